@@ -1,0 +1,16 @@
+"""CPU oracle for the Q4_0 decode path (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU-baseline
+and reference legs) may import this package.  The library's product path never
+calls it, and it shares no code with the CUDA path.
+"""
+from .q4_oracle import (  # noqa: F401
+    bf16_bits_to_f64,
+    f16_bits_to_f64,
+    unpack_superblocks,
+    dequant,
+    gemv,
+    gemv_tolerance,
+    attn_probs,
+    attn_decode,
+)

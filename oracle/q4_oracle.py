@@ -1,0 +1,159 @@
+"""Plain, slow fp64 CPU oracle of the Q4_0 decode path.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline / reference legs may import or run this file.  It
+shares no code, tables or constants with the CUDA path and imports nothing
+from it; both sides read the same input bytes produced by ``synth``.
+
+What it computes, and where the pages stand on it
+-------------------------------------------------
+The pages ("Qwen3.8-27B at 256K on a 24GB RTX PRO 4000 SFF (432 GB/s): 50
+tok/s with MTP", the paragraph beginning "NVIDIA quotes 432 GB/s") attribute
+decode speed to two costs: repeatedly streaming quantised weights, and reading
+a Q4 K/V cache that grows with context.  The same page (paragraph on public
+GGUFs at 40K context) names the Q4_0 weight format; the paragraph on the 16
+full-attention layers says only those layers keep a K/V cache, stored as Q4.
+"Qwen3.8-27B on RTX 4090: 5,000 tok/s Prefill Reproduced" (section "MTP helps
+ordinary prose, but acceptance controls the gain") explains that the target
+model verifies a drafted block of tokens, which is where the M = 1..5 rows of
+one decode step come from.  The pages define none of the formulas; this file
+writes out the definitions the library implements:
+
+* Q4_0 block: 32 weights, one fp16 scale ``d``, 16 bytes of nibbles; byte
+  ``j`` holds element ``j`` (low nibble) and ``j + 16`` (high nibble);
+  ``w = d * (q - 8)``.
+* super-block storage: 8 blocks in 144 bytes, nibbles first (``16*b + j``),
+  then the 8 fp16 scales at ``128 + 2*b`` (little endian).  A row of K
+  elements is K/256 consecutive super-blocks.
+* GEMV: ``y[m, n] = sum_k w[n, k] * x[m, k]`` for M bf16 rows x.
+* decode attention: query head ``h`` reads KV head ``h // (n_q / n_kv)``; draft
+  row ``m`` sits at position ``p_m = ctx_len - M + m`` and sees tokens
+  ``t <= p_m``; ``s = scale * Q . K_hat``, ``P = softmax(s)``, ``out = P V_hat``.
+
+Readings taken where nothing fixes a detail: output is fp32 on the device
+(fp64 here); the softmax scale defaults to 1 (queries arrive pre-scaled);
+GQA groups are contiguous; non-finite inputs are out of scope.
+
+Everything is fp64 numpy; the matrix products are numpy's (a library
+primitive), with no blocking, reordering or fusion beyond the definitions.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+SB_ELEMS = 256          # elements per super-block
+SB_BYTES = 144          # bytes per super-block
+NIBBLE_BYTES = 128      # bytes of nibbles per super-block (8 blocks x 16)
+
+
+def bf16_bits_to_f64(bits) -> np.ndarray:
+    """Exact value of bf16 bit patterns: the 16 bits are the top half of an
+    IEEE binary32 number."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def f16_bits_to_f64(bits) -> np.ndarray:
+    """Exact value of IEEE binary16 bit patterns."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def unpack_superblocks(buf, rows: int, K: int):
+    """Read ``rows`` rows of ``K`` Q4_0 elements from super-block bytes.
+
+    Returns ``q`` (uint8 [rows][K], values 0..15) and ``d`` (float64
+    [rows][K/32], the per-block scale of each group of 32 elements).
+    """
+    if K % SB_ELEMS:
+        raise ValueError("K must be a multiple of 256")
+    nsb = K // SB_ELEMS
+    raw = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    need = rows * nsb * SB_BYTES
+    if raw.size < need:
+        raise ValueError(f"buffer holds {raw.size} bytes, need {need}")
+    sb = raw[:need].reshape(rows, nsb, SB_BYTES)
+    q = np.empty((rows, nsb, 8, 32), dtype=np.uint8)
+    d_bits = np.empty((rows, nsb, 8), dtype=np.uint16)
+    for b in range(8):
+        qs = sb[:, :, 16 * b: 16 * b + 16]           # 16 bytes of block b
+        q[:, :, b, 0:16] = qs & 0x0F                  # element j
+        q[:, :, b, 16:32] = qs >> 4                   # element j + 16
+        lo = sb[:, :, 128 + 2 * b].astype(np.uint16)
+        hi = sb[:, :, 128 + 2 * b + 1].astype(np.uint16)
+        d_bits[:, :, b] = lo | (hi << 8)              # little endian fp16
+    return q.reshape(rows, K), f16_bits_to_f64(d_bits).reshape(rows, K // 32)
+
+
+def dequant(buf, rows: int, K: int) -> np.ndarray:
+    """fp64 weights ``w = d * (q - 8)`` of ``rows x K`` Q4_0 elements."""
+    q, d = unpack_superblocks(buf, rows, K)
+    return np.repeat(d, 32, axis=1) * (q.astype(np.float64) - 8.0)
+
+
+def gemv(W_buf, x_bits, M: int, N: int, K: int):
+    """Dequant-GEMV: ``y[m, n] = sum_k w[n, k] x[m, k]`` in fp64.
+
+    ``W_buf``: N rows of K elements in super-block layout; ``x_bits``: bf16 bit
+    patterns [M][K].  Returns ``(y, S)``, both float64 [M][N], where
+    ``S[m, n] = sum_k |w[n, k] x[m, k]|`` scales the parity tolerance.
+    """
+    w = dequant(W_buf, N, K)
+    x = bf16_bits_to_f64(np.asarray(x_bits).reshape(M, K))
+    y = x @ w.T
+    S = np.abs(x) @ np.abs(w).T
+    return y, S
+
+
+def gemv_tolerance(S: np.ndarray) -> np.ndarray:
+    """Per-element bound ``2e-3 * S + 1e-5`` that the device result must meet."""
+    return 2e-3 * S + 1e-5
+
+
+def _kv_hat(buf, n_kv: int, ctx_len: int, head_dim: int, kv_stride: int) -> np.ndarray:
+    """Dequantised cache [n_kv][ctx_len][head_dim] (rows of one super-block
+    per token when head_dim == 256; ``kv_stride`` tokens between heads)."""
+    out = np.empty((n_kv, ctx_len, head_dim), dtype=np.float64)
+    row_bytes = (head_dim // SB_ELEMS) * SB_BYTES
+    raw = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    for h in range(n_kv):
+        start = h * kv_stride * row_bytes
+        out[h] = dequant(raw[start: start + ctx_len * row_bytes], ctx_len, head_dim)
+    return out
+
+
+def attn_probs(Q_bits, K_buf, ctx_len: int, n_q_heads: int, n_kv_heads: int,
+               head_dim: int, M: int, kv_stride: int | None = None,
+               scale: float = 1.0) -> np.ndarray:
+    """Softmax weights ``P[m, h, t]`` (zero for masked tokens), fp64."""
+    kv_stride = ctx_len if kv_stride is None else kv_stride
+    g = n_q_heads // n_kv_heads
+    Q = bf16_bits_to_f64(np.asarray(Q_bits).reshape(M, n_q_heads, head_dim))
+    Kh = _kv_hat(K_buf, n_kv_heads, ctx_len, head_dim, kv_stride)
+    P = np.zeros((M, n_q_heads, ctx_len), dtype=np.float64)
+    for m in range(M):
+        p_m = ctx_len - M + m                 # absolute position of draft row m
+        for h in range(n_q_heads):
+            kv = h // g
+            s = scale * (Kh[kv, : p_m + 1] @ Q[m, h])
+            e = np.exp(s - s.max())
+            P[m, h, : p_m + 1] = e / e.sum()
+    return P
+
+
+def attn_decode(Q_bits, K_buf, V_buf, ctx_len: int, n_q_heads: int, n_kv_heads: int,
+                head_dim: int, M: int, kv_stride: int | None = None,
+                scale: float = 1.0) -> np.ndarray:
+    """Causal GQA decode attention over a Q4_0 K/V cache, fp64.
+
+    Returns ``out[m, h, :] = sum_t P[m, h, t] * V_hat[h // g, t, :]``.
+    """
+    kv_stride = ctx_len if kv_stride is None else kv_stride
+    g = n_q_heads // n_kv_heads
+    P = attn_probs(Q_bits, K_buf, ctx_len, n_q_heads, n_kv_heads, head_dim, M,
+                   kv_stride, scale)
+    Vh = _kv_hat(V_buf, n_kv_heads, ctx_len, head_dim, kv_stride)
+    out = np.empty((M, n_q_heads, head_dim), dtype=np.float64)
+    for m in range(M):
+        for h in range(n_q_heads):
+            out[m, h] = P[m, h] @ Vh[h // g]
+    return out

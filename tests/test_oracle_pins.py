@@ -1,0 +1,395 @@
+"""Pins for the CPU oracle: each test ties it to something other than itself --
+a hand-worked fixture, literal bit patterns, closed forms, invariants, or a
+brute-force pure-Python evaluation with exact rational arithmetic."""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------- helpers ---
+def _fraction_bf16(bits: int) -> Fraction:
+    """Exact value of a bf16 bit pattern by the IEEE binary32 field definition
+    (sign, 8-bit exponent, 7 stored fraction bits), in rationals."""
+    sign = -1 if bits & 0x8000 else 1
+    exp = (bits >> 7) & 0xFF
+    frac = bits & 0x7F
+    if exp == 0:
+        return sign * Fraction(frac, 128) * Fraction(2) ** (-126)
+    return sign * (1 + Fraction(frac, 128)) * Fraction(2) ** (exp - 127)
+
+
+def _fraction_f16(bits: int) -> Fraction:
+    """Exact value of an IEEE binary16 bit pattern (5-bit exponent, 10 bits)."""
+    sign = -1 if bits & 0x8000 else 1
+    exp = (bits >> 10) & 0x1F
+    frac = bits & 0x3FF
+    if exp == 0:
+        return sign * Fraction(frac, 1024) * Fraction(2) ** (-14)
+    return sign * (1 + Fraction(frac, 1024)) * Fraction(2) ** (exp - 15)
+
+
+def _brute_weights(buf, rows, K):
+    """Pure-Python reading of the super-block layout, in rationals."""
+    raw = bytes(np.asarray(buf, dtype=np.uint8).tobytes())
+    nsb = K // 256
+    w = [[Fraction(0)] * K for _ in range(rows)]
+    for r in range(rows):
+        for s in range(nsb):
+            base = (r * nsb + s) * 144
+            for b in range(8):
+                d = _fraction_f16(raw[base + 128 + 2 * b] | (raw[base + 129 + 2 * b] << 8))
+                for j in range(16):
+                    byte = raw[base + 16 * b + j]
+                    k0 = s * 256 + b * 32
+                    w[r][k0 + j] = d * ((byte & 15) - 8)
+                    w[r][k0 + j + 16] = d * ((byte >> 4) - 8)
+    return w
+
+
+# ------------------------------------------------------- number formats ----
+def test_bf16_literal_values():
+    cases = {0x3F80: 1.0, 0xBF80: -1.0, 0x4049: 3.140625, 0x3E20: 0.15625,
+             0x0000: 0.0, 0x0001: 2.0 ** -133, 0x0080: 2.0 ** -126,
+             0x7F7F: 3.3895313892515355e38, 0xC2F7: -123.5}
+    got = oracle.bf16_bits_to_f64(np.array(list(cases), dtype=np.uint16))
+    assert list(got) == list(cases.values())
+
+
+def test_f16_literal_values():
+    cases = {0x3800: 0.5, 0x3C00: 1.0, 0xB400: -0.25, 0x0001: 2.0 ** -24,
+             0x0400: 2.0 ** -14, 0x7BFF: 65504.0, 0xC500: -5.0, 0x2E66: 0.0999755859375}
+    got = oracle.f16_bits_to_f64(np.array(list(cases), dtype=np.uint16))
+    assert list(got) == list(cases.values())
+
+
+def test_bf16_decode_matches_field_definition_exhaustively():
+    bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    finite = ((bits.astype(np.uint32) >> 7) & 0xFF) != 0xFF
+    got = oracle.bf16_bits_to_f64(bits[finite])
+    sample = np.random.default_rng(5).choice(np.flatnonzero(finite), 2000, replace=False)
+    for i in sample:
+        b = int(bits[i])
+        assert Fraction(got[np.searchsorted(np.flatnonzero(finite), i)]) == _fraction_bf16(b)
+
+
+def test_rounding_helpers_are_nearest_even():
+    # 1 + 2^-8 is halfway between bf16 1.0 and 1.0078125 -> ties to even (1.0)
+    v = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -2.5, 1e-3], dtype=np.float32)
+    bits = synth.f32_to_bf16_bits(v)
+    assert list(bits[:3]) == [0x3F80, 0x3F82, 0xC020]
+    assert abs(oracle.bf16_bits_to_f64(bits[3:])[0] - 1e-3) <= 2 ** -9 * 1e-3
+
+
+# ---------------------------------------------------------- Q4_0 layout ----
+def _read_golden():
+    blocks, expect = [], []
+    with open(os.path.join(GOLDEN, "q4_0_superblock_worked.txt")) as f:
+        lines = [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+    for head, vals in zip(lines[0::2], lines[1::2]):
+        parts = dict(p.split("=") for p in head.split()[2:])
+        blocks.append((int(parts["d"], 16), bytes.fromhex(parts["bytes"])))
+        expect.extend(float(v) for v in vals.split())
+    return blocks, expect
+
+
+def test_worked_superblock_fixture():
+    blocks, expect = _read_golden()
+    assert len(blocks) == 8 and len(expect) == 256
+    sb = bytearray(144)
+    for b, (dbits, qs) in enumerate(blocks):
+        sb[16 * b: 16 * b + 16] = qs
+        sb[128 + 2 * b] = dbits & 0xFF
+        sb[129 + 2 * b] = dbits >> 8
+    w = oracle.dequant(np.frombuffer(bytes(sb), dtype=np.uint8), 1, 256)
+    assert list(w[0]) == expect
+
+
+def test_pack_unpack_roundtrip():
+    rng = np.random.default_rng(11)
+    q = rng.integers(0, 16, size=(7, 768), dtype=np.uint8)
+    dbits = rng.integers(0, 0x7C00, size=(7, 24)).astype(np.uint16)
+    buf = synth.pack_superblocks(q, dbits)
+    assert buf.size == 7 * 3 * 144
+    q2, d2 = oracle.unpack_superblocks(buf, 7, 768)
+    assert np.array_equal(q2, q)
+    assert np.array_equal(d2, oracle.f16_bits_to_f64(dbits))
+
+
+def test_superblock_offsets_single_nibble():
+    # one nonzero nibble (q = 9, all others q = 8) at row 2, super-block 1,
+    # block 5, byte 3, high nibble -> element 256 + 5*32 + 3 + 16 only
+    N, K = 4, 512
+    q = np.full((N, K), 8, dtype=np.uint8)
+    d = np.full((N, K // 32), 0.5, dtype=np.float32)
+    q[2, 256 + 5 * 32 + 3 + 16] = 9
+    buf = synth.from_parts(q, d)
+    raw = buf.reshape(N, 2, 144)
+    assert raw[2, 1, 16 * 5 + 3] == (8 | (9 << 4))
+    w = oracle.dequant(buf, N, K)
+    nz = np.argwhere(w != 0)
+    assert nz.tolist() == [[2, 256 + 5 * 32 + 3 + 16]] and w[2, 435] == 0.5
+
+
+def test_oracle_reading_matches_bruteforce_reader():
+    buf = synth.q4_0_weights(21, 3, 512)
+    w = oracle.dequant(buf, 3, 512)
+    wb = _brute_weights(buf, 3, 512)
+    for r in range(3):
+        assert [Fraction(v) for v in w[r]] == wb[r]
+
+
+# ----------------------------------------------------------------- GEMV ----
+def test_one_hot_x_picks_one_weight_column():
+    N, K = 5, 512
+    buf = synth.q4_0_weights(3, N, K)
+    w = oracle.dequant(buf, N, K)
+    for k in (0, 17, 31, 32, 255, 256, 511):
+        x = np.zeros((1, K), dtype=np.uint16)
+        x[0, k] = 0x3F80  # 1.0
+        y, S = oracle.gemv(buf, x, 1, N, K)
+        assert np.array_equal(y[0], w[:, k]) and np.array_equal(S[0], np.abs(w[:, k]))
+
+
+def test_all_q8_gives_exact_zero():
+    N, K, M = 6, 1024, 3
+    q = np.full((N, K), 8, dtype=np.uint8)
+    d = np.abs(np.random.default_rng(1).standard_normal((N, K // 32))).astype(np.float32)
+    buf = synth.from_parts(q, d)
+    x = synth.activations(2, M, K)
+    y, S = oracle.gemv(buf, x, M, N, K)
+    assert np.all(y == 0.0) and np.all(S == 0.0)
+
+
+def test_linear_in_one_block_scale():
+    # dyadic values keep every fp64 operation exact, so the change must equal
+    # the one block's contribution exactly
+    N, K = 3, 512
+    rng = np.random.default_rng(4)
+    q = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    d = (2.0 ** -rng.integers(1, 6, size=(N, K // 32))).astype(np.float32)
+    x = synth.f32_to_bf16_bits(rng.integers(-4, 5, size=(1, K)).astype(np.float32))
+    y0, _ = oracle.gemv(synth.from_parts(q, d), x, 1, N, K)
+    b = 9
+    d2 = d.copy()
+    d2[:, b] *= 2
+    y1, _ = oracle.gemv(synth.from_parts(q, d2), x, 1, N, K)
+    xs = oracle.bf16_bits_to_f64(x)[0, 32 * b: 32 * b + 32]
+    contrib = (d[:, b:b + 1].astype(np.float64) * (q[:, 32 * b:32 * b + 32] - 8.0)) @ xs
+    assert np.array_equal(y1[0] - y0[0], contrib)
+
+
+def test_linear_in_x():
+    N, K = 4, 768
+    rng = np.random.default_rng(8)
+    buf = synth.from_parts(rng.integers(0, 16, size=(N, K), dtype=np.uint8),
+                           (2.0 ** -rng.integers(2, 8, size=(N, K // 32))).astype(np.float32))
+    a = rng.integers(-3, 4, size=(1, K)).astype(np.float32)
+    b = rng.integers(-3, 4, size=(1, K)).astype(np.float32)
+    ya, _ = oracle.gemv(buf, synth.f32_to_bf16_bits(a), 1, N, K)
+    yb, _ = oracle.gemv(buf, synth.f32_to_bf16_bits(b), 1, N, K)
+    yab, _ = oracle.gemv(buf, synth.f32_to_bf16_bits(3 * a + b), 1, N, K)
+    assert np.array_equal(yab, 3 * ya + yb)
+
+
+def test_rows_are_independent():
+    N, K, M = 8, 512, 5
+    buf = synth.q4_0_weights(12, N, K)
+    x = synth.activations(13, M, K)
+    y5, _ = oracle.gemv(buf, x, M, N, K)
+    for m in range(M):
+        y1, _ = oracle.gemv(buf, x[m:m + 1], 1, N, K)
+        assert np.array_equal(y1[0], y5[m])
+
+
+def test_exact_integer_case_against_python_ints():
+    # d = 2^-k and small-integer x make y an exact dyadic rational
+    N, K, M = 4, 512, 2
+    rng = np.random.default_rng(31)
+    q = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    kexp = rng.integers(0, 6, size=(N, K // 32))
+    xi = rng.integers(-7, 8, size=(M, K))
+    buf = synth.from_parts(q, (2.0 ** -kexp).astype(np.float32))
+    y, _ = oracle.gemv(buf, synth.f32_to_bf16_bits(xi.astype(np.float32)), M, N, K)
+    for m in range(M):
+        for n in range(N):
+            ref = sum(Fraction(int(q[n, k]) - 8, 2 ** int(kexp[n, k // 32])) * int(xi[m, k])
+                      for k in range(K))
+            assert Fraction(y[m, n]) == ref
+
+
+def test_gemv_against_rational_bruteforce():
+    N, K, M = 3, 256, 2
+    buf = synth.q4_0_weights(41, N, K)
+    x = synth.activations(42, M, K)
+    y, S = oracle.gemv(buf, x, M, N, K)
+    w = _brute_weights(buf, N, K)
+    for m in range(M):
+        xs = [_fraction_bf16(int(b)) for b in x[m]]
+        for n in range(N):
+            exact = sum(wk * xk for wk, xk in zip(w[n], xs))
+            sabs = sum(abs(wk * xk) for wk, xk in zip(w[n], xs))
+            assert abs(Fraction(y[m, n]) - exact) <= Fraction(1, 10 ** 12) * (sabs + 1)
+            assert abs(Fraction(S[m, n]) - sabs) <= Fraction(1, 10 ** 12) * (sabs + 1)
+
+
+def test_tolerance_formula():
+    S = np.array([[0.0, 1.0, 250.0]])
+    assert np.allclose(oracle.gemv_tolerance(S), [[1e-5, 2e-3 + 1e-5, 0.5 + 1e-5]])
+
+
+# ------------------------------------------------------------- attention ----
+def _kv_from_parts(q, d):
+    return synth.from_parts(q, d)
+
+
+def _attn_case(seed, ctx, n_q, n_kv, M):
+    K = synth.q4_0_kv_cache(seed, n_kv, ctx)
+    V = synth.q4_0_kv_cache(seed + 1, n_kv, ctx)
+    Q = synth.queries(seed + 2, M, n_q)
+    return Q, K, V
+
+
+def test_softmax_rows_sum_to_one_and_mask():
+    ctx, n_q, n_kv, M = 40, 6, 2, 5
+    Q, K, _ = _attn_case(3, ctx, n_q, n_kv, M)
+    P = oracle.attn_probs(Q, K, ctx, n_q, n_kv, 256, M)
+    assert np.allclose(P.sum(-1), 1.0, rtol=0, atol=1e-14)
+    for m in range(M):
+        assert np.all(P[m, :, ctx - M + m + 1:] == 0) and np.all(P[m, :, : ctx - M + m + 1] > 0)
+
+
+def test_all_keys_q8_gives_mean_of_visible_values():
+    ctx, n_q, n_kv, M = 23, 4, 2, 3
+    kq = np.full((n_kv * ctx, 256), 8, dtype=np.uint8)
+    K = _kv_from_parts(kq, np.ones((n_kv * ctx, 8), dtype=np.float32))
+    V = synth.q4_0_kv_cache(7, n_kv, ctx)
+    Q = synth.queries(8, M, n_q)
+    out = oracle.attn_decode(Q, K, V, ctx, n_q, n_kv, 256, M)
+    Vh = oracle.dequant(V, n_kv * ctx, 256).reshape(n_kv, ctx, 256)
+    for m in range(M):
+        vis = ctx - M + m + 1
+        for h in range(n_q):
+            mean = [math.fsum(Vh[h // 2, t, c] for t in range(vis)) / vis for c in range(256)]
+            assert np.allclose(out[m, h], mean, rtol=0, atol=1e-13)
+
+
+def test_constant_values_give_that_constant():
+    ctx, n_q, n_kv, M = 31, 6, 3, 2
+    vq = np.full((n_kv * ctx, 256), 11, dtype=np.uint8)          # q - 8 = 3
+    V = _kv_from_parts(vq, np.full((n_kv * ctx, 8), 0.25, dtype=np.float32))
+    Q, K, _ = _attn_case(9, ctx, n_q, n_kv, M)
+    out = oracle.attn_decode(Q, K, V, ctx, n_q, n_kv, 256, M)
+    assert np.allclose(out, 0.75, rtol=0, atol=1e-14)
+
+
+def test_single_token_returns_its_value_row():
+    Q, K, V = _attn_case(15, 1, 4, 1, 1)
+    out = oracle.attn_decode(Q, K, V, 1, 4, 1, 256, 1)
+    Vh = oracle.dequant(V, 1, 256)
+    assert np.array_equal(out[0], np.repeat(Vh, 4, axis=0))
+
+
+def test_dominant_key_selects_its_value():
+    ctx, M = 16, 1
+    kq = np.full((ctx, 256), 8, dtype=np.uint8)
+    kq[5, :] = 15                                    # q - 8 = 7 on every dim
+    K = _kv_from_parts(kq, np.full((ctx, 8), 1.0, dtype=np.float32))
+    V = synth.q4_0_kv_cache(17, 1, ctx)
+    Q = synth.f32_to_bf16_bits(np.full((1, 1, 256), 1.0, dtype=np.float32))
+    out = oracle.attn_decode(Q, K, V, ctx, 1, 1, 256, M)     # logit gap 7*256
+    Vh = oracle.dequant(V, ctx, 256)
+    assert np.array_equal(out[0, 0], Vh[5])
+
+
+def test_causal_rows_ignore_later_tokens():
+    ctx, n_q, n_kv, M = 20, 6, 2, 5
+    Q, K, V = _attn_case(19, ctx, n_q, n_kv, M)
+    base = oracle.attn_decode(Q, K, V, ctx, n_q, n_kv, 256, M)
+    # perturb the last token (position ctx-1) of every head: only row M-1 sees it
+    K2 = K.copy().reshape(n_kv, ctx, 144)
+    V2 = V.copy().reshape(n_kv, ctx, 144)
+    K2[:, ctx - 1, :128] ^= 0x5A
+    V2[:, ctx - 1, :128] ^= 0xA5
+    pert = oracle.attn_decode(Q, K2.reshape(-1), V2.reshape(-1), ctx, n_q, n_kv, 256, M)
+    assert np.array_equal(pert[: M - 1], base[: M - 1])
+    assert not np.allclose(pert[M - 1], base[M - 1])
+
+
+def test_gqa_head_mapping_is_contiguous_groups():
+    ctx, n_q, n_kv, M = 9, 6, 3, 1
+    vq = np.concatenate([np.full((ctx, 256), 8 + h, dtype=np.uint8) for h in range(n_kv)])
+    V = _kv_from_parts(vq, np.ones((n_kv * ctx, 8), dtype=np.float32))
+    Q, K, _ = _attn_case(23, ctx, n_q, n_kv, M)
+    out = oracle.attn_decode(Q, K, V, ctx, n_q, n_kv, 256, M)
+    for h in range(n_q):
+        assert np.allclose(out[0, h], h // 2, rtol=0, atol=1e-14)
+
+
+def test_mha_equals_independent_single_heads():
+    ctx, n, M = 12, 3, 2
+    Q, K, V = _attn_case(29, ctx, n, n, M)
+    out = oracle.attn_decode(Q, K, V, ctx, n, n, 256, M)
+    Kr, Vr = K.reshape(n, ctx * 144), V.reshape(n, ctx * 144)
+    Qr = Q.reshape(M, n, 256)
+    for h in range(n):
+        one = oracle.attn_decode(Qr[:, h:h + 1].copy(), Kr[h], Vr[h], ctx, 1, 1, 256, M)
+        assert np.array_equal(one[:, 0], out[:, h])
+
+
+def test_softmax_scale_equals_scaled_queries():
+    ctx, n_q, n_kv, M = 14, 4, 2, 2
+    Q, K, V = _attn_case(33, ctx, n_q, n_kv, M)
+    Q2 = synth.f32_to_bf16_bits(2 * oracle.bf16_bits_to_f64(Q).astype(np.float32))
+    a = oracle.attn_decode(Q, K, V, ctx, n_q, n_kv, 256, M, scale=2.0)
+    b = oracle.attn_decode(Q2, K, V, ctx, n_q, n_kv, 256, M)
+    assert np.allclose(a, b, rtol=0, atol=1e-13)
+
+
+def test_kv_stride_reads_the_right_rows():
+    ctx, cap, n_q, n_kv, M = 10, 16, 4, 2, 2
+    Kf = synth.q4_0_kv_cache(35, n_kv, cap)
+    Vf = synth.q4_0_kv_cache(36, n_kv, cap)
+    Q = synth.queries(37, M, n_q)
+    out = oracle.attn_decode(Q, Kf, Vf, ctx, n_q, n_kv, 256, M, kv_stride=cap)
+    Kc = Kf.reshape(n_kv, cap, 144)[:, :ctx].reshape(-1)
+    Vc = Vf.reshape(n_kv, cap, 144)[:, :ctx].reshape(-1)
+    ref = oracle.attn_decode(Q, Kc, Vc, ctx, n_q, n_kv, 256, M)
+    assert np.array_equal(out, ref)
+
+
+def test_attention_against_python_bruteforce():
+    ctx, n_q, n_kv, M = 7, 4, 2, 3
+    Q, K, V = _attn_case(39, ctx, n_q, n_kv, M)
+    out = oracle.attn_decode(Q, K, V, ctx, n_q, n_kv, 256, M)
+    Kw = _brute_weights(K, n_kv * ctx, 256)
+    Vw = _brute_weights(V, n_kv * ctx, 256)
+    Qf = np.asarray(Q).reshape(M, n_q, 256)
+    for m in range(M):
+        vis = ctx - M + m + 1
+        for h in range(n_q):
+            kv = h // (n_q // n_kv)
+            q = [_fraction_bf16(int(b)) for b in Qf[m, h]]
+            s = [float(sum(a * b for a, b in zip(q, Kw[kv * ctx + t]))) for t in range(vis)]
+            mx = max(s)
+            e = [math.exp(v - mx) for v in s]
+            z = math.fsum(e)
+            for c in range(0, 256, 37):
+                ref = math.fsum(e[t] * float(Vw[kv * ctx + t][c]) for t in range(vis)) / z
+                assert out[m, h, c] == pytest.approx(ref, abs=1e-12)
+
+
+def test_quantizer_recipe_on_literal_block():
+    v = np.zeros((1, 256), dtype=np.float32)
+    v[0, :32] = np.linspace(-1.0, 2.0, 32, dtype=np.float32)   # amax = +2.0
+    q, d = synth.quantize_blocks(v)
+    assert d[0, 0] == 0xB400                                    # fp16(-0.25)
+    assert q[0, 31] == 0 and q[0, 0] == 12                      # 2/-0.25+8.5 -> 0; -1/-0.25+8.5 -> 12
+    assert np.all(q[0, 32:] == 8) and np.all(d[0, 1:] == 0)
