@@ -1,0 +1,512 @@
+#!/usr/bin/env python3
+"""Benchmark of the Q4_0 decode hot path on B200.
+
+One step = one decode pass of the whole path at M draft rows:
+  * the 64-layer Q4_0 weight stream (per layer: gate 5120->17408, up
+    5120->17408, down 17408->5120, in 5120->6144, out 6144->5120) plus the
+    5120->151936 output head: 321 q4_gemv calls, 12.33 GB of weights;
+  * Q4-KV decode attention for 16 layers (24 query heads, 4 KV heads,
+    head_dim 256) at ctx_len 262144: 16 q4kv_attn_decode calls, 4.83 GB.
+Every matrix and cache is distinct (17.2 GB per step, far above the 126 MB
+L2), so no L2 flush is needed between steps.  The metric is achieved HBM
+TB/s = algorithmic bytes / device time.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--M m] [--impl reference]
+Under torchrun each rank runs an independent replica on its own GPU (the
+path has no exchange step); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Q4 decode GEMV/attn: achieved HBM TB/s (% of B200 peak), µs per call at M=1..5"
+HIDDEN, FFN, QKV, HEAD_N, LAYERS = 5120, 17408, 6144, 151936, 64
+ATTN_LAYERS, N_Q, N_KV, HEAD_DIM, CTX = 16, 24, 4, 256, 262144
+LAYER_SHAPES = [(FFN, HIDDEN), (FFN, HIDDEN), (HIDDEN, FFN), (QKV, HIDDEN), (HIDDEN, QKV)]  # (N, K)
+L2_BYTES = 126 * 1024 * 1024
+
+
+def q4_bytes(N, K):
+    return N * (K // 256) * 144
+
+
+def gemv_alg_bytes(M, N, K):
+    return q4_bytes(N, K) + 2 * M * K + 4 * M * N
+
+
+def attn_alg_bytes(M, ctx):
+    return 2 * N_KV * ctx * 144 + M * N_Q * HEAD_DIM * (2 + 4)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_weight_streaming_dequant_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    e = rec.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_uuid}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 7]
+        if not rows:
+            return None
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if "Active" in v
+                          and "Not" not in v})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------- CPU arms --
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        n = 1
+    return int(n)
+
+
+def oracle_sample_step(seed=0):
+    """One bounded sample of the workload on the CPU oracle: a 5120->6144
+    GEMV at M rows and one attention layer at ctx 4096.  Returns
+    (algorithmic bytes, seconds)."""
+    import oracle
+    import synth
+
+    N, K = QKV, HIDDEN
+    W = synth.q4_0_weights(1000 + seed, N, K)
+    x = synth.activations(2000 + seed, ARGS.M, K)
+    ctx = 4096
+    Kc, Vc = synth.q4_0_kv_cache(3000 + seed, N_KV, ctx), synth.q4_0_kv_cache(4000 + seed, N_KV, ctx)
+    Q = synth.queries(5000 + seed, ARGS.M, N_Q)
+    t0 = time.perf_counter()
+    oracle.gemv(W, x, ARGS.M, N, K)
+    oracle.attn_decode(Q, Kc, Vc, ctx, N_Q, N_KV, HEAD_DIM, ARGS.M)
+    dt = time.perf_counter() - t0
+    return gemv_alg_bytes(ARGS.M, N, K) + attn_alg_bytes(ARGS.M, ctx), dt
+
+
+SAMPLE_DESC = ("fp64 numpy oracle: one 5120->6144 Q4_0 GEMV plus one attention layer at "
+               "ctx 4096 (24/4 heads) per sample, M as the GPU arm; inputs generated "
+               "outside the timed part")
+
+
+def cpu_baseline(n_samples=3):
+    total_b, total_t = 0, 0.0
+    for s in range(n_samples):
+        b, t = oracle_sample_step(s)
+        total_b += b
+        total_t += t
+    return {"value": total_b / total_t / 1e12, "unit": "TB/s", "cores": cpu_cores(),
+            "kind": "oracle", "sample": f"{n_samples} samples; " + SAMPLE_DESC}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    for s in range(args.warmup):
+        oracle_sample_step(100 + s)
+    bs, ts = [], []
+    for s in range(args.steps):
+        b, t = oracle_sample_step(s)
+        bs.append(b)
+        ts.append(t)
+    value = sum(bs) / sum(ts) / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(ts) / len(ts), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(args),
+            "cpu_baseline": {"kind": "oracle", "cores": cpu_cores(), "value": value,
+                             "unit": "TB/s", "sample": "each step: " + SAMPLE_DESC},
+            "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(args):
+    return {"workload": (f"decode step at M={args.M}: 64-layer Q4_0 weight stream "
+                         "(5120->17408 x2, 17408->5120, 5120->6144, 6144->5120) + "
+                         "5120->151936 head = 321 GEMVs, then 16-layer Q4-KV attention "
+                         f"(24 q / 4 kv heads, head_dim 256) at ctx_len {CTX}"),
+            "M": args.M, "ctx_len": CTX, "layers": LAYERS, "attn_layers": ATTN_LAYERS,
+            "bytes_per_step": step_bytes(args.M),
+            "l2": "inputs larger than L2 (17.2 GB of distinct weights/caches per step)",
+            "parallelism": f"replicas x{args.gpus}"}
+
+
+def step_bytes(M):
+    g = sum(gemv_alg_bytes(M, N, K) for N, K in LAYER_SHAPES) * LAYERS
+    g += gemv_alg_bytes(M, HEAD_N, HIDDEN)
+    return g + ATTN_LAYERS * attn_alg_bytes(M, CTX)
+
+
+# ------------------------------------------------------------- GPU arm --
+def main():
+    global ARGS
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--M", type=int, default=1, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="libq4dec", choices=["libq4dec", "reference"])
+    ap.add_argument("--no-per-call", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    ARGS = args
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from bit_weight_streaming_dequant_b200 import q4dec
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+    q4dec.lib()
+    M = args.M
+
+    # -------- resident state: weights and caches (generated on the device)
+    gen_t0 = time.time()
+    layers = []
+    for l in range(LAYERS):
+        layers.append([synth.device_q4_0_weights(1000 + 5 * l + i, N, K, device=dev)
+                       for i, (N, K) in enumerate(LAYER_SHAPES)])
+    head = synth.device_q4_0_weights(999, HEAD_N, HIDDEN, device=dev)
+    kv = [(synth.device_q4_0_kv_cache(2000 + l, N_KV, CTX, device=dev),
+           synth.device_q4_0_kv_cache(2100 + l, N_KV, CTX, device=dev))
+          for l in range(ATTN_LAYERS)]
+    # per-step inputs and outputs
+    xs = {K: synth.device_bf16_normal(7 + K, (M, K), device=dev) for K in (HIDDEN, FFN, QKV)}
+    ys = {N: torch.empty((M, N), dtype=torch.float32, device=dev)
+          for N in (FFN, HIDDEN, QKV, HEAD_N)}
+    Qs = [synth.device_bf16_normal(2200 + l, (M, N_Q, HEAD_DIM), scale=1 / 16, device=dev)
+          for l in range(ATTN_LAYERS)]
+    outs = [torch.empty((M, N_Q, HEAD_DIM), dtype=torch.float32, device=dev)
+            for _ in range(ATTN_LAYERS)]
+    L = q4dec.lib()
+    gws = max([L.q4d_gemv_workspace_bytes(M, N, K) for N, K in LAYER_SHAPES + [(HEAD_N, HIDDEN)]])
+    aws = L.q4d_attn_workspace_bytes(CTX, N_Q, N_KV, HEAD_DIM, M)
+    ws = torch.empty(max(gws, aws, 16), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    gen_s = time.time() - gen_t0
+
+    stream = torch.cuda.current_stream()
+    sptr = stream.cuda_stream
+    launches = {"n": 0}
+
+    def gemv(W, x, y, N, K):
+        st = L.q4_gemv_ex(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, sptr,
+                          ws.data_ptr(), ws.numel())
+        if st:
+            raise RuntimeError(f"q4_gemv_ex failed: {st}")
+        launches["n"] += 1 + (1 if L.q4d_gemv_workspace_bytes(M, N, K) else 0)
+
+    def attn(l):
+        Kc, Vc = kv[l]
+        st = L.q4kv_attn_decode_ex(Qs[l].data_ptr(), Kc.data_ptr(), Vc.data_ptr(),
+                                   outs[l].data_ptr(), CTX, N_Q, N_KV, HEAD_DIM, M, CTX,
+                                   1.0, sptr, ws.data_ptr(), ws.numel())
+        if st:
+            raise RuntimeError(f"q4kv_attn_decode_ex failed: {st}")
+        launches["n"] += 2 if aws else 1
+
+    def gemv_stream():
+        for l in range(LAYERS):
+            for i, (N, K) in enumerate(LAYER_SHAPES):
+                gemv(layers[l][i], xs[K], ys[N], N, K)
+        gemv(head, xs[HIDDEN], ys[HEAD_N], HEAD_N, HIDDEN)
+
+    def attn_stream():
+        for l in range(ATTN_LAYERS):
+            attn(l)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+
+    for _ in range(args.warmup):
+        gemv_stream()
+        attn_stream()
+    torch.cuda.synchronize()
+
+    # -------- timed region
+    K_ = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K_)]
+    launches["n"] = 0
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(K_):
+        ev[k][0].record(stream)
+        gemv_stream()
+        ev[k][1].record(stream)
+        attn_stream()
+        ev[k][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    timed_launches = launches["n"]
+    total_ms = t_start.elapsed_time(t_end)
+    gemv_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
+    clock = clocks.stop()
+
+    t = torch.tensor([total_ms, gemv_ms, attn_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, gemv_ms, attn_ms = t.tolist()
+
+    bytes_step = step_bytes(M)
+    value = bytes_step * K_ * world / (total_ms * 1e-3) / 1e12
+    peak_gbs, peak_kind = peaks()
+    n_gemv = LAYERS * len(LAYER_SHAPES) + 1
+    gemv_bytes = sum(gemv_alg_bytes(M, N, K) for N, K in LAYER_SHAPES) * LAYERS + \
+        gemv_alg_bytes(M, HEAD_N, HIDDEN)
+    per_launch_bytes = gemv_bytes / n_gemv
+    per_launch_s = gemv_ms * 1e-3 / (K_ * n_gemv)
+    achieved_gbs = per_launch_bytes / per_launch_s / 1e9
+    attn_gbs = ATTN_LAYERS * attn_alg_bytes(M, CTX) * K_ / (attn_ms * 1e-3) / 1e9
+
+    # -------- end to end through the public API with host buffers
+    import torch as _t
+
+    e2e_steps = max(3, min(K_, 10))
+    h_x = {K: _t.empty((M, K), dtype=_t.bfloat16, pin_memory=True) for K in xs}
+    for K in xs:
+        h_x[K].copy_(xs[K])
+    h_q = [_t.empty((M, N_Q, HEAD_DIM), dtype=_t.bfloat16, pin_memory=True) for _ in Qs]
+    for l in range(ATTN_LAYERS):
+        h_q[l].copy_(Qs[l])
+    h_y = {N: _t.empty((M, N), dtype=_t.float32, pin_memory=True) for N in ys}
+    h_o = [_t.empty((M, N_Q, HEAD_DIM), dtype=_t.float32, pin_memory=True) for _ in outs]
+    h2d = d2h = 0
+
+    def e2e_step():
+        nonlocal h2d, d2h
+        h2d = d2h = 0
+        for l in range(LAYERS):
+            for i, (N, K) in enumerate(LAYER_SHAPES):
+                xs[K].copy_(h_x[K], non_blocking=True)
+                h2d += xs[K].numel() * 2
+                gemv(layers[l][i], xs[K], ys[N], N, K)
+                h_y[N].copy_(ys[N], non_blocking=True)
+                d2h += ys[N].numel() * 4
+        xs[HIDDEN].copy_(h_x[HIDDEN], non_blocking=True)
+        h2d += xs[HIDDEN].numel() * 2
+        gemv(head, xs[HIDDEN], ys[HEAD_N], HEAD_N, HIDDEN)
+        h_y[HEAD_N].copy_(ys[HEAD_N], non_blocking=True)
+        d2h += ys[HEAD_N].numel() * 4
+        for l in range(ATTN_LAYERS):
+            Qs[l].copy_(h_q[l], non_blocking=True)
+            h2d += Qs[l].numel() * 2
+            attn(l)
+            h_o[l].copy_(outs[l], non_blocking=True)
+            d2h += outs[l].numel() * 4
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = bytes_step * e2e_steps * world / (e2e_ms.item() * 1e-3) / 1e12
+
+    # -------- per-call latencies (cold L2), rank 0
+    per_call = None
+    if rank == 0 and not args.no_per_call:
+        per_call = per_call_table(torch, L, dev, layers, kv, ws, peak_gbs)
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        base = cpu_baseline()
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": world, "steps": K_,
+        "warmup": args.warmup, "ms_per_step": total_ms / K_, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(args),
+        "frac_of_peak": value / world / (peak_gbs / 1e3),
+        "roofline": {"bound": "hbm", "kernel": "q4_gemv_kernel", "achieved": achieved_gbs,
+                     "peak": peak_gbs, "peak_source": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                     "frac": achieved_gbs / peak_gbs,
+                     "traffic": recorded_traffic("q4_gemv_kernel"),
+                     "algorithmic_bytes_per_launch": per_launch_bytes,
+                     "launch_us": per_launch_s * 1e6},
+        "attention": {"achieved_gbs": attn_gbs, "frac": attn_gbs / peak_gbs,
+                      "us_per_layer": attn_ms * 1e3 / (K_ * ATTN_LAYERS)},
+        "cpu_baseline": base,
+        "e2e": {"value": e2e_value, "unit": "TB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": timed_launches,
+        "clocks": clock,
+        "per_call": per_call,
+        "setup_s": gen_s,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def per_call_table(torch, L, dev, layers, kv, ws, peak_gbs, reps=15):
+    """Median device time of single calls with L2 flushed before each call."""
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sptr = stream.cuda_stream
+    table = {"gemv": [], "attn": [], "l2": "flushed before every call (256 MB write)"}
+    names = {(FFN, HIDDEN): "5120->17408", (HIDDEN, FFN): "17408->5120",
+             (QKV, HIDDEN): "5120->6144", (HIDDEN, QKV): "6144->5120"}
+    shape_idx = {(FFN, HIDDEN): 0, (HIDDEN, FFN): 2, (QKV, HIDDEN): 3, (HIDDEN, QKV): 4}
+    for (N, K), name in names.items():
+        for M in (1, 2, 3, 4, 5):
+            x = torch.randn((M, K), device=dev).to(torch.bfloat16)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            times = []
+            for r in range(reps + 2):
+                W = layers[r % len(layers)][shape_idx[(N, K)]]
+                flush.fill_(r & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                st = L.q4_gemv_ex(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, sptr,
+                                  ws.data_ptr(), ws.numel())
+                b.record(stream)
+                assert st == 0
+                torch.cuda.synchronize()
+                if r >= 2:
+                    times.append(a.elapsed_time(b) * 1e3)
+            us = statistics.median(times)
+            gbs = gemv_alg_bytes(M, N, K) / (us * 1e-6) / 1e9
+            table["gemv"].append({"shape": name, "M": M, "us": us, "GBps": gbs,
+                                  "frac": gbs / peak_gbs})
+    for ctx in (4096, 65536, 262144):
+        for M in (1, 5):
+            Q = torch.randn((M, N_Q, HEAD_DIM), device=dev).div_(16).to(torch.bfloat16)
+            out = torch.empty((M, N_Q, HEAD_DIM), dtype=torch.float32, device=dev)
+            times = []
+            for r in range(reps + 2):
+                Kc, Vc = kv[r % len(kv)]
+                flush.fill_(r & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                st = L.q4kv_attn_decode_ex(Q.data_ptr(), Kc.data_ptr(), Vc.data_ptr(),
+                                           out.data_ptr(), ctx, N_Q, N_KV, HEAD_DIM, M, CTX,
+                                           1.0, sptr, ws.data_ptr(), ws.numel())
+                b.record(stream)
+                assert st == 0
+                torch.cuda.synchronize()
+                if r >= 2:
+                    times.append(a.elapsed_time(b) * 1e3)
+            us = statistics.median(times)
+            gbs = attn_alg_bytes(M, ctx) / (us * 1e-6) / 1e9
+            table["attn"].append({"ctx": ctx, "M": M, "us": us, "GBps": gbs,
+                                  "frac": gbs / peak_gbs})
+    del flush
+    return table
+
+
+ARGS = None
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,392 @@
+// libq4dec C ABI: argument validation, launch planning, workspace handling
+// and kernel dispatch.  Declarations and the contract live in include/q4dec.h.
+#include "q4dec.h"
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "q4_gemv.cuh"
+#include "q4kv_attn.cuh"
+
+// Device error word (bit q4d::kDevErrWaitTimeout: a bounded wait ran out).
+__device__ unsigned q4d_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kPlanFallbackSms = 148;
+constexpr size_t kGemvStageBudget = 160 * 1024;  // shared memory for the weight ring
+
+struct DeviceState {
+  std::atomic<bool> ready{false};
+  int num_sms = 0;
+  int smem_optin = 0;
+  unsigned* err = nullptr;
+  void* ws = nullptr;  // library-owned workspace of the plain entry points
+  size_t ws_bytes = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+q4d_status current_device(int* dev_out, DeviceState** st_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return Q4D_ERR_CUDA;
+  }
+  DeviceState& s = g_dev[dev];
+  if (!s.ready.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!s.ready.load(std::memory_order_relaxed)) {
+      if (cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&s.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+              cudaSuccess ||
+          cudaGetSymbolAddress(reinterpret_cast<void**>(&s.err), q4d_error_word) != cudaSuccess) {
+        cudaGetLastError();
+        return Q4D_ERR_CUDA;
+      }
+      s.ready.store(true, std::memory_order_release);
+    }
+  }
+  *dev_out = dev;
+  *st_out = &s;
+  return Q4D_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit to the device maximum, once
+// per (kernel, device).
+template <typename Kernel>
+q4d_status allow_smem(Kernel kernel, int dev, const DeviceState& s, std::atomic<bool>* done) {
+  if (done[dev].load(std::memory_order_acquire)) return Q4D_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s.smem_optin) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return Q4D_ERR_CUDA;
+  }
+  done[dev].store(true, std::memory_order_release);
+  return Q4D_OK;
+}
+
+q4d_status library_workspace(DeviceState& s, size_t need, void** ws) {
+  if (need == 0) {
+    *ws = nullptr;
+    return Q4D_OK;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (s.ws_bytes < need) {
+    if (s.ws) cudaFree(s.ws);
+    s.ws = nullptr;
+    s.ws_bytes = 0;
+    if (cudaMalloc(&s.ws, need) != cudaSuccess) {
+      cudaGetLastError();
+      return Q4D_ERR_CUDA;
+    }
+    s.ws_bytes = need;
+  }
+  *ws = s.ws;
+  return Q4D_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int ceil_div(long long a, long long b) { return int((a + b - 1) / b); }
+long long round_up(long long a, long long b) { return (a + b - 1) / b * b; }
+
+// Per-M kernel configuration: 32-bit nibble words per thread and rows per
+// stream per stage.  Must match the dispatch in launch_gemv.
+int gemv_words_per_thread(int M) { return M == 1 ? 4 : (M == 2 ? 2 : 1); }
+int gemv_rows_per_stream(int M) { return M <= 2 ? 4 : 2; }
+
+q4d_status check_gemv_shape(int M, int N, int K) {
+  if (N < 1 || K < 0) return Q4D_ERR_INVALID_ARG;
+  if (M < 1 || M > 5 || K < 256 || K % 256 != 0) return Q4D_ERR_UNSUPPORTED_SHAPE;
+  return Q4D_OK;
+}
+
+q4d_status check_attn_shape(int ctx_len, int n_q, int n_kv, int head_dim, int M, int kv_stride,
+                            float scale) {
+  if (ctx_len < 1 || n_q < 1 || n_kv < 1 || !std::isfinite(scale)) return Q4D_ERR_INVALID_ARG;
+  if (head_dim != 256 || M < 1 || M > 5 || n_q % n_kv != 0 || ctx_len < M ||
+      kv_stride < ctx_len)
+    return Q4D_ERR_UNSUPPORTED_SHAPE;
+  return Q4D_OK;
+}
+
+template <int M, int W, int RSR>
+q4d_status launch_gemv_t(const q4d::GemvArgs& a, const q4d_gemv_plan& p, int dev,
+                         const DeviceState& s, cudaStream_t stream) {
+  static std::atomic<bool> smem_set[kMaxDevices];
+  auto kernel = q4d::q4_gemv_kernel<M, W, RSR>;
+  q4d_status st = allow_smem(kernel, dev, s, smem_set);
+  if (st != Q4D_OK) return st;
+  dim3 grid(p.grid_rows, p.k_splits);
+  kernel<<<grid, p.threads, p.smem_bytes, stream>>>(a);
+  return Q4D_OK;
+}
+
+q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, int K,
+                     cudaStream_t stream, void* workspace, size_t workspace_bytes,
+                     bool library_ws) {
+  q4d_status st = check_gemv_shape(M, N, K);
+  if (st != Q4D_OK) return st;
+  if (!W_q4 || !x || !y) return Q4D_ERR_INVALID_ARG;
+  if (!aligned(W_q4, 16) || !aligned(x, 16) || !aligned(y, 4)) return Q4D_ERR_MISALIGNED;
+  if (workspace && !aligned(workspace, 16)) return Q4D_ERR_MISALIGNED;
+
+  int dev = 0;
+  DeviceState* s = nullptr;
+  if ((st = current_device(&dev, &s)) != Q4D_OK) return st;
+  q4d_gemv_plan p;
+  if ((st = q4d_plan_gemv(M, N, K, s->num_sms, &p)) != Q4D_OK) return st;
+  if (p.smem_bytes > size_t(s->smem_optin)) return Q4D_ERR_UNSUPPORTED_SHAPE;
+  if (library_ws) {
+    if ((st = library_workspace(*s, p.workspace_bytes, &workspace)) != Q4D_OK) return st;
+  } else if (p.workspace_bytes > 0 && (!workspace || workspace_bytes < p.workspace_bytes)) {
+    return Q4D_ERR_WORKSPACE;
+  }
+
+  q4d::GemvArgs a;
+  a.W = static_cast<const uint8_t*>(W_q4);
+  a.x = static_cast<const uint16_t*>(x);
+  a.out = p.k_splits > 1 ? static_cast<float*>(workspace) : y;
+  a.err = s->err;
+  a.N = N;
+  a.K = K;
+  a.nsb = K / 256;
+  a.k_splits = p.k_splits;
+  a.sb_base = a.nsb / p.k_splits;
+  a.sb_rem = a.nsb % p.k_splits;
+  a.row_streams = p.row_streams;
+  a.tpr = p.threads / p.row_streams;
+  a.stages = p.stages;
+  a.grid_rows = p.grid_rows;
+  a.slot_bytes = uint32_t(p.row_streams * p.rows_per_stream * p.sb_per_split * 144);
+
+  switch (M) {
+    case 1: st = launch_gemv_t<1, 4, 4>(a, p, dev, *s, stream); break;
+    case 2: st = launch_gemv_t<2, 2, 4>(a, p, dev, *s, stream); break;
+    case 3: st = launch_gemv_t<3, 1, 2>(a, p, dev, *s, stream); break;
+    case 4: st = launch_gemv_t<4, 1, 2>(a, p, dev, *s, stream); break;
+    default: st = launch_gemv_t<5, 1, 2>(a, p, dev, *s, stream); break;
+  }
+  if (st != Q4D_OK) return st;
+  if (p.k_splits > 1) {
+    const long long mn = (long long)M * N;
+    const int blocks = int(std::min<long long>((mn + 255) / 256, 4LL * s->num_sms));
+    q4d::q4_gemv_splitk_reduce<<<blocks, 256, 0, stream>>>(static_cast<const float*>(workspace), y,
+                                                          mn, p.k_splits);
+  }
+  if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
+  return Q4D_OK;
+}
+
+q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out, int ctx_len,
+                     int n_q, int n_kv, int head_dim, int M, int kv_stride, float scale,
+                     cudaStream_t stream, void* workspace, size_t workspace_bytes,
+                     bool library_ws) {
+  q4d_status st = check_attn_shape(ctx_len, n_q, n_kv, head_dim, M, kv_stride, scale);
+  if (st != Q4D_OK) return st;
+  if (!Q || !Kq4 || !Vq4 || !out) return Q4D_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(Kq4, 16) || !aligned(Vq4, 16) || !aligned(out, 4))
+    return Q4D_ERR_MISALIGNED;
+  if (workspace && !aligned(workspace, 16)) return Q4D_ERR_MISALIGNED;
+
+  int dev = 0;
+  DeviceState* s = nullptr;
+  if ((st = current_device(&dev, &s)) != Q4D_OK) return st;
+  q4d_attn_plan p;
+  if ((st = q4d_plan_attn(ctx_len, n_q, n_kv, head_dim, M, s->num_sms, &p)) != Q4D_OK) return st;
+  if (p.smem_bytes > size_t(s->smem_optin)) return Q4D_ERR_UNSUPPORTED_SHAPE;
+  if (library_ws) {
+    if ((st = library_workspace(*s, p.workspace_bytes, &workspace)) != Q4D_OK) return st;
+  } else if (p.workspace_bytes > 0 && (!workspace || workspace_bytes < p.workspace_bytes)) {
+    return Q4D_ERR_WORKSPACE;
+  }
+
+  q4d::AttnArgs a;
+  a.Q = static_cast<const uint16_t*>(Q);
+  a.K = static_cast<const uint8_t*>(Kq4);
+  a.V = static_cast<const uint8_t*>(Vq4);
+  a.out = out;
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_ml = a.ws_o ? a.ws_o + size_t(p.n_splits) * M * n_q * 256 : nullptr;
+  a.err = s->err;
+  a.ctx_len = ctx_len;
+  a.n_q = n_q;
+  a.n_kv = n_kv;
+  a.M = M;
+  a.g = n_q / n_kv;
+  a.kv_stride = kv_stride;
+  a.scale = scale;
+  a.n_splits = p.n_splits;
+  a.split_tokens = p.split_tokens;
+  a.rows_per_cta = p.rows_per_cta;
+  a.stages = p.stages;
+
+  static std::atomic<bool> smem_set[kMaxDevices];
+  if ((st = allow_smem(q4d::q4kv_attn_split_kernel, dev, *s, smem_set)) != Q4D_OK) return st;
+  dim3 grid(p.n_splits, n_kv, p.row_groups);
+  q4d::q4kv_attn_split_kernel<<<grid, p.threads, p.smem_bytes, stream>>>(a);
+  if (p.n_splits > 1) q4d::q4kv_attn_merge_kernel<<<M * n_q, 256, 0, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
+  return Q4D_OK;
+}
+
+int planning_sms() {
+  int dev = 0;
+  DeviceState* s = nullptr;
+  if (current_device(&dev, &s) != Q4D_OK) return kPlanFallbackSms;
+  return s->num_sms;
+}
+
+}  // namespace
+
+extern "C" {
+
+int q4d_version(void) { return Q4D_VERSION; }
+
+const char* q4d_status_string(int status) {
+  switch (status) {
+    case Q4D_OK: return "ok";
+    case Q4D_ERR_INVALID_ARG: return "invalid argument";
+    case Q4D_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case Q4D_ERR_MISALIGNED: return "misaligned pointer";
+    case Q4D_ERR_WORKSPACE: return "workspace missing or too small";
+    case Q4D_ERR_CUDA: return "CUDA runtime error";
+    case Q4D_ERR_DEVICE_TIMEOUT: return "in-kernel wait timed out";
+    default: return "unknown status";
+  }
+}
+
+q4d_status q4d_plan_gemv(int M, int N, int K, int num_sms, q4d_gemv_plan* plan) {
+  if (!plan || num_sms < 1) return Q4D_ERR_INVALID_ARG;
+  q4d_status st = check_gemv_shape(M, N, K);
+  if (st != Q4D_OK) return st;
+  const int nsb = K / 256;
+  const int W = gemv_words_per_thread(M);
+  const int tps = 32 / W;
+  const int rsr = gemv_rows_per_stream(M);
+  // K ranges: as few as fit the thread budget ...
+  int ks = 1;
+  while (round_up((long long)ceil_div(nsb, ks) * tps, 32) > q4d::kGemvMaxThreads) ++ks;
+  // ... and more while there are fewer (row, range) units than SMs.
+  while (ks < nsb && (long long)N * ks < num_sms) ++ks;
+  const int sbs = ceil_div(nsb, ks);
+  const int tpr = int(round_up((long long)sbs * tps, 32));
+  int grid_rows = std::max(1, num_sms / ks);
+  if (grid_rows > N) grid_rows = N;
+  const int rows_per_cta = ceil_div(N, grid_rows);
+  int streams = std::max(1, q4d::kGemvMaxThreads / tpr);
+  streams = std::min(streams, std::max(1, ceil_div(rows_per_cta, rsr)));
+  const size_t slot = size_t(streams) * rsr * sbs * 144;
+  int stages = int(kGemvStageBudget / slot);
+  stages = std::max(2, std::min(12, stages));
+  const int VPAD = q4d::next_pow2(rsr * M);
+  const int threads = streams * tpr;
+  plan->k_splits = ks;
+  plan->sb_per_split = sbs;
+  plan->words_per_thread = W;
+  plan->row_streams = streams;
+  plan->rows_per_stream = rsr;
+  plan->stages = stages;
+  plan->threads = threads;
+  plan->grid_rows = grid_rows;
+  plan->smem_bytes = stages * slot + size_t(2) * (threads / 32) * VPAD * 4 + size_t(stages) * 8;
+  plan->workspace_bytes = ks > 1 ? size_t(ks) * M * N * 4 : 0;
+  return Q4D_OK;
+}
+
+q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
+                         int num_sms, q4d_attn_plan* plan) {
+  if (!plan || num_sms < 1) return Q4D_ERR_INVALID_ARG;
+  q4d_status st = check_attn_shape(ctx_len, n_q_heads, n_kv_heads, head_dim, M, ctx_len, 1.0f);
+  if (st != Q4D_OK) return st;
+  const int TT = q4d::kAttnTileTokens;
+  const int rows_all = (n_q_heads / n_kv_heads) * M;
+  const int row_groups = ceil_div(rows_all, q4d::kAttnMaxRows);
+  const int rows_per_cta = ceil_div(rows_all, row_groups);
+  const long long ctas_per_split = (long long)n_kv_heads * row_groups;
+  int n_splits = int(std::max<long long>(1, (2LL * num_sms + ctas_per_split - 1) / ctas_per_split));
+  n_splits = std::min(n_splits, std::max(1, ceil_div(ctx_len, 4 * TT)));
+  const int split_tokens = int(round_up(ceil_div(ctx_len, n_splits), TT));
+  n_splits = ceil_div(ctx_len, split_tokens);
+  const int stages = 3;
+  plan->n_splits = n_splits;
+  plan->split_tokens = split_tokens;
+  plan->tile_tokens = TT;
+  plan->row_groups = row_groups;
+  plan->rows_per_cta = rows_per_cta;
+  plan->stages = stages;
+  plan->threads = q4d::kAttnThreads;
+  plan->smem_bytes = size_t(q4d::kAttnMaxRows) * q4d::kHeadDim * 4 +
+                     size_t(stages) * 2 * TT * q4d::kRowBytes + size_t(TT) * q4d::kAttnMaxRows * 4 +
+                     3 * q4d::kAttnMaxRows * 4 + size_t(stages) * 8;
+  plan->workspace_bytes =
+      n_splits > 1 ? size_t(n_splits) * M * n_q_heads * (q4d::kHeadDim + 2) * 4 : 0;
+  return Q4D_OK;
+}
+
+size_t q4d_gemv_workspace_bytes(int M, int N, int K) {
+  q4d_gemv_plan p;
+  if (q4d_plan_gemv(M, N, K, planning_sms(), &p) != Q4D_OK) return 0;
+  return p.workspace_bytes;
+}
+
+size_t q4d_attn_workspace_bytes(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M) {
+  q4d_attn_plan p;
+  if (q4d_plan_attn(ctx_len, n_q_heads, n_kv_heads, head_dim, M, planning_sms(), &p) != Q4D_OK)
+    return 0;
+  return p.workspace_bytes;
+}
+
+q4d_status q4_gemv(const void* W_q4, const void* x, float* y, int M, int N, int K) {
+  return gemv_impl(W_q4, x, y, M, N, K, nullptr, nullptr, 0, true);
+}
+
+q4d_status q4_gemv_ex(const void* W_q4, const void* x, float* y, int M, int N, int K,
+                      void* stream, void* workspace, size_t workspace_bytes) {
+  return gemv_impl(W_q4, x, y, M, N, K, static_cast<cudaStream_t>(stream), workspace,
+                   workspace_bytes, false);
+}
+
+q4d_status q4kv_attn_decode(const void* Q, const void* Kq4, const void* Vq4, float* out,
+                            int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M) {
+  return attn_impl(Q, Kq4, Vq4, out, ctx_len, n_q_heads, n_kv_heads, head_dim, M, ctx_len, 1.0f,
+                   nullptr, nullptr, 0, true);
+}
+
+q4d_status q4kv_attn_decode_ex(const void* Q, const void* Kq4, const void* Vq4, float* out,
+                               int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
+                               int kv_stride_tokens, float softmax_scale, void* stream,
+                               void* workspace, size_t workspace_bytes) {
+  return attn_impl(Q, Kq4, Vq4, out, ctx_len, n_q_heads, n_kv_heads, head_dim, M,
+                   kv_stride_tokens, softmax_scale, static_cast<cudaStream_t>(stream), workspace,
+                   workspace_bytes, false);
+}
+
+q4d_status q4d_device_error(int reset) {
+  int dev = 0;
+  DeviceState* s = nullptr;
+  q4d_status st = current_device(&dev, &s);
+  if (st != Q4D_OK) return st;
+  unsigned word = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpy(&word, s->err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return Q4D_ERR_CUDA;
+  }
+  if (reset && word) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(s->err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return Q4D_ERR_CUDA;
+  }
+  return word ? Q4D_ERR_DEVICE_TIMEOUT : Q4D_OK;
+}
+
+}  // extern "C"

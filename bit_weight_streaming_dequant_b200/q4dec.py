@@ -1,0 +1,209 @@
+"""Python binding of libq4dec: argument marshalling only.
+
+Every step of the decode path runs in the library's CUDA kernels; this module
+checks tensors, takes raw device pointers and the current torch stream, and
+calls the C ABI (``include/q4dec.h``).  There is no fallback: if the shared
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libq4dec.so")
+
+STATUS = {
+    0: "Q4D_OK",
+    1: "Q4D_ERR_INVALID_ARG",
+    2: "Q4D_ERR_UNSUPPORTED_SHAPE",
+    3: "Q4D_ERR_MISALIGNED",
+    4: "Q4D_ERR_WORKSPACE",
+    5: "Q4D_ERR_CUDA",
+    6: "Q4D_ERR_DEVICE_TIMEOUT",
+}
+
+EXPORTS = (
+    "q4d_version", "q4d_status_string",
+    "q4_gemv", "q4_gemv_ex", "q4d_gemv_workspace_bytes",
+    "q4kv_attn_decode", "q4kv_attn_decode_ex", "q4d_attn_workspace_bytes",
+    "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
+)
+
+
+class Q4DecError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({lib().q4d_status_string(status).decode()})")
+
+
+class GemvPlan(ctypes.Structure):
+    _fields_ = [("k_splits", ctypes.c_int), ("sb_per_split", ctypes.c_int),
+                ("words_per_thread", ctypes.c_int), ("row_streams", ctypes.c_int),
+                ("rows_per_stream", ctypes.c_int), ("stages", ctypes.c_int),
+                ("threads", ctypes.c_int), ("grid_rows", ctypes.c_int),
+                ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class AttnPlan(ctypes.Structure):
+    _fields_ = [("n_splits", ctypes.c_int), ("split_tokens", ctypes.c_int),
+                ("tile_tokens", ctypes.c_int), ("row_groups", ctypes.c_int),
+                ("rows_per_cta", ctypes.c_int), ("stages", ctypes.c_int),
+                ("threads", ctypes.c_int), ("smem_bytes", ctypes.c_size_t),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libq4dec.so (built in-tree); raise if it is not there."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m bit_weight_streaming_dequant_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    L.q4d_version.restype = i
+    L.q4d_status_string.argtypes = [i]
+    L.q4d_status_string.restype = ctypes.c_char_p
+    L.q4_gemv.argtypes = [vp, vp, vp, i, i, i]
+    L.q4_gemv_ex.argtypes = [vp, vp, vp, i, i, i, vp, vp, sz]
+    L.q4d_gemv_workspace_bytes.argtypes = [i, i, i]
+    L.q4d_gemv_workspace_bytes.restype = sz
+    L.q4kv_attn_decode.argtypes = [vp, vp, vp, vp, i, i, i, i, i]
+    L.q4kv_attn_decode_ex.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, sz]
+    L.q4d_attn_workspace_bytes.argtypes = [i, i, i, i, i]
+    L.q4d_attn_workspace_bytes.restype = sz
+    L.q4d_plan_gemv.argtypes = [i, i, i, i, ctypes.POINTER(GemvPlan)]
+    L.q4d_plan_attn.argtypes = [i, i, i, i, i, i, ctypes.POINTER(AttnPlan)]
+    L.q4d_device_error.argtypes = [i]
+    for fn in ("q4_gemv", "q4_gemv_ex", "q4kv_attn_decode", "q4kv_attn_decode_ex",
+               "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error"):
+        getattr(L, fn).restype = i
+    _lib = L
+    return L
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise Q4DecError(status, what)
+
+
+def plan_gemv(M: int, N: int, K: int, num_sms: int) -> GemvPlan:
+    p = GemvPlan()
+    _check(lib().q4d_plan_gemv(M, N, K, num_sms, ctypes.byref(p)), "q4d_plan_gemv")
+    return p
+
+
+def plan_attn(ctx_len: int, n_q_heads: int, n_kv_heads: int, head_dim: int, M: int,
+              num_sms: int) -> AttnPlan:
+    p = AttnPlan()
+    _check(lib().q4d_plan_attn(ctx_len, n_q_heads, n_kv_heads, head_dim, M, num_sms,
+                               ctypes.byref(p)), "q4d_plan_attn")
+    return p
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _dev_tensor(t, dtype, what):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{what} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    return t
+
+
+def _stream_ptr(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _workspace(nbytes: int, device, workspace):
+    torch = _torch()
+    if nbytes == 0:
+        return None
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError(f"workspace smaller than the {nbytes} bytes needed")
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def q4_gemv(W, x, y=None, *, N: int, K: int, stream=None, workspace=None):
+    """y[M][N] (fp32) = dequant(W)[N][K] @ x[M][K]^T via ``q4_gemv_ex``.
+
+    ``W``: uint8 CUDA tensor with N*K/256*144 bytes (super-block layout);
+    ``x``: bf16 CUDA tensor [M][K]; ``y``: optional fp32 [M][N] output.
+    """
+    torch = _torch()
+    _dev_tensor(W, torch.uint8, "W")
+    _dev_tensor(x, torch.bfloat16, "x")
+    if x.dim() != 2 or x.shape[1] != K:
+        raise ValueError("x must be [M][K]")
+    M = x.shape[0]
+    if W.numel() != N * (K // 256) * 144:
+        raise ValueError("W has the wrong number of bytes for N x K")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _dev_tensor(y, torch.float32, "y")
+    if tuple(y.shape) != (M, N):
+        raise ValueError("y must be [M][N]")
+    with torch.cuda.device(x.device):
+        need = lib().q4d_gemv_workspace_bytes(M, N, K)
+        ws = _workspace(need, x.device, workspace)
+        st = lib().q4_gemv_ex(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K,
+                              _stream_ptr(stream), None if ws is None else ws.data_ptr(), need)
+    _check(st, "q4_gemv")
+    return y
+
+
+def q4kv_attn_decode(Q, Kq4, Vq4, out=None, *, ctx_len: int, n_kv_heads: int,
+                     head_dim: int = 256, kv_stride_tokens: int | None = None,
+                     softmax_scale: float = 1.0, stream=None, workspace=None):
+    """Causal GQA decode attention over Q4_0 K/V via ``q4kv_attn_decode_ex``.
+
+    ``Q``: bf16 [M][n_q_heads][head_dim]; ``Kq4``/``Vq4``: uint8 caches of
+    ``n_kv_heads * kv_stride_tokens`` super-blocks; returns fp32 ``out`` of
+    Q's shape.
+    """
+    torch = _torch()
+    _dev_tensor(Q, torch.bfloat16, "Q")
+    _dev_tensor(Kq4, torch.uint8, "Kq4")
+    _dev_tensor(Vq4, torch.uint8, "Vq4")
+    if Q.dim() != 3 or Q.shape[2] != head_dim:
+        raise ValueError("Q must be [M][n_q_heads][head_dim]")
+    M, n_q = Q.shape[0], Q.shape[1]
+    stride = ctx_len if kv_stride_tokens is None else kv_stride_tokens
+    need_bytes = n_kv_heads * stride * (head_dim // 256) * 144
+    if Kq4.numel() < need_bytes or Vq4.numel() < need_bytes:
+        raise ValueError("K/V caches are smaller than n_kv_heads * kv_stride_tokens rows")
+    if out is None:
+        out = torch.empty((M, n_q, head_dim), dtype=torch.float32, device=Q.device)
+    _dev_tensor(out, torch.float32, "out")
+    if tuple(out.shape) != (M, n_q, head_dim):
+        raise ValueError("out must match Q's shape")
+    with torch.cuda.device(Q.device):
+        need = lib().q4d_attn_workspace_bytes(ctx_len, n_q, n_kv_heads, head_dim, M)
+        ws = _workspace(need, Q.device, workspace)
+        st = lib().q4kv_attn_decode_ex(Q.data_ptr(), Kq4.data_ptr(), Vq4.data_ptr(),
+                                       out.data_ptr(), ctx_len, n_q, n_kv_heads, head_dim, M,
+                                       stride, float(softmax_scale), _stream_ptr(stream),
+                                       None if ws is None else ws.data_ptr(), need)
+    _check(st, "q4kv_attn_decode")
+    return out
+
+
+def device_error(reset: bool = False) -> int:
+    """Synchronise and read the device error word (0 = clear)."""
+    return lib().q4d_device_error(1 if reset else 0)

@@ -1,0 +1,182 @@
+/*
+ * libq4dec -- Q4_0 decode hot path for NVIDIA B200 (sm_100a).
+ *
+ * Two operations make up one decode step of a quantised dense model:
+ *
+ *  1. q4_gemv: a dequant-fused GEMV / skinny GEMM that streams Q4_0 weights
+ *     once for M = 1..5 activation rows.  The pages ("Qwen3.8-27B at 256K on
+ *     a 24GB RTX PRO 4000 SFF (432 GB/s): 50 tok/s with MTP", the paragraph
+ *     beginning "NVIDIA quotes 432 GB/s") put decode time into "repeatedly
+ *     streaming quantized weights"; M = 1 is plain decode and M = 2..5 is the
+ *     target model verifying a drafted block of up to four tokens
+ *     ("Qwen3.8-27B on RTX 4090: 5,000 tok/s Prefill Reproduced", section
+ *     "MTP helps ordinary prose, but acceptance controls the gain").
+ *
+ *  2. q4kv_attn_decode: causal GQA flash-decode attention over a K/V cache
+ *     stored in the same Q4_0 layout (same first page: "With Q4 K and V ..."
+ *     and "the 16 attention layers add increasingly expensive KV reads as
+ *     context fills").  The context is split across the SMs and the partial
+ *     softmax states are combined by a log-sum-exp merge.
+ *
+ * ---------------------------------------------------------------------------
+ * Storage layout (identical for weights and for the K/V cache)
+ *
+ *   Q4_0 block   : 32 elements, one IEEE fp16 scale d, 16 bytes of nibbles.
+ *                  Byte j (0..15) holds element j in bits 0..3 and element
+ *                  j+16 in bits 4..7.  Element value = d * (q - 8), q in 0..15.
+ *   super-block  : 256 consecutive elements = 8 blocks in 144 bytes:
+ *                  bytes [16*b, 16*b+16) = nibbles of block b (b = 0..7),
+ *                  bytes [128+2*b, 128+2*b+2) = fp16 scale of block b
+ *                  (little endian).  144 is a multiple of 16, so every
+ *                  super-block starts on a 16-byte boundary.
+ *   weight W[N][K]: row n = K/256 consecutive super-blocks; super-block s of
+ *                  row n starts at byte (n*(K/256) + s) * 144.
+ *   K/V cache    : one super-block per (KV head, token) (head_dim = 256);
+ *                  token t of KV head h starts at byte (h*kv_stride + t)*144.
+ *
+ * Conventions
+ *   - Every pointer passed to a compute entry point is a DEVICE pointer of
+ *     the current CUDA device, owned by the caller; the library never frees
+ *     or retains it.  W, x, Q, K, V and workspace must be 16-byte aligned;
+ *     y and out must be 4-byte aligned.
+ *   - "stream" is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; the library never
+ *     synchronises the host on the compute path.
+ *   - Arguments are validated before anything is launched; on any error
+ *     nothing is launched and the outputs are untouched.  Launch failures
+ *     return Q4D_ERR_CUDA.  Faults during execution surface at the caller's
+ *     next synchronisation.  Every wait inside a kernel is bounded in time;
+ *     a wait that runs out sets a device error word readable through
+ *     q4d_device_error().
+ *   - Results are fp32.  Accumulation is fp32; the kernels use no atomics on
+ *     results, so repeated calls with the same inputs and the same device
+ *     give bitwise identical outputs.
+ */
+#ifndef Q4DEC_H
+#define Q4DEC_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define Q4D_VERSION 10000 /* 1.0.0 */
+
+typedef enum {
+  Q4D_OK = 0,
+  Q4D_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad scale */
+  Q4D_ERR_UNSUPPORTED_SHAPE = 2, /* M outside 1..5, K % 256 != 0, head_dim != 256,
+                                    n_q % n_kv != 0, ctx_len < M, stride < ctx_len */
+  Q4D_ERR_MISALIGNED = 3,        /* pointer alignment below the stated minimum */
+  Q4D_ERR_WORKSPACE = 4,         /* workspace missing or smaller than required */
+  Q4D_ERR_CUDA = 5,              /* CUDA runtime error (launch, device query, malloc) */
+  Q4D_ERR_DEVICE_TIMEOUT = 6     /* a bounded in-kernel wait ran out (q4d_device_error) */
+} q4d_status;
+
+/* Library version, Q4D_VERSION of the build. */
+int q4d_version(void);
+
+/* Static, never-NULL description of a status code (unknown codes included). */
+const char* q4d_status_string(int status);
+
+/* ------------------------------------------------------------------ GEMV --
+ * y[m][n] = sum_k (d * (q - 8))[n][k] * x[m][k]   for m < M, n < N.
+ *
+ *   W_q4 : N rows x K elements of Q4_0 in the super-block layout, N*K/256*144 bytes.
+ *   x    : bf16 [M][K] row-major (M activation rows sharing one weight stream).
+ *   y    : fp32 [M][N] row-major, fully overwritten.
+ *   Requirements: 1 <= M <= 5, N >= 1, K >= 256, K % 256 == 0.
+ *
+ * q4_gemv runs on the legacy default stream with a workspace owned by the
+ * library (per device, allocated on first need and grown when a larger one
+ * is needed -- that call synchronises the device and must not be captured
+ * into a CUDA graph).  q4_gemv_ex takes the stream and a caller-owned
+ * workspace of at least q4d_gemv_workspace_bytes(M, N, K) bytes (it may be
+ * NULL when that size is 0); it never allocates.
+ */
+q4d_status q4_gemv(const void* W_q4, const void* x, float* y, int M, int N, int K);
+q4d_status q4_gemv_ex(const void* W_q4, const void* x, float* y, int M, int N, int K,
+                      void* stream, void* workspace, size_t workspace_bytes);
+/* Workspace bytes q4_gemv_ex needs on the CURRENT device (depends on its SM
+ * count; a host without a usable device is planned for 148 SMs).  Returns 0
+ * for invalid shapes as well as for shapes that need none. */
+size_t q4d_gemv_workspace_bytes(int M, int N, int K);
+
+/* ------------------------------------------------------------- attention --
+ * For draft row m (absolute position p_m = ctx_len - M + m) and query head h
+ * (KV head kh = h / (n_q_heads / n_kv_heads)):
+ *   s[t]        = softmax_scale * sum_c Q[m][h][c] * Khat[kh][t][c],  t <= p_m
+ *   out[m][h][:] = sum_t softmax(s)[t] * Vhat[kh][t][:]
+ * where Khat / Vhat are the dequantised caches.  Tokens t > p_m are masked
+ * (the M draft tokens are already in the cache; row M-1 sees all ctx_len).
+ *
+ *   Q    : bf16 [M][n_q_heads][head_dim].
+ *   Kq4, Vq4 : [n_kv_heads][kv_stride] super-blocks (one per token, 144 B).
+ *   out  : fp32 [M][n_q_heads][head_dim], fully overwritten.
+ *   Requirements: head_dim == 256, 1 <= M <= 5, n_kv_heads >= 1,
+ *                 n_q_heads % n_kv_heads == 0, ctx_len >= M,
+ *                 kv_stride_tokens >= ctx_len, softmax_scale finite.
+ *
+ * q4kv_attn_decode uses kv_stride = ctx_len, softmax_scale = 1 (queries are
+ * pre-scaled), the legacy default stream and a library-owned workspace (same
+ * rules as q4_gemv).  The _ex form takes all of them explicitly and never
+ * allocates; workspace must hold q4d_attn_workspace_bytes(...) bytes.
+ */
+q4d_status q4kv_attn_decode(const void* Q, const void* Kq4, const void* Vq4, float* out,
+                            int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M);
+q4d_status q4kv_attn_decode_ex(const void* Q, const void* Kq4, const void* Vq4, float* out,
+                               int ctx_len, int n_q_heads, int n_kv_heads, int head_dim,
+                               int M, int kv_stride_tokens, float softmax_scale,
+                               void* stream, void* workspace, size_t workspace_bytes);
+/* Workspace bytes q4kv_attn_decode_ex needs on the current device (0 for
+ * invalid shapes and for shapes handled in one pass). */
+size_t q4d_attn_workspace_bytes(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim,
+                                int M);
+
+/* ------------------------------------------------------- launch planning --
+ * Pure host functions (no CUDA call) exposing how a call is partitioned on
+ * a device with num_sms SMs; the compute entry points use exactly these.
+ */
+typedef struct {
+  int k_splits;          /* K is cut into this many ranges (1 = no split)        */
+  int sb_per_split;      /* super-blocks in the longest range                    */
+  int words_per_thread;  /* 32-bit nibble words each thread owns per row         */
+  int row_streams;       /* independent row streams per CTA                      */
+  int rows_per_stream;   /* rows each stream handles per pipeline stage          */
+  int stages;            /* shared-memory pipeline depth                         */
+  int threads;           /* threads per CTA                                      */
+  int grid_rows;         /* CTAs per K range (grid = grid_rows * k_splits)       */
+  size_t smem_bytes;     /* dynamic shared memory per CTA                        */
+  size_t workspace_bytes;/* fp32 partials, k_splits * M * N * 4 when k_splits > 1 */
+} q4d_gemv_plan;
+
+typedef struct {
+  int n_splits;          /* context splits per KV head                           */
+  int split_tokens;      /* tokens per split (multiple of tile_tokens)           */
+  int tile_tokens;       /* tokens per shared-memory tile                        */
+  int row_groups;        /* CTAs per (KV head, split) when g*M exceeds one CTA   */
+  int rows_per_cta;      /* query rows (draft rows x grouped heads) per CTA      */
+  int stages;            /* shared-memory pipeline depth                         */
+  int threads;           /* threads per CTA                                      */
+  size_t smem_bytes;     /* dynamic shared memory per CTA                        */
+  size_t workspace_bytes;/* partial (max, sum, o[256]) states for the merge      */
+} q4d_attn_plan;
+
+q4d_status q4d_plan_gemv(int M, int N, int K, int num_sms, q4d_gemv_plan* plan);
+q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
+                         int num_sms, q4d_attn_plan* plan);
+
+/* ------------------------------------------------------- device errors --
+ * Synchronises the current device and reads the library's device error word
+ * (set when an in-kernel wait exceeded its time limit).  Returns Q4D_OK when
+ * clear, Q4D_ERR_DEVICE_TIMEOUT when set, Q4D_ERR_CUDA if the device cannot
+ * be queried.  reset != 0 clears the word after reading.
+ */
+q4d_status q4d_device_error(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4DEC_H */

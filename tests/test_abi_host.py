@@ -1,0 +1,110 @@
+"""Host-only checks of libq4dec: it loads, exports every symbol the header
+declares, validates arguments before touching CUDA, and plans launches."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_weight_streaming_dequant_b200 import q4dec
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "q4dec.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(q4[a-z0-9_]*)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_function():
+    L = q4dec.lib()
+    declared = _declared_functions()
+    assert set(declared) == set(q4dec.EXPORTS)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings():
+    L = q4dec.lib()
+    assert L.q4d_version() == 10000
+    for code in range(7):
+        assert L.q4d_status_string(code)
+    assert L.q4d_status_string(99) == b"unknown status"
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("M,N,K,code", [
+    (0, 16, 256, 2), (6, 16, 256, 2), (1, 16, 100, 2), (1, 16, 0, 2),
+    (1, 0, 256, 1), (1, -3, 256, 1), (1, 16, -256, 1),
+])
+def test_gemv_rejects_bad_shapes_without_cuda(M, N, K, code):
+    L = q4dec.lib()
+    assert L.q4_gemv_ex(FAKE, FAKE, FAKE, M, N, K, None, None, 0) == code
+    assert L.q4_gemv(FAKE, FAKE, FAKE, M, N, K) == code
+
+
+def test_gemv_rejects_null_and_misaligned_pointers():
+    L = q4dec.lib()
+    assert L.q4_gemv_ex(None, FAKE, FAKE, 1, 16, 256, None, None, 0) == 1
+    assert L.q4_gemv_ex(FAKE, None, FAKE, 1, 16, 256, None, None, 0) == 1
+    assert L.q4_gemv_ex(FAKE, FAKE, None, 1, 16, 256, None, None, 0) == 1
+    assert L.q4_gemv_ex(FAKE + 8, FAKE, FAKE, 1, 16, 256, None, None, 0) == 3
+    assert L.q4_gemv_ex(FAKE, FAKE + 2, FAKE, 1, 16, 256, None, None, 0) == 3
+    assert L.q4_gemv_ex(FAKE, FAKE, FAKE + 2, 1, 16, 256, None, None, 0) == 3
+    assert L.q4_gemv_ex(FAKE, FAKE, FAKE, 1, 16, 256, None, FAKE + 4, 64) == 3
+
+
+@pytest.mark.parametrize("ctx,nq,nkv,hd,M,stride,scale,code", [
+    (100, 24, 4, 128, 1, 100, 1.0, 2),    # head_dim != 256
+    (100, 24, 5, 256, 1, 100, 1.0, 2),    # n_q % n_kv
+    (4, 24, 4, 256, 5, 4, 1.0, 2),        # ctx_len < M
+    (100, 24, 4, 256, 6, 100, 1.0, 2),    # M > 5
+    (100, 24, 4, 256, 0, 100, 1.0, 2),    # M < 1
+    (100, 24, 4, 256, 1, 99, 1.0, 2),     # stride < ctx_len
+    (0, 24, 4, 256, 1, 0, 1.0, 1),        # empty context
+    (100, 0, 4, 256, 1, 100, 1.0, 1),
+    (100, 24, 0, 256, 1, 100, 1.0, 1),
+    (100, 24, 4, 256, 1, 100, float("nan"), 1),
+    (100, 24, 4, 256, 1, 100, float("inf"), 1),
+])
+def test_attn_rejects_bad_arguments_without_cuda(ctx, nq, nkv, hd, M, stride, scale, code):
+    L = q4dec.lib()
+    assert L.q4kv_attn_decode_ex(FAKE, FAKE, FAKE, FAKE, ctx, nq, nkv, hd, M, stride,
+                                 ctypes.c_float(scale), None, None, 0) == code
+
+
+def test_attn_rejects_null_and_misaligned():
+    L = q4dec.lib()
+    args = (4096, 24, 4, 256, 1, 4096, ctypes.c_float(1.0), None, None, 0)
+    assert L.q4kv_attn_decode_ex(None, FAKE, FAKE, FAKE, *args) == 1
+    assert L.q4kv_attn_decode_ex(FAKE, FAKE, FAKE, None, *args) == 1
+    assert L.q4kv_attn_decode_ex(FAKE + 8, FAKE, FAKE, FAKE, *args) == 3
+    assert L.q4kv_attn_decode_ex(FAKE, FAKE + 4, FAKE, FAKE, *args) == 3
+    assert L.q4kv_attn_decode_ex(FAKE, FAKE, FAKE + 12, FAKE, *args) == 3
+    assert L.q4kv_attn_decode_ex(FAKE, FAKE, FAKE, FAKE + 1, *args) == 3
+
+
+def test_plan_rejects_bad_inputs():
+    L = q4dec.lib()
+    p = q4dec.GemvPlan()
+    assert L.q4d_plan_gemv(1, 16, 256, 0, ctypes.byref(p)) == 1
+    assert L.q4d_plan_gemv(1, 16, 256, 148, None) == 1
+    assert L.q4d_plan_gemv(7, 16, 256, 148, ctypes.byref(p)) == 2
+    a = q4dec.AttnPlan()
+    assert L.q4d_plan_attn(4096, 24, 4, 256, 1, 0, ctypes.byref(a)) == 1
+    assert L.q4d_plan_attn(4096, 24, 4, 64, 1, 148, ctypes.byref(a)) == 2
+
+
+def test_workspace_queries_without_device_use_the_fallback_plan():
+    L = q4dec.lib()
+    # invalid shapes report 0
+    assert L.q4d_gemv_workspace_bytes(0, 16, 256) == 0
+    assert L.q4d_attn_workspace_bytes(4096, 24, 5, 256, 1) == 0
+    # layer shapes need no split-K workspace; the long context needs merge space
+    assert L.q4d_gemv_workspace_bytes(1, 17408, 5120) == 0
+    assert L.q4d_attn_workspace_bytes(262144, 24, 4, 256, 5) > 0
