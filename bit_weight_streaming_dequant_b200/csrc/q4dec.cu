@@ -390,3 +390,66 @@ q4d_status q4d_device_error(int reset) {
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Allocation-free attention (q4kv_attn_decode_noalloc): the split states live
+// in this file-scope device array instead of a caller or library allocation.
+// In host code the name below is only a host-side stand-in; kernels get the
+// device address looked up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char q4d_noalloc_scratch[Q4D_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+struct NoAllocScratch {
+  std::atomic<bool> ready{false};
+  void* ptr = nullptr;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device, looked up once.
+q4d_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return Q4D_ERR_CUDA;
+  }
+  NoAllocScratch& s = g_noalloc[dev];
+  if (!s.ready.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!s.ready.load(std::memory_order_relaxed)) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, q4d_noalloc_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return Q4D_ERR_CUDA;
+      }
+      s.ptr = p;
+      s.ready.store(true, std::memory_order_release);
+    }
+  }
+  *out = s.ptr;
+  return Q4D_OK;
+}
+
+}  // namespace
+
+extern "C" q4d_status q4kv_attn_decode_noalloc(const void* Q, const void* Kq4, const void* Vq4,
+                                               float* out, int ctx_len, int n_q_heads,
+                                               int n_kv_heads, int head_dim, int M,
+                                               int kv_stride_tokens, float softmax_scale,
+                                               void* stream) {
+  // Reject bad arguments before touching CUDA, as the other entry points do.
+  q4d_status st = check_attn_shape(ctx_len, n_q_heads, n_kv_heads, head_dim, M,
+                                   kv_stride_tokens, softmax_scale);
+  if (st != Q4D_OK) return st;
+  if (!Q || !Kq4 || !Vq4 || !out) return Q4D_ERR_INVALID_ARG;
+  if (!aligned(Q, 16) || !aligned(Kq4, 16) || !aligned(Vq4, 16) || !aligned(out, 4))
+    return Q4D_ERR_MISALIGNED;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != Q4D_OK) return st;
+  // The workspace path never allocates; a plan needing more than the array
+  // holds comes back as Q4D_ERR_WORKSPACE before any launch.
+  return attn_impl(Q, Kq4, Vq4, out, ctx_len, n_q_heads, n_kv_heads, head_dim, M,
+                   kv_stride_tokens, softmax_scale, static_cast<cudaStream_t>(stream), scratch,
+                   Q4D_NOALLOC_SCRATCH_BYTES, false);
+}

@@ -28,6 +28,7 @@ EXPORTS = (
     "q4_gemv", "q4_gemv_ex", "q4d_gemv_workspace_bytes",
     "q4kv_attn_decode", "q4kv_attn_decode_ex", "q4d_attn_workspace_bytes",
     "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
+    "q4kv_attn_decode_noalloc",
 )
 
 
@@ -80,8 +81,10 @@ def lib() -> ctypes.CDLL:
     L.q4d_plan_gemv.argtypes = [i, i, i, i, ctypes.POINTER(GemvPlan)]
     L.q4d_plan_attn.argtypes = [i, i, i, i, i, i, ctypes.POINTER(AttnPlan)]
     L.q4d_device_error.argtypes = [i]
+    L.q4kv_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     for fn in ("q4_gemv", "q4_gemv_ex", "q4kv_attn_decode", "q4kv_attn_decode_ex",
-               "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error"):
+               "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
+               "q4kv_attn_decode_noalloc"):
         getattr(L, fn).restype = i
     _lib = L
     return L
@@ -201,6 +204,37 @@ def q4kv_attn_decode(Q, Kq4, Vq4, out=None, *, ctx_len: int, n_kv_heads: int,
                                        stride, float(softmax_scale), _stream_ptr(stream),
                                        None if ws is None else ws.data_ptr(), need)
     _check(st, "q4kv_attn_decode")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def q4kv_attn_decode_noalloc(Q, Kq4, Vq4, out, *, ctx_len: int, n_kv_heads: int,
+                             head_dim: int = 256, kv_stride_tokens: int | None = None,
+                             softmax_scale: float = 1.0, stream=None):
+    """Decode attention through ``q4kv_attn_decode_noalloc``: for callers that
+    may not allocate device memory while running.  Neither this wrapper nor the
+    library allocates; ``out`` (fp32, Q's shape) must be given.  The library's
+    16 MiB static scratch is shared by all such calls, so calls that overlap on
+    the GPU race."""
+    torch = _torch()
+    _dev_tensor(Q, torch.bfloat16, "Q")
+    _dev_tensor(Kq4, torch.uint8, "Kq4")
+    _dev_tensor(Vq4, torch.uint8, "Vq4")
+    _dev_tensor(out, torch.float32, "out")
+    if Q.dim() != 3 or Q.shape[2] != head_dim or tuple(out.shape) != tuple(Q.shape):
+        raise ValueError("Q must be [M][n_q_heads][head_dim] and out must match it")
+    M, n_q = Q.shape[0], Q.shape[1]
+    stride = ctx_len if kv_stride_tokens is None else kv_stride_tokens
+    need_bytes = n_kv_heads * stride * (head_dim // 256) * 144
+    if Kq4.numel() < need_bytes or Vq4.numel() < need_bytes:
+        raise ValueError("K/V caches are smaller than n_kv_heads * kv_stride_tokens rows")
+    with torch.cuda.device(Q.device):
+        st = lib().q4kv_attn_decode_noalloc(Q.data_ptr(), Kq4.data_ptr(), Vq4.data_ptr(),
+                                            out.data_ptr(), ctx_len, n_q, n_kv_heads, head_dim,
+                                            M, stride, float(softmax_scale), _stream_ptr(stream))
+    _check(st, "q4kv_attn_decode_noalloc")
     return out
 
 

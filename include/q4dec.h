@@ -134,6 +134,38 @@ q4d_status q4kv_attn_decode_ex(const void* Q, const void* Kq4, const void* Vq4, 
 size_t q4d_attn_workspace_bytes(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim,
                                 int M);
 
+/* ------------------------------------------- attention, allocation-free --
+ * The paper has no counterpart to this entry point; it exists for deployment.
+ *
+ * Some callers may not allocate device memory once they are running: runtimes
+ * that reserve all device memory in their own arena at start-up and forbid
+ * allocation afterwards, and latency-critical decode loops in which a
+ * cudaMalloc/cudaFree would synchronise the device and stall the token.  They
+ * cannot use q4kv_attn_decode (which may allocate its workspace) and may have
+ * no spare buffer to hand to the _ex form.  This entry point takes no
+ * workspace and allocates nothing: the per-split softmax states live in one
+ * statically sized device array of Q4D_NOALLOC_SCRATCH_BYTES inside this
+ * library, which every GPU that loads the library holds until the process
+ * exits.
+ *
+ *   - Arguments, layout and results are those of q4kv_attn_decode_ex without
+ *     the workspace.  A call needing more scratch than the array holds
+ *     (q4d_attn_workspace_bytes > Q4D_NOALLOC_SCRATCH_BYTES) returns
+ *     Q4D_ERR_WORKSPACE and launches nothing.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero (each call writes every state it
+ *     reads), but calls whose kernels overlap on the GPU -- e.g. on two
+ *     streams without ordering between them -- race and give wrong results.
+ */
+#define Q4D_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB */
+q4d_status q4kv_attn_decode_noalloc(const void* Q, const void* Kq4, const void* Vq4, float* out,
+                                    int ctx_len, int n_q_heads, int n_kv_heads, int head_dim,
+                                    int M, int kv_stride_tokens, float softmax_scale,
+                                    void* stream);
+
 /* ------------------------------------------------------- launch planning --
  * Pure host functions (no CUDA call) exposing how a call is partitioned on
  * a device with num_sms SMs; the compute entry points use exactly these.
