@@ -1,263 +1,363 @@
-// Dequant-fused Q4_0 GEMV / skinny GEMM for M = 1..5 rows on CUDA cores.
+// Q4_0 GEMV / skinny GEMM for M = 1..5 rows with register dequantisation
+// feeding mma.sync (m16n8k16, bf16 in, fp32 accumulate).
 //
-// What it computes: y[m][n] = sum_k d(n,k) * (q(n,k) - 8) * x[m][k], the weight
-// stream that dominates a decode step ("Qwen3.8-27B at 256K on a 24GB RTX PRO
-// 4000 SFF (432 GB/s): 50 tok/s with MTP", paragraph beginning "NVIDIA quotes
-// 432 GB/s"), with M = 2..5 rows sharing one pass over the weights when the
-// target model verifies a drafted block ("Qwen3.8-27B on RTX 4090: 5,000 tok/s
-// Prefill Reproduced", section "MTP helps ordinary prose ...").
+// Why tensor-core instructions for a bandwidth-bound GEMV: on B200 the
+// logic/integer pipe runs at half the FP32 rate, and unpacking nibbles plus
+// one FMA per weight per row keeps the SM issue-bound well below HBM speed
+// (the CUDA-core formulation measured ~4.8 thread instructions per weight at
+// M = 1).  Letting mma.sync do the multiply-adds leaves ~2 instructions per
+// weight -- the unpack -- for every M up to 8, so M = 2..5 verification rows
+// ("Qwen3.8-27B on RTX 4090: 5,000 tok/s Prefill Reproduced", section "MTP
+// helps ordinary prose ...") cost the same as plain decode.
 //
-// Design (B200):
-//  * Each thread owns a fixed slice of K (W 32-bit nibble words = 8*W
-//    elements) for the whole kernel, so its activations live in registers for
-//    every row it touches; rows stream past it.  The activations are stored
-//    pre-scaled so that the nibble -> float conversion is one LOP3 (nibble
-//    OR'd into the mantissa of 2^23) plus one packed subtraction, and the
-//    products use packed fp32 FMA (FFMA2) -- both exact.
-//  * Each CTA (one per SM) owns a contiguous range of rows and pulls them
-//    through a shared-memory ring with cp.async.bulk, completing on an
-//    mbarrier; with an evict-first L2 policy since each weight is read once.
-//  * Per-thread partial dot products of RSR rows are combined by a warp
-//    reduce-scatter, then across the warps of a row stream in a fixed order
-//    (deterministic, no atomics).
-//  * If K is long relative to the thread budget, or there are fewer rows than
-//    SMs, K is split into ranges whose fp32 partials are summed in a fixed
-//    order by a second small kernel.
+// Exactness: q - 8 is an integer in [-8, 7], exact in bf16; x is bf16; their
+// products are exact in fp32.  Each 32-element block gets its own fresh
+// accumulator, multiplied by the block's fp16 scale d in fp32 and added to the
+// row's fp32 sum -- the Q4_0 definition w = d * (q - 8) ("Qwen3.8-27B at 256K
+// on a 24GB RTX PRO 4000 SFF (432 GB/s): 50 tok/s with MTP", paragraph on
+// public GGUFs at 40K context names the format) with fp32 rounding only.
+//
+// Layout of the work:
+//  * Weights are stored super-block-column-major: column s holds super-block
+//    s of every row, so the rows a CTA owns form one contiguous piece of each
+//    column -- every pipeline stage is a single contiguous bulk copy per
+//    column, the access pattern that streams HBM fastest.
+//  * CTA c owns rows [N*c/G, N*(c+1)/G) of one K range (k_splits > 1 only for
+//    very few rows); rows are processed in passes of up to 8 m16 tiles; a
+//    pass streams its K range KC super-block columns per stage.
+//  * Warp specialisation: one producer warp issues the copies (bulk copy of
+//    the weight piece, TMA box of the activations) into a ring of stages that
+//    complete on "full" mbarriers; eight consumer warps compute and release
+//    each stage on an "empty" mbarrier, so loads and math overlap with no
+//    CTA-wide barrier per stage.  Every wait is bounded in time.
+//  * Consumer warp w takes block w of each super-block; it builds the B
+//    fragment (x) of its block once per column and applies it to every m-tile
+//    of the pass.  At the end of a pass the eight warps' partial sums are
+//    added in a fixed order through shared memory (deterministic).
+//  * A-fragment k order: lane (g, t) dequantises word t of a block (bytes
+//    4t..4t+3) of rows g and g+8; its four bf16 pairs (low nibbles of bytes
+//    0/2, high nibbles of bytes 0/2, low of 1/3, high of 1/3) are the fragment
+//    registers of the block's two k16 steps; the B fragment takes x in the
+//    same element order, so the permutation cancels in the dot product.
+//    Rows land at a 144-byte pitch, at which the 32 lanes' 4-byte nibble
+//    loads hit 32 distinct banks.
 #pragma once
+
+#include <cuda.h>
 
 #include "q4dec_device.cuh"
 
 namespace q4d {
 
-constexpr int kGemvMaxThreads = 640;
+constexpr int kMmaMaxTiles = 8;  // m16 tiles per pass (128 rows)
+constexpr int kMmaMaxStages = 16;
 
-struct GemvArgs {
-  const uint8_t* W;    // super-blocks, N rows of nsb
-  const uint16_t* x;   // bf16 bits [M][K]
+// Kernel parameters.  The tensor map describes x as a bf16 tensor [M][K]
+// with boxes of [M][256] (one super-block column); passed as a
+// __grid_constant__ so the TMA unit reads it from the parameter space.
+struct alignas(64) GemvArgs {
+  CUtensorMap xmap;
+  const uint8_t* W;    // super-block-column-major weights, [K/256][N] x 144 B
   float* out;          // y [M][N] or partials [k_splits][M][N]
-  unsigned* err;       // device error word
-  int N, K, nsb;
-  int k_splits, sb_base, sb_rem;
-  int row_streams, tpr, stages, grid_rows;
-  uint32_t slot_bytes;
+  unsigned* err;
+  int N;
+  int sb_per_split;    // super-blocks per K range
+  int rows_per_pass;   // multiple of 16, <= 128
+  int grid_rows;
+  int stages;
 };
 
-constexpr int next_pow2(int v) { return v <= 1 ? 1 : 2 * next_pow2((v + 1) / 2); }
-
-// Scale applied to nibble position p (0..7) of a word by the extraction below:
-// positions 0..4 are used in place (bits 4p..4p+3), positions 5..7 from the
-// word shifted right by 12 (bits 4p-12..4p-9).
-__device__ __forceinline__ constexpr float nib_scale(int p) {
-  return p <= 4 ? float(1u << (4 * p)) : float(1u << (4 * p - 12));
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
 }
 
-// Word -> 8 floats equal to (q_p - 8) * nib_scale(p).  The nibble placed in
-// the low mantissa bits of 2^23 gives 2^23 + q*scale exactly; subtracting
-// 2^23 + 8*scale (exact) leaves (q - 8) * scale.
-__device__ __forceinline__ void dequant_word(uint32_t w, float2 (&t)[4]) {
-  const uint32_t w12 = w >> 12;
-  const float f0 = __uint_as_float(0x4B000000u | (w & 0x0000000Fu));
-  const float f1 = __uint_as_float(0x4B000000u | (w & 0x000000F0u));
-  const float f2 = __uint_as_float(0x4B000000u | (w & 0x00000F00u));
-  const float f3 = __uint_as_float(0x4B000000u | (w & 0x0000F000u));
-  const float f4 = __uint_as_float(0x4B000000u | (w & 0x000F0000u));
-  const float f5 = __uint_as_float(0x4B000000u | (w12 & 0x00000F00u));
-  const float f6 = __uint_as_float(0x4B000000u | (w12 & 0x0000F000u));
-  const float f7 = __uint_as_float(0x4B000000u | (w12 & 0x000F0000u));
-  constexpr float c23 = 8388608.0f;
-  t[0] = __fadd2_rn(make_float2(f0, f1),
-                    make_float2(-(c23 + 8.0f * nib_scale(0)), -(c23 + 8.0f * nib_scale(1))));
-  t[1] = __fadd2_rn(make_float2(f2, f3),
-                    make_float2(-(c23 + 8.0f * nib_scale(2)), -(c23 + 8.0f * nib_scale(3))));
-  t[2] = __fadd2_rn(make_float2(f4, f5),
-                    make_float2(-(c23 + 8.0f * nib_scale(4)), -(c23 + 8.0f * nib_scale(5))));
-  t[3] = __fadd2_rn(make_float2(f6, f7),
-                    make_float2(-(c23 + 8.0f * nib_scale(6)), -(c23 + 8.0f * nib_scale(7))));
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(magic));
+  return r;  // (a & mask) | magic
 }
 
-template <int W>
-__device__ __forceinline__ void load_words(const uint8_t* p, uint32_t (&wv)[W]) {
-  if constexpr (W == 4) {
-    const uint4 v = *reinterpret_cast<const uint4*>(p);
-    wv[0] = v.x; wv[1] = v.y; wv[2] = v.z; wv[3] = v.w;
-  } else if constexpr (W == 2) {
-    const uint2 v = *reinterpret_cast<const uint2*>(p);
-    wv[0] = v.x; wv[1] = v.y;
-  } else {
-    wv[0] = *reinterpret_cast<const uint32_t*>(p);
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Four bf16x2 registers holding q - 8 (exact) for the 8 nibbles of word w:
+// r[0] = (byte0.lo, byte2.lo), r[1] = (byte0.hi, byte2.hi),
+// r[2] = (byte1.lo, byte3.lo), r[3] = (byte1.hi, byte3.hi).
+// 0x4300 | q is the bf16 value 128 + q; subtracting 136 leaves q - 8.
+__device__ __forceinline__ void dequant_pairs(uint32_t w, uint32_t mask, uint32_t magic,
+                                              uint32_t c136, uint32_t (&r)[4]) {
+  r[0] = bf16x2_sub(lop3_and_or(w, mask, magic), c136);
+  r[1] = bf16x2_sub(lop3_and_or(w >> 4, mask, magic), c136);
+  r[2] = bf16x2_sub(lop3_and_or(w >> 8, mask, magic), c136);
+  r[3] = bf16x2_sub(lop3_and_or(w >> 12, mask, magic), c136);
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_nohint(uint32_t dst, const CUtensorMap* map, int x,
+                                                   int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+constexpr uint32_t kSbBytes = 144;  // one super-block row piece in shared memory
+
+// Bytes of one pipeline stage holding KC super-block columns: KC weight
+// pieces (rows_per_pass x 144 bytes each, rounded up to 128) followed by KC
+// activation boxes (M x 512 bytes each).
+__host__ __device__ constexpr uint32_t gemv_wbox_bytes(int rows_per_pass) {
+  return (uint32_t(rows_per_pass) * kSbBytes + 127u) / 128u * 128u;
+}
+__host__ __device__ constexpr uint32_t gemv_stage_bytes(int M, int KC, int rows_per_pass) {
+  return uint32_t(KC) * (gemv_wbox_bytes(rows_per_pass) + uint32_t(M) * 512u);
+}
+
+constexpr int kConsumerWarps = 8;
+constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
+// One m16 tile x one 32-element block: dequantise rows g (and g+8 when
+// `second`), two MMAs against the block's x fragment, then add the tile's
+// fresh accumulator times each row's block scale into acc.  Columns >= M
+// of the accumulator stay zero and are not scaled.
+template <int M>
+__device__ __forceinline__ void gemv_tile(const uint8_t* pa, uint32_t woff, uint32_t doff,
+                                          bool second, const uint32_t (&bx)[4],
+                                          float (&acc)[4]) {
+  const uint32_t mask = 0x000F000Fu, magic = 0x43004300u, c136 = 0x43084308u;  // bf16 136
+  const uint8_t* pb = pa + 8u * kSbBytes;
+  const uint32_t wa = *reinterpret_cast<const uint32_t*>(pa + woff);
+  const uint32_t wb = second ? *reinterpret_cast<const uint32_t*>(pb + woff) : 0x88888888u;
+  const float da = half_bits_to_float(*reinterpret_cast<const uint16_t*>(pa + doff));
+  const float db = second ? half_bits_to_float(*reinterpret_cast<const uint16_t*>(pb + doff)) : 0.f;
+  uint32_t qa[4], qb[4];
+  dequant_pairs(wa, mask, magic, c136, qa);
+  dequant_pairs(wb, mask, magic, c136, qb);
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
+  mma_bf16(c, qa[0], qb[0], qa[1], qb[1], bx[0], bx[1]);
+  mma_bf16(c, qa[2], qb[2], qa[3], qb[3], bx[2], bx[3]);
+  acc[0] = fmaf(da, c[0], acc[0]);
+  acc[2] = fmaf(db, c[2], acc[2]);
+  if constexpr (M > 1) {
+    acc[1] = fmaf(da, c[1], acc[1]);
+    acc[3] = fmaf(db, c[3], acc[3]);
   }
 }
 
-// M: activation rows, W: nibble words per thread per row, RSR: rows each
-// row stream handles per pipeline stage.
-template <int M, int W, int RSR>
-__global__ void __launch_bounds__(kGemvMaxThreads, 1) q4_gemv_kernel(const GemvArgs a) {
-  constexpr int TPS = 32 / W;                 // threads per super-block
-  constexpr int VPAD = next_pow2(RSR * M);    // reduce-scatter width (<= 32)
-  static_assert(VPAD <= 32, "reduce-scatter holds at most one value per lane");
+// Everything a consumer warp needs to run the stages of one pass.
+struct PassCtx {
+  const uint8_t* ring;
+  uint64_t* full;
+  uint64_t* empty;
+  unsigned* err;
+  uint32_t stage_bytes, wbox, xoff, woff, doff;
+  int S, n_chunks, warp, g, t, lane;
+};
 
+// One pass of T m-tiles (the last one using only rows 0..7 when HALF) over
+// all chunks of the K range: wait for each stage, run every tile of every
+// block fully unrolled (no per-tile guard, so the compiler interleaves the
+// tiles' loads, unpacking and MMAs), then release the stage.  Rows beyond the
+// pass's end hold stale shared memory; their results are never stored.
+template <int M, int KC, int T, bool HALF>
+__device__ __forceinline__ void gemv_pass(const PassCtx& c, int& slot, uint32_t& phase,
+                                          float (&acc)[kMmaMaxTiles][4]) {
+  #pragma unroll
+  for (int p = 0; p < T; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
+  for (int chunk = 0; chunk < c.n_chunks; ++chunk) {
+    mbar_wait(smem_addr(&c.full[slot]), phase, c.err);
+    const uint8_t* wst = c.ring + size_t(slot) * c.stage_bytes;
+    #pragma unroll 1
+    for (int j = 0; j < KC; ++j) {  // kept rolled: one copy of the tile code stays in the I-cache
+      // B fragment (x) of this warp's block of column j for column g
+      uint32_t bx[4] = {0u, 0u, 0u, 0u};
+      if (c.g < M) {
+        const uint8_t* xr = wst + c.xoff + (j * M + c.g) * 512 + (c.warp * 32 + 4 * c.t) * 2;
+        const uint2 lo = *reinterpret_cast<const uint2*>(xr);
+        const uint2 hi = *reinterpret_cast<const uint2*>(xr + 32);
+        bx[0] = prmt(lo.x, lo.y, 0x5410);  // (x[4t+0], x[4t+2])
+        bx[1] = prmt(hi.x, hi.y, 0x5410);  // (x[16+4t+0], x[16+4t+2])
+        bx[2] = prmt(lo.x, lo.y, 0x7632);  // (x[4t+1], x[4t+3])
+        bx[3] = prmt(hi.x, hi.y, 0x7632);  // (x[16+4t+1], x[16+4t+3])
+      }
+      const uint8_t* wj = wst + uint32_t(j) * c.wbox;
+      #pragma unroll
+      for (int p = 0; p < T; ++p)
+        gemv_tile<M>(wj + 16u * p * kSbBytes, c.woff, c.doff, !(HALF && p == T - 1), bx, acc[p]);
+    }
+    __syncwarp();
+    if (c.lane == 0) mbar_arrive(smem_addr(&c.empty[slot]));  // this warp is done with it
+    if (++slot == c.S) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+}
+
+// M: activation rows (B fragment columns; columns M..7 are zero).
+// KC: super-block columns per pipeline stage.
+// Warps 0..7 consume: warp w takes block w of every super-block column and
+// every m-tile of the pass.  Warp 8 produces: it refills a stage as soon as
+// all eight consumers have released it.
+template <int M, int KC>
+__global__ void __launch_bounds__(kGemvThreads, 1)
+    q4_gemv_kernel(const __grid_constant__ GemvArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = blockDim.x >> 5;
   const int ks = blockIdx.y;
-
-  const int sb_count = a.sb_base + (ks < a.sb_rem ? 1 : 0);
-  const int sb0 = ks * a.sb_base + min(ks, a.sb_rem);
-  const uint32_t seg_bytes = uint32_t(sb_count) * 144u;
+  const int S = a.stages;
 
   const int row_begin = int((long long)a.N * blockIdx.x / a.grid_rows);
   const int row_end = int((long long)a.N * (blockIdx.x + 1) / a.grid_rows);
-  const int rows_per_stage = a.row_streams * RSR;
-  const int n_stages = (row_end - row_begin + rows_per_stage - 1) / rows_per_stage;
+  const int n_rows = row_end - row_begin;
+  const int R = a.rows_per_pass;
+  const int n_passes = (n_rows + R - 1) / R;
+  const int n_chunks = a.sb_per_split / KC;
+  const int n_stages = n_passes * n_chunks;
+  const int sb_split0 = ks * a.sb_per_split;
+  const uint32_t wbox = gemv_wbox_bytes(R);
+  const uint32_t stage_bytes = gemv_stage_bytes(M, KC, R);
+  const uint32_t xoff = uint32_t(KC) * wbox;
 
-  uint8_t* slots = smem;
-  float* red = reinterpret_cast<float*>(smem + size_t(a.stages) * a.slot_bytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 2 * nwarps * VPAD);
-
-  const int stream = tid / a.tpr;
-  const int idx = tid - stream * a.tpr;
-  const int sb_local = idx / TPS;
-  const int word0 = (idx % TPS) * W;
-  const int blk = word0 >> 2;
-  const bool active = sb_local < sb_count;
+  uint8_t* ring = smem;
+  float4* red = reinterpret_cast<float4*>(smem + size_t(S) * stage_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + kConsumerWarps * kMmaMaxTiles * 32);
+  uint64_t* empty = full + S;
 
   if (tid == 0) {
-    for (int s = 0; s < a.stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_addr(&full[s]), 1);
+      mbar_init(smem_addr(&empty[s]), kConsumerWarps);
+    }
     mbar_init_fence();
   }
   __syncthreads();
 
-  const uint64_t pol = l2_evict_first_policy();
-  auto issue = [&](int st) {
-    const int slot = st % a.stages;
-    const int r0 = row_begin + st * rows_per_stage;
-    const int nr = min(rows_per_stage, row_end - r0);
-    const uint32_t bar = smem_addr(&bars[slot]);
-    const uint32_t dst = smem_addr(slots + size_t(slot) * a.slot_bytes);
-    mbar_arrive_expect_tx(bar, uint32_t(nr) * seg_bytes);
-    if (a.k_splits == 1) {
-      bulk_g2s(dst, a.W + size_t(r0) * a.nsb * 144u, uint32_t(nr) * seg_bytes, bar, pol);
-    } else {
-      for (int r = 0; r < nr; ++r)
-        bulk_g2s(dst + uint32_t(r) * seg_bytes,
-                 a.W + (size_t(r0 + r) * a.nsb + sb0) * 144u, seg_bytes, bar, pol);
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: one lane issues every copy ----------------
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();
+      int slot = 0, pass = 0, chunk = 0;
+      uint32_t phase = 0;
+      for (int st = 0; st < n_stages; ++st) {
+        if (st >= S) mbar_wait(smem_addr(&empty[slot]), phase ^ 1u, a.err);
+        const int r0 = row_begin + pass * R;
+        const int nr = min(R, row_end - r0);
+        const uint32_t bar = smem_addr(&full[slot]);
+        const uint32_t dst = smem_addr(ring + size_t(slot) * stage_bytes);
+        const int sb = sb_split0 + chunk * KC;
+        mbar_arrive_expect_tx(bar, uint32_t(KC) * (uint32_t(nr) * kSbBytes + uint32_t(M) * 512u));
+        #pragma unroll
+        for (int j = 0; j < KC; ++j) {
+          // rows r0 .. r0+nr of column sb+j are contiguous in the weight layout
+          bulk_g2s(dst + uint32_t(j) * wbox, a.W + (size_t(sb + j) * a.N + r0) * kSbBytes,
+                   uint32_t(nr) * kSbBytes, bar, pol);
+          tma_load_2d_nohint(dst + xoff + uint32_t(j) * uint32_t(M) * 512u, &a.xmap,
+                             (sb + j) * 256, 0, bar);
+        }
+        if (++slot == S) {
+          slot = 0;
+          phase ^= 1u;
+        }
+        if (++chunk == n_chunks) {
+          chunk = 0;
+          ++pass;
+        }
+      }
     }
-  };
-  if (tid == 0) {
-    const int pre = min(a.stages, n_stages);
-    for (int st = 0; st < pre; ++st) issue(st);
+    return;
   }
 
-  // Activations of my words, pre-divided by the extraction scale.
-  float2 xr[M][W][4];
-  #pragma unroll
-  for (int m = 0; m < M; ++m)
+  // ---------------- consumers ----------------
+  PassCtx c;
+  c.ring = ring;
+  c.full = full;
+  c.empty = empty;
+  c.err = a.err;
+  c.stage_bytes = stage_bytes;
+  c.wbox = wbox;
+  c.xoff = xoff;
+  c.warp = warp;
+  c.lane = lane;
+  c.g = lane >> 2;
+  c.t = lane & 3;
+  c.woff = uint32_t(c.g) * kSbBytes + uint32_t(warp) * 16u + uint32_t(c.t) * 4u;
+  c.doff = uint32_t(c.g) * kSbBytes + 128u + uint32_t(warp) * 2u;
+  c.S = S;
+  c.n_chunks = n_chunks;
+  float acc[kMmaMaxTiles][4];
+  int slot = 0;
+  uint32_t phase = 0;
+
+  for (int pass = 0; pass < n_passes; ++pass) {
+    const int nr = min(R, n_rows - pass * R);
+    const int T = (nr + 15) >> 4;
+    const bool half = (nr & 15) != 0 && (nr & 15) <= 8;
+    switch (T * 2 + (half ? 1 : 0)) {
+#define Q4D_PASS(TT)                                                   \
+  case 2 * TT: gemv_pass<M, KC, TT, false>(c, slot, phase, acc); break; \
+  case 2 * TT + 1: gemv_pass<M, KC, TT, true>(c, slot, phase, acc); break;
+      Q4D_PASS(1) Q4D_PASS(2) Q4D_PASS(3) Q4D_PASS(4)
+      Q4D_PASS(5) Q4D_PASS(6) Q4D_PASS(7) Q4D_PASS(8)
+#undef Q4D_PASS
+      default: break;
+    }
+
+    // Cross-warp sum of the pass, in a fixed order.
     #pragma unroll
-    for (int w = 0; w < W; ++w)
+    for (int p = 0; p < kMmaMaxTiles; ++p)
+      if (16 * p < nr)
+        red[(warp * kMmaMaxTiles + p) * 32 + lane] =
+            make_float4(acc[p][0], acc[p][1], acc[p][2], acc[p][3]);
+    consumer_sync();
+    // out[m][row] = sum over the 8 warps; element (row r, column m) sits in
+    // lane (r % 8) * 4 + m / 2 of tile r / 16, component (r >= 8 ? 2 : 0) + m % 2
+    const int r0 = row_begin + pass * R;
+    for (int i = tid; i < nr * M; i += kConsumerWarps * 32) {
+      const int r = i / M, m = i - (i / M) * M;
+      const int p = r >> 4, rr = r & 15;
+      const int ln = (rr & 7) * 4 + (m >> 1);
+      const int comp = (rr >= 8 ? 2 : 0) + (m & 1);
+      float s = 0.f;
       #pragma unroll
-      for (int i = 0; i < 4; ++i) xr[m][w][i] = make_float2(0.f, 0.f);
-  if (active) {
-    const int kb = (sb0 + sb_local) * 256 + blk * 32;
-    #pragma unroll
-    for (int w = 0; w < W; ++w) {
-      const int klo = kb + 4 * ((word0 + w) & 3);
-      #pragma unroll
-      for (int m = 0; m < M; ++m) {
-        const uint2 lo = *reinterpret_cast<const uint2*>(a.x + size_t(m) * a.K + klo);
-        const uint2 hi = *reinterpret_cast<const uint2*>(a.x + size_t(m) * a.K + klo + 16);
-        const uint32_t lv[4] = {lo.x & 0xFFFFu, lo.x >> 16, lo.y & 0xFFFFu, lo.y >> 16};
-        const uint32_t hv[4] = {hi.x & 0xFFFFu, hi.x >> 16, hi.y & 0xFFFFu, hi.y >> 16};
-        #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          // byte c: low nibble = position 2c (element klo+c), high = 2c+1 (klo+16+c)
-          const float xl = bf16_bits_to_float(lv[c]) * (1.0f / nib_scale(2 * c));
-          const float xh = bf16_bits_to_float(hv[c]) * (1.0f / nib_scale(2 * c + 1));
-          if (c == 0) xr[m][w][0] = make_float2(xl, xh);
-          if (c == 1) xr[m][w][1] = make_float2(xl, xh);
-          if (c == 2) xr[m][w][2] = make_float2(xl, xh);
-          if (c == 3) xr[m][w][3] = make_float2(xl, xh);
-        }
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float4 v = red[(w * kMmaMaxTiles + p) * 32 + ln];
+        s += comp == 0 ? v.x : comp == 1 ? v.y : comp == 2 ? v.z : v.w;
       }
+      a.out[(size_t(ks) * M + m) * a.N + r0 + r] = s;
     }
-  }
-
-  const uint32_t word_off = uint32_t(sb_local) * 144u + uint32_t(word0) * 4u;
-  const uint32_t scale_off = uint32_t(sb_local) * 144u + 128u + uint32_t(blk) * 2u;
-  const int wps = a.tpr >> 5;  // warps per row stream
-
-  for (int st = 0; st < n_stages; ++st) {
-    const int slot = st % a.stages;
-    mbar_wait(smem_addr(&bars[slot]), uint32_t(st / a.stages) & 1u, a.err);
-    const uint8_t* sl = slots + size_t(slot) * a.slot_bytes;
-    const int r0 = row_begin + st * rows_per_stage;
-    const int nr = min(rows_per_stage, row_end - r0);
-
-    float v[VPAD];
-    #pragma unroll
-    for (int i = 0; i < VPAD; ++i) v[i] = 0.f;
-    #pragma unroll
-    for (int r = 0; r < RSR; ++r) {
-      const int lr = stream * RSR + r;
-      if (active && lr < nr) {
-        const uint8_t* rowp = sl + uint32_t(lr) * seg_bytes;
-        uint32_t wv[W];
-        load_words<W>(rowp + word_off, wv);
-        const float dsc = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rowp + scale_off));
-        float2 acc[M];
-        #pragma unroll
-        for (int m = 0; m < M; ++m) acc[m] = make_float2(0.f, 0.f);
-        #pragma unroll
-        for (int w = 0; w < W; ++w) {
-          float2 t[4];
-          dequant_word(wv[w], t);
-          #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            #pragma unroll
-            for (int m = 0; m < M; ++m) acc[m] = __ffma2_rn(t[i], xr[m][w][i], acc[m]);
-        }
-        #pragma unroll
-        for (int m = 0; m < M; ++m) v[r * M + m] = dsc * (acc[m].x + acc[m].y);
-      }
-    }
-
-    // Warp reduce-scatter: after it, lane L holds the warp sum of value
-    // L / (32 / VPAD); lanes with L % (32 / VPAD) == 0 publish it.
-    #pragma unroll
-    for (int it = 0; it < 5; ++it) {
-      const int off = 16 >> it;
-      const int width = (VPAD >> it) > 1 ? (VPAD >> it) : 1;
-      if (width > 1) {
-        const bool upper = (lane & off) != 0;
-        #pragma unroll
-        for (int i = 0; i < width / 2; ++i) {
-          const float send = upper ? v[i] : v[i + width / 2];
-          const float keep = upper ? v[i + width / 2] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
-        }
-      } else {
-        v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], off);
-      }
-    }
-    float* redb = red + (st & 1) * nwarps * VPAD;
-    if ((lane % (32 / VPAD)) == 0) redb[warp * VPAD + lane / (32 / VPAD)] = v[0];
-    __syncthreads();
-
-    if (tid == 0 && st + a.stages < n_stages) issue(st + a.stages);
-
-    // Combine the warps of each row stream in a fixed order and store.
-    if (tid < rows_per_stage * M) {
-      const int lr = tid / M, m = tid - (tid / M) * M;
-      if (lr < nr) {
-        const int s = lr / RSR, r = lr - s * RSR;
-        float sum = 0.f;
-        for (int w = 0; w < wps; ++w) sum += redb[(s * wps + w) * VPAD + r * M + m];
-        a.out[(size_t(ks) * M + m) * a.N + r0 + lr] = sum;
-      }
-    }
+    consumer_sync();  // red is rewritten at the next pass end
   }
 }
 
-// y[i] = sum over k ranges of the partials, in range order.
+// y[i] = sum over K ranges of the partials, in range order.
 __global__ void q4_gemv_splitk_reduce(const float* __restrict__ ws, float* __restrict__ y,
                                       long long mn, int k_splits) {
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < mn;

@@ -2,13 +2,17 @@
 // and kernel dispatch.  Declarations and the contract live in include/q4dec.h.
 #include "q4dec.h"
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "q4_gemv.cuh"
 #include "q4kv_attn.cuh"
@@ -20,7 +24,7 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kPlanFallbackSms = 148;
-constexpr size_t kGemvStageBudget = 160 * 1024;  // shared memory for the weight ring
+constexpr size_t kGemvSmemBudget = 224 * 1024;   // shared memory per GEMV CTA
 
 struct DeviceState {
   std::atomic<bool> ready{false};
@@ -98,10 +102,66 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 int ceil_div(long long a, long long b) { return int((a + b - 1) / b); }
 long long round_up(long long a, long long b) { return (a + b - 1) / b * b; }
 
-// Per-M kernel configuration: 32-bit nibble words per thread and rows per
-// stream per stage.  Must match the dispatch in launch_gemv.
-int gemv_words_per_thread(int M) { return M == 1 ? 4 : (M == 2 ? 2 : 1); }
-int gemv_rows_per_stream(int M) { return M <= 2 ? 4 : 2; }
+// ---------------------------------------------------------------------------
+// TMA tensor maps, encoded on the host through the driver entry point (no
+// link-time dependency on libcuda) and cached by (address, shape, box).
+struct MapKey {
+  const void* ptr;
+  uint64_t d0, d1, stride;
+  uint32_t b0, b1;
+  int dtype;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && stride == o.stride && b0 == o.b0 &&
+           b1 == o.b1 && dtype == o.dtype;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    uint64_t h = reinterpret_cast<uintptr_t>(k.ptr);
+    for (uint64_t v : {k.d0, k.d1, k.stride, uint64_t(k.b0) << 32 | k.b1, uint64_t(k.dtype)})
+      h = (h ^ v) * 0x100000001B3ull;
+    return size_t(h);
+  }
+};
+std::mutex g_map_mu;
+std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+q4d_status tensor_map_2d(CUtensorMap* out, CUtensorMapDataType dtype, const void* ptr, uint64_t d0,
+                         uint64_t d1, uint64_t stride_bytes, uint32_t b0, uint32_t b1) {
+  const MapKey key{ptr, d0, d1, stride_bytes, b0, b1, int(dtype)};
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  auto it = g_maps.find(key);
+  if (it != g_maps.end()) {
+    *out = it->second;
+    return Q4D_OK;
+  }
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn) {
+      cudaGetLastError();
+      return Q4D_ERR_CUDA;
+    }
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {stride_bytes};
+  const cuuint32_t box[2] = {b0, b1};
+  const cuuint32_t estr[2] = {1, 1};
+  if (g_encode(&map, dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+      CUDA_SUCCESS)
+    return Q4D_ERR_CUDA;
+  if (g_maps.size() > 8192) g_maps.clear();
+  g_maps.emplace(key, map);
+  *out = map;
+  return Q4D_OK;
+}
 
 q4d_status check_gemv_shape(int M, int N, int K) {
   if (N < 1 || K < 0) return Q4D_ERR_INVALID_ARG;
@@ -118,11 +178,11 @@ q4d_status check_attn_shape(int ctx_len, int n_q, int n_kv, int head_dim, int M,
   return Q4D_OK;
 }
 
-template <int M, int W, int RSR>
+template <int M, int KC>
 q4d_status launch_gemv_t(const q4d::GemvArgs& a, const q4d_gemv_plan& p, int dev,
                          const DeviceState& s, cudaStream_t stream) {
   static std::atomic<bool> smem_set[kMaxDevices];
-  auto kernel = q4d::q4_gemv_kernel<M, W, RSR>;
+  auto kernel = q4d::q4_gemv_kernel<M, KC>;
   q4d_status st = allow_smem(kernel, dev, s, smem_set);
   if (st != Q4D_OK) return st;
   dim3 grid(p.grid_rows, p.k_splits);
@@ -152,28 +212,35 @@ q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, in
   }
 
   q4d::GemvArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if ((st = tensor_map_2d(&a.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, uint64_t(K), uint64_t(M),
+                          uint64_t(K) * 2u, 256u, uint32_t(M))) != Q4D_OK)
+    return st;
   a.W = static_cast<const uint8_t*>(W_q4);
-  a.x = static_cast<const uint16_t*>(x);
   a.out = p.k_splits > 1 ? static_cast<float*>(workspace) : y;
   a.err = s->err;
   a.N = N;
-  a.K = K;
-  a.nsb = K / 256;
-  a.k_splits = p.k_splits;
-  a.sb_base = a.nsb / p.k_splits;
-  a.sb_rem = a.nsb % p.k_splits;
-  a.row_streams = p.row_streams;
-  a.tpr = p.threads / p.row_streams;
-  a.stages = p.stages;
+  a.sb_per_split = p.sb_per_split;
+  a.rows_per_pass = p.rows_per_pass;
   a.grid_rows = p.grid_rows;
-  a.slot_bytes = uint32_t(p.row_streams * p.rows_per_stream * p.sb_per_split * 144);
+  a.stages = p.stages;
 
-  switch (M) {
-    case 1: st = launch_gemv_t<1, 4, 4>(a, p, dev, *s, stream); break;
-    case 2: st = launch_gemv_t<2, 2, 4>(a, p, dev, *s, stream); break;
-    case 3: st = launch_gemv_t<3, 1, 2>(a, p, dev, *s, stream); break;
-    case 4: st = launch_gemv_t<4, 1, 2>(a, p, dev, *s, stream); break;
-    default: st = launch_gemv_t<5, 1, 2>(a, p, dev, *s, stream); break;
+  switch (M * 8 + p.chunk_sb) {
+    case 1 * 8 + 1: st = launch_gemv_t<1, 1>(a, p, dev, *s, stream); break;
+    case 1 * 8 + 2: st = launch_gemv_t<1, 2>(a, p, dev, *s, stream); break;
+    case 1 * 8 + 4: st = launch_gemv_t<1, 4>(a, p, dev, *s, stream); break;
+    case 2 * 8 + 1: st = launch_gemv_t<2, 1>(a, p, dev, *s, stream); break;
+    case 2 * 8 + 2: st = launch_gemv_t<2, 2>(a, p, dev, *s, stream); break;
+    case 2 * 8 + 4: st = launch_gemv_t<2, 4>(a, p, dev, *s, stream); break;
+    case 3 * 8 + 1: st = launch_gemv_t<3, 1>(a, p, dev, *s, stream); break;
+    case 3 * 8 + 2: st = launch_gemv_t<3, 2>(a, p, dev, *s, stream); break;
+    case 3 * 8 + 4: st = launch_gemv_t<3, 4>(a, p, dev, *s, stream); break;
+    case 4 * 8 + 1: st = launch_gemv_t<4, 1>(a, p, dev, *s, stream); break;
+    case 4 * 8 + 2: st = launch_gemv_t<4, 2>(a, p, dev, *s, stream); break;
+    case 4 * 8 + 4: st = launch_gemv_t<4, 4>(a, p, dev, *s, stream); break;
+    case 5 * 8 + 1: st = launch_gemv_t<5, 1>(a, p, dev, *s, stream); break;
+    case 5 * 8 + 2: st = launch_gemv_t<5, 2>(a, p, dev, *s, stream); break;
+    default: st = launch_gemv_t<5, 4>(a, p, dev, *s, stream); break;
   }
   if (st != Q4D_OK) return st;
   if (p.k_splits > 1) {
@@ -269,35 +336,46 @@ q4d_status q4d_plan_gemv(int M, int N, int K, int num_sms, q4d_gemv_plan* plan) 
   q4d_status st = check_gemv_shape(M, N, K);
   if (st != Q4D_OK) return st;
   const int nsb = K / 256;
-  const int W = gemv_words_per_thread(M);
-  const int tps = 32 / W;
-  const int rsr = gemv_rows_per_stream(M);
-  // K ranges: as few as fit the thread budget ...
+  // Rows are shared out exactly (+-1) over up to one CTA per SM, at least 8
+  // rows each.  When that leaves most SMs idle, K is cut into equal ranges
+  // (a divisor of the super-block count, two or more super-blocks each).
+  int grid_rows = std::min(num_sms, std::max(1, N / 8));
   int ks = 1;
-  while (round_up((long long)ceil_div(nsb, ks) * tps, 32) > q4d::kGemvMaxThreads) ++ks;
-  // ... and more while there are fewer (row, range) units than SMs.
-  while (ks < nsb && (long long)N * ks < num_sms) ++ks;
-  const int sbs = ceil_div(nsb, ks);
-  const int tpr = int(round_up((long long)sbs * tps, 32));
-  int grid_rows = std::max(1, num_sms / ks);
-  if (grid_rows > N) grid_rows = N;
+  if (2 * grid_rows < num_sms) {
+    const int want = num_sms / grid_rows;
+    for (int d = std::min(want, nsb / 2); d >= 2; --d)
+      if (nsb % d == 0) {
+        ks = d;
+        break;
+      }
+  }
+  const int sbs = nsb / ks;
   const int rows_per_cta = ceil_div(N, grid_rows);
-  int streams = std::max(1, q4d::kGemvMaxThreads / tpr);
-  streams = std::min(streams, std::max(1, ceil_div(rows_per_cta, rsr)));
-  const size_t slot = size_t(streams) * rsr * sbs * 144;
-  int stages = int(kGemvStageBudget / slot);
-  stages = std::max(2, std::min(12, stages));
-  const int VPAD = q4d::next_pow2(rsr * M);
-  const int threads = streams * tpr;
+  const int tiles = std::min(q4d::kMmaMaxTiles, ceil_div(rows_per_cta, 16));
+  const int rows_per_pass = 16 * tiles;
+  // Super-block columns per stage: the fewest of 1, 2, 4 (dividing the K
+  // range) that give at least 24 KB of weights per stage (fewer, larger
+  // stages amortise the per-stage handshakes); then as many stages as fit,
+  // up to 16.
+  int KC = 1;
+  for (int c : {1, 2, 4}) {
+    if (sbs % c) continue;
+    KC = c;
+    if (size_t(c) * rows_per_pass * 144 >= 24 * 1024) break;
+  }
+  const size_t red = size_t(q4d::kConsumerWarps) * q4d::kMmaMaxTiles * 32 * 16;
+  const size_t stage = q4d::gemv_stage_bytes(M, KC, rows_per_pass);
+  int stages = int((kGemvSmemBudget - red) / (stage + 16));
+  stages = std::max(2, std::min(q4d::kMmaMaxStages, stages));
   plan->k_splits = ks;
   plan->sb_per_split = sbs;
-  plan->words_per_thread = W;
-  plan->row_streams = streams;
-  plan->rows_per_stream = rsr;
+  plan->chunk_sb = KC;
+  plan->rows_per_cta = rows_per_cta;
+  plan->rows_per_pass = rows_per_pass;
   plan->stages = stages;
-  plan->threads = threads;
+  plan->threads = q4d::kGemvThreads;
   plan->grid_rows = grid_rows;
-  plan->smem_bytes = stages * slot + size_t(2) * (threads / 32) * VPAD * 4 + size_t(stages) * 8;
+  plan->smem_bytes = stages * stage + red + size_t(stages) * 16;
   plan->workspace_bytes = ks > 1 ? size_t(ks) * M * N * 4 : 0;
   return Q4D_OK;
 }

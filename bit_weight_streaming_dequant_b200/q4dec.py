@@ -40,8 +40,8 @@ class Q4DecError(RuntimeError):
 
 class GemvPlan(ctypes.Structure):
     _fields_ = [("k_splits", ctypes.c_int), ("sb_per_split", ctypes.c_int),
-                ("words_per_thread", ctypes.c_int), ("row_streams", ctypes.c_int),
-                ("rows_per_stream", ctypes.c_int), ("stages", ctypes.c_int),
+                ("chunk_sb", ctypes.c_int), ("rows_per_cta", ctypes.c_int),
+                ("rows_per_pass", ctypes.c_int), ("stages", ctypes.c_int),
                 ("threads", ctypes.c_int), ("grid_rows", ctypes.c_int),
                 ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
 

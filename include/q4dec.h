@@ -29,8 +29,12 @@
  *                  bytes [128+2*b, 128+2*b+2) = fp16 scale of block b
  *                  (little endian).  144 is a multiple of 16, so every
  *                  super-block starts on a 16-byte boundary.
- *   weight W[N][K]: row n = K/256 consecutive super-blocks; super-block s of
- *                  row n starts at byte (n*(K/256) + s) * 144.
+ *   weight W[N][K]: super-block-column-major: K/256 columns one after
+ *                  another, column s holding super-block s of rows 0..N-1,
+ *                  so super-block (n, s) starts at byte (s*N + n) * 144.
+ *                  (The rows a GPU block streams are then contiguous in
+ *                  every column.)  A row-major Q4_0 matrix converts by
+ *                  moving whole 144-byte super-blocks.
  *   K/V cache    : one super-block per (KV head, token) (head_dim = 256);
  *                  token t of KV head h starts at byte (h*kv_stride + t)*144.
  *
@@ -83,7 +87,7 @@ const char* q4d_status_string(int status);
 /* ------------------------------------------------------------------ GEMV --
  * y[m][n] = sum_k (d * (q - 8))[n][k] * x[m][k]   for m < M, n < N.
  *
- *   W_q4 : N rows x K elements of Q4_0 in the super-block layout, N*K/256*144 bytes.
+ *   W_q4 : N x K elements of Q4_0 in the weight layout above, N*K/256*144 bytes.
  *   x    : bf16 [M][K] row-major (M activation rows sharing one weight stream).
  *   y    : fp32 [M][N] row-major, fully overwritten.
  *   Requirements: 1 <= M <= 5, N >= 1, K >= 256, K % 256 == 0.
@@ -171,11 +175,11 @@ q4d_status q4kv_attn_decode_noalloc(const void* Q, const void* Kq4, const void* 
  * a device with num_sms SMs; the compute entry points use exactly these.
  */
 typedef struct {
-  int k_splits;          /* K is cut into this many ranges (1 = no split)        */
-  int sb_per_split;      /* super-blocks in the longest range                    */
-  int words_per_thread;  /* 32-bit nibble words each thread owns per row         */
-  int row_streams;       /* independent row streams per CTA                      */
-  int rows_per_stream;   /* rows each stream handles per pipeline stage          */
+  int k_splits;          /* K is cut into this many equal ranges (1 = no split)  */
+  int sb_per_split;      /* super-blocks per K range                             */
+  int chunk_sb;          /* super-blocks of K per pipeline stage                 */
+  int rows_per_cta;      /* most rows any CTA owns                               */
+  int rows_per_pass;     /* rows held per pass (multiple of 16, at most 128)     */
   int stages;            /* shared-memory pipeline depth                         */
   int threads;           /* threads per CTA                                      */
   int grid_rows;         /* CTAs per K range (grid = grid_rows * k_splits)       */

@@ -9,6 +9,8 @@ from .q4_oracle import (  # noqa: F401
     f16_bits_to_f64,
     unpack_superblocks,
     dequant,
+    dequant_weights,
+    weight_rows,
     gemv,
     gemv_tolerance,
     attn_probs,

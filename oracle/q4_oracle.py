@@ -23,8 +23,12 @@ writes out the definitions the library implements:
   ``j`` holds element ``j`` (low nibble) and ``j + 16`` (high nibble);
   ``w = d * (q - 8)``.
 * super-block storage: 8 blocks in 144 bytes, nibbles first (``16*b + j``),
-  then the 8 fp16 scales at ``128 + 2*b`` (little endian).  A row of K
-  elements is K/256 consecutive super-blocks.
+  then the 8 fp16 scales at ``128 + 2*b`` (little endian).
+* weight matrix W[N][K]: K/256 super-block columns one after another; column
+  s holds super-block s of rows 0..N-1 in order, i.e. super-block (n, s) sits
+  at byte (s*N + n)*144.
+* K/V cache: one super-block per (KV head, token) at byte
+  (h*kv_stride + t)*144 (head_dim 256).
 * GEMV: ``y[m, n] = sum_k w[n, k] * x[m, k]`` for M bf16 rows x.
 * decode attention: query head ``h`` reads KV head ``h // (n_q / n_kv)``; draft
   row ``m`` sits at position ``p_m = ctx_len - M + m`` and sees tokens
@@ -90,14 +94,28 @@ def dequant(buf, rows: int, K: int) -> np.ndarray:
     return np.repeat(d, 32, axis=1) * (q.astype(np.float64) - 8.0)
 
 
+def weight_rows(W_buf, N: int, K: int) -> np.ndarray:
+    """Reorder a weight matrix stored super-block-column-major ([K/256][N]
+    super-blocks) into row order ([N][K/256] super-blocks), flat bytes."""
+    nsb = K // SB_ELEMS
+    raw = np.asarray(W_buf, dtype=np.uint8).reshape(-1)[: nsb * N * SB_BYTES]
+    return raw.reshape(nsb, N, SB_BYTES).transpose(1, 0, 2).reshape(-1)
+
+
+def dequant_weights(W_buf, N: int, K: int) -> np.ndarray:
+    """fp64 weights [N][K] of a matrix in the column-major super-block layout."""
+    return dequant(weight_rows(W_buf, N, K), N, K)
+
+
 def gemv(W_buf, x_bits, M: int, N: int, K: int):
     """Dequant-GEMV: ``y[m, n] = sum_k w[n, k] x[m, k]`` in fp64.
 
-    ``W_buf``: N rows of K elements in super-block layout; ``x_bits``: bf16 bit
-    patterns [M][K].  Returns ``(y, S)``, both float64 [M][N], where
-    ``S[m, n] = sum_k |w[n, k] x[m, k]|`` scales the parity tolerance.
+    ``W_buf``: the N x K weight matrix in the column-major super-block layout;
+    ``x_bits``: bf16 bit patterns [M][K].  Returns ``(y, S)``, both float64
+    [M][N], where ``S[m, n] = sum_k |w[n, k] x[m, k]|`` scales the parity
+    tolerance.
     """
-    w = dequant(W_buf, N, K)
+    w = dequant_weights(W_buf, N, K)
     x = bf16_bits_to_f64(np.asarray(x_bits).reshape(M, K))
     y = x @ w.T
     S = np.abs(x) @ np.abs(w).T

@@ -14,9 +14,10 @@ Storage layout written here (the library's documented layout):
 * super-block: 256 consecutive elements (8 blocks) in 144 bytes -- the 8
   blocks' 16-byte nibble arrays first (bytes ``16*b .. 16*b+15``), then the 8
   fp16 scales (bytes ``128 + 2*b``, little endian).
-* a row of ``K`` elements is ``K / 256`` consecutive super-blocks; rows follow
-  each other.  A K/V cache row (one token of one KV head, head_dim 256) is one
-  super-block.
+* a weight matrix [N][K] is stored super-block-column-major: K/256 columns,
+  column s holding super-block s of rows 0..N-1, so super-block (n, s) sits at
+  byte (s*N + n)*144.  A K/V cache row (one token of one KV head, head_dim
+  256) is one super-block, tokens of a head consecutive.
 
 Recipes (the workloads of the decode path):
 
@@ -105,12 +106,21 @@ def quantize_blocks(v: np.ndarray):
 # --------------------------------------------------------------------------
 # host generators (numpy PCG64)
 # --------------------------------------------------------------------------
+def column_major(rows_buf: np.ndarray, N: int, K: int) -> np.ndarray:
+    """Reorder super-blocks of a row-ordered matrix ([N][K/256]) into the
+    weight layout ([K/256][N]), flat bytes."""
+    nsb = K // SUPERBLOCK_ELEMS
+    return np.ascontiguousarray(
+        np.asarray(rows_buf, dtype=np.uint8).reshape(N, nsb, SUPERBLOCK_BYTES).transpose(1, 0, 2)
+    ).reshape(-1)
+
+
 def q4_0_weights(seed: int, N: int, K: int) -> np.ndarray:
-    """Random Q4_0 weight matrix [N][K] in super-block layout (flat uint8)."""
+    """Random Q4_0 weight matrix [N][K] in the weight layout (flat uint8)."""
     rng = np.random.default_rng(seed)
     q = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
     d = np.abs(rng.standard_normal(size=(N, K // BLOCK_ELEMS))) * 0.02
-    return pack_superblocks(q, f32_to_f16_bits(d.astype(np.float32)))
+    return column_major(pack_superblocks(q, f32_to_f16_bits(d.astype(np.float32))), N, K)
 
 
 def bf16_normal(seed: int, shape, scale: float = 1.0) -> np.ndarray:
@@ -140,9 +150,15 @@ def queries(seed: int, M: int, n_q_heads: int, head_dim: int = 256) -> np.ndarra
 
 
 def from_parts(q: np.ndarray, d: np.ndarray) -> np.ndarray:
-    """Pack explicit nibbles and float scales (rounded to fp16) -- used to build
-    hand-made cases (all q = 8, powers of two, one-hot ...)."""
+    """Pack explicit nibbles and float scales (rounded to fp16) row after row
+    -- the K/V cache layout; hand-made cases (all q = 8, powers of two ...)."""
     return pack_superblocks(q, f32_to_f16_bits(np.asarray(d, dtype=np.float32)))
+
+
+def weights_from_parts(q: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """Like ``from_parts`` but in the weight layout (column-major super-blocks)."""
+    q = np.asarray(q, dtype=np.uint8)
+    return column_major(from_parts(q, d), q.shape[0], q.shape[1])
 
 
 # --------------------------------------------------------------------------
@@ -156,17 +172,17 @@ def _torch():
 
 def device_q4_0_weights(seed: int, N: int, K: int, device="cuda"):
     """Random Q4_0 weight matrix [N][K] generated on ``device``; returns a
-    flat uint8 tensor in super-block layout (same recipe as ``q4_0_weights``)."""
+    flat uint8 tensor in the weight layout (same recipe as ``q4_0_weights``)."""
     torch = _torch()
     g = torch.Generator(device=device)
     g.manual_seed(seed)
     nsb = K // SUPERBLOCK_ELEMS
-    out = torch.empty((N, nsb, SUPERBLOCK_BYTES), dtype=torch.uint8, device=device)
+    out = torch.empty((nsb, N, SUPERBLOCK_BYTES), dtype=torch.uint8, device=device)
     # q: two uniform nibbles per byte == one uniform byte
-    out[:, :, :128] = torch.randint(0, 256, (N, nsb, 128), generator=g, device=device,
+    out[:, :, :128] = torch.randint(0, 256, (nsb, N, 128), generator=g, device=device,
                                     dtype=torch.int32).to(torch.uint8)
-    d = (torch.randn((N, nsb, 8), generator=g, device=device).abs() * 0.02).to(torch.float16)
-    out[:, :, 128:] = d.view(torch.uint8).reshape(N, nsb, 16)
+    d = (torch.randn((nsb, N, 8), generator=g, device=device).abs() * 0.02).to(torch.float16)
+    out[:, :, 128:] = d.view(torch.uint8).reshape(nsb, N, 16)
     return out.reshape(-1)
 
 

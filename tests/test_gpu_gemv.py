@@ -59,7 +59,7 @@ def test_layer_shapes_m1(cuda_ok, shape):
 def test_layer_shapes_verify_m2_to_m5(cuda_ok, shape):
     N, K = LAYER_SHAPES[shape]
     Wnp = synth.q4_0_weights(10 + shape, N, K)
-    w = oracle.dequant(Wnp, N, K)
+    w = oracle.dequant_weights(Wnp, N, K)
     W = dev_bytes(Wnp)
     for M in (2, 3, 4, 5):
         xnp = synth.activations(100 + M, M, K)
@@ -75,7 +75,7 @@ def test_layer_shapes_verify_m2_to_m5(cuda_ok, shape):
 def test_all_q8_gives_exact_zero(cuda_ok, N, K, M):
     q = np.full((N, K), 8, dtype=np.uint8)
     d = np.abs(np.random.default_rng(N).standard_normal((N, K // 32))).astype(np.float32)
-    y = _run(synth.from_parts(q, d), synth.activations(3, M, K), N, K)
+    y = _run(synth.weights_from_parts(q, d), synth.activations(3, M, K), N, K)
     assert torch.count_nonzero(y).item() == 0
 
 
@@ -86,7 +86,7 @@ def test_dyadic_inputs_are_bit_exact(cuda_ok, M):
     q = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
     d = (2.0 ** -rng.integers(0, 6, size=(N, K // 32))).astype(np.float32)
     xi = rng.integers(-3, 4, size=(M, K)).astype(np.float32)
-    Wnp, xnp = synth.from_parts(q, d), synth.f32_to_bf16_bits(xi)
+    Wnp, xnp = synth.weights_from_parts(q, d), synth.f32_to_bf16_bits(xi)
     y_ref, _ = oracle.gemv(Wnp, xnp, M, N, K)
     y = _run(Wnp, xnp, N, K).cpu().numpy().astype(np.float64)
     assert np.array_equal(y, y_ref)
@@ -149,7 +149,9 @@ def test_output_head_sampled_rows(cuda_ok):
         torch.cuda.synchronize()
         rows = np.sort(np.random.default_rng(M).choice(N, 1024, replace=False))
         rows = np.concatenate([[0, 1, N - 2, N - 1], rows])
-        Wr = host_bytes(W.view(N, -1)[torch.from_numpy(rows).cuda()].reshape(-1))
+        # the sampled rows keep the column-major super-block layout
+        idx = torch.from_numpy(rows).cuda()
+        Wr = host_bytes(W.view(K // 256, N, 144)[:, idx, :].contiguous().reshape(-1))
         xb = x.cpu().view(torch.int16).numpy().view(np.uint16)
         y_ref, S = oracle.gemv(Wr, xb, M, len(rows), K)
         assert_gemv_close(y[:, torch.from_numpy(rows).cuda()], y_ref, S, f"head M={M}")

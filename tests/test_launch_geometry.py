@@ -11,113 +11,87 @@ TX_LIMIT = (1 << 20) - 1           # mbarrier transaction-count range
 SMEM_OPTIN = 227 * 1024            # B200 opt-in shared memory per block
 
 
-def _next_pow2(v):
-    p = 1
-    while p < v:
-        p *= 2
-    return p
+def _wbox(R):
+    return -(-R * 144 // 128) * 128
 
 
-def _gemv_rsr(M):
-    return 4 if M <= 2 else 2
+def _stage_bytes(M, KC, R):
+    return KC * (_wbox(R) + M * 512)
 
 
 GEMV_SHAPES = [(1, 512, 1024), (1, 17408, 5120), (1, 5120, 17408), (1, 6144, 5120),
                (1, 5120, 6144), (1, 151936, 5120), (2, 5120, 17408), (3, 17408, 5120),
                (4, 6144, 5120), (5, 5120, 17408), (5, 151936, 5120), (1, 1, 256),
                (5, 3, 256), (1, 37, 4352), (3, 300, 1280), (2, 64, 65536), (5, 7, 32768),
-               (4, 100, 256), (1, 147, 512), (1, 149, 512)]
+               (4, 100, 256), (1, 147, 512), (1, 149, 512), (5, 1000, 2048), (2, 2, 17408),
+               (1, 1300, 512), (3, 40000, 768)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMV_SHAPES)
 @pytest.mark.parametrize("sms", [148, 132, 7])
 def test_gemv_geometry(M, N, K, sms):
     p = q4dec.plan_gemv(M, N, K, sms)
-    W, rsr = p.words_per_thread, p.rows_per_stream
-    assert rsr == _gemv_rsr(M) and W == {1: 4, 2: 2}.get(M, 1)
-    tps = 32 // W
     nsb = K // 256
-    ks = p.k_splits
-    assert p.threads % 32 == 0 and p.threads <= 640 and p.threads % p.row_streams == 0
-    tpr = p.threads // p.row_streams
-    assert tpr % 32 == 0 and tpr >= p.sb_per_split * tps
-    vpad = _next_pow2(rsr * M)
-    assert vpad <= 32 and p.row_streams * rsr * M <= p.threads
-    slot = p.row_streams * rsr * p.sb_per_split * 144
-    nwarps = p.threads // 32
-    assert p.smem_bytes == p.stages * slot + 2 * nwarps * vpad * 4 + p.stages * 8
-    assert p.smem_bytes <= SMEM_OPTIN and (p.stages * slot + 2 * nwarps * vpad * 4) % 8 == 0
+    ks, KC = p.k_splits, p.chunk_sb
+    assert p.threads == 288 and nsb % ks == 0 and p.sb_per_split == nsb // ks
+    assert KC in (1, 2, 4) and p.sb_per_split % KC == 0
+    assert 1 <= p.grid_rows <= sms and p.grid_rows * ks <= max(sms, p.grid_rows)
+    R = p.rows_per_pass
+    tiles = R // 16
+    assert R % 16 == 0 and 1 <= tiles <= 8 and tiles == min(8, -(-p.rows_per_cta // 16))
+    wbox, stage = _wbox(R), _stage_bytes(M, KC, R)
+    xoff = KC * wbox
+    assert stage % 128 == 0 and xoff % 128 == 0 and wbox >= R * 144
+    red = 8 * 8 * 32 * 16
+    assert p.smem_bytes == p.stages * stage + red + p.stages * 16
+    assert 2 <= p.stages <= 16 and p.smem_bytes <= SMEM_OPTIN
+    assert (p.stages * stage + red) % 8 == 0
     assert p.workspace_bytes == (ks * M * N * 4 if ks > 1 else 0)
     w_bytes = N * nsb * 144
     out_len = ks * M * N if ks > 1 else M * N
+    n_chunks = p.sb_per_split // KC
 
-    # K ranges partition the super-blocks
-    sb_base, sb_rem = nsb // ks, nsb % ks
-    covered = []
-    for k in range(ks):
-        cnt = sb_base + (1 if k < sb_rem else 0)
-        sb0 = k * sb_base + min(k, sb_rem)
-        assert 1 <= cnt <= p.sb_per_split
-        covered.extend(range(sb0, sb0 + cnt))
-    assert covered == list(range(nsb))
+    # bank pattern of the A-word loads: 32 lanes (g, t) read row g, word t at a
+    # 144-byte pitch
+    banks = {((g * 144 + 4 * t) // 4) % 32 for g in range(8) for t in range(4)}
+    assert len(banks) == 32
 
-    # threads of one row stream: words and scales inside the row segment,
-    # activations inside x
-    for k in range(ks):
-        cnt = sb_base + (1 if k < sb_rem else 0)
-        sb0 = k * sb_base + min(k, sb_rem)
-        seg = cnt * 144
-        seen = set()
-        for tid in range(p.threads):
-            stream, idx = divmod(tid, tpr)
-            assert stream < p.row_streams
-            sb_local, word0 = idx // tps, (idx % tps) * W
-            if sb_local >= cnt:
-                continue
-            blk = word0 >> 2
-            word_off = sb_local * 144 + word0 * 4
-            scale_off = sb_local * 144 + 128 + blk * 2
-            assert word_off % (4 * W) == 0 and word_off + 4 * W <= sb_local * 144 + 128
-            assert scale_off + 2 <= seg
-            for w in range(W):
-                klo = (sb0 + sb_local) * 256 + blk * 32 + 4 * ((word0 + w) & 3)
-                assert klo % 4 == 0 and klo + 16 + 4 <= K and (sb0 + sb_local) * 256 <= klo
-                if stream == 0:
-                    for c in range(4):
-                        seen.add(klo + c)
-                        seen.add(klo + 16 + c)
-        assert seen == set(range(sb0 * 256, (sb0 + cnt) * 256))
-
-    # rows: CTAs partition [0, N); copies stay inside W and the slot
     rows = []
-    per_stage = p.row_streams * rsr
-    for k in range(ks):
-        cnt = sb_base + (1 if k < sb_rem else 0)
-        sb0 = k * sb_base + min(k, sb_rem)
-        seg = cnt * 144
-        for cta in range(p.grid_rows):
-            rb, re_ = N * cta // p.grid_rows, N * (cta + 1) // p.grid_rows
-            assert re_ > rb
-            if k == 0:
-                rows.extend(range(rb, re_))
-            n_st = (re_ - rb + per_stage - 1) // per_stage
-            for st in range(n_st):
-                r0 = rb + st * per_stage
-                nr = min(per_stage, re_ - r0)
-                assert nr >= 1 and nr * seg <= slot and nr * seg <= TX_LIMIT
-                if ks == 1:
-                    lo, hi = r0 * nsb * 144, r0 * nsb * 144 + nr * seg
-                    assert lo % 16 == 0 and hi <= w_bytes
-                else:
-                    for r in range(nr):
-                        lo = ((r0 + r) * nsb + sb0) * 144
-                        assert lo % 16 == 0 and lo + seg <= w_bytes
-                # final stores
-                for tid in range(per_stage * M):
-                    lr, m = divmod(tid, M)
-                    if lr < nr:
-                        assert (k * M + m) * N + r0 + lr < out_len
+    for cta in range(p.grid_rows):
+        rb, re_ = N * cta // p.grid_rows, N * (cta + 1) // p.grid_rows
+        assert 1 <= re_ - rb <= p.rows_per_cta
+        rows.extend(range(rb, re_))
+        n_passes = -(-(re_ - rb) // R)
+        for k in range(ks):
+            for st in range(n_passes * n_chunks):
+                pss, chunk = divmod(st, n_chunks)
+                r0 = rb + pss * R
+                nr = min(R, re_ - r0)
+                assert 1 <= nr
+                assert KC * (nr * 144 + M * 512) <= TX_LIMIT
+                for j in range(KC):
+                    sb = k * p.sb_per_split + chunk * KC + j
+                    src = (sb * N + r0) * 144            # contiguous rows of column sb
+                    assert sb < nsb and src % 16 == 0 and src + nr * 144 <= w_bytes
+                    assert (sb * 256 * 2) % 16 == 0      # activation box x coordinate
+                    assert j * wbox + nr * 144 <= xoff
+                    assert xoff + (j + 1) * M * 512 <= stage
+                if chunk == n_chunks - 1:
+                    for r in (0, nr - 1):
+                        for m in range(M):
+                            assert (k * M + m) * N + r0 + r < out_len
     assert rows == list(range(N))
+
+    # per-warp shared-memory reads stay inside the weight piece / activation box
+    for warp in range(8):
+        for t in range(4):
+            woff = 7 * 144 + warp * 16 + t * 4           # largest g
+            assert (16 * (tiles - 1) + 8) * 144 + woff + 4 <= R * 144
+            for j in range(KC):
+                xo = (j * M + (M - 1)) * 512 + (warp * 32 + 4 * t) * 2
+                assert xo + 32 + 8 <= KC * M * 512
+        doff = 7 * 144 + 128 + warp * 2
+        assert (16 * (tiles - 1) + 8) * 144 + doff + 2 <= R * 144
 
 
 ATTN_CASES = [(4096, 24, 4, 1), (4096, 24, 4, 5), (65536, 24, 4, 5), (262144, 24, 4, 1),

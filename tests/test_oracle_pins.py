@@ -36,14 +36,16 @@ def _fraction_f16(bits: int) -> Fraction:
     return sign * (1 + Fraction(frac, 1024)) * Fraction(2) ** (exp - 15)
 
 
-def _brute_weights(buf, rows, K):
-    """Pure-Python reading of the super-block layout, in rationals."""
+def _brute_weights(buf, rows, K, column_major=False):
+    """Pure-Python reading of the super-block layout, in rationals: rows of
+    consecutive super-blocks (K/V caches), or the weight layout where
+    super-block (r, s) sits at (s * rows + r) * 144."""
     raw = bytes(np.asarray(buf, dtype=np.uint8).tobytes())
     nsb = K // 256
     w = [[Fraction(0)] * K for _ in range(rows)]
     for r in range(rows):
         for s in range(nsb):
-            base = (r * nsb + s) * 144
+            base = ((s * rows + r) if column_major else (r * nsb + s)) * 144
             for b in range(8):
                 d = _fraction_f16(raw[base + 128 + 2 * b] | (raw[base + 129 + 2 * b] << 8))
                 for j in range(16):
@@ -139,18 +141,41 @@ def test_superblock_offsets_single_nibble():
 
 
 def test_oracle_reading_matches_bruteforce_reader():
-    buf = synth.q4_0_weights(21, 3, 512)
-    w = oracle.dequant(buf, 3, 512)
-    wb = _brute_weights(buf, 3, 512)
+    rows = synth.pack_superblocks(np.random.default_rng(21).integers(0, 16, size=(3, 512)),
+                                  np.random.default_rng(22).integers(0, 0x7C00, size=(3, 16)))
+    w = oracle.dequant(rows, 3, 512)
+    wb = _brute_weights(rows, 3, 512)
     for r in range(3):
         assert [Fraction(v) for v in w[r]] == wb[r]
+    buf = synth.q4_0_weights(21, 5, 768)
+    w = oracle.dequant_weights(buf, 5, 768)
+    wb = _brute_weights(buf, 5, 768, column_major=True)
+    for r in range(5):
+        assert [Fraction(v) for v in w[r]] == wb[r]
+
+
+def test_weight_layout_single_nibble():
+    # weights are super-block-column-major: super-block (n, s) at (s*N + n)*144
+    N, K = 4, 768
+    q = np.full((N, K), 8, dtype=np.uint8)
+    d = np.full((N, K // 32), 0.25, dtype=np.float32)
+    q[2, 256 + 3 * 32 + 5] = 12                     # row 2, super-block 1, block 3, byte 5 lo
+    buf = synth.weights_from_parts(q, d)
+    assert buf.size == N * 3 * 144
+    off = (1 * N + 2) * 144 + 16 * 3 + 5
+    assert buf[off] == (12 | (8 << 4))
+    assert np.count_nonzero(buf.reshape(-1, 144)[:, :128] != 0x88) == 1
+    w = oracle.dequant_weights(buf, N, K)
+    assert np.argwhere(w != 0).tolist() == [[2, 256 + 3 * 32 + 5]] and w[2, 357] == 1.0
+    assert np.array_equal(oracle.weight_rows(buf, N, K).reshape(N, 3, 144)[2, 1],
+                          buf.reshape(3, N, 144)[1, 2])
 
 
 # ----------------------------------------------------------------- GEMV ----
 def test_one_hot_x_picks_one_weight_column():
     N, K = 5, 512
     buf = synth.q4_0_weights(3, N, K)
-    w = oracle.dequant(buf, N, K)
+    w = oracle.dequant_weights(buf, N, K)
     for k in (0, 17, 31, 32, 255, 256, 511):
         x = np.zeros((1, K), dtype=np.uint16)
         x[0, k] = 0x3F80  # 1.0
@@ -162,7 +187,7 @@ def test_all_q8_gives_exact_zero():
     N, K, M = 6, 1024, 3
     q = np.full((N, K), 8, dtype=np.uint8)
     d = np.abs(np.random.default_rng(1).standard_normal((N, K // 32))).astype(np.float32)
-    buf = synth.from_parts(q, d)
+    buf = synth.weights_from_parts(q, d)
     x = synth.activations(2, M, K)
     y, S = oracle.gemv(buf, x, M, N, K)
     assert np.all(y == 0.0) and np.all(S == 0.0)
@@ -176,11 +201,11 @@ def test_linear_in_one_block_scale():
     q = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
     d = (2.0 ** -rng.integers(1, 6, size=(N, K // 32))).astype(np.float32)
     x = synth.f32_to_bf16_bits(rng.integers(-4, 5, size=(1, K)).astype(np.float32))
-    y0, _ = oracle.gemv(synth.from_parts(q, d), x, 1, N, K)
+    y0, _ = oracle.gemv(synth.weights_from_parts(q, d), x, 1, N, K)
     b = 9
     d2 = d.copy()
     d2[:, b] *= 2
-    y1, _ = oracle.gemv(synth.from_parts(q, d2), x, 1, N, K)
+    y1, _ = oracle.gemv(synth.weights_from_parts(q, d2), x, 1, N, K)
     xs = oracle.bf16_bits_to_f64(x)[0, 32 * b: 32 * b + 32]
     contrib = (d[:, b:b + 1].astype(np.float64) * (q[:, 32 * b:32 * b + 32] - 8.0)) @ xs
     assert np.array_equal(y1[0] - y0[0], contrib)
@@ -189,8 +214,8 @@ def test_linear_in_one_block_scale():
 def test_linear_in_x():
     N, K = 4, 768
     rng = np.random.default_rng(8)
-    buf = synth.from_parts(rng.integers(0, 16, size=(N, K), dtype=np.uint8),
-                           (2.0 ** -rng.integers(2, 8, size=(N, K // 32))).astype(np.float32))
+    buf = synth.weights_from_parts(rng.integers(0, 16, size=(N, K), dtype=np.uint8),
+                                   (2.0 ** -rng.integers(2, 8, size=(N, K // 32))).astype(np.float32))
     a = rng.integers(-3, 4, size=(1, K)).astype(np.float32)
     b = rng.integers(-3, 4, size=(1, K)).astype(np.float32)
     ya, _ = oracle.gemv(buf, synth.f32_to_bf16_bits(a), 1, N, K)
@@ -216,7 +241,7 @@ def test_exact_integer_case_against_python_ints():
     q = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
     kexp = rng.integers(0, 6, size=(N, K // 32))
     xi = rng.integers(-7, 8, size=(M, K))
-    buf = synth.from_parts(q, (2.0 ** -kexp).astype(np.float32))
+    buf = synth.weights_from_parts(q, (2.0 ** -kexp).astype(np.float32))
     y, _ = oracle.gemv(buf, synth.f32_to_bf16_bits(xi.astype(np.float32)), M, N, K)
     for m in range(M):
         for n in range(N):
@@ -230,7 +255,7 @@ def test_gemv_against_rational_bruteforce():
     buf = synth.q4_0_weights(41, N, K)
     x = synth.activations(42, M, K)
     y, S = oracle.gemv(buf, x, M, N, K)
-    w = _brute_weights(buf, N, K)
+    w = _brute_weights(buf, N, K, column_major=True)
     for m in range(M):
         xs = [_fraction_bf16(int(b)) for b in x[m]]
         for n in range(N):
