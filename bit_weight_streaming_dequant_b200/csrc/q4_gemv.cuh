@@ -67,45 +67,6 @@ struct alignas(64) GemvArgs {
   int stages;
 };
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
-  uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(magic));
-  return r;  // (a & mask) | magic
-}
-
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
-// Four bf16x2 registers holding q - 8 (exact) for the 8 nibbles of word w:
-// r[0] = (byte0.lo, byte2.lo), r[1] = (byte0.hi, byte2.hi),
-// r[2] = (byte1.lo, byte3.lo), r[3] = (byte1.hi, byte3.hi).
-// 0x4300 | q is the bf16 value 128 + q; subtracting 136 leaves q - 8.
-__device__ __forceinline__ void dequant_pairs(uint32_t w, uint32_t mask, uint32_t magic,
-                                              uint32_t c136, uint32_t (&r)[4]) {
-  r[0] = bf16x2_sub(lop3_and_or(w, mask, magic), c136);
-  r[1] = bf16x2_sub(lop3_and_or(w >> 4, mask, magic), c136);
-  r[2] = bf16x2_sub(lop3_and_or(w >> 8, mask, magic), c136);
-  r[3] = bf16x2_sub(lop3_and_or(w >> 12, mask, magic), c136);
-}
-
-__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar, uint64_t policy) {
   asm volatile(

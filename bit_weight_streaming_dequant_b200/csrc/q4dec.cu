@@ -25,6 +25,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kPlanFallbackSms = 148;
 constexpr size_t kGemvSmemBudget = 224 * 1024;   // shared memory per GEMV CTA
+constexpr size_t kAttnSmemBudget = 224 * 1024;   // shared memory per attention CTA
 
 struct DeviceState {
   std::atomic<bool> ready{false};
@@ -253,6 +254,18 @@ q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, in
   return Q4D_OK;
 }
 
+template <int NRT>
+q4d_status launch_attn_t(const q4d::AttnArgs& a, const q4d_attn_plan& p, int n_kv, int dev,
+                         const DeviceState& s, cudaStream_t stream) {
+  static std::atomic<bool> smem_set[kMaxDevices];
+  auto kernel = q4d::q4kv_attn_split_kernel<NRT>;
+  q4d_status st = allow_smem(kernel, dev, s, smem_set);
+  if (st != Q4D_OK) return st;
+  dim3 grid(p.n_splits, n_kv, p.row_groups);
+  kernel<<<grid, p.threads, p.smem_bytes, stream>>>(a);
+  return Q4D_OK;
+}
+
 q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out, int ctx_len,
                      int n_q, int n_kv, int head_dim, int M, int kv_stride, float scale,
                      cudaStream_t stream, void* workspace, size_t workspace_bytes,
@@ -277,6 +290,7 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
   }
 
   q4d::AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
   a.Q = static_cast<const uint16_t*>(Q);
   a.K = static_cast<const uint8_t*>(Kq4);
   a.V = static_cast<const uint8_t*>(Vq4);
@@ -290,16 +304,19 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
   a.M = M;
   a.g = n_q / n_kv;
   a.kv_stride = kv_stride;
-  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;  // log2(e): the kernel works in base 2
   a.n_splits = p.n_splits;
   a.split_tokens = p.split_tokens;
   a.rows_per_cta = p.rows_per_cta;
   a.stages = p.stages;
 
-  static std::atomic<bool> smem_set[kMaxDevices];
-  if ((st = allow_smem(q4d::q4kv_attn_split_kernel, dev, *s, smem_set)) != Q4D_OK) return st;
-  dim3 grid(p.n_splits, n_kv, p.row_groups);
-  q4d::q4kv_attn_split_kernel<<<grid, p.threads, p.smem_bytes, stream>>>(a);
+  switch ((p.rows_per_cta + 7) / 8) {
+    case 1: st = launch_attn_t<1>(a, p, n_kv, dev, *s, stream); break;
+    case 2: st = launch_attn_t<2>(a, p, n_kv, dev, *s, stream); break;
+    case 3: st = launch_attn_t<3>(a, p, n_kv, dev, *s, stream); break;
+    default: st = launch_attn_t<4>(a, p, n_kv, dev, *s, stream); break;
+  }
+  if (st != Q4D_OK) return st;
   if (p.n_splits > 1) q4d::q4kv_attn_merge_kernel<<<M * n_q, 256, 0, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
   return Q4D_OK;
@@ -389,12 +406,20 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   const int rows_all = (n_q_heads / n_kv_heads) * M;
   const int row_groups = ceil_div(rows_all, q4d::kAttnMaxRows);
   const int rows_per_cta = ceil_div(rows_all, row_groups);
+  // One CTA per SM (the K/V ring takes most of shared memory): enough context
+  // splits that (splits x KV heads x row groups) fills the SMs once, each
+  // split at least two tiles long and at most 256 splits (the merge kernel's
+  // limit).
   const long long ctas_per_split = (long long)n_kv_heads * row_groups;
-  int n_splits = int(std::max<long long>(1, (2LL * num_sms + ctas_per_split - 1) / ctas_per_split));
-  n_splits = std::min(n_splits, std::max(1, ceil_div(ctx_len, 4 * TT)));
+  int n_splits = int(std::max<long long>(1, (num_sms + ctas_per_split - 1) / ctas_per_split));
+  n_splits = std::min(n_splits, std::max(1, ceil_div(ctx_len, 2 * TT)));
+  n_splits = std::min(n_splits, 256);
   const int split_tokens = int(round_up(ceil_div(ctx_len, n_splits), TT));
   n_splits = ceil_div(ctx_len, split_tokens);
-  const int stages = 3;
+  // As many ring stages as fit next to the fixed buffers, up to 8.
+  const size_t fixed = q4d::attn_smem_bytes(0);
+  int stages = int((kAttnSmemBudget - fixed) / (q4d::kAttnStageBytes + 16));
+  stages = std::max(2, std::min(8, stages));
   plan->n_splits = n_splits;
   plan->split_tokens = split_tokens;
   plan->tile_tokens = TT;
@@ -402,9 +427,7 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   plan->rows_per_cta = rows_per_cta;
   plan->stages = stages;
   plan->threads = q4d::kAttnThreads;
-  plan->smem_bytes = size_t(q4d::kAttnMaxRows) * q4d::kHeadDim * 4 +
-                     size_t(stages) * 2 * TT * q4d::kRowBytes + size_t(TT) * q4d::kAttnMaxRows * 4 +
-                     3 * q4d::kAttnMaxRows * 4 + size_t(stages) * 8;
+  plan->smem_bytes = q4d::attn_smem_bytes(stages);
   plan->workspace_bytes =
       n_splits > 1 ? size_t(n_splits) * M * n_q_heads * (q4d::kHeadDim + 2) * 4 : 0;
   return Q4D_OK;

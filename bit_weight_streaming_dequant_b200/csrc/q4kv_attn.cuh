@@ -1,4 +1,4 @@
-// Causal GQA flash-decode attention over a Q4_0 K/V cache (CUDA cores).
+// Causal GQA flash-decode attention over a Q4_0 K/V cache, on tensor cores.
 //
 // What it computes: for draft row m at position p_m = ctx_len - M + m and
 // query head h, softmax over tokens t <= p_m of s = scale * Q . Khat, applied
@@ -6,29 +6,56 @@
 // 24GB RTX PRO 4000 SFF (432 GB/s): 50 tok/s with MTP", paragraphs on the 16
 // full-attention layers and on the 432 GB/s ceiling).
 //
-// Design:
-//  * Grid = (context split, KV head, query-row group).  One CTA holds every
-//    query row that reads its KV head (g grouped heads x M draft rows, up to
-//    32), so each K/V byte of its split is read from HBM exactly once.
-//  * K and V tiles of 64 tokens stream through a shared-memory ring with
-//    cp.async.bulk completing on mbarriers (bounded waits).
-//  * Per tile: scores (thread = token x row group, block scale applied once
-//    per 32-element block), online softmax (warp per query row), then P.V
-//    (thread = output dimension, nibble dequantised in registers).
-//  * Each split writes its running (max, sum, unnormalised o); a second kernel
-//    merges the splits with log-sum-exp weights.  A single split writes the
-//    normalised output directly.
+// Work split: grid = (context split, KV head, query-row group).  One CTA holds
+// every query row that reads its KV head (g grouped heads x M draft rows, at
+// most 32) so each K/V byte of its split leaves HBM once; the splits' softmax
+// states are merged by a second kernel (log-sum-exp, base 2).
+//
+// Per 128-token tile (one producer warp bulk-copies the K and V tiles --
+// contiguous, one super-block per token -- into a ring of stages on
+// full/empty mbarriers with bounded waits; eight consumer warps compute):
+//  1. Scores, exact: warp w takes tokens 16w..16w+15.  ldmatrix hands lane
+//     (g, t) word t of the 16-byte nibble piece of tokens g and g+8 (the
+//     A-fragment layout); nibbles become exact bf16 (q - 8); Q (bf16) is the
+//     B operand, pre-arranged in shared memory in the same element order; one
+//     fresh MMA accumulator per 32-element block is scaled by that token's
+//     fp32 block scale.  S^T = Khat Q^T arrives as (token, row) fragments.
+//  2. Online softmax in base 2 (scale * log2 e folded in): per-row tile max
+//     across the eight warps through shared memory, running max m and
+//     per-lane partial sums l rescaled by 2^(m_old - m_new); P = 2^(s - m) is
+//     rounded to fp16 and stored as P^T [token][row]; l adds the same rounded
+//     values, so numerator and denominator see identical weights.
+//  3. P.V: warp w owns the 32 dimensions of block w.  ldmatrix.trans pairs two
+//     tokens' bytes of the V piece in one register, so the A operand
+//     (q - 8)^T [dims][tokens] unpacks in registers, exact in fp16; the block
+//     scale d of V goes into the B operand instead: P^T (ldmatrix.trans) times
+//     d of the same tokens, one fp16 multiply, |P d| <= |d| so it cannot
+//     overflow.  O^T [dims][rows] accumulates in fp32 across the split.
 #pragma once
 
 #include "q4dec_device.cuh"
 
 namespace q4d {
 
-constexpr int kAttnThreads = 256;
-constexpr int kAttnTileTokens = 64;
-constexpr int kAttnMaxRows = 32;
+constexpr int kAttnConsumerWarps = 8;
+constexpr int kAttnThreads = (kAttnConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kAttnTileTokens = 128;
+constexpr int kAttnMaxRows = 32;                              // 4 row tiles of 8
 constexpr int kHeadDim = 256;
-constexpr int kRowBytes = 144;  // one super-block per token
+constexpr int kRowBytes = 144;                                // one super-block per token
+constexpr int kPtPitch = 80;                                  // bytes per token row of P^T
+constexpr int kQPitch = 8 * 4 * 16 + 64;                      // bytes per row of Q fragments
+constexpr uint32_t kAttnStageBytes = 2u * kAttnTileTokens * kRowBytes;  // K tile + V tile
+
+// Dynamic shared memory of the split kernel for a given stage count.
+__host__ __device__ constexpr size_t attn_smem_bytes(int stages) {
+  return size_t(stages) * kAttnStageBytes                // K/V ring
+         + size_t(kAttnMaxRows) * kQPitch                // Q fragments [row][block][t] x 16 B
+         + size_t(kAttnTileTokens) * kPtPitch            // P^T fp16
+         + size_t(kAttnMaxRows) * kAttnConsumerWarps * 4 // per-warp row maxima
+         + size_t(kAttnMaxRows) * 4                      // per-row final sums
+         + size_t(stages) * 16;                          // full / empty barriers
+}
 
 struct AttnArgs {
   const uint16_t* Q;   // bf16 bits [M][n_q][256]
@@ -36,27 +63,92 @@ struct AttnArgs {
   const uint8_t* V;
   float* out;          // [M][n_q][256]
   float* ws_o;         // [n_splits][M*n_q][256]
-  float* ws_ml;        // [n_splits][M*n_q][2]
+  float* ws_ml;        // [n_splits][M*n_q][2] (running max in log2 units, sum)
   unsigned* err;
   int ctx_len, n_q, n_kv, M, g, kv_stride;
-  float scale;
+  float scale_log2;    // softmax scale * log2(e)
   int n_splits, split_tokens, rows_per_cta, stages;
 };
 
-__device__ __forceinline__ float nib_minus8(uint32_t q) {
-  return __uint_as_float(0x4B000000u | q) - 8388616.0f;  // (2^23 + q) - (2^23 + 8)
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t f16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
+                                              uint32_t a2, uint32_t a3, uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void attn_consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kAttnConsumerWarps * 32) : "memory");
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 2) q4kv_attn_split_kernel(const AttnArgs a) {
-  constexpr int TT = kAttnTileTokens, RM = kAttnMaxRows;
+// Fp16 pair q - 8 (exact) for the two tokens held in the halves of `r`:
+// the nibble at bits 0-3 (LOW) or 4-7 (!LOW) of each half.  0x6400 | q is the
+// fp16 value 1024 + q and 0x6400 | (q << 4) is 1024 + 16 q; one fma whose
+// exact result is q - 8 finishes it.
+template <bool LOW>
+__device__ __forceinline__ uint32_t q8_pair(uint32_t r) {
+  if (LOW)
+    return f16x2_fma(lop3_and_or(r, 0x000F000Fu, 0x64006400u), 0x3C003C00u,
+                     0xE408E408u /* -1032 */);
+  return f16x2_fma(lop3_and_or(r, 0x00F000F0u, 0x64006400u), 0x2C002C00u /* 1/16 */,
+                   0xD480D480u /* -72 */);
+}
+
+// NRT: row tiles of 8 query rows (1..4).  A single row tile keeps its Q
+// fragments in registers for the whole split; more read them from shared
+// memory at every use.
+template <int NRT>
+__global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const AttnArgs a) {
+  constexpr int TT = kAttnTileTokens;
+  constexpr bool kQReg = NRT == 1;
   extern __shared__ __align__(128) uint8_t smem[];
-  float* Qs = reinterpret_cast<float*>(smem);                       // [RM][256]
-  uint8_t* ring = smem + RM * kHeadDim * 4;                          // [stages][2][TT*144]
-  float* Ps = reinterpret_cast<float*>(ring + size_t(a.stages) * 2 * TT * kRowBytes);  // [TT][RM]
-  float* m_run = Ps + TT * RM;
-  float* l_run = m_run + RM;
-  float* alpha = l_run + RM;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(alpha + RM);
+  const int S = a.stages;
+  uint8_t* ring = smem;
+  uint8_t* Qp = ring + size_t(S) * kAttnStageBytes;                 // [row] x kQPitch
+  uint8_t* Pt = Qp + kAttnMaxRows * kQPitch;                         // [token] x kPtPitch, fp16
+  float* red = reinterpret_cast<float*>(Pt + TT * kPtPitch);        // [row][warp]
+  float* row_sum = red + kAttnMaxRows * kAttnConsumerWarps;          // [row]
+  uint64_t* full = reinterpret_cast<uint64_t*>(row_sum + kAttnMaxRows);
+  uint64_t* empty = full + S;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x, kh = blockIdx.y, rgrp = blockIdx.z;
@@ -70,205 +162,359 @@ __global__ void __launch_bounds__(kAttnThreads, 2) q4kv_attn_split_kernel(const 
   const uint8_t* Vh = a.V + size_t(kh) * a.kv_stride * kRowBytes;
 
   if (tid == 0) {
-    for (int s = 0; s < a.stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_addr(&full[s]), 1);
+      mbar_init(smem_addr(&empty[s]), kAttnConsumerWarps);
+    }
     mbar_init_fence();
   }
   __syncthreads();
 
-  const uint64_t pol = l2_evict_first_policy();
-  auto issue = [&](int tile) {
-    const int slot = tile % a.stages;
-    const int t0 = t_begin + tile * TT;
-    const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * kRowBytes;
-    const uint32_t bar = smem_addr(&bars[slot]);
-    const uint32_t dk = smem_addr(ring + size_t(slot) * 2 * TT * kRowBytes);
-    mbar_arrive_expect_tx(bar, 2 * bytes);
-    bulk_g2s(dk, Kh + size_t(t0) * kRowBytes, bytes, bar, pol);
-    bulk_g2s(dk + TT * kRowBytes, Vh + size_t(t0) * kRowBytes, bytes, bar, pol);
-  };
-  if (tid == 0) {
-    const int pre = min(a.stages, n_tiles);
-    for (int t = 0; t < pre; ++t) issue(t);
+  if (warp == kAttnConsumerWarps) {
+    // ---------------- producer: K and V tiles, one bulk copy each ----------
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();
+      int slot = 0;
+      uint32_t phase = 0;
+      for (int tile = 0; tile < n_tiles; ++tile) {
+        if (tile >= S) mbar_wait(smem_addr(&empty[slot]), phase ^ 1u, a.err);
+        const int t0 = t_begin + tile * TT;
+        const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * kRowBytes;
+        const uint32_t bar = smem_addr(&full[slot]);
+        const uint32_t dk = smem_addr(ring + size_t(slot) * kAttnStageBytes);
+        mbar_arrive_expect_tx(bar, 2 * bytes);
+        bulk_g2s(dk, Kh + size_t(t0) * kRowBytes, bytes, bar, pol);
+        bulk_g2s(dk + TT * kRowBytes, Vh + size_t(t0) * kRowBytes, bytes, bar, pol);
+        if (++slot == S) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    return;
   }
 
-  // Stage the queries (scaled) as fp32, rows r = m*g + j of this row group.
-  for (int i = tid; i < RM * kHeadDim; i += kAttnThreads) {
-    const int r = i / kHeadDim, c = i - r * kHeadDim;
-    float q = 0.f;
+  // ---------------- consumers ----------------
+  const int g = lane >> 2, t = lane & 3;
+
+  // Q fragments.  For row r, block b and lane t, 16 bytes: the bf16 pairs
+  // (q[4t], q[4t+2]), (q[16+4t], q[16+4t+2]), (q[4t+1], q[4t+3]),
+  // (q[16+4t+1], q[16+4t+3]) of the block -- the element order in which the
+  // nibbles of word t of a K row unpack.  Rows past R are zero.
+  for (int i = tid; i < kAttnMaxRows * 32; i += kAttnConsumerWarps * 32) {
+    const int r = i >> 5, b = (i >> 2) & 7, tt = i & 3;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (r < R) {
       const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
-      const int h = kh * a.g + j;
-      q = bf16_bits_to_float(a.Q[(size_t(m) * a.n_q + h) * kHeadDim + c]) * a.scale;
+      const uint16_t* q = a.Q + (size_t(m) * a.n_q + kh * a.g + j) * kHeadDim + b * 32 + 4 * tt;
+      const uint2 lo = *reinterpret_cast<const uint2*>(q);
+      const uint2 hi = *reinterpret_cast<const uint2*>(q + 16);
+      v.x = prmt(lo.x, lo.y, 0x5410);
+      v.y = prmt(hi.x, hi.y, 0x5410);
+      v.z = prmt(lo.x, lo.y, 0x7632);
+      v.w = prmt(hi.x, hi.y, 0x7632);
     }
-    Qs[i] = q;
+    *reinterpret_cast<uint4*>(Qp + r * kQPitch + (i & 31) * 16) = v;
   }
-  if (tid < RM) {
-    m_run[tid] = -INFINITY;
-    l_run[tid] = 0.f;
+  attn_consumer_sync();
+  const uint32_t Qp_addr = smem_addr(Qp), Pt_addr = smem_addr(Pt);
+  uint4 qreg[kQReg ? NRT : 1][kQReg ? 8 : 1];
+  if (kQReg) {
+    #pragma unroll
+    for (int rt = 0; rt < NRT; ++rt)
+      #pragma unroll
+      for (int b = 0; b < 8; ++b)
+        qreg[rt][b] = *reinterpret_cast<const uint4*>(Qp + (8 * rt + g) * kQPitch + (b * 4 + t) * 16);
   }
-  __syncthreads();
 
-  // score-phase mapping: token st, rows sr0 + 4*i
-  const int st = tid & (TT - 1);
-  const int sr0 = tid >> 6;
-  // PV-phase mapping: output dimension pd (block pb, byte pj, high nibble?)
-  const int pd = tid;
-  const int pb = pd >> 5, pe = pd & 31, pj = pe & 15;
-  const bool phi = pe >= 16;
-
-  float o[RM];
+  // rows this lane holds in every row tile: 8*rt + 2t + e, e = 0, 1
+  int row_pos[NRT][2];  // position of the row's draft token; -1 for padding rows
+  float m_run[NRT][2], l_run[NRT][2];
   #pragma unroll
-  for (int r = 0; r < RM; ++r) o[r] = 0.f;
+  for (int rt = 0; rt < NRT; ++rt)
+    #pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int r = 8 * rt + 2 * t + e;
+      row_pos[rt][e] = r < R ? a.ctx_len - a.M + (row0 + r) / a.g : -1;
+      m_run[rt][e] = -INFINITY;
+      l_run[rt][e] = 0.f;
+    }
+  float o[2][NRT][4];  // O^T fragments: [dim tile][row tile]
+  #pragma unroll
+  for (int d = 0; d < 2; ++d)
+    #pragma unroll
+    for (int rt = 0; rt < NRT; ++rt) o[d][rt][0] = o[d][rt][1] = o[d][rt][2] = o[d][rt][3] = 0.f;
 
+  const uint32_t bmask = 0x000F000Fu, bmagic = 0x43004300u, b136 = 0x43084308u;
+  int slot = 0;
+  uint32_t phase = 0;
+
+  #pragma unroll 1
   for (int tile = 0; tile < n_tiles; ++tile) {
-    const int slot = tile % a.stages;
     const int t0 = t_begin + tile * TT;
     const int n_tok = min(TT, t_end - t0);
-    mbar_wait(smem_addr(&bars[slot]), uint32_t(tile / a.stages) & 1u, a.err);
-    const uint8_t* Kt = ring + size_t(slot) * 2 * TT * kRowBytes;
+    mbar_wait(smem_addr(&full[slot]), phase, a.err);
+    const uint8_t* Kt = ring + size_t(slot) * kAttnStageBytes;
     const uint8_t* Vt = Kt + TT * kRowBytes;
+    const uint32_t Kt_addr = smem_addr(Kt), Vt_addr = smem_addr(Vt);
 
-    // ---- scores
+    // ---- 1. S^T for tokens 16*warp + g (a) and + g + 8 (b)
+    const int tok_a = 16 * warp + g, tok_b = tok_a + 8;
+    float s[NRT][4];
+    #pragma unroll
+    for (int rt = 0; rt < NRT; ++rt) s[rt][0] = s[rt][1] = s[rt][2] = s[rt][3] = 0.f;
     {
-      float s[RM / 4];
+      // ldmatrix rows: lanes 0-7 tokens 16w+0..7 block b, 8-15 tokens
+      // 16w+8..15 block b, 16-23 tokens 16w+0..7 block b+1, 24-31 tokens
+      // 16w+8..15 block b+1; lane (g, t) receives word t of each.
+      const uint32_t lbase = Kt_addr + uint32_t(16 * warp + (lane & 15)) * kRowBytes +
+                             uint32_t(lane >> 4) * 16u;
+      const uint8_t* da_p = Kt + tok_a * kRowBytes + 128;
+      const uint8_t* db_p = Kt + tok_b * kRowBytes + 128;
       #pragma unroll
-      for (int i = 0; i < RM / 4; ++i) s[i] = 0.f;
-      if (st < n_tok) {
-        const uint8_t* krow = Kt + st * kRowBytes;
-        #pragma unroll 1
-        for (int b = 0; b < 8; ++b) {
-          const uint4 nb = *reinterpret_cast<const uint4*>(krow + 16 * b);
-          const float db = half_bits_to_float(*reinterpret_cast<const uint16_t*>(krow + 128 + 2 * b));
-          const uint32_t wd[4] = {nb.x, nb.y, nb.z, nb.w};
-          float kv[32];
+      for (int b = 0; b < 8; b += 2) {
+        uint32_t w0a, w0b, w1a, w1b;
+        ldsm_x4(lbase + uint32_t(b) * 16u, w0a, w0b, w1a, w1b);
+        // (d_b, d_b+1) of tokens a and b
+        const float2 dA = __half22float2(*reinterpret_cast<const __half2*>(da_p + 2 * b));
+        const float2 dB = __half22float2(*reinterpret_cast<const __half2*>(db_p + 2 * b));
+        #pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          uint32_t qa[4], qb[4];
+          dequant_pairs(bb ? w1a : w0a, bmask, bmagic, b136, qa);
+          dequant_pairs(bb ? w1b : w0b, bmask, bmagic, b136, qb);
+          const float da = bb ? dA.y : dA.x, db = bb ? dB.y : dB.x;
           #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const uint32_t byte = (wd[j >> 2] >> (8 * (j & 3))) & 0xFFu;
-            kv[j] = nib_minus8(byte & 0xFu);
-            kv[j + 16] = nib_minus8(byte >> 4);
+          for (int rt = 0; rt < NRT; ++rt) {
+            uint4 qf;
+            if (kQReg) {
+              qf = qreg[kQReg ? rt : 0][kQReg ? b + bb : 0];
+            } else {
+              asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                           : "=r"(qf.x), "=r"(qf.y), "=r"(qf.z), "=r"(qf.w)
+                           : "r"(Qp_addr + uint32_t((8 * rt + g) * kQPitch + ((b + bb) * 4 + t) * 16)));
+            }
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_bf16(c, qa[0], qb[0], qa[1], qb[1], qf.x, qf.y);
+            mma_bf16(c, qa[2], qb[2], qa[3], qb[3], qf.z, qf.w);
+            s[rt][0] = fmaf(da, c[0], s[rt][0]);
+            s[rt][1] = fmaf(da, c[1], s[rt][1]);
+            s[rt][2] = fmaf(db, c[2], s[rt][2]);
+            s[rt][3] = fmaf(db, c[3], s[rt][3]);
           }
+        }
+      }
+      // base-2 logits, causal / tile-end mask, this warp's per-row maxima
+      const int ta = t0 + tok_a, tb = t0 + tok_b;
+      #pragma unroll
+      for (int rt = 0; rt < NRT; ++rt)
+        #pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int pos = row_pos[rt][e];
+          s[rt][e] = (tok_a < n_tok && ta <= pos) ? s[rt][e] * a.scale_log2 : -INFINITY;
+          s[rt][2 + e] = (tok_b < n_tok && tb <= pos) ? s[rt][2 + e] * a.scale_log2 : -INFINITY;
+          float mx = fmaxf(s[rt][e], s[rt][2 + e]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
+          if (g == 0) red[(8 * rt + 2 * t + e) * kAttnConsumerWarps + warp] = mx;
+        }
+    }
+    attn_consumer_sync();
+
+    // ---- 2. running max, rescale factors, P = 2^(s - m) as fp16 P^T
+    float alpha[NRT][2];
+    #pragma unroll
+    for (int rt = 0; rt < NRT; ++rt) {
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float4* rm =
+            reinterpret_cast<const float4*>(red + (8 * rt + 2 * t + e) * kAttnConsumerWarps);
+        const float4 x0 = rm[0], x1 = rm[1];
+        const float tile_max = fmaxf(fmaxf(fmaxf(x0.x, x0.y), fmaxf(x0.z, x0.w)),
+                                     fmaxf(fmaxf(x1.x, x1.y), fmaxf(x1.z, x1.w)));
+        const float m_new = fmaxf(m_run[rt][e], tile_max);
+        // a row with no visible token so far keeps m = -inf and weight 0
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        alpha[rt][e] = ex2(m_run[rt][e] - m_use);
+        m_run[rt][e] = m_new;
+        s[rt][e] = ex2(s[rt][e] - m_use);
+        s[rt][2 + e] = ex2(s[rt][2 + e] - m_use);
+      }
+      // P^T entries as fp16; the row sums add the same rounded weights
+      const uint32_t pa = pack_f16x2(s[rt][0], s[rt][1]);
+      const uint32_t pb = pack_f16x2(s[rt][2], s[rt][3]);
+      const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&pa));
+      const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&pb));
+      l_run[rt][0] = l_run[rt][0] * alpha[rt][0] + fa.x + fb.x;
+      l_run[rt][1] = l_run[rt][1] * alpha[rt][1] + fa.y + fb.y;
+      *reinterpret_cast<uint32_t*>(Pt + tok_a * kPtPitch + (8 * rt + 2 * t) * 2) = pa;
+      *reinterpret_cast<uint32_t*>(Pt + tok_b * kPtPitch + (8 * rt + 2 * t) * 2) = pb;
+    }
+    attn_consumer_sync();
+
+    // ---- 3. O^T[dims of block `warp`][rows] += Vhat^T P^T over the tile
+    #pragma unroll
+    for (int d = 0; d < 2; ++d)
+      #pragma unroll
+      for (int rt = 0; rt < NRT; ++rt) {
+        o[d][rt][0] *= alpha[rt][0];
+        o[d][rt][1] *= alpha[rt][1];
+        o[d][rt][2] *= alpha[rt][0];
+        o[d][rt][3] *= alpha[rt][1];
+      }
+    {
+      // ldmatrix.trans over the 16-byte V piece of block `warp`: lane i
+      // addresses token k0 + i, so matrix j covers tokens k0 + 8j .. +7 and
+      // lane (g, t) receives bytes 2g, 2g+1 of tokens k0 + 8j + 2t and +1.
+      const uint32_t vbase = Vt_addr + uint32_t(lane) * kRowBytes + uint32_t(warp) * 16u;
+      const uint32_t pbase = Pt_addr + uint32_t(lane & 15) * kPtPitch + uint32_t(lane >> 4) * 16u;
+      const uint8_t* vd = Vt + 128 + 2 * warp;
+      #pragma unroll 1
+      for (int k0 = 0; k0 < n_tok; k0 += 32) {
+        uint32_t v[4];
+        ldsm_x4_trans(vbase + uint32_t(k0) * kRowBytes, v[0], v[1], v[2], v[3]);
+        #pragma unroll
+        for (int h = 0; h < 2; ++h) {  // k16 step: tokens kb .. kb + 15
+          const int kb = k0 + 16 * h;
+          const int ta = kb + 2 * t, tb = ta + 8;
+          // block scales of tokens (ta, ta+1) and (tb, tb+1); zero past the
+          // tile end, where the shared memory holds no token of this split
+          uint32_t d_lo = uint32_t(*reinterpret_cast<const uint16_t*>(vd + ta * kRowBytes)) |
+                          (uint32_t(*reinterpret_cast<const uint16_t*>(vd + (ta + 1) * kRowBytes)) << 16);
+          uint32_t d_hi = uint32_t(*reinterpret_cast<const uint16_t*>(vd + tb * kRowBytes)) |
+                          (uint32_t(*reinterpret_cast<const uint16_t*>(vd + (tb + 1) * kRowBytes)) << 16);
+          if (kb + 16 > n_tok) {
+            d_lo &= (ta < n_tok ? 0xFFFFu : 0u) | (ta + 1 < n_tok ? 0xFFFF0000u : 0u);
+            d_hi &= (tb < n_tok ? 0xFFFFu : 0u) | (tb + 1 < n_tok ? 0xFFFF0000u : 0u);
+          }
+          const uint32_t ra = v[2 * h], rb = v[2 * h + 1];
+          // A fragments (q - 8, exact): dim tile 0 = block dims {2g, 2g+16},
+          // dim tile 1 = {2g+1, 2g+17}
+          const uint32_t a00 = q8_pair<true>(ra), a01 = q8_pair<false>(ra);
+          const uint32_t a02 = q8_pair<true>(rb), a03 = q8_pair<false>(rb);
+          const uint32_t a10 = q8_pair<true>(ra >> 8), a11 = q8_pair<false>(ra >> 8);
+          const uint32_t a12 = q8_pair<true>(rb >> 8), a13 = q8_pair<false>(rb >> 8);
           #pragma unroll
-          for (int i = 0; i < RM / 4; ++i) {
-            const int r = sr0 + 4 * i;
-            if (r < R) {
-              const float4* q4 = reinterpret_cast<const float4*>(Qs + r * kHeadDim + 32 * b);
-              float dot = 0.f;
-              #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float4 qv = q4[e];
-                dot = fmaf(kv[4 * e + 0], qv.x, dot);
-                dot = fmaf(kv[4 * e + 1], qv.y, dot);
-                dot = fmaf(kv[4 * e + 2], qv.z, dot);
-                dot = fmaf(kv[4 * e + 3], qv.w, dot);
-              }
-              s[i] = fmaf(db, dot, s[i]);
+          for (int rt = 0; rt < NRT; rt += 2) {
+            // B fragments: P^T of tokens (kb + 2t, +1) and (kb + 2t + 8, +9)
+            // times those tokens' block scales -- this warp's block only
+            const uint32_t paddr = pbase + uint32_t(kb) * kPtPitch + uint32_t(rt) * 16u;
+            if (rt + 1 < NRT) {
+              uint32_t p0, p1, p2, p3;
+              ldsm_x4_trans(paddr, p0, p1, p2, p3);
+              p0 = f16x2_mul(p0, d_lo);
+              p1 = f16x2_mul(p1, d_hi);
+              p2 = f16x2_mul(p2, d_lo);
+              p3 = f16x2_mul(p3, d_hi);
+              mma_f16(o[0][rt], a00, a01, a02, a03, p0, p1);
+              mma_f16(o[1][rt], a10, a11, a12, a13, p0, p1);
+              mma_f16(o[0][rt + 1], a00, a01, a02, a03, p2, p3);
+              mma_f16(o[1][rt + 1], a10, a11, a12, a13, p2, p3);
+            } else {
+              uint32_t p0, p1;
+              ldsm_x2_trans(paddr, p0, p1);
+              p0 = f16x2_mul(p0, d_lo);
+              p1 = f16x2_mul(p1, d_hi);
+              mma_f16(o[0][rt], a00, a01, a02, a03, p0, p1);
+              mma_f16(o[1][rt], a10, a11, a12, a13, p0, p1);
             }
           }
         }
       }
-      const int t_abs = t0 + st;
-      #pragma unroll
-      for (int i = 0; i < RM / 4; ++i) {
-        const int r = sr0 + 4 * i;
-        if (r < R) {
-          const int m = (row0 + r) / a.g;
-          const bool vis = st < n_tok && t_abs <= a.ctx_len - a.M + m;
-          Ps[st * RM + r] = vis ? s[i] : -INFINITY;
-        }
-      }
     }
-    __syncthreads();
-
-    // ---- online softmax, one warp per query row
-    for (int r = warp; r < R; r += kAttnThreads / 32) {
-      const float s0 = Ps[lane * RM + r], s1 = Ps[(lane + 32) * RM + r];
-      float mx = fmaxf(s0, s1);
-      #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-      const float m_old = m_run[r];
-      const float m_new = fmaxf(m_old, mx);
-      float p0 = 0.f, p1 = 0.f, al = 1.f;
-      if (m_new != -INFINITY) {
-        al = __expf(m_old - m_new);
-        p0 = __expf(s0 - m_new);
-        p1 = __expf(s1 - m_new);
-      }
-      float ps = p0 + p1;
-      #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, off);
-      Ps[lane * RM + r] = p0;
-      Ps[(lane + 32) * RM + r] = p1;
-      __syncwarp();
-      if (lane == 0) {
-        m_run[r] = m_new;
-        l_run[r] = al * l_run[r] + ps;
-        alpha[r] = al;
-      }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&empty[slot]));
+    if (++slot == S) {
+      slot = 0;
+      phase ^= 1u;
     }
-    __syncthreads();
-
-    // ---- o = alpha * o + P V, thread per output dimension
-    {
-      #pragma unroll
-      for (int r = 0; r < RM; ++r)
-        if (r < R) o[r] *= alpha[r];
-      #pragma unroll 2
-      for (int t = 0; t < n_tok; ++t) {
-        const uint8_t* vrow = Vt + t * kRowBytes;
-        const uint32_t byte = vrow[16 * pb + pj];
-        const float dv = half_bits_to_float(*reinterpret_cast<const uint16_t*>(vrow + 128 + 2 * pb));
-        const float v = dv * nib_minus8(phi ? (byte >> 4) : (byte & 0xFu));
-        const float4* p4 = reinterpret_cast<const float4*>(Ps + t * RM);
-        #pragma unroll
-        for (int q = 0; q < RM / 4; ++q) {
-          if (4 * q < R) {
-            const float4 pv = p4[q];
-            o[4 * q + 0] = fmaf(pv.x, v, o[4 * q + 0]);
-            o[4 * q + 1] = fmaf(pv.y, v, o[4 * q + 1]);
-            o[4 * q + 2] = fmaf(pv.z, v, o[4 * q + 2]);
-            o[4 * q + 3] = fmaf(pv.w, v, o[4 * q + 3]);
-          }
-        }
-      }
-    }
-    __syncthreads();
-    if (tid == 0 && tile + a.stages < n_tiles) issue(tile + a.stages);
   }
 
-  // ---- write this split's state (or the final output for a single split)
+  // ---- split totals: l summed over lanes and warps; O^T of block `warp`
   #pragma unroll
-  for (int r = 0; r < RM; ++r) {
-    if (r < R) {
+  for (int rt = 0; rt < NRT; ++rt)
+    #pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float l = l_run[rt][e];
+      l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
+      l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
+      l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
+      if (g == 0) red[(8 * rt + 2 * t + e) * kAttnConsumerWarps + warp] = l;
+    }
+  attn_consumer_sync();
+  if (tid < 8 * NRT) {
+    float l = 0.f;
+    for (int w = 0; w < kAttnConsumerWarps; ++w) l += red[tid * kAttnConsumerWarps + w];
+    row_sum[tid] = l;
+  }
+  attn_consumer_sync();
+  // O^T element (dim tile d, row tile rt, k): dim 32*warp + 2g + d (+16 for
+  // k >= 2), row 8*rt + 2t + (k & 1)
+  const size_t rows_total = size_t(a.M) * a.n_q;
+  #pragma unroll
+  for (int rt = 0; rt < NRT; ++rt)
+    #pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int r = 8 * rt + 2 * t + (k & 1);
+      if (r >= R) continue;
       const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
-      const int row = m * a.n_q + kh * a.g + j;  // (m, h) flattened
-      if (a.n_splits == 1) {
-        a.out[size_t(row) * kHeadDim + pd] = o[r] / l_run[r];
-      } else {
-        a.ws_o[(size_t(split) * a.M * a.n_q + row) * kHeadDim + pd] = o[r];
-        if (pd == 0) {
-          a.ws_ml[(size_t(split) * a.M * a.n_q + row) * 2 + 0] = m_run[r];
-          a.ws_ml[(size_t(split) * a.M * a.n_q + row) * 2 + 1] = l_run[r];
+      const size_t row = size_t(m) * a.n_q + kh * a.g + j;
+      #pragma unroll
+      for (int d = 0; d < 2; ++d) {
+        const int dim = 32 * warp + 2 * g + d + (k >= 2 ? 16 : 0);
+        if (a.n_splits == 1) {
+          a.out[row * kHeadDim + dim] = o[d][rt][k] / row_sum[r];
+        } else {
+          a.ws_o[(size_t(split) * rows_total + row) * kHeadDim + dim] = o[d][rt][k];
         }
       }
+      if (a.n_splits > 1 && warp == 0 && g == 0 && k < 2) {
+        a.ws_ml[(size_t(split) * rows_total + row) * 2 + 0] = m_run[rt][k];
+        a.ws_ml[(size_t(split) * rows_total + row) * 2 + 1] = row_sum[r];
+      }
     }
-  }
 }
 
-// Log-sum-exp merge of the per-split states; one CTA per (draft row, head).
+// Log-sum-exp merge of the per-split states (base 2); one CTA per (draft
+// row, head), one thread per output dimension; at most 256 splits.
 __global__ void __launch_bounds__(kHeadDim) q4kv_attn_merge_kernel(const AttnArgs a) {
   const int row = blockIdx.x;  // m * n_q + h
   const int d = threadIdx.x;
   const size_t rows = size_t(a.M) * a.n_q;
-  float mx = -INFINITY;
-  for (int c = 0; c < a.n_splits; ++c) mx = fmaxf(mx, a.ws_ml[(c * rows + row) * 2]);
-  float L = 0.f, acc = 0.f;
-  for (int c = 0; c < a.n_splits; ++c) {
-    const float mc = a.ws_ml[(c * rows + row) * 2];
-    const float w = (mc == -INFINITY) ? 0.f : __expf(mc - mx);
-    L = fmaf(a.ws_ml[(c * rows + row) * 2 + 1], w, L);
-    acc = fmaf(a.ws_o[(c * rows + row) * kHeadDim + d], w, acc);
+  __shared__ float wts[256];
+  __shared__ float inv_l;
+  // one thread per split gathers (max, sum); weights 2^(m_c - MX)
+  float mc = -INFINITY, lc = 0.f;
+  if (d < a.n_splits) {
+    mc = a.ws_ml[(d * rows + row) * 2];
+    lc = a.ws_ml[(d * rows + row) * 2 + 1];
   }
-  a.out[size_t(row) * kHeadDim + d] = acc / L;
+  float mx = mc;
+  for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+  __shared__ float wmax[8];
+  if ((d & 31) == 0) wmax[d >> 5] = mx;
+  __syncthreads();
+  mx = wmax[0];
+  for (int w = 1; w < 8; ++w) mx = fmaxf(mx, wmax[w]);
+  const float wc = (d < a.n_splits && mc != -INFINITY) ? ex2(mc - mx) : 0.f;
+  if (d < 256) wts[d] = wc;
+  float lw = lc * wc;
+  for (int off = 16; off >= 1; off >>= 1) lw += __shfl_xor_sync(0xFFFFFFFFu, lw, off);
+  __shared__ float wsum[8];
+  __syncthreads();
+  if ((d & 31) == 0) wsum[d >> 5] = lw;
+  __syncthreads();
+  if (d == 0) {
+    float L = 0.f;
+    for (int w = 0; w < 8; ++w) L += wsum[w];
+    inv_l = 1.f / L;
+  }
+  __syncthreads();
+  float acc = 0.f;
+  #pragma unroll 8
+  for (int c = 0; c < a.n_splits; ++c) acc = fmaf(a.ws_o[(c * rows + row) * kHeadDim + d], wts[c], acc);
+  a.out[size_t(row) * kHeadDim + d] = acc * inv_l;
 }
 
 }  // namespace q4d

@@ -99,16 +99,61 @@ ATTN_CASES = [(4096, 24, 4, 1), (4096, 24, 4, 5), (65536, 24, 4, 5), (262144, 24
               (1000, 8, 1, 5), (300, 64, 4, 5), (129, 4, 4, 2), (70000, 48, 1, 5)]
 
 
+TT_ATTN, Q_PITCH, PT_PITCH, ROW = 128, 576, 80, 144
+
+
+def _attn_smem(stages):
+    return stages * 2 * TT_ATTN * ROW + 32 * Q_PITCH + TT_ATTN * PT_PITCH + 32 * 8 * 4 + 32 * 4 \
+        + stages * 16
+
+
+def _chunks(addrs):
+    """16-byte bank groups hit by eight ldmatrix row addresses (one phase)."""
+    return {(a % 128) // 16 for a in addrs}
+
+
+def test_attn_shared_memory_banks():
+    # K ldmatrix: eight token rows at a 144-byte pitch, same column
+    for col in range(0, 128, 16):
+        assert len(_chunks([r * ROW + col for r in range(8)])) == 8
+    # P^T ldmatrix.trans: eight token rows at an 80-byte pitch
+    for col in range(0, 64, 16):
+        assert len(_chunks([r * PT_PITCH + col for r in range(8)])) == 8
+    # P^T stores: lane (g, t) writes 4 bytes at token g, rows 2t..2t+1
+    for rt in range(4):
+        banks = {((g * PT_PITCH + (8 * rt + 2 * t) * 2) // 4) % 32 for g in range(8) for t in range(4)}
+        assert len(banks) == 32
+    # Q fragment loads (16 bytes per lane): each group of eight lanes covers
+    # eight distinct 16-byte bank groups
+    for rt in range(4):
+        for blk in range(8):
+            for q in range(4):
+                lanes = range(8 * q, 8 * q + 8)
+                assert len(_chunks([(8 * rt + (ln >> 2)) * Q_PITCH + (blk * 4 + (ln & 3)) * 16
+                                    for ln in lanes])) == 8
+    # block scales in the score step: tokens g at a 144-byte pitch, distinct banks
+    assert len({((g * ROW + 128) // 4) % 32 for g in range(8)}) == 8
+
+
 @pytest.mark.parametrize("ctx,nq,nkv,M", ATTN_CASES)
 @pytest.mark.parametrize("stride_extra", [0, 37])
 def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
     sms = 148
     p = q4dec.plan_attn(ctx, nq, nkv, 256, M, sms)
-    TT, RM = p.tile_tokens, 32
+    TT = p.tile_tokens
     stride = ctx + stride_extra
     g = nq // nkv
-    assert TT == 64 and p.split_tokens % TT == 0 and p.threads == 256
-    assert p.rows_per_cta <= RM and p.row_groups * p.rows_per_cta >= g * M
+    assert TT == TT_ATTN and p.split_tokens % TT == 0 and p.threads == 288
+    assert 1 <= p.n_splits <= 256
+    assert p.rows_per_cta <= 32 and p.row_groups * p.rows_per_cta >= g * M
+    assert 2 <= p.stages <= 8 and p.smem_bytes == _attn_smem(p.stages) <= SMEM_OPTIN
+    # carve-up: ring, Q fragments, P^T (16-byte aligned for ldmatrix / v4),
+    # row maxima, row sums, barriers (8-byte aligned)
+    ring = p.stages * 2 * TT * ROW
+    q_off, pt_off = ring, ring + 32 * Q_PITCH
+    bar_off = pt_off + TT * PT_PITCH + 32 * 8 * 4 + 32 * 4
+    assert q_off % 16 == 0 and pt_off % 16 == 0 and bar_off % 8 == 0
+    assert (TT * ROW) % 16 == 0
     cache_bytes = nkv * stride * 144
     tokens = []
     for c in range(p.n_splits):
@@ -118,32 +163,51 @@ def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
         n_tiles = (te - tb + TT - 1) // TT
         for tile in range(n_tiles):
             t0 = tb + tile * TT
-            nbytes = min(TT, te - t0) * 144
-            assert 2 * nbytes <= TX_LIMIT
+            nbytes = min(TT, te - t0) * ROW
+            assert 2 * nbytes <= TX_LIMIT and nbytes % 16 == 0 and nbytes <= TT * ROW
             for kh in range(nkv):
-                lo = (kh * stride + t0) * 144
+                lo = (kh * stride + t0) * ROW
                 assert lo % 16 == 0 and lo + nbytes <= cache_bytes
     assert tokens == list(range(ctx))
     rows = []
     for z in range(p.row_groups):
         r0 = z * p.rows_per_cta
         R = min(p.rows_per_cta, g * M - r0)
-        assert 1 <= R <= RM
+        assert 1 <= R <= 32
         rows.extend(range(r0, r0 + R))
     assert rows == list(range(g * M))
-    # workspace indices of the split states and the output rows
-    nrows = M * nq
-    if p.n_splits > 1:
-        assert p.workspace_bytes == p.n_splits * nrows * 258 * 4
-        assert (p.n_splits - 1) * nrows * 256 + (nrows - 1) * 256 + 255 < p.n_splits * nrows * 256
-    else:
-        assert p.workspace_bytes == 0
+    nrt = -(-p.rows_per_cta // 8)
+    # shared-memory reads inside one tile: K ldmatrix rows / columns, block
+    # scales, V ldmatrix.trans rows, P^T ldmatrix.trans rows / columns
+    for warp in range(8):
+        for lane in range(32):
+            tok = 16 * warp + (lane & 15)
+            for b in range(0, 8, 2):
+                col = (lane >> 4) * 16 + b * 16
+                assert tok < TT and col + 16 <= 128
+                assert 128 + 2 * b + 4 <= ROW
+            for k0 in range(0, TT, 32):
+                assert k0 + lane < TT and warp * 16 + 16 <= 128
+                for h in range(2):
+                    kb = k0 + 16 * h
+                    assert kb + 2 * (lane & 3) + 8 + 1 < TT and 128 + 2 * warp + 2 <= ROW
+                    for rt in range(0, nrt, 2):
+                        pcol = rt * 16 + (lane >> 4) * 16 if rt + 1 < nrt else rt * 16
+                        assert kb + (lane & 15) < TT and pcol + 16 <= 64
+    # Q reads (global, 8-byte vectors) stay inside [M][n_q][256]
+    q_elems = M * nq * 256
     for kh in range(nkv):
         for rr in range(g * M):
             m, j = divmod(rr, g)
             row = m * nq + kh * g + j
-            assert 0 <= row < nrows
-    ring = p.stages * 2 * TT * 144
-    assert p.smem_bytes == RM * 256 * 4 + ring + TT * RM * 4 + 3 * RM * 4 + p.stages * 8
-    assert (RM * 256 * 4 + ring + TT * RM * 4 + 3 * RM * 4) % 8 == 0
-    assert 2 * p.smem_bytes <= 228 * 1024  # two CTAs per SM
+            assert 0 <= row < M * nq
+            for b in range(8):
+                for t in range(4):
+                    e = row * 256 + b * 32 + 4 * t
+                    assert e % 4 == 0 and e + 16 + 4 <= q_elems
+    # workspace: split outputs then (max, sum) pairs
+    nrows = M * nq
+    if p.n_splits > 1:
+        assert p.workspace_bytes == p.n_splits * nrows * 258 * 4
+    else:
+        assert p.workspace_bytes == 0
