@@ -254,11 +254,17 @@ q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, in
   return Q4D_OK;
 }
 
+// NRT = 1: the warp-local kernel (at most 8 query rows per CTA); 2..4: the
+// generic kernel.
 template <int NRT>
 q4d_status launch_attn_t(const q4d::AttnArgs& a, const q4d_attn_plan& p, int n_kv, int dev,
                          const DeviceState& s, cudaStream_t stream) {
   static std::atomic<bool> smem_set[kMaxDevices];
-  auto kernel = q4d::q4kv_attn_split_kernel<NRT>;
+  void (*kernel)(q4d::AttnArgs);
+  if constexpr (NRT == 1)
+    kernel = q4d::q4kv_attn_split_rows8_kernel;
+  else
+    kernel = q4d::q4kv_attn_split_kernel<NRT>;
   q4d_status st = allow_smem(kernel, dev, s, smem_set);
   if (st != Q4D_OK) return st;
   dim3 grid(p.n_splits, n_kv, p.row_groups);
@@ -416,8 +422,10 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   n_splits = std::min(n_splits, 256);
   const int split_tokens = int(round_up(ceil_div(ctx_len, n_splits), TT));
   n_splits = ceil_div(ctx_len, split_tokens);
-  // As many ring stages as fit next to the fixed buffers, up to 8.
-  const size_t fixed = q4d::attn_smem_bytes(0);
+  // As many ring stages as fit next to the variant's fixed buffers, up to 8
+  // (at least 2: the warp-local variant parks 64 KB in the ring at the end).
+  const bool rows8 = rows_per_cta <= 8;
+  const size_t fixed = rows8 ? q4d::attn_rows8_smem_bytes(0) : q4d::attn_smem_bytes(0);
   int stages = int((kAttnSmemBudget - fixed) / (q4d::kAttnStageBytes + 16));
   stages = std::max(2, std::min(8, stages));
   plan->n_splits = n_splits;
@@ -427,7 +435,7 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   plan->rows_per_cta = rows_per_cta;
   plan->stages = stages;
   plan->threads = q4d::kAttnThreads;
-  plan->smem_bytes = q4d::attn_smem_bytes(stages);
+  plan->smem_bytes = rows8 ? q4d::attn_rows8_smem_bytes(stages) : q4d::attn_smem_bytes(stages);
   plan->workspace_bytes =
       n_splits > 1 ? size_t(n_splits) * M * n_q_heads * (q4d::kHeadDim + 2) * 4 : 0;
   return Q4D_OK;

@@ -87,6 +87,11 @@ __device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint3
                : "=r"(r0), "=r"(r1)
                : "r"(addr));
 }
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
 __device__ __forceinline__ uint32_t f16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t r;
   asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
@@ -133,13 +138,299 @@ __device__ __forceinline__ uint32_t q8_pair(uint32_t r) {
                    0xD480D480u /* -72 */);
 }
 
-// NRT: row tiles of 8 query rows (1..4).  A single row tile keeps its Q
-// fragments in registers for the whole split; more read them from shared
-// memory at every use.
+// Shared memory of the warp-local variant: the ring (which also holds the
+// final cross-warp combine, 64 KB) plus per-warp row statistics and barriers.
+__host__ __device__ constexpr size_t attn_rows8_smem_bytes(int stages) {
+  return size_t(stages) * kAttnStageBytes + size_t(kAttnConsumerWarps) * 8 * 2 * 4 + 8 * 2 * 4 +
+         size_t(stages) * 16;
+}
+
+// Warp-local variant for at most 8 query rows per CTA (one row tile: plain
+// decode, M = 1).  Each consumer warp owns tokens 16w .. 16w + 15 of every
+// tile and carries its own online softmax and its own O^T for all 256
+// dimensions (64 fp32 registers), so a tile needs no CTA-wide barrier: the
+// score fragments (token, row) are rounded to fp16 and transposed in
+// registers with movmatrix into the P^T operand of P.V.  The eight warps'
+// states are combined once, at the end of the split.
+__global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_rows8_kernel(const AttnArgs a) {
+  constexpr int TT = kAttnTileTokens;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int S = a.stages;
+  uint8_t* ring = smem;
+  float* wml = reinterpret_cast<float*>(ring + size_t(S) * kAttnStageBytes);  // [warp][row][m, l]
+  float* rml = wml + kAttnConsumerWarps * 8 * 2;                              // [row][M, L]
+  uint64_t* full = reinterpret_cast<uint64_t*>(rml + 8 * 2);
+  uint64_t* empty = full + S;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = blockIdx.x, kh = blockIdx.y, rgrp = blockIdx.z;
+  const int row0 = rgrp * a.rows_per_cta;
+  const int R = min(a.rows_per_cta, a.g * a.M - row0);
+  const int t_begin = split * a.split_tokens;
+  const int t_end = min(a.ctx_len, t_begin + a.split_tokens);
+  const int n_tiles = (t_end - t_begin + TT - 1) / TT;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_addr(&full[s]), 1);
+      mbar_init(smem_addr(&empty[s]), kAttnConsumerWarps);
+    }
+    mbar_init_fence();
+  }
+  __syncthreads();
+
+  if (warp == kAttnConsumerWarps) {
+    if (lane == 0) {
+      const uint8_t* Kh = a.K + size_t(kh) * a.kv_stride * kRowBytes;
+      const uint8_t* Vh = a.V + size_t(kh) * a.kv_stride * kRowBytes;
+      const uint64_t pol = l2_evict_first_policy();
+      int slot = 0;
+      uint32_t phase = 0;
+      for (int tile = 0; tile < n_tiles; ++tile) {
+        if (tile >= S) mbar_wait(smem_addr(&empty[slot]), phase ^ 1u, a.err);
+        const int t0 = t_begin + tile * TT;
+        const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * kRowBytes;
+        const uint32_t bar = smem_addr(&full[slot]);
+        const uint32_t dk = smem_addr(ring + size_t(slot) * kAttnStageBytes);
+        mbar_arrive_expect_tx(bar, 2 * bytes);
+        bulk_g2s(dk, Kh + size_t(t0) * kRowBytes, bytes, bar, pol);
+        bulk_g2s(dk + TT * kRowBytes, Vh + size_t(t0) * kRowBytes, bytes, bar, pol);
+        if (++slot == S) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    return;
+  }
+
+  const int g = lane >> 2, t = lane & 3;
+  // Q fragments of row g (zero for padding rows), in the nibble order of a
+  // K word: see the generic kernel below.
+  uint4 qf[8];
+  {
+    const bool live = g < R;
+    const int rr = row0 + g, m = rr / a.g, j = rr - m * a.g;
+    const uint16_t* q = a.Q + (size_t(live ? m : 0) * a.n_q + kh * a.g + (live ? j : 0)) * kHeadDim + 4 * t;
+    #pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (live) {
+        const uint2 lo = *reinterpret_cast<const uint2*>(q + b * 32);
+        const uint2 hi = *reinterpret_cast<const uint2*>(q + b * 32 + 16);
+        v.x = prmt(lo.x, lo.y, 0x5410);
+        v.y = prmt(hi.x, hi.y, 0x5410);
+        v.z = prmt(lo.x, lo.y, 0x7632);
+        v.w = prmt(hi.x, hi.y, 0x7632);
+      }
+      qf[b] = v;
+    }
+  }
+  int row_pos[2];
+  float m_run[2], l_run[2];
+  #pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int r = 2 * t + e;
+    row_pos[e] = r < R ? a.ctx_len - a.M + (row0 + r) / a.g : -1;
+    m_run[e] = -INFINITY;
+    l_run[e] = 0.f;
+  }
+  float o[8][2][4];  // O^T: [block][dim tile][fragment]
+  #pragma unroll
+  for (int b = 0; b < 8; ++b)
+    #pragma unroll
+    for (int d = 0; d < 2; ++d) o[b][d][0] = o[b][d][1] = o[b][d][2] = o[b][d][3] = 0.f;
+
+  const uint32_t bmask = 0x000F000Fu, bmagic = 0x43004300u, b136 = 0x43084308u;
+  const int tok0 = 16 * warp;
+  // ldmatrix rows of this warp's 16 tokens: lanes 0-15 tokens tok0 + lane at
+  // block b, lanes 16-31 tokens tok0 + lane - 16 at block b + 1
+  const uint32_t lrow = uint32_t(tok0 + (lane & 15)) * kRowBytes + uint32_t(lane >> 4) * 16u;
+  int slot = 0;
+  uint32_t phase = 0;
+
+  #pragma unroll 1
+  for (int tile = 0; tile < n_tiles; ++tile) {
+    const int t0 = t_begin + tile * TT;
+    const int n_tok = min(TT, t_end - t0);
+    mbar_wait(smem_addr(&full[slot]), phase, a.err);
+    const uint8_t* Kt = ring + size_t(slot) * kAttnStageBytes;
+    const uint8_t* Vt = Kt + TT * kRowBytes;
+    if (tok0 < n_tok) {
+      const uint32_t Kt_addr = smem_addr(Kt), Vt_addr = smem_addr(Vt);
+      // ---- scores S^T (tokens tok0 + g, tok0 + g + 8; rows 2t, 2t + 1)
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint8_t* da_p = Kt + (tok0 + g) * kRowBytes + 128;
+      const uint8_t* db_p = da_p + 8 * kRowBytes;
+      #pragma unroll
+      for (int b = 0; b < 8; b += 2) {
+        uint32_t w0a, w0b, w1a, w1b;
+        ldsm_x4(Kt_addr + lrow + uint32_t(b) * 16u, w0a, w0b, w1a, w1b);
+        const float2 dA = __half22float2(*reinterpret_cast<const __half2*>(da_p + 2 * b));
+        const float2 dB = __half22float2(*reinterpret_cast<const __half2*>(db_p + 2 * b));
+        #pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          uint32_t qa[4], qb[4];
+          dequant_pairs(bb ? w1a : w0a, bmask, bmagic, b136, qa);
+          dequant_pairs(bb ? w1b : w0b, bmask, bmagic, b136, qb);
+          const uint4 qv = qf[b + bb];
+          float c[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_bf16(c, qa[0], qb[0], qa[1], qb[1], qv.x, qv.y);
+          mma_bf16(c, qa[2], qb[2], qa[3], qb[3], qv.z, qv.w);
+          const float da = bb ? dA.y : dA.x, db = bb ? dB.y : dB.x;
+          s[0] = fmaf(da, c[0], s[0]);
+          s[1] = fmaf(da, c[1], s[1]);
+          s[2] = fmaf(db, c[2], s[2]);
+          s[3] = fmaf(db, c[3], s[3]);
+        }
+      }
+      // ---- warp-local online softmax (base 2)
+      const int ta = tok0 + g, tb = ta + 8;
+      float alpha[2];
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int pos = row_pos[e];
+        s[e] = (ta < n_tok && t0 + ta <= pos) ? s[e] * a.scale_log2 : -INFINITY;
+        s[2 + e] = (tb < n_tok && t0 + tb <= pos) ? s[2 + e] * a.scale_log2 : -INFINITY;
+        float mx = fmaxf(s[e], s[2 + e]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
+        const float m_new = fmaxf(m_run[e], mx);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        alpha[e] = ex2(m_run[e] - m_use);
+        m_run[e] = m_new;
+        s[e] = ex2(s[e] - m_use);
+        s[2 + e] = ex2(s[2 + e] - m_use);
+      }
+      const uint32_t pa = pack_f16x2(s[0], s[1]);  // token ta, rows 2t, 2t + 1
+      const uint32_t pb = pack_f16x2(s[2], s[3]);  // token tb
+      {
+        const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&pa));
+        const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&pb));
+        l_run[0] = l_run[0] * alpha[0] + fa.x + fb.x;
+        l_run[1] = l_run[1] * alpha[1] + fa.y + fb.y;
+      }
+      // P^T B fragments: (tokens 2t, 2t + 1; row g) and (tokens 2t + 8, 2t + 9; row g)
+      const uint32_t B0 = movmatrix_trans(pa), B1 = movmatrix_trans(pb);
+      if (__any_sync(0xFFFFFFFFu, alpha[0] != 1.f || alpha[1] != 1.f)) {
+        #pragma unroll
+        for (int b = 0; b < 8; ++b)
+          #pragma unroll
+          for (int d = 0; d < 2; ++d) {
+            o[b][d][0] *= alpha[0];
+            o[b][d][1] *= alpha[1];
+            o[b][d][2] *= alpha[0];
+            o[b][d][3] *= alpha[1];
+          }
+      }
+      // ---- V block scales of tokens 2t, 2t + 1, 2t + 8, 2t + 9 (all 8
+      // blocks, as fp16 pairs (d_2i, d_2i+1)); zero past the tile end
+      uint4 dw[4];
+      #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tk = tok0 + 2 * t + (i & 1) + (i >> 1) * 8;
+        dw[i] = *reinterpret_cast<const uint4*>(Vt + tk * kRowBytes + 128);
+        if (tok0 + 16 > n_tok && tk >= n_tok) dw[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      // ---- O^T[dims][rows] += (q - 8)^T (P^T d) over this warp's 16 tokens
+      #pragma unroll
+      for (int b = 0; b < 8; b += 2) {
+        uint32_t v0, v1, v2, v3;  // blocks b (v0, v1) and b + 1 (v2, v3)
+        ldsm_x4_trans(Vt_addr + lrow + uint32_t(b) * 16u, v0, v1, v2, v3);
+        #pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const uint32_t ra = bb ? v2 : v0, rb = bb ? v3 : v1;
+          const int wd = (b + bb) >> 1;
+          const uint32_t sel = ((b + bb) & 1) ? 0x7632u : 0x5410u;
+          const uint32_t x0 = wd == 0 ? dw[0].x : wd == 1 ? dw[0].y : wd == 2 ? dw[0].z : dw[0].w;
+          const uint32_t x1 = wd == 0 ? dw[1].x : wd == 1 ? dw[1].y : wd == 2 ? dw[1].z : dw[1].w;
+          const uint32_t x2 = wd == 0 ? dw[2].x : wd == 1 ? dw[2].y : wd == 2 ? dw[2].z : dw[2].w;
+          const uint32_t x3 = wd == 0 ? dw[3].x : wd == 1 ? dw[3].y : wd == 2 ? dw[3].z : dw[3].w;
+          const uint32_t p0 = f16x2_mul(B0, prmt(x0, x1, sel));
+          const uint32_t p1 = f16x2_mul(B1, prmt(x2, x3, sel));
+          mma_f16(o[b + bb][0], q8_pair<true>(ra), q8_pair<false>(ra), q8_pair<true>(rb),
+                  q8_pair<false>(rb), p0, p1);
+          mma_f16(o[b + bb][1], q8_pair<true>(ra >> 8), q8_pair<false>(ra >> 8),
+                  q8_pair<true>(rb >> 8), q8_pair<false>(rb >> 8), p0, p1);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&empty[slot]));
+    if (++slot == S) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+
+  // ---- combine the eight warps: per-row maxima and sums, then O^T parked in
+  // the (now idle) ring as [warp][row][dim] and summed in warp order
+  #pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    float l = l_run[e];
+    l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
+    l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
+    l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
+    if (g == 0) {
+      wml[(warp * 8 + 2 * t + e) * 2 + 0] = m_run[e];
+      wml[(warp * 8 + 2 * t + e) * 2 + 1] = l;
+    }
+  }
+  attn_consumer_sync();
+  float cw[2];
+  #pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int r = 2 * t + e;
+    float M = -INFINITY;
+    for (int w = 0; w < kAttnConsumerWarps; ++w) M = fmaxf(M, wml[(w * 8 + r) * 2]);
+    const float m_use = M == -INFINITY ? 0.f : M;
+    cw[e] = ex2(m_run[e] - m_use);
+    if (warp == 0 && g == 0) {
+      float L = 0.f;
+      for (int w = 0; w < kAttnConsumerWarps; ++w)
+        L += wml[(w * 8 + r) * 2 + 1] * ex2(wml[(w * 8 + r) * 2] - m_use);
+      rml[r * 2 + 0] = M;
+      rml[r * 2 + 1] = L;
+    }
+  }
+  float* park = reinterpret_cast<float*>(ring) + warp * 8 * kHeadDim;
+  #pragma unroll
+  for (int b = 0; b < 8; ++b)
+    #pragma unroll
+    for (int d = 0; d < 2; ++d)
+      #pragma unroll
+      for (int k = 0; k < 4; ++k)
+        park[(2 * t + (k & 1)) * kHeadDim + 32 * b + 2 * g + d + (k >= 2 ? 16 : 0)] =
+            o[b][d][k] * cw[k & 1];
+  attn_consumer_sync();
+  const float* parked = reinterpret_cast<const float*>(ring);
+  const size_t rows_total = size_t(a.M) * a.n_q;
+  for (int r = 0; r < R; ++r) {
+    float acc = 0.f;
+    #pragma unroll
+    for (int w = 0; w < kAttnConsumerWarps; ++w) acc += parked[(w * 8 + r) * kHeadDim + tid];
+    const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
+    const size_t row = size_t(m) * a.n_q + kh * a.g + j;
+    if (a.n_splits == 1) {
+      a.out[row * kHeadDim + tid] = acc / rml[r * 2 + 1];
+    } else {
+      a.ws_o[(size_t(split) * rows_total + row) * kHeadDim + tid] = acc;
+      if (tid == 0) {
+        a.ws_ml[(size_t(split) * rows_total + row) * 2 + 0] = rml[r * 2 + 0];
+        a.ws_ml[(size_t(split) * rows_total + row) * 2 + 1] = rml[r * 2 + 1];
+      }
+    }
+  }
+}
+
+// Generic variant, NRT row tiles of 8 query rows (2..4, up to 32 rows): the
+// warps split the tile's tokens for the scores and the head dimensions for
+// P.V, exchanging the running maxima and P^T through shared memory with two
+// CTA-wide barriers per tile.  Q fragments are read from shared memory.
 template <int NRT>
 __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const AttnArgs a) {
   constexpr int TT = kAttnTileTokens;
-  constexpr bool kQReg = NRT == 1;
   extern __shared__ __align__(128) uint8_t smem[];
   const int S = a.stages;
   uint8_t* ring = smem;
@@ -218,14 +509,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const 
   }
   attn_consumer_sync();
   const uint32_t Qp_addr = smem_addr(Qp), Pt_addr = smem_addr(Pt);
-  uint4 qreg[kQReg ? NRT : 1][kQReg ? 8 : 1];
-  if (kQReg) {
-    #pragma unroll
-    for (int rt = 0; rt < NRT; ++rt)
-      #pragma unroll
-      for (int b = 0; b < 8; ++b)
-        qreg[rt][b] = *reinterpret_cast<const uint4*>(Qp + (8 * rt + g) * kQPitch + (b * 4 + t) * 16);
-  }
 
   // rows this lane holds in every row tile: 8*rt + 2t + e, e = 0, 1
   int row_pos[NRT][2];  // position of the row's draft token; -1 for padding rows
@@ -287,13 +570,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const 
           #pragma unroll
           for (int rt = 0; rt < NRT; ++rt) {
             uint4 qf;
-            if (kQReg) {
-              qf = qreg[kQReg ? rt : 0][kQReg ? b + bb : 0];
-            } else {
-              asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                           : "=r"(qf.x), "=r"(qf.y), "=r"(qf.z), "=r"(qf.w)
-                           : "r"(Qp_addr + uint32_t((8 * rt + g) * kQPitch + ((b + bb) * 4 + t) * 16)));
-            }
+            asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(qf.x), "=r"(qf.y), "=r"(qf.z), "=r"(qf.w)
+                         : "r"(Qp_addr + uint32_t((8 * rt + g) * kQPitch + ((b + bb) * 4 + t) * 16)));
             float c[4] = {0.f, 0.f, 0.f, 0.f};
             mma_bf16(c, qa[0], qb[0], qa[1], qb[1], qf.x, qf.y);
             mma_bf16(c, qa[2], qb[2], qa[3], qb[3], qf.z, qf.w);
@@ -476,45 +755,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const 
     }
 }
 
-// Log-sum-exp merge of the per-split states (base 2); one CTA per (draft
-// row, head), one thread per output dimension; at most 256 splits.
-__global__ void __launch_bounds__(kHeadDim) q4kv_attn_merge_kernel(const AttnArgs a) {
+// Log-sum-exp merge of the per-split states (base 2); one CTA of eight warps
+// per (draft row, head).  Every warp finds the global maximum and the total
+// weight itself; warp w then adds splits w, w + 8, ... for all 256
+// dimensions (two float4 per lane), and the eight partial vectors are summed
+// in warp order.
+__global__ void __launch_bounds__(256) q4kv_attn_merge_kernel(const AttnArgs a) {
   const int row = blockIdx.x;  // m * n_q + h
-  const int d = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t rows = size_t(a.M) * a.n_q;
-  __shared__ float wts[256];
-  __shared__ float inv_l;
-  // one thread per split gathers (max, sum); weights 2^(m_c - MX)
-  float mc = -INFINITY, lc = 0.f;
-  if (d < a.n_splits) {
-    mc = a.ws_ml[(d * rows + row) * 2];
-    lc = a.ws_ml[(d * rows + row) * 2 + 1];
-  }
-  float mx = mc;
+  __shared__ float part[8 * kHeadDim];
+  const int n = a.n_splits;
+  float mx = -INFINITY;
+  for (int c = lane; c < n; c += 32) mx = fmaxf(mx, a.ws_ml[(c * rows + row) * 2]);
+  #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-  __shared__ float wmax[8];
-  if ((d & 31) == 0) wmax[d >> 5] = mx;
-  __syncthreads();
-  mx = wmax[0];
-  for (int w = 1; w < 8; ++w) mx = fmaxf(mx, wmax[w]);
-  const float wc = (d < a.n_splits && mc != -INFINITY) ? ex2(mc - mx) : 0.f;
-  if (d < 256) wts[d] = wc;
-  float lw = lc * wc;
-  for (int off = 16; off >= 1; off >>= 1) lw += __shfl_xor_sync(0xFFFFFFFFu, lw, off);
-  __shared__ float wsum[8];
-  __syncthreads();
-  if ((d & 31) == 0) wsum[d >> 5] = lw;
-  __syncthreads();
-  if (d == 0) {
-    float L = 0.f;
-    for (int w = 0; w < 8; ++w) L += wsum[w];
-    inv_l = 1.f / L;
+  float L = 0.f;
+  for (int c = lane; c < n; c += 32) {
+    const float mc = a.ws_ml[(c * rows + row) * 2];
+    if (mc != -INFINITY) L += a.ws_ml[(c * rows + row) * 2 + 1] * ex2(mc - mx);
   }
+  #pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, off);
+  float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+  #pragma unroll 4
+  for (int c = warp; c < n; c += 8) {
+    const float mc = a.ws_ml[(c * rows + row) * 2];
+    const float wc = mc == -INFINITY ? 0.f : ex2(mc - mx);
+    const float4* src = reinterpret_cast<const float4*>(a.ws_o + (c * rows + row) * kHeadDim);
+    const float4 v0 = src[lane], v1 = src[32 + lane];
+    acc0.x = fmaf(wc, v0.x, acc0.x);
+    acc0.y = fmaf(wc, v0.y, acc0.y);
+    acc0.z = fmaf(wc, v0.z, acc0.z);
+    acc0.w = fmaf(wc, v0.w, acc0.w);
+    acc1.x = fmaf(wc, v1.x, acc1.x);
+    acc1.y = fmaf(wc, v1.y, acc1.y);
+    acc1.z = fmaf(wc, v1.z, acc1.z);
+    acc1.w = fmaf(wc, v1.w, acc1.w);
+  }
+  reinterpret_cast<float4*>(part + warp * kHeadDim)[lane] = acc0;
+  reinterpret_cast<float4*>(part + warp * kHeadDim)[32 + lane] = acc1;
   __syncthreads();
-  float acc = 0.f;
-  #pragma unroll 8
-  for (int c = 0; c < a.n_splits; ++c) acc = fmaf(a.ws_o[(c * rows + row) * kHeadDim + d], wts[c], acc);
-  a.out[size_t(row) * kHeadDim + d] = acc * inv_l;
+  float sum = 0.f;
+  #pragma unroll
+  for (int w = 0; w < 8; ++w) sum += part[w * kHeadDim + tid];
+  a.out[size_t(row) * kHeadDim + tid] = sum / L;
 }
 
 }  // namespace q4d

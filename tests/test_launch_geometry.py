@@ -102,9 +102,11 @@ ATTN_CASES = [(4096, 24, 4, 1), (4096, 24, 4, 5), (65536, 24, 4, 5), (262144, 24
 TT_ATTN, Q_PITCH, PT_PITCH, ROW = 128, 576, 80, 144
 
 
-def _attn_smem(stages):
-    return stages * 2 * TT_ATTN * ROW + 32 * Q_PITCH + TT_ATTN * PT_PITCH + 32 * 8 * 4 + 32 * 4 \
-        + stages * 16
+def _attn_smem(stages, rows_per_cta):
+    ring = stages * 2 * TT_ATTN * ROW
+    if rows_per_cta <= 8:      # warp-local variant: ring + per-warp / per-row stats
+        return ring + 8 * 8 * 2 * 4 + 8 * 2 * 4 + stages * 16
+    return ring + 32 * Q_PITCH + TT_ATTN * PT_PITCH + 32 * 8 * 4 + 32 * 4 + stages * 16
 
 
 def _chunks(addrs):
@@ -146,13 +148,19 @@ def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
     assert TT == TT_ATTN and p.split_tokens % TT == 0 and p.threads == 288
     assert 1 <= p.n_splits <= 256
     assert p.rows_per_cta <= 32 and p.row_groups * p.rows_per_cta >= g * M
-    assert 2 <= p.stages <= 8 and p.smem_bytes == _attn_smem(p.stages) <= SMEM_OPTIN
-    # carve-up: ring, Q fragments, P^T (16-byte aligned for ldmatrix / v4),
-    # row maxima, row sums, barriers (8-byte aligned)
+    assert 2 <= p.stages <= 8
+    assert p.smem_bytes == _attn_smem(p.stages, p.rows_per_cta) <= SMEM_OPTIN
     ring = p.stages * 2 * TT * ROW
-    q_off, pt_off = ring, ring + 32 * Q_PITCH
-    bar_off = pt_off + TT * PT_PITCH + 32 * 8 * 4 + 32 * 4
-    assert q_off % 16 == 0 and pt_off % 16 == 0 and bar_off % 8 == 0
+    if p.rows_per_cta <= 8:
+        # warp-local: the final combine parks [8 warps][8 rows][256] fp32 in the ring
+        assert ring >= 8 * 8 * 256 * 4
+        assert (ring + 8 * 8 * 2 * 4 + 8 * 2 * 4) % 8 == 0
+    else:
+        # carve-up: ring, Q fragments, P^T (16-byte aligned for ldmatrix / v4),
+        # row maxima, row sums, barriers (8-byte aligned)
+        q_off, pt_off = ring, ring + 32 * Q_PITCH
+        bar_off = pt_off + TT * PT_PITCH + 32 * 8 * 4 + 32 * 4
+        assert q_off % 16 == 0 and pt_off % 16 == 0 and bar_off % 8 == 0
     assert (TT * ROW) % 16 == 0
     cache_bytes = nkv * stride * 144
     tokens = []
@@ -177,8 +185,18 @@ def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
         rows.extend(range(r0, r0 + R))
     assert rows == list(range(g * M))
     nrt = -(-p.rows_per_cta // 8)
-    # shared-memory reads inside one tile: K ldmatrix rows / columns, block
-    # scales, V ldmatrix.trans rows, P^T ldmatrix.trans rows / columns
+    for warp in range(8):
+        for lane in range(32):
+            # warp-local variant: ldmatrix rows (K and V) and the 16-byte
+            # scale vectors of tokens 2t, 2t + 1, 2t + 8, 2t + 9
+            tok = 16 * warp + (lane & 15)
+            for b in range(0, 8, 2):
+                assert tok < TT and (lane >> 4) * 16 + b * 16 + 16 <= 128
+            for i in range(4):
+                tk = 16 * warp + 2 * (lane & 3) + (i & 1) + (i >> 1) * 8
+                assert tk < TT and (tk * ROW + 128) % 16 == 0
+    # generic variant: K ldmatrix rows / columns, block scales, V
+    # ldmatrix.trans rows, P^T ldmatrix.trans rows / columns
     for warp in range(8):
         for lane in range(32):
             tok = 16 * warp + (lane & 15)
