@@ -86,45 +86,75 @@ def recorded_traffic(kernel):
 
 # ------------------------------------------------------------------ clocks --
 class ClockSampler:
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons sampled every few milliseconds
+    from a background thread through NVML (read-only queries) while the timed
+    region runs; nvidia-smi polling is the fallback when NVML is missing."""
 
-    def __init__(self, gpu_uuid):
-        self.proc = None
+    REASONS = [("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown")]
+
+    def __init__(self, torch_dev_index, period_s=0.002):
+        import threading
+
+        self.samples = []
+        self.err = None
+        self._stop = threading.Event()
+        self._nvml = None
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={gpu_uuid}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except Exception:
-            self.proc = None
+            import pynvml
+
+            pynvml.nvmlInit()
+            visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = torch_dev_index
+            if visible:
+                ids = [v.strip() for v in visible.split(",") if v.strip()]
+                if torch_dev_index < len(ids) and ids[torch_dev_index].isdigit():
+                    idx = int(ids[torch_dev_index])
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self._nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.err = f"nvml: {e}"
+            self.max_mhz = None
+        self._period = period_s
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nvml
+        masks = [(name, getattr(nv, attr, 0)) for name, attr in self.REASONS]
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                pw = nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+                self.samples.append((mhz, pw, [n for n, m in masks if m and rs & m]))
+            except Exception as e:  # noqa: BLE001
+                self.err = f"nvml sample: {e}"
+                break
+            self._stop.wait(self._period)
+
+    def start(self):
+        if self._nvml is not None:
+            self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=10)
-        except Exception:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 7]
-        if not rows:
-            return None
-        def num(v):
-            try:
-                return float(v)
-            except ValueError:
-                return None
-        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
-        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if "Active" in v
-                          and "Not" not in v})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "error": self.err}
+        self._stop.set()
+        self._thread.join(timeout=5)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "error": self.err or "no sample inside the timed region"}
+        mhz = [m for m, _, _ in self.samples]
+        reasons = sorted({r for _, _, rs in self.samples for r in rs})
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "sm_min_mhz": min(mhz), "power_w_median": statistics.median(
+                    [p for _, p, _ in self.samples]),
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
 
 # --------------------------------------------------------------- CPU arms --
@@ -204,6 +234,7 @@ def workload_config(args):
             "M": args.M, "ctx_len": CTX, "layers": LAYERS, "attn_layers": ATTN_LAYERS,
             "bytes_per_step": step_bytes(args.M),
             "l2": "inputs larger than L2 (17.2 GB of distinct weights/caches per step)",
+            "gemv_launch": "q4_gemv_ex2 with Q4D_GEMV_WEIGHT_PREFETCH",
             "parallelism": f"replicas x{args.gpus}"}
 
 
@@ -290,10 +321,12 @@ def main():
     launches = {"n": 0}
 
     def gemv(W, x, y, N, K):
-        st = L.q4_gemv_ex(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, sptr,
-                          ws.data_ptr(), ws.numel())
+        # weights are immutable: each call may stream its first stages while
+        # the kernel before it finishes (programmatic dependent launch)
+        st = L.q4_gemv_ex2(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, sptr,
+                           ws.data_ptr(), ws.numel(), q4dec.GEMV_WEIGHT_PREFETCH)
         if st:
-            raise RuntimeError(f"q4_gemv_ex failed: {st}")
+            raise RuntimeError(f"q4_gemv_ex2 failed: {st}")
         launches["n"] += 1 + (1 if L.q4d_gemv_workspace_bytes(M, N, K) else 0)
 
     def attn(l):
@@ -319,8 +352,7 @@ def main():
         if world > 1:
             dist.barrier()
 
-    uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    clocks = ClockSampler(local)
 
     for _ in range(args.warmup):
         gemv_stream()
@@ -336,6 +368,7 @@ def main():
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    clocks.start()
     t_start.record(stream)
     for k in range(K_):
         ev[k][0].record(stream)

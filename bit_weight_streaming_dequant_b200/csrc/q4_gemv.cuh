@@ -213,6 +213,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   uint64_t* empty = full + S;
 
   if (tid == 0) {
+    // the next kernel on the stream may start its own weight prefetch
+    griddep_launch_dependents();
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_addr(&full[s]), 1);
       mbar_init(smem_addr(&empty[s]), kConsumerWarps);
@@ -225,10 +227,37 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     // ---------------- producer: one lane issues every copy ----------------
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();
-      int slot = 0, pass = 0, chunk = 0;
-      uint32_t phase = 0;
-      for (int st = 0; st < n_stages; ++st) {
-        if (st >= S) mbar_wait(smem_addr(&empty[slot]), phase ^ 1u, a.err);
+      // First ring fill: the weights (no earlier kernel writes them) go out
+      // before waiting on the previous kernel; the activations, which it may
+      // produce, only after.  Under a plain launch the wait returns at once.
+      const int pre = min(S, n_stages);
+      for (int st = 0; st < pre; ++st) {
+        const int ps = st / n_chunks, ch = st - ps * n_chunks;
+        const int r0 = row_begin + ps * R;
+        const int nr = min(R, row_end - r0);
+        const int sb = sb_split0 + ch * KC;
+        const uint32_t bar = smem_addr(&full[st]);
+        const uint32_t dst = smem_addr(ring + size_t(st) * stage_bytes);
+        mbar_arrive_expect_tx(bar, uint32_t(KC) * (uint32_t(nr) * kSbBytes + uint32_t(M) * 512u));
+        #pragma unroll
+        for (int j = 0; j < KC; ++j)
+          bulk_g2s(dst + uint32_t(j) * wbox, a.W + (size_t(sb + j) * a.N + r0) * kSbBytes,
+                   uint32_t(nr) * kSbBytes, bar, pol);
+      }
+      griddep_wait();
+      for (int st = 0; st < pre; ++st) {
+        const int sb = sb_split0 + (st % n_chunks) * KC;
+        const uint32_t bar = smem_addr(&full[st]);
+        const uint32_t dst = smem_addr(ring + size_t(st) * stage_bytes);
+        #pragma unroll
+        for (int j = 0; j < KC; ++j)
+          tma_load_2d_nohint(dst + xoff + uint32_t(j) * uint32_t(M) * 512u, &a.xmap,
+                             (sb + j) * 256, 0, bar);
+      }
+      int slot = 0, pass = pre / n_chunks, chunk = pre % n_chunks;
+      uint32_t phase = pre == S ? 1u : 0u;
+      for (int st = pre; st < n_stages; ++st) {
+        mbar_wait(smem_addr(&empty[slot]), phase ^ 1u, a.err);
         const int r0 = row_begin + pass * R;
         const int nr = min(R, row_end - r0);
         const uint32_t bar = smem_addr(&full[slot]);
@@ -321,6 +350,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 // y[i] = sum over K ranges of the partials, in range order.
 __global__ void q4_gemv_splitk_reduce(const float* __restrict__ ws, float* __restrict__ y,
                                       long long mn, int k_splits) {
+  if (threadIdx.x == 0) griddep_launch_dependents();
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < mn;
        i += (long long)gridDim.x * blockDim.x) {
     float s = 0.f;

@@ -181,19 +181,32 @@ q4d_status check_attn_shape(int ctx_len, int n_q, int n_kv, int head_dim, int M,
 
 template <int M, int KC>
 q4d_status launch_gemv_t(const q4d::GemvArgs& a, const q4d_gemv_plan& p, int dev,
-                         const DeviceState& s, cudaStream_t stream) {
+                         const DeviceState& s, cudaStream_t stream, bool pdl) {
   static std::atomic<bool> smem_set[kMaxDevices];
   auto kernel = q4d::q4_gemv_kernel<M, KC>;
   q4d_status st = allow_smem(kernel, dev, s, smem_set);
   if (st != Q4D_OK) return st;
   dim3 grid(p.grid_rows, p.k_splits);
-  kernel<<<grid, p.threads, p.smem_bytes, stream>>>(a);
-  return Q4D_OK;
+  if (!pdl) {
+    kernel<<<grid, p.threads, p.smem_bytes, stream>>>(a);
+    return Q4D_OK;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(p.threads);
+  cfg.dynamicSmemBytes = p.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a) == cudaSuccess ? Q4D_OK : Q4D_ERR_CUDA;
 }
 
 q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, int K,
                      cudaStream_t stream, void* workspace, size_t workspace_bytes,
-                     bool library_ws) {
+                     bool library_ws, bool pdl = false) {
   q4d_status st = check_gemv_shape(M, N, K);
   if (st != Q4D_OK) return st;
   if (!W_q4 || !x || !y) return Q4D_ERR_INVALID_ARG;
@@ -227,21 +240,21 @@ q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, in
   a.stages = p.stages;
 
   switch (M * 8 + p.chunk_sb) {
-    case 1 * 8 + 1: st = launch_gemv_t<1, 1>(a, p, dev, *s, stream); break;
-    case 1 * 8 + 2: st = launch_gemv_t<1, 2>(a, p, dev, *s, stream); break;
-    case 1 * 8 + 4: st = launch_gemv_t<1, 4>(a, p, dev, *s, stream); break;
-    case 2 * 8 + 1: st = launch_gemv_t<2, 1>(a, p, dev, *s, stream); break;
-    case 2 * 8 + 2: st = launch_gemv_t<2, 2>(a, p, dev, *s, stream); break;
-    case 2 * 8 + 4: st = launch_gemv_t<2, 4>(a, p, dev, *s, stream); break;
-    case 3 * 8 + 1: st = launch_gemv_t<3, 1>(a, p, dev, *s, stream); break;
-    case 3 * 8 + 2: st = launch_gemv_t<3, 2>(a, p, dev, *s, stream); break;
-    case 3 * 8 + 4: st = launch_gemv_t<3, 4>(a, p, dev, *s, stream); break;
-    case 4 * 8 + 1: st = launch_gemv_t<4, 1>(a, p, dev, *s, stream); break;
-    case 4 * 8 + 2: st = launch_gemv_t<4, 2>(a, p, dev, *s, stream); break;
-    case 4 * 8 + 4: st = launch_gemv_t<4, 4>(a, p, dev, *s, stream); break;
-    case 5 * 8 + 1: st = launch_gemv_t<5, 1>(a, p, dev, *s, stream); break;
-    case 5 * 8 + 2: st = launch_gemv_t<5, 2>(a, p, dev, *s, stream); break;
-    default: st = launch_gemv_t<5, 4>(a, p, dev, *s, stream); break;
+    case 1 * 8 + 1: st = launch_gemv_t<1, 1>(a, p, dev, *s, stream, pdl); break;
+    case 1 * 8 + 2: st = launch_gemv_t<1, 2>(a, p, dev, *s, stream, pdl); break;
+    case 1 * 8 + 4: st = launch_gemv_t<1, 4>(a, p, dev, *s, stream, pdl); break;
+    case 2 * 8 + 1: st = launch_gemv_t<2, 1>(a, p, dev, *s, stream, pdl); break;
+    case 2 * 8 + 2: st = launch_gemv_t<2, 2>(a, p, dev, *s, stream, pdl); break;
+    case 2 * 8 + 4: st = launch_gemv_t<2, 4>(a, p, dev, *s, stream, pdl); break;
+    case 3 * 8 + 1: st = launch_gemv_t<3, 1>(a, p, dev, *s, stream, pdl); break;
+    case 3 * 8 + 2: st = launch_gemv_t<3, 2>(a, p, dev, *s, stream, pdl); break;
+    case 3 * 8 + 4: st = launch_gemv_t<3, 4>(a, p, dev, *s, stream, pdl); break;
+    case 4 * 8 + 1: st = launch_gemv_t<4, 1>(a, p, dev, *s, stream, pdl); break;
+    case 4 * 8 + 2: st = launch_gemv_t<4, 2>(a, p, dev, *s, stream, pdl); break;
+    case 4 * 8 + 4: st = launch_gemv_t<4, 4>(a, p, dev, *s, stream, pdl); break;
+    case 5 * 8 + 1: st = launch_gemv_t<5, 1>(a, p, dev, *s, stream, pdl); break;
+    case 5 * 8 + 2: st = launch_gemv_t<5, 2>(a, p, dev, *s, stream, pdl); break;
+    default: st = launch_gemv_t<5, 4>(a, p, dev, *s, stream, pdl); break;
   }
   if (st != Q4D_OK) return st;
   if (p.k_splits > 1) {
@@ -408,10 +421,14 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   if (!plan || num_sms < 1) return Q4D_ERR_INVALID_ARG;
   q4d_status st = check_attn_shape(ctx_len, n_q_heads, n_kv_heads, head_dim, M, ctx_len, 1.0f);
   if (st != Q4D_OK) return st;
-  const int TT = q4d::kAttnTileTokens;
   const int rows_all = (n_q_heads / n_kv_heads) * M;
   const int row_groups = ceil_div(rows_all, q4d::kAttnMaxRows);
   const int rows_per_cta = ceil_div(rows_all, row_groups);
+  // Variant: warp-local (12 warps, 192-token tiles) for at most 8 rows per
+  // CTA, else generic (8 warps + a producer warp, 128-token tiles).
+  const bool rows8 = rows_per_cta <= 8;
+  const int TT = rows8 ? q4d::kR8Tile : q4d::kAttnTileTokens;
+  const size_t stage_bytes = rows8 ? q4d::kR8StageBytes : q4d::kAttnStageBytes;
   // One CTA per SM (the K/V ring takes most of shared memory): enough context
   // splits that (splits x KV heads x row groups) fills the SMs once, each
   // split at least two tiles long and at most 256 splits (the merge kernel's
@@ -423,10 +440,9 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   const int split_tokens = int(round_up(ceil_div(ctx_len, n_splits), TT));
   n_splits = ceil_div(ctx_len, split_tokens);
   // As many ring stages as fit next to the variant's fixed buffers, up to 8
-  // (at least 2: the warp-local variant parks 64 KB in the ring at the end).
-  const bool rows8 = rows_per_cta <= 8;
+  // (at least 2: the warp-local variant parks 96 KB in the ring at the end).
   const size_t fixed = rows8 ? q4d::attn_rows8_smem_bytes(0) : q4d::attn_smem_bytes(0);
-  int stages = int((kAttnSmemBudget - fixed) / (q4d::kAttnStageBytes + 16));
+  int stages = int((kAttnSmemBudget - fixed) / (stage_bytes + 16));
   stages = std::max(2, std::min(8, stages));
   plan->n_splits = n_splits;
   plan->split_tokens = split_tokens;
@@ -434,7 +450,7 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   plan->row_groups = row_groups;
   plan->rows_per_cta = rows_per_cta;
   plan->stages = stages;
-  plan->threads = q4d::kAttnThreads;
+  plan->threads = rows8 ? q4d::kR8Threads : q4d::kAttnThreads;
   plan->smem_bytes = rows8 ? q4d::attn_rows8_smem_bytes(stages) : q4d::attn_smem_bytes(stages);
   plan->workspace_bytes =
       n_splits > 1 ? size_t(n_splits) * M * n_q_heads * (q4d::kHeadDim + 2) * 4 : 0;
@@ -462,6 +478,13 @@ q4d_status q4_gemv_ex(const void* W_q4, const void* x, float* y, int M, int N, i
                       void* stream, void* workspace, size_t workspace_bytes) {
   return gemv_impl(W_q4, x, y, M, N, K, static_cast<cudaStream_t>(stream), workspace,
                    workspace_bytes, false);
+}
+
+q4d_status q4_gemv_ex2(const void* W_q4, const void* x, float* y, int M, int N, int K,
+                       void* stream, void* workspace, size_t workspace_bytes, unsigned flags) {
+  if (flags & ~Q4D_GEMV_WEIGHT_PREFETCH) return Q4D_ERR_INVALID_ARG;
+  return gemv_impl(W_q4, x, y, M, N, K, static_cast<cudaStream_t>(stream), workspace,
+                   workspace_bytes, false, (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0);
 }
 
 q4d_status q4kv_attn_decode(const void* Q, const void* Kq4, const void* Vq4, float* out,

@@ -9,28 +9,29 @@
 // Work split: grid = (context split, KV head, query-row group).  One CTA holds
 // every query row that reads its KV head (g grouped heads x M draft rows, at
 // most 32) so each K/V byte of its split leaves HBM once; the splits' softmax
-// states are merged by a second kernel (log-sum-exp, base 2).
+// states are merged by a second kernel (log-sum-exp, base 2).  K and V tiles
+// (contiguous: one super-block per token) stream into a ring of shared-memory
+// stages by bulk copies on full/empty mbarriers with bounded waits.
 //
-// Per 128-token tile (one producer warp bulk-copies the K and V tiles --
-// contiguous, one super-block per token -- into a ring of stages on
-// full/empty mbarriers with bounded waits; eight consumer warps compute):
-//  1. Scores, exact: warp w takes tokens 16w..16w+15.  ldmatrix hands lane
-//     (g, t) word t of the 16-byte nibble piece of tokens g and g+8 (the
-//     A-fragment layout); nibbles become exact bf16 (q - 8); Q (bf16) is the
-//     B operand, pre-arranged in shared memory in the same element order; one
-//     fresh MMA accumulator per 32-element block is scaled by that token's
-//     fp32 block scale.  S^T = Khat Q^T arrives as (token, row) fragments.
-//  2. Online softmax in base 2 (scale * log2 e folded in): per-row tile max
-//     across the eight warps through shared memory, running max m and
-//     per-lane partial sums l rescaled by 2^(m_old - m_new); P = 2^(s - m) is
-//     rounded to fp16 and stored as P^T [token][row]; l adds the same rounded
-//     values, so numerator and denominator see identical weights.
-//  3. P.V: warp w owns the 32 dimensions of block w.  ldmatrix.trans pairs two
-//     tokens' bytes of the V piece in one register, so the A operand
-//     (q - 8)^T [dims][tokens] unpacks in registers, exact in fp16; the block
-//     scale d of V goes into the B operand instead: P^T (ldmatrix.trans) times
-//     d of the same tokens, one fp16 multiply, |P d| <= |d| so it cannot
-//     overflow.  O^T [dims][rows] accumulates in fp32 across the split.
+// Both variants below compute, per tile:
+//  1. Scores, exact up to fp32 rounding: ldmatrix hands lane (g, t) word t
+//     of the 16-byte nibble piece of tokens g and g+8 (the A-fragment layout);
+//     the nibbles become exact fp16 (q - 8); Q, converted to fp16 once, is
+//     the B operand in the same element order; one fresh MMA accumulator per
+//     32-element block is scaled by the token's block scale in fp32.
+//     S^T = Khat Q^T arrives as (token, row) fragments.
+//  2. Online softmax in base 2 (scale * log2 e folded in); P = 2^(s - m) is
+//     rounded to fp16 and the row sums add the same rounded values, so
+//     numerator and denominator see identical weights.
+//  3. P.V as O^T = (q - 8)^T (P^T d): ldmatrix.trans pairs two tokens' bytes
+//     of a V piece in one register, so the A operand (q - 8)^T [dims][tokens]
+//     unpacks in registers, exact in fp16; the V block scale d goes into the
+//     B operand, P^T times d of the same tokens in one fp16 multiply
+//     (|P d| <= |d|: no overflow).  O^T accumulates in fp32.
+// The warp-local variant (at most 8 query rows) gives each warp its own
+// tokens, softmax and full O^T; the generic one (up to 32 rows) splits tokens
+// across warps for the scores and dimensions for P.V, exchanging maxima and
+// P^T through shared memory.
 #pragma once
 
 #include "q4dec_device.cuh"
@@ -138,27 +139,64 @@ __device__ __forceinline__ uint32_t q8_pair(uint32_t r) {
                    0xD480D480u /* -72 */);
 }
 
+// Q fragments of one row, block b, lane t (16 bytes, fp16): the pairs
+// (q[4t], q[4t+2]), (q[16+4t], q[16+4t+2]), (q[4t+1], q[4t+3]),
+// (q[16+4t+1], q[16+4t+3]) of the block -- the element order in which word t
+// of a K row's nibbles unpacks (k_pairs).  bf16 -> fp16 is exact for
+// |q| in [2^-14, 65504]; smaller magnitudes round to fp16 subnormals.
+__device__ __forceinline__ uint4 q_frag_f16(const uint16_t* q /* row + 32 b + 4 t */) {
+  const uint2 lo = *reinterpret_cast<const uint2*>(q);
+  const uint2 hi = *reinterpret_cast<const uint2*>(q + 16);
+  auto f = [](uint32_t bits16) { return __uint_as_float(bits16 << 16); };
+  uint4 v;
+  v.x = pack_f16x2(f(lo.x & 0xFFFFu), f(lo.y & 0xFFFFu));
+  v.y = pack_f16x2(f(hi.x & 0xFFFFu), f(hi.y & 0xFFFFu));
+  v.z = pack_f16x2(f(lo.x >> 16), f(lo.y >> 16));
+  v.w = pack_f16x2(f(hi.x >> 16), f(hi.y >> 16));
+  return v;
+}
+
+// The eight nibbles of K word w as exact fp16 pairs q - 8, in the order
+// (byte0.lo, byte2.lo), (byte0.hi, byte2.hi), (byte1.lo, byte3.lo),
+// (byte1.hi, byte3.hi): one shift per word.
+__device__ __forceinline__ void k_pairs(uint32_t w, uint32_t (&r)[4]) {
+  r[0] = q8_pair<true>(w);
+  r[1] = q8_pair<false>(w);
+  r[2] = q8_pair<true>(w >> 8);
+  r[3] = q8_pair<false>(w >> 8);
+}
+
+constexpr int kR8Warps = 12;                                   // consumer warps
+constexpr int kR8QPitch = 8 * 4 * 16 + 64;                     // bytes per row of Q fragments
+constexpr int kR8Threads = kR8Warps * 32;
+constexpr int kR8Tile = 16 * kR8Warps;                         // 192 tokens per tile
+constexpr uint32_t kR8StageBytes = 2u * kR8Tile * kRowBytes;   // K tile + V tile
+
 // Shared memory of the warp-local variant: the ring (which also holds the
-// final cross-warp combine, 64 KB) plus per-warp row statistics and barriers.
+// final cross-warp combine, 96 KB), Q fragments of 8 rows, per-warp and
+// per-row statistics, barriers.
 __host__ __device__ constexpr size_t attn_rows8_smem_bytes(int stages) {
-  return size_t(stages) * kAttnStageBytes + size_t(kAttnConsumerWarps) * 8 * 2 * 4 + 8 * 2 * 4 +
-         size_t(stages) * 16;
+  return size_t(stages) * kR8StageBytes + 8 * kR8QPitch + size_t(kR8Warps) * 8 * 2 * 4 +
+         8 * 2 * 4 + size_t(stages) * 16;
 }
 
 // Warp-local variant for at most 8 query rows per CTA (one row tile: plain
-// decode, M = 1).  Each consumer warp owns tokens 16w .. 16w + 15 of every
-// tile and carries its own online softmax and its own O^T for all 256
-// dimensions (64 fp32 registers), so a tile needs no CTA-wide barrier: the
+// decode, M = 1).  Twelve warps, each owning tokens 16w .. 16w + 15 of every
+// 192-token tile, carry their own online softmax and their own O^T for all
+// 256 dimensions (64 fp32 registers): a tile needs no CTA-wide barrier.  The
 // score fragments (token, row) are rounded to fp16 and transposed in
-// registers with movmatrix into the P^T operand of P.V.  The eight warps'
-// states are combined once, at the end of the split.
-__global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_rows8_kernel(const AttnArgs a) {
-  constexpr int TT = kAttnTileTokens;
+// registers with movmatrix into the P^T operand of P.V.  Lane 0 of warp 0
+// also issues the bulk copies (a separate producer warp would cut every
+// thread's register budget); it blocks only for the tile it needs next.  The
+// warps' states are combined once, at the end of the split.
+__global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(const AttnArgs a) {
+  constexpr int TT = kR8Tile;
   extern __shared__ __align__(128) uint8_t smem[];
   const int S = a.stages;
   uint8_t* ring = smem;
-  float* wml = reinterpret_cast<float*>(ring + size_t(S) * kAttnStageBytes);  // [warp][row][m, l]
-  float* rml = wml + kAttnConsumerWarps * 8 * 2;                              // [row][M, L]
+  uint8_t* Qf = ring + size_t(S) * kR8StageBytes;                 // [row] x kR8QPitch
+  float* wml = reinterpret_cast<float*>(Qf + 8 * kR8QPitch);       // [warp][row][m, l]
+  float* rml = wml + kR8Warps * 8 * 2;                              // [row][M, L]
   uint64_t* full = reinterpret_cast<uint64_t*>(rml + 8 * 2);
   uint64_t* empty = full + S;
 
@@ -169,63 +207,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_rows8_kernel(
   const int t_begin = split * a.split_tokens;
   const int t_end = min(a.ctx_len, t_begin + a.split_tokens);
   const int n_tiles = (t_end - t_begin + TT - 1) / TT;
+  const bool producer = tid == 0;
+  const uint8_t* Kh = a.K + size_t(kh) * a.kv_stride * kRowBytes;
+  const uint8_t* Vh = a.V + size_t(kh) * a.kv_stride * kRowBytes;
+  const uint64_t pol = l2_evict_first_policy();
+  auto issue = [&](int tile) {
+    const int t0 = t_begin + tile * TT;
+    const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * kRowBytes;
+    const int slot = tile % S;
+    const uint32_t bar = smem_addr(&full[slot]);
+    const uint32_t dk = smem_addr(ring + size_t(slot) * kR8StageBytes);
+    mbar_arrive_expect_tx(bar, 2 * bytes);
+    bulk_g2s(dk, Kh + size_t(t0) * kRowBytes, bytes, bar, pol);
+    bulk_g2s(dk + TT * kRowBytes, Vh + size_t(t0) * kRowBytes, bytes, bar, pol);
+  };
 
-  if (tid == 0) {
+  int issued = 0;
+  if (producer) {
+    griddep_launch_dependents();  // a following weight-prefetching GEMV may start
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_addr(&full[s]), 1);
-      mbar_init(smem_addr(&empty[s]), kAttnConsumerWarps);
+      mbar_init(smem_addr(&empty[s]), kR8Warps);
     }
     mbar_init_fence();
+    // start streaming before anything else
+    for (; issued < min(S, n_tiles); ++issued) issue(issued);
+  }
+  // Q fragments (zero for padding rows)
+  for (int i = tid; i < 8 * 32; i += kR8Threads) {
+    const int r = i >> 5, b = (i >> 2) & 7, tt = i & 3;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < R) {
+      const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
+      v = q_frag_f16(a.Q + (size_t(m) * a.n_q + kh * a.g + j) * kHeadDim + b * 32 + 4 * tt);
+    }
+    *reinterpret_cast<uint4*>(Qf + r * kR8QPitch + (i & 31) * 16) = v;
   }
   __syncthreads();
 
-  if (warp == kAttnConsumerWarps) {
-    if (lane == 0) {
-      const uint8_t* Kh = a.K + size_t(kh) * a.kv_stride * kRowBytes;
-      const uint8_t* Vh = a.V + size_t(kh) * a.kv_stride * kRowBytes;
-      const uint64_t pol = l2_evict_first_policy();
-      int slot = 0;
-      uint32_t phase = 0;
-      for (int tile = 0; tile < n_tiles; ++tile) {
-        if (tile >= S) mbar_wait(smem_addr(&empty[slot]), phase ^ 1u, a.err);
-        const int t0 = t_begin + tile * TT;
-        const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * kRowBytes;
-        const uint32_t bar = smem_addr(&full[slot]);
-        const uint32_t dk = smem_addr(ring + size_t(slot) * kAttnStageBytes);
-        mbar_arrive_expect_tx(bar, 2 * bytes);
-        bulk_g2s(dk, Kh + size_t(t0) * kRowBytes, bytes, bar, pol);
-        bulk_g2s(dk + TT * kRowBytes, Vh + size_t(t0) * kRowBytes, bytes, bar, pol);
-        if (++slot == S) {
-          slot = 0;
-          phase ^= 1u;
-        }
-      }
-    }
-    return;
-  }
-
   const int g = lane >> 2, t = lane & 3;
-  // Q fragments of row g (zero for padding rows), in the nibble order of a
-  // K word: see the generic kernel below.
-  uint4 qf[8];
-  {
-    const bool live = g < R;
-    const int rr = row0 + g, m = rr / a.g, j = rr - m * a.g;
-    const uint16_t* q = a.Q + (size_t(live ? m : 0) * a.n_q + kh * a.g + (live ? j : 0)) * kHeadDim + 4 * t;
-    #pragma unroll
-    for (int b = 0; b < 8; ++b) {
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (live) {
-        const uint2 lo = *reinterpret_cast<const uint2*>(q + b * 32);
-        const uint2 hi = *reinterpret_cast<const uint2*>(q + b * 32 + 16);
-        v.x = prmt(lo.x, lo.y, 0x5410);
-        v.y = prmt(hi.x, hi.y, 0x5410);
-        v.z = prmt(lo.x, lo.y, 0x7632);
-        v.w = prmt(hi.x, hi.y, 0x7632);
-      }
-      qf[b] = v;
-    }
-  }
   int row_pos[2];
   float m_run[2], l_run[2];
   #pragma unroll
@@ -241,20 +261,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_rows8_kernel(
     #pragma unroll
     for (int d = 0; d < 2; ++d) o[b][d][0] = o[b][d][1] = o[b][d][2] = o[b][d][3] = 0.f;
 
-  const uint32_t bmask = 0x000F000Fu, bmagic = 0x43004300u, b136 = 0x43084308u;
   const int tok0 = 16 * warp;
   // ldmatrix rows of this warp's 16 tokens: lanes 0-15 tokens tok0 + lane at
   // block b, lanes 16-31 tokens tok0 + lane - 16 at block b + 1
   const uint32_t lrow = uint32_t(tok0 + (lane & 15)) * kRowBytes + uint32_t(lane >> 4) * 16u;
+  const uint4* qrow = reinterpret_cast<const uint4*>(Qf + g * kR8QPitch) + t;  // + 4 b
   int slot = 0;
   uint32_t phase = 0;
 
   #pragma unroll 1
   for (int tile = 0; tile < n_tiles; ++tile) {
+    if (producer) {
+      // refill the slots every warp has released; block only for this tile
+      while (issued < n_tiles && issued < tile + S) {
+        const uint32_t bar = smem_addr(&empty[issued % S]);
+        const uint32_t parity = uint32_t(issued / S - 1) & 1u;
+        if (issued > tile) {
+          if (!mbar_test_wait(bar, parity)) break;
+        } else if (!mbar_wait(bar, parity, a.err)) {
+          break;
+        }
+        issue(issued++);
+      }
+    }
+    __syncwarp();
     const int t0 = t_begin + tile * TT;
     const int n_tok = min(TT, t_end - t0);
     mbar_wait(smem_addr(&full[slot]), phase, a.err);
-    const uint8_t* Kt = ring + size_t(slot) * kAttnStageBytes;
+    const uint8_t* Kt = ring + size_t(slot) * kR8StageBytes;
     const uint8_t* Vt = Kt + TT * kRowBytes;
     if (tok0 < n_tok) {
       const uint32_t Kt_addr = smem_addr(Kt), Vt_addr = smem_addr(Vt);
@@ -271,12 +305,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_rows8_kernel(
         #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
           uint32_t qa[4], qb[4];
-          dequant_pairs(bb ? w1a : w0a, bmask, bmagic, b136, qa);
-          dequant_pairs(bb ? w1b : w0b, bmask, bmagic, b136, qb);
-          const uint4 qv = qf[b + bb];
+          k_pairs(bb ? w1a : w0a, qa);
+          k_pairs(bb ? w1b : w0b, qb);
+          const uint4 qv = qrow[4 * (b + bb)];
           float c[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_bf16(c, qa[0], qb[0], qa[1], qb[1], qv.x, qv.y);
-          mma_bf16(c, qa[2], qb[2], qa[3], qb[3], qv.z, qv.w);
+          mma_f16(c, qa[0], qb[0], qa[1], qb[1], qv.x, qv.y);
+          mma_f16(c, qa[2], qb[2], qa[3], qb[3], qv.z, qv.w);
           const float da = bb ? dA.y : dA.x, db = bb ? dB.y : dB.x;
           s[0] = fmaf(da, c[0], s[0]);
           s[1] = fmaf(da, c[1], s[1]);
@@ -297,8 +331,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_rows8_kernel(
         mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
         const float m_new = fmaxf(m_run[e], mx);
+        // a row with no visible token so far (or a padding row) keeps
+        // m = -inf, weight 0 and alpha = 1: nothing to rescale
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        alpha[e] = ex2(m_run[e] - m_use);
+        alpha[e] = m_new == -INFINITY ? 1.f : ex2(m_run[e] - m_use);
         m_run[e] = m_new;
         s[e] = ex2(s[e] - m_use);
         s[2 + e] = ex2(s[2 + e] - m_use);
@@ -364,8 +400,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_rows8_kernel(
     }
   }
 
-  // ---- combine the eight warps: per-row maxima and sums, then O^T parked in
-  // the (now idle) ring as [warp][row][dim] and summed in warp order
+  // ---- combine the warps: per-row maxima and sums, then O^T parked in the
+  // (now idle) ring as [warp][row][dim] and summed in warp order
   #pragma unroll
   for (int e = 0; e < 2; ++e) {
     float l = l_run[e];
@@ -377,18 +413,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_rows8_kernel(
       wml[(warp * 8 + 2 * t + e) * 2 + 1] = l;
     }
   }
-  attn_consumer_sync();
+  __syncthreads();
   float cw[2];
   #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int r = 2 * t + e;
     float M = -INFINITY;
-    for (int w = 0; w < kAttnConsumerWarps; ++w) M = fmaxf(M, wml[(w * 8 + r) * 2]);
+    for (int w = 0; w < kR8Warps; ++w) M = fmaxf(M, wml[(w * 8 + r) * 2]);
     const float m_use = M == -INFINITY ? 0.f : M;
     cw[e] = ex2(m_run[e] - m_use);
     if (warp == 0 && g == 0) {
       float L = 0.f;
-      for (int w = 0; w < kAttnConsumerWarps; ++w)
+      for (int w = 0; w < kR8Warps; ++w)
         L += wml[(w * 8 + r) * 2 + 1] * ex2(wml[(w * 8 + r) * 2] - m_use);
       rml[r * 2 + 0] = M;
       rml[r * 2 + 1] = L;
@@ -403,20 +439,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_rows8_kernel(
       for (int k = 0; k < 4; ++k)
         park[(2 * t + (k & 1)) * kHeadDim + 32 * b + 2 * g + d + (k >= 2 ? 16 : 0)] =
             o[b][d][k] * cw[k & 1];
-  attn_consumer_sync();
+  __syncthreads();
   const float* parked = reinterpret_cast<const float*>(ring);
   const size_t rows_total = size_t(a.M) * a.n_q;
-  for (int r = 0; r < R; ++r) {
+  for (int i = tid; i < R * kHeadDim; i += kR8Threads) {
+    const int r = i / kHeadDim, dim = i - r * kHeadDim;
     float acc = 0.f;
     #pragma unroll
-    for (int w = 0; w < kAttnConsumerWarps; ++w) acc += parked[(w * 8 + r) * kHeadDim + tid];
+    for (int w = 0; w < kR8Warps; ++w) acc += parked[(w * 8 + r) * kHeadDim + dim];
     const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
     const size_t row = size_t(m) * a.n_q + kh * a.g + j;
     if (a.n_splits == 1) {
-      a.out[row * kHeadDim + tid] = acc / rml[r * 2 + 1];
+      a.out[row * kHeadDim + dim] = acc / rml[r * 2 + 1];
     } else {
-      a.ws_o[(size_t(split) * rows_total + row) * kHeadDim + tid] = acc;
-      if (tid == 0) {
+      a.ws_o[(size_t(split) * rows_total + row) * kHeadDim + dim] = acc;
+      if (dim == 0) {
         a.ws_ml[(size_t(split) * rows_total + row) * 2 + 0] = rml[r * 2 + 0];
         a.ws_ml[(size_t(split) * rows_total + row) * 2 + 1] = rml[r * 2 + 1];
       }
@@ -453,6 +490,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const 
   const uint8_t* Vh = a.V + size_t(kh) * a.kv_stride * kRowBytes;
 
   if (tid == 0) {
+    griddep_launch_dependents();  // a following weight-prefetching GEMV may start
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_addr(&full[s]), 1);
       mbar_init(smem_addr(&empty[s]), kAttnConsumerWarps);
@@ -488,22 +526,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const 
   // ---------------- consumers ----------------
   const int g = lane >> 2, t = lane & 3;
 
-  // Q fragments.  For row r, block b and lane t, 16 bytes: the bf16 pairs
-  // (q[4t], q[4t+2]), (q[16+4t], q[16+4t+2]), (q[4t+1], q[4t+3]),
-  // (q[16+4t+1], q[16+4t+3]) of the block -- the element order in which the
-  // nibbles of word t of a K row unpack.  Rows past R are zero.
+  // Q fragments (fp16, zero for padding rows): see q_frag_f16.
   for (int i = tid; i < kAttnMaxRows * 32; i += kAttnConsumerWarps * 32) {
     const int r = i >> 5, b = (i >> 2) & 7, tt = i & 3;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (r < R) {
       const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
-      const uint16_t* q = a.Q + (size_t(m) * a.n_q + kh * a.g + j) * kHeadDim + b * 32 + 4 * tt;
-      const uint2 lo = *reinterpret_cast<const uint2*>(q);
-      const uint2 hi = *reinterpret_cast<const uint2*>(q + 16);
-      v.x = prmt(lo.x, lo.y, 0x5410);
-      v.y = prmt(hi.x, hi.y, 0x5410);
-      v.z = prmt(lo.x, lo.y, 0x7632);
-      v.w = prmt(hi.x, hi.y, 0x7632);
+      v = q_frag_f16(a.Q + (size_t(m) * a.n_q + kh * a.g + j) * kHeadDim + b * 32 + 4 * tt);
     }
     *reinterpret_cast<uint4*>(Qp + r * kQPitch + (i & 31) * 16) = v;
   }
@@ -528,7 +557,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const 
     #pragma unroll
     for (int rt = 0; rt < NRT; ++rt) o[d][rt][0] = o[d][rt][1] = o[d][rt][2] = o[d][rt][3] = 0.f;
 
-  const uint32_t bmask = 0x000F000Fu, bmagic = 0x43004300u, b136 = 0x43084308u;
   int slot = 0;
   uint32_t phase = 0;
 
@@ -564,8 +592,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const 
         #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
           uint32_t qa[4], qb[4];
-          dequant_pairs(bb ? w1a : w0a, bmask, bmagic, b136, qa);
-          dequant_pairs(bb ? w1b : w0b, bmask, bmagic, b136, qb);
+          k_pairs(bb ? w1a : w0a, qa);
+          k_pairs(bb ? w1b : w0b, qb);
           const float da = bb ? dA.y : dA.x, db = bb ? dB.y : dB.x;
           #pragma unroll
           for (int rt = 0; rt < NRT; ++rt) {
@@ -574,8 +602,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const 
                          : "=r"(qf.x), "=r"(qf.y), "=r"(qf.z), "=r"(qf.w)
                          : "r"(Qp_addr + uint32_t((8 * rt + g) * kQPitch + ((b + bb) * 4 + t) * 16)));
             float c[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_bf16(c, qa[0], qb[0], qa[1], qb[1], qf.x, qf.y);
-            mma_bf16(c, qa[2], qb[2], qa[3], qb[3], qf.z, qf.w);
+            mma_f16(c, qa[0], qb[0], qa[1], qb[1], qf.x, qf.y);
+            mma_f16(c, qa[2], qb[2], qa[3], qb[3], qf.z, qf.w);
             s[rt][0] = fmaf(da, c[0], s[rt][0]);
             s[rt][1] = fmaf(da, c[1], s[rt][1]);
             s[rt][2] = fmaf(db, c[2], s[rt][2]);
@@ -613,9 +641,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const 
         const float tile_max = fmaxf(fmaxf(fmaxf(x0.x, x0.y), fmaxf(x0.z, x0.w)),
                                      fmaxf(fmaxf(x1.x, x1.y), fmaxf(x1.z, x1.w)));
         const float m_new = fmaxf(m_run[rt][e], tile_max);
-        // a row with no visible token so far keeps m = -inf and weight 0
+        // a row with no visible token so far keeps m = -inf, weight 0, alpha 1
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        alpha[rt][e] = ex2(m_run[rt][e] - m_use);
+        alpha[rt][e] = m_new == -INFINITY ? 1.f : ex2(m_run[rt][e] - m_use);
         m_run[rt][e] = m_new;
         s[rt][e] = ex2(s[rt][e] - m_use);
         s[rt][2 + e] = ex2(s[rt][2 + e] - m_use);
@@ -763,6 +791,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const 
 __global__ void __launch_bounds__(256) q4kv_attn_merge_kernel(const AttnArgs a) {
   const int row = blockIdx.x;  // m * n_q + h
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) griddep_launch_dependents();
   const size_t rows = size_t(a.M) * a.n_q;
   __shared__ float part[8 * kHeadDim];
   const int n = a.n_splits;

@@ -25,7 +25,7 @@ STATUS = {
 
 EXPORTS = (
     "q4d_version", "q4d_status_string",
-    "q4_gemv", "q4_gemv_ex", "q4d_gemv_workspace_bytes",
+    "q4_gemv", "q4_gemv_ex", "q4_gemv_ex2", "q4d_gemv_workspace_bytes",
     "q4kv_attn_decode", "q4kv_attn_decode_ex", "q4d_attn_workspace_bytes",
     "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
     "q4kv_attn_decode_noalloc",
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
     L.q4d_status_string.restype = ctypes.c_char_p
     L.q4_gemv.argtypes = [vp, vp, vp, i, i, i]
     L.q4_gemv_ex.argtypes = [vp, vp, vp, i, i, i, vp, vp, sz]
+    L.q4_gemv_ex2.argtypes = [vp, vp, vp, i, i, i, vp, vp, sz, ctypes.c_uint]
     L.q4d_gemv_workspace_bytes.argtypes = [i, i, i]
     L.q4d_gemv_workspace_bytes.restype = sz
     L.q4kv_attn_decode.argtypes = [vp, vp, vp, vp, i, i, i, i, i]
@@ -82,7 +83,7 @@ def lib() -> ctypes.CDLL:
     L.q4d_plan_attn.argtypes = [i, i, i, i, i, i, ctypes.POINTER(AttnPlan)]
     L.q4d_device_error.argtypes = [i]
     L.q4kv_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
-    for fn in ("q4_gemv", "q4_gemv_ex", "q4kv_attn_decode", "q4kv_attn_decode_ex",
+    for fn in ("q4_gemv", "q4_gemv_ex", "q4_gemv_ex2", "q4kv_attn_decode", "q4kv_attn_decode_ex",
                "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
                "q4kv_attn_decode_noalloc"):
         getattr(L, fn).restype = i
@@ -143,11 +144,17 @@ def _workspace(nbytes: int, device, workspace):
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
-def q4_gemv(W, x, y=None, *, N: int, K: int, stream=None, workspace=None):
-    """y[M][N] (fp32) = dequant(W)[N][K] @ x[M][K]^T via ``q4_gemv_ex``.
+GEMV_WEIGHT_PREFETCH = 1  # Q4D_GEMV_WEIGHT_PREFETCH
+
+
+def q4_gemv(W, x, y=None, *, N: int, K: int, stream=None, workspace=None,
+            weight_prefetch: bool = False):
+    """y[M][N] (fp32) = dequant(W)[N][K] @ x[M][K]^T via ``q4_gemv_ex2``.
 
     ``W``: uint8 CUDA tensor with N*K/256*144 bytes (super-block layout);
     ``x``: bf16 CUDA tensor [M][K]; ``y``: optional fp32 [M][N] output.
+    ``weight_prefetch``: Q4D_GEMV_WEIGHT_PREFETCH (programmatic dependent
+    launch; W must not be written by earlier kernels still in flight).
     """
     torch = _torch()
     _dev_tensor(W, torch.uint8, "W")
@@ -165,8 +172,9 @@ def q4_gemv(W, x, y=None, *, N: int, K: int, stream=None, workspace=None):
     with torch.cuda.device(x.device):
         need = lib().q4d_gemv_workspace_bytes(M, N, K)
         ws = _workspace(need, x.device, workspace)
-        st = lib().q4_gemv_ex(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K,
-                              _stream_ptr(stream), None if ws is None else ws.data_ptr(), need)
+        st = lib().q4_gemv_ex2(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K,
+                               _stream_ptr(stream), None if ws is None else ws.data_ptr(), need,
+                               GEMV_WEIGHT_PREFETCH if weight_prefetch else 0)
     _check(st, "q4_gemv")
     return y
 

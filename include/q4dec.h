@@ -102,6 +102,23 @@ const char* q4d_status_string(int status);
 q4d_status q4_gemv(const void* W_q4, const void* x, float* y, int M, int N, int K);
 q4d_status q4_gemv_ex(const void* W_q4, const void* x, float* y, int M, int N, int K,
                       void* stream, void* workspace, size_t workspace_bytes);
+
+/* q4_gemv_ex2: q4_gemv_ex plus launch flags (0 behaves exactly as q4_gemv_ex;
+ * any other bit is Q4D_ERR_INVALID_ARG).
+ *
+ *   Q4D_GEMV_WEIGHT_PREFETCH: launch with programmatic dependent launch.  The
+ *   kernel's CTAs may start while the kernel before it on the stream is still
+ *   running, and stream the first pipeline stages of W_q4 at once; they read
+ *   x, and write y and the workspace, only after that kernel has completed
+ *   and its writes are visible.  The caller guarantees that no kernel issued
+ *   earlier on the stream still writes W_q4 (true for inference weights).
+ *   Back-to-back GEMVs then overlap one call's start-up with the previous
+ *   call's tail.  No counterpart in the source pages: a launch-time option of
+ *   this library.
+ */
+#define Q4D_GEMV_WEIGHT_PREFETCH 1u
+q4d_status q4_gemv_ex2(const void* W_q4, const void* x, float* y, int M, int N, int K,
+                       void* stream, void* workspace, size_t workspace_bytes, unsigned flags);
 /* Workspace bytes q4_gemv_ex needs on the CURRENT device (depends on its SM
  * count; a host without a usable device is planned for 148 SMs).  Returns 0
  * for invalid shapes as well as for shapes that need none. */

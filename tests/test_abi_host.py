@@ -48,6 +48,16 @@ def test_gemv_rejects_bad_shapes_without_cuda(M, N, K, code):
     assert L.q4_gemv(FAKE, FAKE, FAKE, M, N, K) == code
 
 
+def test_gemv_ex2_rejects_unknown_flags_and_bad_shapes_without_cuda():
+    L = q4dec.lib()
+    for flags in (2, 4, 0x80000000, 3):
+        assert L.q4_gemv_ex2(FAKE, FAKE, FAKE, 1, 16, 256, None, None, 0, flags) == 1
+    for flags in (0, q4dec.GEMV_WEIGHT_PREFETCH):
+        assert L.q4_gemv_ex2(FAKE, FAKE, FAKE, 6, 16, 256, None, None, 0, flags) == 2
+        assert L.q4_gemv_ex2(FAKE + 8, FAKE, FAKE, 1, 16, 256, None, None, 0, flags) == 3
+        assert L.q4_gemv_ex2(None, FAKE, FAKE, 1, 16, 256, None, None, 0, flags) == 1
+
+
 def test_gemv_rejects_null_and_misaligned_pointers():
     L = q4dec.lib()
     assert L.q4_gemv_ex(None, FAKE, FAKE, 1, 16, 256, None, None, 0) == 1

@@ -100,13 +100,15 @@ ATTN_CASES = [(4096, 24, 4, 1), (4096, 24, 4, 5), (65536, 24, 4, 5), (262144, 24
 
 
 TT_ATTN, Q_PITCH, PT_PITCH, ROW = 128, 576, 80, 144
+TT_R8, WARPS_R8 = 192, 12          # warp-local variant (at most 8 rows per CTA)
 
 
 def _attn_smem(stages, rows_per_cta):
-    ring = stages * 2 * TT_ATTN * ROW
-    if rows_per_cta <= 8:      # warp-local variant: ring + per-warp / per-row stats
-        return ring + 8 * 8 * 2 * 4 + 8 * 2 * 4 + stages * 16
-    return ring + 32 * Q_PITCH + TT_ATTN * PT_PITCH + 32 * 8 * 4 + 32 * 4 + stages * 16
+    if rows_per_cta <= 8:      # ring + Q fragments + per-warp / per-row stats + barriers
+        return stages * 2 * TT_R8 * ROW + 8 * Q_PITCH + WARPS_R8 * 8 * 2 * 4 + 8 * 2 * 4 \
+            + stages * 16
+    return stages * 2 * TT_ATTN * ROW + 32 * Q_PITCH + TT_ATTN * PT_PITCH + 32 * 8 * 4 + 32 * 4 \
+        + stages * 16
 
 
 def _chunks(addrs):
@@ -145,16 +147,19 @@ def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
     TT = p.tile_tokens
     stride = ctx + stride_extra
     g = nq // nkv
-    assert TT == TT_ATTN and p.split_tokens % TT == 0 and p.threads == 288
+    rows8 = p.rows_per_cta <= 8
+    assert TT == (TT_R8 if rows8 else TT_ATTN) and p.split_tokens % TT == 0
+    assert p.threads == (WARPS_R8 * 32 if rows8 else 288)
     assert 1 <= p.n_splits <= 256
     assert p.rows_per_cta <= 32 and p.row_groups * p.rows_per_cta >= g * M
     assert 2 <= p.stages <= 8
     assert p.smem_bytes == _attn_smem(p.stages, p.rows_per_cta) <= SMEM_OPTIN
     ring = p.stages * 2 * TT * ROW
-    if p.rows_per_cta <= 8:
-        # warp-local: the final combine parks [8 warps][8 rows][256] fp32 in the ring
-        assert ring >= 8 * 8 * 256 * 4
-        assert (ring + 8 * 8 * 2 * 4 + 8 * 2 * 4) % 8 == 0
+    if rows8:
+        # the final combine parks [12 warps][8 rows][256] fp32 in the ring;
+        # Q fragments follow the ring (16-byte aligned), barriers 8-aligned
+        assert ring >= WARPS_R8 * 8 * 256 * 4
+        assert ring % 16 == 0 and (ring + 8 * Q_PITCH + WARPS_R8 * 64 + 64) % 8 == 0
     else:
         # carve-up: ring, Q fragments, P^T (16-byte aligned for ldmatrix / v4),
         # row maxima, row sums, barriers (8-byte aligned)
@@ -185,16 +190,23 @@ def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
         rows.extend(range(r0, r0 + R))
     assert rows == list(range(g * M))
     nrt = -(-p.rows_per_cta // 8)
-    for warp in range(8):
-        for lane in range(32):
-            # warp-local variant: ldmatrix rows (K and V) and the 16-byte
-            # scale vectors of tokens 2t, 2t + 1, 2t + 8, 2t + 9
-            tok = 16 * warp + (lane & 15)
-            for b in range(0, 8, 2):
-                assert tok < TT and (lane >> 4) * 16 + b * 16 + 16 <= 128
-            for i in range(4):
-                tk = 16 * warp + 2 * (lane & 3) + (i & 1) + (i >> 1) * 8
-                assert tk < TT and (tk * ROW + 128) % 16 == 0
+    if rows8:
+        for warp in range(WARPS_R8):
+            for lane in range(32):
+                # ldmatrix rows (K and V) and the 16-byte scale vectors of
+                # tokens 2t, 2t + 1, 2t + 8, 2t + 9
+                tok = 16 * warp + (lane & 15)
+                for b in range(0, 8, 2):
+                    assert tok < TT and (lane >> 4) * 16 + b * 16 + 16 <= 128
+                for i in range(4):
+                    tk = 16 * warp + 2 * (lane & 3) + (i & 1) + (i >> 1) * 8
+                    assert tk < TT and (tk * ROW + 128) % 16 == 0
+                # park index of the final combine
+                g_, t_ = lane >> 2, lane & 3
+                hi = (warp * 8 + 2 * t_ + 1) * 256 + 32 * 7 + 2 * g_ + 1 + 16
+                assert hi < WARPS_R8 * 8 * 256
+        _attn_q_and_workspace(p, M, nq, nkv, g)
+        return
     # generic variant: K ldmatrix rows / columns, block scales, V
     # ldmatrix.trans rows, P^T ldmatrix.trans rows / columns
     for warp in range(8):
@@ -212,6 +224,10 @@ def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
                     for rt in range(0, nrt, 2):
                         pcol = rt * 16 + (lane >> 4) * 16 if rt + 1 < nrt else rt * 16
                         assert kb + (lane & 15) < TT and pcol + 16 <= 64
+    _attn_q_and_workspace(p, M, nq, nkv, g)
+
+
+def _attn_q_and_workspace(p, M, nq, nkv, g):
     # Q reads (global, 8-byte vectors) stay inside [M][n_q][256]
     q_elems = M * nq * 256
     for kh in range(nkv):
@@ -229,3 +245,60 @@ def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
         assert p.workspace_bytes == p.n_splits * nrows * 258 * 4
     else:
         assert p.workspace_bytes == 0
+
+
+def _simulate_in_warp_producer(n_tiles, S, warps, seed):
+    """Random schedules of the warp-local variant's copy protocol: lane 0 of
+    warp 0 issues tile k into slot k % S only once every warp has released
+    tile k - S; at the start of its tile i it issues what it can without
+    waiting, and waits only when tile i itself is not issued yet.  Every
+    schedule must finish (no state where all warps wait forever)."""
+    import random
+
+    rnd = random.Random(seed)
+    done = [0] * warps              # tiles finished per warp
+    issued = min(S, n_tiles)        # prologue
+    pending = [True] * warps        # warp 0's refill step still to run at its current tile
+    released = lambda k: all(d > k for d in done)
+    steps = 0
+    while min(done) < n_tiles:
+        steps += 1
+        assert steps < 100000
+        movable = []
+        for w in range(warps):
+            i = done[w]
+            if i >= n_tiles:
+                continue
+            if w == 0 and pending[0]:
+                # can the refill step finish now?
+                blocked = False
+                k = issued
+                while k < n_tiles and k < i + S:
+                    if not released(k - S):
+                        blocked = k <= i
+                        break
+                    k += 1
+                if not blocked:
+                    movable.append(w)
+                continue
+            if issued > i:          # tile i's copies were issued: its full barrier completes
+                movable.append(w)
+        assert movable, f"deadlock: done={done} issued={issued}"
+        w = rnd.choice(movable)
+        if w == 0 and pending[0]:
+            i = done[0]
+            while issued < n_tiles and issued < i + S and released(issued - S):
+                # slot issued % S held tile issued - S, which every warp has left
+                assert all(d >= issued - S + 1 for d in done)
+                issued += 1
+            pending[0] = False
+            continue
+        done[w] += 1
+        if w == 0:
+            pending[0] = True
+
+
+@pytest.mark.parametrize("n_tiles,S", [(1, 2), (2, 2), (3, 2), (7, 3), (37, 4), (40, 4), (5, 8)])
+def test_in_warp_producer_never_deadlocks(n_tiles, S):
+    for seed in range(40):
+        _simulate_in_warp_producer(n_tiles, S, WARPS_R8, seed)
