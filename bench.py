@@ -70,12 +70,14 @@ def kernel_source_hash():
 
 
 def recorded_traffic(kernel):
-    """DRAM bytes per launch from a committed ncu capture, if it was taken on
-    the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    """DRAM bytes per launch from a committed ncu capture (the json block of
+    profiles/dram_traffic.md), if it was taken on the current kernel sources
+    (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
     try:
         with open(path) as f:
-            rec = json.load(f)
+            text = f.read()
+        rec = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
     except Exception:
         return None
     e = rec.get(kernel)
