@@ -502,6 +502,71 @@ q4d_status q4kv_attn_decode_ex(const void* Q, const void* Kq4, const void* Vq4, 
                    workspace_bytes, false);
 }
 
+}  // extern "C"
+
+// ---- host layout helpers: canonical 18-byte blocks <-> 144-byte super-blocks
+namespace {
+q4d_status check_pack_args(const void* a, const void* b, int rows, int K) {
+  if (!a || !b || rows < 1 || K < 0) return Q4D_ERR_INVALID_ARG;
+  if (K < 256 || K % 256 != 0) return Q4D_ERR_UNSUPPORTED_SHAPE;
+  return Q4D_OK;
+}
+// super-block index of (row r, column s) in either layout
+size_t sb_index(bool column_major, int rows, int nsb, int r, int s) {
+  return column_major ? size_t(s) * rows + r : size_t(r) * nsb + s;
+}
+q4d_status pack_impl(const void* blocks18, void* out, int rows, int K, bool column_major) {
+  q4d_status st = check_pack_args(blocks18, out, rows, K);
+  if (st != Q4D_OK) return st;
+  const int nsb = K / 256;
+  const uint8_t* in = static_cast<const uint8_t*>(blocks18);
+  uint8_t* o = static_cast<uint8_t*>(out);
+  for (int r = 0; r < rows; ++r)
+    for (int s = 0; s < nsb; ++s) {
+      uint8_t* sb = o + sb_index(column_major, rows, nsb, r, s) * 144;
+      for (int b = 0; b < 8; ++b) {
+        const uint8_t* blk = in + (size_t(r) * (K / 32) + size_t(s) * 8 + b) * 18;
+        std::memcpy(sb + 16 * b, blk + 2, 16);     // nibbles
+        std::memcpy(sb + 128 + 2 * b, blk, 2);     // fp16 scale
+      }
+    }
+  return Q4D_OK;
+}
+q4d_status unpack_impl(const void* in_q4, void* blocks18, int rows, int K, bool column_major) {
+  q4d_status st = check_pack_args(in_q4, blocks18, rows, K);
+  if (st != Q4D_OK) return st;
+  const int nsb = K / 256;
+  const uint8_t* in = static_cast<const uint8_t*>(in_q4);
+  uint8_t* o = static_cast<uint8_t*>(blocks18);
+  for (int r = 0; r < rows; ++r)
+    for (int s = 0; s < nsb; ++s) {
+      const uint8_t* sb = in + sb_index(column_major, rows, nsb, r, s) * 144;
+      for (int b = 0; b < 8; ++b) {
+        uint8_t* blk = o + (size_t(r) * (K / 32) + size_t(s) * 8 + b) * 18;
+        std::memcpy(blk, sb + 128 + 2 * b, 2);
+        std::memcpy(blk + 2, sb + 16 * b, 16);
+      }
+    }
+  return Q4D_OK;
+}
+}  // namespace
+
+extern "C" {
+q4d_status q4d_pack_q4_0_weights(const void* blocks18, void* W_q4, int N, int K) {
+  return pack_impl(blocks18, W_q4, N, K, true);
+}
+q4d_status q4d_unpack_q4_0_weights(const void* W_q4, void* blocks18, int N, int K) {
+  return unpack_impl(W_q4, blocks18, N, K, true);
+}
+q4d_status q4d_pack_q4_0_rows(const void* blocks18, void* rows_q4, int rows, int K) {
+  return pack_impl(blocks18, rows_q4, rows, K, false);
+}
+q4d_status q4d_unpack_q4_0_rows(const void* rows_q4, void* blocks18, int rows, int K) {
+  return unpack_impl(rows_q4, blocks18, rows, K, false);
+}
+}  // extern "C"
+
+extern "C" {
 q4d_status q4d_device_error(int reset) {
   int dev = 0;
   DeviceState* s = nullptr;

@@ -29,6 +29,8 @@ EXPORTS = (
     "q4kv_attn_decode", "q4kv_attn_decode_ex", "q4d_attn_workspace_bytes",
     "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
     "q4kv_attn_decode_noalloc",
+    "q4d_pack_q4_0_weights", "q4d_unpack_q4_0_weights", "q4d_pack_q4_0_rows",
+    "q4d_unpack_q4_0_rows",
 )
 
 
@@ -83,6 +85,10 @@ def lib() -> ctypes.CDLL:
     L.q4d_plan_attn.argtypes = [i, i, i, i, i, i, ctypes.POINTER(AttnPlan)]
     L.q4d_device_error.argtypes = [i]
     L.q4kv_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
+    for fn in ("q4d_pack_q4_0_weights", "q4d_unpack_q4_0_weights", "q4d_pack_q4_0_rows",
+               "q4d_unpack_q4_0_rows"):
+        getattr(L, fn).argtypes = [vp, vp, i, i]
+        getattr(L, fn).restype = i
     for fn in ("q4_gemv", "q4_gemv_ex", "q4_gemv_ex2", "q4kv_attn_decode", "q4kv_attn_decode_ex",
                "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
                "q4kv_attn_decode_noalloc"):
@@ -108,6 +114,39 @@ def plan_attn(ctx_len: int, n_q_heads: int, n_kv_heads: int, head_dim: int, M: i
     _check(lib().q4d_plan_attn(ctx_len, n_q_heads, n_kv_heads, head_dim, M, num_sms,
                                ctypes.byref(p)), "q4d_plan_attn")
     return p
+
+
+def _host_convert(fn: str, src, rows: int, K: int, out_bytes: int, what: str):
+    import numpy as np
+
+    a = np.ascontiguousarray(src, dtype=np.uint8).reshape(-1)
+    out = np.empty(out_bytes, dtype=np.uint8)
+    if a.size < (rows * K // 32 * 18 if "unpack" not in fn else rows * K // 256 * 144):
+        raise ValueError(f"{what}: input buffer too small")
+    _check(getattr(lib(), fn)(a.ctypes.data, out.ctypes.data, rows, K), fn)
+    return out
+
+
+def pack_q4_0_weights(blocks18, N: int, K: int):
+    """Canonical 18-byte Q4_0 blocks, row-major [N][K/32] (host bytes) -> the
+    library's weight layout (host bytes, N*K/256*144)."""
+    return _host_convert("q4d_pack_q4_0_weights", blocks18, N, K, N * K // 256 * 144, "blocks18")
+
+
+def unpack_q4_0_weights(W_q4, N: int, K: int):
+    """Inverse of :func:`pack_q4_0_weights`."""
+    return _host_convert("q4d_unpack_q4_0_weights", W_q4, N, K, N * K // 32 * 18, "W_q4")
+
+
+def pack_q4_0_rows(blocks18, rows: int, K: int):
+    """Canonical 18-byte Q4_0 blocks [rows][K/32] -> super-blocks in row order
+    (the K/V cache layout)."""
+    return _host_convert("q4d_pack_q4_0_rows", blocks18, rows, K, rows * K // 256 * 144, "blocks18")
+
+
+def unpack_q4_0_rows(rows_q4, rows: int, K: int):
+    """Inverse of :func:`pack_q4_0_rows`."""
+    return _host_convert("q4d_unpack_q4_0_rows", rows_q4, rows, K, rows * K // 32 * 18, "rows_q4")
 
 
 def _torch():

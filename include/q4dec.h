@@ -220,6 +220,31 @@ q4d_status q4d_plan_gemv(int M, int N, int K, int num_sms, q4d_gemv_plan* plan);
 q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
                          int num_sms, q4d_attn_plan* plan);
 
+/* ------------------------------------------------ host layout helpers --
+ * Conversions between the canonical 18-byte Q4_0 block (GGUF order: fp16 d,
+ * little endian, then 16 bytes where byte j holds element j in its low nibble
+ * and element j + 16 in its high nibble) and this library's 144-byte
+ * super-block (the 8 blocks' 16 nibble bytes, then their 8 fp16 scales).
+ * The canonical input is row-major: rows of K/32 blocks.  Plain host code on
+ * host pointers, no CUDA; no counterpart on the source pages (format
+ * plumbing for data quantised elsewhere).
+ *
+ *   q4d_pack_q4_0_weights:   blocks18 [N][K/32] -> W_q4 in the weight layout
+ *                            (super-block (n, s) at byte (s*N + n) * 144).
+ *   q4d_unpack_q4_0_weights: the inverse.
+ *   q4d_pack_q4_0_rows:      blocks18 [rows][K/32] -> rows of super-blocks in
+ *                            row order (super-block (r, s) at (r*K/256 + s) * 144),
+ *                            the K/V cache layout (one row per token, K = 256).
+ *   q4d_unpack_q4_0_rows:    the inverse.
+ * Requirements: non-null pointers, rows (N) >= 1, K >= 256, K % 256 == 0; the
+ * buffers hold rows*K/32*18 and rows*K/256*144 bytes and do not overlap.
+ * Errors: Q4D_ERR_INVALID_ARG (null, rows < 1), Q4D_ERR_UNSUPPORTED_SHAPE (K).
+ */
+q4d_status q4d_pack_q4_0_weights(const void* blocks18, void* W_q4, int N, int K);
+q4d_status q4d_unpack_q4_0_weights(const void* W_q4, void* blocks18, int N, int K);
+q4d_status q4d_pack_q4_0_rows(const void* blocks18, void* rows_q4, int rows, int K);
+q4d_status q4d_unpack_q4_0_rows(const void* rows_q4, void* blocks18, int rows, int K);
+
 /* ------------------------------------------------------- device errors --
  * Synchronises the current device and reads the library's device error word
  * (set when an in-kernel wait exceeded its time limit).  Returns Q4D_OK when
