@@ -15,4 +15,6 @@ from .q4_oracle import (  # noqa: F401
     gemv_tolerance,
     attn_probs,
     attn_decode,
+    quantize_q4_0_rows,
+    kv_append,
 )

@@ -34,6 +34,13 @@ writes out the definitions the library implements:
   row ``m`` sits at position ``p_m = ctx_len - M + m`` and sees tokens
   ``t <= p_m``; ``s = scale * Q . K_hat``, ``P = softmax(s)``, ``out = P V_hat``.
 
+* K/V append: new K/V values (fp32) are quantised per 32-element block: amax =
+  the signed element of largest magnitude (first on ties), d = fp16(amax/-8),
+  q = clamp(floor(v/d + 8.5), 0, 15) with the division and the addition
+  rounded in fp32 (the precision the device decides the codes in); a block
+  whose d is zero stores d = +0 and q = 8.  The pages say only that the
+  cache is Q4 (the paragraph on the 16 full-attention layers).
+
 Readings taken where nothing fixes a detail: output is fp32 on the device
 (fp64 here); the softmax scale defaults to 1 (queries arrive pre-scaled);
 GQA groups are contiguous; non-finite inputs are out of scope.
@@ -175,3 +182,48 @@ def attn_decode(Q_bits, K_buf, V_buf, ctx_len: int, n_q_heads: int, n_kv_heads: 
         for h in range(n_q_heads):
             out[m, h] = P[m, h] @ Vh[h // g]
     return out
+
+
+def quantize_q4_0_rows(v) -> np.ndarray:
+    """Quantise fp32 rows ``v[rows][K]`` (K % 256 == 0) into super-blocks in
+    row order (the K/V layout), following the K/V append reading above: the
+    codes are decided in fp32 (numpy float32 division and addition, each
+    rounded to nearest), the scale is rounded to fp16."""
+    v = np.asarray(v, dtype=np.float32)
+    rows, K = v.shape
+    if K % SB_ELEMS:
+        raise ValueError("K must be a multiple of 256")
+    out = np.zeros((rows, K // SB_ELEMS, SB_BYTES), dtype=np.uint8)
+    for r in range(rows):
+        for blk in range(K // 32):
+            vals = v[r, 32 * blk: 32 * blk + 32]
+            i = int(np.argmax(np.abs(vals)))            # first index of the largest |v|
+            d16 = np.float16(vals[i] / np.float32(-8.0))
+            if d16 == 0:
+                d16 = np.float16(0.0)                   # +0, and every code 8
+                q = np.full(32, 8, dtype=np.int64)
+            else:
+                d32 = np.float32(d16)
+                q = np.floor(vals / d32 + np.float32(8.5)).astype(np.int64)
+                q = np.clip(q, 0, 15)
+            s_, b = divmod(blk, 8)
+            sb = out[r, s_]
+            sb[16 * b: 16 * b + 16] = (q[:16] | (q[16:] << 4)).astype(np.uint8)
+            sb[128 + 2 * b: 130 + 2 * b] = np.array([d16], dtype=np.float16).view(np.uint8)
+    return out.reshape(-1)
+
+
+def kv_append(K_buf, V_buf, k_new, v_new, n_kv_heads: int, kv_stride: int, pos: int, M: int):
+    """Caches after appending M tokens at positions pos .. pos+M-1 of every KV
+    head: token m of head h gets quantize_q4_0_rows(new[m][h]).  ``k_new`` /
+    ``v_new``: fp32 [M][n_kv_heads][256].  Returns new (K, V) byte arrays."""
+    outs = []
+    for buf, new in ((K_buf, k_new), (V_buf, v_new)):
+        b = np.array(buf, dtype=np.uint8).reshape(-1).copy()
+        new = np.asarray(new, dtype=np.float32).reshape(M, n_kv_heads, SB_ELEMS)
+        for m in range(M):
+            for h in range(n_kv_heads):
+                at = (h * kv_stride + pos + m) * SB_BYTES
+                b[at: at + SB_BYTES] = quantize_q4_0_rows(new[m, h][None, :])
+        outs.append(b)
+    return outs[0], outs[1]

@@ -418,3 +418,79 @@ def test_quantizer_recipe_on_literal_block():
     assert d[0, 0] == 0xB400                                    # fp16(-0.25)
     assert q[0, 31] == 0 and q[0, 0] == 12                      # 2/-0.25+8.5 -> 0; -1/-0.25+8.5 -> 12
     assert np.all(q[0, 32:] == 8) and np.all(d[0, 1:] == 0)
+
+
+# ---------------------------------------------------------------- K/V append
+def _one_block_row(vals):
+    """A 256-element row whose first block is ``vals`` and the rest zero."""
+    row = np.zeros((1, 256), dtype=np.float32)
+    row[0, :len(vals)] = vals
+    return row
+
+
+def test_quantizer_hand_worked_block():
+    # amax = -4 (largest |v|, negative) -> d = -4 / -8 = 0.5 (exact in fp16);
+    # q = floor(v / 0.5 + 8.5): -4 -> 0, -3.9 -> 0 (floor(0.7)), 0 -> 8,
+    # 0.25 -> 9, 3.5 -> 15, 3.74 -> 15 (floor(15.98)), 3.76 -> 16 -> clamp 15,
+    # -0.26 -> floor(7.98) = 7, 1.0 -> 10, -1.25 -> floor(6.0) = 6
+    vals = [-4.0, -3.9, 0.0, 0.25, 3.5, 3.74, 3.76, -0.26, 1.0, -1.25]
+    sb = oracle.quantize_q4_0_rows(_one_block_row(vals))
+    q = np.concatenate([sb[0:16] & 0x0F, sb[0:16] >> 4])
+    assert list(q[:10]) == [0, 0, 8, 9, 15, 15, 15, 7, 10, 6]
+    assert all(q[10:] == 8)                                 # zeros -> code 8
+    assert sb[128:130].view(np.float16)[0] == np.float16(0.5)
+    # blocks 1..7 are all-zero: d = +0 (bits 0x0000), every code 8
+    assert all(sb[16:128] == 0x88) and all(sb[130:144] == 0)
+
+
+def test_quantizer_positive_amax_flips_sign_and_maps_exactly():
+    # amax = +2 -> d = -0.25; the amax element itself maps to q = 0, i.e.
+    # -0.25 * (0 - 8) = 2 exactly; -2 maps to q = 16 -> 15 (one step short)
+    vals = [2.0, -2.0, 0.5, -0.5]
+    sb = oracle.quantize_q4_0_rows(_one_block_row(vals))
+    q = np.concatenate([sb[0:16] & 0x0F, sb[0:16] >> 4])
+    assert list(q[:4]) == [0, 15, 6, 10]
+    assert sb[128:130].view(np.float16)[0] == np.float16(-0.25)
+    w = oracle.dequant(sb, 1, 256)[0]
+    assert w[0] == 2.0 and w[1] == -1.75 and w[2] == 0.5 and w[3] == -0.5
+
+
+def test_quantizer_ties_take_the_first_index_and_zero_block_stores_plus_zero():
+    sb = oracle.quantize_q4_0_rows(_one_block_row([-3.0, 3.0]))
+    assert sb[128:130].view(np.float16)[0] == np.float16(0.375)   # from -3 (first)
+    z = oracle.quantize_q4_0_rows(np.zeros((1, 256), dtype=np.float32))
+    assert all(z[:128] == 0x88) and all(z[128:] == 0)
+    # -0.0 everywhere is an all-zero block too: d = +0, not -0
+    nz = oracle.quantize_q4_0_rows(np.full((1, 256), -0.0, dtype=np.float32))
+    assert all(nz[128:] == 0)
+
+
+def test_quantizer_error_bound_on_random_rows():
+    # |dequant(quant(v)) - v| <= |d| / 2, except the clamped top code (<= |d|)
+    rng = np.random.default_rng(9)
+    v = rng.standard_normal((6, 512)).astype(np.float32) * np.float32(3.0)
+    sb = oracle.quantize_q4_0_rows(v)
+    w = oracle.dequant(sb, 6, 512)
+    _, d = oracle.unpack_superblocks(sb, 6, 512)
+    dd = np.repeat(np.abs(d), 32, axis=1)
+    err = np.abs(w - v.astype(np.float64))
+    assert np.all(err <= dd * 1.0 + 1e-12)
+    assert np.mean(err <= dd * 0.5 + 1e-12) > 0.95
+
+
+def test_kv_append_writes_only_the_target_tokens():
+    n_kv, stride, pos, M = 2, 10, 3, 2
+    K0 = np.arange(n_kv * stride * 144, dtype=np.int64).astype(np.uint8)
+    V0 = K0[::-1].copy()
+    rng = np.random.default_rng(4)
+    kn = rng.standard_normal((M, n_kv, 256)).astype(np.float32)
+    vn = rng.standard_normal((M, n_kv, 256)).astype(np.float32)
+    K1, V1 = oracle.kv_append(K0, V0, kn, vn, n_kv, stride, pos, M)
+    for h in range(n_kv):
+        for t in range(stride):
+            at = slice((h * stride + t) * 144, (h * stride + t + 1) * 144)
+            if pos <= t < pos + M:
+                assert np.array_equal(K1[at], oracle.quantize_q4_0_rows(kn[t - pos, h][None]))
+                assert np.array_equal(V1[at], oracle.quantize_q4_0_rows(vn[t - pos, h][None]))
+            else:
+                assert np.array_equal(K1[at], K0[at]) and np.array_equal(V1[at], V0[at])
