@@ -201,8 +201,17 @@ def cpu_baseline(n_samples=3):
         b, t = oracle_sample_step(s)
         total_b += b
         total_t += t
-    return {"value": total_b / total_t / 1e12, "unit": "TB/s", "cores": cpu_cores(),
-            "kind": "oracle", "sample": f"{n_samples} samples; " + SAMPLE_DESC}
+    out = {"value": total_b / total_t / 1e12, "unit": "TB/s", "cores": cpu_cores(),
+           "kind": "oracle", "sample": f"{n_samples} samples; " + SAMPLE_DESC}
+    try:  # the same oracle on one thread
+        from threadpoolctl import threadpool_limits
+
+        with threadpool_limits(limits=1):
+            b, t = oracle_sample_step(n_samples)
+        out["single_thread"] = {"value": b / t / 1e12, "cores": 1, "sample": "1 sample"}
+    except Exception as e:  # noqa: BLE001
+        out["single_thread"] = {"error": str(e)[:200]}
+    return out
 
 
 def run_reference(args, rank, world):
@@ -325,8 +334,9 @@ def main():
     def gemv(W, x, y, N, K):
         # weights are immutable: each call may stream its first stages while
         # the kernel before it finishes (programmatic dependent launch)
-        st = L.q4_gemv_ex2(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, sptr,
-                           ws.data_ptr(), ws.numel(), q4dec.GEMV_WEIGHT_PREFETCH)
+        st = L.q4_gemv_ex2(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K,
+                           torch.cuda.current_stream().cuda_stream, ws.data_ptr(), ws.numel(),
+                           q4dec.GEMV_WEIGHT_PREFETCH)
         if st:
             raise RuntimeError(f"q4_gemv_ex2 failed: {st}")
         launches["n"] += 1 + (1 if L.q4d_gemv_workspace_bytes(M, N, K) else 0)
@@ -335,7 +345,8 @@ def main():
         Kc, Vc = kv[l]
         st = L.q4kv_attn_decode_ex(Qs[l].data_ptr(), Kc.data_ptr(), Vc.data_ptr(),
                                    outs[l].data_ptr(), CTX, N_Q, N_KV, HEAD_DIM, M, CTX,
-                                   1.0, sptr, ws.data_ptr(), ws.numel())
+                                   1.0, torch.cuda.current_stream().cuda_stream,
+                                   ws.data_ptr(), ws.numel())
         if st:
             raise RuntimeError(f"q4kv_attn_decode_ex failed: {st}")
         launches["n"] += 2 if aws else 1
@@ -402,6 +413,53 @@ def main():
     per_launch_s = gemv_ms * 1e-3 / (K_ * n_gemv)
     achieved_gbs = per_launch_bytes / per_launch_s / 1e9
     attn_gbs = ATTN_LAYERS * attn_alg_bytes(M, CTX) * K_ / (attn_ms * 1e-3) / 1e9
+
+    # -------- the same step replayed as one CUDA graph (353 kernel nodes; the
+    # weight-prefetching GEMVs keep their programmatic dependencies)
+    graph = None
+    g = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        s_cap = torch.cuda.Stream()
+        s_cap.wait_stream(stream)
+        with torch.cuda.stream(s_cap):
+            gemv_stream()
+            attn_stream()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s_cap):
+            gemv_stream()
+            attn_stream()
+        torch.cuda.synchronize()
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        graph_err = None
+    except Exception as e:  # noqa: BLE001 - report, keep the eager numbers
+        graph_err = f"{type(e).__name__}: {e}"[:300]
+        torch.cuda.synchronize()
+    ok = torch.tensor([0.0 if graph_err else 1.0], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ok, op=dist.ReduceOp.MIN)
+    if ok.item() == 1.0:
+        barrier()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(K_):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        gms = torch.tensor([g0.elapsed_time(g1) / K_], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(gms, op=dist.ReduceOp.MAX)
+        graph = {"ms_per_step": gms.item(),
+                 "value": bytes_step * world / (gms.item() * 1e-3) / 1e12,
+                 "unit": "TB/s", "replays": K_}
+    else:
+        graph = {"error": graph_err or "capture failed on another rank"}
+    del g
+    torch.cuda.synchronize()
 
     # -------- end to end through the public API with host buffers
     import torch as _t
@@ -487,6 +545,7 @@ def main():
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": timed_launches,
         "clocks": clock,
+        "graph": graph,
         "per_call": per_call,
         "setup_s": gen_s,
     }
@@ -552,6 +611,32 @@ def per_call_table(torch, L, dev, layers, kv, ws, peak_gbs, reps=15):
             gbs = attn_alg_bytes(M, ctx) / (us * 1e-6) / 1e9
             table["attn"].append({"ctx": ctx, "M": M, "us": us, "GBps": gbs,
                                   "frac": gbs / peak_gbs})
+    # t(M=5) / t(M=1) per GEMV shape: about 1 is what makes verification cheap
+    by = {(r["shape"], r["M"]): r["us"] for r in table["gemv"]}
+    table["gemv_m5_over_m1"] = {name: by[(name, 5)] / by[(name, 1)] for name in names.values()}
+    # K/V append of M verified tokens (4 KV heads), a small cache of its own
+    stride = 4096
+    Kc = torch.zeros(N_KV * stride * 144, dtype=torch.uint8, device=dev)
+    Vc = torch.zeros_like(Kc)
+    table["kv_append"] = []
+    for M in (1, 5):
+        kn = torch.randn((M, N_KV, HEAD_DIM), device=dev)
+        vn = torch.randn((M, N_KV, HEAD_DIM), device=dev)
+        times = []
+        for r in range(reps + 2):
+            flush.fill_(r & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            st = L.q4kv_append(Kc.data_ptr(), Vc.data_ptr(), kn.data_ptr(), vn.data_ptr(), N_KV,
+                               stride, stride - M, M, sptr)
+            b.record(stream)
+            if st:
+                raise RuntimeError(f"q4kv_append failed: {st}")
+            torch.cuda.synchronize()
+            if r >= 2:
+                times.append(a.elapsed_time(b) * 1e3)
+        table["kv_append"].append({"M": M, "n_kv_heads": N_KV, "us": statistics.median(times),
+                                   "bytes_written": 2 * M * N_KV * 144})
     del flush
     return table
 

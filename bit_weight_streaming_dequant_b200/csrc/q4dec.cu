@@ -16,6 +16,7 @@
 
 #include "q4_gemv.cuh"
 #include "q4kv_attn.cuh"
+#include "q4kv_append.cuh"
 
 // Device error word (bit q4d::kDevErrWaitTimeout: a bounded wait ran out).
 __device__ unsigned q4d_error_word;
@@ -503,6 +504,33 @@ q4d_status q4kv_attn_decode_ex(const void* Q, const void* Kq4, const void* Vq4, 
 }
 
 }  // extern "C"
+
+// ---- K/V append
+extern "C" q4d_status q4kv_append(void* Kq4, void* Vq4, const float* k_new, const float* v_new,
+                                  int n_kv_heads, int kv_stride_tokens, int pos, int M,
+                                  void* stream) {
+  if (!Kq4 || !Vq4 || !k_new || !v_new || n_kv_heads < 1 || M < 1 || pos < 0 ||
+      kv_stride_tokens < 1)
+    return Q4D_ERR_INVALID_ARG;
+  if ((long long)pos + M > kv_stride_tokens) return Q4D_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(Kq4, 16) || !aligned(Vq4, 16) || !aligned(k_new, 4) || !aligned(v_new, 4))
+    return Q4D_ERR_MISALIGNED;
+  int dev = 0;
+  DeviceState* s = nullptr;
+  q4d_status st = current_device(&dev, &s);
+  if (st != Q4D_OK) return st;
+  q4d::AppendArgs a;
+  a.K = static_cast<uint8_t*>(Kq4);
+  a.V = static_cast<uint8_t*>(Vq4);
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.n_kv = n_kv_heads;
+  a.kv_stride = kv_stride_tokens;
+  a.pos = pos;
+  a.M = M;
+  q4d::q4kv_append_kernel<<<dim3(M * n_kv_heads, 2), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return cudaGetLastError() == cudaSuccess ? Q4D_OK : Q4D_ERR_CUDA;
+}
 
 // ---- host layout helpers: canonical 18-byte blocks <-> 144-byte super-blocks
 namespace {

@@ -30,7 +30,7 @@ EXPORTS = (
     "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
     "q4kv_attn_decode_noalloc",
     "q4d_pack_q4_0_weights", "q4d_unpack_q4_0_weights", "q4d_pack_q4_0_rows",
-    "q4d_unpack_q4_0_rows",
+    "q4d_unpack_q4_0_rows", "q4kv_append",
 )
 
 
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
                "q4d_unpack_q4_0_rows"):
         getattr(L, fn).argtypes = [vp, vp, i, i]
         getattr(L, fn).restype = i
+    L.q4kv_append.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
+    L.q4kv_append.restype = i
     for fn in ("q4_gemv", "q4_gemv_ex", "q4_gemv_ex2", "q4kv_attn_decode", "q4kv_attn_decode_ex",
                "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
                "q4kv_attn_decode_noalloc"):
@@ -216,6 +218,26 @@ def q4_gemv(W, x, y=None, *, N: int, K: int, stream=None, workspace=None,
                                GEMV_WEIGHT_PREFETCH if weight_prefetch else 0)
     _check(st, "q4_gemv")
     return y
+
+
+def q4kv_append(Kq4, Vq4, k_new, v_new, *, pos: int, kv_stride_tokens: int, stream=None):
+    """Quantise the fp32 K/V rows ``k_new`` / ``v_new`` [M][n_kv_heads][256] into
+    the Q4_0 caches at token positions pos .. pos+M-1 (``q4kv_append``)."""
+    torch = _torch()
+    _dev_tensor(Kq4, torch.uint8, "Kq4")
+    _dev_tensor(Vq4, torch.uint8, "Vq4")
+    _dev_tensor(k_new, torch.float32, "k_new")
+    _dev_tensor(v_new, torch.float32, "v_new")
+    if k_new.dim() != 3 or k_new.shape[2] != 256 or tuple(v_new.shape) != tuple(k_new.shape):
+        raise ValueError("k_new / v_new must be [M][n_kv_heads][256]")
+    M, n_kv = k_new.shape[0], k_new.shape[1]
+    need = n_kv * kv_stride_tokens * 144
+    if Kq4.numel() < need or Vq4.numel() < need:
+        raise ValueError("caches are smaller than n_kv_heads * kv_stride_tokens rows")
+    with torch.cuda.device(k_new.device):
+        st = lib().q4kv_append(Kq4.data_ptr(), Vq4.data_ptr(), k_new.data_ptr(), v_new.data_ptr(),
+                               n_kv, kv_stride_tokens, pos, M, _stream_ptr(stream))
+    _check(st, "q4kv_append")
 
 
 def q4kv_attn_decode(Q, Kq4, Vq4, out=None, *, ctx_len: int, n_kv_heads: int,

@@ -220,6 +220,28 @@ q4d_status q4d_plan_gemv(int M, int N, int K, int num_sms, q4d_gemv_plan* plan);
 q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
                          int num_sms, q4d_attn_plan* plan);
 
+/* ------------------------------------------------------- K/V append --
+ * Quantise the K and V rows of M new tokens and write them at token positions
+ * pos .. pos+M-1 of every KV head of the Q4_0 caches ("Qwen3.8-27B at 256K on
+ * a 24GB RTX PRO 4000 SFF (432 GB/s): 50 tok/s with MTP", paragraph on the
+ * 16 full-attention layers: the K/V cache is Q4 and grows by the verified
+ * tokens).  Per 32-element block: amax = the element of largest magnitude
+ * (first on ties), d = fp16(amax / -8), q = clamp(floor(v/d + 8.5), 0, 15)
+ * with the division and addition rounded to nearest in fp32; a zero d is
+ * stored as +0 with every q = 8.
+ *
+ *   Kq4, Vq4     : caches, [n_kv_heads][kv_stride_tokens] super-blocks (head_dim 256).
+ *   k_new, v_new : fp32 [M][n_kv_heads][256], device pointers.
+ *   Requirements: n_kv_heads >= 1, M >= 1, pos >= 0, pos + M <= kv_stride_tokens;
+ *   caches 16-byte and k_new / v_new 4-byte aligned.  Runs on `stream`
+ *   (NULL = legacy default stream); allocates nothing; only the M target
+ *   tokens' super-blocks are written.
+ *   Errors: Q4D_ERR_INVALID_ARG, Q4D_ERR_UNSUPPORTED_SHAPE (pos + M beyond
+ *   the stride), Q4D_ERR_MISALIGNED, Q4D_ERR_CUDA; nothing is launched on error.
+ */
+q4d_status q4kv_append(void* Kq4, void* Vq4, const float* k_new, const float* v_new,
+                       int n_kv_heads, int kv_stride_tokens, int pos, int M, void* stream);
+
 /* ------------------------------------------------ host layout helpers --
  * Conversions between the canonical 18-byte Q4_0 block (GGUF order: fp16 d,
  * little endian, then 16 bytes where byte j holds element j in its low nibble

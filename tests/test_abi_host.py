@@ -118,3 +118,14 @@ def test_workspace_queries_without_device_use_the_fallback_plan():
     # layer shapes need no split-K workspace; the long context needs merge space
     assert L.q4d_gemv_workspace_bytes(1, 17408, 5120) == 0
     assert L.q4d_attn_workspace_bytes(262144, 24, 4, 256, 5) > 0
+
+
+def test_append_rejects_bad_arguments_without_cuda():
+    L = q4dec.lib()
+    assert L.q4kv_append(None, FAKE, FAKE, FAKE, 4, 64, 0, 1, None) == 1
+    assert L.q4kv_append(FAKE, FAKE, FAKE, FAKE, 0, 64, 0, 1, None) == 1
+    assert L.q4kv_append(FAKE, FAKE, FAKE, FAKE, 4, 64, -1, 1, None) == 1
+    assert L.q4kv_append(FAKE, FAKE, FAKE, FAKE, 4, 64, 0, 0, None) == 1
+    assert L.q4kv_append(FAKE, FAKE, FAKE, FAKE, 4, 64, 60, 5, None) == 2
+    assert L.q4kv_append(FAKE + 8, FAKE, FAKE, FAKE, 4, 64, 0, 1, None) == 3
+    assert L.q4kv_append(FAKE, FAKE, FAKE + 2, FAKE, 4, 64, 0, 1, None) == 3
