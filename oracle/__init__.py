@@ -16,5 +16,7 @@ from .q4_oracle import (  # noqa: F401
     attn_probs,
     attn_decode,
     quantize_q4_0_rows,
+    silu,
+    gemv_swiglu,
     kv_append,
 )

@@ -34,6 +34,10 @@ writes out the definitions the library implements:
   row ``m`` sits at position ``p_m = ctx_len - M + m`` and sees tokens
   ``t <= p_m``; ``s = scale * Q . K_hat``, ``P = softmax(s)``, ``out = P V_hat``.
 
+* fused gate/up GEMV with a SwiGLU epilogue (the feed-forward block the page
+  on the 64-layer model describes as gate, up and down projections): the
+  weight matrix holds 2N rows, gate row n at 2n and up row n at 2n + 1;
+  ``h[m, n] = silu(g) * u`` with ``silu(g) = g / (1 + exp(-g))``.
 * K/V append: new K/V values (fp32) are quantised per 32-element block: amax =
   the signed element of largest magnitude (first on ties), d = fp16(amax/-8),
   q = clamp(floor(v/d + 8.5), 0, 15) with the division and the addition
@@ -227,3 +231,31 @@ def kv_append(K_buf, V_buf, k_new, v_new, n_kv_heads: int, kv_stride: int, pos: 
                 b[at: at + SB_BYTES] = quantize_q4_0_rows(new[m, h][None, :])
         outs.append(b)
     return outs[0], outs[1]
+
+
+def silu(g):
+    """``g / (1 + exp(-g))`` in fp64 (written so that it does not overflow)."""
+    g = np.asarray(g, dtype=np.float64)
+    out = np.empty_like(g)
+    pos = g >= 0
+    out[pos] = g[pos] / (1.0 + np.exp(-g[pos]))
+    e = np.exp(g[~pos])
+    out[~pos] = g[~pos] * e / (1.0 + e)
+    return out
+
+
+def gemv_swiglu(W_buf, x_bits, M: int, N: int, K: int):
+    """Fused gate/up GEMV + SwiGLU: ``W_buf`` holds 2N rows in the weight
+    layout (gate row n at 2n, up row n at 2n + 1).  Returns ``(h, tol)``:
+    ``h[m, n] = silu(g) * u`` in fp64 and the per-element bound the device
+    result must meet, propagated from the GEMV bound ``t = 2e-3 S + 1e-5`` of
+    g and u through the product: ``|silu'(g) u| t_g + |silu(g)| t_u + c t_g t_u``
+    with ``c = max |silu''| <= 0.5``, plus 1e-6 relative for the fp32 epilogue."""
+    y, S = gemv(W_buf, x_bits, M, 2 * N, K)
+    g, u = y[:, 0::2], y[:, 1::2]
+    tg, tu = gemv_tolerance(S[:, 0::2]), gemv_tolerance(S[:, 1::2])
+    sg = 1.0 / (1.0 + np.exp(-np.clip(g, -700, 700)))
+    dsilu = sg * (1.0 + g * (1.0 - sg))
+    h = silu(g) * u
+    tol = np.abs(dsilu * u) * tg + np.abs(silu(g)) * tu + 0.5 * tg * tu + 1e-6 * np.abs(h)
+    return h, tol

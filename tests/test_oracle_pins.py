@@ -494,3 +494,51 @@ def test_kv_append_writes_only_the_target_tokens():
                 assert np.array_equal(V1[at], oracle.quantize_q4_0_rows(vn[t - pos, h][None]))
             else:
                 assert np.array_equal(K1[at], K0[at]) and np.array_equal(V1[at], V0[at])
+
+
+# ------------------------------------------------------- gate/up + SwiGLU
+def test_silu_closed_forms():
+    g = np.array([0.0, 1.0, -1.0, 40.0, -40.0, 800.0, -800.0])
+    s = oracle.silu(g)
+    assert s[0] == 0.0
+    assert abs(s[1] - 1.0 / (1.0 + math.exp(-1.0))) < 1e-15
+    assert abs(s[2] - (-1.0) / (1.0 + math.exp(1.0))) < 1e-15
+    assert abs(s[3] - 40.0) < 1e-12 and abs(s[4]) < 1e-15
+    assert s[5] == 800.0
+    assert abs(s[6]) < 1e-300
+
+
+def test_gemv_swiglu_composes_two_plain_gemvs():
+    # interleaving gate and up rows and fusing must equal silu(gate GEMV) * up GEMV
+    N, K, M = 6, 512, 2
+    Wg = synth.q4_0_weights(31, N, K)
+    Wu = synth.q4_0_weights(32, N, K)
+    x = synth.activations(33, M, K)
+    rows_g = oracle.weight_rows(Wg, N, K).reshape(N, -1)
+    rows_u = oracle.weight_rows(Wu, N, K).reshape(N, -1)
+    inter = np.empty((2 * N, rows_g.shape[1]), dtype=np.uint8)
+    inter[0::2], inter[1::2] = rows_g, rows_u
+    Wgu = synth.column_major(inter.reshape(-1), 2 * N, K)
+    h, tol = oracle.gemv_swiglu(Wgu, x, M, N, K)
+    g, _ = oracle.gemv(Wg, x, M, N, K)
+    u, _ = oracle.gemv(Wu, x, M, N, K)
+    np.testing.assert_allclose(h, oracle.silu(g) * u, rtol=0, atol=1e-12)
+    assert np.all(tol > 0)
+
+
+def test_gemv_swiglu_hand_worked():
+    # K = 256, one row pair: gate weights all d * (q - 8) = 0.5 * 1 on element 0
+    # only (others q = 8), up weights 0.25 * (-2) on element 1 only; x[0] = 2,
+    # x[1] = 3: g = 1.0, u = -1.5, h = silu(1) * -1.5
+    q = np.full((2, 256), 8, dtype=np.uint8)
+    q[0, 0] = 9
+    q[1, 1] = 6
+    d = np.zeros((2, 8), dtype=np.float32)
+    d[0, 0] = 0.5
+    d[1, 0] = 0.25
+    W = synth.weights_from_parts(q, d)
+    x = np.zeros((1, 256), dtype=np.float32)
+    x[0, 0], x[0, 1] = 2.0, 3.0
+    xb = synth.f32_to_bf16_bits(x)
+    h, _ = oracle.gemv_swiglu(W, xb, 1, 1, 256)
+    assert abs(h[0, 0] - (1.0 / (1.0 + math.exp(-1.0))) * -1.5) < 1e-15
