@@ -614,6 +614,32 @@ def per_call_table(torch, L, dev, layers, kv, ws, peak_gbs, reps=15):
     # t(M=5) / t(M=1) per GEMV shape: about 1 is what makes verification cheap
     by = {(r["shape"], r["M"]): r["us"] for r in table["gemv"]}
     table["gemv_m5_over_m1"] = {name: by[(name, 5)] / by[(name, 1)] for name in names.values()}
+    # fused gate / up + SwiGLU (one 2 x 17408 x 5120 interleaved matrix) vs the
+    # two separate 5120 -> 17408 GEMVs of the table above
+    import synth
+    Wgu = [synth.device_q4_0_weights(7000 + i, 2 * FFN, HIDDEN, device=dev) for i in range(2)]
+    table["gate_up_swiglu"] = []
+    for M in (1, 5):
+        x = torch.randn((M, HIDDEN), device=dev).to(torch.bfloat16)
+        h = torch.empty((M, FFN), dtype=torch.float32, device=dev)
+        times = []
+        for r in range(reps + 2):
+            flush.fill_(r & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            st = L.q4_gemv_swiglu_ex(Wgu[r % 2].data_ptr(), x.data_ptr(), h.data_ptr(), M, FFN,
+                                     HIDDEN, sptr, ws.data_ptr(), ws.numel(), 0)
+            b.record(stream)
+            if st:
+                raise RuntimeError(f"q4_gemv_swiglu_ex failed: {st}")
+            torch.cuda.synchronize()
+            if r >= 2:
+                times.append(a.elapsed_time(b) * 1e3)
+        us = statistics.median(times)
+        gbs = (2 * q4_bytes(FFN, HIDDEN) + 2 * M * HIDDEN + 4 * M * FFN) / (us * 1e-6) / 1e9
+        table["gate_up_swiglu"].append({"M": M, "us": us, "GBps": gbs, "frac": gbs / peak_gbs,
+                                        "separate_gate_plus_up_us": 2 * by[("5120->17408", M)]})
+    del Wgu
     # K/V append of M verified tokens (4 KV heads), a small cache of its own
     stride = 4096
     Kc = torch.zeros(N_KV * stride * 144, dtype=torch.uint8, device=dev)

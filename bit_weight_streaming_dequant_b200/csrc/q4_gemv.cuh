@@ -187,7 +187,9 @@ __device__ __forceinline__ void gemv_pass(const PassCtx& c, int& slot, uint32_t&
 // Warps 0..7 consume: warp w takes block w of every super-block column and
 // every m-tile of the pass.  Warp 8 produces: it refills a stage as soon as
 // all eight consumers have released it.
-template <int M, int KC>
+// SWIGLU: the matrix holds gate / up row pairs (rows 2n, 2n + 1); CTAs own
+// whole pairs and, without a K split, store h = silu(gate) * up per pair.
+template <int M, int KC, bool SWIGLU>
 __global__ void __launch_bounds__(kGemvThreads, 1)
     q4_gemv_kernel(const __grid_constant__ GemvArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -195,8 +197,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   const int ks = blockIdx.y;
   const int S = a.stages;
 
-  const int row_begin = int((long long)a.N * blockIdx.x / a.grid_rows);
-  const int row_end = int((long long)a.N * (blockIdx.x + 1) / a.grid_rows);
+  const int unit = SWIGLU ? 2 : 1;  // rows per partition unit
+  const int units = a.N / unit;
+  const int row_begin = unit * int((long long)units * blockIdx.x / a.grid_rows);
+  const int row_end = unit * int((long long)units * (blockIdx.x + 1) / a.grid_rows);
   const int n_rows = row_end - row_begin;
   const int R = a.rows_per_pass;
   const int n_passes = (n_rows + R - 1) / R;
@@ -330,8 +334,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     // out[m][row] = sum over the 8 warps; element (row r, column m) sits in
     // lane (r % 8) * 4 + m / 2 of tile r / 16, component (r >= 8 ? 2 : 0) + m % 2
     const int r0 = row_begin + pass * R;
-    for (int i = tid; i < nr * M; i += kConsumerWarps * 32) {
-      const int r = i / M, m = i - (i / M) * M;
+    auto row_sum = [&](int r, int m) {
       const int p = r >> 4, rr = r & 15;
       const int ln = (rr & 7) * 4 + (m >> 1);
       const int comp = (rr >= 8 ? 2 : 0) + (m & 1);
@@ -341,9 +344,40 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
         const float4 v = red[(w * kMmaMaxTiles + p) * 32 + ln];
         s += comp == 0 ? v.x : comp == 1 ? v.y : comp == 2 ? v.z : v.w;
       }
-      a.out[(size_t(ks) * M + m) * a.N + r0 + r] = s;
+      return s;
+    };
+    if (SWIGLU && gridDim.y == 1) {
+      // h[m][n] = silu(g) * u for the pairs of this pass (passes hold whole pairs)
+      for (int i = tid; i < (nr >> 1) * M; i += kConsumerWarps * 32) {
+        const int j = i / M, m = i - (i / M) * M;
+        const float g = row_sum(2 * j, m), u = row_sum(2 * j + 1, m);
+        a.out[size_t(m) * (a.N >> 1) + ((r0 >> 1) + j)] = g / (1.f + __expf(-g)) * u;
+      }
+    } else {
+      for (int i = tid; i < nr * M; i += kConsumerWarps * 32) {
+        const int r = i / M, m = i - (i / M) * M;
+        a.out[(size_t(ks) * M + m) * a.N + r0 + r] = row_sum(r, m);
+      }
     }
     consumer_sync();  // red is rewritten at the next pass end
+  }
+}
+
+// h[m][n] = silu(g) * u from the partials of the 2N gate / up rows, each
+// summed over the K ranges in range order.
+__global__ void q4_gemv_splitk_reduce_swiglu(const float* __restrict__ ws, float* __restrict__ h,
+                                             int M, int N, int k_splits) {
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  const long long mn = (long long)M * N, rows = 2LL * N;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < mn;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long m = i / N, n = i - m * N;
+    float g = 0.f, u = 0.f;
+    for (int k = 0; k < k_splits; ++k) {
+      g += ws[(k * M + m) * rows + 2 * n];
+      u += ws[(k * M + m) * rows + 2 * n + 1];
+    }
+    h[i] = g / (1.f + __expf(-g)) * u;
   }
 }
 

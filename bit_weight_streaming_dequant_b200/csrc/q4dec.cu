@@ -180,11 +180,64 @@ q4d_status check_attn_shape(int ctx_len, int n_q, int n_kv, int head_dim, int M,
   return Q4D_OK;
 }
 
-template <int M, int KC>
+// Plan for `rows` weight rows shared out in units of `unit` rows (2 for the
+// gate / up pairs of the SwiGLU variant).
+q4d_status plan_gemv_rows(int M, int rows, int K, int num_sms, int unit, q4d_gemv_plan* plan) {
+  if (!plan || num_sms < 1) return Q4D_ERR_INVALID_ARG;
+  q4d_status st = check_gemv_shape(M, rows, K);
+  if (st != Q4D_OK) return st;
+  const int N = rows, units = rows / unit;
+  const int nsb = K / 256;
+  // Rows are shared out exactly (+-1) over up to one CTA per SM, at least 8
+  // rows each.  When that leaves most SMs idle, K is cut into equal ranges
+  // (a divisor of the super-block count, two or more super-blocks each).
+  int grid_rows = std::min(num_sms, std::max(1, std::min(units, N / 8)));
+  int ks = 1;
+  if (2 * grid_rows < num_sms) {
+    const int want = num_sms / grid_rows;
+    for (int d = std::min(want, nsb / 2); d >= 2; --d)
+      if (nsb % d == 0) {
+        ks = d;
+        break;
+      }
+  }
+  const int sbs = nsb / ks;
+  const int rows_per_cta = unit * ceil_div(units, grid_rows);
+  const int tiles = std::min(q4d::kMmaMaxTiles, ceil_div(rows_per_cta, 16));
+  const int rows_per_pass = 16 * tiles;
+  // Super-block columns per stage: the fewest of 1, 2, 4 (dividing the K
+  // range) that give at least 24 KB of weights per stage (fewer, larger
+  // stages amortise the per-stage handshakes); then as many stages as fit,
+  // up to 16.
+  int KC = 1;
+  for (int c : {1, 2, 4}) {
+    if (sbs % c) continue;
+    KC = c;
+    if (size_t(c) * rows_per_pass * 144 >= 24 * 1024) break;
+  }
+  const size_t red = size_t(q4d::kConsumerWarps) * q4d::kMmaMaxTiles * 32 * 16;
+  const size_t stage = q4d::gemv_stage_bytes(M, KC, rows_per_pass);
+  int stages = int((kGemvSmemBudget - red) / (stage + 16));
+  stages = std::max(2, std::min(q4d::kMmaMaxStages, stages));
+  plan->k_splits = ks;
+  plan->sb_per_split = sbs;
+  plan->chunk_sb = KC;
+  plan->rows_per_cta = rows_per_cta;
+  plan->rows_per_pass = rows_per_pass;
+  plan->stages = stages;
+  plan->threads = q4d::kGemvThreads;
+  plan->grid_rows = grid_rows;
+  plan->smem_bytes = stages * stage + red + size_t(stages) * 16;
+  plan->workspace_bytes = ks > 1 ? size_t(ks) * M * N * 4 : 0;
+  return Q4D_OK;
+}
+
+
+template <int M, int KC, bool SWIGLU>
 q4d_status launch_gemv_t(const q4d::GemvArgs& a, const q4d_gemv_plan& p, int dev,
                          const DeviceState& s, cudaStream_t stream, bool pdl) {
   static std::atomic<bool> smem_set[kMaxDevices];
-  auto kernel = q4d::q4_gemv_kernel<M, KC>;
+  auto kernel = q4d::q4_gemv_kernel<M, KC, SWIGLU>;
   q4d_status st = allow_smem(kernel, dev, s, smem_set);
   if (st != Q4D_OK) return st;
   dim3 grid(p.grid_rows, p.k_splits);
@@ -205,10 +258,13 @@ q4d_status launch_gemv_t(const q4d::GemvArgs& a, const q4d_gemv_plan& p, int dev
   return cudaLaunchKernelEx(&cfg, kernel, a) == cudaSuccess ? Q4D_OK : Q4D_ERR_CUDA;
 }
 
+// y = W x (rows = N), or with `swiglu` h[m][n] = silu(g) * u over the N gate /
+// up row pairs of W (2N rows).
 q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, int K,
                      cudaStream_t stream, void* workspace, size_t workspace_bytes,
-                     bool library_ws, bool pdl = false) {
-  q4d_status st = check_gemv_shape(M, N, K);
+                     bool library_ws, bool pdl = false, bool swiglu = false) {
+  if (swiglu && N > (1 << 29)) return Q4D_ERR_UNSUPPORTED_SHAPE;
+  q4d_status st = check_gemv_shape(M, swiglu ? 2 * N : N, K);
   if (st != Q4D_OK) return st;
   if (!W_q4 || !x || !y) return Q4D_ERR_INVALID_ARG;
   if (!aligned(W_q4, 16) || !aligned(x, 16) || !aligned(y, 4)) return Q4D_ERR_MISALIGNED;
@@ -217,8 +273,9 @@ q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, in
   int dev = 0;
   DeviceState* s = nullptr;
   if ((st = current_device(&dev, &s)) != Q4D_OK) return st;
+  const int rows = swiglu ? 2 * N : N;
   q4d_gemv_plan p;
-  if ((st = q4d_plan_gemv(M, N, K, s->num_sms, &p)) != Q4D_OK) return st;
+  if ((st = plan_gemv_rows(M, rows, K, s->num_sms, swiglu ? 2 : 1, &p)) != Q4D_OK) return st;
   if (p.smem_bytes > size_t(s->smem_optin)) return Q4D_ERR_UNSUPPORTED_SHAPE;
   if (library_ws) {
     if ((st = library_workspace(*s, p.workspace_bytes, &workspace)) != Q4D_OK) return st;
@@ -234,35 +291,39 @@ q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, in
   a.W = static_cast<const uint8_t*>(W_q4);
   a.out = p.k_splits > 1 ? static_cast<float*>(workspace) : y;
   a.err = s->err;
-  a.N = N;
+  a.N = rows;
   a.sb_per_split = p.sb_per_split;
   a.rows_per_pass = p.rows_per_pass;
   a.grid_rows = p.grid_rows;
   a.stages = p.stages;
 
   switch (M * 8 + p.chunk_sb) {
-    case 1 * 8 + 1: st = launch_gemv_t<1, 1>(a, p, dev, *s, stream, pdl); break;
-    case 1 * 8 + 2: st = launch_gemv_t<1, 2>(a, p, dev, *s, stream, pdl); break;
-    case 1 * 8 + 4: st = launch_gemv_t<1, 4>(a, p, dev, *s, stream, pdl); break;
-    case 2 * 8 + 1: st = launch_gemv_t<2, 1>(a, p, dev, *s, stream, pdl); break;
-    case 2 * 8 + 2: st = launch_gemv_t<2, 2>(a, p, dev, *s, stream, pdl); break;
-    case 2 * 8 + 4: st = launch_gemv_t<2, 4>(a, p, dev, *s, stream, pdl); break;
-    case 3 * 8 + 1: st = launch_gemv_t<3, 1>(a, p, dev, *s, stream, pdl); break;
-    case 3 * 8 + 2: st = launch_gemv_t<3, 2>(a, p, dev, *s, stream, pdl); break;
-    case 3 * 8 + 4: st = launch_gemv_t<3, 4>(a, p, dev, *s, stream, pdl); break;
-    case 4 * 8 + 1: st = launch_gemv_t<4, 1>(a, p, dev, *s, stream, pdl); break;
-    case 4 * 8 + 2: st = launch_gemv_t<4, 2>(a, p, dev, *s, stream, pdl); break;
-    case 4 * 8 + 4: st = launch_gemv_t<4, 4>(a, p, dev, *s, stream, pdl); break;
-    case 5 * 8 + 1: st = launch_gemv_t<5, 1>(a, p, dev, *s, stream, pdl); break;
-    case 5 * 8 + 2: st = launch_gemv_t<5, 2>(a, p, dev, *s, stream, pdl); break;
-    default: st = launch_gemv_t<5, 4>(a, p, dev, *s, stream, pdl); break;
+    case 1 * 8 + 1: st = (swiglu ? launch_gemv_t<1, 1, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<1, 1, false>(a, p, dev, *s, stream, pdl)); break;
+    case 1 * 8 + 2: st = (swiglu ? launch_gemv_t<1, 2, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<1, 2, false>(a, p, dev, *s, stream, pdl)); break;
+    case 1 * 8 + 4: st = (swiglu ? launch_gemv_t<1, 4, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<1, 4, false>(a, p, dev, *s, stream, pdl)); break;
+    case 2 * 8 + 1: st = (swiglu ? launch_gemv_t<2, 1, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<2, 1, false>(a, p, dev, *s, stream, pdl)); break;
+    case 2 * 8 + 2: st = (swiglu ? launch_gemv_t<2, 2, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<2, 2, false>(a, p, dev, *s, stream, pdl)); break;
+    case 2 * 8 + 4: st = (swiglu ? launch_gemv_t<2, 4, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<2, 4, false>(a, p, dev, *s, stream, pdl)); break;
+    case 3 * 8 + 1: st = (swiglu ? launch_gemv_t<3, 1, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<3, 1, false>(a, p, dev, *s, stream, pdl)); break;
+    case 3 * 8 + 2: st = (swiglu ? launch_gemv_t<3, 2, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<3, 2, false>(a, p, dev, *s, stream, pdl)); break;
+    case 3 * 8 + 4: st = (swiglu ? launch_gemv_t<3, 4, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<3, 4, false>(a, p, dev, *s, stream, pdl)); break;
+    case 4 * 8 + 1: st = (swiglu ? launch_gemv_t<4, 1, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<4, 1, false>(a, p, dev, *s, stream, pdl)); break;
+    case 4 * 8 + 2: st = (swiglu ? launch_gemv_t<4, 2, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<4, 2, false>(a, p, dev, *s, stream, pdl)); break;
+    case 4 * 8 + 4: st = (swiglu ? launch_gemv_t<4, 4, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<4, 4, false>(a, p, dev, *s, stream, pdl)); break;
+    case 5 * 8 + 1: st = (swiglu ? launch_gemv_t<5, 1, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<5, 1, false>(a, p, dev, *s, stream, pdl)); break;
+    case 5 * 8 + 2: st = (swiglu ? launch_gemv_t<5, 2, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<5, 2, false>(a, p, dev, *s, stream, pdl)); break;
+    default: st = (swiglu ? launch_gemv_t<5, 4, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<5, 4, false>(a, p, dev, *s, stream, pdl)); break;
   }
   if (st != Q4D_OK) return st;
   if (p.k_splits > 1) {
     const long long mn = (long long)M * N;
     const int blocks = int(std::min<long long>((mn + 255) / 256, 4LL * s->num_sms));
-    q4d::q4_gemv_splitk_reduce<<<blocks, 256, 0, stream>>>(static_cast<const float*>(workspace), y,
-                                                          mn, p.k_splits);
+    if (swiglu)
+      q4d::q4_gemv_splitk_reduce_swiglu<<<blocks, 256, 0, stream>>>(
+          static_cast<const float*>(workspace), y, M, N, p.k_splits);
+    else
+      q4d::q4_gemv_splitk_reduce<<<blocks, 256, 0, stream>>>(static_cast<const float*>(workspace),
+                                                            y, mn, p.k_splits);
   }
   if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
   return Q4D_OK;
@@ -369,52 +430,7 @@ const char* q4d_status_string(int status) {
 }
 
 q4d_status q4d_plan_gemv(int M, int N, int K, int num_sms, q4d_gemv_plan* plan) {
-  if (!plan || num_sms < 1) return Q4D_ERR_INVALID_ARG;
-  q4d_status st = check_gemv_shape(M, N, K);
-  if (st != Q4D_OK) return st;
-  const int nsb = K / 256;
-  // Rows are shared out exactly (+-1) over up to one CTA per SM, at least 8
-  // rows each.  When that leaves most SMs idle, K is cut into equal ranges
-  // (a divisor of the super-block count, two or more super-blocks each).
-  int grid_rows = std::min(num_sms, std::max(1, N / 8));
-  int ks = 1;
-  if (2 * grid_rows < num_sms) {
-    const int want = num_sms / grid_rows;
-    for (int d = std::min(want, nsb / 2); d >= 2; --d)
-      if (nsb % d == 0) {
-        ks = d;
-        break;
-      }
-  }
-  const int sbs = nsb / ks;
-  const int rows_per_cta = ceil_div(N, grid_rows);
-  const int tiles = std::min(q4d::kMmaMaxTiles, ceil_div(rows_per_cta, 16));
-  const int rows_per_pass = 16 * tiles;
-  // Super-block columns per stage: the fewest of 1, 2, 4 (dividing the K
-  // range) that give at least 24 KB of weights per stage (fewer, larger
-  // stages amortise the per-stage handshakes); then as many stages as fit,
-  // up to 16.
-  int KC = 1;
-  for (int c : {1, 2, 4}) {
-    if (sbs % c) continue;
-    KC = c;
-    if (size_t(c) * rows_per_pass * 144 >= 24 * 1024) break;
-  }
-  const size_t red = size_t(q4d::kConsumerWarps) * q4d::kMmaMaxTiles * 32 * 16;
-  const size_t stage = q4d::gemv_stage_bytes(M, KC, rows_per_pass);
-  int stages = int((kGemvSmemBudget - red) / (stage + 16));
-  stages = std::max(2, std::min(q4d::kMmaMaxStages, stages));
-  plan->k_splits = ks;
-  plan->sb_per_split = sbs;
-  plan->chunk_sb = KC;
-  plan->rows_per_cta = rows_per_cta;
-  plan->rows_per_pass = rows_per_pass;
-  plan->stages = stages;
-  plan->threads = q4d::kGemvThreads;
-  plan->grid_rows = grid_rows;
-  plan->smem_bytes = stages * stage + red + size_t(stages) * 16;
-  plan->workspace_bytes = ks > 1 ? size_t(ks) * M * N * 4 : 0;
-  return Q4D_OK;
+  return plan_gemv_rows(M, N, K, num_sms, 1, plan);
 }
 
 q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
@@ -486,6 +502,21 @@ q4d_status q4_gemv_ex2(const void* W_q4, const void* x, float* y, int M, int N, 
   if (flags & ~Q4D_GEMV_WEIGHT_PREFETCH) return Q4D_ERR_INVALID_ARG;
   return gemv_impl(W_q4, x, y, M, N, K, static_cast<cudaStream_t>(stream), workspace,
                    workspace_bytes, false, (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0);
+}
+
+q4d_status q4_gemv_swiglu_ex(const void* W_gu, const void* x, float* h, int M, int N, int K,
+                             void* stream, void* workspace, size_t workspace_bytes,
+                             unsigned flags) {
+  if (flags & ~Q4D_GEMV_WEIGHT_PREFETCH) return Q4D_ERR_INVALID_ARG;
+  return gemv_impl(W_gu, x, h, M, N, K, static_cast<cudaStream_t>(stream), workspace,
+                   workspace_bytes, false, (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0, true);
+}
+
+size_t q4d_gemv_swiglu_workspace_bytes(int M, int N, int K) {
+  if (N < 1 || N > (1 << 29)) return 0;
+  q4d_gemv_plan p;
+  if (plan_gemv_rows(M, 2 * N, K, planning_sms(), 2, &p) != Q4D_OK) return 0;
+  return p.workspace_bytes;
 }
 
 q4d_status q4kv_attn_decode(const void* Q, const void* Kq4, const void* Vq4, float* out,

@@ -30,7 +30,8 @@ EXPORTS = (
     "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
     "q4kv_attn_decode_noalloc",
     "q4d_pack_q4_0_weights", "q4d_unpack_q4_0_weights", "q4d_pack_q4_0_rows",
-    "q4d_unpack_q4_0_rows", "q4kv_append",
+    "q4d_unpack_q4_0_rows", "q4kv_append", "q4_gemv_swiglu_ex",
+    "q4d_gemv_swiglu_workspace_bytes",
 )
 
 
@@ -91,6 +92,10 @@ def lib() -> ctypes.CDLL:
         getattr(L, fn).restype = i
     L.q4kv_append.argtypes = [vp, vp, vp, vp, i, i, i, i, vp]
     L.q4kv_append.restype = i
+    L.q4_gemv_swiglu_ex.argtypes = [vp, vp, vp, i, i, i, vp, vp, sz, ctypes.c_uint]
+    L.q4_gemv_swiglu_ex.restype = i
+    L.q4d_gemv_swiglu_workspace_bytes.argtypes = [i, i, i]
+    L.q4d_gemv_swiglu_workspace_bytes.restype = sz
     for fn in ("q4_gemv", "q4_gemv_ex", "q4_gemv_ex2", "q4kv_attn_decode", "q4kv_attn_decode_ex",
                "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
                "q4kv_attn_decode_noalloc"):
@@ -218,6 +223,33 @@ def q4_gemv(W, x, y=None, *, N: int, K: int, stream=None, workspace=None,
                                GEMV_WEIGHT_PREFETCH if weight_prefetch else 0)
     _check(st, "q4_gemv")
     return y
+
+
+def q4_gemv_swiglu(W_gu, x, h=None, *, N: int, K: int, stream=None, workspace=None,
+                   weight_prefetch: bool = False):
+    """h[M][N] (fp32) = silu(gate) * up from one interleaved gate / up matrix
+    ``W_gu`` (2N rows: gate n at row 2n, up n at 2n + 1) via ``q4_gemv_swiglu_ex``."""
+    torch = _torch()
+    _dev_tensor(W_gu, torch.uint8, "W_gu")
+    _dev_tensor(x, torch.bfloat16, "x")
+    if x.dim() != 2 or x.shape[1] != K:
+        raise ValueError("x must be [M][K]")
+    M = x.shape[0]
+    if W_gu.numel() != 2 * N * (K // 256) * 144:
+        raise ValueError("W_gu has the wrong number of bytes for 2N x K")
+    if h is None:
+        h = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _dev_tensor(h, torch.float32, "h")
+    if tuple(h.shape) != (M, N):
+        raise ValueError("h must be [M][N]")
+    with torch.cuda.device(x.device):
+        need = lib().q4d_gemv_swiglu_workspace_bytes(M, N, K)
+        ws = _workspace(need, x.device, workspace)
+        st = lib().q4_gemv_swiglu_ex(W_gu.data_ptr(), x.data_ptr(), h.data_ptr(), M, N, K,
+                                     _stream_ptr(stream), None if ws is None else ws.data_ptr(),
+                                     need, GEMV_WEIGHT_PREFETCH if weight_prefetch else 0)
+    _check(st, "q4_gemv_swiglu")
+    return h
 
 
 def q4kv_append(Kq4, Vq4, k_new, v_new, *, pos: int, kv_stride_tokens: int, stream=None):

@@ -129,3 +129,16 @@ def test_append_rejects_bad_arguments_without_cuda():
     assert L.q4kv_append(FAKE, FAKE, FAKE, FAKE, 4, 64, 60, 5, None) == 2
     assert L.q4kv_append(FAKE + 8, FAKE, FAKE, FAKE, 4, 64, 0, 1, None) == 3
     assert L.q4kv_append(FAKE, FAKE, FAKE + 2, FAKE, 4, 64, 0, 1, None) == 3
+
+
+def test_swiglu_rejects_bad_arguments_without_cuda():
+    L = q4dec.lib()
+    assert L.q4_gemv_swiglu_ex(FAKE, FAKE, FAKE, 1, 16, 256, None, None, 0, 2) == 1
+    assert L.q4_gemv_swiglu_ex(None, FAKE, FAKE, 1, 16, 256, None, None, 0, 0) == 1
+    assert L.q4_gemv_swiglu_ex(FAKE, FAKE, FAKE, 6, 16, 256, None, None, 0, 0) == 2
+    assert L.q4_gemv_swiglu_ex(FAKE, FAKE, FAKE, 1, 16, 100, None, None, 0, 0) == 2
+    assert L.q4_gemv_swiglu_ex(FAKE, FAKE, FAKE, 1, 0, 256, None, None, 0, 0) == 1
+    assert L.q4_gemv_swiglu_ex(FAKE + 8, FAKE, FAKE, 1, 16, 256, None, None, 0, 0) == 3
+    # workspace: a plan over 2N rows in pairs
+    assert L.q4d_gemv_swiglu_workspace_bytes(1, 8, 65536) > 0
+    assert L.q4d_gemv_swiglu_workspace_bytes(1, 0, 256) == 0

@@ -302,3 +302,21 @@ def _simulate_in_warp_producer(n_tiles, S, warps, seed):
 def test_in_warp_producer_never_deadlocks(n_tiles, S):
     for seed in range(40):
         _simulate_in_warp_producer(n_tiles, S, WARPS_R8, seed)
+
+
+@pytest.mark.parametrize("N,K", [(1, 256), (3, 512), (37, 4352), (17408, 5120), (2048, 5120),
+                                 (8, 65536), (75968, 5120)])
+@pytest.mark.parametrize("sms", [148, 7])
+def test_swiglu_partition_keeps_row_pairs_together(N, K, sms):
+    # the fused variant shares out gate / up row pairs: every CTA starts on an
+    # even row and owns whole pairs, so a pass (a multiple of 16 rows from an
+    # even start) never splits a pair
+    rows = 2 * N
+    units = N
+    grid = min(sms, max(1, min(units, rows // 8)))
+    owned = []
+    for c in range(grid):
+        rb, re_ = 2 * (units * c // grid), 2 * (units * (c + 1) // grid)
+        assert rb % 2 == 0 and re_ % 2 == 0 and re_ > rb
+        owned.extend(range(rb, re_))
+    assert owned == list(range(rows))
