@@ -195,19 +195,22 @@ SAMPLE_DESC = ("fp64 numpy oracle: one 5120->6144 Q4_0 GEMV plus one attention l
                "outside the timed part")
 
 
-def cpu_baseline(n_samples=3):
-    total_b, total_t = 0, 0.0
-    for s in range(n_samples):
-        b, t = oracle_sample_step(s)
+def cpu_baseline(min_seconds=10.0, max_samples=40):
+    """The oracle on the host cores: samples until ~10 s of oracle time (at
+    most 40 samples), so the default bench run stays within minutes."""
+    total_b, total_t, n = 0, 0.0, 0
+    while n < max_samples and total_t < min_seconds:
+        b, t = oracle_sample_step(n)
         total_b += b
         total_t += t
+        n += 1
     out = {"value": total_b / total_t / 1e12, "unit": "TB/s", "cores": cpu_cores(),
-           "kind": "oracle", "sample": f"{n_samples} samples; " + SAMPLE_DESC}
+           "kind": "oracle", "seconds": total_t, "sample": f"{n} samples; " + SAMPLE_DESC}
     try:  # the same oracle on one thread
         from threadpoolctl import threadpool_limits
 
         with threadpool_limits(limits=1):
-            b, t = oracle_sample_step(n_samples)
+            b, t = oracle_sample_step(n)
         out["single_thread"] = {"value": b / t / 1e12, "cores": 1, "sample": "1 sample"}
     except Exception as e:  # noqa: BLE001
         out["single_thread"] = {"error": str(e)[:200]}
