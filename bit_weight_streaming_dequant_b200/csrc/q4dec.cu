@@ -16,6 +16,7 @@
 
 #include "q4_gemv.cuh"
 #include "q4kv_attn.cuh"
+#include "q4kv_attn_tc.cuh"
 #include "q4kv_append.cuh"
 
 // Device error word (bit q4d::kDevErrWaitTimeout: a bounded wait ran out).
@@ -347,6 +348,18 @@ q4d_status launch_attn_t(const q4d::AttnArgs& a, const q4d_attn_plan& p, int n_k
   return Q4D_OK;
 }
 
+// The tensor-memory kernel with NR (16 or 32) MMA columns of query rows.
+template <int NR>
+q4d_status launch_attn_tc(const q4d::AttnArgs& a, const q4d_attn_plan& p, int n_kv, int dev,
+                          const DeviceState& s, cudaStream_t stream) {
+  static std::atomic<bool> smem_set[kMaxDevices];
+  q4d_status st = allow_smem(q4d::q4kv_attn_tc_kernel<NR>, dev, s, smem_set);
+  if (st != Q4D_OK) return st;
+  dim3 grid(p.n_splits, n_kv, p.row_groups);
+  q4d::q4kv_attn_tc_kernel<NR><<<grid, p.threads, p.smem_bytes, stream>>>(a);
+  return Q4D_OK;
+}
+
 q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out, int ctx_len,
                      int n_q, int n_kv, int head_dim, int M, int kv_stride, float scale,
                      cudaStream_t stream, void* workspace, size_t workspace_bytes,
@@ -391,12 +404,12 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
   a.rows_per_cta = p.rows_per_cta;
   a.stages = p.stages;
 
-  switch ((p.rows_per_cta + 7) / 8) {
-    case 1: st = launch_attn_t<1>(a, p, n_kv, dev, *s, stream); break;
-    case 2: st = launch_attn_t<2>(a, p, n_kv, dev, *s, stream); break;
-    case 3: st = launch_attn_t<3>(a, p, n_kv, dev, *s, stream); break;
-    default: st = launch_attn_t<4>(a, p, n_kv, dev, *s, stream); break;
-  }
+  if (p.rows_per_cta <= 8)
+    st = launch_attn_t<1>(a, p, n_kv, dev, *s, stream);
+  else if (p.rows_per_cta <= 16)
+    st = launch_attn_tc<16>(a, p, n_kv, dev, *s, stream);
+  else
+    st = launch_attn_tc<32>(a, p, n_kv, dev, *s, stream);
   if (st != Q4D_OK) return st;
   if (p.n_splits > 1) q4d::q4kv_attn_merge_kernel<<<M * n_q, 256, 0, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
@@ -441,11 +454,13 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   const int rows_all = (n_q_heads / n_kv_heads) * M;
   const int row_groups = ceil_div(rows_all, q4d::kAttnMaxRows);
   const int rows_per_cta = ceil_div(rows_all, row_groups);
-  // Variant: warp-local (12 warps, 192-token tiles) for at most 8 rows per
-  // CTA, else generic (8 warps + a producer warp, 128-token tiles).
+  // Variant: warp-local mma.sync kernel (12 warps, 192-token tiles) for at
+  // most 8 rows per CTA, else the tensor-memory kernel (8 token warps, a
+  // producer warp and an MMA warp; 128-token tiles; 16 or 32 MMA columns).
   const bool rows8 = rows_per_cta <= 8;
-  const int TT = rows8 ? q4d::kR8Tile : q4d::kAttnTileTokens;
-  const size_t stage_bytes = rows8 ? q4d::kR8StageBytes : q4d::kAttnStageBytes;
+  const int nr = rows_per_cta <= 16 ? 16 : 32;
+  const int TT = rows8 ? q4d::kR8Tile : q4d::kTcaTile;
+  const size_t stage_bytes = rows8 ? q4d::kR8StageBytes : q4d::kTcaStage;
   // One CTA per SM (the K/V ring takes most of shared memory): enough context
   // splits that (splits x KV heads x row groups) fills the SMs once, each
   // split at least two tiles long and at most 256 splits (the merge kernel's
@@ -458,7 +473,7 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   n_splits = ceil_div(ctx_len, split_tokens);
   // As many ring stages as fit next to the variant's fixed buffers, up to 8
   // (at least 2: the warp-local variant parks 96 KB in the ring at the end).
-  const size_t fixed = rows8 ? q4d::attn_rows8_smem_bytes(0) : q4d::attn_smem_bytes(0);
+  const size_t fixed = rows8 ? q4d::attn_rows8_smem_bytes(0) : q4d::tca_smem_bytes(nr, 0);
   int stages = int((kAttnSmemBudget - fixed) / (stage_bytes + 16));
   stages = std::max(2, std::min(8, stages));
   plan->n_splits = n_splits;
@@ -467,8 +482,8 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   plan->row_groups = row_groups;
   plan->rows_per_cta = rows_per_cta;
   plan->stages = stages;
-  plan->threads = rows8 ? q4d::kR8Threads : q4d::kAttnThreads;
-  plan->smem_bytes = rows8 ? q4d::attn_rows8_smem_bytes(stages) : q4d::attn_smem_bytes(stages);
+  plan->threads = rows8 ? q4d::kR8Threads : q4d::kTcaThreads;
+  plan->smem_bytes = rows8 ? q4d::attn_rows8_smem_bytes(stages) : q4d::tca_smem_bytes(nr, stages);
   plan->workspace_bytes =
       n_splits > 1 ? size_t(n_splits) * M * n_q_heads * (q4d::kHeadDim + 2) * 4 : 0;
   return Q4D_OK;

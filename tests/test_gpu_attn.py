@@ -84,8 +84,13 @@ def test_uniform_keys_give_mean_of_visible_values(cuda_ok):
     out = _gpu(Q, K, V, ctx, n_q, n_kv, M).cpu().numpy()
     Vh = oracle.dequant(V, n_kv * ctx, 256).reshape(n_kv, ctx, 256)
     for m in range(M):
-        mean = Vh[:, : ctx - M + m + 1].mean(axis=1)          # [n_kv][256]
-        assert np.abs(out[m] - np.repeat(mean, n_q // n_kv, axis=0)).max() <= 1e-5
+        vis = Vh[:, : ctx - M + m + 1]
+        mean = vis.mean(axis=1)                                 # [n_kv][256]
+        # the kernels may round each product d*(q - 8) once to fp16 before the
+        # P.V contraction: at most 2^-11 of |v| per term, so of the mean |v|
+        bound = 2.0 ** -11 * np.abs(vis).mean(axis=1) + 1e-6
+        err = np.abs(out[m] - np.repeat(mean, n_q // n_kv, axis=0))
+        assert (err <= np.repeat(bound, n_q // n_kv, axis=0)).all(), err.max()
 
 
 def test_constant_values_and_single_token(cuda_ok):

@@ -103,12 +103,35 @@ TT_ATTN, Q_PITCH, PT_PITCH, ROW = 128, 576, 80, 144
 TT_R8, WARPS_R8 = 192, 12          # warp-local variant (at most 8 rows per CTA)
 
 
+TC_THREADS, TC_V_BYTES = 448, 256 * 128 * 2   # tensor-memory variant: 14 warps, fp16 V tile
+
+
+def _tc_nr(rows_per_cta):
+    return 16 if rows_per_cta <= 16 else 32
+
+
+def _tc_offsets(stages, nr):
+    """Carve-up of the tensor-memory variant's shared memory: ring, Q (fp16,
+    K-major), V tile (fp16, M-major), two P^T buffers (fp16, N-major), row
+    statistics ([4][32] warp partials, running max, max used, alpha, sums,
+    causal limits), flags, barriers (2 per ring stage + 12) and the
+    tensor-memory address."""
+    ring = stages * 2 * TT_ATTN * ROW
+    q = ring
+    v = q + 512 * nr
+    pt = v + TC_V_BYTES
+    stats = pt + 2 * (nr // 8) * 2048
+    flags = stats + 4 * 32 * 4 + 5 * 32 * 4
+    bars = flags + 16
+    end = bars + (2 * stages + 12) * 8 + 8
+    return dict(ring=ring, q=q, v=v, pt=pt, stats=stats, flags=flags, bars=bars, end=end)
+
+
 def _attn_smem(stages, rows_per_cta):
     if rows_per_cta <= 8:      # ring + Q fragments + per-warp / per-row stats + barriers
         return stages * 2 * TT_R8 * ROW + 8 * Q_PITCH + WARPS_R8 * 8 * 2 * 4 + 8 * 2 * 4 \
             + stages * 16
-    return stages * 2 * TT_ATTN * ROW + 32 * Q_PITCH + TT_ATTN * PT_PITCH + 32 * 8 * 4 + 32 * 4 \
-        + stages * 16
+    return _tc_offsets(stages, _tc_nr(rows_per_cta))["end"]
 
 
 def _chunks(addrs):
@@ -149,7 +172,7 @@ def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
     g = nq // nkv
     rows8 = p.rows_per_cta <= 8
     assert TT == (TT_R8 if rows8 else TT_ATTN) and p.split_tokens % TT == 0
-    assert p.threads == (WARPS_R8 * 32 if rows8 else 288)
+    assert p.threads == (WARPS_R8 * 32 if rows8 else TC_THREADS)
     assert 1 <= p.n_splits <= 256
     assert p.rows_per_cta <= 32 and p.row_groups * p.rows_per_cta >= g * M
     assert 2 <= p.stages <= 8
@@ -161,11 +184,9 @@ def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
         assert ring >= WARPS_R8 * 8 * 256 * 4
         assert ring % 16 == 0 and (ring + 8 * Q_PITCH + WARPS_R8 * 64 + 64) % 8 == 0
     else:
-        # carve-up: ring, Q fragments, P^T (16-byte aligned for ldmatrix / v4),
-        # row maxima, row sums, barriers (8-byte aligned)
-        q_off, pt_off = ring, ring + 32 * Q_PITCH
-        bar_off = pt_off + TT * PT_PITCH + 32 * 8 * 4 + 32 * 4
-        assert q_off % 16 == 0 and pt_off % 16 == 0 and bar_off % 8 == 0
+        o = _tc_offsets(p.stages, _tc_nr(p.rows_per_cta))
+        # operands of the tensor-core descriptors 16-byte aligned, barriers 8
+        assert all(o[k] % 16 == 0 for k in ("q", "v", "pt", "stats", "flags", "bars"))
     assert (TT * ROW) % 16 == 0
     cache_bytes = nkv * stride * 144
     tokens = []
@@ -207,24 +228,80 @@ def test_attn_geometry(ctx, nq, nkv, M, stride_extra):
                 assert hi < WARPS_R8 * 8 * 256
         _attn_q_and_workspace(p, M, nq, nkv, g)
         return
-    # generic variant: K ldmatrix rows / columns, block scales, V
-    # ldmatrix.trans rows, P^T ldmatrix.trans rows / columns
-    for warp in range(8):
-        for lane in range(32):
-            tok = 16 * warp + (lane & 15)
-            for b in range(0, 8, 2):
-                col = (lane >> 4) * 16 + b * 16
-                assert tok < TT and col + 16 <= 128
-                assert 128 + 2 * b + 4 <= ROW
-            for k0 in range(0, TT, 32):
-                assert k0 + lane < TT and warp * 16 + 16 <= 128
-                for h in range(2):
-                    kb = k0 + 16 * h
-                    assert kb + 2 * (lane & 3) + 8 + 1 < TT and 128 + 2 * warp + 2 <= ROW
-                    for rt in range(0, nrt, 2):
-                        pcol = rt * 16 + (lane >> 4) * 16 if rt + 1 < nrt else rt * 16
-                        assert kb + (lane & 15) < TT and pcol + 16 <= 64
+    _tc_layout_checks(_tc_nr(p.rows_per_cta))
     _attn_q_and_workspace(p, M, nq, nkv, g)
+
+
+def _pair_elements(word, low):
+    """Elements of a Q4_0 block held by the fp16 pair unpacked from bits 0-3
+    (low) or 4-7 of bytes 0 and 2 of `word` (a 4-byte group, word 0 = bytes
+    0..3): byte j holds element j in its low nibble, j + 16 in its high."""
+    b0, b2 = 4 * (word // 4) + (word % 4), 4 * (word // 4) + (word % 4) + 2
+    return (b0, b2) if low else (b0 + 16, b2 + 16)
+
+
+def _tc_unpacked_element(kk):
+    # restatement of the kernel's element order: column c = kk // 2 holds
+    # pair i = c % 4 of word t = c // 4
+    c, h = kk >> 1, kk & 1
+    t, i = c >> 2, c & 3
+    return (16 if i & 1 else 0) + 4 * t + (i >> 1) + 2 * h
+
+
+def test_tc_element_order_matches_nibble_unpacking():
+    # word t of a block unpacks as q8_pair<low>(w), q8_pair<high>(w),
+    # q8_pair<low>(w >> 8), q8_pair<high>(w >> 8): bytes (4t, 4t+2) then
+    # (4t+1, 4t+3)
+    order = []
+    for t in range(4):
+        order += _pair_elements(4 * t, True) + _pair_elements(4 * t, False)
+        order += _pair_elements(4 * t + 1, True) + _pair_elements(4 * t + 1, False)
+    assert order == [_tc_unpacked_element(kk) for kk in range(32)]
+    assert sorted(order) == list(range(32))
+
+
+def _tc_layout_checks(nr):
+    # Q, K-major canonical layout: (kp, n) -> (kp>>3)*nr*16 + (n>>3)*128 + (n&7)*16 + (kp&7)*2
+    q_off = {(kp >> 3) * nr * 16 + (n >> 3) * 128 + (n & 7) * 16 + (kp & 7) * 2
+             for kp in range(256) for n in range(nr)}
+    assert q_off == set(range(0, 512 * nr, 2))
+    # QK B operand, step s: core matrices at base + s*nr*32 + kg*LBO + ng*SBO (LBO nr*16, SBO 128)
+    reads = set()
+    for s_ in range(16):
+        for kg in range(2):
+            for ng in range(nr // 8):
+                reads.add(s_ * nr * 32 + kg * nr * 16 + ng * 128)
+    assert reads == set(range(0, 512 * nr, 128))
+    # V tile, M-major: V warp (8..11) lane -> token k, chunk (4b + t) of 8 dimensions
+    v_off = []
+    for warp in range(8, 12):
+        for lane in range(32):
+            k = 32 * (warp & 3) + lane
+            for b in range(8):
+                for t in range(4):
+                    v_off.append((4 * b + t) * 2048 + (k >> 3) * 128 + (k & 7) * 16)
+    assert sorted(v_off) == list(range(0, TC_V_BYTES, 16))
+    # PV A operand (half h, step j): core matrices base + h*32768 + j*256 + kg*128 + mg*2048
+    a_reads = {h * 32768 + j * 256 + kg * 128 + mg * 2048
+               for h in range(2) for j in range(8) for kg in range(2) for mg in range(16)}
+    assert a_reads == set(range(0, TC_V_BYTES, 128))
+    # P^T, N-major: softmax warp (0..3) lane -> token k, rows 8c .. 8c + 7
+    p_off = []
+    for warp in range(4):
+        for lane in range(32):
+            k = 32 * warp + lane
+            for c in range(nr // 8):
+                p_off.append(c * 2048 + (k >> 3) * 128 + (k & 7) * 16)
+    assert sorted(p_off) == list(range(0, (nr // 8) * 2048, 16))
+    b_reads = {j * 256 + kg * 128 + ng * 2048 for j in range(8) for kg in range(2)
+               for ng in range(nr // 8)}
+    assert b_reads == set(range(0, (nr // 8) * 2048, 128))
+    # tensor memory: K tiles [2][128], S^T [2][nr], O^T [2][nr] in 512 columns
+    assert 256 + 4 * nr <= 512
+    # the epilogue's lane -> dimension map is a bijection of 0..255 that
+    # inverts the Q element order
+    dims = [(mm & ~31) + _tc_unpacked_element(mm & 31) for mm in range(256)]
+    assert sorted(dims) == list(range(256))
 
 
 def _attn_q_and_workspace(p, M, nq, nkv, g):
