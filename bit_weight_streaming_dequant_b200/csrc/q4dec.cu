@@ -330,21 +330,14 @@ q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, in
   return Q4D_OK;
 }
 
-// NRT = 1: the warp-local kernel (at most 8 query rows per CTA); 2..4: the
-// generic kernel.
-template <int NRT>
-q4d_status launch_attn_t(const q4d::AttnArgs& a, const q4d_attn_plan& p, int n_kv, int dev,
-                         const DeviceState& s, cudaStream_t stream) {
+// The warp-local mma.sync kernel (at most 8 query rows per CTA).
+q4d_status launch_attn_rows8(const q4d::AttnArgs& a, const q4d_attn_plan& p, int n_kv, int dev,
+                             const DeviceState& s, cudaStream_t stream) {
   static std::atomic<bool> smem_set[kMaxDevices];
-  void (*kernel)(q4d::AttnArgs);
-  if constexpr (NRT == 1)
-    kernel = q4d::q4kv_attn_split_rows8_kernel;
-  else
-    kernel = q4d::q4kv_attn_split_kernel<NRT>;
-  q4d_status st = allow_smem(kernel, dev, s, smem_set);
+  q4d_status st = allow_smem(q4d::q4kv_attn_split_rows8_kernel, dev, s, smem_set);
   if (st != Q4D_OK) return st;
   dim3 grid(p.n_splits, n_kv, p.row_groups);
-  kernel<<<grid, p.threads, p.smem_bytes, stream>>>(a);
+  q4d::q4kv_attn_split_rows8_kernel<<<grid, p.threads, p.smem_bytes, stream>>>(a);
   return Q4D_OK;
 }
 
@@ -405,7 +398,7 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
   a.stages = p.stages;
 
   if (p.rows_per_cta <= 8)
-    st = launch_attn_t<1>(a, p, n_kv, dev, *s, stream);
+    st = launch_attn_rows8(a, p, n_kv, dev, *s, stream);
   else if (p.rows_per_cta <= 16)
     st = launch_attn_tc<16>(a, p, n_kv, dev, *s, stream);
   else

@@ -13,7 +13,7 @@
 // (contiguous: one super-block per token) stream into a ring of shared-memory
 // stages by bulk copies on full/empty mbarriers with bounded waits.
 //
-// Both variants below compute, per tile:
+// The kernel below (at most 8 query rows per CTA) computes, per tile:
 //  1. Scores, exact up to fp32 rounding: ldmatrix hands lane (g, t) word t
 //     of the 16-byte nibble piece of tokens g and g+8 (the A-fragment layout);
 //     the nibbles become exact fp16 (q - 8); Q, converted to fp16 once, is
@@ -28,35 +28,18 @@
 //     unpacks in registers, exact in fp16; the V block scale d goes into the
 //     B operand, P^T times d of the same tokens in one fp16 multiply
 //     (|P d| <= |d|: no overflow).  O^T accumulates in fp32.
-// The warp-local variant (at most 8 query rows) gives each warp its own
-// tokens, softmax and full O^T; the generic one (up to 32 rows) splits tokens
-// across warps for the scores and dimensions for P.V, exchanging maxima and
-// P^T through shared memory.
+// Each warp owns its own tokens, softmax state and full O^T.  More query rows
+// per CTA (9..32) go to the tensor-memory kernel in q4kv_attn_tc.cuh; both
+// write the same split states for the merge kernel at the end of this file.
 #pragma once
 
 #include "q4dec_device.cuh"
 
 namespace q4d {
 
-constexpr int kAttnConsumerWarps = 8;
-constexpr int kAttnThreads = (kAttnConsumerWarps + 1) * 32;  // + one producer warp
-constexpr int kAttnTileTokens = 128;
-constexpr int kAttnMaxRows = 32;                              // 4 row tiles of 8
+constexpr int kAttnMaxRows = 32;                              // query rows per CTA, at most
 constexpr int kHeadDim = 256;
 constexpr int kRowBytes = 144;                                // one super-block per token
-constexpr int kPtPitch = 80;                                  // bytes per token row of P^T
-constexpr int kQPitch = 8 * 4 * 16 + 64;                      // bytes per row of Q fragments
-constexpr uint32_t kAttnStageBytes = 2u * kAttnTileTokens * kRowBytes;  // K tile + V tile
-
-// Dynamic shared memory of the split kernel for a given stage count.
-__host__ __device__ constexpr size_t attn_smem_bytes(int stages) {
-  return size_t(stages) * kAttnStageBytes                // K/V ring
-         + size_t(kAttnMaxRows) * kQPitch                // Q fragments [row][block][t] x 16 B
-         + size_t(kAttnTileTokens) * kPtPitch            // P^T fp16
-         + size_t(kAttnMaxRows) * kAttnConsumerWarps * 4 // per-warp row maxima
-         + size_t(kAttnMaxRows) * 4                      // per-row final sums
-         + size_t(stages) * 16;                          // full / empty barriers
-}
 
 struct AttnArgs {
   const uint16_t* Q;   // bf16 bits [M][n_q][256]
@@ -116,9 +99,6 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void attn_consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kAttnConsumerWarps * 32) : "memory");
 }
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -459,328 +439,6 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
       }
     }
   }
-}
-
-// Generic variant, NRT row tiles of 8 query rows (2..4, up to 32 rows): the
-// warps split the tile's tokens for the scores and the head dimensions for
-// P.V, exchanging the running maxima and P^T through shared memory with two
-// CTA-wide barriers per tile.  Q fragments are read from shared memory.
-template <int NRT>
-__global__ void __launch_bounds__(kAttnThreads, 1) q4kv_attn_split_kernel(const AttnArgs a) {
-  constexpr int TT = kAttnTileTokens;
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int S = a.stages;
-  uint8_t* ring = smem;
-  uint8_t* Qp = ring + size_t(S) * kAttnStageBytes;                 // [row] x kQPitch
-  uint8_t* Pt = Qp + kAttnMaxRows * kQPitch;                         // [token] x kPtPitch, fp16
-  float* red = reinterpret_cast<float*>(Pt + TT * kPtPitch);        // [row][warp]
-  float* row_sum = red + kAttnMaxRows * kAttnConsumerWarps;          // [row]
-  uint64_t* full = reinterpret_cast<uint64_t*>(row_sum + kAttnMaxRows);
-  uint64_t* empty = full + S;
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int split = blockIdx.x, kh = blockIdx.y, rgrp = blockIdx.z;
-  const int R_all = a.g * a.M;
-  const int row0 = rgrp * a.rows_per_cta;
-  const int R = min(a.rows_per_cta, R_all - row0);
-  const int t_begin = split * a.split_tokens;
-  const int t_end = min(a.ctx_len, t_begin + a.split_tokens);
-  const int n_tiles = (t_end - t_begin + TT - 1) / TT;
-  const uint8_t* Kh = a.K + size_t(kh) * a.kv_stride * kRowBytes;
-  const uint8_t* Vh = a.V + size_t(kh) * a.kv_stride * kRowBytes;
-
-  if (tid == 0) {
-    griddep_launch_dependents();  // a following weight-prefetching GEMV may start
-    for (int s = 0; s < S; ++s) {
-      mbar_init(smem_addr(&full[s]), 1);
-      mbar_init(smem_addr(&empty[s]), kAttnConsumerWarps);
-    }
-    mbar_init_fence();
-  }
-  __syncthreads();
-
-  if (warp == kAttnConsumerWarps) {
-    // ---------------- producer: K and V tiles, one bulk copy each ----------
-    if (lane == 0) {
-      const uint64_t pol = l2_evict_first_policy();
-      int slot = 0;
-      uint32_t phase = 0;
-      for (int tile = 0; tile < n_tiles; ++tile) {
-        if (tile >= S) mbar_wait(smem_addr(&empty[slot]), phase ^ 1u, a.err);
-        const int t0 = t_begin + tile * TT;
-        const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * kRowBytes;
-        const uint32_t bar = smem_addr(&full[slot]);
-        const uint32_t dk = smem_addr(ring + size_t(slot) * kAttnStageBytes);
-        mbar_arrive_expect_tx(bar, 2 * bytes);
-        bulk_g2s(dk, Kh + size_t(t0) * kRowBytes, bytes, bar, pol);
-        bulk_g2s(dk + TT * kRowBytes, Vh + size_t(t0) * kRowBytes, bytes, bar, pol);
-        if (++slot == S) {
-          slot = 0;
-          phase ^= 1u;
-        }
-      }
-    }
-    return;
-  }
-
-  // ---------------- consumers ----------------
-  const int g = lane >> 2, t = lane & 3;
-
-  // Q fragments (fp16, zero for padding rows): see q_frag_f16.
-  for (int i = tid; i < kAttnMaxRows * 32; i += kAttnConsumerWarps * 32) {
-    const int r = i >> 5, b = (i >> 2) & 7, tt = i & 3;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < R) {
-      const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
-      v = q_frag_f16(a.Q + (size_t(m) * a.n_q + kh * a.g + j) * kHeadDim + b * 32 + 4 * tt);
-    }
-    *reinterpret_cast<uint4*>(Qp + r * kQPitch + (i & 31) * 16) = v;
-  }
-  attn_consumer_sync();
-  const uint32_t Qp_addr = smem_addr(Qp), Pt_addr = smem_addr(Pt);
-
-  // rows this lane holds in every row tile: 8*rt + 2t + e, e = 0, 1
-  int row_pos[NRT][2];  // position of the row's draft token; -1 for padding rows
-  float m_run[NRT][2], l_run[NRT][2];
-  #pragma unroll
-  for (int rt = 0; rt < NRT; ++rt)
-    #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int r = 8 * rt + 2 * t + e;
-      row_pos[rt][e] = r < R ? a.ctx_len - a.M + (row0 + r) / a.g : -1;
-      m_run[rt][e] = -INFINITY;
-      l_run[rt][e] = 0.f;
-    }
-  float o[2][NRT][4];  // O^T fragments: [dim tile][row tile]
-  #pragma unroll
-  for (int d = 0; d < 2; ++d)
-    #pragma unroll
-    for (int rt = 0; rt < NRT; ++rt) o[d][rt][0] = o[d][rt][1] = o[d][rt][2] = o[d][rt][3] = 0.f;
-
-  int slot = 0;
-  uint32_t phase = 0;
-
-  #pragma unroll 1
-  for (int tile = 0; tile < n_tiles; ++tile) {
-    const int t0 = t_begin + tile * TT;
-    const int n_tok = min(TT, t_end - t0);
-    mbar_wait(smem_addr(&full[slot]), phase, a.err);
-    const uint8_t* Kt = ring + size_t(slot) * kAttnStageBytes;
-    const uint8_t* Vt = Kt + TT * kRowBytes;
-    const uint32_t Kt_addr = smem_addr(Kt), Vt_addr = smem_addr(Vt);
-
-    // ---- 1. S^T for tokens 16*warp + g (a) and + g + 8 (b)
-    const int tok_a = 16 * warp + g, tok_b = tok_a + 8;
-    float s[NRT][4];
-    #pragma unroll
-    for (int rt = 0; rt < NRT; ++rt) s[rt][0] = s[rt][1] = s[rt][2] = s[rt][3] = 0.f;
-    {
-      // ldmatrix rows: lanes 0-7 tokens 16w+0..7 block b, 8-15 tokens
-      // 16w+8..15 block b, 16-23 tokens 16w+0..7 block b+1, 24-31 tokens
-      // 16w+8..15 block b+1; lane (g, t) receives word t of each.
-      const uint32_t lbase = Kt_addr + uint32_t(16 * warp + (lane & 15)) * kRowBytes +
-                             uint32_t(lane >> 4) * 16u;
-      const uint8_t* da_p = Kt + tok_a * kRowBytes + 128;
-      const uint8_t* db_p = Kt + tok_b * kRowBytes + 128;
-      #pragma unroll
-      for (int b = 0; b < 8; b += 2) {
-        uint32_t w0a, w0b, w1a, w1b;
-        ldsm_x4(lbase + uint32_t(b) * 16u, w0a, w0b, w1a, w1b);
-        // (d_b, d_b+1) of tokens a and b
-        const float2 dA = __half22float2(*reinterpret_cast<const __half2*>(da_p + 2 * b));
-        const float2 dB = __half22float2(*reinterpret_cast<const __half2*>(db_p + 2 * b));
-        #pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          uint32_t qa[4], qb[4];
-          k_pairs(bb ? w1a : w0a, qa);
-          k_pairs(bb ? w1b : w0b, qb);
-          const float da = bb ? dA.y : dA.x, db = bb ? dB.y : dB.x;
-          #pragma unroll
-          for (int rt = 0; rt < NRT; ++rt) {
-            uint4 qf;
-            asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                         : "=r"(qf.x), "=r"(qf.y), "=r"(qf.z), "=r"(qf.w)
-                         : "r"(Qp_addr + uint32_t((8 * rt + g) * kQPitch + ((b + bb) * 4 + t) * 16)));
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_f16(c, qa[0], qb[0], qa[1], qb[1], qf.x, qf.y);
-            mma_f16(c, qa[2], qb[2], qa[3], qb[3], qf.z, qf.w);
-            s[rt][0] = fmaf(da, c[0], s[rt][0]);
-            s[rt][1] = fmaf(da, c[1], s[rt][1]);
-            s[rt][2] = fmaf(db, c[2], s[rt][2]);
-            s[rt][3] = fmaf(db, c[3], s[rt][3]);
-          }
-        }
-      }
-      // base-2 logits, causal / tile-end mask, this warp's per-row maxima
-      const int ta = t0 + tok_a, tb = t0 + tok_b;
-      #pragma unroll
-      for (int rt = 0; rt < NRT; ++rt)
-        #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int pos = row_pos[rt][e];
-          s[rt][e] = (tok_a < n_tok && ta <= pos) ? s[rt][e] * a.scale_log2 : -INFINITY;
-          s[rt][2 + e] = (tok_b < n_tok && tb <= pos) ? s[rt][2 + e] * a.scale_log2 : -INFINITY;
-          float mx = fmaxf(s[rt][e], s[rt][2 + e]);
-          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 4));
-          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 8));
-          mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
-          if (g == 0) red[(8 * rt + 2 * t + e) * kAttnConsumerWarps + warp] = mx;
-        }
-    }
-    attn_consumer_sync();
-
-    // ---- 2. running max, rescale factors, P = 2^(s - m) as fp16 P^T
-    float alpha[NRT][2];
-    #pragma unroll
-    for (int rt = 0; rt < NRT; ++rt) {
-      #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float4* rm =
-            reinterpret_cast<const float4*>(red + (8 * rt + 2 * t + e) * kAttnConsumerWarps);
-        const float4 x0 = rm[0], x1 = rm[1];
-        const float tile_max = fmaxf(fmaxf(fmaxf(x0.x, x0.y), fmaxf(x0.z, x0.w)),
-                                     fmaxf(fmaxf(x1.x, x1.y), fmaxf(x1.z, x1.w)));
-        const float m_new = fmaxf(m_run[rt][e], tile_max);
-        // a row with no visible token so far keeps m = -inf, weight 0, alpha 1
-        const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        alpha[rt][e] = m_new == -INFINITY ? 1.f : ex2(m_run[rt][e] - m_use);
-        m_run[rt][e] = m_new;
-        s[rt][e] = ex2(s[rt][e] - m_use);
-        s[rt][2 + e] = ex2(s[rt][2 + e] - m_use);
-      }
-      // P^T entries as fp16; the row sums add the same rounded weights
-      const uint32_t pa = pack_f16x2(s[rt][0], s[rt][1]);
-      const uint32_t pb = pack_f16x2(s[rt][2], s[rt][3]);
-      const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&pa));
-      const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&pb));
-      l_run[rt][0] = l_run[rt][0] * alpha[rt][0] + fa.x + fb.x;
-      l_run[rt][1] = l_run[rt][1] * alpha[rt][1] + fa.y + fb.y;
-      *reinterpret_cast<uint32_t*>(Pt + tok_a * kPtPitch + (8 * rt + 2 * t) * 2) = pa;
-      *reinterpret_cast<uint32_t*>(Pt + tok_b * kPtPitch + (8 * rt + 2 * t) * 2) = pb;
-    }
-    attn_consumer_sync();
-
-    // ---- 3. O^T[dims of block `warp`][rows] += Vhat^T P^T over the tile
-    #pragma unroll
-    for (int d = 0; d < 2; ++d)
-      #pragma unroll
-      for (int rt = 0; rt < NRT; ++rt) {
-        o[d][rt][0] *= alpha[rt][0];
-        o[d][rt][1] *= alpha[rt][1];
-        o[d][rt][2] *= alpha[rt][0];
-        o[d][rt][3] *= alpha[rt][1];
-      }
-    {
-      // ldmatrix.trans over the 16-byte V piece of block `warp`: lane i
-      // addresses token k0 + i, so matrix j covers tokens k0 + 8j .. +7 and
-      // lane (g, t) receives bytes 2g, 2g+1 of tokens k0 + 8j + 2t and +1.
-      const uint32_t vbase = Vt_addr + uint32_t(lane) * kRowBytes + uint32_t(warp) * 16u;
-      const uint32_t pbase = Pt_addr + uint32_t(lane & 15) * kPtPitch + uint32_t(lane >> 4) * 16u;
-      const uint8_t* vd = Vt + 128 + 2 * warp;
-      #pragma unroll 1
-      for (int k0 = 0; k0 < n_tok; k0 += 32) {
-        uint32_t v[4];
-        ldsm_x4_trans(vbase + uint32_t(k0) * kRowBytes, v[0], v[1], v[2], v[3]);
-        #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // k16 step: tokens kb .. kb + 15
-          const int kb = k0 + 16 * h;
-          const int ta = kb + 2 * t, tb = ta + 8;
-          // block scales of tokens (ta, ta+1) and (tb, tb+1); zero past the
-          // tile end, where the shared memory holds no token of this split
-          uint32_t d_lo = uint32_t(*reinterpret_cast<const uint16_t*>(vd + ta * kRowBytes)) |
-                          (uint32_t(*reinterpret_cast<const uint16_t*>(vd + (ta + 1) * kRowBytes)) << 16);
-          uint32_t d_hi = uint32_t(*reinterpret_cast<const uint16_t*>(vd + tb * kRowBytes)) |
-                          (uint32_t(*reinterpret_cast<const uint16_t*>(vd + (tb + 1) * kRowBytes)) << 16);
-          if (kb + 16 > n_tok) {
-            d_lo &= (ta < n_tok ? 0xFFFFu : 0u) | (ta + 1 < n_tok ? 0xFFFF0000u : 0u);
-            d_hi &= (tb < n_tok ? 0xFFFFu : 0u) | (tb + 1 < n_tok ? 0xFFFF0000u : 0u);
-          }
-          const uint32_t ra = v[2 * h], rb = v[2 * h + 1];
-          // A fragments (q - 8, exact): dim tile 0 = block dims {2g, 2g+16},
-          // dim tile 1 = {2g+1, 2g+17}
-          const uint32_t a00 = q8_pair<true>(ra), a01 = q8_pair<false>(ra);
-          const uint32_t a02 = q8_pair<true>(rb), a03 = q8_pair<false>(rb);
-          const uint32_t a10 = q8_pair<true>(ra >> 8), a11 = q8_pair<false>(ra >> 8);
-          const uint32_t a12 = q8_pair<true>(rb >> 8), a13 = q8_pair<false>(rb >> 8);
-          #pragma unroll
-          for (int rt = 0; rt < NRT; rt += 2) {
-            // B fragments: P^T of tokens (kb + 2t, +1) and (kb + 2t + 8, +9)
-            // times those tokens' block scales -- this warp's block only
-            const uint32_t paddr = pbase + uint32_t(kb) * kPtPitch + uint32_t(rt) * 16u;
-            if (rt + 1 < NRT) {
-              uint32_t p0, p1, p2, p3;
-              ldsm_x4_trans(paddr, p0, p1, p2, p3);
-              p0 = f16x2_mul(p0, d_lo);
-              p1 = f16x2_mul(p1, d_hi);
-              p2 = f16x2_mul(p2, d_lo);
-              p3 = f16x2_mul(p3, d_hi);
-              mma_f16(o[0][rt], a00, a01, a02, a03, p0, p1);
-              mma_f16(o[1][rt], a10, a11, a12, a13, p0, p1);
-              mma_f16(o[0][rt + 1], a00, a01, a02, a03, p2, p3);
-              mma_f16(o[1][rt + 1], a10, a11, a12, a13, p2, p3);
-            } else {
-              uint32_t p0, p1;
-              ldsm_x2_trans(paddr, p0, p1);
-              p0 = f16x2_mul(p0, d_lo);
-              p1 = f16x2_mul(p1, d_hi);
-              mma_f16(o[0][rt], a00, a01, a02, a03, p0, p1);
-              mma_f16(o[1][rt], a10, a11, a12, a13, p0, p1);
-            }
-          }
-        }
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_addr(&empty[slot]));
-    if (++slot == S) {
-      slot = 0;
-      phase ^= 1u;
-    }
-  }
-
-  // ---- split totals: l summed over lanes and warps; O^T of block `warp`
-  #pragma unroll
-  for (int rt = 0; rt < NRT; ++rt)
-    #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float l = l_run[rt][e];
-      l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
-      l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
-      l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
-      if (g == 0) red[(8 * rt + 2 * t + e) * kAttnConsumerWarps + warp] = l;
-    }
-  attn_consumer_sync();
-  if (tid < 8 * NRT) {
-    float l = 0.f;
-    for (int w = 0; w < kAttnConsumerWarps; ++w) l += red[tid * kAttnConsumerWarps + w];
-    row_sum[tid] = l;
-  }
-  attn_consumer_sync();
-  // O^T element (dim tile d, row tile rt, k): dim 32*warp + 2g + d (+16 for
-  // k >= 2), row 8*rt + 2t + (k & 1)
-  const size_t rows_total = size_t(a.M) * a.n_q;
-  #pragma unroll
-  for (int rt = 0; rt < NRT; ++rt)
-    #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int r = 8 * rt + 2 * t + (k & 1);
-      if (r >= R) continue;
-      const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
-      const size_t row = size_t(m) * a.n_q + kh * a.g + j;
-      #pragma unroll
-      for (int d = 0; d < 2; ++d) {
-        const int dim = 32 * warp + 2 * g + d + (k >= 2 ? 16 : 0);
-        if (a.n_splits == 1) {
-          a.out[row * kHeadDim + dim] = o[d][rt][k] / row_sum[r];
-        } else {
-          a.ws_o[(size_t(split) * rows_total + row) * kHeadDim + dim] = o[d][rt][k];
-        }
-      }
-      if (a.n_splits > 1 && warp == 0 && g == 0 && k < 2) {
-        a.ws_ml[(size_t(split) * rows_total + row) * 2 + 0] = m_run[rt][k];
-        a.ws_ml[(size_t(split) * rows_total + row) * 2 + 1] = row_sum[r];
-      }
-    }
 }
 
 // Log-sum-exp merge of the per-split states (base 2); one CTA of eight warps

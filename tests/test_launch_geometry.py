@@ -99,7 +99,7 @@ ATTN_CASES = [(4096, 24, 4, 1), (4096, 24, 4, 5), (65536, 24, 4, 5), (262144, 24
               (1000, 8, 1, 5), (300, 64, 4, 5), (129, 4, 4, 2), (70000, 48, 1, 5)]
 
 
-TT_ATTN, Q_PITCH, PT_PITCH, ROW = 128, 576, 80, 144
+TT_ATTN, Q_PITCH, ROW = 128, 576, 144
 TT_R8, WARPS_R8 = 192, 12          # warp-local variant (at most 8 rows per CTA)
 
 
@@ -140,26 +140,25 @@ def _chunks(addrs):
 
 
 def test_attn_shared_memory_banks():
-    # K ldmatrix: eight token rows at a 144-byte pitch, same column
-    for col in range(0, 128, 16):
+    # K ldmatrix (warp-local kernel) and 16-byte row loads (tensor-memory
+    # kernel): eight token rows at a 144-byte pitch, same column
+    for col in range(0, 144, 16):
         assert len(_chunks([r * ROW + col for r in range(8)])) == 8
-    # P^T ldmatrix.trans: eight token rows at an 80-byte pitch
-    for col in range(0, 64, 16):
-        assert len(_chunks([r * PT_PITCH + col for r in range(8)])) == 8
-    # P^T stores: lane (g, t) writes 4 bytes at token g, rows 2t..2t+1
-    for rt in range(4):
-        banks = {((g * PT_PITCH + (8 * rt + 2 * t) * 2) // 4) % 32 for g in range(8) for t in range(4)}
-        assert len(banks) == 32
     # Q fragment loads (16 bytes per lane): each group of eight lanes covers
     # eight distinct 16-byte bank groups
-    for rt in range(4):
-        for blk in range(8):
-            for q in range(4):
-                lanes = range(8 * q, 8 * q + 8)
-                assert len(_chunks([(8 * rt + (ln >> 2)) * Q_PITCH + (blk * 4 + (ln & 3)) * 16
-                                    for ln in lanes])) == 8
+    for blk in range(8):
+        for q in range(4):
+            lanes = range(8 * q, 8 * q + 8)
+            assert len(_chunks([(ln >> 2) * Q_PITCH + (blk * 4 + (ln & 3)) * 16
+                                for ln in lanes])) == 8
     # block scales in the score step: tokens g at a 144-byte pitch, distinct banks
     assert len({((g * ROW + 128) // 4) % 32 for g in range(8)}) == 8
+    # tensor-memory kernel: V-tile and P^T stores, lane = token k of a 32-token
+    # quadrant, 16 bytes at (k >> 3) * 128 + (k & 7) * 16 from the chunk base
+    for quad in range(4):
+        for phase in range(4):
+            ks = [32 * quad + 8 * phase + i for i in range(8)]
+            assert len(_chunks([(k >> 3) * 128 + (k & 7) * 16 for k in ks])) == 8
 
 
 @pytest.mark.parametrize("ctx,nq,nkv,M", ATTN_CASES)
