@@ -620,28 +620,35 @@ def per_call_table(torch, L, dev, layers, kv, ws, peak_gbs, reps=15):
     # fused gate / up + SwiGLU (one 2 x 17408 x 5120 interleaved matrix) vs the
     # two separate 5120 -> 17408 GEMVs of the table above
     import synth
+    from bit_weight_streaming_dequant_b200 import q4dec
     Wgu = [synth.device_q4_0_weights(7000 + i, 2 * FFN, HIDDEN, device=dev) for i in range(2)]
     table["gate_up_swiglu"] = []
     for M in (1, 5):
         x = torch.randn((M, HIDDEN), device=dev).to(torch.bfloat16)
-        h = torch.empty((M, FFN), dtype=torch.float32, device=dev)
-        times = []
-        for r in range(reps + 2):
-            flush.fill_(r & 0xFF)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            st = L.q4_gemv_swiglu_ex(Wgu[r % 2].data_ptr(), x.data_ptr(), h.data_ptr(), M, FFN,
-                                     HIDDEN, sptr, ws.data_ptr(), ws.numel(), 0)
-            b.record(stream)
-            if st:
-                raise RuntimeError(f"q4_gemv_swiglu_ex failed: {st}")
-            torch.cuda.synchronize()
-            if r >= 2:
-                times.append(a.elapsed_time(b) * 1e3)
-        us = statistics.median(times)
+        row = {"M": M}
+        # fp32 h, and bf16 h (Q4D_GEMV_OUT_BF16: the down projection's input format)
+        for key, dt, flags in (("us", torch.float32, 0),
+                               ("us_bf16_out", torch.bfloat16, q4dec.GEMV_OUT_BF16)):
+            h = torch.empty((M, FFN), dtype=dt, device=dev)
+            times = []
+            for r in range(reps + 2):
+                flush.fill_(r & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                st = L.q4_gemv_swiglu_ex(Wgu[r % 2].data_ptr(), x.data_ptr(), h.data_ptr(), M,
+                                         FFN, HIDDEN, sptr, ws.data_ptr(), ws.numel(), flags)
+                b.record(stream)
+                if st:
+                    raise RuntimeError(f"q4_gemv_swiglu_ex failed: {st}")
+                torch.cuda.synchronize()
+                if r >= 2:
+                    times.append(a.elapsed_time(b) * 1e3)
+            row[key] = statistics.median(times)
+        us = row["us"]
         gbs = (2 * q4_bytes(FFN, HIDDEN) + 2 * M * HIDDEN + 4 * M * FFN) / (us * 1e-6) / 1e9
-        table["gate_up_swiglu"].append({"M": M, "us": us, "GBps": gbs, "frac": gbs / peak_gbs,
-                                        "separate_gate_plus_up_us": 2 * by[("5120->17408", M)]})
+        row.update({"GBps": gbs, "frac": gbs / peak_gbs,
+                    "separate_gate_plus_up_us": 2 * by[("5120->17408", M)]})
+        table["gate_up_swiglu"].append(row)
     del Wgu
     # K/V append of M verified tokens (4 KV heads), a small cache of its own
     stride = 4096

@@ -44,6 +44,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include "q4dec_device.cuh"
 
@@ -60,6 +61,7 @@ struct alignas(64) GemvArgs {
   const uint8_t* W;    // super-block-column-major weights, [K/256][N] x 144 B
   float* out;          // y [M][N] or partials [k_splits][M][N]
   unsigned* err;
+  int out_bf16;        // 1: y (no K split) is stored as bf16 [M][N], rounded to nearest even
   int N;
   int sb_per_split;    // super-blocks per K range
   int rows_per_pass;   // multiple of 16, <= 128
@@ -95,6 +97,15 @@ __host__ __device__ constexpr uint32_t gemv_wbox_bytes(int rows_per_pass) {
 }
 __host__ __device__ constexpr uint32_t gemv_stage_bytes(int M, int KC, int rows_per_pass) {
   return uint32_t(KC) * (gemv_wbox_bytes(rows_per_pass) + uint32_t(M) * 512u);
+}
+
+// Element i of the output: fp32, or bf16 (round to nearest even) when the
+// caller asked for bf16 outputs.  Partials of a K split are always fp32.
+__device__ __forceinline__ void store_out(float* out, size_t i, float v, int bf16) {
+  if (bf16)
+    reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
+  else
+    out[i] = v;
 }
 
 constexpr int kConsumerWarps = 8;
@@ -351,12 +362,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       for (int i = tid; i < (nr >> 1) * M; i += kConsumerWarps * 32) {
         const int j = i / M, m = i - (i / M) * M;
         const float g = row_sum(2 * j, m), u = row_sum(2 * j + 1, m);
-        a.out[size_t(m) * (a.N >> 1) + ((r0 >> 1) + j)] = g / (1.f + __expf(-g)) * u;
+        store_out(a.out, size_t(m) * (a.N >> 1) + ((r0 >> 1) + j), g / (1.f + __expf(-g)) * u,
+                  a.out_bf16);
       }
     } else {
       for (int i = tid; i < nr * M; i += kConsumerWarps * 32) {
         const int r = i / M, m = i - (i / M) * M;
-        a.out[(size_t(ks) * M + m) * a.N + r0 + r] = row_sum(r, m);
+        store_out(a.out, (size_t(ks) * M + m) * a.N + r0 + r, row_sum(r, m), a.out_bf16);
       }
     }
     consumer_sync();  // red is rewritten at the next pass end
@@ -366,7 +378,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 // h[m][n] = silu(g) * u from the partials of the 2N gate / up rows, each
 // summed over the K ranges in range order.
 __global__ void q4_gemv_splitk_reduce_swiglu(const float* __restrict__ ws, float* __restrict__ h,
-                                             int M, int N, int k_splits) {
+                                             int M, int N, int k_splits, int out_bf16) {
   if (threadIdx.x == 0) griddep_launch_dependents();
   const long long mn = (long long)M * N, rows = 2LL * N;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < mn;
@@ -377,19 +389,19 @@ __global__ void q4_gemv_splitk_reduce_swiglu(const float* __restrict__ ws, float
       g += ws[(k * M + m) * rows + 2 * n];
       u += ws[(k * M + m) * rows + 2 * n + 1];
     }
-    h[i] = g / (1.f + __expf(-g)) * u;
+    store_out(h, size_t(i), g / (1.f + __expf(-g)) * u, out_bf16);
   }
 }
 
 // y[i] = sum over K ranges of the partials, in range order.
 __global__ void q4_gemv_splitk_reduce(const float* __restrict__ ws, float* __restrict__ y,
-                                      long long mn, int k_splits) {
+                                      long long mn, int k_splits, int out_bf16) {
   if (threadIdx.x == 0) griddep_launch_dependents();
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < mn;
        i += (long long)gridDim.x * blockDim.x) {
     float s = 0.f;
     for (int k = 0; k < k_splits; ++k) s += ws[k * mn + i];
-    y[i] = s;
+    store_out(y, size_t(i), s, out_bf16);
   }
 }
 

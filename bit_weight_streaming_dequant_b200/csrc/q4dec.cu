@@ -261,14 +261,16 @@ q4d_status launch_gemv_t(const q4d::GemvArgs& a, const q4d_gemv_plan& p, int dev
 
 // y = W x (rows = N), or with `swiglu` h[m][n] = silu(g) * u over the N gate /
 // up row pairs of W (2N rows).
-q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, int K,
+q4d_status gemv_impl(const void* W_q4, const void* x, void* y, int M, int N, int K,
                      cudaStream_t stream, void* workspace, size_t workspace_bytes,
-                     bool library_ws, bool pdl = false, bool swiglu = false) {
+                     bool library_ws, bool pdl = false, bool swiglu = false,
+                     bool out_bf16 = false) {
   if (swiglu && N > (1 << 29)) return Q4D_ERR_UNSUPPORTED_SHAPE;
   q4d_status st = check_gemv_shape(M, swiglu ? 2 * N : N, K);
   if (st != Q4D_OK) return st;
   if (!W_q4 || !x || !y) return Q4D_ERR_INVALID_ARG;
-  if (!aligned(W_q4, 16) || !aligned(x, 16) || !aligned(y, 4)) return Q4D_ERR_MISALIGNED;
+  if (!aligned(W_q4, 16) || !aligned(x, 16) || !aligned(y, out_bf16 ? 2 : 4))
+    return Q4D_ERR_MISALIGNED;
   if (workspace && !aligned(workspace, 16)) return Q4D_ERR_MISALIGNED;
 
   int dev = 0;
@@ -290,7 +292,8 @@ q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, in
                           uint64_t(K) * 2u, 256u, uint32_t(M))) != Q4D_OK)
     return st;
   a.W = static_cast<const uint8_t*>(W_q4);
-  a.out = p.k_splits > 1 ? static_cast<float*>(workspace) : y;
+  a.out = p.k_splits > 1 ? static_cast<float*>(workspace) : static_cast<float*>(y);
+  a.out_bf16 = (out_bf16 && p.k_splits == 1) ? 1 : 0;
   a.err = s->err;
   a.N = rows;
   a.sb_per_split = p.sb_per_split;
@@ -321,10 +324,12 @@ q4d_status gemv_impl(const void* W_q4, const void* x, float* y, int M, int N, in
     const int blocks = int(std::min<long long>((mn + 255) / 256, 4LL * s->num_sms));
     if (swiglu)
       q4d::q4_gemv_splitk_reduce_swiglu<<<blocks, 256, 0, stream>>>(
-          static_cast<const float*>(workspace), y, M, N, p.k_splits);
+          static_cast<const float*>(workspace), static_cast<float*>(y), M, N, p.k_splits,
+          out_bf16 ? 1 : 0);
     else
-      q4d::q4_gemv_splitk_reduce<<<blocks, 256, 0, stream>>>(static_cast<const float*>(workspace),
-                                                            y, mn, p.k_splits);
+      q4d::q4_gemv_splitk_reduce<<<blocks, 256, 0, stream>>>(
+          static_cast<const float*>(workspace), static_cast<float*>(y), mn, p.k_splits,
+          out_bf16 ? 1 : 0);
   }
   if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
   return Q4D_OK;
@@ -505,19 +510,21 @@ q4d_status q4_gemv_ex(const void* W_q4, const void* x, float* y, int M, int N, i
                    workspace_bytes, false);
 }
 
-q4d_status q4_gemv_ex2(const void* W_q4, const void* x, float* y, int M, int N, int K,
+q4d_status q4_gemv_ex2(const void* W_q4, const void* x, void* y, int M, int N, int K,
                        void* stream, void* workspace, size_t workspace_bytes, unsigned flags) {
-  if (flags & ~Q4D_GEMV_WEIGHT_PREFETCH) return Q4D_ERR_INVALID_ARG;
+  if (flags & ~(Q4D_GEMV_WEIGHT_PREFETCH | Q4D_GEMV_OUT_BF16)) return Q4D_ERR_INVALID_ARG;
   return gemv_impl(W_q4, x, y, M, N, K, static_cast<cudaStream_t>(stream), workspace,
-                   workspace_bytes, false, (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0);
+                   workspace_bytes, false, (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0, false,
+                   (flags & Q4D_GEMV_OUT_BF16) != 0);
 }
 
-q4d_status q4_gemv_swiglu_ex(const void* W_gu, const void* x, float* h, int M, int N, int K,
+q4d_status q4_gemv_swiglu_ex(const void* W_gu, const void* x, void* h, int M, int N, int K,
                              void* stream, void* workspace, size_t workspace_bytes,
                              unsigned flags) {
-  if (flags & ~Q4D_GEMV_WEIGHT_PREFETCH) return Q4D_ERR_INVALID_ARG;
+  if (flags & ~(Q4D_GEMV_WEIGHT_PREFETCH | Q4D_GEMV_OUT_BF16)) return Q4D_ERR_INVALID_ARG;
   return gemv_impl(W_gu, x, h, M, N, K, static_cast<cudaStream_t>(stream), workspace,
-                   workspace_bytes, false, (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0, true);
+                   workspace_bytes, false, (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0, true,
+                   (flags & Q4D_GEMV_OUT_BF16) != 0);
 }
 
 size_t q4d_gemv_swiglu_workspace_bytes(int M, int N, int K) {

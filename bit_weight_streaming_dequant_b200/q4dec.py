@@ -191,14 +191,25 @@ def _workspace(nbytes: int, device, workspace):
 
 
 GEMV_WEIGHT_PREFETCH = 1  # Q4D_GEMV_WEIGHT_PREFETCH
+GEMV_OUT_BF16 = 2         # Q4D_GEMV_OUT_BF16
+
+
+def _out_flags(out_dtype, torch):
+    if out_dtype == torch.float32:
+        return 0
+    if out_dtype == torch.bfloat16:
+        return GEMV_OUT_BF16
+    raise ValueError("out_dtype must be torch.float32 or torch.bfloat16")
 
 
 def q4_gemv(W, x, y=None, *, N: int, K: int, stream=None, workspace=None,
-            weight_prefetch: bool = False):
-    """y[M][N] (fp32) = dequant(W)[N][K] @ x[M][K]^T via ``q4_gemv_ex2``.
+            weight_prefetch: bool = False, out_dtype=None):
+    """y[M][N] = dequant(W)[N][K] @ x[M][K]^T via ``q4_gemv_ex2``.
 
     ``W``: uint8 CUDA tensor with N*K/256*144 bytes (super-block layout);
-    ``x``: bf16 CUDA tensor [M][K]; ``y``: optional fp32 [M][N] output.
+    ``x``: bf16 CUDA tensor [M][K]; ``y``: optional [M][N] output.
+    ``out_dtype``: torch.float32 (default) or torch.bfloat16 (Q4D_GEMV_OUT_BF16:
+    the fp32 result rounded to nearest even); taken from ``y`` when given.
     ``weight_prefetch``: Q4D_GEMV_WEIGHT_PREFETCH (programmatic dependent
     launch; W must not be written by earlier kernels still in flight).
     """
@@ -210,9 +221,12 @@ def q4_gemv(W, x, y=None, *, N: int, K: int, stream=None, workspace=None,
     M = x.shape[0]
     if W.numel() != N * (K // 256) * 144:
         raise ValueError("W has the wrong number of bytes for N x K")
+    if out_dtype is None:
+        out_dtype = torch.float32 if y is None else y.dtype
+    flags = _out_flags(out_dtype, torch) | (GEMV_WEIGHT_PREFETCH if weight_prefetch else 0)
     if y is None:
-        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
-    _dev_tensor(y, torch.float32, "y")
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _dev_tensor(y, out_dtype, "y")
     if tuple(y.shape) != (M, N):
         raise ValueError("y must be [M][N]")
     with torch.cuda.device(x.device):
@@ -220,15 +234,16 @@ def q4_gemv(W, x, y=None, *, N: int, K: int, stream=None, workspace=None,
         ws = _workspace(need, x.device, workspace)
         st = lib().q4_gemv_ex2(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K,
                                _stream_ptr(stream), None if ws is None else ws.data_ptr(), need,
-                               GEMV_WEIGHT_PREFETCH if weight_prefetch else 0)
+                               flags)
     _check(st, "q4_gemv")
     return y
 
 
 def q4_gemv_swiglu(W_gu, x, h=None, *, N: int, K: int, stream=None, workspace=None,
-                   weight_prefetch: bool = False):
-    """h[M][N] (fp32) = silu(gate) * up from one interleaved gate / up matrix
-    ``W_gu`` (2N rows: gate n at row 2n, up n at 2n + 1) via ``q4_gemv_swiglu_ex``."""
+                   weight_prefetch: bool = False, out_dtype=None):
+    """h[M][N] = silu(gate) * up from one interleaved gate / up matrix
+    ``W_gu`` (2N rows: gate n at row 2n, up n at 2n + 1) via ``q4_gemv_swiglu_ex``;
+    ``out_dtype`` as for :func:`q4_gemv`."""
     torch = _torch()
     _dev_tensor(W_gu, torch.uint8, "W_gu")
     _dev_tensor(x, torch.bfloat16, "x")
@@ -237,9 +252,12 @@ def q4_gemv_swiglu(W_gu, x, h=None, *, N: int, K: int, stream=None, workspace=No
     M = x.shape[0]
     if W_gu.numel() != 2 * N * (K // 256) * 144:
         raise ValueError("W_gu has the wrong number of bytes for 2N x K")
+    if out_dtype is None:
+        out_dtype = torch.float32 if h is None else h.dtype
+    flags = _out_flags(out_dtype, torch) | (GEMV_WEIGHT_PREFETCH if weight_prefetch else 0)
     if h is None:
-        h = torch.empty((M, N), dtype=torch.float32, device=x.device)
-    _dev_tensor(h, torch.float32, "h")
+        h = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _dev_tensor(h, out_dtype, "h")
     if tuple(h.shape) != (M, N):
         raise ValueError("h must be [M][N]")
     with torch.cuda.device(x.device):
@@ -247,7 +265,7 @@ def q4_gemv_swiglu(W_gu, x, h=None, *, N: int, K: int, stream=None, workspace=No
         ws = _workspace(need, x.device, workspace)
         st = lib().q4_gemv_swiglu_ex(W_gu.data_ptr(), x.data_ptr(), h.data_ptr(), M, N, K,
                                      _stream_ptr(stream), None if ws is None else ws.data_ptr(),
-                                     need, GEMV_WEIGHT_PREFETCH if weight_prefetch else 0)
+                                     need, flags)
     _check(st, "q4_gemv_swiglu")
     return h
 

@@ -42,7 +42,7 @@
  *   - Every pointer passed to a compute entry point is a DEVICE pointer of
  *     the current CUDA device, owned by the caller; the library never frees
  *     or retains it.  W, x, Q, K, V and workspace must be 16-byte aligned;
- *     y and out must be 4-byte aligned.
+ *     y and out must be 4-byte aligned (2-byte for bf16 outputs).
  *   - "stream" is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Work is enqueued asynchronously; the library never
  *     synchronises the host on the compute path.
@@ -103,8 +103,8 @@ q4d_status q4_gemv(const void* W_q4, const void* x, float* y, int M, int N, int 
 q4d_status q4_gemv_ex(const void* W_q4, const void* x, float* y, int M, int N, int K,
                       void* stream, void* workspace, size_t workspace_bytes);
 
-/* q4_gemv_ex2: q4_gemv_ex plus launch flags (0 behaves exactly as q4_gemv_ex;
- * any other bit is Q4D_ERR_INVALID_ARG).
+/* q4_gemv_ex2: q4_gemv_ex plus flags (0 behaves exactly as q4_gemv_ex; a bit
+ * other than the two below is Q4D_ERR_INVALID_ARG).
  *
  *   Q4D_GEMV_WEIGHT_PREFETCH: launch with programmatic dependent launch.  The
  *   kernel's CTAs may start while the kernel before it on the stream is still
@@ -117,7 +117,16 @@ q4d_status q4_gemv_ex(const void* W_q4, const void* x, float* y, int M, int N, i
  *   this library.
  */
 #define Q4D_GEMV_WEIGHT_PREFETCH 1u
-q4d_status q4_gemv_ex2(const void* W_q4, const void* x, float* y, int M, int N, int K,
+/*   Q4D_GEMV_OUT_BF16: y is bf16 [M][N] (2 bytes per element, 2-byte
+ *   aligned) instead of fp32: each element is the fp32 result of the plain
+ *   call rounded to nearest even -- bit for bit the fp32 output converted --
+ *   so that a GEMV's output can feed the next GEMV's bf16 activations
+ *   directly.  A K split still reduces its partials in fp32 (the workspace
+ *   size does not change).  No counterpart in the source pages, which keep
+ *   activations in 16 bits between layers without fixing the format.
+ */
+#define Q4D_GEMV_OUT_BF16 2u
+q4d_status q4_gemv_ex2(const void* W_q4, const void* x, void* y, int M, int N, int K,
                        void* stream, void* workspace, size_t workspace_bytes, unsigned flags);
 
 /* q4_gemv_swiglu_ex: fused gate / up projections with the SwiGLU epilogue of
@@ -127,13 +136,14 @@ q4d_status q4_gemv_ex2(const void* W_q4, const void* x, float* y, int M, int N, 
  *   W_gu : 2N x K elements of Q4_0 in the weight layout above, the gate row n
  *          stored as row 2n and the up row n as row 2n + 1 (interleaved).
  *   x    : bf16 [M][K];  h : fp32 [M][N] = silu(g) * u, silu(g) = g / (1 + e^-g),
- *          g and u the fp32 gate / up outputs of row pair n.
+ *          g and u the fp32 gate / up outputs of row pair n (bf16 [M][N] with
+ *          Q4D_GEMV_OUT_BF16: the fp32 h rounded to nearest even).
  *   Requirements as q4_gemv (with 2N rows); workspace of at least
  *   q4d_gemv_swiglu_workspace_bytes(M, N, K) bytes; flags as q4_gemv_ex2.
  * One weight stream and one launch (plus a reduction launch when K is split)
  * instead of two GEMVs and an elementwise pass.
  */
-q4d_status q4_gemv_swiglu_ex(const void* W_gu, const void* x, float* h, int M, int N, int K,
+q4d_status q4_gemv_swiglu_ex(const void* W_gu, const void* x, void* h, int M, int N, int K,
                              void* stream, void* workspace, size_t workspace_bytes,
                              unsigned flags);
 size_t q4d_gemv_swiglu_workspace_bytes(int M, int N, int K);

@@ -50,12 +50,19 @@ def test_gemv_rejects_bad_shapes_without_cuda(M, N, K, code):
 
 def test_gemv_ex2_rejects_unknown_flags_and_bad_shapes_without_cuda():
     L = q4dec.lib()
-    for flags in (2, 4, 0x80000000, 3):
+    for flags in (4, 0x80000000, 5, 7):
         assert L.q4_gemv_ex2(FAKE, FAKE, FAKE, 1, 16, 256, None, None, 0, flags) == 1
-    for flags in (0, q4dec.GEMV_WEIGHT_PREFETCH):
+        assert L.q4_gemv_swiglu_ex(FAKE, FAKE, FAKE, 1, 16, 256, None, None, 0, flags) == 1
+    bf16 = q4dec.GEMV_OUT_BF16
+    for flags in (0, q4dec.GEMV_WEIGHT_PREFETCH, bf16, bf16 | q4dec.GEMV_WEIGHT_PREFETCH):
         assert L.q4_gemv_ex2(FAKE, FAKE, FAKE, 6, 16, 256, None, None, 0, flags) == 2
         assert L.q4_gemv_ex2(FAKE + 8, FAKE, FAKE, 1, 16, 256, None, None, 0, flags) == 3
         assert L.q4_gemv_ex2(None, FAKE, FAKE, 1, 16, 256, None, None, 0, flags) == 1
+        # y: 4-byte alignment for fp32 outputs, 2-byte for bf16
+        assert L.q4_gemv_ex2(FAKE, FAKE, FAKE + 1, 1, 16, 256, None, None, 0, flags) == 3
+        assert L.q4_gemv_swiglu_ex(FAKE, FAKE, FAKE + 1, 1, 16, 256, None, None, 0, flags) == 3
+    for flags in (0, q4dec.GEMV_WEIGHT_PREFETCH):
+        assert L.q4_gemv_ex2(FAKE, FAKE, FAKE + 2, 1, 16, 256, None, None, 0, flags) == 3
 
 
 def test_gemv_rejects_null_and_misaligned_pointers():
@@ -133,7 +140,7 @@ def test_append_rejects_bad_arguments_without_cuda():
 
 def test_swiglu_rejects_bad_arguments_without_cuda():
     L = q4dec.lib()
-    assert L.q4_gemv_swiglu_ex(FAKE, FAKE, FAKE, 1, 16, 256, None, None, 0, 2) == 1
+    assert L.q4_gemv_swiglu_ex(FAKE, FAKE, FAKE, 1, 16, 256, None, None, 0, 4) == 1
     assert L.q4_gemv_swiglu_ex(None, FAKE, FAKE, 1, 16, 256, None, None, 0, 0) == 1
     assert L.q4_gemv_swiglu_ex(FAKE, FAKE, FAKE, 6, 16, 256, None, None, 0, 0) == 2
     assert L.q4_gemv_swiglu_ex(FAKE, FAKE, FAKE, 1, 16, 100, None, None, 0, 0) == 2
