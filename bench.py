@@ -46,8 +46,10 @@ def gemv_alg_bytes(M, N, K):
     return q4_bytes(N, K) + 2 * M * K + 4 * M * N
 
 
-def attn_alg_bytes(M, ctx):
-    return 2 * N_KV * ctx * 144 + M * N_Q * HEAD_DIM * (2 + 4)
+def attn_alg_bytes(M, ctx, row_bytes=144):
+    """K and V rows (144 B per token and KV head for Q4_0, 272 B for Q8_0)
+    plus the bf16 queries and fp32 outputs."""
+    return 2 * N_KV * ctx * row_bytes + M * N_Q * HEAD_DIM * (2 + 4)
 
 
 def peaks():
@@ -561,7 +563,9 @@ def per_call_table(torch, L, dev, layers, kv, ws, peak_gbs, reps=15):
     need = max([L.q4d_gemv_workspace_bytes(M, N, K) for M in range(1, 6)
                 for N, K in LAYER_SHAPES] +
                [L.q4d_attn_workspace_bytes(c, N_Q, N_KV, HEAD_DIM, M) for M in (1, 5)
-                for c in (4096, 65536, CTX)] + [16])
+                for c in (4096, 65536, CTX)] +
+               [L.q8kv_attn_workspace_bytes(c, N_Q, N_KV, HEAD_DIM, M) for M in (1, 5)
+                for c in (65536, CTX)] + [16])
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     sptr = stream.cuda_stream
@@ -614,6 +618,35 @@ def per_call_table(torch, L, dev, layers, kv, ws, peak_gbs, reps=15):
             gbs = attn_alg_bytes(M, ctx) / (us * 1e-6) / 1e9
             table["attn"].append({"ctx": ctx, "M": M, "us": us, "GBps": gbs,
                                   "frac": gbs / peak_gbs})
+    # the same attention over the Q8_0 cache (272-byte rows), own caches
+    import synth
+    kv8 = [(synth.device_q8_0_kv_cache(9000 + 2 * i, N_KV, CTX, device=dev),
+            synth.device_q8_0_kv_cache(9001 + 2 * i, N_KV, CTX, device=dev)) for i in range(2)]
+    table["attn_q8"] = []
+    for ctx in (65536, 262144):
+        for M in (1, 5):
+            Q = torch.randn((M, N_Q, HEAD_DIM), device=dev).div_(16).to(torch.bfloat16)
+            out = torch.empty((M, N_Q, HEAD_DIM), dtype=torch.float32, device=dev)
+            times = []
+            for r in range(reps + 2):
+                Kc, Vc = kv8[r % len(kv8)]
+                flush.fill_(r & 0xFF)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                st = L.q8kv_attn_decode_ex(Q.data_ptr(), Kc.data_ptr(), Vc.data_ptr(),
+                                           out.data_ptr(), ctx, N_Q, N_KV, HEAD_DIM, M, CTX,
+                                           1.0, sptr, ws.data_ptr(), ws.numel())
+                b.record(stream)
+                if st:
+                    raise RuntimeError(f"q8kv_attn_decode_ex failed: {st}")
+                torch.cuda.synchronize()
+                if r >= 2:
+                    times.append(a.elapsed_time(b) * 1e3)
+            us = statistics.median(times)
+            gbs = attn_alg_bytes(M, ctx, 272) / (us * 1e-6) / 1e9
+            table["attn_q8"].append({"ctx": ctx, "M": M, "us": us, "GBps": gbs,
+                                     "frac": gbs / peak_gbs})
+    del kv8
     # t(M=5) / t(M=1) per GEMV shape: about 1 is what makes verification cheap
     by = {(r["shape"], r["M"]): r["us"] for r in table["gemv"]}
     table["gemv_m5_over_m1"] = {name: by[(name, 5)] / by[(name, 1)] for name in names.values()}

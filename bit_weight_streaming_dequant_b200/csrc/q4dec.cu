@@ -28,6 +28,9 @@ constexpr int kMaxDevices = 64;
 constexpr int kPlanFallbackSms = 148;
 constexpr size_t kGemvSmemBudget = 224 * 1024;   // shared memory per GEMV CTA
 constexpr size_t kAttnSmemBudget = 224 * 1024;   // shared memory per attention CTA
+// The 8-bit cache's 70 KB ring stages need the device's whole opt-in shared
+// memory per block (227 KB on B200) for two stages next to the V tile.
+constexpr size_t kAttnSmemMax = 227 * 1024;
 
 struct DeviceState {
   std::atomic<bool> ready{false};
@@ -346,22 +349,30 @@ q4d_status launch_attn_rows8(const q4d::AttnArgs& a, const q4d_attn_plan& p, int
   return Q4D_OK;
 }
 
-// The tensor-memory kernel with NR (16 or 32) MMA columns of query rows.
-template <int NR>
+// The tensor-memory kernel with NR (16 or 32) MMA columns of query rows, the
+// Q4 or Q8 cache and PB P^T buffers.
+template <int NR, bool Q8, int PB>
 q4d_status launch_attn_tc(const q4d::AttnArgs& a, const q4d_attn_plan& p, int n_kv, int dev,
                           const DeviceState& s, cudaStream_t stream) {
   static std::atomic<bool> smem_set[kMaxDevices];
-  q4d_status st = allow_smem(q4d::q4kv_attn_tc_kernel<NR>, dev, s, smem_set);
+  q4d_status st = allow_smem(q4d::q4kv_attn_tc_kernel<NR, Q8, PB>, dev, s, smem_set);
   if (st != Q4D_OK) return st;
   dim3 grid(p.n_splits, n_kv, p.row_groups);
-  q4d::q4kv_attn_tc_kernel<NR><<<grid, p.threads, p.smem_bytes, stream>>>(a);
+  q4d::q4kv_attn_tc_kernel<NR, Q8, PB><<<grid, p.threads, p.smem_bytes, stream>>>(a);
   return Q4D_OK;
 }
+
+// P^T buffers of the tensor-memory kernel: two, except for the 8-bit cache
+// with 32 MMA columns, whose shared memory holds only one next to two stages.
+int tca_pbufs(int nr, bool q8) { return (q8 && nr == 32) ? 1 : 2; }
+
+q4d_status plan_attn_impl(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
+                          int num_sms, bool q8, q4d_attn_plan* plan);
 
 q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out, int ctx_len,
                      int n_q, int n_kv, int head_dim, int M, int kv_stride, float scale,
                      cudaStream_t stream, void* workspace, size_t workspace_bytes,
-                     bool library_ws) {
+                     bool library_ws, bool q8 = false) {
   q4d_status st = check_attn_shape(ctx_len, n_q, n_kv, head_dim, M, kv_stride, scale);
   if (st != Q4D_OK) return st;
   if (!Q || !Kq4 || !Vq4 || !out) return Q4D_ERR_INVALID_ARG;
@@ -373,7 +384,8 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
   DeviceState* s = nullptr;
   if ((st = current_device(&dev, &s)) != Q4D_OK) return st;
   q4d_attn_plan p;
-  if ((st = q4d_plan_attn(ctx_len, n_q, n_kv, head_dim, M, s->num_sms, &p)) != Q4D_OK) return st;
+  if ((st = plan_attn_impl(ctx_len, n_q, n_kv, head_dim, M, s->num_sms, q8, &p)) != Q4D_OK)
+    return st;
   if (p.smem_bytes > size_t(s->smem_optin)) return Q4D_ERR_UNSUPPORTED_SHAPE;
   if (library_ws) {
     if ((st = library_workspace(*s, p.workspace_bytes, &workspace)) != Q4D_OK) return st;
@@ -402,12 +414,14 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
   a.rows_per_cta = p.rows_per_cta;
   a.stages = p.stages;
 
-  if (p.rows_per_cta <= 8)
+  if (!q8 && p.rows_per_cta <= 8)
     st = launch_attn_rows8(a, p, n_kv, dev, *s, stream);
   else if (p.rows_per_cta <= 16)
-    st = launch_attn_tc<16>(a, p, n_kv, dev, *s, stream);
+    st = q8 ? launch_attn_tc<16, true, 2>(a, p, n_kv, dev, *s, stream)
+            : launch_attn_tc<16, false, 2>(a, p, n_kv, dev, *s, stream);
   else
-    st = launch_attn_tc<32>(a, p, n_kv, dev, *s, stream);
+    st = q8 ? launch_attn_tc<32, true, 1>(a, p, n_kv, dev, *s, stream)
+            : launch_attn_tc<32, false, 2>(a, p, n_kv, dev, *s, stream);
   if (st != Q4D_OK) return st;
   if (p.n_splits > 1) q4d::q4kv_attn_merge_kernel<<<M * n_q, 256, 0, stream>>>(a);
   if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
@@ -446,19 +460,35 @@ q4d_status q4d_plan_gemv(int M, int N, int K, int num_sms, q4d_gemv_plan* plan) 
 
 q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
                          int num_sms, q4d_attn_plan* plan) {
+  return plan_attn_impl(ctx_len, n_q_heads, n_kv_heads, head_dim, M, num_sms, false, plan);
+}
+
+q4d_status q8kv_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
+                          int num_sms, q4d_attn_plan* plan) {
+  return plan_attn_impl(ctx_len, n_q_heads, n_kv_heads, head_dim, M, num_sms, true, plan);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Variant: warp-local mma.sync kernel (12 warps, 192-token tiles) for at
+// most 8 rows per CTA of the Q4 cache, else the tensor-memory kernel (8 token
+// warps, a producer warp and an MMA warp; 128-token tiles; 16 or 32 MMA
+// columns), which also serves every row count of the Q8 cache.
+q4d_status plan_attn_impl(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
+                          int num_sms, bool q8, q4d_attn_plan* plan) {
   if (!plan || num_sms < 1) return Q4D_ERR_INVALID_ARG;
   q4d_status st = check_attn_shape(ctx_len, n_q_heads, n_kv_heads, head_dim, M, ctx_len, 1.0f);
   if (st != Q4D_OK) return st;
   const int rows_all = (n_q_heads / n_kv_heads) * M;
   const int row_groups = ceil_div(rows_all, q4d::kAttnMaxRows);
   const int rows_per_cta = ceil_div(rows_all, row_groups);
-  // Variant: warp-local mma.sync kernel (12 warps, 192-token tiles) for at
-  // most 8 rows per CTA, else the tensor-memory kernel (8 token warps, a
-  // producer warp and an MMA warp; 128-token tiles; 16 or 32 MMA columns).
-  const bool rows8 = rows_per_cta <= 8;
+  const bool rows8 = !q8 && rows_per_cta <= 8;
   const int nr = rows_per_cta <= 16 ? 16 : 32;
+  const int pb = tca_pbufs(nr, q8);
   const int TT = rows8 ? q4d::kR8Tile : q4d::kTcaTile;
-  const size_t stage_bytes = rows8 ? q4d::kR8StageBytes : q4d::kTcaStage;
+  const size_t stage_bytes = rows8 ? q4d::kR8StageBytes : q4d::tca_stage_bytes(q8);
   // One CTA per SM (the K/V ring takes most of shared memory): enough context
   // splits that (splits x KV heads x row groups) fills the SMs once, each
   // split at least two tiles long and at most 256 splits (the merge kernel's
@@ -471,8 +501,9 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   n_splits = ceil_div(ctx_len, split_tokens);
   // As many ring stages as fit next to the variant's fixed buffers, up to 8
   // (at least 2: the warp-local variant parks 96 KB in the ring at the end).
-  const size_t fixed = rows8 ? q4d::attn_rows8_smem_bytes(0) : q4d::tca_smem_bytes(nr, 0);
-  int stages = int((kAttnSmemBudget - fixed) / (stage_bytes + 16));
+  const size_t fixed = rows8 ? q4d::attn_rows8_smem_bytes(0) : q4d::tca_smem_bytes(nr, 0, q8, pb);
+  const size_t budget = q8 ? kAttnSmemMax : kAttnSmemBudget;
+  int stages = int((budget - fixed) / (stage_bytes + 16));
   stages = std::max(2, std::min(8, stages));
   plan->n_splits = n_splits;
   plan->split_tokens = split_tokens;
@@ -481,11 +512,16 @@ q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_di
   plan->rows_per_cta = rows_per_cta;
   plan->stages = stages;
   plan->threads = rows8 ? q4d::kR8Threads : q4d::kTcaThreads;
-  plan->smem_bytes = rows8 ? q4d::attn_rows8_smem_bytes(stages) : q4d::tca_smem_bytes(nr, stages);
+  plan->smem_bytes =
+      rows8 ? q4d::attn_rows8_smem_bytes(stages) : q4d::tca_smem_bytes(nr, stages, q8, pb);
   plan->workspace_bytes =
       n_splits > 1 ? size_t(n_splits) * M * n_q_heads * (q4d::kHeadDim + 2) * 4 : 0;
   return Q4D_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 size_t q4d_gemv_workspace_bytes(int M, int N, int K) {
   q4d_gemv_plan p;
@@ -496,6 +532,13 @@ size_t q4d_gemv_workspace_bytes(int M, int N, int K) {
 size_t q4d_attn_workspace_bytes(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M) {
   q4d_attn_plan p;
   if (q4d_plan_attn(ctx_len, n_q_heads, n_kv_heads, head_dim, M, planning_sms(), &p) != Q4D_OK)
+    return 0;
+  return p.workspace_bytes;
+}
+
+size_t q8kv_attn_workspace_bytes(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M) {
+  q4d_attn_plan p;
+  if (q8kv_plan_attn(ctx_len, n_q_heads, n_kv_heads, head_dim, M, planning_sms(), &p) != Q4D_OK)
     return 0;
   return p.workspace_bytes;
 }
@@ -547,6 +590,15 @@ q4d_status q4kv_attn_decode_ex(const void* Q, const void* Kq4, const void* Vq4, 
   return attn_impl(Q, Kq4, Vq4, out, ctx_len, n_q_heads, n_kv_heads, head_dim, M,
                    kv_stride_tokens, softmax_scale, static_cast<cudaStream_t>(stream), workspace,
                    workspace_bytes, false);
+}
+
+q4d_status q8kv_attn_decode_ex(const void* Q, const void* Kq8, const void* Vq8, float* out,
+                               int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
+                               int kv_stride_tokens, float softmax_scale, void* stream,
+                               void* workspace, size_t workspace_bytes) {
+  return attn_impl(Q, Kq8, Vq8, out, ctx_len, n_q_heads, n_kv_heads, head_dim, M,
+                   kv_stride_tokens, softmax_scale, static_cast<cudaStream_t>(stream), workspace,
+                   workspace_bytes, false, true);
 }
 
 }  // extern "C"

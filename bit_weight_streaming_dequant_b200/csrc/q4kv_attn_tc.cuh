@@ -25,6 +25,11 @@
 //  * producer warp: K and V tiles through a ring of bulk copies.
 // The split states use the workspace layout of the other split kernels, so the
 // same merge kernel finishes the job.  Every wait is bounded in time.
+//
+// The same kernel serves the 8-bit cache variant (Q8: 272-byte super-blocks
+// of 256 int8 values and 8 fp16 scales, the `--cache-type-k/v q8_0` cache of
+// "Running Qwen3.8-27B on an RTX 4090"): only the row size and the unpack
+// (fp16 d * q, elements in their natural order) change.
 #pragma once
 
 #include <climits>
@@ -39,8 +44,14 @@ constexpr int kTcaProducerWarp = 3 * kTcaRoleWarps;    // warps 0-3 softmax, 4-7
 constexpr int kTcaMmaWarp = kTcaProducerWarp + 1;
 constexpr int kTcaThreads = (kTcaMmaWarp + 1) * 32;
 constexpr int kTcaTile = 128;                          // tokens per tile (TMEM lanes)
-constexpr uint32_t kTcaStage = 2u * kTcaTile * kRowBytes;
 constexpr uint32_t kTcaVBytes = 256u * kTcaTile * 2u;  // unpacked V tile, fp16
+
+// Bytes of one token row (one super-block) of the cache, and of a ring stage
+// (a K tile and a V tile).
+__host__ __device__ constexpr uint32_t tca_row_bytes(bool q8) { return q8 ? 272u : 144u; }
+__host__ __device__ constexpr uint32_t tca_stage_bytes(bool q8) {
+  return 2u * kTcaTile * tca_row_bytes(q8);
+}
 constexpr int kTcaBarriers = 12;                       // besides the ring's 2 per stage
 
 // Element (within its 32-element block) that K position kk (0..31) of the
@@ -53,11 +64,12 @@ __host__ __device__ constexpr int unpacked_element(int kk) {
          2 * (kk & 1);
 }
 
-// Shared memory for NR (16 or 32) MMA columns of query rows and S stages:
-// ring, Q, V tile, P^T [2], row statistics ([4][32] + 5 x [32]), flags,
-// barriers.
-__host__ __device__ constexpr size_t tca_smem_bytes(int NR, int stages) {
-  return size_t(stages) * kTcaStage + size_t(512) * NR + kTcaVBytes + size_t(NR) * 512 +
+// Shared memory for NR (16 or 32) MMA columns of query rows, S stages and PB
+// (1 or 2) P^T buffers: ring, Q, V tile, P^T, row statistics ([4][32] +
+// 5 x [32]), flags, barriers.
+__host__ __device__ constexpr size_t tca_smem_bytes(int NR, int stages, bool q8, int PB) {
+  return size_t(stages) * tca_stage_bytes(q8) + size_t(512) * NR + kTcaVBytes +
+         size_t(NR) * 256 * PB +
          4 * 32 * 4 + 5 * 32 * 4 + 16 + size_t(2 * stages + kTcaBarriers) * 8 + 8;
 }
 
@@ -67,6 +79,48 @@ __device__ __forceinline__ uint4 tca_scaled_word(uint32_t w, uint32_t d2) {
                     f16x2_mul(q8_pair<true>(w >> 8), d2), f16x2_mul(q8_pair<false>(w >> 8), d2));
 }
 
+// Q8: fp16 pairs d * q of the four int8 values of w, (byte 0, byte 1) and
+// (byte 2, byte 3).  q ^ 0x80 = q + 128 is the low byte of the fp16 value
+// 1024 + q + 128 (high byte 0x64); subtracting 1152 leaves q exactly; one
+// multiply rounds d * q once.
+__device__ __forceinline__ void tca_scaled_q8_word(uint32_t w, uint32_t d2, uint32_t& lo,
+                                                   uint32_t& hi) {
+  const uint32_t x = w ^ 0x80808080u;
+  lo = f16x2_mul(f16x2_fma(prmt(x, 0x64646464u, 0x4140u), 0x3C003C00u, 0xE480E480u), d2);
+  hi = f16x2_mul(f16x2_fma(prmt(x, 0x64646464u, 0x4342u), 0x3C003C00u, 0xE480E480u), d2);
+}
+
+// The 16 fp16 pairs (d folded) of block b of a token row, in tensor-memory
+// column order: Q4 in the unpacked element order, Q8 in element order.
+template <bool Q8>
+__device__ __forceinline__ void tca_block(const uint8_t* row, int b, uint32_t d2,
+                                          uint32_t (&o)[16]) {
+  if constexpr (!Q8) {
+    const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * b);
+    const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+    #pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint4 v = tca_scaled_word(w4[t], d2);
+      o[4 * t + 0] = v.x;
+      o[4 * t + 1] = v.y;
+      o[4 * t + 2] = v.z;
+      o[4 * t + 3] = v.w;
+    }
+  } else {
+    const uint4 w0 = *reinterpret_cast<const uint4*>(row + 32 * b);
+    const uint4 w1 = *reinterpret_cast<const uint4*>(row + 32 * b + 16);
+    const uint32_t w8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) tca_scaled_q8_word(w8[i], d2, o[2 * i], o[2 * i + 1]);
+  }
+}
+
+// Element of a block that position kk (0..31) of the column order holds.
+template <bool Q8>
+__host__ __device__ constexpr int tca_element(int kk) {
+  return Q8 ? kk : unpacked_element(kk);
+}
+
 // fp16 scale of block b (0..7) from the row's 16 scale bytes, in both halves
 // (0 for a token past the end of the tile's data).
 __device__ __forceinline__ uint32_t tca_scale2(const uint4& dv, int b, bool live) {
@@ -74,19 +128,26 @@ __device__ __forceinline__ uint32_t tca_scale2(const uint4& dv, int b, bool live
   return live ? prmt(w, 0u, (b & 1) ? 0x3232u : 0x1010u) : 0u;
 }
 
-template <int NR>
+// NR: MMA columns of query rows (16 or 32); Q8: the 8-bit cache; PB: P^T
+// buffers (2 lets the softmax of a tile overlap the previous P.V; 1 when
+// shared memory holds no more).
+template <int NR, bool Q8, int PB>
 __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const AttnArgs a) {
   static_assert(NR == 16 || NR == 32, "query rows per CTA: 16 or 32 MMA columns");
+  static_assert(PB == 1 || PB == 2, "one or two P^T buffers");
   constexpr int TT = kTcaTile;
+  constexpr uint32_t RB = tca_row_bytes(Q8);           // bytes per token row
+  constexpr uint32_t kStage = tca_stage_bytes(Q8);
+  constexpr uint32_t kScales = Q8 ? 256u : 128u;       // offset of the 8 fp16 scales
   constexpr uint32_t kIdescQK = idesc_f16(128, NR, 0, 0);
   constexpr uint32_t kIdescPV = idesc_f16(128, NR, 1, 1);
   extern __shared__ __align__(128) uint8_t smem[];
   const int S = a.stages;
   uint8_t* ring = smem;
-  uint8_t* Qs = ring + size_t(S) * kTcaStage;
+  uint8_t* Qs = ring + size_t(S) * kStage;
   uint8_t* Vs = Qs + 512 * NR;
   uint8_t* Ps = Vs + kTcaVBytes;
-  float* wred = reinterpret_cast<float*>(Ps + NR * 512);   // [4][32]; P^T [2][NR * 256]
+  float* wred = reinterpret_cast<float*>(Ps + NR * 256 * PB);   // [4][32]; P^T [PB][NR * 256]
   float* m_run = wred + 4 * 32;
   float* m_use = m_run + 32;
   float* alph = m_use + 32;
@@ -137,7 +198,7 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
     float v = 0.f;
     if (n < R) {
       const int rr = row0 + n, m = rr / a.g, j = rr - m * a.g;
-      const int e = (kp & ~31) + unpacked_element(kp & 31);
+      const int e = (kp & ~31) + tca_element<Q8>(kp & 31);
       v = bf16_bits_to_float(a.Q[(size_t(m) * a.n_q + kh * a.g + j) * kHeadDim + e]);
     }
     *reinterpret_cast<__half*>(Qs + (kp >> 3) * (NR * 16) + (n >> 3) * 128 + (n & 7) * 16 +
@@ -165,19 +226,19 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
   if (warp == kTcaProducerWarp) {
     // ------------------------------ producer ------------------------------
     if (lane == 0) {
-      const uint8_t* Kh = a.K + size_t(kh) * a.kv_stride * kRowBytes;
-      const uint8_t* Vh = a.V + size_t(kh) * a.kv_stride * kRowBytes;
+      const uint8_t* Kh = a.K + size_t(kh) * a.kv_stride * RB;
+      const uint8_t* Vh = a.V + size_t(kh) * a.kv_stride * RB;
       const uint64_t pol = l2_evict_first_policy();
       for (int tile = 0; tile < n_tiles; ++tile) {
         const int slot = tile % S;
         if (tile >= S) mbar_wait(smem_addr(&empty[slot]), uint32_t(tile / S - 1) & 1u, a.err);
         const int t0 = t_begin + tile * TT;
-        const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * kRowBytes;
+        const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * RB;
         const uint32_t bar = smem_addr(&full[slot]);
-        const uint32_t dk = smem_addr(ring + size_t(slot) * kTcaStage);
+        const uint32_t dk = smem_addr(ring + size_t(slot) * kStage);
         mbar_arrive_expect_tx(bar, 2 * bytes);
-        bulk_g2s(dk, Kh + size_t(t0) * kRowBytes, bytes, bar, pol);
-        bulk_g2s(dk + TT * kRowBytes, Vh + size_t(t0) * kRowBytes, bytes, bar, pol);
+        bulk_g2s(dk, Kh + size_t(t0) * RB, bytes, bar, pol);
+        bulk_g2s(dk + TT * RB, Vh + size_t(t0) * RB, bytes, bar, pol);
       }
     }
   } else if (warp == kTcaMmaWarp) {
@@ -200,8 +261,8 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
       const uint32_t vs = smem_addr(Vs), ps = smem_addr(Ps);
       for (int tile = 0; tile < n_tiles; ++tile) {
         if (tile + 1 < n_tiles) qk(tile + 1);
-        const int pb = tile & 1;
-        mbar_wait(smem_addr(&pready[pb]), uint32_t(tile >> 1) & 1u, a.err);
+        const int pb = tile % PB;
+        mbar_wait(smem_addr(&pready[pb]), uint32_t(tile / PB) & 1u, a.err);
         const uint32_t psb = ps + uint32_t(pb) * (NR * 256);
         #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -227,26 +288,19 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
       if (tile >= 2) mbar_wait(smem_addr(&sdone[tile & 1]), uint32_t((tile - 2) >> 1) & 1u, a.err);
       __syncwarp();  // the tensor-memory stores below are warp-collective
       tc_fence_after();
-      const uint8_t* row = ring + size_t(slot) * kTcaStage + k * kRowBytes;
+      const uint8_t* row = ring + size_t(slot) * kStage + k * RB;
       const bool live = k < t_end - (t_begin + tile * TT);
-      const uint4 dv = *reinterpret_cast<const uint4*>(row + 128);
+      const uint4 dv = *reinterpret_cast<const uint4*>(row + kScales);
       #pragma unroll 1
       for (int c = 0; c < 4; ++c) {  // blocks 2c, 2c + 1: 32 tensor-memory columns
         uint32_t r[32];
         #pragma unroll
         for (int bb = 0; bb < 2; ++bb) {
           const int b = 2 * c + bb;
-          const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * b);
-          const uint32_t d2 = tca_scale2(dv, b, live);
-          const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+          uint32_t o[16];
+          tca_block<Q8>(row, b, tca_scale2(dv, b, live), o);
           #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const uint4 o = tca_scaled_word(w4[t], d2);
-            r[16 * bb + 4 * t + 0] = o.x;
-            r[16 * bb + 4 * t + 1] = o.y;
-            r[16 * bb + 4 * t + 2] = o.z;
-            r[16 * bb + 4 * t + 3] = o.w;
-          }
+          for (int i = 0; i < 16; ++i) r[16 * bb + i] = o[i];
         }
         tc_st32(tm_ak + lane_base + uint32_t((tile & 1) * 128 + 32 * c), r);
       }
@@ -261,9 +315,9 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
     for (int tile = 0; tile < n_tiles; ++tile) {
       const int slot = tile % S;
       mbar_wait(smem_addr(&full[slot]), uint32_t(tile / S) & 1u, a.err);
-      const uint8_t* row = ring + size_t(slot) * kTcaStage + (TT + k) * kRowBytes;
+      const uint8_t* row = ring + size_t(slot) * kStage + (TT + k) * RB;
       const bool live = k < t_end - (t_begin + tile * TT);
-      const uint4 dv = *reinterpret_cast<const uint4*>(row + 128);
+      const uint4 dv = *reinterpret_cast<const uint4*>(row + kScales);
       #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         // half h of the V tile was last read by the P.V chain of tile - 1
@@ -271,13 +325,12 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
         #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
           const int b = 4 * h + bb;
-          const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * b);
-          const uint32_t d2 = tca_scale2(dv, b, live);
-          const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+          uint32_t o[16];
+          tca_block<Q8>(row, b, tca_scale2(dv, b, live), o);
           #pragma unroll
-          for (int t = 0; t < 4; ++t)  // one 16-byte chunk of the M-major tile
+          for (int t = 0; t < 4; ++t)  // 8 dimensions: one 16-byte chunk of the M-major tile
             *reinterpret_cast<uint4*>(Vs + (4 * b + t) * 2048 + (k >> 3) * 128 + (k & 7) * 16) =
-                tca_scaled_word(w4[t], d2);
+                make_uint4(o[4 * t], o[4 * t + 1], o[4 * t + 2], o[4 * t + 3]);
         }
         fence_proxy_async_smem();
         mbar_arrive(smem_addr(&vready[h]));
@@ -348,9 +401,10 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
         l_part[i + 2] = fmaf(l_part[i + 2], al4.z, f1.x);
         l_part[i + 3] = fmaf(l_part[i + 3], al4.w, f1.y);
       }
-      // P^T buffer (tile & 1) is free once the P.V of tile - 2 has read it;
+      // P^T buffer (tile % PB) is free once the P.V of tile - PB has read it;
       // O^T may be rescaled only after the P.V of tile - 1 has finished
-      if (tile >= 2) mbar_wait(smem_addr(&pfree[tile & 1]), uint32_t((tile - 2) >> 1) & 1u, a.err);
+      if (tile >= PB)
+        mbar_wait(smem_addr(&pfree[tile % PB]), uint32_t((tile - PB) / PB) & 1u, a.err);
       if (rescale && tile > 0) {
         mbar_wait(smem_addr(&pvdone[1]), uint32_t(tile - 1) & 1u, a.err);
         __syncwarp();
@@ -370,18 +424,18 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
           tc_wait_st();
         }
       }
-      uint8_t* Pb = Ps + (tile & 1) * (NR * 256);
+      uint8_t* Pb = Ps + (tile % PB) * (NR * 256);
       #pragma unroll
       for (int c = 0; c < NR / 8; ++c)  // rows 8c .. 8c + 7 of token k
         *reinterpret_cast<uint4*>(Pb + c * 2048 + (k >> 3) * 128 + (k & 7) * 16) =
             make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(smem_addr(&pready[tile & 1]));
+      mbar_arrive(smem_addr(&pready[tile % PB]));
     }
     // ---- split totals: row sums of the rounded P (after the last P.V)
     if (n_tiles > 0) {
-      mbar_wait(smem_addr(&pfree[(n_tiles - 1) & 1]), uint32_t((n_tiles - 1) >> 1) & 1u, a.err);
+      mbar_wait(smem_addr(&pfree[(n_tiles - 1) % PB]), uint32_t((n_tiles - 1) / PB) & 1u, a.err);
       __syncwarp();
     }
     #pragma unroll
@@ -402,7 +456,7 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
   if (warp < 2 * kTcaRoleWarps) {
     const int half = warp / kTcaRoleWarps;
     const int mm = 128 * half + k;                      // lane = unpacked dimension position
-    const int dim = (mm & ~31) + unpacked_element(mm & 31);
+    const int dim = (mm & ~31) + tca_element<Q8>(mm & 31);
     const size_t rows_total = size_t(a.M) * a.n_q;
     #pragma unroll
     for (int c0 = 0; c0 < NR; c0 += 16) {

@@ -31,7 +31,8 @@ EXPORTS = (
     "q4kv_attn_decode_noalloc",
     "q4d_pack_q4_0_weights", "q4d_unpack_q4_0_weights", "q4d_pack_q4_0_rows",
     "q4d_unpack_q4_0_rows", "q4kv_append", "q4_gemv_swiglu_ex",
-    "q4d_gemv_swiglu_workspace_bytes",
+    "q4d_gemv_swiglu_workspace_bytes", "q8kv_attn_decode_ex", "q8kv_attn_workspace_bytes",
+    "q8kv_plan_attn",
 )
 
 
@@ -96,6 +97,12 @@ def lib() -> ctypes.CDLL:
     L.q4_gemv_swiglu_ex.restype = i
     L.q4d_gemv_swiglu_workspace_bytes.argtypes = [i, i, i]
     L.q4d_gemv_swiglu_workspace_bytes.restype = sz
+    L.q8kv_attn_decode_ex.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, sz]
+    L.q8kv_attn_decode_ex.restype = i
+    L.q8kv_attn_workspace_bytes.argtypes = [i, i, i, i, i]
+    L.q8kv_attn_workspace_bytes.restype = sz
+    L.q8kv_plan_attn.argtypes = [i, i, i, i, i, i, ctypes.POINTER(AttnPlan)]
+    L.q8kv_plan_attn.restype = i
     for fn in ("q4_gemv", "q4_gemv_ex", "q4_gemv_ex2", "q4kv_attn_decode", "q4kv_attn_decode_ex",
                "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
                "q4kv_attn_decode_noalloc"):
@@ -116,10 +123,12 @@ def plan_gemv(M: int, N: int, K: int, num_sms: int) -> GemvPlan:
 
 
 def plan_attn(ctx_len: int, n_q_heads: int, n_kv_heads: int, head_dim: int, M: int,
-              num_sms: int) -> AttnPlan:
+              num_sms: int, q8: bool = False) -> AttnPlan:
+    """Launch plan of the attention over the Q4_0 cache (``q8``: the Q8_0 cache)."""
     p = AttnPlan()
-    _check(lib().q4d_plan_attn(ctx_len, n_q_heads, n_kv_heads, head_dim, M, num_sms,
-                               ctypes.byref(p)), "q4d_plan_attn")
+    fn = "q8kv_plan_attn" if q8 else "q4d_plan_attn"
+    _check(getattr(lib(), fn)(ctx_len, n_q_heads, n_kv_heads, head_dim, M, num_sms,
+                              ctypes.byref(p)), fn)
     return p
 
 
@@ -299,30 +308,47 @@ def q4kv_attn_decode(Q, Kq4, Vq4, out=None, *, ctx_len: int, n_kv_heads: int,
     ``n_kv_heads * kv_stride_tokens`` super-blocks; returns fp32 ``out`` of
     Q's shape.
     """
+    return _attn(Q, Kq4, Vq4, out, ctx_len, n_kv_heads, head_dim, kv_stride_tokens,
+                 softmax_scale, stream, workspace, q8=False)
+
+
+def q8kv_attn_decode(Q, Kq8, Vq8, out=None, *, ctx_len: int, n_kv_heads: int,
+                     head_dim: int = 256, kv_stride_tokens: int | None = None,
+                     softmax_scale: float = 1.0, stream=None, workspace=None):
+    """The same attention over Q8_0 K/V caches (272-byte super-blocks) via
+    ``q8kv_attn_decode_ex``."""
+    return _attn(Q, Kq8, Vq8, out, ctx_len, n_kv_heads, head_dim, kv_stride_tokens,
+                 softmax_scale, stream, workspace, q8=True)
+
+
+def _attn(Q, Kc, Vc, out, ctx_len, n_kv_heads, head_dim, kv_stride_tokens, softmax_scale,
+          stream, workspace, q8):
     torch = _torch()
     _dev_tensor(Q, torch.bfloat16, "Q")
-    _dev_tensor(Kq4, torch.uint8, "Kq4")
-    _dev_tensor(Vq4, torch.uint8, "Vq4")
+    _dev_tensor(Kc, torch.uint8, "K cache")
+    _dev_tensor(Vc, torch.uint8, "V cache")
     if Q.dim() != 3 or Q.shape[2] != head_dim:
         raise ValueError("Q must be [M][n_q_heads][head_dim]")
     M, n_q = Q.shape[0], Q.shape[1]
     stride = ctx_len if kv_stride_tokens is None else kv_stride_tokens
-    need_bytes = n_kv_heads * stride * (head_dim // 256) * 144
-    if Kq4.numel() < need_bytes or Vq4.numel() < need_bytes:
+    need_bytes = n_kv_heads * stride * (head_dim // 256) * (272 if q8 else 144)
+    if Kc.numel() < need_bytes or Vc.numel() < need_bytes:
         raise ValueError("K/V caches are smaller than n_kv_heads * kv_stride_tokens rows")
     if out is None:
         out = torch.empty((M, n_q, head_dim), dtype=torch.float32, device=Q.device)
     _dev_tensor(out, torch.float32, "out")
     if tuple(out.shape) != (M, n_q, head_dim):
         raise ValueError("out must match Q's shape")
+    name = "q8kv_attn_decode_ex" if q8 else "q4kv_attn_decode_ex"
     with torch.cuda.device(Q.device):
-        need = lib().q4d_attn_workspace_bytes(ctx_len, n_q, n_kv_heads, head_dim, M)
+        wsfn = lib().q8kv_attn_workspace_bytes if q8 else lib().q4d_attn_workspace_bytes
+        need = wsfn(ctx_len, n_q, n_kv_heads, head_dim, M)
         ws = _workspace(need, Q.device, workspace)
-        st = lib().q4kv_attn_decode_ex(Q.data_ptr(), Kq4.data_ptr(), Vq4.data_ptr(),
-                                       out.data_ptr(), ctx_len, n_q, n_kv_heads, head_dim, M,
-                                       stride, float(softmax_scale), _stream_ptr(stream),
-                                       None if ws is None else ws.data_ptr(), need)
-    _check(st, "q4kv_attn_decode")
+        st = getattr(lib(), name)(Q.data_ptr(), Kc.data_ptr(), Vc.data_ptr(), out.data_ptr(),
+                                  ctx_len, n_q, n_kv_heads, head_dim, M, stride,
+                                  float(softmax_scale), _stream_ptr(stream),
+                                  None if ws is None else ws.data_ptr(), need)
+    _check(st, name)
     return out
 
 

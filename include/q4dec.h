@@ -183,6 +183,28 @@ q4d_status q4kv_attn_decode_ex(const void* Q, const void* Kq4, const void* Vq4, 
 size_t q4d_attn_workspace_bytes(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim,
                                 int M);
 
+/* -------------------------------------------- attention, Q8_0 K/V cache --
+ * The same attention over the 8-bit cache type the page "Running
+ * Qwen3.8-27B on an RTX 4090" launches its server with (--cache-type-k /
+ * --cache-type-v q8_0): Q8_0 blocks of 32 int8 values q and one fp16 scale d,
+ * value d * q.
+ *
+ *   Kq8, Vq8 : [n_kv_heads][kv_stride_tokens] 272-byte super-blocks, one per
+ *              token: bytes 0..255 the int8 values (element j of block b at
+ *              byte 32*b + j, two's complement), bytes 256 + 2*b the fp16
+ *              scale of block b (little endian); 16-byte aligned.
+ *   Everything else (Q, out, requirements, workspace, errors) as
+ *   q4kv_attn_decode_ex, with the workspace size from
+ *   q8kv_attn_workspace_bytes.  Every row count runs on the tensor-memory
+ *   kernel; K and V enter the tensor core as fp16 d * q, each rounded once.
+ */
+q4d_status q8kv_attn_decode_ex(const void* Q, const void* Kq8, const void* Vq8, float* out,
+                               int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
+                               int kv_stride_tokens, float softmax_scale, void* stream,
+                               void* workspace, size_t workspace_bytes);
+size_t q8kv_attn_workspace_bytes(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim,
+                                 int M);
+
 /* ------------------------------------------- attention, allocation-free --
  * The paper has no counterpart to this entry point; it exists for deployment.
  *
@@ -247,6 +269,9 @@ typedef struct {
 q4d_status q4d_plan_gemv(int M, int N, int K, int num_sms, q4d_gemv_plan* plan);
 q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
                          int num_sms, q4d_attn_plan* plan);
+/* The plan of q8kv_attn_decode_ex (the Q8_0 cache). */
+q4d_status q8kv_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
+                          int num_sms, q4d_attn_plan* plan);
 
 /* ------------------------------------------------------- K/V append --
  * Quantise the K and V rows of M new tokens and write them at token positions

@@ -1,4 +1,4 @@
-"""CPU oracle for the Q4_0 decode path (test infrastructure only).
+"""CPU oracle for the Q4_0 decode path (and the Q8_0 K/V cache variant) (test infrastructure only).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU-baseline
 and reference legs) may import this package.  The library's product path never
@@ -9,6 +9,8 @@ from .q4_oracle import (  # noqa: F401
     f16_bits_to_f64,
     unpack_superblocks,
     dequant,
+    unpack_q8_superblocks,
+    dequant_q8,
     dequant_weights,
     weight_rows,
     gemv,

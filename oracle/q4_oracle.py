@@ -45,6 +45,14 @@ writes out the definitions the library implements:
   whose d is zero stores d = +0 and q = 8.  The pages say only that the
   cache is Q4 (the paragraph on the 16 full-attention layers).
 
+* Q8_0 K/V cache (the 8-bit cache type the page "Running Qwen3.8-27B on an
+  RTX 4090" launches its server with, ``--cache-type-k/v q8_0``): 32 int8
+  values and one fp16 scale per block, value ``d * q``; stored, like the Q4
+  cache, as one super-block per token: the 256 int8 values first (element
+  ``j`` of block ``b`` at byte ``32*b + j``), then the 8 fp16 scales at
+  ``256 + 2*b`` -- 272 bytes.  Attention over it is the same computation with
+  this dequantisation.
+
 Readings taken where nothing fixes a detail: output is fp32 on the device
 (fp64 here); the softmax scale defaults to 1 (queries arrive pre-scaled);
 GQA groups are contiguous; non-finite inputs are out of scope.
@@ -59,6 +67,7 @@ import numpy as np
 SB_ELEMS = 256          # elements per super-block
 SB_BYTES = 144          # bytes per super-block
 NIBBLE_BYTES = 128      # bytes of nibbles per super-block (8 blocks x 16)
+Q8_SB_BYTES = 272       # bytes per Q8_0 super-block (256 int8 values + 8 fp16 scales)
 
 
 def bf16_bits_to_f64(bits) -> np.ndarray:
@@ -138,26 +147,57 @@ def gemv_tolerance(S: np.ndarray) -> np.ndarray:
     return 2e-3 * S + 1e-5
 
 
-def _kv_hat(buf, n_kv: int, ctx_len: int, head_dim: int, kv_stride: int) -> np.ndarray:
+def unpack_q8_superblocks(buf, rows: int, K: int):
+    """Read ``rows`` rows of ``K`` Q8_0 elements from 272-byte super-blocks.
+
+    Returns ``q`` (int64 [rows][K], values -128..127) and ``d`` (float64
+    [rows][K/32])."""
+    if K % SB_ELEMS:
+        raise ValueError("K must be a multiple of 256")
+    nsb = K // SB_ELEMS
+    raw = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    need = rows * nsb * Q8_SB_BYTES
+    if raw.size < need:
+        raise ValueError(f"buffer holds {raw.size} bytes, need {need}")
+    sb = raw[:need].reshape(rows, nsb, Q8_SB_BYTES)
+    u = sb[:, :, :256].astype(np.int64)
+    q = np.where(u >= 128, u - 256, u)                # two's complement bytes
+    lo = sb[:, :, 256::2].astype(np.uint16)
+    hi = sb[:, :, 257::2].astype(np.uint16)
+    d_bits = lo | (hi << 8)                           # little endian fp16, block b at 256 + 2b
+    return q.reshape(rows, K), f16_bits_to_f64(d_bits).reshape(rows, K // 32)
+
+
+def dequant_q8(buf, rows: int, K: int) -> np.ndarray:
+    """fp64 values ``d * q`` of ``rows x K`` Q8_0 elements."""
+    q, d = unpack_q8_superblocks(buf, rows, K)
+    return np.repeat(d, 32, axis=1) * q.astype(np.float64)
+
+
+def _kv_hat(buf, n_kv: int, ctx_len: int, head_dim: int, kv_stride: int,
+            fmt: str = "q4_0") -> np.ndarray:
     """Dequantised cache [n_kv][ctx_len][head_dim] (rows of one super-block
     per token when head_dim == 256; ``kv_stride`` tokens between heads)."""
+    if fmt not in ("q4_0", "q8_0"):
+        raise ValueError(f"unknown cache format {fmt!r}")
+    sb_bytes, deq = (SB_BYTES, dequant) if fmt == "q4_0" else (Q8_SB_BYTES, dequant_q8)
     out = np.empty((n_kv, ctx_len, head_dim), dtype=np.float64)
-    row_bytes = (head_dim // SB_ELEMS) * SB_BYTES
+    row_bytes = (head_dim // SB_ELEMS) * sb_bytes
     raw = np.asarray(buf, dtype=np.uint8).reshape(-1)
     for h in range(n_kv):
         start = h * kv_stride * row_bytes
-        out[h] = dequant(raw[start: start + ctx_len * row_bytes], ctx_len, head_dim)
+        out[h] = deq(raw[start: start + ctx_len * row_bytes], ctx_len, head_dim)
     return out
 
 
 def attn_probs(Q_bits, K_buf, ctx_len: int, n_q_heads: int, n_kv_heads: int,
                head_dim: int, M: int, kv_stride: int | None = None,
-               scale: float = 1.0) -> np.ndarray:
+               scale: float = 1.0, fmt: str = "q4_0") -> np.ndarray:
     """Softmax weights ``P[m, h, t]`` (zero for masked tokens), fp64."""
     kv_stride = ctx_len if kv_stride is None else kv_stride
     g = n_q_heads // n_kv_heads
     Q = bf16_bits_to_f64(np.asarray(Q_bits).reshape(M, n_q_heads, head_dim))
-    Kh = _kv_hat(K_buf, n_kv_heads, ctx_len, head_dim, kv_stride)
+    Kh = _kv_hat(K_buf, n_kv_heads, ctx_len, head_dim, kv_stride, fmt)
     P = np.zeros((M, n_q_heads, ctx_len), dtype=np.float64)
     for m in range(M):
         p_m = ctx_len - M + m                 # absolute position of draft row m
@@ -171,16 +211,17 @@ def attn_probs(Q_bits, K_buf, ctx_len: int, n_q_heads: int, n_kv_heads: int,
 
 def attn_decode(Q_bits, K_buf, V_buf, ctx_len: int, n_q_heads: int, n_kv_heads: int,
                 head_dim: int, M: int, kv_stride: int | None = None,
-                scale: float = 1.0) -> np.ndarray:
-    """Causal GQA decode attention over a Q4_0 K/V cache, fp64.
+                scale: float = 1.0, fmt: str = "q4_0") -> np.ndarray:
+    """Causal GQA decode attention over a Q4_0 (or, ``fmt="q8_0"``, Q8_0) K/V
+    cache, fp64.
 
     Returns ``out[m, h, :] = sum_t P[m, h, t] * V_hat[h // g, t, :]``.
     """
     kv_stride = ctx_len if kv_stride is None else kv_stride
     g = n_q_heads // n_kv_heads
     P = attn_probs(Q_bits, K_buf, ctx_len, n_q_heads, n_kv_heads, head_dim, M,
-                   kv_stride, scale)
-    Vh = _kv_hat(V_buf, n_kv_heads, ctx_len, head_dim, kv_stride)
+                   kv_stride, scale, fmt)
+    Vh = _kv_hat(V_buf, n_kv_heads, ctx_len, head_dim, kv_stride, fmt)
     out = np.empty((M, n_q_heads, head_dim), dtype=np.float64)
     for m in range(M):
         for h in range(n_q_heads):

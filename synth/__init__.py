@@ -27,7 +27,13 @@ Recipes (the workloads of the decode path):
 * K/V caches: ``N(0,1)`` values quantised per 32-block with ``amax`` = the
   signed element of largest magnitude, ``d = fp16(amax / -8)``,
   ``q = clamp(floor(v / d + 8.5), 0, 15)`` (``d = 0`` gives ``q = 8``);
-* queries: ``bf16(N(0,1) / 16)``.
+* queries: ``bf16(N(0,1) / 16)``;
+* Q8_0 K/V caches (the 8-bit cache variant): one 272-byte super-block per
+  token: 256 int8 values (element ``j`` of block ``b`` at byte ``32*b + j``,
+  two's complement), then the 8 fp16 scales (bytes ``256 + 2*b``); the value
+  is ``d * q``.  Recipe: ``N(0,1)`` values per 32-block, ``d = fp16(amax/127)``
+  with ``amax`` the largest magnitude, ``q = clamp(rint(v / d), -127, 127)``
+  (``d = 0`` gives ``q = 0``).
 
 Host generation uses ``numpy.random.default_rng(seed)`` (PCG64).  The large
 workloads (gigabytes) are generated directly on the GPU with a seeded
@@ -144,6 +150,45 @@ def q4_0_kv_cache(seed: int, n_kv_heads: int, ctx: int, head_dim: int = 256) -> 
     return pack_superblocks(q, d)
 
 
+Q8_SUPERBLOCK_BYTES = 272
+
+
+def quantize_q8_blocks(v: np.ndarray):
+    """Quantise float values ``v[rows][K]`` per 32-block to 8 bits (Q8_0 recipe
+    in the module docstring).  Returns ``(q int8[rows][K], d_bits uint16[rows][K/32])``."""
+    v = np.asarray(v, dtype=np.float32)
+    rows, K = v.shape
+    vb = v.reshape(rows, K // BLOCK_ELEMS, BLOCK_ELEMS)
+    amax = np.abs(vb).max(axis=-1)
+    d16 = (amax / np.float32(127.0)).astype(np.float16)
+    d32 = d16.astype(np.float32)
+    safe = np.where(d32 == 0, np.float32(1.0), d32)
+    q = np.clip(np.rint(vb / safe[..., None]), -127, 127).astype(np.int8)
+    q[d32 == 0] = 0
+    return q.reshape(rows, K), d16.view(np.uint16)
+
+
+def pack_q8_superblocks(q: np.ndarray, d_bits: np.ndarray) -> np.ndarray:
+    """int8 ``q[rows][K]`` and fp16 scale bits ``d_bits[rows][K/32]`` -> flat
+    uint8 of ``rows * K/256`` Q8_0 super-blocks in row order."""
+    rows, K = q.shape
+    nsb = K // SUPERBLOCK_ELEMS
+    out = np.empty((rows, nsb, Q8_SUPERBLOCK_BYTES), dtype=np.uint8)
+    out[:, :, :256] = np.asarray(q, dtype=np.int8).view(np.uint8).reshape(rows, nsb, 256)
+    out[:, :, 256:] = (np.asarray(d_bits, dtype=np.uint16).reshape(rows, nsb, 8)
+                       .view(np.uint8).reshape(rows, nsb, 16))
+    return out.reshape(-1)
+
+
+def q8_0_kv_cache(seed: int, n_kv_heads: int, ctx: int, head_dim: int = 256) -> np.ndarray:
+    """One Q8_0 K (or V) cache: N(0,1) values quantised per block, laid out as
+    ``[n_kv_heads][ctx]`` 272-byte super-blocks (flat uint8)."""
+    rng = np.random.default_rng(seed)
+    v = rng.standard_normal(size=(n_kv_heads * ctx, head_dim)).astype(np.float32)
+    q, d = quantize_q8_blocks(v)
+    return pack_q8_superblocks(q, d)
+
+
 def queries(seed: int, M: int, n_q_heads: int, head_dim: int = 256) -> np.ndarray:
     """bf16 bits of ``N(0,1)/16`` queries, shape [M][n_q_heads][head_dim]."""
     return bf16_normal(seed, (M, n_q_heads, head_dim), scale=1.0 / 16.0)
@@ -219,4 +264,28 @@ def device_q4_0_kv_cache(seed: int, n_kv_heads: int, ctx: int, head_dim: int = 2
         nib = q[..., 0, :] | (q[..., 1, :] << 4)
         out[r0:r1, :, :128] = nib.reshape(r1 - r0, nsb, 128)
         out[r0:r1, :, 128:] = d16.view(torch.uint8).reshape(r1 - r0, nsb, 16)
+    return out.reshape(-1)
+
+
+def device_q8_0_kv_cache(seed: int, n_kv_heads: int, ctx: int, head_dim: int = 256,
+                         device="cuda", chunk_tokens: int = 1 << 16):
+    """Q8_0 K (or V) cache of N(0,1) values quantised per block, generated on
+    the device in chunks; flat uint8 tensor ``[n_kv_heads][ctx]`` super-blocks."""
+    torch = _torch()
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    rows = n_kv_heads * ctx
+    nsb = head_dim // SUPERBLOCK_ELEMS
+    out = torch.empty((rows, nsb, Q8_SUPERBLOCK_BYTES), dtype=torch.uint8, device=device)
+    for r0 in range(0, rows, chunk_tokens):
+        r1 = min(rows, r0 + chunk_tokens)
+        v = torch.randn((r1 - r0, head_dim), generator=g, device=device)
+        vb = v.reshape(r1 - r0, head_dim // BLOCK_ELEMS, BLOCK_ELEMS)
+        d16 = (vb.abs().amax(dim=-1) / 127.0).to(torch.float16)
+        d32 = d16.to(torch.float32)
+        safe = torch.where(d32 == 0, torch.ones_like(d32), d32)
+        q = torch.round(vb / safe[..., None]).clamp_(-127, 127).to(torch.int8)
+        q[d32 == 0] = 0
+        out[r0:r1, :, :256] = q.view(torch.uint8).reshape(r1 - r0, nsb, 256)
+        out[r0:r1, :, 256:] = d16.view(torch.uint8).reshape(r1 - r0, nsb, 16)
     return out.reshape(-1)

@@ -15,7 +15,7 @@ HEADER = os.path.join(ROOT, "include", "q4dec.h")
 def _declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    names = re.findall(r"\b(q4[a-z0-9_]*)\s*\(", text)
+    names = re.findall(r"\b(q[48][a-z0-9_]*)\s*\(", text)
     return sorted(set(names))
 
 
@@ -91,19 +91,33 @@ def test_gemv_rejects_null_and_misaligned_pointers():
 ])
 def test_attn_rejects_bad_arguments_without_cuda(ctx, nq, nkv, hd, M, stride, scale, code):
     L = q4dec.lib()
-    assert L.q4kv_attn_decode_ex(FAKE, FAKE, FAKE, FAKE, ctx, nq, nkv, hd, M, stride,
-                                 ctypes.c_float(scale), None, None, 0) == code
+    for fn in (L.q4kv_attn_decode_ex, L.q8kv_attn_decode_ex):
+        assert fn(FAKE, FAKE, FAKE, FAKE, ctx, nq, nkv, hd, M, stride,
+                  ctypes.c_float(scale), None, None, 0) == code
 
 
 def test_attn_rejects_null_and_misaligned():
     L = q4dec.lib()
     args = (4096, 24, 4, 256, 1, 4096, ctypes.c_float(1.0), None, None, 0)
-    assert L.q4kv_attn_decode_ex(None, FAKE, FAKE, FAKE, *args) == 1
-    assert L.q4kv_attn_decode_ex(FAKE, FAKE, FAKE, None, *args) == 1
-    assert L.q4kv_attn_decode_ex(FAKE + 8, FAKE, FAKE, FAKE, *args) == 3
-    assert L.q4kv_attn_decode_ex(FAKE, FAKE + 4, FAKE, FAKE, *args) == 3
-    assert L.q4kv_attn_decode_ex(FAKE, FAKE, FAKE + 12, FAKE, *args) == 3
-    assert L.q4kv_attn_decode_ex(FAKE, FAKE, FAKE, FAKE + 1, *args) == 3
+    for fn in (L.q4kv_attn_decode_ex, L.q8kv_attn_decode_ex):
+        assert fn(None, FAKE, FAKE, FAKE, *args) == 1
+        assert fn(FAKE, FAKE, FAKE, None, *args) == 1
+        assert fn(FAKE + 8, FAKE, FAKE, FAKE, *args) == 3
+        assert fn(FAKE, FAKE + 4, FAKE, FAKE, *args) == 3
+        assert fn(FAKE, FAKE, FAKE + 12, FAKE, *args) == 3
+        assert fn(FAKE, FAKE, FAKE, FAKE + 1, *args) == 3
+
+
+def test_q8_plan_and_workspace_queries():
+    L = q4dec.lib()
+    a = q4dec.AttnPlan()
+    assert L.q8kv_plan_attn(4096, 24, 4, 256, 1, 0, ctypes.byref(a)) == 1
+    assert L.q8kv_plan_attn(4096, 24, 4, 64, 1, 148, ctypes.byref(a)) == 2
+    assert L.q8kv_plan_attn(4096, 24, 4, 256, 1, 148, None) == 1
+    assert L.q8kv_attn_workspace_bytes(4096, 24, 4, 64, 1) == 0       # invalid shape
+    # one row per CTA still takes the tensor-memory kernel (448 threads)
+    assert L.q8kv_plan_attn(4096, 4, 4, 256, 1, 148, ctypes.byref(a)) == 0
+    assert a.threads == 448 and a.tile_tokens == 128
 
 
 def test_plan_rejects_bad_inputs():

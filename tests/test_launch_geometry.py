@@ -3,6 +3,7 @@ planner: every row, K range and token is covered exactly once, every bulk
 copy stays inside its source buffer and its shared-memory slot, and every
 load, store and workspace index stays in bounds.  These run before anything
 touches a GPU."""
+import numpy as np
 import pytest
 
 from bit_weight_streaming_dequant_b200 import q4dec
@@ -110,17 +111,25 @@ def _tc_nr(rows_per_cta):
     return 16 if rows_per_cta <= 16 else 32
 
 
-def _tc_offsets(stages, nr):
+ROW_Q8 = 272                        # bytes per token row of the Q8_0 cache
+SMEM_Q8_BUDGET = 227 * 1024
+
+
+def _tc_pbufs(nr, q8):
+    return 1 if (q8 and nr == 32) else 2
+
+
+def _tc_offsets(stages, nr, row=ROW, pb=2):
     """Carve-up of the tensor-memory variant's shared memory: ring, Q (fp16,
-    K-major), V tile (fp16, M-major), two P^T buffers (fp16, N-major), row
+    K-major), V tile (fp16, M-major), `pb` P^T buffers (fp16, N-major), row
     statistics ([4][32] warp partials, running max, max used, alpha, sums,
     causal limits), flags, barriers (2 per ring stage + 12) and the
     tensor-memory address."""
-    ring = stages * 2 * TT_ATTN * ROW
+    ring = stages * 2 * TT_ATTN * row
     q = ring
     v = q + 512 * nr
     pt = v + TC_V_BYTES
-    stats = pt + 2 * (nr // 8) * 2048
+    stats = pt + pb * (nr // 8) * 2048
     flags = stats + 4 * 32 * 4 + 5 * 32 * 4
     bars = flags + 16
     end = bars + (2 * stages + 12) * 8 + 8
@@ -396,3 +405,73 @@ def test_swiglu_partition_keeps_row_pairs_together(N, K, sms):
         assert rb % 2 == 0 and re_ % 2 == 0 and re_ > rb
         owned.extend(range(rb, re_))
     assert owned == list(range(rows))
+
+
+@pytest.mark.parametrize("ctx,nq,nkv,M", ATTN_CASES + [(1, 4, 1, 1), (200, 48, 1, 5)])
+@pytest.mark.parametrize("stride_extra", [0, 37])
+def test_attn_q8_geometry(ctx, nq, nkv, M, stride_extra):
+    # the Q8_0 cache: every row count on the tensor-memory kernel, 272-byte rows
+    sms = 148
+    p = q4dec.plan_attn(ctx, nq, nkv, 256, M, sms, q8=True)
+    g = nq // nkv
+    nr = _tc_nr(p.rows_per_cta)
+    pb = _tc_pbufs(nr, True)
+    assert p.tile_tokens == TT_ATTN and p.threads == TC_THREADS and p.split_tokens % TT_ATTN == 0
+    assert 2 <= p.stages <= 8 and 1 <= p.n_splits <= 256
+    o = _tc_offsets(p.stages, nr, ROW_Q8, pb)
+    assert p.smem_bytes == o["end"] <= SMEM_Q8_BUDGET
+    assert all(o[k] % 16 == 0 for k in ("q", "v", "pt", "stats", "flags", "bars"))
+    # a third stage would not fit: the planner takes as many as fit
+    assert _tc_offsets(p.stages + 1, nr, ROW_Q8, pb)["end"] > SMEM_Q8_BUDGET or p.stages == 8
+    stride = ctx + stride_extra
+    cache_bytes = nkv * stride * ROW_Q8
+    tokens = []
+    for c in range(p.n_splits):
+        tb, te = c * p.split_tokens, min(ctx, (c + 1) * p.split_tokens)
+        assert te > tb
+        tokens.extend(range(tb, te))
+        for tile in range((te - tb + TT_ATTN - 1) // TT_ATTN):
+            t0 = tb + tile * TT_ATTN
+            nbytes = min(TT_ATTN, te - t0) * ROW_Q8
+            assert 2 * nbytes <= TX_LIMIT and nbytes % 16 == 0
+            for kh in range(nkv):
+                lo = (kh * stride + t0) * ROW_Q8
+                assert lo % 16 == 0 and lo + nbytes <= cache_bytes
+    assert tokens == list(range(ctx))
+    # per token row: block b's 32 values at 32b .. 32b+31 (two 16-byte loads),
+    # the 16 scale bytes at 256; rows at a 272-byte pitch hit distinct 16-byte
+    # bank groups for eight consecutive tokens
+    for b in range(8):
+        assert 32 * b + 32 <= 256
+    for col in range(0, ROW_Q8, 16):
+        assert len(_chunks([r * ROW_Q8 + col for r in range(8)])) == 8
+    _tc_layout_checks(nr)
+    _attn_q_and_workspace(p, M, nq, nkv, g)
+    assert p.workspace_bytes == q4dec.lib().q8kv_attn_workspace_bytes(ctx, nq, nkv, 256, M) or \
+        sms != 148
+
+
+def _prmt(a, b, sel):
+    """PTX prmt.b32 (default mode): result byte i = byte (sel >> 4i) & 7 of
+    the eight bytes {a, b} (a's bytes 0..3, b's bytes 4..7)."""
+    src = [(a >> (8 * i)) & 0xFF for i in range(4)] + [(b >> (8 * i)) & 0xFF for i in range(4)]
+    return sum(src[(sel >> (4 * i)) & 7] << (8 * i) for i in range(4))
+
+
+def test_q8_unpack_constants_give_exact_codes():
+    # the tensor-memory kernel's Q8 unpack: x = w ^ 0x80808080, pairs
+    # prmt(x, 0x64646464, 0x4140 / 0x4342) read as fp16 are 1024 + q + 128;
+    # fma(., 1.0 (0x3C00), -1152 (0xE480)) is exactly q, in element order
+    one, m1152 = np.uint16(0x3C00).view(np.float16), np.uint16(0xE480).view(np.float16)
+    assert float(one) == 1.0 and float(m1152) == -1152.0
+    for q0 in range(-128, 128, 7):
+        qs = [q0, (q0 + 37) % 256 - 128, (q0 + 101) % 256 - 128, -q0 - 1]
+        w = sum((q & 0xFF) << (8 * i) for i, q in enumerate(qs))
+        x = w ^ 0x80808080
+        got = []
+        for sel in (0x4140, 0x4342):
+            r = _prmt(x, 0x64646464, sel)
+            for half in (r & 0xFFFF, r >> 16):
+                v = np.uint16(half).view(np.float16)
+                got.append(float(np.float16(np.float32(v) * np.float32(one) + np.float32(m1152))))
+        assert got == [float(q) for q in qs]

@@ -542,3 +542,97 @@ def test_gemv_swiglu_hand_worked():
     xb = synth.f32_to_bf16_bits(x)
     h, _ = oracle.gemv_swiglu(W, xb, 1, 1, 256)
     assert abs(h[0, 0] - (1.0 / (1.0 + math.exp(-1.0))) * -1.5) < 1e-15
+
+
+# ---------------------------------------------------- Q8_0 K/V variant ----
+def _read_q8_golden():
+    blocks, expect = [], []
+    with open(os.path.join(GOLDEN, "q8_0_superblock_worked.txt")) as f:
+        lines = [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+    for head, vals in zip(lines[0::2], lines[1::2]):
+        parts = dict(p.split("=") for p in head.split()[2:])
+        blocks.append((int(parts["d"], 16), bytes.fromhex(parts["bytes"])))
+        expect.extend(float(v) for v in vals.split())
+    return blocks, expect
+
+
+def test_q8_worked_superblock_fixture():
+    blocks, expect = _read_q8_golden()
+    assert len(blocks) == 8 and len(expect) == 256
+    sb = bytearray(272)
+    for b, (dbits, qs) in enumerate(blocks):
+        assert len(qs) == 32
+        sb[32 * b: 32 * b + 32] = qs
+        sb[256 + 2 * b] = dbits & 0xFF
+        sb[257 + 2 * b] = dbits >> 8
+    v = oracle.dequant_q8(np.frombuffer(bytes(sb), dtype=np.uint8), 1, 256)
+    assert list(v[0]) == expect
+
+
+def test_q8_superblock_offsets_single_value():
+    # one nonzero value (q = -3) at row 1, super-block 2, block 6, element 17:
+    # byte 32*6 + 17 of that super-block; its block scale is the only 1.0
+    rows, K = 3, 768
+    buf = np.zeros(rows * 3 * 272, dtype=np.uint8)
+    at = (1 * 3 + 2) * 272
+    buf[at + 32 * 6 + 17] = 0xFD
+    buf[at + 256 + 2 * 6: at + 258 + 2 * 6] = [0x00, 0x3C]
+    v = oracle.dequant_q8(buf, rows, K)
+    nz = np.argwhere(v != 0)
+    assert nz.tolist() == [[1, 512 + 6 * 32 + 17]]
+    assert v[1, 512 + 6 * 32 + 17] == -3.0
+
+
+def test_q8_generator_recipe():
+    # every block: d = fp16(amax / 127), |q| <= 127, and the largest |q| is 127
+    # (the element that set amax) unless the block is all zero
+    c = synth.q8_0_kv_cache(5, 2, 9)
+    q, d = oracle.unpack_q8_superblocks(c, 18, 256)
+    assert np.abs(q).max() <= 127
+    qb = np.abs(q.reshape(18, 8, 32)).max(axis=-1)
+    assert ((qb == 127) | (d == 0)).all()
+    assert (d > 0).all()
+
+
+def _q4_cache_as_q8(buf4, rows):
+    """The same values in the 8-bit layout: q8 = q4 - 8 with the same scale,
+    written byte by byte from the nibble definition (no oracle code)."""
+    raw = np.asarray(buf4, dtype=np.uint8).reshape(rows, 144)
+    out = np.zeros((rows, 272), dtype=np.uint8)
+    for b in range(8):
+        nib = raw[:, 16 * b: 16 * b + 16]
+        lo = (nib & 0x0F).astype(np.int16) - 8           # elements j
+        hi = (nib >> 4).astype(np.int16) - 8              # elements j + 16
+        out[:, 32 * b: 32 * b + 16] = lo.astype(np.int8).view(np.uint8)
+        out[:, 32 * b + 16: 32 * b + 32] = hi.astype(np.int8).view(np.uint8)
+    out[:, 256:272] = raw[:, 128:144]
+    return out.reshape(-1)
+
+
+@pytest.mark.parametrize("ctx,n_q,n_kv,M", [(5, 4, 1, 1), (33, 24, 4, 5), (70, 8, 2, 3)])
+def test_q8_attention_equals_q4_attention_on_the_same_values(ctx, n_q, n_kv, M):
+    # a Q4 cache re-expressed exactly in the 8-bit layout must give the same
+    # attention output: pins the Q8 path to the Q4 path's pins
+    K4 = synth.q4_0_kv_cache(90 + ctx, n_kv, ctx)
+    V4 = synth.q4_0_kv_cache(91 + ctx, n_kv, ctx)
+    Q = synth.queries(92 + ctx, M, n_q)
+    K8, V8 = _q4_cache_as_q8(K4, n_kv * ctx), _q4_cache_as_q8(V4, n_kv * ctx)
+    assert np.array_equal(oracle.dequant_q8(K8, n_kv * ctx, 256), oracle.dequant(K4, n_kv * ctx, 256))
+    o4 = oracle.attn_decode(Q, K4, V4, ctx, n_q, n_kv, 256, M)
+    o8 = oracle.attn_decode(Q, K8, V8, ctx, n_q, n_kv, 256, M, fmt="q8_0")
+    assert np.allclose(o8, o4, rtol=0, atol=1e-13)
+
+
+def test_q8_attention_single_token_and_stride():
+    # one visible token: the output is that token's V row for every query
+    # head of the group; a stride leaves the tokens beyond ctx unread
+    n_kv, cap = 2, 7
+    V = synth.q8_0_kv_cache(3, n_kv, cap)
+    K = synth.q8_0_kv_cache(4, n_kv, cap)
+    Q = synth.queries(5, 1, 6)
+    out = oracle.attn_decode(Q, K, V, 1, 6, n_kv, 256, 1, kv_stride=cap, fmt="q8_0")
+    Vh = oracle.dequant_q8(V, n_kv * cap, 256).reshape(n_kv, cap, 256)
+    for h in range(6):
+        assert np.array_equal(out[0, h], Vh[h // 3, 0])
+    with pytest.raises(ValueError):
+        oracle.attn_decode(Q, K, V, 1, 6, n_kv, 256, 1, fmt="q5_0")

@@ -1,7 +1,7 @@
 """Host model of the synchronisation in the tensor-memory attention kernel
 (q4kv_attn_tc.cuh): a producer thread (bulk copies into an S-slot ring), an
-MMA thread, four K warps, four V warps and four softmax warps (two P^T
-buffers; O^T rescaled only in tiles where a row maximum grows), coupled by
+MMA thread, four K warps, four V warps and four softmax warps (one or two
+P^T buffers; O^T rescaled only in tiles where a row maximum grows), coupled by
 mbarriers that are waited on by phase parity.  Random interleavings
 (asynchronous completions included) must always finish, every parity wait
 must start while its barrier is at the awaited phase or one past it (else the
@@ -26,14 +26,14 @@ class Bar:
             self.phase += 1
 
 
-def simulate(n_tiles, S, seed):
+def simulate(n_tiles, S, seed, PB=2):
     rnd = random.Random(seed)
     full = [Bar(f"full{s}", 1) for s in range(S)]
     empty = [Bar(f"empty{s}", 2 * ROLE) for s in range(S)]
     kready = [Bar(f"kready{b}", ROLE) for b in range(2)]
     sdone = [Bar(f"sdone{b}", 1) for b in range(2)]
-    pready = [Bar(f"pready{b}", ROLE) for b in range(2)]
-    pfree = [Bar(f"pfree{b}", 1) for b in range(2)]
+    pready = [Bar(f"pready{b}", ROLE) for b in range(PB)]
+    pfree = [Bar(f"pfree{b}", 1) for b in range(PB)]
     vready = [Bar(f"vready{h}", ROLE) for h in range(2)]
     pvdone = [Bar(f"pvdone{h}", 1) for h in range(2)]
     pending_copies = []      # complete in any order
@@ -74,7 +74,7 @@ def simulate(n_tiles, S, seed):
         for t in range(n_tiles):
             if t + 1 < n_tiles:
                 yield from qk(t + 1)
-            yield from wait(pready[t & 1], t >> 1)
+            yield from wait(pready[t % PB], t // PB)
             for h in range(2):
                 yield from wait(vready[h], t)
                 assert (t, h) in state["v_written"] and t in state["p_written"]
@@ -121,17 +121,17 @@ def simulate(n_tiles, S, seed):
             # the CTA-wide rescale decision of tile t (same for every warp)
             rescale = state["rescale"].setdefault(t, rnd.random() < 0.3)
             yield "barrier"
-            if t >= 2:
-                yield from wait(pfree[t & 1], (t - 2) >> 1)
-                assert ("pv", 1, t - 2) in done                # P^T buffer free
+            if t >= PB:
+                yield from wait(pfree[t % PB], (t - PB) // PB)
+                assert ("pv", 1, t - PB) in done               # P^T buffer free
             if rescale and t > 0:
                 yield from wait(pvdone[1], t - 1)
                 assert ("pv", 0, t - 1) in done and ("pv", 1, t - 1) in done   # O^T idle
             state["p_written"].add(t)
-            pready[t & 1].arrive()
+            pready[t % PB].arrive()
             yield
         if n_tiles:
-            yield from wait(pfree[(n_tiles - 1) & 1], (n_tiles - 1) >> 1)
+            yield from wait(pfree[(n_tiles - 1) % PB], (n_tiles - 1) // PB)
             assert all(("pv", h, n_tiles - 1) in done for h in range(2))
 
     actors = {"producer": producer(), "mma": mma()}
@@ -162,7 +162,7 @@ def simulate(n_tiles, S, seed):
             elif job[0] == "pv":
                 pvdone[job[1]].arrive()
             else:
-                pfree[job[1] & 1].arrive()
+                pfree[job[1] % PB].arrive()
             continue
         try:
             if next(actors[c]) == "barrier":
@@ -176,6 +176,7 @@ def simulate(n_tiles, S, seed):
 
 
 @pytest.mark.parametrize("n_tiles,S", [(1, 2), (2, 2), (3, 2), (3, 3), (5, 3), (9, 4), (16, 3), (4, 8)])
-def test_tc_attention_protocol(n_tiles, S):
+@pytest.mark.parametrize("PB", [1, 2])
+def test_tc_attention_protocol(n_tiles, S, PB):
     for seed in range(60):
-        simulate(n_tiles, S, seed)
+        simulate(n_tiles, S, seed, PB)
