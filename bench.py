@@ -276,6 +276,7 @@ def main():
     ap.add_argument("--shape", default="17408x5120", help="--case gemv: NxK")
     ap.add_argument("--ctx", type=int, default=65536, help="--case attn: ctx_len")
     ap.add_argument("--launches", type=int, default=8, help="--case gemv/attn: launches")
+    ap.add_argument("--q8", action="store_true", help="--case attn: the Q8_0 K/V cache")
     args = ap.parse_args()
     ARGS = args
     if args.warmup < 3:
@@ -744,28 +745,30 @@ def run_case(args, torch, dev):
         what = f"q4_gemv {N}x{K} M={M}"
     else:
         ctx = args.ctx
-        copies = max(2, -(-3 * L2_BYTES // (2 * N_KV * ctx * 144)))
-        caches = [(synth.device_q4_0_kv_cache(60 + i, N_KV, ctx, device=dev),
-                   synth.device_q4_0_kv_cache(80 + i, N_KV, ctx, device=dev))
+        row = 272 if args.q8 else 144
+        gen = synth.device_q8_0_kv_cache if args.q8 else synth.device_q4_0_kv_cache
+        fn = L.q8kv_attn_decode_ex if args.q8 else L.q4kv_attn_decode_ex
+        wsfn = L.q8kv_attn_workspace_bytes if args.q8 else L.q4d_attn_workspace_bytes
+        copies = max(2, -(-3 * L2_BYTES // (2 * N_KV * ctx * row)))
+        caches = [(gen(60 + i, N_KV, ctx, device=dev), gen(80 + i, N_KV, ctx, device=dev))
                   for i in range(copies)]
         Q = synth.device_bf16_normal(2, (M, N_Q, HEAD_DIM), scale=1 / 16, device=dev)
         out = torch.empty((M, N_Q, HEAD_DIM), dtype=torch.float32, device=dev)
-        ws = torch.empty(max(16, L.q4d_attn_workspace_bytes(ctx, N_Q, N_KV, HEAD_DIM, M)),
-                         dtype=torch.uint8, device=dev)
+        ws = torch.empty(max(16, wsfn(ctx, N_Q, N_KV, HEAD_DIM, M)), dtype=torch.uint8,
+                         device=dev)
         for i in range(args.launches):
             Kc, Vc = caches[i % copies]
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            st = L.q4kv_attn_decode_ex(Q.data_ptr(), Kc.data_ptr(), Vc.data_ptr(),
-                                       out.data_ptr(), ctx, N_Q, N_KV, HEAD_DIM, M, ctx, 1.0,
-                                       sptr, ws.data_ptr(), ws.numel())
+            st = fn(Q.data_ptr(), Kc.data_ptr(), Vc.data_ptr(), out.data_ptr(), ctx, N_Q, N_KV,
+                    HEAD_DIM, M, ctx, 1.0, sptr, ws.data_ptr(), ws.numel())
             b.record(stream)
             if st:
-                raise RuntimeError(f"q4kv_attn_decode_ex failed: {st}")
+                raise RuntimeError(f"attention call failed: {st}")
             torch.cuda.synchronize()
             times.append(a.elapsed_time(b) * 1e3)
-        nbytes = attn_alg_bytes(M, ctx)
-        what = f"q4kv_attn ctx={ctx} M={M}"
+        nbytes = attn_alg_bytes(M, ctx, row)
+        what = f"{'q8' if args.q8 else 'q4'}kv_attn ctx={ctx} M={M}"
     us = statistics.median(times[1:] if len(times) > 1 else times)
     print(json.dumps({"case": what, "us_median": us, "GBps": nbytes / (us * 1e-6) / 1e9,
                       "copies": copies, "launches": args.launches}), flush=True)
