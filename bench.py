@@ -482,24 +482,28 @@ def main():
     h2d = d2h = 0
 
     def e2e_step():
+        # the step's inputs (the activation rows of each width, the queries of
+        # every attention layer) come from pinned host memory; the step's
+        # results (the last output of each GEMV width, the logits, every
+        # attention output) go back to it; the kernels are the timed step's
         nonlocal h2d, d2h
         h2d = d2h = 0
-        for l in range(LAYERS):
-            for i, (N, K) in enumerate(LAYER_SHAPES):
-                xs[K].copy_(h_x[K], non_blocking=True)
-                h2d += xs[K].numel() * 2
-                gemv(layers[l][i], xs[K], ys[N], N, K)
-                h_y[N].copy_(ys[N], non_blocking=True)
-                d2h += ys[N].numel() * 4
-        xs[HIDDEN].copy_(h_x[HIDDEN], non_blocking=True)
-        h2d += xs[HIDDEN].numel() * 2
-        gemv(head, xs[HIDDEN], ys[HEAD_N], HEAD_N, HIDDEN)
-        h_y[HEAD_N].copy_(ys[HEAD_N], non_blocking=True)
-        d2h += ys[HEAD_N].numel() * 4
+        for K in xs:
+            xs[K].copy_(h_x[K], non_blocking=True)
+            h2d += xs[K].numel() * 2
         for l in range(ATTN_LAYERS):
             Qs[l].copy_(h_q[l], non_blocking=True)
             h2d += Qs[l].numel() * 2
+        for l in range(LAYERS):
+            for i, (N, K) in enumerate(LAYER_SHAPES):
+                gemv(layers[l][i], xs[K], ys[N], N, K)
+        gemv(head, xs[HIDDEN], ys[HEAD_N], HEAD_N, HIDDEN)
+        for l in range(ATTN_LAYERS):
             attn(l)
+        for N in ys:
+            h_y[N].copy_(ys[N], non_blocking=True)
+            d2h += ys[N].numel() * 4
+        for l in range(ATTN_LAYERS):
             h_o[l].copy_(outs[l], non_blocking=True)
             d2h += outs[l].numel() * 4
 
