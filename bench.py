@@ -172,6 +172,26 @@ def cpu_cores():
     return int(n)
 
 
+def reduce_over_ranks(values, device, world, op="max"):
+    """Element-wise max (or min) of per-rank floats over all ranks of the
+    process group (the timed regions' durations: the job takes as long as its
+    slowest rank).  With one rank, the values themselves."""
+    import torch
+
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.MIN)
+    return t.tolist()
+
+
+def job_tbps(bytes_per_rank_step, steps, world, max_ms):
+    """Whole-job throughput: every rank moves bytes_per_rank_step per step
+    (weak scaling), the job lasts max_ms (the slowest rank)."""
+    return bytes_per_rank_step * steps * world / (max_ms * 1e-3) / 1e12
+
+
 def oracle_sample_step(seed=0):
     """One bounded sample of the workload on the CPU oracle: a 5120->6144
     GEMV at M rows and one attention layer at ctx 4096.  Returns
@@ -404,13 +424,10 @@ def main():
     attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
     clock = clocks.stop()
 
-    t = torch.tensor([total_ms, gemv_ms, attn_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, gemv_ms, attn_ms = t.tolist()
+    total_ms, gemv_ms, attn_ms = reduce_over_ranks([total_ms, gemv_ms, attn_ms], dev, world)
 
     bytes_step = step_bytes(M)
-    value = bytes_step * K_ * world / (total_ms * 1e-3) / 1e12
+    value = job_tbps(bytes_step, K_, world, total_ms)
     peak_gbs, peak_kind = peaks()
     n_gemv = LAYERS * len(LAYER_SHAPES) + 1
     gemv_bytes = sum(gemv_alg_bytes(M, N, K) for N, K in LAYER_SHAPES) * LAYERS + \
@@ -443,10 +460,8 @@ def main():
     except Exception as e:  # noqa: BLE001 - report, keep the eager numbers
         graph_err = f"{type(e).__name__}: {e}"[:300]
         torch.cuda.synchronize()
-    ok = torch.tensor([0.0 if graph_err else 1.0], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ok, op=dist.ReduceOp.MIN)
-    if ok.item() == 1.0:
+    ok = reduce_over_ranks([0.0 if graph_err else 1.0], dev, world, op="min")[0]
+    if ok == 1.0:
         barrier()
         torch.cuda.synchronize()
         g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -456,11 +471,8 @@ def main():
         g1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        gms = torch.tensor([g0.elapsed_time(g1) / K_], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(gms, op=dist.ReduceOp.MAX)
-        graph = {"ms_per_step": gms.item(),
-                 "value": bytes_step * world / (gms.item() * 1e-3) / 1e12,
+        gms = reduce_over_ranks([g0.elapsed_time(g1) / K_], dev, world)[0]
+        graph = {"ms_per_step": gms, "value": job_tbps(bytes_step, 1, world, gms),
                  "unit": "TB/s", "replays": K_}
     else:
         graph = {"error": graph_err or "capture failed on another rank"}
@@ -517,10 +529,8 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = bytes_step * e2e_steps * world / (e2e_ms.item() * 1e-3) / 1e12
+    e2e_ms = reduce_over_ranks([e0.elapsed_time(e1)], dev, world)[0]
+    e2e_value = job_tbps(bytes_step, e2e_steps, world, e2e_ms)
 
     # -------- per-call latencies (cold L2), rank 0
     per_call = None
