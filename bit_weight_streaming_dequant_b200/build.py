@@ -34,7 +34,7 @@ def nvcc() -> str:
 
 
 def build(verbose: bool = False, extra_flags=None) -> str:
-    srcs = [os.path.join(CSRC, "q4dec.cu")]
+    srcs = [os.path.join(CSRC, "q4dec.cu"), os.path.join(CSRC, "q4d_selftest.cu")]
     cmd = [nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC,
            *srcs, "-o", LIB + ".tmp"]
     if verbose:

@@ -32,7 +32,7 @@ EXPORTS = (
     "q4d_pack_q4_0_weights", "q4d_unpack_q4_0_weights", "q4d_pack_q4_0_rows",
     "q4d_unpack_q4_0_rows", "q4kv_append", "q4_gemv_swiglu_ex",
     "q4d_gemv_swiglu_workspace_bytes", "q8kv_attn_decode_ex", "q8kv_attn_workspace_bytes",
-    "q8kv_plan_attn",
+    "q8kv_plan_attn", "q4d_wait_selftest",
 )
 
 
@@ -103,6 +103,8 @@ def lib() -> ctypes.CDLL:
     L.q8kv_attn_workspace_bytes.restype = sz
     L.q8kv_plan_attn.argtypes = [i, i, i, i, i, i, ctypes.POINTER(AttnPlan)]
     L.q8kv_plan_attn.restype = i
+    L.q4d_wait_selftest.argtypes = [vp, ctypes.c_uint, i, vp]
+    L.q4d_wait_selftest.restype = i
     for fn in ("q4_gemv", "q4_gemv_ex", "q4_gemv_ex2", "q4kv_attn_decode", "q4kv_attn_decode_ex",
                "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
                "q4kv_attn_decode_noalloc"):

@@ -328,6 +328,20 @@ q4d_status q4d_unpack_q4_0_rows(const void* rows_q4, void* blocks18, int rows, i
  */
 q4d_status q4d_device_error(int reset);
 
+/* Self-test of the bounded in-kernel wait (the mechanism behind
+ * Q4D_ERR_DEVICE_TIMEOUT), for failure-detection tests: one CTA waits on an
+ * mbarrier phase that completes only if `arrive` != 0, giving up after
+ * limit_us microseconds of wall-clock time.  The kernel ORs 2u into *word if
+ * the phase completed and 1u if the wait ran out, then returns normally (the
+ * CUDA context stays usable).
+ *   word     : device pointer to one unsigned, 4-byte aligned, caller-owned.
+ *   limit_us : 1 .. 10,000,000.
+ * Returns Q4D_ERR_INVALID_ARG / Q4D_ERR_MISALIGNED (nothing launched) or the
+ * launch status; the result is in *word after the stream synchronises.
+ * No counterpart in the source pages: a test hook of this library.
+ */
+q4d_status q4d_wait_selftest(unsigned* word, unsigned limit_us, int arrive, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -163,3 +163,11 @@ def test_swiglu_rejects_bad_arguments_without_cuda():
     # workspace: a plan over 2N rows in pairs
     assert L.q4d_gemv_swiglu_workspace_bytes(1, 8, 65536) > 0
     assert L.q4d_gemv_swiglu_workspace_bytes(1, 0, 256) == 0
+
+
+def test_wait_selftest_rejects_bad_arguments_without_cuda():
+    L = q4dec.lib()
+    assert L.q4d_wait_selftest(None, 1000, 0, None) == 1
+    assert L.q4d_wait_selftest(FAKE, 0, 0, None) == 1
+    assert L.q4d_wait_selftest(FAKE, 10_000_001, 0, None) == 1
+    assert L.q4d_wait_selftest(FAKE + 2, 1000, 0, None) == 3
