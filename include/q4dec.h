@@ -18,6 +18,11 @@
  *     context fills").  The context is split across the SMs and the partial
  *     softmax states are combined by a log-sum-exp merge.
  *
+ * Around them: q4_gemv_swiglu_ex (the feed-forward block's gate and up
+ * projections in one weight stream, with the SwiGLU epilogue), q4kv_append
+ * (quantises the verified tokens' K/V rows into the cache), and
+ * q8kv_attn_decode_ex (the same attention over an 8-bit Q8_0 cache).
+ *
  * ---------------------------------------------------------------------------
  * Storage layout (identical for weights and for the K/V cache)
  *
@@ -52,9 +57,9 @@
  *     next synchronisation.  Every wait inside a kernel is bounded in time;
  *     a wait that runs out sets a device error word readable through
  *     q4d_device_error().
- *   - Results are fp32.  Accumulation is fp32; the kernels use no atomics on
- *     results, so repeated calls with the same inputs and the same device
- *     give bitwise identical outputs.
+ *   - Results are fp32 (the GEMVs store bf16 on request).  Accumulation is
+ *     fp32; the kernels use no atomics on results, so repeated calls with
+ *     the same inputs and the same device give bitwise identical outputs.
  */
 #ifndef Q4DEC_H
 #define Q4DEC_H
