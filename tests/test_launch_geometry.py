@@ -475,3 +475,30 @@ def test_q8_unpack_constants_give_exact_codes():
                 v = np.uint16(half).view(np.float16)
                 got.append(float(np.float16(np.float32(v) * np.float32(one) + np.float32(m1152))))
         assert got == [float(q) for q in qs]
+
+
+def _bf16(bits):
+    return float(np.array([bits << 16], dtype=np.uint32).view(np.float32)[0])
+
+
+def _f16(bits):
+    return float(np.uint16(bits).view(np.float16))
+
+
+def test_q4_unpack_constants_give_exact_codes():
+    # GEMV (bf16): (w & 0x000F000F) | 0x43004300 is 128 + q in each half;
+    # subtracting bf16 136 (0x4308) leaves q - 8 exactly
+    assert _bf16(0x4300) == 128.0 and _bf16(0x4308) == 136.0
+    for q in range(16):
+        v = _bf16(0x4300 | q)
+        assert v == 128.0 + q and float(np.float32(v) - np.float32(136.0)) == q - 8
+    # attention (fp16): low nibble 0x6400 | q = 1024 + q, fma(., 1, -1032);
+    # high nibble 0x6400 | (q << 4) = 1024 + 16 q, fma(., 1/16, -72); both q - 8
+    assert _f16(0x3C00) == 1.0 and _f16(0xE408) == -1032.0
+    assert _f16(0x2C00) == 1.0 / 16 and _f16(0xD480) == -72.0
+    for q in range(16):
+        lo, hi = _f16(0x6400 | q), _f16(0x6400 | (q << 4))
+        assert lo == 1024.0 + q and hi == 1024.0 + 16 * q
+        # each fma is exact (the result is a small integer), so fp16 rounding is moot
+        assert float(np.float16(lo * 1.0 - 1032.0)) == q - 8
+        assert float(np.float16(hi * (1.0 / 16) - 72.0)) == q - 8
