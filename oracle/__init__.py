@@ -19,6 +19,11 @@ from .q4_oracle import (  # noqa: F401
     attn_decode,
     quantize_q4_0_rows,
     silu,
+    silu_prime,
+    SILU_PRIME_CRIT,
+    silu_prime_max,
+    SWIGLU_EPILOGUE_REL,
+    swiglu_tolerance,
     gemv_swiglu,
     kv_append,
 )

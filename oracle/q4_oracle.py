@@ -285,18 +285,80 @@ def silu(g):
     return out
 
 
+def silu_prime(g):
+    """d/dg silu(g) = s + g s (1 - s), s = 1 / (1 + e^-g), in fp64."""
+    g = np.asarray(g, dtype=np.float64)
+    s = 1.0 / (1.0 + np.exp(-np.clip(g, -700.0, 700.0)))
+    return s * (1.0 + g * (1.0 - s))
+
+
+def _silu_prime_critical_point() -> float:
+    """The positive root of silu''(g) = s(1 - s)(2 - g tanh(g / 2)), i.e. of
+    g tanh(g / 2) = 2 (increasing in g > 0), by bisection in fp64.  silu' has
+    its only extrema at +-this point (a maximum at +, a minimum at -)."""
+    lo, hi = 1.0, 4.0
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        if mid * np.tanh(mid / 2.0) < 2.0:
+            lo = mid
+        else:
+            hi = mid
+    return 0.5 * (lo + hi)
+
+
+SILU_PRIME_CRIT = _silu_prime_critical_point()
+
+# Relative error of the device's fp32 SwiGLU epilogue h = g / (1 + expf(-g)) * u
+# for given fp32 g and u: expf is documented to 2 ulp (2 * 2^-23 relative),
+# and the add, the IEEE division and the multiply each round once to nearest
+# (2^-24 relative each); the errors compound to at most
+# (1 + 2^-22)(1 + 2^-24)^3 - 1 < 7 * 2^-24 * (1 + 1e-6).
+SWIGLU_EPILOGUE_REL = 7.0 * 2.0 ** -24 * (1.0 + 1e-6)
+
+
+def silu_prime_max(g, t):
+    """max |silu'(xi)| over xi in [g - t, g + t]: silu' is monotonic between
+    its extrema at -SILU_PRIME_CRIT and +SILU_PRIME_CRIT, so the maximum of
+    its magnitude is at an end of the interval or at an extremum inside it."""
+    g, t = np.broadcast_arrays(np.asarray(g, dtype=np.float64), np.asarray(t, dtype=np.float64))
+    lo, hi = g - t, g + t
+    best = np.maximum(np.abs(silu_prime(lo)), np.abs(silu_prime(hi)))
+    for c in (-SILU_PRIME_CRIT, SILU_PRIME_CRIT):
+        inside = (lo <= c) & (c <= hi)
+        best = np.where(inside, np.maximum(best, abs(float(silu_prime(c)))), best)
+    return best
+
+
+def swiglu_tolerance(g, u, tg, tu):
+    """Bound on |h_dev - silu(g) u| when the device computed g and u to within
+    tg and tu (the GEMV bound) and then evaluated the SwiGLU epilogue in fp32.
+
+    With g~ = g + dg, u~ = u + du (|dg| <= tg, |du| <= tu):
+      silu(g~) u~ - silu(g) u = (silu(g~) - silu(g)) u~ + silu(g) du,
+    and by the mean value theorem |silu(g~) - silu(g)| <= D tg with
+    D = max |silu'| over [g - tg, g + tg] (D <= |silu'(g)| + tg / 2, since
+    |silu''| <= 1/2); |u~| <= |u| + tu.  So
+      |dh| <= D tg (|u| + tu) + |silu(g)| tu:
+    the first-order terms |silu'(g) u| tg + |silu(g)| tu, the cross term
+    D tg tu, and the curvature of silu over the interval through D.  The fp32
+    epilogue adds SWIGLU_EPILOGUE_REL times a bound on |silu(g~) u~|, and 1e-30
+    absolute covers fp32 underflow of silu(g~) for g~ < -87."""
+    g, u = np.asarray(g, dtype=np.float64), np.asarray(u, dtype=np.float64)
+    dsilu_span = silu_prime_max(g, tg) * tg
+    u_span = np.abs(u) + tu
+    prop = dsilu_span * u_span + np.abs(silu(g)) * tu
+    h_max = (np.abs(silu(g)) + dsilu_span) * u_span
+    return prop + SWIGLU_EPILOGUE_REL * h_max + 1e-30 * u_span
+
+
 def gemv_swiglu(W_buf, x_bits, M: int, N: int, K: int):
     """Fused gate/up GEMV + SwiGLU: ``W_buf`` holds 2N rows in the weight
     layout (gate row n at 2n, up row n at 2n + 1).  Returns ``(h, tol)``:
     ``h[m, n] = silu(g) * u`` in fp64 and the per-element bound the device
-    result must meet, propagated from the GEMV bound ``t = 2e-3 S + 1e-5`` of
-    g and u through the product: ``|silu'(g) u| t_g + |silu(g)| t_u + c t_g t_u``
-    with ``c = max |silu''| <= 0.5``, plus 1e-6 relative for the fp32 epilogue."""
+    result must meet: the GEMV bound ``t = 2e-3 S + 1e-5`` of g and of u,
+    carried through the SwiGLU by ``swiglu_tolerance``."""
     y, S = gemv(W_buf, x_bits, M, 2 * N, K)
     g, u = y[:, 0::2], y[:, 1::2]
     tg, tu = gemv_tolerance(S[:, 0::2]), gemv_tolerance(S[:, 1::2])
-    sg = 1.0 / (1.0 + np.exp(-np.clip(g, -700, 700)))
-    dsilu = sg * (1.0 + g * (1.0 - sg))
     h = silu(g) * u
-    tol = np.abs(dsilu * u) * tg + np.abs(silu(g)) * tu + 0.5 * tg * tu + 1e-6 * np.abs(h)
-    return h, tol
+    return h, swiglu_tolerance(g, u, tg, tu)

@@ -636,3 +636,109 @@ def test_q8_attention_single_token_and_stride():
         assert np.array_equal(out[0, h], Vh[h // 3, 0])
     with pytest.raises(ValueError):
         oracle.attn_decode(Q, K, V, 1, 6, n_kv, 256, 1, fmt="q5_0")
+
+
+# ------------------------------------------- SwiGLU propagated tolerance ----
+def _f32_ulps(v, k):
+    """fp32 value v moved by k ulps (k may be negative)."""
+    v = np.float32(v)
+    for _ in range(abs(k)):
+        v = np.nextafter(v, np.float32(np.inf if k > 0 else -np.inf), dtype=np.float32)
+    return v
+
+
+def _device_epilogue(g32, u32, exp_ulps):
+    """h = g / (1 + expf(-g)) * u with every fp32 operation rounded to nearest
+    and expf off by exp_ulps ulps (the documented bound is 2)."""
+    e = _f32_ulps(np.float32(math.exp(-float(g32))), exp_ulps)
+    den = np.float32(np.float32(1.0) + e)
+    return float(np.float32(np.float32(g32 / den) * u32))
+
+
+def _within(v, center, t):
+    """Closest fp32 value to v that lies within [center - t, center + t]."""
+    v = np.float32(v)
+    while abs(float(v) - center) > t:
+        v = np.nextafter(v, np.float32(center), dtype=np.float32)
+    return v
+
+
+def _worst_ratio(g, u, tg, tu, scale=1.0):
+    """max over a grid of device results (g~, u~ within tg, tu of g, u; expf
+    off by -2, 0, +2 ulps) of |h_dev - silu(g) u| / (scale * tolerance)."""
+    tol = float(oracle.swiglu_tolerance(np.array(g), np.array(u), tg, tu)) * scale
+    exact = float(oracle.silu(np.array([g]))[0]) * u
+    worst = 0.0
+    for dg in np.linspace(-tg, tg, 21):
+        g32 = _within(g + dg, g, tg)
+        for du in np.linspace(-tu, tu, 11):
+            u32 = _within(u + du, u, tu)
+            for k in (-2, 0, 2):
+                worst = max(worst, abs(_device_epilogue(g32, u32, k) - exact) / tol)
+    return worst
+
+
+SWIGLU_CASES = [(g, u, tg, tu) for g in (-30.0, -8.0, -1.278, 0.0, 0.7, 2.4, 8.0, 30.0)
+                for u in (-3.0, 1e-3, 5.0)
+                for tg, tu in ((0.02, 0.03), (0.5, 0.8), (2.0, 1.5))]
+
+
+def test_silu_prime_extrema_and_interval_maximum():
+    # silu'' = s(1 - s)(2 - g tanh(g / 2)) vanishes at +-SILU_PRIME_CRIT only,
+    # and max |silu'| over an interval (the bound's D) equals a dense-grid
+    # maximum of |silu'| over that interval
+    c = oracle.SILU_PRIME_CRIT
+    assert abs(c * math.tanh(c / 2) - 2.0) < 1e-12 and 2.39 < c < 2.41
+    g = np.linspace(-30.0, 30.0, 240001)  # 1 - s stays > 0 in fp64 here
+    s = 1.0 / (1.0 + np.exp(-g))
+    d2 = s * (1.0 - s) * (2.0 - g * np.tanh(g / 2.0))
+    sign_changes = g[1:][np.sign(d2[1:]) != np.sign(d2[:-1])]
+    assert len(sign_changes) == 2 and np.allclose(sign_changes, [-c, c], atol=1e-3)
+    h = 1e-5
+    fd = (oracle.silu_prime(g[::997] + h) - oracle.silu_prime(g[::997] - h)) / (2 * h)
+    np.testing.assert_allclose(fd, d2[::997], atol=1e-8)
+    for center in (-30.0, -8.0, -2.4, -1.0, 0.0, 1.5, 2.4, 3.0, 30.0):
+        for t in (0.01, 0.3, 2.0, 6.0):
+            grid = np.linspace(center - t, center + t, 200001)
+            dense = np.abs(oracle.silu_prime(grid)).max()
+            got = float(oracle.silu_prime_max(center, t))
+            assert dense * (1 - 1e-12) <= got <= dense * (1 + 1e-9) + 1e-15
+
+
+def test_silu_prime_is_the_derivative():
+    g = np.linspace(-40.0, 40.0, 4001)
+    h = 1e-6
+    fd = (oracle.silu(g + h) - oracle.silu(g - h)) / (2 * h)
+    np.testing.assert_allclose(oracle.silu_prime(g), fd, atol=1e-8)
+
+
+@pytest.mark.parametrize("g,u,tg,tu", SWIGLU_CASES)
+def test_swiglu_tolerance_covers_every_perturbation(g, u, tg, tu):
+    # every (g~, u~) within the GEMV bound of (g, u), evaluated as the device
+    # does in fp32 with expf at its documented 2-ulp limit, stays within the bound
+    assert _worst_ratio(g, u, tg, tu) <= 1.0
+
+
+@pytest.mark.parametrize("g", [-30.0, -8.0, 0.0, 8.0, 30.0])
+def test_swiglu_tolerance_halved_fails(g):
+    # the bound is tight to within a factor 2 at these gates: half of it is
+    # exceeded by some perturbation inside (tg, tu)
+    worst = max(_worst_ratio(g, u, tg, tu, scale=0.5)
+                for (gg, u, tg, tu) in SWIGLU_CASES if gg == g)
+    assert worst > 1.0
+
+
+def test_swiglu_tolerance_is_the_propagated_gemv_bound():
+    # the fused oracle carries the GEMV bound of each output through the SwiGLU
+    N, K, M = 5, 512, 2
+    W = synth.q4_0_weights(71, 2 * N, K)
+    x = synth.activations(72, M, K)
+    h, tol = oracle.gemv_swiglu(W, x, M, N, K)
+    y, S = oracle.gemv(W, x, M, 2 * N, K)
+    t = oracle.gemv_tolerance(S)
+    np.testing.assert_array_equal(
+        tol, oracle.swiglu_tolerance(y[:, 0::2], y[:, 1::2], t[:, 0::2], t[:, 1::2]))
+    # first-order part alone is a lower bound of it
+    g, u = y[:, 0::2], y[:, 1::2]
+    first = np.abs(oracle.silu_prime(g) * u) * t[:, 0::2] + np.abs(oracle.silu(g)) * t[:, 1::2]
+    assert np.all(tol >= first)
