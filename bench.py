@@ -75,21 +75,20 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel):
-    """DRAM bytes per launch from a committed ncu capture (the json block of
-    profiles/dram_traffic.md), if it was taken on the current kernel sources
-    (else None)."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+def recorded_traffic(kernel, M):
+    """DRAM bytes (read + write) per launch of the step's kernel at M rows, from
+    the committed ncu record profiles/dram_traffic.json, if it was taken on the
+    current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
-            text = f.read()
-        rec = json.loads(text.split("```json", 1)[1].split("```", 1)[0])
+            rec = json.load(f)
     except Exception:
         return None
-    e = rec.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if rec.get("source_hash") != kernel_source_hash():
         return None
-    return e.get("bytes_per_launch")
+    e = rec.get("step", {}).get(kernel, {}).get(f"M{M}")
+    return None if not e else e.get("bytes_per_launch")
 
 
 # ------------------------------------------------------------------ clocks --
@@ -274,7 +273,8 @@ def workload_config(args):
             "M": args.M, "ctx_len": CTX, "layers": LAYERS, "attn_layers": ATTN_LAYERS,
             "bytes_per_step": step_bytes(args.M),
             "l2": "inputs larger than L2 (17.2 GB of distinct weights/caches per step)",
-            "gemv_launch": "q4_gemv_ex2 with Q4D_GEMV_WEIGHT_PREFETCH",
+            "gemv_launch": ("one q4_gemv_batch_ex launch of the 321 matrices per step, each "
+                            "waiting for its predecessor in the layer chain"),
             "parallelism": f"replicas x{args.gpus}"}
 
 
@@ -295,8 +295,10 @@ def main():
     ap.add_argument("--impl", default="libq4dec", choices=["libq4dec", "reference"])
     ap.add_argument("--no-per-call", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--case", default="step", choices=["step", "gemv", "attn"],
-                    help="gemv/attn: a few launches of one kernel (small case for profilers)")
+    ap.add_argument("--case", default="step", choices=["step", "gemv", "gemv_batch", "attn"],
+                    help="gemv/gemv_batch/attn: a few launches of one kernel (small case for "
+                         "profilers)")
+    ap.add_argument("--layers", type=int, default=2, help="--case gemv_batch: layers per launch")
     ap.add_argument("--shape", default="17408x5120", help="--case gemv: NxK")
     ap.add_argument("--ctx", type=int, default=65536, help="--case attn: ctx_len")
     ap.add_argument("--launches", type=int, default=8, help="--case gemv/attn: launches")
@@ -342,71 +344,29 @@ def main():
     kv = [(synth.device_q4_0_kv_cache(2000 + l, N_KV, CTX, device=dev),
            synth.device_q4_0_kv_cache(2100 + l, N_KV, CTX, device=dev))
           for l in range(ATTN_LAYERS)]
-    # per-step inputs and outputs
-    xs = {K: synth.device_bf16_normal(7 + K, (M, K), device=dev) for K in (HIDDEN, FFN, QKV)}
-    ys = {N: torch.empty((M, N), dtype=torch.float32, device=dev)
-          for N in (FFN, HIDDEN, QKV, HEAD_N)}
-    Qs = [synth.device_bf16_normal(2200 + l, (M, N_Q, HEAD_DIM), scale=1 / 16, device=dev)
-          for l in range(ATTN_LAYERS)]
-    outs = [torch.empty((M, N_Q, HEAD_DIM), dtype=torch.float32, device=dev)
-            for _ in range(ATTN_LAYERS)]
     L = q4dec.lib()
-    gws = max([L.q4d_gemv_workspace_bytes(M, N, K) for N, K in LAYER_SHAPES + [(HEAD_N, HIDDEN)]])
-    aws = L.q4d_attn_workspace_bytes(CTX, N_Q, N_KV, HEAD_DIM, M)
-    ws = torch.empty(max(gws, aws, 16), dtype=torch.uint8, device=dev)
+    step = DecodeStep(torch, q4dec, synth, dev, layers, head, kv, M)
+    m5 = DecodeStep(torch, q4dec, synth, dev, layers, head, kv, 5) if M != 5 else None
     torch.cuda.synchronize()
     gen_s = time.time() - gen_t0
 
     stream = torch.cuda.current_stream()
-    sptr = stream.cuda_stream
-    launches = {"n": 0}
-
-    def gemv(W, x, y, N, K):
-        # weights are immutable: each call may stream its first stages while
-        # the kernel before it finishes (programmatic dependent launch)
-        st = L.q4_gemv_ex2(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K,
-                           torch.cuda.current_stream().cuda_stream, ws.data_ptr(), ws.numel(),
-                           q4dec.GEMV_WEIGHT_PREFETCH)
-        if st:
-            raise RuntimeError(f"q4_gemv_ex2 failed: {st}")
-        launches["n"] += 1 + (1 if L.q4d_gemv_workspace_bytes(M, N, K) else 0)
-
-    def attn(l):
-        Kc, Vc = kv[l]
-        st = L.q4kv_attn_decode_ex(Qs[l].data_ptr(), Kc.data_ptr(), Vc.data_ptr(),
-                                   outs[l].data_ptr(), CTX, N_Q, N_KV, HEAD_DIM, M, CTX,
-                                   1.0, torch.cuda.current_stream().cuda_stream,
-                                   ws.data_ptr(), ws.numel())
-        if st:
-            raise RuntimeError(f"q4kv_attn_decode_ex failed: {st}")
-        launches["n"] += 2 if aws else 1
-
-    def gemv_stream():
-        for l in range(LAYERS):
-            for i, (N, K) in enumerate(LAYER_SHAPES):
-                gemv(layers[l][i], xs[K], ys[N], N, K)
-        gemv(head, xs[HIDDEN], ys[HEAD_N], HEAD_N, HIDDEN)
-
-    def attn_stream():
-        for l in range(ATTN_LAYERS):
-            attn(l)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     clocks = ClockSampler(local)
-
     for _ in range(args.warmup):
-        gemv_stream()
-        attn_stream()
+        step.gemv_stream()
+        step.attn_stream()
     torch.cuda.synchronize()
 
     # -------- timed region
     K_ = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(K_)]
-    launches["n"] = 0
+    step.launches = 0
     barrier()
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
@@ -415,14 +375,14 @@ def main():
     t_start.record(stream)
     for k in range(K_):
         ev[k][0].record(stream)
-        gemv_stream()
+        step.gemv_stream()
         ev[k][1].record(stream)
-        attn_stream()
+        step.attn_stream()
         ev[k][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
-    timed_launches = launches["n"]
+    timed_launches = step.launches
     total_ms = t_start.elapsed_time(t_end)
     gemv_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
     attn_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
@@ -433,16 +393,42 @@ def main():
     bytes_step = step_bytes(M)
     value = job_tbps(bytes_step, K_, world, total_ms)
     peak_gbs, peak_kind = peaks()
-    n_gemv = LAYERS * len(LAYER_SHAPES) + 1
-    gemv_bytes = sum(gemv_alg_bytes(M, N, K) for N, K in LAYER_SHAPES) * LAYERS + \
-        gemv_alg_bytes(M, HEAD_N, HIDDEN)
-    per_launch_bytes = gemv_bytes / n_gemv
-    per_launch_s = gemv_ms * 1e-3 / (K_ * n_gemv)
-    achieved_gbs = per_launch_bytes / per_launch_s / 1e9
+    gemv_bytes = gemv_step_bytes(M)
+    gemv_launch_s = gemv_ms * 1e-3 / K_            # one batch launch per step
+    achieved_gbs = gemv_bytes / gemv_launch_s / 1e9
     attn_gbs = ATTN_LAYERS * attn_alg_bytes(M, CTX) * K_ / (attn_ms * 1e-3) / 1e9
 
-    # -------- the same step replayed as one CUDA graph (353 kernel nodes; the
-    # weight-prefetching GEMVs keep their programmatic dependencies)
+    # -------- the same weight stream as 321 separate launches (one per matrix,
+    # weight prefetch under programmatic dependent launch), for comparison
+    sep = time_region(torch, stream, lambda: step.gemv_stream_per_matrix(), max(3, K_ // 5))
+    sep_ms = reduce_over_ranks([sep], dev, world)[0]
+    per_matrix = {"ms_per_step": sep_ms, "value": gemv_bytes / (sep_ms * 1e-3) / 1e12,
+                  "unit": "TB/s", "launches_per_step": step.n_gemv}
+
+    # -------- the step at M = 5 (target verification of a 4-token draft)
+    m5_rec = None
+    if m5 is not None:
+        for _ in range(args.warmup):
+            m5.gemv_stream()
+            m5.attn_stream()
+        k5 = max(5, K_ // 5)
+        g5 = time_region(torch, stream, m5.gemv_stream, k5)
+        a5 = time_region(torch, stream, m5.attn_stream, k5)
+        t5 = time_region(torch, stream, lambda: (m5.gemv_stream(), m5.attn_stream()), k5)
+        g5, a5, t5 = reduce_over_ranks([g5, a5, t5], dev, world)
+        gb5 = gemv_step_bytes(5) / (g5 * 1e-3) / 1e9
+        ab5 = ATTN_LAYERS * attn_alg_bytes(5, CTX) / (a5 * 1e-3) / 1e9
+        m5_rec = {"M": 5, "steps": k5, "ms_per_step": t5,
+                  "value": job_tbps(step_bytes(5), 1, world, t5), "unit": "TB/s",
+                  "bytes_per_step": step_bytes(5),
+                  "roofline": {"bound": "hbm", "kernel": "q4_gemv_kernel<5> (one launch)",
+                               "achieved": gb5, "peak": peak_gbs, "unit": "GB/s",
+                               "frac": gb5 / peak_gbs, "launch_us": g5 * 1e3},
+                  "attention": {"achieved_gbs": ab5, "frac": ab5 / peak_gbs,
+                                "us_per_layer": a5 * 1e3 / ATTN_LAYERS}}
+        del m5
+
+    # -------- the same step replayed as one CUDA graph
     graph = None
     g = None
     try:
@@ -450,12 +436,12 @@ def main():
         s_cap = torch.cuda.Stream()
         s_cap.wait_stream(stream)
         with torch.cuda.stream(s_cap):
-            gemv_stream()
-            attn_stream()
+            step.gemv_stream()
+            step.attn_stream()
         torch.cuda.synchronize()
         with torch.cuda.graph(g, stream=s_cap):
-            gemv_stream()
-            attn_stream()
+            step.gemv_stream()
+            step.attn_stream()
         torch.cuda.synchronize()
         for _ in range(args.warmup):
             g.replay()
@@ -467,15 +453,9 @@ def main():
     ok = reduce_over_ranks([0.0 if graph_err else 1.0], dev, world, op="min")[0]
     if ok == 1.0:
         barrier()
-        torch.cuda.synchronize()
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        g0.record(stream)
-        for _ in range(K_):
-            g.replay()
-        g1.record(stream)
-        torch.cuda.synchronize()
+        gms = time_region(torch, stream, g.replay, K_)
         barrier()
-        gms = reduce_over_ranks([g0.elapsed_time(g1) / K_], dev, world)[0]
+        gms = reduce_over_ranks([gms], dev, world)[0]
         graph = {"ms_per_step": gms, "value": job_tbps(bytes_step, 1, world, gms),
                  "unit": "TB/s", "replays": K_}
     else:
@@ -484,62 +464,19 @@ def main():
     torch.cuda.synchronize()
 
     # -------- end to end through the public API with host buffers
-    import torch as _t
-
     e2e_steps = max(3, min(K_, 10))
-    h_x = {K: _t.empty((M, K), dtype=_t.bfloat16, pin_memory=True) for K in xs}
-    for K in xs:
-        h_x[K].copy_(xs[K])
-    h_q = [_t.empty((M, N_Q, HEAD_DIM), dtype=_t.bfloat16, pin_memory=True) for _ in Qs]
-    for l in range(ATTN_LAYERS):
-        h_q[l].copy_(Qs[l])
-    h_y = {N: _t.empty((M, N), dtype=_t.float32, pin_memory=True) for N in ys}
-    h_o = [_t.empty((M, N_Q, HEAD_DIM), dtype=_t.float32, pin_memory=True) for _ in outs]
-    h2d = d2h = 0
-
-    def e2e_step():
-        # the step's inputs (the activation rows of each width, the queries of
-        # every attention layer) come from pinned host memory; the step's
-        # results (the last output of each GEMV width, the logits, every
-        # attention output) go back to it; the kernels are the timed step's
-        nonlocal h2d, d2h
-        h2d = d2h = 0
-        for K in xs:
-            xs[K].copy_(h_x[K], non_blocking=True)
-            h2d += xs[K].numel() * 2
-        for l in range(ATTN_LAYERS):
-            Qs[l].copy_(h_q[l], non_blocking=True)
-            h2d += Qs[l].numel() * 2
-        for l in range(LAYERS):
-            for i, (N, K) in enumerate(LAYER_SHAPES):
-                gemv(layers[l][i], xs[K], ys[N], N, K)
-        gemv(head, xs[HIDDEN], ys[HEAD_N], HEAD_N, HIDDEN)
-        for l in range(ATTN_LAYERS):
-            attn(l)
-        for N in ys:
-            h_y[N].copy_(ys[N], non_blocking=True)
-            d2h += ys[N].numel() * 4
-        for l in range(ATTN_LAYERS):
-            h_o[l].copy_(outs[l], non_blocking=True)
-            d2h += outs[l].numel() * 4
-
-    e2e_step()
+    step.e2e_step()
     torch.cuda.synchronize()
     barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    e2e_ms = time_region(torch, stream, step.e2e_step, e2e_steps)
     barrier()
-    e2e_ms = reduce_over_ranks([e0.elapsed_time(e1)], dev, world)[0]
-    e2e_value = job_tbps(bytes_step, e2e_steps, world, e2e_ms)
+    e2e_ms = reduce_over_ranks([e2e_ms], dev, world)[0]
+    e2e_value = job_tbps(bytes_step, 1, world, e2e_ms)
 
     # -------- per-call latencies (cold L2), rank 0
     per_call = None
     if rank == 0 and not args.no_per_call:
-        per_call = per_call_table(torch, L, dev, layers, kv, ws, peak_gbs)
+        per_call = per_call_table(torch, L, dev, layers, kv, peak_gbs)
 
     base = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -556,17 +493,22 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(args),
         "frac_of_peak": value / world / (peak_gbs / 1e3),
-        "roofline": {"bound": "hbm", "kernel": "q4_gemv_kernel", "achieved": achieved_gbs,
+        "roofline": {"bound": "hbm", "kernel": f"q4_gemv_kernel<{M}> (one launch per step)",
+                     "achieved": achieved_gbs,
                      "peak": peak_gbs, "peak_source": f"{peak_kind} hbm_gbs", "unit": "GB/s",
                      "frac": achieved_gbs / peak_gbs,
-                     "traffic": recorded_traffic("q4_gemv_kernel"),
-                     "algorithmic_bytes_per_launch": per_launch_bytes,
-                     "launch_us": per_launch_s * 1e6},
+                     "traffic": recorded_traffic("q4_gemv_kernel", M),
+                     "algorithmic_bytes_per_launch": gemv_bytes,
+                     "launch_us": gemv_launch_s * 1e6,
+                     "matrices_per_launch": step.n_gemv},
         "attention": {"achieved_gbs": attn_gbs, "frac": attn_gbs / peak_gbs,
-                      "us_per_layer": attn_ms * 1e3 / (K_ * ATTN_LAYERS)},
+                      "us_per_layer": attn_ms * 1e3 / (K_ * ATTN_LAYERS),
+                      "traffic": recorded_traffic("q4kv_attn", M)},
+        "m5": m5_rec,
+        "gemv_one_launch_per_matrix": per_matrix,
         "cpu_baseline": base,
-        "e2e": {"value": e2e_value, "unit": "TB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "e2e": {"value": e2e_value, "unit": "TB/s", "h2d_bytes_per_step": step.h2d,
+                "d2h_bytes_per_step": step.d2h, "steps": e2e_steps},
         "gpu_launches": timed_launches,
         "clocks": clock,
         "graph": graph,
@@ -576,9 +518,147 @@ def main():
     print(json.dumps(line), flush=True)
 
 
-def per_call_table(torch, L, dev, layers, kv, ws, peak_gbs, reps=15):
-    """Median device time of single calls with L2 flushed before each call."""
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+def time_region(torch, stream, fn, reps):
+    """Device time of `reps` calls of fn on `stream` (CUDA events, synchronised
+    on both sides); ms per call."""
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def gemv_step_bytes(M):
+    return sum(gemv_alg_bytes(M, N, K) for N, K in LAYER_SHAPES) * LAYERS + \
+        gemv_alg_bytes(M, HEAD_N, HIDDEN)
+
+
+class DecodeStep:
+    """One decode step at M rows on resident weights and caches.
+
+    The 321 GEMVs run as one batch launch (q4_gemv_batch_ex) in the order of a
+    layer -- in-projection, out-projection, gate, up, down -- then the head,
+    with the dependencies of a real layer: out waits for in, gate and up for
+    out (not for each other), down for up (and so gate), the next layer's in
+    for down, the head for the last down.  Each matrix type writes its own
+    output buffer; the activations are fixed synthetic inputs (a real chain
+    would feed each output on, through the attention and norm steps that are
+    not part of this path)."""
+
+    def __init__(self, torch, q4dec, synth, dev, layers, head, kv, M):
+        self.torch, self.q4dec, self.L, self.dev, self.M = torch, q4dec, q4dec.lib(), dev, M
+        self.layers, self.head, self.kv = layers, head, kv
+        self.xs = {K: synth.device_bf16_normal(7 + K + 100 * M, (M, K), device=dev)
+                   for K in (HIDDEN, FFN, QKV)}
+        names = ("gate", "up", "down", "in", "out")
+        self.ys = {n: torch.empty((M, N), dtype=torch.float32, device=dev)
+                   for n, (N, K) in zip(names, LAYER_SHAPES)}
+        self.ys["head"] = torch.empty((M, HEAD_N), dtype=torch.float32, device=dev)
+        self.Qs = [synth.device_bf16_normal(2200 + l + 100 * M, (M, N_Q, HEAD_DIM), scale=1 / 16,
+                                            device=dev) for l in range(ATTN_LAYERS)]
+        self.outs = [torch.empty((M, N_Q, HEAD_DIM), dtype=torch.float32, device=dev)
+                     for _ in range(ATTN_LAYERS)]
+        order = (3, 4, 0, 1, 2)                      # in, out, gate, up, down
+        jobs, prev_down = [], -1
+        for l in range(LAYERS):
+            base = len(jobs)
+            waits = {3: prev_down, 4: base, 0: base + 1, 1: base + 1, 2: base + 3}
+            for i in order:
+                N, K = LAYER_SHAPES[i]
+                jobs.append(dict(W=layers[l][i], x=self.xs[K], y=self.ys[names[i]], N=N, K=K,
+                                 wait_for=waits[i]))
+            prev_down = base + 4
+        jobs.append(dict(W=head, x=self.xs[HIDDEN], y=self.ys["head"], N=HEAD_N, K=HIDDEN,
+                         wait_for=prev_down))
+        self.jobs = jobs
+        self.n_gemv = len(jobs)
+        self.batch = q4dec.GemvBatch(jobs)
+        self.aws = self.L.q4d_attn_workspace_bytes(CTX, N_Q, N_KV, HEAD_DIM, M)
+        self.attn_ws = torch.empty(max(self.aws, 16), dtype=torch.uint8, device=dev)
+        self.gemv_ws = torch.empty(max(16, max(self.L.q4d_gemv_workspace_bytes(M, N, K)
+                                               for N, K in LAYER_SHAPES + [(HEAD_N, HIDDEN)])),
+                                   dtype=torch.uint8, device=dev)
+        self.launches = 0
+        self.h2d = self.d2h = 0
+        self.h_x = {K: torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
+                    for K in self.xs}
+        for K in self.xs:
+            self.h_x[K].copy_(self.xs[K])
+        self.h_q = [torch.empty((M, N_Q, HEAD_DIM), dtype=torch.bfloat16, pin_memory=True)
+                    for _ in self.Qs]
+        for q, h in zip(self.Qs, self.h_q):
+            h.copy_(q)
+        self.h_y = {n: torch.empty_like(y, device="cpu").pin_memory() for n, y in self.ys.items()}
+        self.h_o = [torch.empty((M, N_Q, HEAD_DIM), dtype=torch.float32, pin_memory=True)
+                    for _ in self.outs]
+
+    def gemv_stream(self):
+        # one launch; the weights of later matrices stream while earlier ones
+        # finish (programmatic dependent launch against the previous kernel)
+        self.batch.run(weight_prefetch=True)
+        self.launches += 1
+
+    def gemv_stream_per_matrix(self):
+        torch, L, M = self.torch, self.L, self.M
+        sptr = torch.cuda.current_stream().cuda_stream
+        for j in self.jobs:
+            st = L.q4_gemv_ex2(j["W"].data_ptr(), j["x"].data_ptr(), j["y"].data_ptr(), M,
+                               j["N"], j["K"], sptr, self.gemv_ws.data_ptr(),
+                               self.gemv_ws.numel(), self.q4dec.GEMV_WEIGHT_PREFETCH)
+            if st:
+                raise RuntimeError(f"q4_gemv_ex2 failed: {st}")
+
+    def attn(self, l):
+        torch, L, M = self.torch, self.L, self.M
+        Kc, Vc = self.kv[l]
+        st = L.q4kv_attn_decode_ex(self.Qs[l].data_ptr(), Kc.data_ptr(), Vc.data_ptr(),
+                                   self.outs[l].data_ptr(), CTX, N_Q, N_KV, HEAD_DIM, M, CTX,
+                                   1.0, torch.cuda.current_stream().cuda_stream,
+                                   self.attn_ws.data_ptr(), self.attn_ws.numel())
+        if st:
+            raise RuntimeError(f"q4kv_attn_decode_ex failed: {st}")
+        self.launches += 2 if self.aws else 1
+
+    def attn_stream(self):
+        for l in range(ATTN_LAYERS):
+            self.attn(l)
+
+    def e2e_step(self):
+        # the step's inputs (the activation rows of each width, every attention
+        # layer's queries) come from pinned host memory; its results (the last
+        # output of each matrix type, the logits, every attention output) go
+        # back to it; the kernels are the timed step's
+        self.h2d = self.d2h = 0
+        for K in self.xs:
+            self.xs[K].copy_(self.h_x[K], non_blocking=True)
+            self.h2d += self.xs[K].numel() * 2
+        for q, h in zip(self.Qs, self.h_q):
+            q.copy_(h, non_blocking=True)
+            self.h2d += q.numel() * 2
+        self.gemv_stream()
+        self.attn_stream()
+        for n, y in self.ys.items():
+            self.h_y[n].copy_(y, non_blocking=True)
+            self.d2h += y.numel() * 4
+        for o, h in zip(self.outs, self.h_o):
+            h.copy_(o, non_blocking=True)
+            self.d2h += o.numel() * 4
+
+
+def per_call_table(torch, L, dev, layers, kv, peak_gbs, reps=15):
+    """Median device time of single calls, L2 flushed before each call by
+    reading a buffer twice its size (which also writes back any dirty lines
+    before the timed call starts)."""
+    flush_buf = torch.ones(2 * L2_BYTES // 4, dtype=torch.int32, device=dev)
+
+    class _Flush:
+        def fill_(self, _):
+            flush_buf.sum()
+
+    flush = _Flush()
     need = max([L.q4d_gemv_workspace_bytes(M, N, K) for M in range(1, 6)
                 for N, K in LAYER_SHAPES] +
                [L.q4d_attn_workspace_bytes(c, N_Q, N_KV, HEAD_DIM, M) for M in (1, 5)
@@ -588,7 +668,7 @@ def per_call_table(torch, L, dev, layers, kv, ws, peak_gbs, reps=15):
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     sptr = stream.cuda_stream
-    table = {"gemv": [], "attn": [], "l2": "flushed before every call (256 MB write)"}
+    table = {"gemv": [], "attn": [], "l2": "flushed before every call (252 MB read)"}
     names = {(FFN, HIDDEN): "5120->17408", (HIDDEN, FFN): "17408->5120",
              (QKV, HIDDEN): "5120->6144", (HIDDEN, QKV): "6144->5120"}
     shape_idx = {(FFN, HIDDEN): 0, (HIDDEN, FFN): 2, (QKV, HIDDEN): 3, (HIDDEN, QKV): 4}
@@ -740,7 +820,24 @@ def run_case(args, torch, dev):
     stream = torch.cuda.current_stream()
     sptr = stream.cuda_stream
     times = []
-    if args.case == "gemv":
+    if args.case == "gemv_batch":
+        # the step's batch launch over `layers` layers (5 matrices each, in the
+        # step's order and dependencies), on distinct weights per launch
+        copies = 2
+        sets = [[[synth.device_q4_0_weights(300 + 50 * c + 5 * l + i, N, K, device=dev)
+                  for i, (N, K) in enumerate(LAYER_SHAPES)] for l in range(args.layers)]
+                for c in range(copies)]
+        steps = [DecodeStepGemvOnly(torch, q4dec, synth, dev, sets[c], M) for c in range(copies)]
+        for i in range(args.launches):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            steps[i % copies].batch.run()
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b) * 1e3)
+        nbytes = sum(gemv_alg_bytes(M, N, K) for N, K in LAYER_SHAPES) * args.layers
+        what = f"q4_gemv batch of {args.layers} layers ({5 * args.layers} matrices) M={M}"
+    elif args.case == "gemv":
         N, K = (int(v) for v in args.shape.lower().split("x"))
         copies = max(2, -(-3 * L2_BYTES // q4_bytes(N, K)))
         Ws = [synth.device_q4_0_weights(50 + i, N, K, device=dev) for i in range(copies)]
@@ -790,6 +887,27 @@ def run_case(args, torch, dev):
     us = statistics.median(times[1:] if len(times) > 1 else times)
     print(json.dumps({"case": what, "us_median": us, "GBps": nbytes / (us * 1e-6) / 1e9,
                       "copies": copies, "launches": args.launches}), flush=True)
+
+
+class DecodeStepGemvOnly:
+    """The step's GEMV batch over the given layers only (no head, no caches):
+    a small case of the same launch for profilers."""
+
+    def __init__(self, torch, q4dec, synth, dev, layers, M):
+        xs = {K: synth.device_bf16_normal(7 + K, (M, K), device=dev) for K in (HIDDEN, FFN, QKV)}
+        names = ("gate", "up", "down", "in", "out")
+        ys = {n: torch.empty((M, N), dtype=torch.float32, device=dev)
+              for n, (N, K) in zip(names, LAYER_SHAPES)}
+        jobs, prev_down = [], -1
+        for layer in layers:
+            base = len(jobs)
+            waits = {3: prev_down, 4: base, 0: base + 1, 1: base + 1, 2: base + 3}
+            for i in (3, 4, 0, 1, 2):
+                N, K = LAYER_SHAPES[i]
+                jobs.append(dict(W=layer[i], x=xs[K], y=ys[names[i]], N=N, K=K, wait_for=waits[i]))
+            prev_down = base + 4
+        self.keep = (xs, ys)
+        self.batch = q4dec.GemvBatch(jobs)
 
 
 ARGS = None

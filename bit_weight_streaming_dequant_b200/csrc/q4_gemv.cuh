@@ -1,407 +1,693 @@
-// Q4_0 GEMV / skinny GEMM for M = 1..5 rows with register dequantisation
-// feeding mma.sync (m16n8k16, bf16 in, fp32 accumulate).
+// Q4_0 GEMV / skinny GEMM for M = 1..5 activation rows, one or many matrices
+// per launch, with register dequantisation feeding mma.sync (m16n8k16, bf16
+// in, fp32 accumulate).
 //
-// Why tensor-core instructions for a bandwidth-bound GEMV: on B200 the
-// logic/integer pipe runs at half the FP32 rate, and unpacking nibbles plus
-// one FMA per weight per row keeps the SM issue-bound well below HBM speed
-// (the CUDA-core formulation measured ~4.8 thread instructions per weight at
-// M = 1).  Letting mma.sync do the multiply-adds leaves ~2 instructions per
-// weight -- the unpack -- for every M up to 8, so M = 2..5 verification rows
+// What it computes: y[m][n] = sum_k d * (q - 8) * x[m][k] over the Q4_0 blocks
+// of weight row n -- the quantised weight stream that decode repeatedly
+// reads ("Qwen3.8-27B at 256K on a 24GB RTX PRO 4000 SFF (432 GB/s): 50 tok/s
+// with MTP", paragraph beginning "NVIDIA quotes 432 GB/s"); M = 2..5 rows are
+// the target model verifying a drafted block, which shares one weight stream
 // ("Qwen3.8-27B on RTX 4090: 5,000 tok/s Prefill Reproduced", section "MTP
-// helps ordinary prose ...") cost the same as plain decode.
+// helps ordinary prose, but acceptance controls the gain").
 //
 // Exactness: q - 8 is an integer in [-8, 7], exact in bf16; x is bf16; their
-// products are exact in fp32.  Each 32-element block gets its own fresh
+// products are exact in fp32.  Each 32-element block gets its own fresh MMA
 // accumulator, multiplied by the block's fp16 scale d in fp32 and added to the
-// row's fp32 sum -- the Q4_0 definition w = d * (q - 8) ("Qwen3.8-27B at 256K
-// on a 24GB RTX PRO 4000 SFF (432 GB/s): 50 tok/s with MTP", paragraph on
-// public GGUFs at 40K context names the format) with fp32 rounding only.
+// row's fp32 sum, so the only roundings are fp32 additions.
 //
-// Layout of the work:
-//  * Weights are stored super-block-column-major: column s holds super-block
-//    s of every row, so the rows a CTA owns form one contiguous piece of each
-//    column -- every pipeline stage is a single contiguous bulk copy per
-//    column, the access pattern that streams HBM fastest.
-//  * CTA c owns rows [N*c/G, N*(c+1)/G) of one K range (k_splits > 1 only for
-//    very few rows); rows are processed in passes of up to 8 m16 tiles; a
-//    pass streams its K range KC super-block columns per stage.
-//  * Warp specialisation: one producer warp issues the copies (bulk copy of
-//    the weight piece, TMA box of the activations) into a ring of stages that
-//    complete on "full" mbarriers; eight consumer warps compute and release
-//    each stage on an "empty" mbarrier, so loads and math overlap with no
-//    CTA-wide barrier per stage.  Every wait is bounded in time.
-//  * Consumer warp w takes block w of each super-block; it builds the B
-//    fragment (x) of its block once per column and applies it to every m-tile
-//    of the pass.  At the end of a pass the eight warps' partial sums are
-//    added in a fixed order through shared memory (deterministic).
-//  * A-fragment k order: lane (g, t) dequantises word t of a block (bytes
-//    4t..4t+3) of rows g and g+8; its four bf16 pairs (low nibbles of bytes
-//    0/2, high nibbles of bytes 0/2, low of 1/3, high of 1/3) are the fragment
-//    registers of the block's two k16 steps; the B fragment takes x in the
-//    same element order, so the permutation cancels in the dot product.
-//    Rows land at a 144-byte pitch, at which the 32 lanes' 4-byte nibble
-//    loads hit 32 distinct banks.
+// Why tensor-core instructions for a bandwidth-bound GEMV: unpacking nibbles
+// keeps the half-rate integer pipe busy (three shifts and four masks per eight
+// weights, plus four bf16 subtractions on the fp16 pipe); letting mma.sync do
+// the multiply-adds leaves that unpack as the only per-weight work, for every
+// M up to 8.
+//
+// Work decomposition (stream-K):
+//  * A matrix is cut into row blocks of 128 rows (8 m16 tiles) and, along K,
+//    into units of two super-block columns (512 elements).  The units, row
+//    block after row block, are shared out in equal contiguous ranges over the
+//    CTAs (one CTA per SM), so every CTA streams the same number of bytes
+//    whatever N and K are, and every pass keeps 8 tiles of independent work.
+//    Where the units do not divide evenly, some CTAs get one more; a job's
+//    CTA numbering is rotated by the units of the jobs before it, so that
+//    over a batch those extra units land on different CTAs.
+//  * A CTA's range covers the tail of one row block, whole row blocks and the
+//    head of another.  A row block covered by one CTA is written directly; a
+//    row block shared by several CTAs is finished by the last contributor to
+//    arrive: each writes its partial sums into its own slot of the workspace
+//    and counts itself in on the row block's counter; the last one adds the
+//    slots in slot (K) order -- the result does not depend on arrival order --
+//    and resets the counter to zero.  Counters carry the launch's 48-bit tag
+//    next to their 16-bit count: a counter holding another tag (left over by
+//    another use of the memory) counts as zero, so the workspace needs no
+//    clearing, and the resets keep replays of a captured launch (same tag)
+//    correct.
+//  * Several matrices ("jobs") can run in one launch.  The producer keeps
+//    streaming the next job's weights (they depend on nothing) while a job's
+//    activations wait for the job they depend on: each CTA counts itself in on
+//    a per-job counter when it has finished that job, and a job's activation
+//    copies are issued only once its prerequisite's counter is complete.  These
+//    counters live in the launch descriptor, which the host hands over zeroed;
+//    the last CTA to leave the launch sets them back to zero.
+//  * Weights are stored super-block-column-major: the 128 rows of a row block
+//    are one contiguous piece of each column, so a unit is two bulk copies of
+//    18 KB plus one copy of each activation row's 1 KB, issued by a producer
+//    warp into a ring of stages that complete on "full" mbarriers.  Sixteen
+//    consumer warps take one (column, block) task each per stage and release
+//    it on an "empty" mbarrier.  At the end of each row block segment they add
+//    their 16 partial sums in a fixed order through shared memory into one of
+//    four segment buffers and go on with the next stage; two epilogue warps,
+//    taking alternate segments, write them out (y, or the partial slot and,
+//    when last, the sum of the slots), publish them with one release fence
+//    each and count the CTA in for a job once both have written all of its
+//    segments, so no global write, fence or atomic stalls the consumers.
+//  * Every wait is bounded in time.  A wait that runs out sets the device
+//    error word and a per-CTA abort flag; from then on no wait blocks, the
+//    producer issues no further copies and waits for the ones in flight, and
+//    every role still runs its loop to the end, so the kernel terminates.
+//
+// A-fragment k order: lane (g, t) dequantises word t of a block (bytes
+// 4t..4t+3) of rows g and g+8; its four bf16 pairs (low nibbles of bytes 0/2,
+// high nibbles of bytes 0/2, low of 1/3, high of 1/3) are the fragment
+// registers of the block's two k16 steps; the B fragment takes x in the same
+// element order, so the permutation cancels in the dot product.  Rows land at
+// a 144-byte pitch, at which the 32 lanes' 4-byte nibble loads hit 32
+// distinct banks.
 #pragma once
 
-#include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "q4dec_device.cuh"
 
 namespace q4d {
 
-constexpr int kMmaMaxTiles = 8;  // m16 tiles per pass (128 rows)
-constexpr int kMmaMaxStages = 16;
+constexpr int kGemvTiles = 8;                              // m16 tiles per row block
+constexpr int kGemvRows = 16 * kGemvTiles;                 // 128 weight rows
+constexpr int kGemvCols = 2;                               // super-block columns per unit
+constexpr int kGemvConsumerWarps = 8 * kGemvCols;          // one (column, block) task each
+constexpr int kGemvProducerWarp = kGemvConsumerWarps;      // bulk copies
+constexpr int kGemvEpilogueWarps = 2;                      // output writes, counters
+constexpr int kGemvThreads = (kGemvConsumerWarps + 1 + kGemvEpilogueWarps) * 32;
+constexpr int kGemvSegBufs = 4;                            // segment buffers (consumers -> epilogue)
+constexpr int kGemvMaxStages = 8;
+constexpr uint32_t kSbBytes = 144;                         // one super-block
+constexpr uint32_t kGemvWBox = kGemvRows * kSbBytes;       // one column of a row block
+constexpr uint32_t kJobOutBf16 = 1u;                       // y stored as bf16 (RNE)
+constexpr uint32_t kJobSwiglu = 2u;                        // rows are gate / up pairs
 
-// Kernel parameters.  The tensor map describes x as a bf16 tensor [M][K]
-// with boxes of [M][256] (one super-block column); passed as a
-// __grid_constant__ so the TMA unit reads it from the parameter space.
-struct alignas(64) GemvArgs {
-  CUtensorMap xmap;
-  const uint8_t* W;    // super-block-column-major weights, [K/256][N] x 144 B
-  float* out;          // y [M][N] or partials [k_splits][M][N]
-  unsigned* err;
-  int out_bf16;        // 1: y (no K split) is stored as bf16 [M][N], rounded to nearest even
-  int N;
-  int sb_per_split;    // super-blocks per K range
-  int rows_per_pass;   // multiple of 16, <= 128
-  int grid_rows;
-  int stages;
+// One pipeline stage: the unit's two weight pieces, then M activation rows of
+// two columns (1 KB each, the second half unused when the unit has one column).
+__host__ __device__ constexpr uint32_t gemv_stage_bytes(int M) {
+  return kGemvCols * kGemvWBox + uint32_t(M) * kGemvCols * 512u;
+}
+// Cross-warp reduction buffer: 8 slots x 8 tiles x 16 rows x M columns, fp32.
+__host__ __device__ constexpr uint32_t gemv_red_bytes(int M) {
+  return 8u * kGemvTiles * 16u * uint32_t(M) * 4u;
+}
+// Segment buffers: [4][M][128] fp32.
+__host__ __device__ constexpr uint32_t gemv_fin_bytes(int M) {
+  return uint32_t(kGemvSegBufs) * uint32_t(M) * kGemvRows * 4u;
+}
+// Shared memory: ring, reduction buffer, segment buffers, flags (abort, two
+// epilogue progress counts; padded to 16), 2 barriers per stage and 2 per
+// segment buffer.
+__host__ __device__ constexpr size_t gemv_smem_bytes(int M, int stages) {
+  return size_t(stages) * gemv_stage_bytes(M) + gemv_red_bytes(M) + gemv_fin_bytes(M) + 16 +
+         size_t(stages) * 16 + size_t(kGemvSegBufs) * 16;
+}
+
+// First unit of (job-local) CTA c when U units are shared out over G CTAs
+// (G <= U), and the CTA whose range holds unit u.  32-bit arithmetic: the host
+// accepts only U * G < 2^31.
+__host__ __device__ __forceinline__ int unit_begin(int c, int U, int G) {
+  return int(unsigned(c) * unsigned(U) / unsigned(G));
+}
+__host__ __device__ __forceinline__ int unit_owner(int u, int U, int G) {
+  return int((unsigned(u + 1) * unsigned(G) - 1u) / unsigned(U));
+}
+
+// Everything the kernel needs to know about one matrix; the host planner
+// fills it (the same for every M row count except the partial-slot size).
+struct alignas(16) GemvJobDesc {
+  const uint8_t* W;      // super-block-column-major weights
+  const uint16_t* x;     // bf16 [M][K]
+  void* y;               // fp32 or bf16 [M][N] ([M][N/2] for gate / up pairs)
+  long long part_off;    // this job's partial slots: floats into the partial area
+  int N;                 // weight rows
+  int nsb;               // K / 256
+  int flags;             // kJobOutBf16 | kJobSwiglu
+  int wait_for;          // -1: x is ready at launch; j: x is read after job j finished
+  int rbs;               // row blocks, ceil(N / 128)
+  int upr;               // units per row block, ceil(nsb / 2)
+  int units;             // rbs * upr
+  int grid;              // CTAs that work on this job (min(launch grid, units))
+  int slots;             // partial slots per row block (0: no row block is shared)
+  int cnt_off;           // this job's row-block counters: index into the counter area
+  int rot;               // job-local CTA index = (blockIdx.x + rot) mod launch grid
+  int pad_;
 };
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                            uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
-      : "memory");
+struct GemvArgs {
+  const GemvJobDesc* jobs;        // device array of n_jobs descriptors, or null: `job` below
+  unsigned* sync;                 // [n_jobs] jobs finished by all CTAs, [1] CTAs gone (zeroed)
+  unsigned long long* counters;   // workspace: row-block counters (tagged)
+  float* partials;                // workspace: partial slots
+  unsigned* err;                  // device error word
+  unsigned long long tag;         // this launch's counter tag (48 bits, non-zero)
+  int n_jobs;
+  int grid;                       // CTAs of the launch
+  int stages;                     // ring stages
+  int pad_;
+  GemvJobDesc job;                // the single job of a one-matrix launch
+};
+
+// Count one arrival on a tagged counter (tag in bits 16..63, count in 0..15;
+// a counter with another tag counts as zero).  Returns the count after it.
+__device__ __forceinline__ unsigned tagged_arrive(unsigned long long* w, unsigned long long tag) {
+  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(w);
+  for (;;) {
+    const unsigned long long nw = ((old >> 16) == tag) ? old + 1ull : ((tag << 16) | 1ull);
+    const unsigned long long prev = atomicCAS(w, old, nw);
+    if (prev == old) return unsigned(nw & 0xFFFFull);
+    old = prev;
+  }
 }
 
-__device__ __forceinline__ void tma_load_2d_nohint(uint32_t dst, const CUtensorMap* map, int x,
-                                                   int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
-constexpr uint32_t kSbBytes = 144;  // one super-block row piece in shared memory
-
-// Bytes of one pipeline stage holding KC super-block columns: KC weight
-// pieces (rows_per_pass x 144 bytes each, rounded up to 128) followed by KC
-// activation boxes (M x 512 bytes each).
-__host__ __device__ constexpr uint32_t gemv_wbox_bytes(int rows_per_pass) {
-  return (uint32_t(rows_per_pass) * kSbBytes + 127u) / 128u * 128u;
-}
-__host__ __device__ constexpr uint32_t gemv_stage_bytes(int M, int KC, int rows_per_pass) {
-  return uint32_t(KC) * (gemv_wbox_bytes(rows_per_pass) + uint32_t(M) * 512u);
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
-// Element i of the output: fp32, or bf16 (round to nearest even) when the
-// caller asked for bf16 outputs.  Partials of a K split are always fp32.
-__device__ __forceinline__ void store_out(float* out, size_t i, float v, int bf16) {
+// Make generic-proxy writes of other CTAs (observed through an acquire) visible
+// to this thread's subsequent bulk copies (async proxy) from global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Element i of an output: fp32, or bf16 (round to nearest even).
+__device__ __forceinline__ void store_out(void* out, size_t i, float v, bool bf16) {
   if (bf16)
     reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
   else
-    out[i] = v;
+    reinterpret_cast<float*>(out)[i] = v;
 }
 
-constexpr int kConsumerWarps = 8;
-constexpr int kGemvThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
-
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+__device__ __forceinline__ void gemv_consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kGemvConsumerWarps * 32) : "memory");
 }
 
-// One m16 tile x one 32-element block: dequantise rows g (and g+8 when
-// `second`), two MMAs against the block's x fragment, then add the tile's
-// fresh accumulator times each row's block scale into acc.  Columns >= M
-// of the accumulator stay zero and are not scaled.
-template <int M>
-__device__ __forceinline__ void gemv_tile(const uint8_t* pa, uint32_t woff, uint32_t doff,
-                                          bool second, const uint32_t (&bx)[4],
-                                          float (&acc)[4]) {
-  const uint32_t mask = 0x000F000Fu, magic = 0x43004300u, c136 = 0x43084308u;  // bf16 136
-  const uint8_t* pb = pa + 8u * kSbBytes;
-  const uint32_t wa = *reinterpret_cast<const uint32_t*>(pa + woff);
-  const uint32_t wb = second ? *reinterpret_cast<const uint32_t*>(pb + woff) : 0x88888888u;
-  const float da = half_bits_to_float(*reinterpret_cast<const uint16_t*>(pa + doff));
-  const float db = second ? half_bits_to_float(*reinterpret_cast<const uint16_t*>(pb + doff)) : 0.f;
-  uint32_t qa[4], qb[4];
-  dequant_pairs(wa, mask, magic, c136, qa);
-  dequant_pairs(wb, mask, magic, c136, qb);
-  float c[4] = {0.f, 0.f, 0.f, 0.f};
-  mma_bf16(c, qa[0], qb[0], qa[1], qb[1], bx[0], bx[1]);
-  mma_bf16(c, qa[2], qb[2], qa[3], qb[3], bx[2], bx[3]);
-  acc[0] = fmaf(da, c[0], acc[0]);
-  acc[2] = fmaf(db, c[2], acc[2]);
-  if constexpr (M > 1) {
-    acc[1] = fmaf(da, c[1], acc[1]);
-    acc[3] = fmaf(db, c[3], acc[3]);
+// Wait for the barrier phase with the given parity, for at most kWaitLimitNs,
+// unless the CTA has already given up (abort flag): then return false at
+// once.  A wait that runs out sets the abort flag and the device error word.
+__device__ __forceinline__ bool gemv_wait(uint32_t bar, uint32_t parity, unsigned* err,
+                                          volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  if (*abort_flag) return false;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t polls = 1;; ++polls) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((polls & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(err, kDevErrWaitTimeout);
+        return false;
+      }
+    }
   }
 }
 
-// Everything a consumer warp needs to run the stages of one pass.
-struct PassCtx {
-  const uint8_t* ring;
-  uint64_t* full;
-  uint64_t* empty;
-  unsigned* err;
-  uint32_t stage_bytes, wbox, xoff, woff, doff;
-  int S, n_chunks, warp, g, t, lane;
+__device__ __forceinline__ const GemvJobDesc* gemv_job(const GemvArgs& a, int i) {
+  return a.jobs ? a.jobs + i : &a.job;
+}
+
+// This CTA's place in job J: its job-local index (-1 when it has no unit of
+// the job) and its unit range [ub, ue).
+struct JobRange {
+  int cj, ub, ue;
+};
+__device__ __forceinline__ JobRange job_range(const GemvArgs& a, const GemvJobDesc* J) {
+  JobRange r;
+  int c = int(blockIdx.x) + J->rot;
+  if (c >= a.grid) c -= a.grid;
+  r.cj = c < J->grid ? c : -1;
+  r.ub = r.cj < 0 ? 0 : unit_begin(r.cj, J->units, J->grid);
+  r.ue = r.cj < 0 ? 0 : unit_begin(r.cj + 1, J->units, J->grid);
+  return r;
+}
+
+// The sequence of units a CTA works through, job after job (jobs it has no
+// units of are skipped), for the producer.  The row block rb and column pair
+// cp of unit u are kept up to date incrementally (no division per unit).
+struct UnitCursor {
+  int job, u, ue, rb, cp;
+  const uint8_t* W;
+  const uint16_t* x;
+  int N, nsb, upr, wait_for;
 };
 
-// One pass of T m-tiles (the last one using only rows 0..7 when HALF) over
-// all chunks of the K range: wait for each stage, run every tile of every
-// block fully unrolled (no per-tile guard, so the compiler interleaves the
-// tiles' loads, unpacking and MMAs), then release the stage.  Rows beyond the
-// pass's end hold stale shared memory; their results are never stored.
-template <int M, int KC, int T, bool HALF>
-__device__ __forceinline__ void gemv_pass(const PassCtx& c, int& slot, uint32_t& phase,
-                                          float (&acc)[kMmaMaxTiles][4]) {
-  #pragma unroll
-  for (int p = 0; p < T; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
-  for (int chunk = 0; chunk < c.n_chunks; ++chunk) {
-    mbar_wait(smem_addr(&c.full[slot]), phase, c.err);
-    const uint8_t* wst = c.ring + size_t(slot) * c.stage_bytes;
-    #pragma unroll 1
-    for (int j = 0; j < KC; ++j) {  // kept rolled: one copy of the tile code stays in the I-cache
-      // B fragment (x) of this warp's block of column j for column g
-      uint32_t bx[4] = {0u, 0u, 0u, 0u};
-      if (c.g < M) {
-        const uint8_t* xr = wst + c.xoff + (j * M + c.g) * 512 + (c.warp * 32 + 4 * c.t) * 2;
-        const uint2 lo = *reinterpret_cast<const uint2*>(xr);
-        const uint2 hi = *reinterpret_cast<const uint2*>(xr + 32);
-        bx[0] = prmt(lo.x, lo.y, 0x5410);  // (x[4t+0], x[4t+2])
-        bx[1] = prmt(hi.x, hi.y, 0x5410);  // (x[16+4t+0], x[16+4t+2])
-        bx[2] = prmt(lo.x, lo.y, 0x7632);  // (x[4t+1], x[4t+3])
-        bx[3] = prmt(hi.x, hi.y, 0x7632);  // (x[16+4t+1], x[16+4t+3])
-      }
-      const uint8_t* wj = wst + uint32_t(j) * c.wbox;
-      #pragma unroll
-      for (int p = 0; p < T; ++p)
-        gemv_tile<M>(wj + 16u * p * kSbBytes, c.woff, c.doff, !(HALF && p == T - 1), bx, acc[p]);
+__device__ __forceinline__ void cursor_enter(UnitCursor& c, const GemvArgs& a, int i) {
+  for (; i < a.n_jobs; ++i) {
+    const GemvJobDesc* J = gemv_job(a, i);
+    const JobRange r = job_range(a, J);
+    if (r.cj < 0) continue;
+    c.u = r.ub;
+    c.ue = r.ue;
+    c.rb = c.u / J->upr;
+    c.cp = c.u - c.rb * J->upr;
+    c.W = J->W;
+    c.x = J->x;
+    c.N = J->N;
+    c.nsb = J->nsb;
+    c.upr = J->upr;
+    c.wait_for = J->wait_for;
+    break;
+  }
+  c.job = i;
+}
+
+__device__ __forceinline__ void cursor_next(UnitCursor& c, const GemvArgs& a) {
+  if (++c.u == c.ue) {
+    cursor_enter(c, a, c.job + 1);
+  } else if (++c.cp == c.upr) {
+    c.cp = 0;
+    ++c.rb;
+  }
+}
+
+// The rows of a row block, fully summed, given as `v` (element i = m * 128 +
+// r; lane L holds elements L, L + 32, ...): write y (or, for gate / up pairs,
+// h = silu(g) * u, pairing rows 2j and 2j + 1 across lanes).
+template <int M>
+__device__ __forceinline__ void gemv_store_rows(const GemvJobDesc* J, int rb, int lane,
+                                                const float (&v)[4 * M]) {
+  const bool bf16 = (J->flags & kJobOutBf16) != 0;
+  const int r0 = rb * kGemvRows;
+  if (J->flags & kJobSwiglu) {
+    const int n_out = J->N >> 1;
+    #pragma unroll
+    for (int k = 0; k < 4 * M; ++k) {
+      const int i = lane + 32 * k, m = i >> 7, r = i & 127;
+      // rows 2j (even lane) and 2j + 1 (the next lane) of the same column
+      const float other = __shfl_down_sync(0xFFFFFFFFu, v[k], 1);
+      if ((r & 1) == 0 && r0 + r + 1 < J->N)
+        store_out(J->y, size_t(m) * n_out + ((r0 + r) >> 1), v[k] / (1.f + expf(-v[k])) * other,
+                  bf16);
     }
-    __syncwarp();
-    if (c.lane == 0) mbar_arrive(smem_addr(&c.empty[slot]));  // this warp is done with it
-    if (++slot == c.S) {
-      slot = 0;
-      phase ^= 1u;
+  } else {
+    #pragma unroll
+    for (int k = 0; k < 4 * M; ++k) {
+      const int i = lane + 32 * k, m = i >> 7, r = i & 127;
+      if (r0 + r < J->N) store_out(J->y, size_t(m) * J->N + r0 + r, v[k], bf16);
     }
   }
 }
 
-// M: activation rows (B fragment columns; columns M..7 are zero).
-// KC: super-block columns per pipeline stage.
-// Warps 0..7 consume: warp w takes block w of every super-block column and
-// every m-tile of the pass.  Warp 8 produces: it refills a stage as soon as
-// all eight consumers have released it.
-// SWIGLU: the matrix holds gate / up row pairs (rows 2n, 2n + 1); CTAs own
-// whole pairs and, without a K split, store h = silu(gate) * up per pair.
-template <int M, int KC, bool SWIGLU>
-__global__ void __launch_bounds__(kGemvThreads, 1)
-    q4_gemv_kernel(const __grid_constant__ GemvArgs a) {
+// End of a row block segment, consumer side: add the 16 warps' partial sums in
+// a fixed order (warp w + 8 into warp w, then the 8 slots in order) into the
+// segment buffer `fin` ([M][128]).
+template <int M>
+__device__ __forceinline__ void gemv_segment_reduce(float* red, float* fin,
+                                                    const float (&acc)[kGemvTiles][4], int warp,
+                                                    int lane, int tid) {
+  const int g = lane >> 2, t = lane & 3;
+  auto red_at = [&](int s, int p, int row, int m) -> float& {
+    return red[((s * kGemvTiles + p) * 16 + row) * M + m];
+  };
+  if (warp >= 8) {
+    #pragma unroll
+    for (int p = 0; p < kGemvTiles; ++p)
+      #pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (2 * t + e < M) {
+          red_at(warp - 8, p, g, 2 * t + e) = acc[p][e];
+          red_at(warp - 8, p, g + 8, 2 * t + e) = acc[p][2 + e];
+        }
+  }
+  gemv_consumer_sync();
+  if (warp < 8) {
+    #pragma unroll
+    for (int p = 0; p < kGemvTiles; ++p)
+      #pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (2 * t + e < M) {
+          red_at(warp, p, g, 2 * t + e) = acc[p][e] + red_at(warp, p, g, 2 * t + e);
+          red_at(warp, p, g + 8, 2 * t + e) = acc[p][2 + e] + red_at(warp, p, g + 8, 2 * t + e);
+        }
+  }
+  gemv_consumer_sync();
+  for (int i = tid; i < kGemvRows * M; i += kGemvConsumerWarps * 32) {
+    const int m = i / kGemvRows, r = i - m * kGemvRows;
+    float s = 0.f;
+    #pragma unroll
+    for (int w = 0; w < 8; ++w) s += red_at(w, r >> 4, r & 15, m);
+    fin[i] = s;
+  }
+  gemv_consumer_sync();
+}
+
+// End of a row block segment, epilogue side (one warp): write the row block
+// (covered by this CTA alone), or this CTA's partial slot and, if it is the
+// last contributor to arrive, the sum of all slots in slot order.  The
+// segment buffer is released as soon as it has been read.
+template <int M>
+__device__ __forceinline__ void gemv_segment_write(const GemvArgs& a, const GemvJobDesc* J, int cj,
+                                                   int rb, const float* fin, uint64_t* fin_empty,
+                                                   int lane) {
+  const int G = J->grid, first_u = rb * J->upr;
+  const int c_first = unit_owner(first_u, J->units, G);
+  const int c_last = unit_owner(first_u + J->upr - 1, J->units, G);
+  const int n_contrib = c_last - c_first + 1;
+  float v[4 * M];
+  #pragma unroll
+  for (int k = 0; k < 4 * M; ++k) v[k] = fin[lane + 32 * k];
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_addr(fin_empty));  // the segment buffer is free again
+  if (n_contrib == 1) {
+    gemv_store_rows<M>(J, rb, lane, v);
+    return;
+  }
+  // this CTA's partial sums into its slot ([M][128] floats; rows past N unused)
+  float* part = a.partials + J->part_off + size_t(rb) * J->slots * M * kGemvRows;
+  float* mine = part + size_t(cj - c_first) * M * kGemvRows;
+  #pragma unroll
+  for (int k = 0; k < 4 * M; ++k) mine[lane + 32 * k] = v[k];
+  __syncwarp();
+  int last = 0;
+  if (lane == 0) {
+    fence_acq_rel_gpu();  // this slot's writes (all lanes, ordered by the warp barrier) first
+    unsigned long long* cnt = a.counters + J->cnt_off + rb;
+    last = tagged_arrive(cnt, a.tag) == unsigned(n_contrib);
+    if (last) {
+      *cnt = 0ull;  // every contributor has counted itself in: ready for a replay
+      fence_acq_rel_gpu();  // the other slots' writes become visible to this warp
+    }
+  }
+  last = __shfl_sync(0xFFFFFFFFu, last, 0);
+  if (!last) return;
+  // the last contributor: every slot's values first (all loads in flight),
+  // added in slot order, then the stores
+  #pragma unroll
+  for (int k = 0; k < 4 * M; ++k) v[k] = 0.f;
+  for (int sl = 0; sl < n_contrib; ++sl) {
+    float w[4 * M];
+    #pragma unroll
+    for (int k = 0; k < 4 * M; ++k) w[k] = __ldcg(part + size_t(sl) * M * kGemvRows + lane + 32 * k);
+    #pragma unroll
+    for (int k = 0; k < 4 * M; ++k) v[k] += w[k];
+  }
+  gemv_store_rows<M>(J, rb, lane, v);
+}
+
+template <int M>
+__global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_constant__ GemvArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int ks = blockIdx.y;
   const int S = a.stages;
-
-  const int unit = SWIGLU ? 2 : 1;  // rows per partition unit
-  const int units = a.N / unit;
-  const int row_begin = unit * int((long long)units * blockIdx.x / a.grid_rows);
-  const int row_end = unit * int((long long)units * (blockIdx.x + 1) / a.grid_rows);
-  const int n_rows = row_end - row_begin;
-  const int R = a.rows_per_pass;
-  const int n_passes = (n_rows + R - 1) / R;
-  const int n_chunks = a.sb_per_split / KC;
-  const int n_stages = n_passes * n_chunks;
-  const int sb_split0 = ks * a.sb_per_split;
-  const uint32_t wbox = gemv_wbox_bytes(R);
-  const uint32_t stage_bytes = gemv_stage_bytes(M, KC, R);
-  const uint32_t xoff = uint32_t(KC) * wbox;
-
+  constexpr uint32_t kStage = gemv_stage_bytes(M);
+  constexpr uint32_t kXOff = kGemvCols * kGemvWBox;
   uint8_t* ring = smem;
-  float4* red = reinterpret_cast<float4*>(smem + size_t(S) * stage_bytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(red + kConsumerWarps * kMmaMaxTiles * 32);
+  float* red = reinterpret_cast<float*>(smem + size_t(S) * kStage);
+  float* fin = red + gemv_red_bytes(M) / 4;                       // [4][M][128]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(fin + kGemvSegBufs * M * kGemvRows);
+  volatile int* epi_done = abort_flag + 1;                        // [2] segments written per epilogue warp
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(S) * kStage + gemv_red_bytes(M) +
+                                               gemv_fin_bytes(M) + 16);
   uint64_t* empty = full + S;
+  uint64_t* fin_full = empty + S;                 // [4] segment buffer written by the consumers
+  uint64_t* fin_empty = fin_full + kGemvSegBufs;  // [4] segment buffer released by the epilogue
 
   if (tid == 0) {
-    // the next kernel on the stream may start its own weight prefetch
-    griddep_launch_dependents();
+    griddep_launch_dependents();  // the next kernel on the stream may start its prologue
     for (int s = 0; s < S; ++s) {
       mbar_init(smem_addr(&full[s]), 1);
-      mbar_init(smem_addr(&empty[s]), kConsumerWarps);
+      mbar_init(smem_addr(&empty[s]), kGemvConsumerWarps);
     }
+    for (int b = 0; b < kGemvSegBufs; ++b) {
+      mbar_init(smem_addr(&fin_full[b]), 1);
+      mbar_init(smem_addr(&fin_empty[b]), 1);
+    }
+    *abort_flag = 0;
+    epi_done[0] = 0;
+    epi_done[1] = 0;
     mbar_init_fence();
   }
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
-    // ---------------- producer: one lane issues every copy ----------------
-    if (lane == 0) {
-      const uint64_t pol = l2_evict_first_policy();
-      // First ring fill: the weights (no earlier kernel writes them) go out
-      // before waiting on the previous kernel; the activations, which it may
-      // produce, only after.  Under a plain launch the wait returns at once.
-      const int pre = min(S, n_stages);
-      for (int st = 0; st < pre; ++st) {
-        const int ps = st / n_chunks, ch = st - ps * n_chunks;
-        const int r0 = row_begin + ps * R;
-        const int nr = min(R, row_end - r0);
-        const int sb = sb_split0 + ch * KC;
-        const uint32_t bar = smem_addr(&full[st]);
-        const uint32_t dst = smem_addr(ring + size_t(st) * stage_bytes);
-        mbar_arrive_expect_tx(bar, uint32_t(KC) * (uint32_t(nr) * kSbBytes + uint32_t(M) * 512u));
-        #pragma unroll
-        for (int j = 0; j < KC; ++j)
-          bulk_g2s(dst + uint32_t(j) * wbox, a.W + (size_t(sb + j) * a.N + r0) * kSbBytes,
-                   uint32_t(nr) * kSbBytes, bar, pol);
+  if (warp == kGemvProducerWarp) {
+    // ------------------------------ producer ------------------------------
+    if (lane != 0) return;
+    const uint64_t pol = l2_evict_first_policy();
+    UnitCursor w, xs;   // next unit whose weights / whose activations to issue
+    cursor_enter(w, a, 0);
+    xs = w;
+    int stw = 0, stx = 0, x_job_ready = -1;
+    int w_slot = 0, x_slot = 0;
+    uint32_t w_par = 0;  // parity of the ring pass of stage stw
+    bool prior_grid_done = false;
+    // Is the input of the job of the oldest stage without activations ready?
+    auto x_ready = [&]() {
+      if (x_job_ready == xs.job) return true;
+      bool ready;
+      if (xs.wait_for < 0) {
+        if (!prior_grid_done) {
+          griddep_wait();  // the kernel before this one has finished, its writes visible
+          prior_grid_done = true;
+        }
+        ready = true;
+      } else {
+        ready = ld_acquire_gpu(a.sync + xs.wait_for) >= unsigned(a.grid);
       }
-      griddep_wait();
-      for (int st = 0; st < pre; ++st) {
-        const int sb = sb_split0 + (st % n_chunks) * KC;
-        const uint32_t bar = smem_addr(&full[st]);
-        const uint32_t dst = smem_addr(ring + size_t(st) * stage_bytes);
-        #pragma unroll
-        for (int j = 0; j < KC; ++j)
-          tma_load_2d_nohint(dst + xoff + uint32_t(j) * uint32_t(M) * 512u, &a.xmap,
-                             (sb + j) * 256, 0, bar);
+      if (ready) {
+        fence_proxy_async_global();
+        x_job_ready = xs.job;
       }
-      int slot = 0, pass = pre / n_chunks, chunk = pre % n_chunks;
-      uint32_t phase = pre == S ? 1u : 0u;
-      for (int st = pre; st < n_stages; ++st) {
-        mbar_wait(smem_addr(&empty[slot]), phase ^ 1u, a.err);
-        const int r0 = row_begin + pass * R;
-        const int nr = min(R, row_end - r0);
-        const uint32_t bar = smem_addr(&full[slot]);
-        const uint32_t dst = smem_addr(ring + size_t(slot) * stage_bytes);
-        const int sb = sb_split0 + chunk * KC;
-        mbar_arrive_expect_tx(bar, uint32_t(KC) * (uint32_t(nr) * kSbBytes + uint32_t(M) * 512u));
-        #pragma unroll
-        for (int j = 0; j < KC; ++j) {
-          // rows r0 .. r0+nr of column sb+j are contiguous in the weight layout
-          bulk_g2s(dst + uint32_t(j) * wbox, a.W + (size_t(sb + j) * a.N + r0) * kSbBytes,
-                   uint32_t(nr) * kSbBytes, bar, pol);
-          tma_load_2d_nohint(dst + xoff + uint32_t(j) * uint32_t(M) * 512u, &a.xmap,
-                             (sb + j) * 256, 0, bar);
+      return ready;
+    };
+    auto issue_x = [&]() {
+      const uint32_t bar = smem_addr(&full[x_slot]);
+      const uint32_t dst = smem_addr(ring + size_t(x_slot) * kStage) + kXOff;
+      const int col0 = 2 * xs.cp;
+      const int kc = min(kGemvCols, xs.nsb - col0);
+      #pragma unroll
+      for (int m = 0; m < M; ++m)
+        bulk_g2s_nohint(dst + uint32_t(m) * (kGemvCols * 512u),
+                        xs.x + (size_t(m) * xs.nsb + col0) * 256, uint32_t(kc) * 512u, bar);
+      ++stx;
+      if (++x_slot == S) x_slot = 0;
+      cursor_next(xs, a);
+    };
+    unsigned long long dep_since = 0;
+    while (xs.job < a.n_jobs && !*abort_flag) {
+      // activations of every armed stage whose job's input is ready
+      while (stx < stw && x_ready()) issue_x();
+      if (w.job < a.n_jobs &&
+          (stw < S || mbar_test_wait(smem_addr(&empty[w_slot]), w_par ^ 1u))) {
+        // weights of the next unit: its ring slot is free
+        const int col0 = 2 * w.cp;
+        const int kc = min(kGemvCols, w.nsb - col0);
+        const int rows = min(kGemvRows, w.N - w.rb * kGemvRows);
+        const uint32_t bar = smem_addr(&full[w_slot]);
+        const uint32_t dst = smem_addr(ring + size_t(w_slot) * kStage);
+        mbar_arrive_expect_tx(bar, uint32_t(kc) * (uint32_t(rows) * kSbBytes + uint32_t(M) * 512u));
+        for (int j = 0; j < kc; ++j)
+          bulk_g2s(dst + uint32_t(j) * kGemvWBox,
+                   w.W + (size_t(col0 + j) * w.N + size_t(w.rb) * kGemvRows) * kSbBytes,
+                   uint32_t(rows) * kSbBytes, bar, pol);
+        ++stw;
+        if (++w_slot == S) {
+          w_slot = 0;
+          w_par ^= 1u;
         }
-        if (++slot == S) {
-          slot = 0;
-          phase ^= 1u;
+        cursor_next(w, a);
+        dep_since = 0;
+        continue;
+      }
+      if (stx < stw) {
+        // an armed stage waits for its job's input (another job of the launch)
+        const unsigned long long now = global_timer_ns();
+        if (dep_since == 0) {
+          dep_since = now;
+        } else if (now - dep_since > kWaitLimitNs) {
+          *abort_flag = 1;
+          atomicOr(a.err, kDevErrWaitTimeout);
         }
-        if (++chunk == n_chunks) {
-          chunk = 0;
-          ++pass;
-        }
+        __nanosleep(200);
+      } else if (w.job < a.n_jobs) {
+        // ring full, every armed stage complete: sleep until a slot is free
+        gemv_wait(smem_addr(&empty[w_slot]), w_par ^ 1u, a.err, abort_flag);
+      }
+    }
+    // After an abort: complete every armed stage with its activation copies
+    // (valid memory, stale values: the results are void anyway), so that each
+    // armed barrier phase can complete.
+    for (; stx < stw; ++stx) {
+      const uint32_t bar = smem_addr(&full[x_slot]);
+      const uint32_t dst = smem_addr(ring + size_t(x_slot) * kStage) + kXOff;
+      const int col0 = 2 * xs.cp;
+      const int kc = min(kGemvCols, xs.nsb - col0);
+      for (int m = 0; m < M; ++m)
+        bulk_g2s_nohint(dst + uint32_t(m) * (kGemvCols * 512u),
+                        xs.x + (size_t(m) * xs.nsb + col0) * 256, uint32_t(kc) * 512u, bar);
+      if (++x_slot == S) x_slot = 0;
+      cursor_next(xs, a);
+    }
+    // Wait for the copies still in flight (bounded), so that none lands after
+    // the CTA has exited: the last stage issued into each slot.
+    for (int k = 0; k < S && k < stw; ++k) {
+      const int st = stw - 1 - k;
+      const uint32_t bar = smem_addr(&full[st % S]);
+      const unsigned long long t0 = global_timer_ns();
+      while (!mbar_try_wait(bar, uint32_t(st / S) & 1u) && global_timer_ns() - t0 < kWaitLimitNs) {
       }
     }
     return;
   }
 
-  // ---------------- consumers ----------------
-  PassCtx c;
-  c.ring = ring;
-  c.full = full;
-  c.empty = empty;
-  c.err = a.err;
-  c.stage_bytes = stage_bytes;
-  c.wbox = wbox;
-  c.xoff = xoff;
-  c.warp = warp;
-  c.lane = lane;
-  c.g = lane >> 2;
-  c.t = lane & 3;
-  c.woff = uint32_t(c.g) * kSbBytes + uint32_t(warp) * 16u + uint32_t(c.t) * 4u;
-  c.doff = uint32_t(c.g) * kSbBytes + 128u + uint32_t(warp) * 2u;
-  c.S = S;
-  c.n_chunks = n_chunks;
-  float acc[kMmaMaxTiles][4];
-  int slot = 0;
-  uint32_t phase = 0;
-
-  for (int pass = 0; pass < n_passes; ++pass) {
-    const int nr = min(R, n_rows - pass * R);
-    const int T = (nr + 15) >> 4;
-    const bool half = (nr & 15) != 0 && (nr & 15) <= 8;
-    switch (T * 2 + (half ? 1 : 0)) {
-#define Q4D_PASS(TT)                                                   \
-  case 2 * TT: gemv_pass<M, KC, TT, false>(c, slot, phase, acc); break; \
-  case 2 * TT + 1: gemv_pass<M, KC, TT, true>(c, slot, phase, acc); break;
-      Q4D_PASS(1) Q4D_PASS(2) Q4D_PASS(3) Q4D_PASS(4)
-      Q4D_PASS(5) Q4D_PASS(6) Q4D_PASS(7) Q4D_PASS(8)
-#undef Q4D_PASS
-      default: break;
-    }
-
-    // Cross-warp sum of the pass, in a fixed order.
-    #pragma unroll
-    for (int p = 0; p < kMmaMaxTiles; ++p)
-      if (16 * p < nr)
-        red[(warp * kMmaMaxTiles + p) * 32 + lane] =
-            make_float4(acc[p][0], acc[p][1], acc[p][2], acc[p][3]);
-    consumer_sync();
-    // out[m][row] = sum over the 8 warps; element (row r, column m) sits in
-    // lane (r % 8) * 4 + m / 2 of tile r / 16, component (r >= 8 ? 2 : 0) + m % 2
-    const int r0 = row_begin + pass * R;
-    auto row_sum = [&](int r, int m) {
-      const int p = r >> 4, rr = r & 15;
-      const int ln = (rr & 7) * 4 + (m >> 1);
-      const int comp = (rr >= 8 ? 2 : 0) + (m & 1);
-      float s = 0.f;
-      #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float4 v = red[(w * kMmaMaxTiles + p) * 32 + ln];
-        s += comp == 0 ? v.x : comp == 1 ? v.y : comp == 2 ? v.z : v.w;
+  if (warp > kGemvProducerWarp) {
+    // ------------------------------ epilogue ------------------------------
+    // Warp e writes segments e, e + 2, ...; the warp writing a job's last
+    // segment in this CTA waits until the other warp has written the job's
+    // earlier ones, then counts the CTA in for the job.  Nothing of the
+    // workspace or the outputs is touched before the previous kernel on the
+    // stream is complete (it may still use the same buffers).
+    griddep_wait();
+    const int e = warp - kGemvProducerWarp - 1, o = 1 - e;
+    // other warp's segments among [0, s): o, o + 2, ...
+    auto other_written = [&](int s_end) {
+      const int need = (s_end + 1 - o) / 2;
+      const unsigned long long t0 = global_timer_ns();
+      while (epi_done[o] < need && !*abort_flag) {
+        __nanosleep(64);
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          atomicOr(a.err, kDevErrWaitTimeout);
+        }
       }
-      return s;
     };
-    if (SWIGLU && gridDim.y == 1) {
-      // h[m][n] = silu(g) * u for the pairs of this pass (passes hold whole pairs)
-      for (int i = tid; i < (nr >> 1) * M; i += kConsumerWarps * 32) {
-        const int j = i / M, m = i - (i / M) * M;
-        const float g = row_sum(2 * j, m), u = row_sum(2 * j + 1, m);
-        store_out(a.out, size_t(m) * (a.N >> 1) + ((r0 >> 1) + j), g / (1.f + __expf(-g)) * u,
-                  a.out_bf16);
+    int seg = 0, mine = 0;
+    for (int job = 0; job < a.n_jobs; ++job) {
+      const GemvJobDesc* J = gemv_job(a, job);
+      const JobRange r = job_range(a, J);
+      int last_seg_writer = 0;  // jobs without units here: warp 0 counts the CTA in
+      for (int u = r.ub; u < r.ue;) {
+        const int rb = u / J->upr;
+        const int u_end = min(r.ue, (rb + 1) * J->upr);
+        if ((seg & 1) == e) {
+          const int b = seg & (kGemvSegBufs - 1);
+          gemv_wait(smem_addr(&fin_full[b]), uint32_t(seg >> 2) & 1u, a.err, abort_flag);
+          gemv_segment_write<M>(a, J, r.cj, rb, fin + b * M * kGemvRows, &fin_empty[b], lane);
+          __syncwarp();
+          if (lane == 0) {
+            fence_acq_rel_gpu();  // this warp's writes before its progress count
+            epi_done[e] = ++mine;
+          }
+          __syncwarp();
+        }
+        last_seg_writer = seg & 1;
+        ++seg;
+        u = u_end;
       }
-    } else {
-      for (int i = tid; i < nr * M; i += kConsumerWarps * 32) {
-        const int r = i / M, m = i - (i / M) * M;
-        store_out(a.out, (size_t(ks) * M + m) * a.N + r0 + r, row_sum(r, m), a.out_bf16);
+      if (a.n_jobs > 1 && last_seg_writer == e) {
+        if (lane == 0) {
+          other_written(seg);
+          fence_acq_rel_gpu();
+          atomicAdd(a.sync + job, 1u);
+        }
+        __syncwarp();
       }
     }
-    consumer_sync();  // red is rewritten at the next pass end
-  }
-}
-
-// h[m][n] = silu(g) * u from the partials of the 2N gate / up rows, each
-// summed over the K ranges in range order.
-__global__ void q4_gemv_splitk_reduce_swiglu(const float* __restrict__ ws, float* __restrict__ h,
-                                             int M, int N, int k_splits, int out_bf16) {
-  if (threadIdx.x == 0) griddep_launch_dependents();
-  const long long mn = (long long)M * N, rows = 2LL * N;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < mn;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long m = i / N, n = i - m * N;
-    float g = 0.f, u = 0.f;
-    for (int k = 0; k < k_splits; ++k) {
-      g += ws[(k * M + m) * rows + 2 * n];
-      u += ws[(k * M + m) * rows + 2 * n + 1];
+    if (a.n_jobs > 1 && e == 0 && lane == 0) {
+      // the last CTA to leave sets the per-job counters back to zero
+      other_written(seg);
+      if (atomicAdd(a.sync + a.n_jobs, 1u) == unsigned(a.grid - 1)) {
+        fence_acq_rel_gpu();
+        for (int i = 0; i <= a.n_jobs; ++i) a.sync[i] = 0u;
+      }
     }
-    store_out(h, size_t(i), g / (1.f + __expf(-g)) * u, out_bf16);
+    return;
   }
-}
 
-// y[i] = sum over K ranges of the partials, in range order.
-__global__ void q4_gemv_splitk_reduce(const float* __restrict__ ws, float* __restrict__ y,
-                                      long long mn, int k_splits, int out_bf16) {
-  if (threadIdx.x == 0) griddep_launch_dependents();
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < mn;
-       i += (long long)gridDim.x * blockDim.x) {
-    float s = 0.f;
-    for (int k = 0; k < k_splits; ++k) s += ws[k * mn + i];
-    store_out(y, size_t(i), s, out_bf16);
+  // ------------------------------ consumers ------------------------------
+  const int g = lane >> 2, t = lane & 3;
+  const int task_col = warp >> 3, task_blk = warp & 7;
+  const uint32_t mask = 0x000F000Fu, magic = 0x43004300u, c136 = 0x43084308u;  // bf16 136
+  const uint32_t x_lane = kXOff + g * (kGemvCols * 512) + task_col * 512 + (task_blk * 32 + 4 * t) * 2;
+  const uint32_t w_lane = task_col * kGemvWBox + g * kSbBytes + task_blk * 16 + t * 4;
+  const uint32_t d_lane = task_col * kGemvWBox + g * kSbBytes + 128 + task_blk * 2;
+  int slot = 0, seg = 0;
+  uint32_t phase = 0;
+  for (int job = 0; job < a.n_jobs; ++job) {
+    const GemvJobDesc* J = gemv_job(a, job);
+    const JobRange r = job_range(a, J);
+    const int upr = J->upr, nsb = J->nsb;
+    for (int u = r.ub; u < r.ue;) {
+      const int rb = u / upr;
+      const int cp0 = u - rb * upr;
+      const int n_units = min(r.ue, (rb + 1) * upr) - u;
+      float acc[kGemvTiles][4];
+      #pragma unroll
+      for (int p = 0; p < kGemvTiles; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
+      #pragma unroll 1
+      for (int k = 0; k < n_units; ++k) {
+        gemv_wait(smem_addr(&full[slot]), phase, a.err, abort_flag);
+        const uint8_t* stage = ring + size_t(slot) * kStage;
+        if (task_col < nsb - 2 * (cp0 + k)) {
+          // B fragment (x) of this warp's block of its column, for column g
+          uint32_t bx[4] = {0u, 0u, 0u, 0u};
+          if (g < M) {
+            const uint2 lo = *reinterpret_cast<const uint2*>(stage + x_lane);
+            const uint2 hi = *reinterpret_cast<const uint2*>(stage + x_lane + 32);
+            bx[0] = prmt(lo.x, lo.y, 0x5410);  // (x[4t+0], x[4t+2])
+            bx[1] = prmt(hi.x, hi.y, 0x5410);  // (x[16+4t+0], x[16+4t+2])
+            bx[2] = prmt(lo.x, lo.y, 0x7632);  // (x[4t+1], x[4t+3])
+            bx[3] = prmt(hi.x, hi.y, 0x7632);  // (x[16+4t+1], x[16+4t+3])
+          }
+          // rows beyond the matrix's last row hold stale data; their sums are never stored
+          #pragma unroll
+          for (int p = 0; p < kGemvTiles; ++p) {
+            const uint8_t* pa = stage + w_lane + 16 * p * kSbBytes;
+            const uint8_t* pd = stage + d_lane + 16 * p * kSbBytes;
+            const uint32_t wa = *reinterpret_cast<const uint32_t*>(pa);
+            const uint32_t wb = *reinterpret_cast<const uint32_t*>(pa + 8 * kSbBytes);
+            const float da = half_bits_to_float(*reinterpret_cast<const uint16_t*>(pd));
+            const float db = half_bits_to_float(*reinterpret_cast<const uint16_t*>(pd + 8 * kSbBytes));
+            uint32_t qa[4], qb[4];
+            dequant_pairs(wa, mask, magic, c136, qa);
+            dequant_pairs(wb, mask, magic, c136, qb);
+            float cc[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_bf16(cc, qa[0], qb[0], qa[1], qb[1], bx[0], bx[1]);
+            mma_bf16(cc, qa[2], qb[2], qa[3], qb[3], bx[2], bx[3]);
+            acc[p][0] = fmaf(da, cc[0], acc[p][0]);
+            acc[p][2] = fmaf(db, cc[2], acc[p][2]);
+            if constexpr (M > 1) {
+              acc[p][1] = fmaf(da, cc[1], acc[p][1]);
+              acc[p][3] = fmaf(db, cc[3], acc[p][3]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&empty[slot]));
+        if (++slot == S) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+      // hand the row block's sums to the epilogue (buffer seg % 4 must have
+      // been released: segment seg - 4)
+      const int b = seg & (kGemvSegBufs - 1);
+      if (seg >= kGemvSegBufs)
+        gemv_wait(smem_addr(&fin_empty[b]), uint32_t((seg - kGemvSegBufs) >> 2) & 1u, a.err,
+                  abort_flag);
+      gemv_segment_reduce<M>(red, fin + b * M * kGemvRows, acc, warp, lane, tid);
+      if (tid == 0) mbar_arrive(smem_addr(&fin_full[b]));
+      ++seg;
+      u += n_units;
+    }
   }
 }
 

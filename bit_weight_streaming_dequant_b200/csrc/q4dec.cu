@@ -2,8 +2,6 @@
 // and kernel dispatch.  Declarations and the contract live in include/q4dec.h.
 #include "q4dec.h"
 
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -11,7 +9,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <unordered_map>
 
 #include "q4_gemv.cuh"
@@ -26,12 +26,6 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kPlanFallbackSms = 148;
-// Shared memory per GEMV CTA: at most half an SM's (228 KB, 1 KB reserved per
-// block), so that with the weight prefetch (programmatic dependent launch) the
-// next GEMV's CTA fits next to the running one and streams its first stages
-// during the running one's tail: 5.34 -> 5.21 ms per decode step measured,
-// against the whole SM for one CTA (more ring stages, no overlap).
-constexpr size_t kGemvSmemBudget = 113 * 1024;
 constexpr size_t kAttnSmemBudget = 224 * 1024;   // shared memory per attention CTA
 // The 8-bit cache's 70 KB ring stages need the device's whole opt-in shared
 // memory per block (227 KB on B200) for two stages next to the V tile.
@@ -42,8 +36,10 @@ struct DeviceState {
   int num_sms = 0;
   int smem_optin = 0;
   unsigned* err = nullptr;
-  void* ws = nullptr;  // library-owned workspace of the plain entry points
+  void* ws = nullptr;  // library-owned workspace of the plain attention entry point
   size_t ws_bytes = 0;
+  void* gemv_ws = nullptr;  // library-owned workspace of the plain GEMV entry point
+  size_t gemv_ws_bytes = 0;
 };
 
 std::mutex g_mu;
@@ -88,23 +84,23 @@ q4d_status allow_smem(Kernel kernel, int dev, const DeviceState& s, std::atomic<
   return Q4D_OK;
 }
 
-q4d_status library_workspace(DeviceState& s, size_t need, void** ws) {
+q4d_status library_workspace(void*& buf, size_t& bytes, size_t need, void** ws) {
   if (need == 0) {
     *ws = nullptr;
     return Q4D_OK;
   }
   std::lock_guard<std::mutex> lk(g_mu);
-  if (s.ws_bytes < need) {
-    if (s.ws) cudaFree(s.ws);
-    s.ws = nullptr;
-    s.ws_bytes = 0;
-    if (cudaMalloc(&s.ws, need) != cudaSuccess) {
+  if (bytes < need) {
+    if (buf) cudaFree(buf);
+    buf = nullptr;
+    bytes = 0;
+    if (cudaMalloc(&buf, need) != cudaSuccess) {
       cudaGetLastError();
       return Q4D_ERR_CUDA;
     }
-    s.ws_bytes = need;
+    bytes = need;
   }
-  *ws = s.ws;
+  *ws = buf;
   return Q4D_OK;
 }
 
@@ -112,67 +108,6 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 int ceil_div(long long a, long long b) { return int((a + b - 1) / b); }
 long long round_up(long long a, long long b) { return (a + b - 1) / b * b; }
-
-// ---------------------------------------------------------------------------
-// TMA tensor maps, encoded on the host through the driver entry point (no
-// link-time dependency on libcuda) and cached by (address, shape, box).
-struct MapKey {
-  const void* ptr;
-  uint64_t d0, d1, stride;
-  uint32_t b0, b1;
-  int dtype;
-  bool operator==(const MapKey& o) const {
-    return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && stride == o.stride && b0 == o.b0 &&
-           b1 == o.b1 && dtype == o.dtype;
-  }
-};
-struct MapKeyHash {
-  size_t operator()(const MapKey& k) const {
-    uint64_t h = reinterpret_cast<uintptr_t>(k.ptr);
-    for (uint64_t v : {k.d0, k.d1, k.stride, uint64_t(k.b0) << 32 | k.b1, uint64_t(k.dtype)})
-      h = (h ^ v) * 0x100000001B3ull;
-    return size_t(h);
-  }
-};
-std::mutex g_map_mu;
-std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-
-q4d_status tensor_map_2d(CUtensorMap* out, CUtensorMapDataType dtype, const void* ptr, uint64_t d0,
-                         uint64_t d1, uint64_t stride_bytes, uint32_t b0, uint32_t b1) {
-  const MapKey key{ptr, d0, d1, stride_bytes, b0, b1, int(dtype)};
-  std::lock_guard<std::mutex> lk(g_map_mu);
-  auto it = g_maps.find(key);
-  if (it != g_maps.end()) {
-    *out = it->second;
-    return Q4D_OK;
-  }
-  if (!g_encode) {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !fn) {
-      cudaGetLastError();
-      return Q4D_ERR_CUDA;
-    }
-    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  }
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {d0, d1};
-  const cuuint64_t strides[1] = {stride_bytes};
-  const cuuint32_t box[2] = {b0, b1};
-  const cuuint32_t estr[2] = {1, 1};
-  if (g_encode(&map, dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-      CUDA_SUCCESS)
-    return Q4D_ERR_CUDA;
-  if (g_maps.size() > 8192) g_maps.clear();
-  g_maps.emplace(key, map);
-  *out = map;
-  return Q4D_OK;
-}
 
 q4d_status check_gemv_shape(int M, int N, int K) {
   if (N < 1 || K < 0) return Q4D_ERR_INVALID_ARG;
@@ -189,87 +124,139 @@ q4d_status check_attn_shape(int ctx_len, int n_q, int n_kv, int head_dim, int M,
   return Q4D_OK;
 }
 
-// Plan for `rows` weight rows shared out in units of `unit` rows (2 for the
-// gate / up pairs of the SwiGLU variant).
-q4d_status plan_gemv_rows(int M, int rows, int K, int num_sms, int unit, q4d_gemv_plan* plan) {
+// ---------------------------------------------------------------------------
+// GEMV planning (stream-K over row blocks of 128 rows and units of two
+// super-block columns; see q4_gemv.cuh).
+
+// Shape of one job's partition over G CTAs.
+struct JobShape {
+  int rbs, upr, units, grid, slots;
+};
+
+// Most CTAs that share one row block (0 when every row block has one CTA).
+int max_contributors(int rbs, int upr, int units, int G) {
+  int slots = 0;
+  for (int rb = 0; rb < rbs; ++rb) {
+    const int first = q4d::unit_owner(rb * upr, units, G);
+    const int last = q4d::unit_owner(rb * upr + upr - 1, units, G);
+    if (last > first) slots = std::max(slots, last - first + 1);
+  }
+  return slots;
+}
+
+std::mutex g_shape_mu;
+std::map<std::tuple<int, int, int>, int> g_slots_cache;
+
+// Row blocks x units per row block must stay below 2^31 / grid (the kernel's
+// 32-bit partition arithmetic); true for any matrix below ~500 GB.
+bool shape_fits(int rows, int nsb, int launch_grid) {
+  const long long units = (long long)ceil_div(rows, q4d::kGemvRows) * ceil_div(nsb, q4d::kGemvCols);
+  return units * (long long)launch_grid < (1ll << 31);
+}
+
+JobShape job_shape(int rows, int nsb, int launch_grid) {
+  JobShape j;
+  j.rbs = ceil_div(rows, q4d::kGemvRows);
+  j.upr = ceil_div(nsb, q4d::kGemvCols);
+  j.units = j.rbs * j.upr;
+  j.grid = std::min(launch_grid, j.units);
+  const auto key = std::make_tuple(rows, nsb, j.grid);
+  {
+    std::lock_guard<std::mutex> lk(g_shape_mu);
+    auto it = g_slots_cache.find(key);
+    if (it != g_slots_cache.end()) {
+      j.slots = it->second;
+      return j;
+    }
+  }
+  j.slots = max_contributors(j.rbs, j.upr, j.units, j.grid);
+  std::lock_guard<std::mutex> lk(g_shape_mu);
+  if (g_slots_cache.size() > 4096) g_slots_cache.clear();
+  g_slots_cache.emplace(key, j.slots);
+  return j;
+}
+
+// Ring stages that fit next to the reduction and segment buffers in
+// `smem_limit` bytes (at most kGemvMaxStages).
+int gemv_stages(int M, size_t smem_limit) {
+  int stages = 0;
+  while (stages < q4d::kGemvMaxStages && q4d::gemv_smem_bytes(M, stages + 1) <= smem_limit)
+    ++stages;
+  return stages;
+}
+
+constexpr size_t kGemvCounterBytes = 8;   // one tagged counter
+constexpr int kSmemOptinB200 = 232448;    // planning default: B200's opt-in shared memory
+
+size_t round_up16(size_t v) { return (v + 15) / 16 * 16; }
+
+q4d_status plan_gemv_rows(int M, int rows, int K, int num_sms, int smem_optin,
+                          q4d_gemv_plan* plan) {
   if (!plan || num_sms < 1) return Q4D_ERR_INVALID_ARG;
   q4d_status st = check_gemv_shape(M, rows, K);
   if (st != Q4D_OK) return st;
-  const int N = rows, units = rows / unit;
-  const int nsb = K / 256;
-  // Rows are shared out exactly (+-1) over up to one CTA per SM, at least 8
-  // rows each.  When that leaves most SMs idle, K is cut into equal ranges
-  // (a divisor of the super-block count, two or more super-blocks each).
-  int grid_rows = std::min(num_sms, std::max(1, std::min(units, N / 8)));
-  int ks = 1;
-  if (2 * grid_rows < num_sms) {
-    const int want = num_sms / grid_rows;
-    for (int d = std::min(want, nsb / 2); d >= 2; --d)
-      if (nsb % d == 0) {
-        ks = d;
-        break;
-      }
-  }
-  const int sbs = nsb / ks;
-  const int rows_per_cta = unit * ceil_div(units, grid_rows);
-  const int tiles = std::min(q4d::kMmaMaxTiles, ceil_div(rows_per_cta, 16));
-  const int rows_per_pass = 16 * tiles;
-  // Super-block columns per stage: the fewest of 1, 2, 4 (dividing the K
-  // range) that give at least 12 KB of weights per stage (stages that small
-  // still amortise the per-stage handshakes, and more of them keep the half-SM
-  // ring busy: 5.21 -> 5.11 ms per decode step against a 24 KB floor); then as
-  // many stages as fit, up to 16.
-  int KC = 1;
-  for (int c : {1, 2, 4}) {
-    if (sbs % c) continue;
-    KC = c;
-    if (size_t(c) * rows_per_pass * 144 >= 12 * 1024) break;
-  }
-  const size_t red = size_t(q4d::kConsumerWarps) * q4d::kMmaMaxTiles * 32 * 16;
-  const size_t stage = q4d::gemv_stage_bytes(M, KC, rows_per_pass);
-  int stages = int((kGemvSmemBudget - red) / (stage + 16));
-  stages = std::max(2, std::min(q4d::kMmaMaxStages, stages));
-  plan->k_splits = ks;
-  plan->sb_per_split = sbs;
-  plan->chunk_sb = KC;
-  plan->rows_per_cta = rows_per_cta;
-  plan->rows_per_pass = rows_per_pass;
-  plan->stages = stages;
+  if (!shape_fits(rows, K / 256, num_sms)) return Q4D_ERR_UNSUPPORTED_SHAPE;
+  const JobShape j = job_shape(rows, K / 256, num_sms);
+  plan->grid = j.grid;
   plan->threads = q4d::kGemvThreads;
-  plan->grid_rows = grid_rows;
-  plan->smem_bytes = stages * stage + red + size_t(stages) * 16;
-  plan->workspace_bytes = ks > 1 ? size_t(ks) * M * N * 4 : 0;
+  plan->row_blocks = j.rbs;
+  plan->units_per_row_block = j.upr;
+  plan->units = j.units;
+  plan->slots = j.slots;
+  plan->stages = gemv_stages(M, size_t(smem_optin));
+  plan->reserved = 0;
+  plan->smem_bytes = q4d::gemv_smem_bytes(M, plan->stages);
+  // row-block counters (8 bytes each), then the partial slots
+  plan->workspace_bytes =
+      j.slots > 0 ? round_up16(size_t(j.rbs) * kGemvCounterBytes) +
+                        size_t(j.rbs) * j.slots * M * q4d::kGemvRows * 4
+                  : 0;
   return Q4D_OK;
 }
 
+std::atomic<unsigned long long> g_gemv_tag{0};
 
-template <int M, int KC, bool SWIGLU>
-q4d_status launch_gemv_t(const q4d::GemvArgs& a, const q4d_gemv_plan& p, int dev,
-                         const DeviceState& s, cudaStream_t stream, bool pdl) {
+// A fresh 48-bit counter tag for every launch (never 0: zeroed memory means
+// "no arrival yet").
+unsigned long long next_gemv_tag() {
+  unsigned long long t = (g_gemv_tag.fetch_add(1, std::memory_order_relaxed) + 1) &
+                         ((1ull << 48) - 1);
+  return t ? t : 1ull;
+}
+
+template <int M>
+q4d_status launch_gemv_t(const q4d::GemvArgs& a, size_t smem, int dev, const DeviceState& s,
+                         cudaStream_t stream, bool pdl) {
   static std::atomic<bool> smem_set[kMaxDevices];
-  auto kernel = q4d::q4_gemv_kernel<M, KC, SWIGLU>;
+  auto kernel = q4d::q4_gemv_kernel<M>;
   q4d_status st = allow_smem(kernel, dev, s, smem_set);
   if (st != Q4D_OK) return st;
-  dim3 grid(p.grid_rows, p.k_splits);
-  if (!pdl) {
-    kernel<<<grid, p.threads, p.smem_bytes, stream>>>(a);
-    return Q4D_OK;
-  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(p.threads);
-  cfg.dynamicSmemBytes = p.smem_bytes;
+  cfg.gridDim = dim3(a.grid);
+  cfg.blockDim = dim3(q4d::kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kernel, a) == cudaSuccess ? Q4D_OK : Q4D_ERR_CUDA;
 }
 
-// y = W x (rows = N), or with `swiglu` h[m][n] = silu(g) * u over the N gate /
-// up row pairs of W (2N rows).
+q4d_status launch_gemv(int M, const q4d::GemvArgs& a, size_t smem, int dev, const DeviceState& s,
+                       cudaStream_t stream, bool pdl) {
+  switch (M) {
+    case 1: return launch_gemv_t<1>(a, smem, dev, s, stream, pdl);
+    case 2: return launch_gemv_t<2>(a, smem, dev, s, stream, pdl);
+    case 3: return launch_gemv_t<3>(a, smem, dev, s, stream, pdl);
+    case 4: return launch_gemv_t<4>(a, smem, dev, s, stream, pdl);
+    default: return launch_gemv_t<5>(a, smem, dev, s, stream, pdl);
+  }
+}
+
+// y = W x (N output rows), or with `swiglu` h[m][n] = silu(g) * u over the N
+// gate / up row pairs of W (2N weight rows): one job in one launch.
 q4d_status gemv_impl(const void* W_q4, const void* x, void* y, int M, int N, int K,
                      cudaStream_t stream, void* workspace, size_t workspace_bytes,
                      bool library_ws, bool pdl = false, bool swiglu = false,
@@ -287,59 +274,46 @@ q4d_status gemv_impl(const void* W_q4, const void* x, void* y, int M, int N, int
   if ((st = current_device(&dev, &s)) != Q4D_OK) return st;
   const int rows = swiglu ? 2 * N : N;
   q4d_gemv_plan p;
-  if ((st = plan_gemv_rows(M, rows, K, s->num_sms, swiglu ? 2 : 1, &p)) != Q4D_OK) return st;
-  if (p.smem_bytes > size_t(s->smem_optin)) return Q4D_ERR_UNSUPPORTED_SHAPE;
+  if ((st = plan_gemv_rows(M, rows, K, s->num_sms, s->smem_optin, &p)) != Q4D_OK) return st;
+  if (p.stages < 2) return Q4D_ERR_UNSUPPORTED_SHAPE;
   if (library_ws) {
-    if ((st = library_workspace(*s, p.workspace_bytes, &workspace)) != Q4D_OK) return st;
+    if ((st = library_workspace(s->gemv_ws, s->gemv_ws_bytes, p.workspace_bytes, &workspace)) !=
+        Q4D_OK)
+      return st;
   } else if (p.workspace_bytes > 0 && (!workspace || workspace_bytes < p.workspace_bytes)) {
     return Q4D_ERR_WORKSPACE;
   }
 
   q4d::GemvArgs a;
   std::memset(&a, 0, sizeof(a));
-  if ((st = tensor_map_2d(&a.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, uint64_t(K), uint64_t(M),
-                          uint64_t(K) * 2u, 256u, uint32_t(M))) != Q4D_OK)
-    return st;
-  a.W = static_cast<const uint8_t*>(W_q4);
-  a.out = p.k_splits > 1 ? static_cast<float*>(workspace) : static_cast<float*>(y);
-  a.out_bf16 = (out_bf16 && p.k_splits == 1) ? 1 : 0;
-  a.err = s->err;
-  a.N = rows;
-  a.sb_per_split = p.sb_per_split;
-  a.rows_per_pass = p.rows_per_pass;
-  a.grid_rows = p.grid_rows;
+  a.jobs = nullptr;
+  a.n_jobs = 1;
+  a.grid = p.grid;
   a.stages = p.stages;
-
-  switch (M * 8 + p.chunk_sb) {
-    case 1 * 8 + 1: st = (swiglu ? launch_gemv_t<1, 1, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<1, 1, false>(a, p, dev, *s, stream, pdl)); break;
-    case 1 * 8 + 2: st = (swiglu ? launch_gemv_t<1, 2, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<1, 2, false>(a, p, dev, *s, stream, pdl)); break;
-    case 1 * 8 + 4: st = (swiglu ? launch_gemv_t<1, 4, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<1, 4, false>(a, p, dev, *s, stream, pdl)); break;
-    case 2 * 8 + 1: st = (swiglu ? launch_gemv_t<2, 1, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<2, 1, false>(a, p, dev, *s, stream, pdl)); break;
-    case 2 * 8 + 2: st = (swiglu ? launch_gemv_t<2, 2, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<2, 2, false>(a, p, dev, *s, stream, pdl)); break;
-    case 2 * 8 + 4: st = (swiglu ? launch_gemv_t<2, 4, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<2, 4, false>(a, p, dev, *s, stream, pdl)); break;
-    case 3 * 8 + 1: st = (swiglu ? launch_gemv_t<3, 1, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<3, 1, false>(a, p, dev, *s, stream, pdl)); break;
-    case 3 * 8 + 2: st = (swiglu ? launch_gemv_t<3, 2, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<3, 2, false>(a, p, dev, *s, stream, pdl)); break;
-    case 3 * 8 + 4: st = (swiglu ? launch_gemv_t<3, 4, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<3, 4, false>(a, p, dev, *s, stream, pdl)); break;
-    case 4 * 8 + 1: st = (swiglu ? launch_gemv_t<4, 1, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<4, 1, false>(a, p, dev, *s, stream, pdl)); break;
-    case 4 * 8 + 2: st = (swiglu ? launch_gemv_t<4, 2, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<4, 2, false>(a, p, dev, *s, stream, pdl)); break;
-    case 4 * 8 + 4: st = (swiglu ? launch_gemv_t<4, 4, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<4, 4, false>(a, p, dev, *s, stream, pdl)); break;
-    case 5 * 8 + 1: st = (swiglu ? launch_gemv_t<5, 1, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<5, 1, false>(a, p, dev, *s, stream, pdl)); break;
-    case 5 * 8 + 2: st = (swiglu ? launch_gemv_t<5, 2, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<5, 2, false>(a, p, dev, *s, stream, pdl)); break;
-    default: st = (swiglu ? launch_gemv_t<5, 4, true>(a, p, dev, *s, stream, pdl) : launch_gemv_t<5, 4, false>(a, p, dev, *s, stream, pdl)); break;
+  a.err = s->err;
+  a.tag = next_gemv_tag();
+  if (p.workspace_bytes > 0) {
+    a.counters = static_cast<unsigned long long*>(workspace);
+    a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                          round_up16(size_t(p.row_blocks) * kGemvCounterBytes));
   }
-  if (st != Q4D_OK) return st;
-  if (p.k_splits > 1) {
-    const long long mn = (long long)M * N;
-    const int blocks = int(std::min<long long>((mn + 255) / 256, 4LL * s->num_sms));
-    if (swiglu)
-      q4d::q4_gemv_splitk_reduce_swiglu<<<blocks, 256, 0, stream>>>(
-          static_cast<const float*>(workspace), static_cast<float*>(y), M, N, p.k_splits,
-          out_bf16 ? 1 : 0);
-    else
-      q4d::q4_gemv_splitk_reduce<<<blocks, 256, 0, stream>>>(
-          static_cast<const float*>(workspace), static_cast<float*>(y), mn, p.k_splits,
-          out_bf16 ? 1 : 0);
-  }
+  q4d::GemvJobDesc& J = a.job;
+  J.W = static_cast<const uint8_t*>(W_q4);
+  J.x = static_cast<const uint16_t*>(x);
+  J.y = y;
+  J.part_off = 0;
+  J.N = rows;
+  J.nsb = K / 256;
+  J.flags = (out_bf16 ? q4d::kJobOutBf16 : 0u) | (swiglu ? q4d::kJobSwiglu : 0u);
+  J.wait_for = -1;
+  J.rbs = p.row_blocks;
+  J.upr = p.units_per_row_block;
+  J.units = p.units;
+  J.grid = p.grid;
+  J.slots = p.slots;
+  J.cnt_off = 0;
+  J.rot = 0;
+  if ((st = launch_gemv(M, a, p.smem_bytes, dev, *s, stream, pdl)) != Q4D_OK) return st;
   if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
   return Q4D_OK;
 }
@@ -394,7 +368,8 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
     return st;
   if (p.smem_bytes > size_t(s->smem_optin)) return Q4D_ERR_UNSUPPORTED_SHAPE;
   if (library_ws) {
-    if ((st = library_workspace(*s, p.workspace_bytes, &workspace)) != Q4D_OK) return st;
+    if ((st = library_workspace(s->ws, s->ws_bytes, p.workspace_bytes, &workspace)) != Q4D_OK)
+      return st;
   } else if (p.workspace_bytes > 0 && (!workspace || workspace_bytes < p.workspace_bytes)) {
     return Q4D_ERR_WORKSPACE;
   }
@@ -461,7 +436,7 @@ const char* q4d_status_string(int status) {
 }
 
 q4d_status q4d_plan_gemv(int M, int N, int K, int num_sms, q4d_gemv_plan* plan) {
-  return plan_gemv_rows(M, N, K, num_sms, 1, plan);
+  return plan_gemv_rows(M, N, K, num_sms, kSmemOptinB200, plan);
 }
 
 q4d_status q4d_plan_attn(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
@@ -531,7 +506,12 @@ extern "C" {
 
 size_t q4d_gemv_workspace_bytes(int M, int N, int K) {
   q4d_gemv_plan p;
-  if (q4d_plan_gemv(M, N, K, planning_sms(), &p) != Q4D_OK) return 0;
+  int dev = 0;
+  DeviceState* s = nullptr;
+  const bool have = current_device(&dev, &s) == Q4D_OK;
+  if (plan_gemv_rows(M, N, K, have ? s->num_sms : kPlanFallbackSms,
+                     have ? s->smem_optin : kSmemOptinB200, &p) != Q4D_OK)
+    return 0;
   return p.workspace_bytes;
 }
 
@@ -578,9 +558,150 @@ q4d_status q4_gemv_swiglu_ex(const void* W_gu, const void* x, void* h, int M, in
 
 size_t q4d_gemv_swiglu_workspace_bytes(int M, int N, int K) {
   if (N < 1 || N > (1 << 29)) return 0;
-  q4d_gemv_plan p;
-  if (plan_gemv_rows(M, 2 * N, K, planning_sms(), 2, &p) != Q4D_OK) return 0;
-  return p.workspace_bytes;
+  return q4d_gemv_workspace_bytes(M, 2 * N, K);
+}
+
+// ---- GEMV batches: many matrices in one launch
+namespace {
+
+constexpr uint32_t kBatchMagic = 0x42443451u;  // "Q4DB"
+constexpr size_t kBatchHeader = 64;
+
+struct BatchHeader {
+  uint32_t magic;
+  int n_jobs, M, num_sms, grid;
+  int pad_;
+  size_t workspace_bytes;
+  size_t counter_bytes;
+};
+static_assert(sizeof(BatchHeader) <= kBatchHeader, "batch header");
+static_assert(sizeof(q4d::GemvJobDesc) % 16 == 0, "job descriptor alignment");
+
+}  // namespace
+
+// Descriptor: header, the jobs, then the per-job completion counters and the
+// exit counter (zero when handed to the device; each launch leaves them zero).
+size_t batch_sync_offset(int n_jobs) {
+  return kBatchHeader + size_t(n_jobs) * sizeof(q4d::GemvJobDesc);
+}
+
+size_t q4d_gemv_batch_desc_bytes(int n_jobs) {
+  if (n_jobs < 1 || n_jobs > (1 << 20)) return 0;
+  return batch_sync_offset(n_jobs) + round_up16(size_t(n_jobs + 1) * 4);
+}
+
+q4d_status q4d_gemv_batch_prepare(const q4d_gemv_job* jobs, int n_jobs, int M, int num_sms,
+                                  void* desc, size_t desc_bytes, size_t* workspace_bytes) {
+  if (!jobs || !desc || n_jobs < 1 || n_jobs > (1 << 20) || num_sms < 1 || num_sms > 65535)
+    return Q4D_ERR_INVALID_ARG;
+  if (M < 1 || M > 5) return Q4D_ERR_UNSUPPORTED_SHAPE;
+  if (desc_bytes < q4d_gemv_batch_desc_bytes(n_jobs)) return Q4D_ERR_INVALID_ARG;
+  // grid: one CTA per SM, fewer if no job has that many units
+  int grid = 1;
+  for (int i = 0; i < n_jobs; ++i) {
+    const q4d_gemv_job& j = jobs[i];
+    const bool swiglu = (j.flags & Q4D_GEMV_SWIGLU) != 0;
+    if (j.flags & ~(Q4D_GEMV_OUT_BF16 | Q4D_GEMV_SWIGLU)) return Q4D_ERR_INVALID_ARG;
+    if (swiglu && j.N > (1 << 29)) return Q4D_ERR_UNSUPPORTED_SHAPE;
+    q4d_status st = check_gemv_shape(M, swiglu ? 2 * j.N : j.N, j.K);
+    if (st != Q4D_OK) return st;
+    if (!j.W_q4 || !j.x || !j.y) return Q4D_ERR_INVALID_ARG;
+    if (!aligned(j.W_q4, 16) || !aligned(j.x, 16) ||
+        !aligned(j.y, (j.flags & Q4D_GEMV_OUT_BF16) ? 2 : 4))
+      return Q4D_ERR_MISALIGNED;
+    if (j.wait_for < -1 || j.wait_for >= i) return Q4D_ERR_INVALID_ARG;
+    if (!shape_fits(swiglu ? 2 * j.N : j.N, j.K / 256, num_sms)) return Q4D_ERR_UNSUPPORTED_SHAPE;
+    const JobShape sh = job_shape(swiglu ? 2 * j.N : j.N, j.K / 256, num_sms);
+    grid = std::max(grid, sh.grid);
+  }
+  q4d::GemvJobDesc* out =
+      reinterpret_cast<q4d::GemvJobDesc*>(static_cast<uint8_t*>(desc) + kBatchHeader);
+  size_t counters = 0;  // tagged row-block counters
+  size_t partials = 0;  // floats
+  long long units_before = 0;  // rotates each job's CTA numbering (balance across the batch)
+  for (int i = 0; i < n_jobs; ++i) {
+    const q4d_gemv_job& j = jobs[i];
+    const bool swiglu = (j.flags & Q4D_GEMV_SWIGLU) != 0;
+    const int rows = swiglu ? 2 * j.N : j.N;
+    const JobShape sh = job_shape(rows, j.K / 256, grid);
+    q4d::GemvJobDesc d;
+    std::memset(&d, 0, sizeof(d));
+    d.W = static_cast<const uint8_t*>(j.W_q4);
+    d.x = static_cast<const uint16_t*>(j.x);
+    d.y = j.y;
+    d.N = rows;
+    d.nsb = j.K / 256;
+    d.flags = ((j.flags & Q4D_GEMV_OUT_BF16) ? q4d::kJobOutBf16 : 0u) |
+              (swiglu ? q4d::kJobSwiglu : 0u);
+    d.wait_for = j.wait_for;
+    d.rbs = sh.rbs;
+    d.upr = sh.upr;
+    d.units = sh.units;
+    d.grid = sh.grid;
+    d.slots = sh.slots;
+    d.cnt_off = int(counters);
+    d.part_off = (long long)partials;
+    d.rot = int(units_before % grid);
+    units_before += sh.units;
+    if (sh.slots > 0) {
+      counters += size_t(sh.rbs);
+      partials += size_t(sh.rbs) * sh.slots * M * q4d::kGemvRows;
+    }
+    std::memcpy(out + i, &d, sizeof(d));
+  }
+  BatchHeader h;
+  std::memset(&h, 0, sizeof(h));
+  h.magic = kBatchMagic;
+  h.n_jobs = n_jobs;
+  h.M = M;
+  h.num_sms = num_sms;
+  h.grid = grid;
+  h.counter_bytes = round_up16(counters * kGemvCounterBytes);
+  h.workspace_bytes = h.counter_bytes + partials * 4;
+  std::memset(desc, 0, kBatchHeader);
+  std::memcpy(desc, &h, sizeof(h));
+  std::memset(static_cast<uint8_t*>(desc) + batch_sync_offset(n_jobs), 0,
+              q4d_gemv_batch_desc_bytes(n_jobs) - batch_sync_offset(n_jobs));
+  if (workspace_bytes) *workspace_bytes = h.workspace_bytes;
+  return Q4D_OK;
+}
+
+q4d_status q4_gemv_batch_ex(const void* desc_host, void* desc_dev, void* stream,
+                            void* workspace, size_t workspace_bytes, unsigned flags) {
+  if (!desc_host || !desc_dev) return Q4D_ERR_INVALID_ARG;
+  if (flags & ~Q4D_GEMV_WEIGHT_PREFETCH) return Q4D_ERR_INVALID_ARG;
+  BatchHeader h;
+  std::memcpy(&h, desc_host, sizeof(h));
+  if (h.magic != kBatchMagic || h.n_jobs < 1 || h.M < 1 || h.M > 5 || h.grid < 1)
+    return Q4D_ERR_INVALID_ARG;
+  if (!aligned(desc_dev, 16) || (workspace && !aligned(workspace, 16))) return Q4D_ERR_MISALIGNED;
+  if (h.workspace_bytes > 0 && (!workspace || workspace_bytes < h.workspace_bytes))
+    return Q4D_ERR_WORKSPACE;
+  int dev = 0;
+  DeviceState* s = nullptr;
+  q4d_status st = current_device(&dev, &s);
+  if (st != Q4D_OK) return st;
+  if (h.num_sms != s->num_sms) return Q4D_ERR_INVALID_ARG;  // prepared for another device
+  const int stages = gemv_stages(h.M, size_t(s->smem_optin));
+  if (stages < 2) return Q4D_ERR_UNSUPPORTED_SHAPE;
+  q4d::GemvArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.jobs = reinterpret_cast<const q4d::GemvJobDesc*>(static_cast<const uint8_t*>(desc_dev) +
+                                                      kBatchHeader);
+  a.sync = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(desc_dev) +
+                                       batch_sync_offset(h.n_jobs));
+  a.n_jobs = h.n_jobs;
+  a.grid = h.grid;
+  a.stages = stages;
+  a.err = s->err;
+  a.tag = next_gemv_tag();
+  a.counters = static_cast<unsigned long long*>(workspace);
+  a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + h.counter_bytes);
+  if ((st = launch_gemv(h.M, a, q4d::gemv_smem_bytes(h.M, stages), dev, *s,
+                        static_cast<cudaStream_t>(stream), (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0)) !=
+      Q4D_OK)
+    return st;
+  return cudaGetLastError() == cudaSuccess ? Q4D_OK : Q4D_ERR_CUDA;
 }
 
 q4d_status q4kv_attn_decode(const void* Q, const void* Kq4, const void* Vq4, float* out,

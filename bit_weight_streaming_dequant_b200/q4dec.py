@@ -33,6 +33,7 @@ EXPORTS = (
     "q4d_unpack_q4_0_rows", "q4kv_append", "q4_gemv_swiglu_ex",
     "q4d_gemv_swiglu_workspace_bytes", "q8kv_attn_decode_ex", "q8kv_attn_workspace_bytes",
     "q8kv_plan_attn", "q4d_wait_selftest",
+    "q4d_gemv_batch_desc_bytes", "q4d_gemv_batch_prepare", "q4_gemv_batch_ex",
 )
 
 
@@ -43,11 +44,18 @@ class Q4DecError(RuntimeError):
 
 
 class GemvPlan(ctypes.Structure):
-    _fields_ = [("k_splits", ctypes.c_int), ("sb_per_split", ctypes.c_int),
-                ("chunk_sb", ctypes.c_int), ("rows_per_cta", ctypes.c_int),
-                ("rows_per_pass", ctypes.c_int), ("stages", ctypes.c_int),
-                ("threads", ctypes.c_int), ("grid_rows", ctypes.c_int),
+    _fields_ = [("grid", ctypes.c_int), ("threads", ctypes.c_int),
+                ("row_blocks", ctypes.c_int), ("units_per_row_block", ctypes.c_int),
+                ("units", ctypes.c_int), ("slots", ctypes.c_int),
+                ("stages", ctypes.c_int), ("reserved", ctypes.c_int),
                 ("smem_bytes", ctypes.c_size_t), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class GemvJob(ctypes.Structure):
+    """``q4d_gemv_job``: one GEMV of a batch launch."""
+    _fields_ = [("W_q4", ctypes.c_void_p), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("N", ctypes.c_int), ("K", ctypes.c_int), ("flags", ctypes.c_uint),
+                ("wait_for", ctypes.c_int)]
 
 
 class AttnPlan(ctypes.Structure):
@@ -97,6 +105,13 @@ def lib() -> ctypes.CDLL:
     L.q4_gemv_swiglu_ex.restype = i
     L.q4d_gemv_swiglu_workspace_bytes.argtypes = [i, i, i]
     L.q4d_gemv_swiglu_workspace_bytes.restype = sz
+    L.q4d_gemv_batch_desc_bytes.argtypes = [i]
+    L.q4d_gemv_batch_desc_bytes.restype = sz
+    L.q4d_gemv_batch_prepare.argtypes = [ctypes.POINTER(GemvJob), i, i, i, vp, sz,
+                                         ctypes.POINTER(ctypes.c_size_t)]
+    L.q4d_gemv_batch_prepare.restype = i
+    L.q4_gemv_batch_ex.argtypes = [vp, vp, vp, vp, sz, ctypes.c_uint]
+    L.q4_gemv_batch_ex.restype = i
     L.q8kv_attn_decode_ex.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, vp, vp, sz]
     L.q8kv_attn_decode_ex.restype = i
     L.q8kv_attn_workspace_bytes.argtypes = [i, i, i, i, i]
@@ -203,6 +218,7 @@ def _workspace(nbytes: int, device, workspace):
 
 GEMV_WEIGHT_PREFETCH = 1  # Q4D_GEMV_WEIGHT_PREFETCH
 GEMV_OUT_BF16 = 2         # Q4D_GEMV_OUT_BF16
+GEMV_SWIGLU = 4           # Q4D_GEMV_SWIGLU (batch jobs)
 
 
 def _out_flags(out_dtype, torch):
@@ -352,6 +368,69 @@ def _attn(Q, Kc, Vc, out, ctx_len, n_kv_heads, head_dim, kv_stride_tokens, softm
                                   None if ws is None else ws.data_ptr(), need)
     _check(st, name)
     return out
+
+
+class GemvBatch:
+    """Many GEMVs in one launch (``q4d_gemv_batch_prepare`` + ``q4_gemv_batch_ex``).
+
+    ``jobs``: list of dicts with keys ``W`` (uint8 weights), ``x`` (bf16
+    [M][K]), ``y`` (fp32 or bf16 output [M][N]), ``N``, ``K`` and optional
+    ``swiglu`` (W holds 2N interleaved gate / up rows, y = h [M][N]) and
+    ``wait_for`` (-1, or the index of the job whose outputs, and those of every
+    job before it, must be written before this job reads x).  All tensors must
+    stay alive and in place for as long as the batch is used.  The descriptor
+    is prepared and copied to the device once; :meth:`run` only launches."""
+
+    def __init__(self, jobs, *, device=None):
+        torch = _torch()
+        if not jobs:
+            raise ValueError("a batch needs at least one job")
+        M = None
+        arr = (GemvJob * len(jobs))()
+        self._keep = []
+        for i, j in enumerate(jobs):
+            W, x, y, N, K = j["W"], j["x"], j["y"], int(j["N"]), int(j["K"])
+            swiglu = bool(j.get("swiglu", False))
+            _dev_tensor(W, torch.uint8, f"jobs[{i}].W")
+            _dev_tensor(x, torch.bfloat16, f"jobs[{i}].x")
+            if x.dim() != 2 or x.shape[1] != K:
+                raise ValueError(f"jobs[{i}].x must be [M][K]")
+            if M is None:
+                M = x.shape[0]
+            if x.shape[0] != M:
+                raise ValueError("every job of a batch has the same M")
+            rows = 2 * N if swiglu else N
+            if W.numel() != rows * (K // 256) * 144:
+                raise ValueError(f"jobs[{i}].W has the wrong number of bytes")
+            _dev_tensor(y, y.dtype, f"jobs[{i}].y")
+            flags = _out_flags(y.dtype, torch) | (GEMV_SWIGLU if swiglu else 0)
+            if tuple(y.shape) != (M, N):
+                raise ValueError(f"jobs[{i}].y must be [M][N]")
+            arr[i] = GemvJob(W.data_ptr(), x.data_ptr(), y.data_ptr(), N, K, flags,
+                             int(j.get("wait_for", -1)))
+            self._keep += [W, x, y]
+        self.device = x.device if device is None else device
+        self.M, self.n_jobs = M, len(jobs)
+        L = lib()
+        with torch.cuda.device(self.device):
+            sms = torch.cuda.get_device_properties(self.device).multi_processor_count
+            nbytes = L.q4d_gemv_batch_desc_bytes(len(jobs))
+            self.desc_host = torch.zeros(nbytes, dtype=torch.uint8)
+            ws = ctypes.c_size_t(0)
+            _check(L.q4d_gemv_batch_prepare(arr, len(jobs), M, sms, self.desc_host.data_ptr(),
+                                            nbytes, ctypes.byref(ws)), "q4d_gemv_batch_prepare")
+            self.desc_dev = self.desc_host.to(self.device)
+            self.workspace_bytes = ws.value
+            self.workspace = torch.empty(max(16, ws.value), dtype=torch.uint8, device=self.device)
+
+    def run(self, stream=None, weight_prefetch: bool = False):
+        torch = _torch()
+        with torch.cuda.device(self.device):
+            st = lib().q4_gemv_batch_ex(self.desc_host.data_ptr(), self.desc_dev.data_ptr(),
+                                        _stream_ptr(stream), self.workspace.data_ptr(),
+                                        self.workspace.numel(),
+                                        GEMV_WEIGHT_PREFETCH if weight_prefetch else 0)
+        _check(st, "q4_gemv_batch_ex")
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

@@ -70,7 +70,7 @@
 extern "C" {
 #endif
 
-#define Q4D_VERSION 10000 /* 1.0.0 */
+#define Q4D_VERSION 20000 /* 2.0.0 */
 
 typedef enum {
   Q4D_OK = 0,
@@ -103,6 +103,15 @@ const char* q4d_status_string(int status);
  * into a CUDA graph).  q4_gemv_ex takes the stream and a caller-owned
  * workspace of at least q4d_gemv_workspace_bytes(M, N, K) bytes (it may be
  * NULL when that size is 0); it never allocates.
+ *
+ * Partition (q4d_plan_gemv): rows are cut into blocks of 128 and K into units
+ * of 512 elements; the units are shared out in equal contiguous ranges over
+ * one CTA per SM, so a row block may be summed by several CTAs.  Those CTAs
+ * write fp32 partial sums into the workspace and the last one to finish adds
+ * them in a fixed order, so results are deterministic.  The workspace holds
+ * small counters besides the partial sums; it needs no initialisation (its
+ * previous contents are ignored), but calls whose kernels may overlap on the
+ * GPU must not share one workspace.
  */
 q4d_status q4_gemv(const void* W_q4, const void* x, float* y, int M, int N, int K);
 q4d_status q4_gemv_ex(const void* W_q4, const void* x, float* y, int M, int N, int K,
@@ -140,13 +149,14 @@ q4d_status q4_gemv_ex2(const void* W_q4, const void* x, void* y, int M, int N, i
  *
  *   W_gu : 2N x K elements of Q4_0 in the weight layout above, the gate row n
  *          stored as row 2n and the up row n as row 2n + 1 (interleaved).
- *   x    : bf16 [M][K];  h : fp32 [M][N] = silu(g) * u, silu(g) = g / (1 + e^-g),
- *          g and u the fp32 gate / up outputs of row pair n (bf16 [M][N] with
- *          Q4D_GEMV_OUT_BF16: the fp32 h rounded to nearest even).
+ *   x    : bf16 [M][K];  h : fp32 [M][N] = silu(g) * u, silu(g) = g / (1 + e^-g)
+ *          evaluated in fp32 with expf, g and u the fp32 gate / up outputs of
+ *          row pair n (bf16 [M][N] with Q4D_GEMV_OUT_BF16: the fp32 h rounded
+ *          to nearest even).
  *   Requirements as q4_gemv (with 2N rows); workspace of at least
  *   q4d_gemv_swiglu_workspace_bytes(M, N, K) bytes; flags as q4_gemv_ex2.
- * One weight stream and one launch (plus a reduction launch when K is split)
- * instead of two GEMVs and an elementwise pass.
+ * One weight stream and one launch instead of two GEMVs and an elementwise
+ * pass.
  */
 q4d_status q4_gemv_swiglu_ex(const void* W_gu, const void* x, void* h, int M, int N, int K,
                              void* stream, void* workspace, size_t workspace_bytes,
@@ -156,6 +166,70 @@ size_t q4d_gemv_swiglu_workspace_bytes(int M, int N, int K);
  * count; a host without a usable device is planned for 148 SMs).  Returns 0
  * for invalid shapes as well as for shapes that need none. */
 size_t q4d_gemv_workspace_bytes(int M, int N, int K);
+
+/* ------------------------------------------------------------ GEMV batch --
+ * Many GEMVs in ONE launch: the weight stream of a whole decode step (every
+ * layer's projections and the output head, "Qwen3.8-27B at 256K on a 24GB RTX
+ * PRO 4000 SFF (432 GB/s): 50 tok/s with MTP", paragraph beginning "NVIDIA
+ * quotes 432 GB/s") without a launch, ramp-up and tail per matrix.  The jobs
+ * run in order on one CTA per SM; while a job waits for its input, the CTAs
+ * already stream the weights of the jobs after it (weights depend on
+ * nothing).  No counterpart in the pages: a launch form of this library.
+ *
+ *   q4d_gemv_job: one GEMV of the batch.
+ *     W_q4, x, y, N, K : as q4_gemv (device pointers; y is [M][N]);
+ *     flags   : Q4D_GEMV_OUT_BF16 (y in bf16) and/or Q4D_GEMV_SWIGLU (W_q4
+ *               holds 2N interleaved gate / up rows and y receives
+ *               h = silu(g) * u [M][N], as q4_gemv_swiglu_ex);
+ *     wait_for: -1 -- x may be read as soon as the kernel before the launch on
+ *               the stream has completed (every job can use -1 when no job of
+ *               the batch writes another job's x);
+ *               j (0 <= j < this job's index) -- x is read only after job j
+ *               and every job before it have written their outputs, e.g. x is
+ *               job j's y.
+ *   Each job must also not overwrite an x or y that an earlier job, not yet
+ *   finished, still uses: give it a wait_for at least as late as that job.
+ *
+ *   q4d_gemv_batch_desc_bytes(n_jobs): bytes of the launch descriptor.
+ *   q4d_gemv_batch_prepare: host only (no CUDA call).  Validates every job as
+ *     q4_gemv would (same status codes), plans the launch for a device with
+ *     num_sms SMs and M activation rows (every job has M rows), writes the
+ *     descriptor into the host buffer `desc` (desc_bytes >= the size above)
+ *     and the workspace size into *workspace_bytes.
+ *   q4_gemv_batch_ex: launches the batch on `stream`.  desc_host is the
+ *     prepared host buffer, desc_dev a byte-for-byte copy of it in device
+ *     memory (16-byte aligned): copy it once, launch many times.  Its tail
+ *     holds the per-job completion counters, zero as prepared; a launch counts
+ *     on them and sets them back to zero before it ends, so launches that may
+ *     overlap on the GPU must not share a descriptor copy, and a copy must not
+ *     be rewritten while a launch may run.  num_sms
+ *     must be the current device's SM count, else Q4D_ERR_INVALID_ARG.
+ *     workspace: device memory of at least *workspace_bytes (16-byte aligned;
+ *     no initialisation needed; launches that may overlap on the GPU must not
+ *     share it), else Q4D_ERR_WORKSPACE.  flags: 0 or
+ *     Q4D_GEMV_WEIGHT_PREFETCH (as q4_gemv_ex2: the first weights stream while
+ *     the previous kernel on the stream still runs).  Never allocates; the
+ *     launch can be captured into a CUDA graph and replayed.
+ *   The CTAs of a batch wait for one another between dependent jobs, so all
+ *   of them must be resident together: one CTA per SM, as launched, on an
+ *   otherwise idle device (each wait is bounded; see q4d_device_error).
+ *   Results are those of the single-GEMV entry points, bit for bit.
+ */
+#define Q4D_GEMV_SWIGLU 4u
+typedef struct {
+  const void* W_q4;
+  const void* x;
+  void* y;
+  int N;
+  int K;
+  unsigned flags;
+  int wait_for;
+} q4d_gemv_job;
+size_t q4d_gemv_batch_desc_bytes(int n_jobs);
+q4d_status q4d_gemv_batch_prepare(const q4d_gemv_job* jobs, int n_jobs, int M, int num_sms,
+                                  void* desc, size_t desc_bytes, size_t* workspace_bytes);
+q4d_status q4_gemv_batch_ex(const void* desc_host, void* desc_dev, void* stream,
+                            void* workspace, size_t workspace_bytes, unsigned flags);
 
 /* ------------------------------------------------------------- attention --
  * For draft row m (absolute position p_m = ctx_len - M + m) and query head h
@@ -176,6 +250,20 @@ size_t q4d_gemv_workspace_bytes(int M, int N, int K);
  * pre-scaled), the legacy default stream and a library-owned workspace (same
  * rules as q4_gemv).  The _ex form takes all of them explicitly and never
  * allocates; workspace must hold q4d_attn_workspace_bytes(...) bytes.
+ *
+ * Supported value range (the same for every M and both cache formats): the
+ * kernels feed Q and the dequantised K/V values to the tensor cores as IEEE
+ * fp16, so
+ *   - |Q| <= 65504 (bf16 queries beyond the fp16 range are not supported;
+ *     |Q| < 2^-14 is rounded to an fp16 subnormal, absolute error <= 2^-25);
+ *   - Q4_0 cache: |d| <= 8188 for every block scale, so that every value
+ *     d * (q - 8) lies within +-65504 (q4kv_append stores such scales for
+ *     any input |v| <= 65504);
+ *   - Q8_0 cache: |d| <= 511.75, so that every value d * q (q = -128..127)
+ *     lies within +-65504.
+ * Inside this range the result meets the stated accuracy for any row count;
+ * outside it the result is undefined (it may be inf or NaN).  The scales are
+ * device data, so the library does not check them.
  */
 q4d_status q4kv_attn_decode(const void* Q, const void* Kq4, const void* Vq4, float* out,
                             int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M);
@@ -247,16 +335,16 @@ q4d_status q4kv_attn_decode_noalloc(const void* Q, const void* Kq4, const void* 
  * a device with num_sms SMs; the compute entry points use exactly these.
  */
 typedef struct {
-  int k_splits;          /* K is cut into this many equal ranges (1 = no split)  */
-  int sb_per_split;      /* super-blocks per K range                             */
-  int chunk_sb;          /* super-blocks of K per pipeline stage                 */
-  int rows_per_cta;      /* most rows any CTA owns                               */
-  int rows_per_pass;     /* rows held per pass (multiple of 16, at most 128)     */
-  int stages;            /* shared-memory pipeline depth                         */
-  int threads;           /* threads per CTA                                      */
-  int grid_rows;         /* CTAs per K range (grid = grid_rows * k_splits)       */
-  size_t smem_bytes;     /* dynamic shared memory per CTA                        */
-  size_t workspace_bytes;/* fp32 partials, k_splits * M * N * 4 when k_splits > 1 */
+  int grid;              /* CTAs, one per SM at most (fewer only for tiny shapes)  */
+  int threads;           /* threads per CTA                                        */
+  int row_blocks;        /* ceil(N / 128): blocks of 128 weight rows               */
+  int units_per_row_block; /* ceil(K / 512): units of two 256-element columns      */
+  int units;             /* row_blocks * units_per_row_block, shared out evenly    */
+  int slots;             /* most CTAs sharing one row block (0: none is shared)    */
+  int stages;            /* shared-memory pipeline depth (one unit per stage)      */
+  int reserved;
+  size_t smem_bytes;     /* dynamic shared memory per CTA                          */
+  size_t workspace_bytes;/* counters + fp32 partial sums of shared row blocks      */
 } q4d_gemv_plan;
 
 typedef struct {

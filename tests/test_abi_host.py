@@ -29,7 +29,7 @@ def test_library_exports_every_declared_function():
 
 def test_version_and_status_strings():
     L = q4dec.lib()
-    assert L.q4d_version() == 10000
+    assert L.q4d_version() == 20000
     for code in range(7):
         assert L.q4d_status_string(code)
     assert L.q4d_status_string(99) == b"unknown status"
@@ -123,6 +123,7 @@ def test_q8_plan_and_workspace_queries():
 def test_plan_rejects_bad_inputs():
     L = q4dec.lib()
     p = q4dec.GemvPlan()
+    assert ctypes.sizeof(p) == 8 * 4 + 2 * 8
     assert L.q4d_plan_gemv(1, 16, 256, 0, ctypes.byref(p)) == 1
     assert L.q4d_plan_gemv(1, 16, 256, 148, None) == 1
     assert L.q4d_plan_gemv(7, 16, 256, 148, ctypes.byref(p)) == 2
@@ -136,9 +137,60 @@ def test_workspace_queries_without_device_use_the_fallback_plan():
     # invalid shapes report 0
     assert L.q4d_gemv_workspace_bytes(0, 16, 256) == 0
     assert L.q4d_attn_workspace_bytes(4096, 24, 5, 256, 1) == 0
-    # layer shapes need no split-K workspace; the long context needs merge space
-    assert L.q4d_gemv_workspace_bytes(1, 17408, 5120) == 0
+    # row blocks shared between CTAs need partial-sum space; one CTA does not;
+    # the long context needs merge space
+    p = q4dec.plan_gemv(1, 17408, 5120, 148)
+    assert L.q4d_gemv_workspace_bytes(1, 17408, 5120) == p.workspace_bytes > 0
+    assert L.q4d_gemv_workspace_bytes(1, 1, 256) == 0
     assert L.q4d_attn_workspace_bytes(262144, 24, 4, 256, 5) > 0
+
+
+def _batch_jobs(n, **kw):
+    jobs = (q4dec.GemvJob * n)()
+    for i in range(n):
+        jobs[i] = q4dec.GemvJob(FAKE, FAKE, FAKE, kw.get("N", 256), kw.get("K", 512),
+                                kw.get("flags", 0), kw.get("wait_for", -1 if i == 0 else i - 1))
+    return jobs
+
+
+def test_gemv_batch_prepare_validates_without_cuda():
+    L = q4dec.lib()
+    n = 3
+    nbytes = L.q4d_gemv_batch_desc_bytes(n)
+    assert nbytes > 0 and L.q4d_gemv_batch_desc_bytes(0) == 0
+    buf = ctypes.create_string_buffer(nbytes)
+    ws = ctypes.c_size_t(0)
+    assert L.q4d_gemv_batch_prepare(_batch_jobs(n, N=17408, K=5120), n, 1, 148, buf, nbytes,
+                                    ctypes.byref(ws)) == 0
+    assert ws.value == 3 * q4dec.plan_gemv(1, 17408, 5120, 148).workspace_bytes
+    # two row blocks, one CTA each: nothing to share, no workspace
+    assert L.q4d_gemv_batch_prepare(_batch_jobs(n), n, 1, 148, buf, nbytes, ctypes.byref(ws)) == 0
+    assert ws.value == 0
+    # the completion counters at the descriptor's end are handed over zeroed
+    assert set(buf.raw[nbytes - 16:]) == {0}
+    assert L.q4d_gemv_batch_prepare(_batch_jobs(n), n, 6, 148, buf, nbytes, None) == 2
+    assert L.q4d_gemv_batch_prepare(_batch_jobs(n), n, 1, 0, buf, nbytes, None) == 1
+    assert L.q4d_gemv_batch_prepare(_batch_jobs(n), n, 1, 148, buf, nbytes - 1, None) == 1
+    assert L.q4d_gemv_batch_prepare(_batch_jobs(n, K=100), n, 1, 148, buf, nbytes, None) == 2
+    assert L.q4d_gemv_batch_prepare(_batch_jobs(n, flags=1), n, 1, 148, buf, nbytes, None) == 1
+    bad = _batch_jobs(n)
+    bad[2].wait_for = 2                       # a job cannot wait for itself
+    assert L.q4d_gemv_batch_prepare(bad, n, 1, 148, buf, nbytes, None) == 1
+    bad = _batch_jobs(n)
+    bad[1].x = FAKE + 8                       # activations 16-byte aligned
+    assert L.q4d_gemv_batch_prepare(bad, n, 1, 148, buf, nbytes, None) == 3
+    bad = _batch_jobs(n)
+    bad[0].y = None
+    assert L.q4d_gemv_batch_prepare(bad, n, 1, 148, buf, nbytes, None) == 1
+    # a launch refuses a foreign or bad descriptor before touching CUDA
+    assert L.q4d_gemv_batch_prepare(_batch_jobs(n, N=17408, K=5120), n, 1, 148, buf, nbytes,
+                                    ctypes.byref(ws)) == 0
+    assert L.q4_gemv_batch_ex(None, FAKE, None, FAKE, 1 << 20, 0) == 1
+    assert L.q4_gemv_batch_ex(buf, FAKE, None, FAKE, 1 << 20, 2) == 1
+    junk = ctypes.create_string_buffer(nbytes)
+    assert L.q4_gemv_batch_ex(junk, FAKE, None, FAKE, 1 << 20, 0) == 1
+    assert L.q4_gemv_batch_ex(buf, FAKE + 8, None, FAKE, 1 << 20, 0) == 3
+    assert L.q4_gemv_batch_ex(buf, FAKE, None, None, 0, 0) == 4
 
 
 def test_append_rejects_bad_arguments_without_cuda():

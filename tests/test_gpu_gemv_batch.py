@@ -1,0 +1,139 @@
+"""GPU tests of the multi-matrix GEMV launch (q4d_gemv_batch_prepare +
+q4_gemv_batch_ex, through the C ABI via the binding's GemvBatch).
+
+Every job of a batch must give, bit for bit, what the single-GEMV entry point
+gives (same partition, same summation order); dependent jobs must read their
+input only after the job they wait for has written it; the completion and
+row-block counters must leave the descriptor and workspace ready for the next
+launch (repeated launches, CUDA-graph replays, a workspace full of garbage)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from bit_weight_streaming_dequant_b200 import q4dec
+from gpu_util import assert_gemv_close, dev_bf16, dev_bytes
+
+pytestmark = pytest.mark.gpu
+
+
+def _weights(seed, N, K, device_gen=False):
+    if device_gen:
+        return synth.device_q4_0_weights(seed, N, K)
+    return dev_bytes(synth.q4_0_weights(seed, N, K))
+
+
+def test_independent_jobs_equal_single_calls(cuda_ok):
+    M = 3
+    shapes = [(512, 1024), (6144, 5120), (5120, 6144), (37, 4352), (17408, 5120), (5120, 17408)]
+    jobs, refs = [], []
+    for i, (N, K) in enumerate(shapes):
+        W = _weights(700 + i, N, K, device_gen=N * K > 1 << 24)
+        x = dev_bf16(synth.activations(710 + i, M, K))
+        y = torch.full((M, N), float("nan"), device="cuda")
+        jobs.append(dict(W=W, x=x, y=y, N=N, K=K))
+        refs.append(q4dec.q4_gemv(W, x, N=N, K=K))
+    b = q4dec.GemvBatch(jobs)
+    for launch in range(3):
+        for j in jobs:
+            j["y"].fill_(float("nan"))
+        b.run()
+        torch.cuda.synchronize()
+        for i, (j, r) in enumerate(zip(jobs, refs)):
+            assert torch.equal(j["y"], r), f"launch {launch} job {i} {shapes[i]}"
+    assert q4dec.device_error() == 0
+
+
+def test_small_jobs_against_the_oracle(cuda_ok):
+    M = 2
+    shapes = [(1, 256), (3, 512), (300, 1280), (64, 65536), (129, 2048)]
+    jobs, ref = [], []
+    for i, (N, K) in enumerate(shapes):
+        Wnp, xnp = synth.q4_0_weights(720 + i, N, K), synth.activations(730 + i, M, K)
+        jobs.append(dict(W=dev_bytes(Wnp), x=dev_bf16(xnp),
+                         y=torch.empty((M, N), device="cuda"), N=N, K=K,
+                         wait_for=-1 if i == 0 else i - 1))
+        ref.append(oracle.gemv(Wnp, xnp, M, N, K))
+    q4dec.GemvBatch(jobs).run()
+    torch.cuda.synchronize()
+    for i, (j, (y_ref, S)) in enumerate(zip(jobs, ref)):
+        assert_gemv_close(j["y"], y_ref, S, f"job {i} {shapes[i]}")
+
+
+def test_dependent_chain_reads_the_previous_output(cuda_ok):
+    # job k reads job k-1's bf16 output as its x: a chain 5120 -> 6144 ->
+    # 5120 -> 17408 -> 5120 with every link waiting for the one before
+    M = 2
+    dims = [5120, 6144, 5120, 17408, 5120]
+    Ws = [_weights(740 + k, dims[k + 1], dims[k], device_gen=True) for k in range(len(dims) - 1)]
+    x0 = dev_bf16(synth.activations(750, M, dims[0]))
+    outs = [torch.empty((M, dims[k + 1]), dtype=torch.bfloat16, device="cuda")
+            for k in range(len(Ws))]
+    jobs = [dict(W=Ws[k], x=x0 if k == 0 else outs[k - 1], y=outs[k], N=dims[k + 1],
+                 K=dims[k], wait_for=k - 1) for k in range(len(Ws))]
+    b = q4dec.GemvBatch(jobs)
+    # reference: the same chain as single calls, one after another
+    ref, x = [], x0
+    for k in range(len(Ws)):
+        ref.append(q4dec.q4_gemv(Ws[k], x, N=dims[k + 1], K=dims[k], out_dtype=torch.bfloat16))
+        x = ref[-1]
+    torch.cuda.synchronize()
+    for launch in range(3):
+        for o in outs:
+            o.fill_(float("nan"))
+        b.run()
+        torch.cuda.synchronize()
+        for k in range(len(Ws)):
+            assert torch.equal(outs[k], ref[k]), f"launch {launch} link {k}"
+    assert q4dec.device_error() == 0
+
+
+def test_swiglu_job_and_garbage_workspace(cuda_ok):
+    M = 5
+    N, K = 1024, 5120
+    Wgu = _weights(760, 2 * N, K)
+    W2 = _weights(761, 6144, 5120)
+    x = dev_bf16(synth.activations(762, M, K))
+    h = torch.empty((M, N), device="cuda")
+    y2 = torch.empty((M, 6144), dtype=torch.bfloat16, device="cuda")
+    b = q4dec.GemvBatch([dict(W=Wgu, x=x, y=h, N=N, K=K, swiglu=True),
+                         dict(W=W2, x=x, y=y2, N=6144, K=5120, wait_for=0)])
+    h_ref = q4dec.q4_gemv_swiglu(Wgu, x, N=N, K=K)
+    y2_ref = q4dec.q4_gemv(W2, x, N=6144, K=5120, out_dtype=torch.bfloat16)
+    for fill in (0xFF, 0x00, 0x5A):
+        b.workspace.fill_(fill)          # leftovers of other uses are ignored
+        b.run()
+        torch.cuda.synchronize()
+        assert torch.equal(h, h_ref) and torch.equal(y2, y2_ref), f"workspace fill {fill:#x}"
+    assert q4dec.device_error() == 0
+
+
+def test_batch_replays_as_a_cuda_graph(cuda_ok):
+    M = 1
+    shapes = [(6144, 5120), (5120, 6144), (17408, 5120)]
+    jobs = []
+    for i, (N, K) in enumerate(shapes):
+        jobs.append(dict(W=_weights(770 + i, N, K, device_gen=True),
+                         x=dev_bf16(synth.activations(780 + i, M, K)),
+                         y=torch.empty((M, N), device="cuda"), N=N, K=K,
+                         wait_for=i - 1))
+    b = q4dec.GemvBatch(jobs)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        b.run(weight_prefetch=True)
+    torch.cuda.synchronize()
+    eager = [j["y"].clone() for j in jobs]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        b.run(weight_prefetch=True)
+    for _ in range(3):
+        for j in jobs:
+            j["y"].fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for i, j in enumerate(jobs):
+            assert torch.equal(j["y"], eager[i]), f"replay job {i}"
+    del g
+    assert q4dec.device_error() == 0

@@ -43,14 +43,22 @@ def test_swiglu_matches_oracle(cuda_ok, N, K, M):
 def test_swiglu_equals_two_plain_gemvs_then_silu(cuda_ok):
     N, K, M = 1024, 5120, 2
     Wg, Wu = synth.q4_0_weights(61, N, K), synth.q4_0_weights(62, N, K)
-    x = dev_bf16(synth.activations(63, M, K))
+    xnp = synth.activations(63, M, K)
+    x = dev_bf16(xnp)
     h = q4dec.q4_gemv_swiglu(dev_bytes(_interleave(Wg, Wu, N, K)), x, N=N, K=K,
                              weight_prefetch=True)
     g = q4dec.q4_gemv(dev_bytes(Wg), x, N=N, K=K)
     u = q4dec.q4_gemv(dev_bytes(Wu), x, N=N, K=K)
     torch.cuda.synchronize()
-    ref = (g / (1 + torch.exp(-g)) * u)
-    # the fused kernel's g and u are the plain GEMV's bit for bit; only the
-    # epilogue's exp and division may differ in the last bits
-    torch.testing.assert_close(h, ref, rtol=1e-5, atol=1e-6)
+    ref = (g / (1 + torch.exp(-g)) * u).double().cpu().numpy()
+    # The fused matrix has 2N rows, so its K ranges split at other places than
+    # the plain N-row GEMVs': g and u agree up to fp32 reassociation of their
+    # sums (far below 1e-5 of sum |w x|), carried through silu(g) * u, plus
+    # the two epilogues' fp32 roundings.
+    _, Sg = oracle.gemv(Wg, xnp, M, N, K)
+    _, Su = oracle.gemv(Wu, xnp, M, N, K)
+    gd, ud = g.double().cpu().numpy(), u.double().cpu().numpy()
+    bound = oracle.swiglu_tolerance(gd, ud, 1e-5 * Sg, 1e-5 * Su) + 1e-6 * np.abs(ref)
+    err = np.abs(h.double().cpu().numpy() - ref)
+    assert (err <= bound).all(), f"worst {(err / bound).max():.3f} of the bound"
     assert q4dec.device_error() == 0

@@ -12,12 +12,20 @@ TX_LIMIT = (1 << 20) - 1           # mbarrier transaction-count range
 SMEM_OPTIN = 227 * 1024            # B200 opt-in shared memory per block
 
 
-def _wbox(R):
-    return -(-R * 144 // 128) * 128
+GEMV_ROWS, GEMV_COLS, GEMV_WARPS, GEMV_THREADS = 128, 2, 16, 608
+GEMV_WBOX = GEMV_ROWS * 144
 
 
-def _stage_bytes(M, KC, R):
-    return KC * (_wbox(R) + M * 512)
+def _gemv_stage_bytes(M):
+    return GEMV_COLS * GEMV_WBOX + M * GEMV_COLS * 512
+
+
+def _unit_begin(c, U, G):
+    return c * U // G
+
+
+def _unit_owner(u, U, G):
+    return ((u + 1) * G - 1) // U
 
 
 GEMV_SHAPES = [(1, 512, 1024), (1, 17408, 5120), (1, 5120, 17408), (1, 6144, 5120),
@@ -25,7 +33,7 @@ GEMV_SHAPES = [(1, 512, 1024), (1, 17408, 5120), (1, 5120, 17408), (1, 6144, 512
                (4, 6144, 5120), (5, 5120, 17408), (5, 151936, 5120), (1, 1, 256),
                (5, 3, 256), (1, 37, 4352), (3, 300, 1280), (2, 64, 65536), (5, 7, 32768),
                (4, 100, 256), (1, 147, 512), (1, 149, 512), (5, 1000, 2048), (2, 2, 17408),
-               (1, 1300, 512), (3, 40000, 768)]
+               (1, 1300, 512), (3, 40000, 768), (5, 34816, 5120)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMV_SHAPES)
@@ -33,66 +41,109 @@ GEMV_SHAPES = [(1, 512, 1024), (1, 17408, 5120), (1, 5120, 17408), (1, 6144, 512
 def test_gemv_geometry(M, N, K, sms):
     p = q4dec.plan_gemv(M, N, K, sms)
     nsb = K // 256
-    ks, KC = p.k_splits, p.chunk_sb
-    assert p.threads == 288 and nsb % ks == 0 and p.sb_per_split == nsb // ks
-    assert KC in (1, 2, 4) and p.sb_per_split % KC == 0
-    assert 1 <= p.grid_rows <= sms and p.grid_rows * ks <= max(sms, p.grid_rows)
-    R = p.rows_per_pass
-    tiles = R // 16
-    assert R % 16 == 0 and 1 <= tiles <= 8 and tiles == min(8, -(-p.rows_per_cta // 16))
-    wbox, stage = _wbox(R), _stage_bytes(M, KC, R)
-    xoff = KC * wbox
-    assert stage % 128 == 0 and xoff % 128 == 0 and wbox >= R * 144
-    red = 8 * 8 * 32 * 16
-    assert p.smem_bytes == p.stages * stage + red + p.stages * 16
-    assert 2 <= p.stages <= 16 and p.smem_bytes <= SMEM_OPTIN
-    assert (p.stages * stage + red) % 8 == 0
-    assert p.workspace_bytes == (ks * M * N * 4 if ks > 1 else 0)
-    w_bytes = N * nsb * 144
-    out_len = ks * M * N if ks > 1 else M * N
-    n_chunks = p.sb_per_split // KC
-
+    rbs, upr = -(-N // GEMV_ROWS), -(-nsb // GEMV_COLS)
+    U, G = rbs * upr, p.grid
+    assert p.threads == GEMV_THREADS and p.row_blocks == rbs and p.units_per_row_block == upr
+    assert p.units == U and 1 <= G <= min(sms, U)
+    stage = _gemv_stage_bytes(M)
+    red = 8 * 8 * 16 * M * 4
+    assert stage % 128 == 0 and (p.stages * stage) % 128 == 0
+    fin = 4 * M * 128 * 4                      # four segment buffers (consumers -> epilogue)
+    assert p.smem_bytes == p.stages * stage + red + fin + 16 + p.stages * 16 + 4 * 16
+    assert p.smem_bytes + stage + 16 > SMEM_OPTIN or p.stages == 8   # as many stages as fit
+    assert 2 <= p.stages <= 8 and p.smem_bytes <= SMEM_OPTIN
+    # the units are shared out exactly once, every CTA getting at least one
+    ranges = [(_unit_begin(c, U, G), _unit_begin(c + 1, U, G)) for c in range(G)]
+    assert ranges[0][0] == 0 and ranges[-1][1] == U
+    assert all(b > a for a, b in ranges) and all(ranges[i][1] == ranges[i + 1][0]
+                                                   for i in range(G - 1))
+    assert max(b - a for a, b in ranges) - min(b - a for a, b in ranges) <= 1
+    for c, (a, b) in enumerate(ranges):
+        assert _unit_owner(a, U, G) == c and _unit_owner(b - 1, U, G) == c
+    # contributors per row block, their slots, the workspace carve-up
+    slots = 0
+    for rb in range(rbs):
+        first, last = _unit_owner(rb * upr, U, G), _unit_owner(rb * upr + upr - 1, U, G)
+        if last > first:
+            slots = max(slots, last - first + 1)
+            for c in range(first, last + 1):        # every one of them holds a unit of rb
+                a, b = ranges[c]
+                assert a < (rb + 1) * upr and b > rb * upr
+    assert p.slots == slots
+    counters = -(-rbs * 8 // 16) * 16
+    assert p.workspace_bytes == (counters + rbs * slots * M * 128 * 4 if slots else 0)
+    # every copy stays inside its source buffer and its stage slot
+    w_bytes, x_bytes = N * nsb * 144, M * K * 2
+    for c in {0, G // 2, G - 1}:
+        a, b = ranges[c]
+        for u in range(a, b):
+            rb, cp = divmod(u, upr)
+            col0 = 2 * cp
+            kc = min(2, nsb - col0)
+            rows = min(GEMV_ROWS, N - rb * GEMV_ROWS)
+            assert kc >= 1 and rows >= 1
+            assert kc * (rows * 144 + M * 512) <= TX_LIMIT
+            for j in range(kc):
+                src = ((col0 + j) * N + rb * GEMV_ROWS) * 144
+                assert src % 16 == 0 and src + rows * 144 <= w_bytes
+                assert j * GEMV_WBOX + rows * 144 <= GEMV_COLS * GEMV_WBOX
+            for m in range(M):
+                xsrc = (m * nsb + col0) * 256 * 2
+                assert xsrc % 16 == 0 and xsrc + kc * 512 <= x_bytes
+                assert GEMV_COLS * GEMV_WBOX + m * 1024 + kc * 512 <= stage
+    # per-warp shared-memory reads stay inside the stage: weights (rows g and
+    # g + 8 of 8 tiles), scales, activations (column g < M)
+    for warp in range(GEMV_WARPS):
+        col, blk = warp >> 3, warp & 7
+        for g in range(8):
+            for t in range(4):
+                pa = col * GEMV_WBOX + g * 144 + blk * 16 + t * 4
+                assert pa + (16 * 7 + 8) * 144 + 4 <= (col + 1) * GEMV_WBOX
+                pd = col * GEMV_WBOX + g * 144 + 128 + blk * 2
+                assert pd + (16 * 7 + 8) * 144 + 2 <= (col + 1) * GEMV_WBOX
+                if g < M:
+                    xo = GEMV_COLS * GEMV_WBOX + g * 1024 + col * 512 + (blk * 32 + 4 * t) * 2
+                    assert xo + 32 + 8 <= stage
     # bank pattern of the A-word loads: 32 lanes (g, t) read row g, word t at a
     # 144-byte pitch
     banks = {((g * 144 + 4 * t) // 4) % 32 for g in range(8) for t in range(4)}
     assert len(banks) == 32
 
-    rows = []
-    for cta in range(p.grid_rows):
-        rb, re_ = N * cta // p.grid_rows, N * (cta + 1) // p.grid_rows
-        assert 1 <= re_ - rb <= p.rows_per_cta
-        rows.extend(range(rb, re_))
-        n_passes = -(-(re_ - rb) // R)
-        for k in range(ks):
-            for st in range(n_passes * n_chunks):
-                pss, chunk = divmod(st, n_chunks)
-                r0 = rb + pss * R
-                nr = min(R, re_ - r0)
-                assert 1 <= nr
-                assert KC * (nr * 144 + M * 512) <= TX_LIMIT
-                for j in range(KC):
-                    sb = k * p.sb_per_split + chunk * KC + j
-                    src = (sb * N + r0) * 144            # contiguous rows of column sb
-                    assert sb < nsb and src % 16 == 0 and src + nr * 144 <= w_bytes
-                    assert (sb * 256 * 2) % 16 == 0      # activation box x coordinate
-                    assert j * wbox + nr * 144 <= xoff
-                    assert xoff + (j + 1) * M * 512 <= stage
-                if chunk == n_chunks - 1:
-                    for r in (0, nr - 1):
-                        for m in range(M):
-                            assert (k * M + m) * N + r0 + r < out_len
-    assert rows == list(range(N))
 
-    # per-warp shared-memory reads stay inside the weight piece / activation box
-    for warp in range(8):
-        for t in range(4):
-            woff = 7 * 144 + warp * 16 + t * 4           # largest g
-            assert (16 * (tiles - 1) + 8) * 144 + woff + 4 <= R * 144
-            for j in range(KC):
-                xo = (j * M + (M - 1)) * 512 + (warp * 32 + 4 * t) * 2
-                assert xo + 32 + 8 <= KC * M * 512
-        doff = 7 * 144 + 128 + warp * 2
-        assert (16 * (tiles - 1) + 8) * 144 + doff + 2 <= R * 144
+@pytest.mark.parametrize("M,N,K", [(1, 17408, 5120), (3, 5120, 17408), (2, 6144, 5120),
+                                   (5, 37, 4352), (1, 300, 1280), (4, 1000, 2048)])
+def test_gemv_stream_k_sums_every_product_once(M, N, K):
+    # a model of the partition and of the last-arriver reduction: partial sums
+    # of each CTA's segments, slot by slot, rebuild the full product exactly
+    p = q4dec.plan_gemv(M, N, K, 148)
+    nsb = K // 256
+    rbs, upr, U, G = p.row_blocks, p.units_per_row_block, p.units, p.grid
+    rng = np.random.default_rng(N + K)
+    w = rng.integers(-8, 8, size=(N, K)).astype(np.float64)
+    x = rng.integers(-4, 5, size=(M, K)).astype(np.float64)
+    y = np.zeros((M, N))
+    parts = {}
+    for c in range(G):
+        a, b = _unit_begin(c, U, G), _unit_begin(c + 1, U, G)
+        u = a
+        while u < b:
+            rb = u // upr
+            seg_end = min(b, (rb + 1) * upr)
+            cols = slice(2 * (u - rb * upr) * 256, min(2 * (seg_end - rb * upr), nsb) * 256)
+            rows = slice(rb * 128, min(N, rb * 128 + 128))
+            s = x[:, cols] @ w[rows, cols].T
+            first = _unit_owner(rb * upr, U, G)
+            last = _unit_owner(rb * upr + upr - 1, U, G)
+            if first == last:
+                y[:, rows] = s
+            else:
+                assert 0 <= c - first < p.slots
+                parts.setdefault(rb, {})[c - first] = s
+            u = seg_end
+    for rb, d in parts.items():
+        assert sorted(d) == list(range(len(d)))
+        y[:, rb * 128: min(N, rb * 128 + 128)] = sum(d[k] for k in range(len(d)))
+    assert np.array_equal(y, x @ w.T)
 
 
 ATTN_CASES = [(4096, 24, 4, 1), (4096, 24, 4, 5), (65536, 24, 4, 5), (262144, 24, 4, 1),
@@ -393,18 +444,17 @@ def test_in_warp_producer_never_deadlocks(n_tiles, S):
                                  (8, 65536), (75968, 5120)])
 @pytest.mark.parametrize("sms", [148, 7])
 def test_swiglu_partition_keeps_row_pairs_together(N, K, sms):
-    # the fused variant shares out gate / up row pairs: every CTA starts on an
-    # even row and owns whole pairs, so a pass (a multiple of 16 rows from an
-    # even start) never splits a pair
-    rows = 2 * N
-    units = N
-    grid = min(sms, max(1, min(units, rows // 8)))
+    # the fused variant plans 2N rows; row blocks (128 rows) start on even rows,
+    # so a gate / up pair (rows 2n, 2n + 1) never straddles two row blocks and
+    # the final write of a block sees both rows of each of its pairs
+    p = q4dec.plan_gemv(1, 2 * N, K, sms)
+    assert p.row_blocks == -(-2 * N // 128)
     owned = []
-    for c in range(grid):
-        rb, re_ = 2 * (units * c // grid), 2 * (units * (c + 1) // grid)
-        assert rb % 2 == 0 and re_ % 2 == 0 and re_ > rb
-        owned.extend(range(rb, re_))
-    assert owned == list(range(rows))
+    for rb in range(p.row_blocks):
+        r0, r1 = rb * 128, min(2 * N, rb * 128 + 128)
+        assert r0 % 2 == 0 and (r1 - r0) % 2 == 0
+        owned.extend(range(r0 // 2, r1 // 2))
+    assert owned == list(range(N))
 
 
 @pytest.mark.parametrize("ctx,nq,nkv,M", ATTN_CASES + [(1, 4, 1, 1), (200, 48, 1, 5)])
