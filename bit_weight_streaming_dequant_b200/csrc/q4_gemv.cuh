@@ -31,23 +31,26 @@
 //    CTA numbering is rotated by the units of the jobs before it, so that
 //    over a batch those extra units land on different CTAs.
 //  * A CTA's range covers the tail of one row block, whole row blocks and the
-//    head of another.  A row block covered by one CTA is written directly; a
-//    row block shared by several CTAs is finished by the last contributor to
-//    arrive: each writes its partial sums into its own slot of the workspace
-//    and counts itself in on the row block's counter; the last one adds the
-//    slots in slot (K) order -- the result does not depend on arrival order --
-//    and resets the counter to zero.  Counters carry the launch's 48-bit tag
-//    next to their 16-bit count: a counter holding another tag (left over by
-//    another use of the memory) counts as zero, so the workspace needs no
-//    clearing, and the resets keep replays of a captured launch (same tag)
-//    correct.
+//    head of another.  A row block covered by one CTA is written directly.  A
+//    row block shared by several CTAs has one slot of partial sums per
+//    contributor, in K order; slot 0 belongs to the CTA whose range ends in
+//    the row block, which reaches it last (the others reach it at the start
+//    of their ranges or cover nothing else), so that CTA finishes it: the
+//    others write their slots and raise the slot's flag (a release store of
+//    the launch's 48-bit tag, no round trip); the finisher waits for the
+//    flags, adds the slots in slot order -- its own from registers -- writes
+//    the rows and lowers the flags again.  A flag holding another value (left
+//    over by another use of the memory) counts as down, so the workspace needs
+//    no clearing, and lowering them keeps replays of a captured launch (same
+//    tag) correct.
 //  * Several matrices ("jobs") can run in one launch.  The producer keeps
 //    streaming the next job's weights (they depend on nothing) while a job's
-//    activations wait for the job they depend on: each CTA counts itself in on
-//    a per-job counter when it has finished that job, and a job's activation
-//    copies are issued only once its prerequisite's counter is complete.  These
-//    counters live in the launch descriptor, which the host hands over zeroed;
-//    the last CTA to leave the launch sets them back to zero.
+//    activations wait for the job they depend on: whoever writes a row block's
+//    final values counts it on a per-job counter, and a job's activation
+//    copies are issued only once its prerequisite's count has reached that
+//    job's number of row blocks.  These counters live in the launch
+//    descriptor, which the host hands over zeroed; the last CTA to leave the
+//    launch sets them back to zero.
 //  * Weights are stored super-block-column-major: the 128 rows of a row block
 //    are one contiguous piece of each column, so a unit is two bulk copies of
 //    18 KB plus one copy of each activation row's 1 KB, issued by a producer
@@ -56,10 +59,10 @@
 //    it on an "empty" mbarrier.  At the end of each row block segment they add
 //    their 16 partial sums in a fixed order through shared memory into one of
 //    four segment buffers and go on with the next stage; two epilogue warps,
-//    taking alternate segments, write them out (y, or the partial slot and,
-//    when last, the sum of the slots), publish them with one release fence
-//    each and count the CTA in for a job once both have written all of its
-//    segments, so no global write, fence or atomic stalls the consumers.
+//    taking alternate segments, write them out (y, or the partial slot, or
+//    the sum of the slots), publish them with one release fence each and count
+//    finished row blocks for their job, so no global write, fence or atomic
+//    stalls the consumers.
 //  * Every wait is bounded in time.  A wait that runs out sets the device
 //    error word and a per-CTA abort flag; from then on no wait blocks, the
 //    producer issues no further copies and waits for the ones in flight, and
@@ -85,7 +88,7 @@ constexpr int kGemvRows = 16 * kGemvTiles;                 // 128 weight rows
 constexpr int kGemvCols = 2;                               // super-block columns per unit
 constexpr int kGemvConsumerWarps = 8 * kGemvCols;          // one (column, block) task each
 constexpr int kGemvProducerWarp = kGemvConsumerWarps;      // bulk copies
-constexpr int kGemvEpilogueWarps = 2;                      // output writes, counters
+constexpr int kGemvEpilogueWarps = 2;                      // output writes, flags, counts
 constexpr int kGemvThreads = (kGemvConsumerWarps + 1 + kGemvEpilogueWarps) * 32;
 constexpr int kGemvSegBufs = 4;                            // segment buffers (consumers -> epilogue)
 constexpr int kGemvMaxStages = 8;
@@ -107,9 +110,8 @@ __host__ __device__ constexpr uint32_t gemv_red_bytes(int M) {
 __host__ __device__ constexpr uint32_t gemv_fin_bytes(int M) {
   return uint32_t(kGemvSegBufs) * uint32_t(M) * kGemvRows * 4u;
 }
-// Shared memory: ring, reduction buffer, segment buffers, flags (abort, two
-// epilogue progress counts; padded to 16), 2 barriers per stage and 2 per
-// segment buffer.
+// Shared memory: ring, reduction buffer, segment buffers, the abort flag
+// (padded to 16), 2 barriers per stage and 2 per segment buffer.
 __host__ __device__ constexpr size_t gemv_smem_bytes(int M, int stages) {
   return size_t(stages) * gemv_stage_bytes(M) + gemv_red_bytes(M) + gemv_fin_bytes(M) + 16 +
          size_t(stages) * 16 + size_t(kGemvSegBufs) * 16;
@@ -141,18 +143,18 @@ struct alignas(16) GemvJobDesc {
   int units;             // rbs * upr
   int grid;              // CTAs that work on this job (min(launch grid, units))
   int slots;             // partial slots per row block (0: no row block is shared)
-  int cnt_off;           // this job's row-block counters: index into the counter area
+  int flag_off;          // this job's slot flags ([rbs][slots]): index into the flag area
   int rot;               // job-local CTA index = (blockIdx.x + rot) mod launch grid
   int pad_;
 };
 
 struct GemvArgs {
   const GemvJobDesc* jobs;        // device array of n_jobs descriptors, or null: `job` below
-  unsigned* sync;                 // [n_jobs] jobs finished by all CTAs, [1] CTAs gone (zeroed)
-  unsigned long long* counters;   // workspace: row-block counters (tagged)
+  unsigned* sync;                 // [n_jobs] row blocks finished per job, [1] CTAs gone (zeroed)
+  unsigned long long* flags;      // workspace: partial-slot flags (tag = raised)
   float* partials;                // workspace: partial slots
   unsigned* err;                  // device error word
-  unsigned long long tag;         // this launch's counter tag (48 bits, non-zero)
+  unsigned long long tag;         // this launch's flag value (48 bits, non-zero)
   int n_jobs;
   int grid;                       // CTAs of the launch
   int stages;                     // ring stages
@@ -160,22 +162,24 @@ struct GemvArgs {
   GemvJobDesc job;                // the single job of a one-matrix launch
 };
 
-// Count one arrival on a tagged counter (tag in bits 16..63, count in 0..15;
-// a counter with another tag counts as zero).  Returns the count after it.
-__device__ __forceinline__ unsigned tagged_arrive(unsigned long long* w, unsigned long long tag) {
-  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(w);
-  for (;;) {
-    const unsigned long long nw = ((old >> 16) == tag) ? old + 1ull : ((tag << 16) | 1ull);
-    const unsigned long long prev = atomicCAS(w, old, nw);
-    if (prev == old) return unsigned(nw & 0xFFFFull);
-    old = prev;
-  }
-}
-
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_release_gpu_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ void fence_acq_rel_gpu() {
@@ -248,6 +252,7 @@ struct UnitCursor {
   const uint8_t* W;
   const uint16_t* x;
   int N, nsb, upr, wait_for;
+  unsigned wait_rbs;  // row blocks of job wait_for (its count once finished)
 };
 
 __device__ __forceinline__ void cursor_enter(UnitCursor& c, const GemvArgs& a, int i) {
@@ -265,6 +270,7 @@ __device__ __forceinline__ void cursor_enter(UnitCursor& c, const GemvArgs& a, i
     c.nsb = J->nsb;
     c.upr = J->upr;
     c.wait_for = J->wait_for;
+    c.wait_rbs = c.wait_for >= 0 ? unsigned(gemv_job(a, c.wait_for)->rbs) : 0u;
     break;
   }
   c.job = i;
@@ -351,17 +357,19 @@ __device__ __forceinline__ void gemv_segment_reduce(float* red, float* fin,
 }
 
 // End of a row block segment, epilogue side (one warp): write the row block
-// (covered by this CTA alone), or this CTA's partial slot and, if it is the
-// last contributor to arrive, the sum of all slots in slot order.  The
-// segment buffer is released as soon as it has been read.
+// (covered by this CTA alone); or, in a shared row block, publish this CTA's
+// slot (slots 1, 2, ...), or finish the row block (slot 0): wait for the other
+// slots' flags, add the slots in slot order and write the rows.  The segment
+// buffer is released as soon as it has been read.  Returns whether this warp
+// wrote the row block's final values.
 template <int M>
-__device__ __forceinline__ void gemv_segment_write(const GemvArgs& a, const GemvJobDesc* J, int cj,
+__device__ __forceinline__ bool gemv_segment_write(const GemvArgs& a, const GemvJobDesc* J, int cj,
                                                    int rb, const float* fin, uint64_t* fin_empty,
-                                                   int lane) {
+                                                   int lane, volatile int* abort_flag) {
   const int G = J->grid, first_u = rb * J->upr;
   const int c_first = unit_owner(first_u, J->units, G);
   const int c_last = unit_owner(first_u + J->upr - 1, J->units, G);
-  const int n_contrib = c_last - c_first + 1;
+  const int n_contrib = c_last - c_first + 1, my = cj - c_first;
   float v[4 * M];
   #pragma unroll
   for (int k = 0; k < 4 * M; ++k) v[k] = fin[lane + 32 * k];
@@ -369,38 +377,50 @@ __device__ __forceinline__ void gemv_segment_write(const GemvArgs& a, const Gemv
   if (lane == 0) mbar_arrive(smem_addr(fin_empty));  // the segment buffer is free again
   if (n_contrib == 1) {
     gemv_store_rows<M>(J, rb, lane, v);
-    return;
+    return true;
   }
-  // this CTA's partial sums into its slot ([M][128] floats; rows past N unused)
+  // slot sl of the row block: [M][128] floats (rows past N unused)
   float* part = a.partials + J->part_off + size_t(rb) * J->slots * M * kGemvRows;
-  float* mine = part + size_t(cj - c_first) * M * kGemvRows;
-  #pragma unroll
-  for (int k = 0; k < 4 * M; ++k) mine[lane + 32 * k] = v[k];
-  __syncwarp();
-  int last = 0;
-  if (lane == 0) {
-    fence_acq_rel_gpu();  // this slot's writes (all lanes, ordered by the warp barrier) first
-    unsigned long long* cnt = a.counters + J->cnt_off + rb;
-    last = tagged_arrive(cnt, a.tag) == unsigned(n_contrib);
-    if (last) {
-      *cnt = 0ull;  // every contributor has counted itself in: ready for a replay
-      fence_acq_rel_gpu();  // the other slots' writes become visible to this warp
-    }
+  unsigned long long* flag = a.flags + J->flag_off + size_t(rb) * J->slots;
+  if (my != 0) {
+    float* mine = part + size_t(my) * M * kGemvRows;
+    #pragma unroll
+    for (int k = 0; k < 4 * M; ++k) mine[lane + 32 * k] = v[k];
+    __syncwarp();
+    // the slot's writes (all lanes, ordered by the warp barrier) before its flag
+    if (lane == 0) st_release_gpu_u64(flag + my, a.tag);
+    return false;
   }
-  last = __shfl_sync(0xFFFFFFFFu, last, 0);
-  if (!last) return;
-  // the last contributor: every slot's values first (all loads in flight),
-  // added in slot order, then the stores
+  // The finisher: every lane acquires every other slot's flag (bounded wait).
+  const unsigned long long t0 = global_timer_ns();
+  for (;;) {
+    bool up = true;
+    for (int sl = 1; sl < n_contrib; ++sl) up &= ld_acquire_gpu_u64(flag + sl) == a.tag;
+    if (__all_sync(0xFFFFFFFFu, up) || *abort_flag) break;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (lane == 0) {
+        *abort_flag = 1;
+        atomicOr(a.err, kDevErrWaitTimeout);
+      }
+      break;
+    }
+    __nanosleep(32);
+  }
+  // slot 0 (this CTA's, from registers), then the others in order
   #pragma unroll
-  for (int k = 0; k < 4 * M; ++k) v[k] = 0.f;
-  for (int sl = 0; sl < n_contrib; ++sl) {
+  for (int k = 0; k < 4 * M; ++k) v[k] = 0.f + v[k];
+  for (int sl = 1; sl < n_contrib; ++sl) {
     float w[4 * M];
     #pragma unroll
     for (int k = 0; k < 4 * M; ++k) w[k] = __ldcg(part + size_t(sl) * M * kGemvRows + lane + 32 * k);
     #pragma unroll
     for (int k = 0; k < 4 * M; ++k) v[k] += w[k];
   }
+  // lower the flags for the next launch with this tag (a replay); that launch
+  // starts only after this one has ended
+  for (int sl = 1 + lane; sl < n_contrib; sl += 32) flag[sl] = 0ull;
   gemv_store_rows<M>(J, rb, lane, v);
+  return true;
 }
 
 template <int M>
@@ -414,7 +434,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
   float* red = reinterpret_cast<float*>(smem + size_t(S) * kStage);
   float* fin = red + gemv_red_bytes(M) / 4;                       // [4][M][128]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(fin + kGemvSegBufs * M * kGemvRows);
-  volatile int* epi_done = abort_flag + 1;                        // [2] segments written per epilogue warp
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(S) * kStage + gemv_red_bytes(M) +
                                                gemv_fin_bytes(M) + 16);
   uint64_t* empty = full + S;
@@ -432,8 +451,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
       mbar_init(smem_addr(&fin_empty[b]), 1);
     }
     *abort_flag = 0;
-    epi_done[0] = 0;
-    epi_done[1] = 0;
     mbar_init_fence();
   }
   __syncthreads();
@@ -460,7 +477,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
         }
         ready = true;
       } else {
-        ready = ld_acquire_gpu(a.sync + xs.wait_for) >= unsigned(a.grid);
+        ready = ld_acquire_gpu(a.sync + xs.wait_for) >= xs.wait_rbs;
       }
       if (ready) {
         fence_proxy_async_global();
@@ -550,61 +567,39 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
 
   if (warp > kGemvProducerWarp) {
     // ------------------------------ epilogue ------------------------------
-    // Warp e writes segments e, e + 2, ...; the warp writing a job's last
-    // segment in this CTA waits until the other warp has written the job's
-    // earlier ones, then counts the CTA in for the job.  Nothing of the
-    // workspace or the outputs is touched before the previous kernel on the
-    // stream is complete (it may still use the same buffers).
+    // Warp e writes segments e, e + 2, ...; each row block it finishes is
+    // counted for its job (after a release fence, so that a CTA which sees the
+    // count complete also sees the rows).  Nothing of the workspace or the
+    // outputs is touched before the previous kernel on the stream is complete
+    // (it may still use the same buffers).
     griddep_wait();
-    const int e = warp - kGemvProducerWarp - 1, o = 1 - e;
-    // other warp's segments among [0, s): o, o + 2, ...
-    auto other_written = [&](int s_end) {
-      const int need = (s_end + 1 - o) / 2;
-      const unsigned long long t0 = global_timer_ns();
-      while (epi_done[o] < need && !*abort_flag) {
-        __nanosleep(64);
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-          *abort_flag = 1;
-          atomicOr(a.err, kDevErrWaitTimeout);
-        }
-      }
-    };
-    int seg = 0, mine = 0;
+    const int e = warp - kGemvProducerWarp - 1;
+    int seg = 0;
     for (int job = 0; job < a.n_jobs; ++job) {
       const GemvJobDesc* J = gemv_job(a, job);
       const JobRange r = job_range(a, J);
-      int last_seg_writer = 0;  // jobs without units here: warp 0 counts the CTA in
       for (int u = r.ub; u < r.ue;) {
         const int rb = u / J->upr;
         const int u_end = min(r.ue, (rb + 1) * J->upr);
         if ((seg & 1) == e) {
           const int b = seg & (kGemvSegBufs - 1);
           gemv_wait(smem_addr(&fin_full[b]), uint32_t(seg >> 2) & 1u, a.err, abort_flag);
-          gemv_segment_write<M>(a, J, r.cj, rb, fin + b * M * kGemvRows, &fin_empty[b], lane);
-          __syncwarp();
-          if (lane == 0) {
-            fence_acq_rel_gpu();  // this warp's writes before its progress count
-            epi_done[e] = ++mine;
+          const bool wrote = gemv_segment_write<M>(a, J, r.cj, rb, fin + b * M * kGemvRows,
+                                                   &fin_empty[b], lane, abort_flag);
+          if (wrote && a.n_jobs > 1) {
+            __syncwarp();
+            if (lane == 0) red_release_gpu_add(a.sync + job, 1u);
           }
-          __syncwarp();
         }
-        last_seg_writer = seg & 1;
         ++seg;
         u = u_end;
       }
-      if (a.n_jobs > 1 && last_seg_writer == e) {
-        if (lane == 0) {
-          other_written(seg);
-          fence_acq_rel_gpu();
-          atomicAdd(a.sync + job, 1u);
-        }
-        __syncwarp();
-      }
     }
-    if (a.n_jobs > 1 && e == 0 && lane == 0) {
-      // the last CTA to leave sets the per-job counters back to zero
-      other_written(seg);
-      if (atomicAdd(a.sync + a.n_jobs, 1u) == unsigned(a.grid - 1)) {
+    if (a.n_jobs > 1) {
+      // both epilogue warps are done; the last CTA to leave sets the per-job
+      // counts back to zero (every count of every CTA is in by then)
+      asm volatile("bar.sync 2, %0;" ::"n"(kGemvEpilogueWarps * 32) : "memory");
+      if (e == 0 && lane == 0 && atomicAdd(a.sync + a.n_jobs, 1u) == unsigned(a.grid - 1)) {
         fence_acq_rel_gpu();
         for (int i = 0; i <= a.n_jobs; ++i) a.sync[i] = 0u;
       }

@@ -185,7 +185,7 @@ int gemv_stages(int M, size_t smem_limit) {
   return stages;
 }
 
-constexpr size_t kGemvCounterBytes = 8;   // one tagged counter
+constexpr size_t kGemvFlagBytes = 8;      // one partial-slot flag
 constexpr int kSmemOptinB200 = 232448;    // planning default: B200's opt-in shared memory
 
 size_t round_up16(size_t v) { return (v + 15) / 16 * 16; }
@@ -206,9 +206,9 @@ q4d_status plan_gemv_rows(int M, int rows, int K, int num_sms, int smem_optin,
   plan->stages = gemv_stages(M, size_t(smem_optin));
   plan->reserved = 0;
   plan->smem_bytes = q4d::gemv_smem_bytes(M, plan->stages);
-  // row-block counters (8 bytes each), then the partial slots
+  // slot flags (8 bytes per row block and slot), then the partial slots
   plan->workspace_bytes =
-      j.slots > 0 ? round_up16(size_t(j.rbs) * kGemvCounterBytes) +
+      j.slots > 0 ? round_up16(size_t(j.rbs) * j.slots * kGemvFlagBytes) +
                         size_t(j.rbs) * j.slots * M * q4d::kGemvRows * 4
                   : 0;
   return Q4D_OK;
@@ -216,8 +216,7 @@ q4d_status plan_gemv_rows(int M, int rows, int K, int num_sms, int smem_optin,
 
 std::atomic<unsigned long long> g_gemv_tag{0};
 
-// A fresh 48-bit counter tag for every launch (never 0: zeroed memory means
-// "no arrival yet").
+// A fresh 48-bit flag value for every launch (never 0: a lowered flag is 0).
 unsigned long long next_gemv_tag() {
   unsigned long long t = (g_gemv_tag.fetch_add(1, std::memory_order_relaxed) + 1) &
                          ((1ull << 48) - 1);
@@ -293,9 +292,10 @@ q4d_status gemv_impl(const void* W_q4, const void* x, void* y, int M, int N, int
   a.err = s->err;
   a.tag = next_gemv_tag();
   if (p.workspace_bytes > 0) {
-    a.counters = static_cast<unsigned long long*>(workspace);
-    a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                          round_up16(size_t(p.row_blocks) * kGemvCounterBytes));
+    a.flags = static_cast<unsigned long long*>(workspace);
+    a.partials = reinterpret_cast<float*>(
+        static_cast<uint8_t*>(workspace) +
+        round_up16(size_t(p.row_blocks) * p.slots * kGemvFlagBytes));
   }
   q4d::GemvJobDesc& J = a.job;
   J.W = static_cast<const uint8_t*>(W_q4);
@@ -311,7 +311,7 @@ q4d_status gemv_impl(const void* W_q4, const void* x, void* y, int M, int N, int
   J.units = p.units;
   J.grid = p.grid;
   J.slots = p.slots;
-  J.cnt_off = 0;
+  J.flag_off = 0;
   J.rot = 0;
   if ((st = launch_gemv(M, a, p.smem_bytes, dev, *s, stream, pdl)) != Q4D_OK) return st;
   if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
@@ -572,7 +572,7 @@ struct BatchHeader {
   int n_jobs, M, num_sms, grid;
   int pad_;
   size_t workspace_bytes;
-  size_t counter_bytes;
+  size_t flag_bytes;
 };
 static_assert(sizeof(BatchHeader) <= kBatchHeader, "batch header");
 static_assert(sizeof(q4d::GemvJobDesc) % 16 == 0, "job descriptor alignment");
@@ -616,7 +616,7 @@ q4d_status q4d_gemv_batch_prepare(const q4d_gemv_job* jobs, int n_jobs, int M, i
   }
   q4d::GemvJobDesc* out =
       reinterpret_cast<q4d::GemvJobDesc*>(static_cast<uint8_t*>(desc) + kBatchHeader);
-  size_t counters = 0;  // tagged row-block counters
+  size_t flags = 0;     // partial-slot flags
   size_t partials = 0;  // floats
   long long units_before = 0;  // rotates each job's CTA numbering (balance across the batch)
   for (int i = 0; i < n_jobs; ++i) {
@@ -639,12 +639,13 @@ q4d_status q4d_gemv_batch_prepare(const q4d_gemv_job* jobs, int n_jobs, int M, i
     d.units = sh.units;
     d.grid = sh.grid;
     d.slots = sh.slots;
-    d.cnt_off = int(counters);
+    if (flags > size_t(1 << 30)) return Q4D_ERR_UNSUPPORTED_SHAPE;
+    d.flag_off = int(flags);
     d.part_off = (long long)partials;
     d.rot = int(units_before % grid);
     units_before += sh.units;
     if (sh.slots > 0) {
-      counters += size_t(sh.rbs);
+      flags += size_t(sh.rbs) * sh.slots;
       partials += size_t(sh.rbs) * sh.slots * M * q4d::kGemvRows;
     }
     std::memcpy(out + i, &d, sizeof(d));
@@ -656,8 +657,8 @@ q4d_status q4d_gemv_batch_prepare(const q4d_gemv_job* jobs, int n_jobs, int M, i
   h.M = M;
   h.num_sms = num_sms;
   h.grid = grid;
-  h.counter_bytes = round_up16(counters * kGemvCounterBytes);
-  h.workspace_bytes = h.counter_bytes + partials * 4;
+  h.flag_bytes = round_up16(flags * kGemvFlagBytes);
+  h.workspace_bytes = h.flag_bytes + partials * 4;
   std::memset(desc, 0, kBatchHeader);
   std::memcpy(desc, &h, sizeof(h));
   std::memset(static_cast<uint8_t*>(desc) + batch_sync_offset(n_jobs), 0,
@@ -695,8 +696,8 @@ q4d_status q4_gemv_batch_ex(const void* desc_host, void* desc_dev, void* stream,
   a.stages = stages;
   a.err = s->err;
   a.tag = next_gemv_tag();
-  a.counters = static_cast<unsigned long long*>(workspace);
-  a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + h.counter_bytes);
+  a.flags = static_cast<unsigned long long*>(workspace);
+  a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + h.flag_bytes);
   if ((st = launch_gemv(h.M, a, q4d::gemv_smem_bytes(h.M, stages), dev, *s,
                         static_cast<cudaStream_t>(stream), (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0)) !=
       Q4D_OK)

@@ -106,12 +106,14 @@ const char* q4d_status_string(int status);
  *
  * Partition (q4d_plan_gemv): rows are cut into blocks of 128 and K into units
  * of 512 elements; the units are shared out in equal contiguous ranges over
- * one CTA per SM, so a row block may be summed by several CTAs.  Those CTAs
- * write fp32 partial sums into the workspace and the last one to finish adds
- * them in a fixed order, so results are deterministic.  The workspace holds
- * small counters besides the partial sums; it needs no initialisation (its
- * previous contents are ignored), but calls whose kernels may overlap on the
- * GPU must not share one workspace.
+ * one CTA per SM, so a row block may be summed by several CTAs.  All but
+ * one of them write fp32 partial sums into the workspace and raise a flag;
+ * the CTA whose range ends in the row block waits for the flags and adds the
+ * partial sums in a fixed (K) order, so results are deterministic.  The
+ * workspace holds the flags (8 bytes per row block and slot) besides the
+ * partial sums; it needs no initialisation (its previous contents are
+ * ignored), but calls whose kernels may overlap on the GPU must not share
+ * one workspace.
  */
 q4d_status q4_gemv(const void* W_q4, const void* x, float* y, int M, int N, int K);
 q4d_status q4_gemv_ex(const void* W_q4, const void* x, float* y, int M, int N, int K,
@@ -199,8 +201,9 @@ size_t q4d_gemv_workspace_bytes(int M, int N, int K);
  *   q4_gemv_batch_ex: launches the batch on `stream`.  desc_host is the
  *     prepared host buffer, desc_dev a byte-for-byte copy of it in device
  *     memory (16-byte aligned): copy it once, launch many times.  Its tail
- *     holds the per-job completion counters, zero as prepared; a launch counts
- *     on them and sets them back to zero before it ends, so launches that may
+ *     holds the per-job completion counters (row blocks written), zero as
+ *     prepared; a launch counts on them and sets them back to zero before it
+ *     ends, so launches that may
  *     overlap on the GPU must not share a descriptor copy, and a copy must not
  *     be rewritten while a launch may run.  num_sms
  *     must be the current device's SM count, else Q4D_ERR_INVALID_ARG.
