@@ -578,7 +578,8 @@ class DecodeStep:
         self.batch = q4dec.GemvBatch(jobs)
         self.aws = self.L.q4d_attn_workspace_bytes(CTX, N_Q, N_KV, HEAD_DIM, M)
         self.attn_ws = torch.empty(max(self.aws, 16), dtype=torch.uint8, device=dev)
-        self.gemv_ws = torch.empty(max(16, max(self.L.q4d_gemv_workspace_bytes(M, N, K)
+        # GEMV workspace: zero-filled once, every launch leaves it so
+        self.gemv_ws = torch.zeros(max(16, max(self.L.q4d_gemv_workspace_bytes(M, N, K)
                                                for N, K in LAYER_SHAPES + [(HEAD_N, HIDDEN)])),
                                    dtype=torch.uint8, device=dev)
         self.launches = 0
@@ -659,9 +660,10 @@ def per_call_table(torch, L, dev, layers, kv, peak_gbs, reps=15):
             flush_buf.sum()
 
     flush = _Flush()
-    need = max([L.q4d_gemv_workspace_bytes(M, N, K) for M in range(1, 6)
-                for N, K in LAYER_SHAPES] +
-               [L.q4d_attn_workspace_bytes(c, N_Q, N_KV, HEAD_DIM, M) for M in (1, 5)
+    gemv_need = max([L.q4d_gemv_workspace_bytes(M, N, K) for M in range(1, 6)
+                     for N, K in LAYER_SHAPES] + [16])
+    gemv_ws = torch.zeros(gemv_need, dtype=torch.uint8, device=dev)  # kept zero by the GEMV
+    need = max([L.q4d_attn_workspace_bytes(c, N_Q, N_KV, HEAD_DIM, M) for M in (1, 5)
                 for c in (4096, 65536, CTX)] +
                [L.q8kv_attn_workspace_bytes(c, N_Q, N_KV, HEAD_DIM, M) for M in (1, 5)
                 for c in (65536, CTX)] + [16])
@@ -683,7 +685,7 @@ def per_call_table(torch, L, dev, layers, kv, peak_gbs, reps=15):
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
                 st = L.q4_gemv_ex(W.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K, sptr,
-                                  ws.data_ptr(), ws.numel())
+                                  gemv_ws.data_ptr(), gemv_ws.numel())
                 b.record(stream)
                 if st:
                     raise RuntimeError(f"q4_gemv_ex failed: {st}")
@@ -843,7 +845,7 @@ def run_case(args, torch, dev):
         Ws = [synth.device_q4_0_weights(50 + i, N, K, device=dev) for i in range(copies)]
         x = synth.device_bf16_normal(1, (M, K), device=dev)
         y = torch.empty((M, N), dtype=torch.float32, device=dev)
-        ws = torch.empty(max(16, L.q4d_gemv_workspace_bytes(M, N, K)), dtype=torch.uint8,
+        ws = torch.zeros(max(16, L.q4d_gemv_workspace_bytes(M, N, K)), dtype=torch.uint8,
                          device=dev)
         for i in range(args.launches):
             W = Ws[i % copies]

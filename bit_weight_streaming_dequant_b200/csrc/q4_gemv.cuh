@@ -35,14 +35,16 @@
 //    row block shared by several CTAs has one slot of partial sums per
 //    contributor, in K order; slot 0 belongs to the CTA whose range ends in
 //    the row block, which reaches it last (the others reach it at the start
-//    of their ranges or cover nothing else), so that CTA finishes it: the
-//    others write their slots and raise the slot's flag (a release store of
-//    the launch's 48-bit tag, no round trip); the finisher waits for the
-//    flags, adds the slots in slot order -- its own from registers -- writes
-//    the rows and lowers the flags again.  A flag holding another value (left
-//    over by another use of the memory) counts as down, so the workspace needs
-//    no clearing, and lowering them keeps replays of a captured launch (same
-//    tag) correct.
+//    of their ranges or cover nothing else), so that CTA finishes it.  The
+//    others write their slots, each entry one 64-bit word holding the fp32
+//    value and the launch's 32-bit tag, so an entry is valid exactly when it
+//    carries the tag (no flag, no fence, no round trip); the finisher reads
+//    the entries until they are valid -- those of a partner that finished
+//    early are read while its own sums are still being made -- adds the slots
+//    in slot order, its own from registers, writes the rows and clears the
+//    entries.  An entry holding another value (left over by another use of
+//    the memory) is not valid, so the workspace needs no clearing, and the
+//    clearing keeps replays of a captured launch (same tag) correct.
 //  * Several matrices ("jobs") can run in one launch.  The producer keeps
 //    streaming the next job's weights (they depend on nothing) while a job's
 //    activations wait for the job they depend on: whoever writes a row block's
@@ -59,10 +61,10 @@
 //    it on an "empty" mbarrier.  At the end of each row block segment they add
 //    their 16 partial sums in a fixed order through shared memory into one of
 //    four segment buffers and go on with the next stage; two epilogue warps,
-//    taking alternate segments, write them out (y, or the partial slot, or
-//    the sum of the slots), publish them with one release fence each and count
-//    finished row blocks for their job, so no global write, fence or atomic
-//    stalls the consumers.
+//    each taking one half (64 rows) of every segment, write them out (y, the
+//    partial slot, or the sum of the slots) and count the halves written in
+//    final form for their job, so no global write or atomic stalls the
+//    consumers.
 //  * Every wait is bounded in time.  A wait that runs out sets the device
 //    error word and a per-CTA abort flag; from then on no wait blocks, the
 //    producer issues no further copies and waits for the ones in flight, and
@@ -143,7 +145,7 @@ struct alignas(16) GemvJobDesc {
   int units;             // rbs * upr
   int grid;              // CTAs that work on this job (min(launch grid, units))
   int slots;             // partial slots per row block (0: no row block is shared)
-  int flag_off;          // this job's slot flags ([rbs][slots]): index into the flag area
+  int pad0_;
   int rot;               // job-local CTA index = (blockIdx.x + rot) mod launch grid
   int pad_;
 };
@@ -151,10 +153,9 @@ struct alignas(16) GemvJobDesc {
 struct GemvArgs {
   const GemvJobDesc* jobs;        // device array of n_jobs descriptors, or null: `job` below
   unsigned* sync;                 // [n_jobs] row blocks finished per job, [1] CTAs gone (zeroed)
-  unsigned long long* flags;      // workspace: partial-slot flags (tag = raised)
-  float* partials;                // workspace: partial slots
+  unsigned long long* partials;   // workspace: partial slots of {fp32 value, tag} entries
   unsigned* err;                  // device error word
-  unsigned long long tag;         // this launch's flag value (48 bits, non-zero)
+  unsigned long long tag;         // this launch's tag (low 32 bits non-zero)
   int n_jobs;
   int grid;                       // CTAs of the launch
   int stages;                     // ring stages
@@ -174,8 +175,19 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned 
   return v;
 }
 
-__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+__device__ __forceinline__ void st_relaxed_gpu_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// A partial-slot entry: the fp32 value's bits, the launch tag above them.
+__device__ __forceinline__ unsigned long long slot_entry(float v, unsigned tag32) {
+  return (static_cast<unsigned long long>(tag32) << 32) | __float_as_uint(v);
 }
 
 __device__ __forceinline__ void red_release_gpu_add(unsigned* p, unsigned v) {
@@ -252,7 +264,7 @@ struct UnitCursor {
   const uint8_t* W;
   const uint16_t* x;
   int N, nsb, upr, wait_for;
-  unsigned wait_rbs;  // row blocks of job wait_for (its count once finished)
+  unsigned wait_rbs;  // count of job wait_for once finished (row-block halves)
 };
 
 __device__ __forceinline__ void cursor_enter(UnitCursor& c, const GemvArgs& a, int i) {
@@ -270,7 +282,7 @@ __device__ __forceinline__ void cursor_enter(UnitCursor& c, const GemvArgs& a, i
     c.nsb = J->nsb;
     c.upr = J->upr;
     c.wait_for = J->wait_for;
-    c.wait_rbs = c.wait_for >= 0 ? unsigned(gemv_job(a, c.wait_for)->rbs) : 0u;
+    c.wait_rbs = c.wait_for >= 0 ? unsigned(kGemvEpilogueWarps * gemv_job(a, c.wait_for)->rbs) : 0u;
     break;
   }
   c.job = i;
@@ -285,20 +297,26 @@ __device__ __forceinline__ void cursor_next(UnitCursor& c, const GemvArgs& a) {
   }
 }
 
-// The rows of a row block, fully summed, given as `v` (element i = m * 128 +
-// r; lane L holds elements L, L + 32, ...): write y (or, for gate / up pairs,
-// h = silu(g) * u, pairing rows 2j and 2j + 1 across lanes).
+// Element k of lane `lane` in epilogue warp e's half of a segment: column
+// m = k / 2 of the [M][128] layout, row r = 64 e + 32 (k % 2) + lane.
+__device__ __forceinline__ int seg_row(int e, int lane, int k) { return 64 * e + 32 * (k & 1) + lane; }
+__device__ __forceinline__ int seg_index(int e, int lane, int k) {
+  return (k >> 1) * kGemvRows + seg_row(e, lane, k);
+}
+
+// Epilogue warp e's half of a row block, fully summed (v[k]: element k as
+// above): write y (or, for gate / up pairs, h = silu(g) * u, pairing rows 2j
+// and 2j + 1, held by neighbouring lanes).
 template <int M>
-__device__ __forceinline__ void gemv_store_rows(const GemvJobDesc* J, int rb, int lane,
-                                                const float (&v)[4 * M]) {
+__device__ __forceinline__ void gemv_store_rows(const GemvJobDesc* J, int rb, int e, int lane,
+                                                const float (&v)[2 * M]) {
   const bool bf16 = (J->flags & kJobOutBf16) != 0;
   const int r0 = rb * kGemvRows;
   if (J->flags & kJobSwiglu) {
     const int n_out = J->N >> 1;
     #pragma unroll
-    for (int k = 0; k < 4 * M; ++k) {
-      const int i = lane + 32 * k, m = i >> 7, r = i & 127;
-      // rows 2j (even lane) and 2j + 1 (the next lane) of the same column
+    for (int k = 0; k < 2 * M; ++k) {
+      const int m = k >> 1, r = seg_row(e, lane, k);
       const float other = __shfl_down_sync(0xFFFFFFFFu, v[k], 1);
       if ((r & 1) == 0 && r0 + r + 1 < J->N)
         store_out(J->y, size_t(m) * n_out + ((r0 + r) >> 1), v[k] / (1.f + expf(-v[k])) * other,
@@ -306,8 +324,8 @@ __device__ __forceinline__ void gemv_store_rows(const GemvJobDesc* J, int rb, in
     }
   } else {
     #pragma unroll
-    for (int k = 0; k < 4 * M; ++k) {
-      const int i = lane + 32 * k, m = i >> 7, r = i & 127;
+    for (int k = 0; k < 2 * M; ++k) {
+      const int m = k >> 1, r = seg_row(e, lane, k);
       if (r0 + r < J->N) store_out(J->y, size_t(m) * J->N + r0 + r, v[k], bf16);
     }
   }
@@ -356,70 +374,104 @@ __device__ __forceinline__ void gemv_segment_reduce(float* red, float* fin,
   gemv_consumer_sync();
 }
 
-// End of a row block segment, epilogue side (one warp): write the row block
-// (covered by this CTA alone); or, in a shared row block, publish this CTA's
-// slot (slots 1, 2, ...), or finish the row block (slot 0): wait for the other
-// slots' flags, add the slots in slot order and write the rows.  The segment
-// buffer is released as soon as it has been read.  Returns whether this warp
-// wrote the row block's final values.
+// Who shares row block rb of job J, and this CTA's slot among them.
+struct RowBlockShare {
+  int n, my;
+};
+__device__ __forceinline__ RowBlockShare row_block_share(const GemvJobDesc* J, int cj, int rb) {
+  const int first_u = rb * J->upr;
+  const int c_first = unit_owner(first_u, J->units, J->grid);
+  const int c_last = unit_owner(first_u + J->upr - 1, J->units, J->grid);
+  return RowBlockShare{c_last - c_first + 1, cj - c_first};
+}
+
+// Entries of slot sl of row block rb ([M][128]; rows past N unused).
+template <int M>
+__device__ __forceinline__ unsigned long long* slot_entries(const GemvArgs& a,
+                                                            const GemvJobDesc* J, int rb, int sl) {
+  return a.partials + J->part_off + (size_t(rb) * J->slots + sl) * M * kGemvRows;
+}
+
+// Read this lane's entries (epilogue warp e's half) of a slot if they are all
+// valid (tag): values into w.  Returns false (w unspecified) if any is not yet
+// written.
+template <int M>
+__device__ __forceinline__ bool read_slot(const unsigned long long* s_e, int e, int lane,
+                                          unsigned tag32, float (&w)[2 * M]) {
+  unsigned long long r[2 * M];
+  #pragma unroll
+  for (int k = 0; k < 2 * M; ++k) r[k] = ld_relaxed_gpu_u64(s_e + seg_index(e, lane, k));
+  bool ok = true;
+  #pragma unroll
+  for (int k = 0; k < 2 * M; ++k) {
+    ok &= unsigned(r[k] >> 32) == tag32;
+    w[k] = __uint_as_float(unsigned(r[k]));
+  }
+  return ok;
+}
+
+// End of a row block segment, epilogue side: warp e takes rows [64 e, 64 e +
+// 64) of it.  Write the rows (row block covered by this CTA alone); or, in a
+// shared row block, publish this CTA's slot (slots 1, 2, ...), or finish the
+// row block (slot 0): read the other slots until valid (slot 1 may have been
+// read already: pv, when `pre`), add the slots in slot order, write the rows
+// and clear the slots read.  The segment buffer is released as soon as it
+// has been read.  Returns whether this warp wrote final values.
 template <int M>
 __device__ __forceinline__ bool gemv_segment_write(const GemvArgs& a, const GemvJobDesc* J, int cj,
                                                    int rb, const float* fin, uint64_t* fin_empty,
-                                                   int lane, volatile int* abort_flag) {
-  const int G = J->grid, first_u = rb * J->upr;
-  const int c_first = unit_owner(first_u, J->units, G);
-  const int c_last = unit_owner(first_u + J->upr - 1, J->units, G);
-  const int n_contrib = c_last - c_first + 1, my = cj - c_first;
-  float v[4 * M];
+                                                   int e, int lane, volatile int* abort_flag,
+                                                   bool pre, const float (&pv)[2 * M]) {
+  const RowBlockShare sh = row_block_share(J, cj, rb);
+  const unsigned tag32 = unsigned(a.tag);
+  float v[2 * M];
   #pragma unroll
-  for (int k = 0; k < 4 * M; ++k) v[k] = fin[lane + 32 * k];
+  for (int k = 0; k < 2 * M; ++k) v[k] = fin[seg_index(e, lane, k)];
   __syncwarp();
-  if (lane == 0) mbar_arrive(smem_addr(fin_empty));  // the segment buffer is free again
-  if (n_contrib == 1) {
-    gemv_store_rows<M>(J, rb, lane, v);
+  if (lane == 0) mbar_arrive(smem_addr(fin_empty));  // this warp is done with the buffer
+  if (sh.n == 1) {
+    gemv_store_rows<M>(J, rb, e, lane, v);
     return true;
   }
-  // slot sl of the row block: [M][128] floats (rows past N unused)
-  float* part = a.partials + J->part_off + size_t(rb) * J->slots * M * kGemvRows;
-  unsigned long long* flag = a.flags + J->flag_off + size_t(rb) * J->slots;
-  if (my != 0) {
-    float* mine = part + size_t(my) * M * kGemvRows;
+  if (sh.my != 0) {
+    unsigned long long* s_e = slot_entries<M>(a, J, rb, sh.my);
     #pragma unroll
-    for (int k = 0; k < 4 * M; ++k) mine[lane + 32 * k] = v[k];
-    __syncwarp();
-    // the slot's writes (all lanes, ordered by the warp barrier) before its flag
-    if (lane == 0) st_release_gpu_u64(flag + my, a.tag);
+    for (int k = 0; k < 2 * M; ++k)
+      st_relaxed_gpu_u64(s_e + seg_index(e, lane, k), slot_entry(v[k], tag32));
     return false;
   }
-  // The finisher: every lane acquires every other slot's flag (bounded wait).
-  const unsigned long long t0 = global_timer_ns();
-  for (;;) {
-    bool up = true;
-    for (int sl = 1; sl < n_contrib; ++sl) up &= ld_acquire_gpu_u64(flag + sl) == a.tag;
-    if (__all_sync(0xFFFFFFFFu, up) || *abort_flag) break;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      if (lane == 0) {
-        *abort_flag = 1;
-        atomicOr(a.err, kDevErrWaitTimeout);
-      }
-      break;
-    }
-    __nanosleep(32);
-  }
-  // slot 0 (this CTA's, from registers), then the others in order
+  // the finisher: slot 0 (its own, from registers), then the others in order
   #pragma unroll
-  for (int k = 0; k < 4 * M; ++k) v[k] = 0.f + v[k];
-  for (int sl = 1; sl < n_contrib; ++sl) {
-    float w[4 * M];
+  for (int k = 0; k < 2 * M; ++k) v[k] = 0.f + v[k];
+  for (int sl = 1; sl < sh.n; ++sl) {
+    float w[2 * M];
+    if (sl == 1 && pre) {
+      #pragma unroll
+      for (int k = 0; k < 2 * M; ++k) w[k] = pv[k];
+    } else {
+      const unsigned long long* s_e = slot_entries<M>(a, J, rb, sl);
+      const unsigned long long t0 = global_timer_ns();
+      while (!read_slot<M>(s_e, e, lane, tag32, w)) {  // bounded wait for the partner's entries
+        if (*abort_flag) break;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          atomicOr(a.err, kDevErrWaitTimeout);
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
     #pragma unroll
-    for (int k = 0; k < 4 * M; ++k) w[k] = __ldcg(part + size_t(sl) * M * kGemvRows + lane + 32 * k);
-    #pragma unroll
-    for (int k = 0; k < 4 * M; ++k) v[k] += w[k];
+    for (int k = 0; k < 2 * M; ++k) v[k] += w[k];
   }
-  // lower the flags for the next launch with this tag (a replay); that launch
-  // starts only after this one has ended
-  for (int sl = 1 + lane; sl < n_contrib; sl += 32) flag[sl] = 0ull;
-  gemv_store_rows<M>(J, rb, lane, v);
+  // clear the entries read, for the next launch with this tag (a replay),
+  // which starts only after this one has ended
+  for (int sl = 1; sl < sh.n; ++sl) {
+    unsigned long long* s_e = slot_entries<M>(a, J, rb, sl);
+    #pragma unroll
+    for (int k = 0; k < 2 * M; ++k) s_e[seg_index(e, lane, k)] = 0ull;
+  }
+  gemv_store_rows<M>(J, rb, e, lane, v);
   return true;
 }
 
@@ -448,7 +500,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
     }
     for (int b = 0; b < kGemvSegBufs; ++b) {
       mbar_init(smem_addr(&fin_full[b]), 1);
-      mbar_init(smem_addr(&fin_empty[b]), 1);
+      mbar_init(smem_addr(&fin_empty[b]), kGemvEpilogueWarps);
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -567,11 +619,12 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
 
   if (warp > kGemvProducerWarp) {
     // ------------------------------ epilogue ------------------------------
-    // Warp e writes segments e, e + 2, ...; each row block it finishes is
-    // counted for its job (after a release fence, so that a CTA which sees the
-    // count complete also sees the rows).  Nothing of the workspace or the
-    // outputs is touched before the previous kernel on the stream is complete
-    // (it may still use the same buffers).
+    // Both warps take every segment, warp e rows [64 e, 64 e + 64) of it; each
+    // half of a row block written in final form is counted for its job (a
+    // release reduction, so that a CTA which sees the count complete also sees
+    // the rows).  Nothing of the workspace or the outputs is touched before
+    // the previous kernel on the stream is complete (it may still use the same
+    // buffers).
     griddep_wait();
     const int e = warp - kGemvProducerWarp - 1;
     int seg = 0;
@@ -581,15 +634,27 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
       for (int u = r.ub; u < r.ue;) {
         const int rb = u / J->upr;
         const int u_end = min(r.ue, (rb + 1) * J->upr);
-        if ((seg & 1) == e) {
-          const int b = seg & (kGemvSegBufs - 1);
-          gemv_wait(smem_addr(&fin_full[b]), uint32_t(seg >> 2) & 1u, a.err, abort_flag);
-          const bool wrote = gemv_segment_write<M>(a, J, r.cj, rb, fin + b * M * kGemvRows,
-                                                   &fin_empty[b], lane, abort_flag);
-          if (wrote && a.n_jobs > 1) {
-            __syncwarp();
-            if (lane == 0) red_release_gpu_add(a.sync + job, 1u);
+        const int b = seg & (kGemvSegBufs - 1);
+        const uint32_t fb = smem_addr(&fin_full[b]), fpar = uint32_t(seg >> 2) & 1u;
+        // Finishing a row block shared with one CTA, whose part came at the
+        // start of its range: read that CTA's slot while this CTA's own sums
+        // are still being made (it is usually written by then).
+        bool pre = false;
+        float pv[2 * M];
+        const RowBlockShare sh = row_block_share(J, r.cj, rb);
+        if (sh.n == 2 && sh.my == 0) {
+          const unsigned long long* s_e = slot_entries<M>(a, J, rb, 1);
+          while (!pre && !mbar_test_wait(fb, fpar) && !*abort_flag) {
+            pre = read_slot<M>(s_e, e, lane, unsigned(a.tag), pv);
+            if (!pre) __nanosleep(256);
           }
+        }
+        gemv_wait(fb, fpar, a.err, abort_flag);
+        const bool wrote = gemv_segment_write<M>(a, J, r.cj, rb, fin + b * M * kGemvRows,
+                                                 &fin_empty[b], e, lane, abort_flag, pre, pv);
+        if (wrote && a.n_jobs > 1) {
+          __syncwarp();
+          if (lane == 0) red_release_gpu_add(a.sync + job, 1u);
         }
         ++seg;
         u = u_end;

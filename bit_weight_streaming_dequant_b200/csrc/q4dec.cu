@@ -98,6 +98,13 @@ q4d_status library_workspace(void*& buf, size_t& bytes, size_t need, void** ws) 
       cudaGetLastError();
       return Q4D_ERR_CUDA;
     }
+    // zero-filled, as the GEMV's partial slots require (launches keep it so)
+    if (cudaMemset(buf, 0, need) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(buf);
+      buf = nullptr;
+      return Q4D_ERR_CUDA;
+    }
     bytes = need;
   }
   *ws = buf;
@@ -185,7 +192,7 @@ int gemv_stages(int M, size_t smem_limit) {
   return stages;
 }
 
-constexpr size_t kGemvFlagBytes = 8;      // one partial-slot flag
+constexpr size_t kGemvEntryBytes = 8;     // one partial-slot entry: fp32 value + tag
 constexpr int kSmemOptinB200 = 232448;    // planning default: B200's opt-in shared memory
 
 size_t round_up16(size_t v) { return (v + 15) / 16 * 16; }
@@ -206,20 +213,18 @@ q4d_status plan_gemv_rows(int M, int rows, int K, int num_sms, int smem_optin,
   plan->stages = gemv_stages(M, size_t(smem_optin));
   plan->reserved = 0;
   plan->smem_bytes = q4d::gemv_smem_bytes(M, plan->stages);
-  // slot flags (8 bytes per row block and slot), then the partial slots
-  plan->workspace_bytes =
-      j.slots > 0 ? round_up16(size_t(j.rbs) * j.slots * kGemvFlagBytes) +
-                        size_t(j.rbs) * j.slots * M * q4d::kGemvRows * 4
-                  : 0;
+  // the partial slots: [row block][slot][M][128] entries
+  plan->workspace_bytes = size_t(j.rbs) * j.slots * M * q4d::kGemvRows * kGemvEntryBytes;
   return Q4D_OK;
 }
 
 std::atomic<unsigned long long> g_gemv_tag{0};
 
-// A fresh 48-bit flag value for every launch (never 0: a lowered flag is 0).
+// A fresh tag for every launch; its low 32 bits, the ones partial-slot entries
+// carry, are never 0 (a cleared entry is 0).
 unsigned long long next_gemv_tag() {
   unsigned long long t = (g_gemv_tag.fetch_add(1, std::memory_order_relaxed) + 1) &
-                         ((1ull << 48) - 1);
+                         0xFFFFFFFFull;
   return t ? t : 1ull;
 }
 
@@ -292,10 +297,7 @@ q4d_status gemv_impl(const void* W_q4, const void* x, void* y, int M, int N, int
   a.err = s->err;
   a.tag = next_gemv_tag();
   if (p.workspace_bytes > 0) {
-    a.flags = static_cast<unsigned long long*>(workspace);
-    a.partials = reinterpret_cast<float*>(
-        static_cast<uint8_t*>(workspace) +
-        round_up16(size_t(p.row_blocks) * p.slots * kGemvFlagBytes));
+    a.partials = static_cast<unsigned long long*>(workspace);
   }
   q4d::GemvJobDesc& J = a.job;
   J.W = static_cast<const uint8_t*>(W_q4);
@@ -311,7 +313,6 @@ q4d_status gemv_impl(const void* W_q4, const void* x, void* y, int M, int N, int
   J.units = p.units;
   J.grid = p.grid;
   J.slots = p.slots;
-  J.flag_off = 0;
   J.rot = 0;
   if ((st = launch_gemv(M, a, p.smem_bytes, dev, *s, stream, pdl)) != Q4D_OK) return st;
   if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
@@ -572,7 +573,7 @@ struct BatchHeader {
   int n_jobs, M, num_sms, grid;
   int pad_;
   size_t workspace_bytes;
-  size_t flag_bytes;
+  size_t reserved_;
 };
 static_assert(sizeof(BatchHeader) <= kBatchHeader, "batch header");
 static_assert(sizeof(q4d::GemvJobDesc) % 16 == 0, "job descriptor alignment");
@@ -616,8 +617,7 @@ q4d_status q4d_gemv_batch_prepare(const q4d_gemv_job* jobs, int n_jobs, int M, i
   }
   q4d::GemvJobDesc* out =
       reinterpret_cast<q4d::GemvJobDesc*>(static_cast<uint8_t*>(desc) + kBatchHeader);
-  size_t flags = 0;     // partial-slot flags
-  size_t partials = 0;  // floats
+  size_t partials = 0;  // partial-slot entries
   long long units_before = 0;  // rotates each job's CTA numbering (balance across the batch)
   for (int i = 0; i < n_jobs; ++i) {
     const q4d_gemv_job& j = jobs[i];
@@ -639,13 +639,10 @@ q4d_status q4d_gemv_batch_prepare(const q4d_gemv_job* jobs, int n_jobs, int M, i
     d.units = sh.units;
     d.grid = sh.grid;
     d.slots = sh.slots;
-    if (flags > size_t(1 << 30)) return Q4D_ERR_UNSUPPORTED_SHAPE;
-    d.flag_off = int(flags);
     d.part_off = (long long)partials;
     d.rot = int(units_before % grid);
     units_before += sh.units;
     if (sh.slots > 0) {
-      flags += size_t(sh.rbs) * sh.slots;
       partials += size_t(sh.rbs) * sh.slots * M * q4d::kGemvRows;
     }
     std::memcpy(out + i, &d, sizeof(d));
@@ -657,8 +654,7 @@ q4d_status q4d_gemv_batch_prepare(const q4d_gemv_job* jobs, int n_jobs, int M, i
   h.M = M;
   h.num_sms = num_sms;
   h.grid = grid;
-  h.flag_bytes = round_up16(flags * kGemvFlagBytes);
-  h.workspace_bytes = h.flag_bytes + partials * 4;
+  h.workspace_bytes = partials * kGemvEntryBytes;
   std::memset(desc, 0, kBatchHeader);
   std::memcpy(desc, &h, sizeof(h));
   std::memset(static_cast<uint8_t*>(desc) + batch_sync_offset(n_jobs), 0,
@@ -696,8 +692,7 @@ q4d_status q4_gemv_batch_ex(const void* desc_host, void* desc_dev, void* stream,
   a.stages = stages;
   a.err = s->err;
   a.tag = next_gemv_tag();
-  a.flags = static_cast<unsigned long long*>(workspace);
-  a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + h.flag_bytes);
+  a.partials = static_cast<unsigned long long*>(workspace);
   if ((st = launch_gemv(h.M, a, q4d::gemv_smem_bytes(h.M, stages), dev, *s,
                         static_cast<cudaStream_t>(stream), (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0)) !=
       Q4D_OK)

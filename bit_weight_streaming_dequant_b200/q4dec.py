@@ -213,7 +213,8 @@ def _workspace(nbytes: int, device, workspace):
         if workspace.numel() * workspace.element_size() < nbytes:
             raise ValueError(f"workspace smaller than the {nbytes} bytes needed")
         return workspace
-    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    # zero-filled: the GEMV workspace's partial-slot entries must start at 0
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
 
 
 GEMV_WEIGHT_PREFETCH = 1  # Q4D_GEMV_WEIGHT_PREFETCH
@@ -421,7 +422,7 @@ class GemvBatch:
                                             nbytes, ctypes.byref(ws)), "q4d_gemv_batch_prepare")
             self.desc_dev = self.desc_host.to(self.device)
             self.workspace_bytes = ws.value
-            self.workspace = torch.empty(max(16, ws.value), dtype=torch.uint8, device=self.device)
+            self.workspace = torch.zeros(max(16, ws.value), dtype=torch.uint8, device=self.device)
 
     def run(self, stream=None, weight_prefetch: bool = False):
         torch = _torch()

@@ -109,11 +109,15 @@ const char* q4d_status_string(int status);
  * one CTA per SM, so a row block may be summed by several CTAs.  All but
  * one of them write fp32 partial sums into the workspace and raise a flag;
  * the CTA whose range ends in the row block waits for the flags and adds the
- * partial sums in a fixed (K) order, so results are deterministic.  The
- * workspace holds the flags (8 bytes per row block and slot) besides the
- * partial sums; it needs no initialisation (its previous contents are
- * ignored), but calls whose kernels may overlap on the GPU must not share
- * one workspace.
+ * partial sums in a fixed (K) order, so results are deterministic.  Each
+ * workspace entry (8 bytes) holds a partial sum and the launch's tag, which
+ * marks it as written.  The workspace must therefore be zero-filled before
+ * its first use; every launch that returns Q4D_OK and leaves the device error
+ * word at 0 leaves it zero-filled again, so one zeroing serves any number of
+ * GEMV calls of any shape (zero it again after a reported error, and do not
+ * share it with other kernels).  Calls whose kernels may overlap on the GPU
+ * must not share one workspace.  The library's own workspace (q4_gemv) is
+ * zeroed when allocated.
  */
 q4d_status q4_gemv(const void* W_q4, const void* x, float* y, int M, int N, int K);
 q4d_status q4_gemv_ex(const void* W_q4, const void* x, float* y, int M, int N, int K,
@@ -208,8 +212,8 @@ size_t q4d_gemv_workspace_bytes(int M, int N, int K);
  *     be rewritten while a launch may run.  num_sms
  *     must be the current device's SM count, else Q4D_ERR_INVALID_ARG.
  *     workspace: device memory of at least *workspace_bytes (16-byte aligned;
- *     no initialisation needed; launches that may overlap on the GPU must not
- *     share it), else Q4D_ERR_WORKSPACE.  flags: 0 or
+ *     zero-filled before first use and kept so, as for q4_gemv_ex; launches
+ *     that may overlap on the GPU must not share it), else Q4D_ERR_WORKSPACE.  flags: 0 or
  *     Q4D_GEMV_WEIGHT_PREFETCH (as q4_gemv_ex2: the first weights stream while
  *     the previous kernel on the stream still runs).  Never allocates; the
  *     launch can be captured into a CUDA graph and replayed.

@@ -116,11 +116,12 @@ def test_decode_layer_calls_replay_as_one_cuda_graph(cuda_ok):
         L = q4dec.lib()
         ws = {"attn": torch.empty(max(16, L.q4d_attn_workspace_bytes(ctx, n_q, n_kv, 256, M)),
                                   dtype=torch.uint8, device=dev),
-              "o": torch.empty(max(16, L.q4d_gemv_workspace_bytes(M, hid, n_q * 256)),
+              # GEMV workspaces: zero-filled before first use
+              "o": torch.zeros(max(16, L.q4d_gemv_workspace_bytes(M, hid, n_q * 256)),
                                dtype=torch.uint8, device=dev),
-              "gu": torch.empty(max(16, L.q4d_gemv_swiglu_workspace_bytes(M, ffn, hid)),
+              "gu": torch.zeros(max(16, L.q4d_gemv_swiglu_workspace_bytes(M, ffn, hid)),
                                 dtype=torch.uint8, device=dev),
-              "dn": torch.empty(max(16, L.q4d_gemv_workspace_bytes(M, hid, ffn)),
+              "dn": torch.zeros(max(16, L.q4d_gemv_workspace_bytes(M, hid, ffn)),
                                 dtype=torch.uint8, device=dev)}
         return (dev_bytes(K0), dev_bytes(V0), torch.empty((M, n_q, 256), device=dev),
                 torch.empty((M, n_q * 256), dtype=torch.bfloat16, device=dev),

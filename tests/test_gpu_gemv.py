@@ -121,6 +121,26 @@ def test_plain_entry_point_and_side_stream(cuda_ok):
     assert torch.equal(y, y2)
 
 
+def test_one_zeroed_workspace_serves_every_shape(cuda_ok):
+    # a caller-owned workspace, zero-filled once, is used by calls of several
+    # shapes and M (each sharing row blocks across CTAs); after every call all
+    # of it is zero again and the results equal calls with fresh workspaces
+    L = q4dec.lib()
+    shapes = [(64, 65536, 2), (17408, 5120, 1), (5120, 17408, 5), (6144, 5120, 3), (300, 1280, 4)]
+    need = max(L.q4d_gemv_workspace_bytes(M, N, K) for N, K, M in shapes)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for i, (N, K, M) in enumerate(shapes * 2):
+        assert L.q4d_gemv_workspace_bytes(M, N, K) > 0, (N, K, M)
+        W = synth.device_q4_0_weights(1100 + i % len(shapes), N, K)
+        x = synth.device_bf16_normal(1110 + i % len(shapes), (M, K))
+        ref = q4dec.q4_gemv(W, x, N=N, K=K)
+        y = q4dec.q4_gemv(W, x, N=N, K=K, workspace=ws, weight_prefetch=bool(i & 1))
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref), (N, K, M)
+        assert int(torch.count_nonzero(ws)) == 0, (N, K, M)
+    assert q4dec.device_error() == 0
+
+
 def test_bad_calls_launch_nothing(cuda_ok):
     N, K = 64, 512
     W = dev_bytes(synth.q4_0_weights(1, N, K))

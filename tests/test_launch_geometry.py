@@ -70,8 +70,8 @@ def test_gemv_geometry(M, N, K, sms):
                 a, b = ranges[c]
                 assert a < (rb + 1) * upr and b > rb * upr
     assert p.slots == slots
-    flags = -(-rbs * slots * 8 // 16) * 16           # one 8-byte flag per row block and slot
-    assert p.workspace_bytes == (flags + rbs * slots * M * 128 * 4 if slots else 0)
+    # one 8-byte entry (fp32 value + tag) per row, column and slot of each row block
+    assert p.workspace_bytes == rbs * slots * M * 128 * 8
     # every copy stays inside its source buffer and its stage slot
     w_bytes, x_bytes = N * nsb * 144, M * K * 2
     for c in {0, G // 2, G - 1}:
