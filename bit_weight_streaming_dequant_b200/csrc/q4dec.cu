@@ -405,7 +405,24 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
     st = q8 ? launch_attn_tc<32, true, 1>(a, p, n_kv, dev, *s, stream)
             : launch_attn_tc<32, false, 2>(a, p, n_kv, dev, *s, stream);
   if (st != Q4D_OK) return st;
-  if (p.n_splits > 1) q4d::q4kv_attn_merge_kernel<<<M * n_q, 256, 0, stream>>>(a);
+  if (p.n_splits > 1) {
+    // the merge may launch while the split kernel runs; it waits for it on
+    // the device (griddepcontrol.wait) before reading the split states
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(unsigned(M * n_q));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, q4d::q4kv_attn_merge_kernel, a) != cudaSuccess) {
+      cudaGetLastError();
+      return Q4D_ERR_CUDA;
+    }
+  }
   if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
   return Q4D_OK;
 }

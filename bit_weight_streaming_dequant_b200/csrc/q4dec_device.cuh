@@ -88,6 +88,27 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   }
 }
 
+// mbar_wait for kernels with a per-CTA abort flag: gives up at once while
+// *abort is set, and sets it (and the error word) when it times out itself, so
+// that after one time-out no wait of the CTA blocks again.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t parity, unsigned* err,
+                                                   volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  if (*abort) return false;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t polls = 1;; ++polls) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((polls & 255u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(err, kDevErrWaitTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 // L2 policy for data that is read exactly once (weights, K/V tiles).
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol;

@@ -154,10 +154,10 @@ constexpr uint32_t kR8StageBytes = 2u * kR8Tile * kRowBytes;   // K tile + V til
 
 // Shared memory of the warp-local variant: the ring (which also holds the
 // final cross-warp combine, 96 KB), Q fragments of 8 rows, per-warp and
-// per-row statistics, barriers.
+// per-row statistics, barriers, the abort flag (padded to 16).
 __host__ __device__ constexpr size_t attn_rows8_smem_bytes(int stages) {
   return size_t(stages) * kR8StageBytes + 8 * kR8QPitch + size_t(kR8Warps) * 8 * 2 * 4 +
-         8 * 2 * 4 + size_t(stages) * 16;
+         8 * 2 * 4 + size_t(stages) * 16 + 16;
 }
 
 // Warp-local variant for at most 8 query rows per CTA (one row tile: plain
@@ -179,6 +179,9 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
   float* rml = wml + kR8Warps * 8 * 2;                              // [row][M, L]
   uint64_t* full = reinterpret_cast<uint64_t*>(rml + 8 * 2);
   uint64_t* empty = full + S;
+  // set by the first wait that times out: from then on no wait blocks and no
+  // further copy is issued (the results are void; the error word says so)
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + S);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x, kh = blockIdx.y, rgrp = blockIdx.z;
@@ -209,6 +212,7 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
       mbar_init(smem_addr(&full[s]), 1);
       mbar_init(smem_addr(&empty[s]), kR8Warps);
     }
+    *abort_flag = 0;
     mbar_init_fence();
     // start streaming before anything else
     for (; issued < min(S, n_tiles); ++issued) issue(issued);
@@ -253,12 +257,12 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
   for (int tile = 0; tile < n_tiles; ++tile) {
     if (producer) {
       // refill the slots every warp has released; block only for this tile
-      while (issued < n_tiles && issued < tile + S) {
+      while (issued < n_tiles && issued < tile + S && !*abort_flag) {
         const uint32_t bar = smem_addr(&empty[issued % S]);
         const uint32_t parity = uint32_t(issued / S - 1) & 1u;
         if (issued > tile) {
           if (!mbar_test_wait(bar, parity)) break;
-        } else if (!mbar_wait(bar, parity, a.err)) {
+        } else if (!mbar_wait_or_abort(bar, parity, a.err, abort_flag)) {
           break;
         }
         issue(issued++);
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
     __syncwarp();
     const int t0 = t_begin + tile * TT;
     const int n_tok = min(TT, t_end - t0);
-    mbar_wait(smem_addr(&full[slot]), phase, a.err);
+    mbar_wait_or_abort(smem_addr(&full[slot]), phase, a.err, abort_flag);
     const uint8_t* Kt = ring + size_t(slot) * kR8StageBytes;
     const uint8_t* Vt = Kt + TT * kRowBytes;
     if (tok0 < n_tok) {
@@ -380,6 +384,13 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
     }
   }
 
+  // After a time-out: wait (bounded) for the copies still in flight -- the
+  // last tile issued into each slot -- before the ring is reused below and
+  // before the CTA exits.
+  if (producer && *abort_flag)
+    for (int tile = max(0, issued - S); tile < issued; ++tile)
+      mbar_wait(smem_addr(&full[tile % S]), uint32_t(tile / S) & 1u, a.err);
+
   // ---- combine the warps: per-row maxima and sums, then O^T parked in the
   // (now idle) ring as [warp][row][dim] and summed in warp order
   #pragma unroll
@@ -442,7 +453,9 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
 }
 
 // Log-sum-exp merge of the per-split states (base 2); one CTA of eight warps
-// per (draft row, head).  Every warp finds the global maximum and the total
+// per (draft row, head).  Launched so that its CTAs may start while the split
+// kernel still runs (programmatic dependent launch): they read the split
+// states only once that kernel has completed.  Every warp finds the global maximum and the total
 // weight itself; warp w then adds splits w, w + 8, ... for all 256
 // dimensions (two float4 per lane), and the eight partial vectors are summed
 // in warp order.
@@ -450,6 +463,7 @@ __global__ void __launch_bounds__(256) q4kv_attn_merge_kernel(const AttnArgs a) 
   const int row = blockIdx.x;  // m * n_q + h
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) griddep_launch_dependents();
+  griddep_wait();  // the split kernel has finished: its states are visible
   const size_t rows = size_t(a.M) * a.n_q;
   __shared__ float part[8 * kHeadDim];
   const int n = a.n_splits;

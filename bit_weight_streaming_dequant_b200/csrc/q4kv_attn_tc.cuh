@@ -153,7 +153,10 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
   float* alph = m_use + 32;
   float* lsum = alph + 32;
   int* rpos = reinterpret_cast<int*>(lsum + 32);            // causal limit of each row
-  int* flags = rpos + 32;
+  int* flags = rpos + 32;          // [0] some row's maximum grew, [1] abort
+  // set by the first wait that times out: from then on no wait blocks and no
+  // further copy is issued (the results are void; the error word says so)
+  volatile int* abort_flag = flags + 1;
   uint64_t* full = reinterpret_cast<uint64_t*>(flags + 4);
   uint64_t* empty = full + S;
   uint64_t* kready = empty + S;   // [2] K tile in tensor memory
@@ -188,6 +191,7 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
       mbar_init(smem_addr(&pready[i]), kTcaRoleWarps * 32);
       mbar_init(smem_addr(&pfree[i]), 1);
     }
+    flags[1] = 0;
     mbar_init_fence();
   }
   // Q in the unpacked element order, K-major canonical layout (core matrices
@@ -229,9 +233,12 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
       const uint8_t* Kh = a.K + size_t(kh) * a.kv_stride * RB;
       const uint8_t* Vh = a.V + size_t(kh) * a.kv_stride * RB;
       const uint64_t pol = l2_evict_first_policy();
+      int issued = 0;
       for (int tile = 0; tile < n_tiles; ++tile) {
         const int slot = tile % S;
-        if (tile >= S) mbar_wait(smem_addr(&empty[slot]), uint32_t(tile / S - 1) & 1u, a.err);
+        if (tile >= S && !mbar_wait_or_abort(smem_addr(&empty[slot]), uint32_t(tile / S - 1) & 1u,
+                                             a.err, abort_flag))
+          break;  // no further copies after a time-out
         const int t0 = t_begin + tile * TT;
         const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * RB;
         const uint32_t bar = smem_addr(&full[slot]);
@@ -239,7 +246,13 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
         mbar_arrive_expect_tx(bar, 2 * bytes);
         bulk_g2s(dk, Kh + size_t(t0) * RB, bytes, bar, pol);
         bulk_g2s(dk + TT * RB, Vh + size_t(t0) * RB, bytes, bar, pol);
+        issued = tile + 1;
       }
+      // after a time-out: wait (bounded) for the copies still in flight, the
+      // last tile issued into each slot, before the CTA can exit
+      if (*abort_flag)
+        for (int tile = max(0, issued - S); tile < issued; ++tile)
+          mbar_wait(smem_addr(&full[tile % S]), uint32_t(tile / S) & 1u, a.err);
     }
   } else if (warp == kTcaMmaWarp) {
     // ------------------------------ MMA issuer -----------------------------
@@ -248,7 +261,7 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
         const int b = tile & 1;
         // S^T[b] is free: the P.V of tile - 2, issued before, waited for the
         // softmax warps to have read it (they read S^T before storing P^T)
-        mbar_wait(smem_addr(&kready[b]), uint32_t(tile >> 1) & 1u, a.err);
+        mbar_wait_or_abort(smem_addr(&kready[b]), uint32_t(tile >> 1) & 1u, a.err, abort_flag);
         tc_fence_after();
         const uint32_t qs = smem_addr(Qs);
         #pragma unroll
@@ -262,11 +275,11 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
       for (int tile = 0; tile < n_tiles; ++tile) {
         if (tile + 1 < n_tiles) qk(tile + 1);
         const int pb = tile % PB;
-        mbar_wait(smem_addr(&pready[pb]), uint32_t(tile / PB) & 1u, a.err);
+        mbar_wait_or_abort(smem_addr(&pready[pb]), uint32_t(tile / PB) & 1u, a.err, abort_flag);
         const uint32_t psb = ps + uint32_t(pb) * (NR * 256);
         #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          mbar_wait(smem_addr(&vready[h]), uint32_t(tile) & 1u, a.err);
+          mbar_wait_or_abort(smem_addr(&vready[h]), uint32_t(tile) & 1u, a.err, abort_flag);
           tc_fence_after();
           #pragma unroll
           for (int j = 0; j < 8; ++j)  // 16 tokens per step
@@ -278,14 +291,19 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
         }
         tc_commit(smem_addr(&pfree[pb]));
       }
+      // every MMA issued has completed (the last commit tracks them all)
+      // before tensor memory is read by the epilogue and freed -- also after a
+      // time-out, when the waits above no longer hold the chain back
+      if (n_tiles > 0)
+        mbar_wait(smem_addr(&pfree[(n_tiles - 1) % PB]), uint32_t((n_tiles - 1) / PB) & 1u, a.err);
     }
   } else if (warp >= kTcaRoleWarps && warp < 2 * kTcaRoleWarps) {
     // ------------------------------ K warps --------------------------------
     for (int tile = 0; tile < n_tiles; ++tile) {
       const int slot = tile % S;
-      mbar_wait(smem_addr(&full[slot]), uint32_t(tile / S) & 1u, a.err);
+      mbar_wait_or_abort(smem_addr(&full[slot]), uint32_t(tile / S) & 1u, a.err, abort_flag);
       // K buffer (tile & 1) was last read by QK(tile - 2)
-      if (tile >= 2) mbar_wait(smem_addr(&sdone[tile & 1]), uint32_t((tile - 2) >> 1) & 1u, a.err);
+      if (tile >= 2) mbar_wait_or_abort(smem_addr(&sdone[tile & 1]), uint32_t((tile - 2) >> 1) & 1u, a.err, abort_flag);
       __syncwarp();  // the tensor-memory stores below are warp-collective
       tc_fence_after();
       const uint8_t* row = ring + size_t(slot) * kStage + k * RB;
@@ -314,14 +332,14 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
     // ------------------------------ V warps --------------------------------
     for (int tile = 0; tile < n_tiles; ++tile) {
       const int slot = tile % S;
-      mbar_wait(smem_addr(&full[slot]), uint32_t(tile / S) & 1u, a.err);
+      mbar_wait_or_abort(smem_addr(&full[slot]), uint32_t(tile / S) & 1u, a.err, abort_flag);
       const uint8_t* row = ring + size_t(slot) * kStage + (TT + k) * RB;
       const bool live = k < t_end - (t_begin + tile * TT);
       const uint4 dv = *reinterpret_cast<const uint4*>(row + kScales);
       #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         // half h of the V tile was last read by the P.V chain of tile - 1
-        if (tile > 0) mbar_wait(smem_addr(&pvdone[h]), uint32_t(tile - 1) & 1u, a.err);
+        if (tile > 0) mbar_wait_or_abort(smem_addr(&pvdone[h]), uint32_t(tile - 1) & 1u, a.err, abort_flag);
         #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
           const int b = 4 * h + bb;
@@ -347,7 +365,7 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
     for (int tile = 0; tile < n_tiles; ++tile) {
       const int t0 = t_begin + tile * TT;
       const int n_tok = min(TT, t_end - t0);
-      mbar_wait(smem_addr(&sdone[tile & 1]), uint32_t(tile >> 1) & 1u, a.err);
+      mbar_wait_or_abort(smem_addr(&sdone[tile & 1]), uint32_t(tile >> 1) & 1u, a.err, abort_flag);
       __syncwarp();
       tc_fence_after();
       float s[NR];
@@ -404,9 +422,9 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
       // P^T buffer (tile % PB) is free once the P.V of tile - PB has read it;
       // O^T may be rescaled only after the P.V of tile - 1 has finished
       if (tile >= PB)
-        mbar_wait(smem_addr(&pfree[tile % PB]), uint32_t((tile - PB) / PB) & 1u, a.err);
+        mbar_wait_or_abort(smem_addr(&pfree[tile % PB]), uint32_t((tile - PB) / PB) & 1u, a.err, abort_flag);
       if (rescale && tile > 0) {
-        mbar_wait(smem_addr(&pvdone[1]), uint32_t(tile - 1) & 1u, a.err);
+        mbar_wait_or_abort(smem_addr(&pvdone[1]), uint32_t(tile - 1) & 1u, a.err, abort_flag);
         __syncwarp();
         tc_fence_after();
         {
@@ -435,7 +453,7 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
     }
     // ---- split totals: row sums of the rounded P (after the last P.V)
     if (n_tiles > 0) {
-      mbar_wait(smem_addr(&pfree[(n_tiles - 1) % PB]), uint32_t((n_tiles - 1) / PB) & 1u, a.err);
+      mbar_wait_or_abort(smem_addr(&pfree[(n_tiles - 1) % PB]), uint32_t((n_tiles - 1) / PB) & 1u, a.err, abort_flag);
       __syncwarp();
     }
     #pragma unroll

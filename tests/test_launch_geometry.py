@@ -188,9 +188,9 @@ def _tc_offsets(stages, nr, row=ROW, pb=2):
 
 
 def _attn_smem(stages, rows_per_cta):
-    if rows_per_cta <= 8:      # ring + Q fragments + per-warp / per-row stats + barriers
+    if rows_per_cta <= 8:      # ring + Q fragments + per-warp / per-row stats + barriers + abort
         return stages * 2 * TT_R8 * ROW + 8 * Q_PITCH + WARPS_R8 * 8 * 2 * 4 + 8 * 2 * 4 \
-            + stages * 16
+            + stages * 16 + 16
     return _tc_offsets(stages, _tc_nr(rows_per_cta))["end"]
 
 
