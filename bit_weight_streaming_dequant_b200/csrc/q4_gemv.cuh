@@ -58,13 +58,14 @@
 //    18 KB plus one copy of each activation row's 1 KB, issued by a producer
 //    warp into a ring of stages that complete on "full" mbarriers.  Sixteen
 //    consumer warps take one (column, block) task each per stage and release
-//    it on an "empty" mbarrier.  At the end of each row block segment they add
-//    their 16 partial sums in a fixed order through shared memory into one of
-//    four segment buffers and go on with the next stage; two epilogue warps,
-//    each taking one half (64 rows) of every segment, write them out (y, the
-//    partial slot, or the sum of the slots) and count the halves written in
-//    final form for their job, so no global write or atomic stalls the
-//    consumers.
+//    it on an "empty" mbarrier.  At the end of each row block segment each
+//    consumer warp stores its partial sums into its own slot of a reduction
+//    buffer, signals it on an mbarrier and goes on with the next stage -- no
+//    CTA-wide barrier; two epilogue warps, each taking one half (64 rows) of
+//    every segment, add the 16 slots in warp order, release the buffer, write
+//    the sums out (y, the partial slot, or the sum of the slots) and count the
+//    halves written in final form for their job, so no global write, atomic
+//    or cross-warp reduction stalls the consumers.
 //  * Every wait is bounded in time.  A wait that runs out sets the device
 //    error word and a per-CTA abort flag; from then on no wait blocks, the
 //    producer issues no further copies and waits for the ones in flight, and
@@ -92,7 +93,7 @@ constexpr int kGemvConsumerWarps = 8 * kGemvCols;          // one (column, block
 constexpr int kGemvProducerWarp = kGemvConsumerWarps;      // bulk copies
 constexpr int kGemvEpilogueWarps = 2;                      // output writes, flags, counts
 constexpr int kGemvThreads = (kGemvConsumerWarps + 1 + kGemvEpilogueWarps) * 32;
-constexpr int kGemvSegBufs = 4;                            // segment buffers (consumers -> epilogue)
+constexpr int kGemvRedStride = kGemvRows + 4;              // floats per column of a slot (banks)
 constexpr int kGemvMaxStages = 8;
 constexpr uint32_t kSbBytes = 144;                         // one super-block
 constexpr uint32_t kGemvWBox = kGemvRows * kSbBytes;       // one column of a row block
@@ -104,19 +105,17 @@ constexpr uint32_t kJobSwiglu = 2u;                        // rows are gate / up
 __host__ __device__ constexpr uint32_t gemv_stage_bytes(int M) {
   return kGemvCols * kGemvWBox + uint32_t(M) * kGemvCols * 512u;
 }
-// Cross-warp reduction buffer: 8 slots x 8 tiles x 16 rows x M columns, fp32.
+// Reduction buffers (consumers -> epilogue): two for M <= 2, one otherwise
+// (shared memory), each 16 warp slots of [M][kGemvRedStride] fp32.
+__host__ __device__ constexpr int gemv_red_bufs(int M) { return M <= 2 ? 2 : 1; }
 __host__ __device__ constexpr uint32_t gemv_red_bytes(int M) {
-  return 8u * kGemvTiles * 16u * uint32_t(M) * 4u;
+  return uint32_t(gemv_red_bufs(M)) * kGemvConsumerWarps * uint32_t(M) * kGemvRedStride * 4u;
 }
-// Segment buffers: [4][M][128] fp32.
-__host__ __device__ constexpr uint32_t gemv_fin_bytes(int M) {
-  return uint32_t(kGemvSegBufs) * uint32_t(M) * kGemvRows * 4u;
-}
-// Shared memory: ring, reduction buffer, segment buffers, the abort flag
-// (padded to 16), 2 barriers per stage and 2 per segment buffer.
+// Shared memory: ring, reduction buffers, the abort flag (padded to 16), 2
+// barriers per stage and 2 per reduction buffer.
 __host__ __device__ constexpr size_t gemv_smem_bytes(int M, int stages) {
-  return size_t(stages) * gemv_stage_bytes(M) + gemv_red_bytes(M) + gemv_fin_bytes(M) + 16 +
-         size_t(stages) * 16 + size_t(kGemvSegBufs) * 16;
+  return size_t(stages) * gemv_stage_bytes(M) + gemv_red_bytes(M) + 16 + size_t(stages) * 16 +
+         size_t(gemv_red_bufs(M)) * 16;
 }
 
 // First unit of (job-local) CTA c when U units are shared out over G CTAs
@@ -210,10 +209,6 @@ __device__ __forceinline__ void store_out(void* out, size_t i, float v, bool bf1
     reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
   else
     reinterpret_cast<float*>(out)[i] = v;
-}
-
-__device__ __forceinline__ void gemv_consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kGemvConsumerWarps * 32) : "memory");
 }
 
 // Wait for the barrier phase with the given parity, for at most kWaitLimitNs,
@@ -331,49 +326,6 @@ __device__ __forceinline__ void gemv_store_rows(const GemvJobDesc* J, int rb, in
   }
 }
 
-// End of a row block segment, consumer side: add the 16 warps' partial sums in
-// a fixed order (warp w + 8 into warp w, then the 8 slots in order) into the
-// segment buffer `fin` ([M][128]).
-template <int M>
-__device__ __forceinline__ void gemv_segment_reduce(float* red, float* fin,
-                                                    const float (&acc)[kGemvTiles][4], int warp,
-                                                    int lane, int tid) {
-  const int g = lane >> 2, t = lane & 3;
-  auto red_at = [&](int s, int p, int row, int m) -> float& {
-    return red[((s * kGemvTiles + p) * 16 + row) * M + m];
-  };
-  if (warp >= 8) {
-    #pragma unroll
-    for (int p = 0; p < kGemvTiles; ++p)
-      #pragma unroll
-      for (int e = 0; e < 2; ++e)
-        if (2 * t + e < M) {
-          red_at(warp - 8, p, g, 2 * t + e) = acc[p][e];
-          red_at(warp - 8, p, g + 8, 2 * t + e) = acc[p][2 + e];
-        }
-  }
-  gemv_consumer_sync();
-  if (warp < 8) {
-    #pragma unroll
-    for (int p = 0; p < kGemvTiles; ++p)
-      #pragma unroll
-      for (int e = 0; e < 2; ++e)
-        if (2 * t + e < M) {
-          red_at(warp, p, g, 2 * t + e) = acc[p][e] + red_at(warp, p, g, 2 * t + e);
-          red_at(warp, p, g + 8, 2 * t + e) = acc[p][2 + e] + red_at(warp, p, g + 8, 2 * t + e);
-        }
-  }
-  gemv_consumer_sync();
-  for (int i = tid; i < kGemvRows * M; i += kGemvConsumerWarps * 32) {
-    const int m = i / kGemvRows, r = i - m * kGemvRows;
-    float s = 0.f;
-    #pragma unroll
-    for (int w = 0; w < 8; ++w) s += red_at(w, r >> 4, r & 15, m);
-    fin[i] = s;
-  }
-  gemv_consumer_sync();
-}
-
 // Who shares row block rb of job J, and this CTA's slot among them.
 struct RowBlockShare {
   int n, my;
@@ -410,25 +362,38 @@ __device__ __forceinline__ bool read_slot(const unsigned long long* s_e, int e, 
   return ok;
 }
 
+// This CTA's sums of a row block segment, epilogue side (warp e: rows [64 e,
+// 64 e + 64)): the 16 consumer warps' slots of reduction buffer `buf` added in
+// warp order into v; then the buffer is released (this warp's arrival).
+template <int M>
+__device__ __forceinline__ void gemv_segment_sum(const float* buf, uint64_t* buf_empty, int e,
+                                                 int lane, float (&v)[2 * M]) {
+  #pragma unroll
+  for (int k = 0; k < 2 * M; ++k) {
+    const float* col = buf + (k >> 1) * kGemvRedStride + seg_row(e, lane, k);
+    float acc = col[0];
+    #pragma unroll
+    for (int w = 1; w < kGemvConsumerWarps; ++w) acc += col[w * M * kGemvRedStride];
+    v[k] = acc;
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(smem_addr(buf_empty));  // this warp is done with the buffer
+}
+
 // End of a row block segment, epilogue side: warp e takes rows [64 e, 64 e +
-// 64) of it.  Write the rows (row block covered by this CTA alone); or, in a
-// shared row block, publish this CTA's slot (slots 1, 2, ...), or finish the
-// row block (slot 0): read the other slots until valid (slot 1 may have been
-// read already: pv, when `pre`), add the slots in slot order, write the rows
-// and clear the slots read.  The segment buffer is released as soon as it
-// has been read.  Returns whether this warp wrote final values.
+// 64) of it, this CTA's sums in v.  Write the rows (row block covered by this
+// CTA alone); or, in a shared row block, publish this CTA's slot (slots 1,
+// 2, ...), or finish the row block (slot 0): read the other slots until valid
+// (slot 1 may have been read already: pv, when `pre`), add the slots in slot
+// order, write the rows and clear the slots read.  Returns whether this warp
+// wrote final values.
 template <int M>
 __device__ __forceinline__ bool gemv_segment_write(const GemvArgs& a, const GemvJobDesc* J, int cj,
-                                                   int rb, const float* fin, uint64_t* fin_empty,
-                                                   int e, int lane, volatile int* abort_flag,
-                                                   bool pre, const float (&pv)[2 * M]) {
+                                                   int rb, int e, int lane,
+                                                   volatile int* abort_flag, bool pre,
+                                                   const float (&pv)[2 * M], float (&v)[2 * M]) {
   const RowBlockShare sh = row_block_share(J, cj, rb);
   const unsigned tag32 = unsigned(a.tag);
-  float v[2 * M];
-  #pragma unroll
-  for (int k = 0; k < 2 * M; ++k) v[k] = fin[seg_index(e, lane, k)];
-  __syncwarp();
-  if (lane == 0) mbar_arrive(smem_addr(fin_empty));  // this warp is done with the buffer
   if (sh.n == 1) {
     gemv_store_rows<M>(J, rb, e, lane, v);
     return true;
@@ -483,14 +448,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
   constexpr uint32_t kStage = gemv_stage_bytes(M);
   constexpr uint32_t kXOff = kGemvCols * kGemvWBox;
   uint8_t* ring = smem;
-  float* red = reinterpret_cast<float*>(smem + size_t(S) * kStage);
-  float* fin = red + gemv_red_bytes(M) / 4;                       // [4][M][128]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(fin + kGemvSegBufs * M * kGemvRows);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(S) * kStage + gemv_red_bytes(M) +
-                                               gemv_fin_bytes(M) + 16);
+  constexpr int kRedBufs = gemv_red_bufs(M);
+  float* red = reinterpret_cast<float*>(smem + size_t(S) * kStage);  // [bufs][16 warps][M][stride]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red + gemv_red_bytes(M) / 4);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(S) * kStage + gemv_red_bytes(M) + 16);
   uint64_t* empty = full + S;
-  uint64_t* fin_full = empty + S;                 // [4] segment buffer written by the consumers
-  uint64_t* fin_empty = fin_full + kGemvSegBufs;  // [4] segment buffer released by the epilogue
+  uint64_t* red_full = empty + S;            // [bufs] every consumer warp's slot written
+  uint64_t* red_empty = red_full + kRedBufs; // [bufs] buffer read by both epilogue warps
 
   if (tid == 0) {
     griddep_launch_dependents();  // the next kernel on the stream may start its prologue
@@ -498,9 +462,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
       mbar_init(smem_addr(&full[s]), 1);
       mbar_init(smem_addr(&empty[s]), kGemvConsumerWarps);
     }
-    for (int b = 0; b < kGemvSegBufs; ++b) {
-      mbar_init(smem_addr(&fin_full[b]), 1);
-      mbar_init(smem_addr(&fin_empty[b]), kGemvEpilogueWarps);
+    for (int b = 0; b < kRedBufs; ++b) {
+      mbar_init(smem_addr(&red_full[b]), kGemvConsumerWarps);
+      mbar_init(smem_addr(&red_empty[b]), kGemvEpilogueWarps);
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -634,8 +598,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
       for (int u = r.ub; u < r.ue;) {
         const int rb = u / J->upr;
         const int u_end = min(r.ue, (rb + 1) * J->upr);
-        const int b = seg & (kGemvSegBufs - 1);
-        const uint32_t fb = smem_addr(&fin_full[b]), fpar = uint32_t(seg >> 2) & 1u;
+        const int b = seg % kRedBufs;
+        const uint32_t fb = smem_addr(&red_full[b]), fpar = uint32_t(seg / kRedBufs) & 1u;
         // Finishing a row block shared with one CTA, whose part came at the
         // start of its range: read that CTA's slot while this CTA's own sums
         // are still being made (it is usually written by then).
@@ -650,8 +614,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
           }
         }
         gemv_wait(fb, fpar, a.err, abort_flag);
-        const bool wrote = gemv_segment_write<M>(a, J, r.cj, rb, fin + b * M * kGemvRows,
-                                                 &fin_empty[b], e, lane, abort_flag, pre, pv);
+        float v[2 * M];
+        gemv_segment_sum<M>(red + size_t(b) * kGemvConsumerWarps * M * kGemvRedStride,
+                            &red_empty[b], e, lane, v);
+        const bool wrote =
+            gemv_segment_write<M>(a, J, r.cj, rb, e, lane, abort_flag, pre, pv, v);
         if (wrote && a.n_jobs > 1) {
           __syncwarp();
           if (lane == 0) red_release_gpu_add(a.sync + job, 1u);
@@ -737,14 +704,24 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
           phase ^= 1u;
         }
       }
-      // hand the row block's sums to the epilogue (buffer seg % 4 must have
-      // been released: segment seg - 4)
-      const int b = seg & (kGemvSegBufs - 1);
-      if (seg >= kGemvSegBufs)
-        gemv_wait(smem_addr(&fin_empty[b]), uint32_t((seg - kGemvSegBufs) >> 2) & 1u, a.err,
+      // hand this warp's sums of the row block to the epilogue: its slot of
+      // reduction buffer seg % bufs (released by the epilogue after segment
+      // seg - bufs), element (m, row) at m * stride + row
+      const int b = seg % kRedBufs;
+      if (seg >= kRedBufs)
+        gemv_wait(smem_addr(&red_empty[b]), uint32_t((seg - kRedBufs) / kRedBufs) & 1u, a.err,
                   abort_flag);
-      gemv_segment_reduce<M>(red, fin + b * M * kGemvRows, acc, warp, lane, tid);
-      if (tid == 0) mbar_arrive(smem_addr(&fin_full[b]));
+      float* slot = red + (size_t(b) * kGemvConsumerWarps + warp) * M * kGemvRedStride;
+      #pragma unroll
+      for (int p = 0; p < kGemvTiles; ++p)
+        #pragma unroll
+        for (int e = 0; e < 2; ++e)
+          if (2 * t + e < M) {
+            slot[(2 * t + e) * kGemvRedStride + 16 * p + g] = acc[p][e];
+            slot[(2 * t + e) * kGemvRedStride + 16 * p + g + 8] = acc[p][2 + e];
+          }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&red_full[b]));
       ++seg;
       u += n_units;
     }

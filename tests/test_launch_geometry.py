@@ -46,10 +46,16 @@ def test_gemv_geometry(M, N, K, sms):
     assert p.threads == GEMV_THREADS and p.row_blocks == rbs and p.units_per_row_block == upr
     assert p.units == U and 1 <= G <= min(sms, U)
     stage = _gemv_stage_bytes(M)
-    red = 8 * 8 * 16 * M * 4
     assert stage % 128 == 0 and (p.stages * stage) % 128 == 0
-    fin = 4 * M * 128 * 4                      # four segment buffers (consumers -> epilogue)
-    assert p.smem_bytes == p.stages * stage + red + fin + 16 + p.stages * 16 + 4 * 16
+    # reduction buffers (consumers -> epilogue): 2 for M <= 2, else 1, each a
+    # slot per consumer warp of [M][132] fp32 (128 rows + 4 floats of padding:
+    # the 8 rows x 4 columns a warp stores at once hit distinct banks)
+    bufs = 2 if M <= 2 else 1
+    red = bufs * 16 * M * 132 * 4
+    assert p.smem_bytes == p.stages * stage + red + 16 + p.stages * 16 + bufs * 16
+    banks = {((2 * t + e) * 132 + g) % 32 for t in range(4) for g in range(8) for e in (0,)
+             if 2 * t + e < M}
+    assert len(banks) == 8 * len([t for t in range(4) if 2 * t < M])
     assert p.smem_bytes + stage + 16 > SMEM_OPTIN or p.stages == 8   # as many stages as fit
     assert 2 <= p.stages <= 8 and p.smem_bytes <= SMEM_OPTIN
     # the units are shared out exactly once, every CTA getting at least one
