@@ -503,12 +503,11 @@ q4d_status plan_attn_impl(int ctx_len, int n_q_heads, int n_kv_heads, int head_d
   const size_t stage_bytes = rows8 ? q4d::kR8StageBytes : q4d::tca_stage_bytes(q8);
   // One CTA per SM (the K/V ring takes most of shared memory): enough context
   // splits that (splits x KV heads x row groups) fills the SMs once, each
-  // split at least two tiles long (one for the warp-local kernel, whose
-  // splits merge in the same launch) and at most 256 splits (the merge
-  // kernel's limit).
+  // split at least two tiles long and at most 256 splits (the merge kernel's
+  // limit).
   const long long ctas_per_split = (long long)n_kv_heads * row_groups;
   int n_splits = int(std::max<long long>(1, (num_sms + ctas_per_split - 1) / ctas_per_split));
-  n_splits = std::min(n_splits, std::max(1, ceil_div(ctx_len, rows8 ? TT : 2 * TT)));
+  n_splits = std::min(n_splits, std::max(1, ceil_div(ctx_len, 2 * TT)));
   n_splits = std::min(n_splits, 256);
   const int split_tokens = int(round_up(ceil_div(ctx_len, n_splits), TT));
   n_splits = ceil_div(ctx_len, split_tokens);
