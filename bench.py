@@ -577,8 +577,7 @@ class DecodeStep:
         self.n_gemv = len(jobs)
         self.batch = q4dec.GemvBatch(jobs)
         self.aws = self.L.q4d_attn_workspace_bytes(CTX, N_Q, N_KV, HEAD_DIM, M)
-        # zero-filled: the split counters of the one-launch merge start at 0
-        self.attn_ws = torch.zeros(max(self.aws, 16), dtype=torch.uint8, device=dev)
+        self.attn_ws = torch.empty(max(self.aws, 16), dtype=torch.uint8, device=dev)
         # GEMV workspace: zero-filled once, every launch leaves it so
         self.gemv_ws = torch.zeros(max(16, max(self.L.q4d_gemv_workspace_bytes(M, N, K)
                                                for N, K in LAYER_SHAPES + [(HEAD_N, HIDDEN)])),
@@ -668,7 +667,7 @@ def per_call_table(torch, L, dev, layers, kv, peak_gbs, reps=15):
                 for c in (4096, 65536, CTX)] +
                [L.q8kv_attn_workspace_bytes(c, N_Q, N_KV, HEAD_DIM, M) for M in (1, 5)
                 for c in (65536, CTX)] + [16])
-    ws = torch.zeros(need, dtype=torch.uint8, device=dev)  # attention: kept zero by each call
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     sptr = stream.cuda_stream
     table = {"gemv": [], "attn": [], "l2": "flushed before every call (252 MB read)"}
@@ -872,7 +871,7 @@ def run_case(args, torch, dev):
                   for i in range(copies)]
         Q = synth.device_bf16_normal(2, (M, N_Q, HEAD_DIM), scale=1 / 16, device=dev)
         out = torch.empty((M, N_Q, HEAD_DIM), dtype=torch.float32, device=dev)
-        ws = torch.zeros(max(16, wsfn(ctx, N_Q, N_KV, HEAD_DIM, M)), dtype=torch.uint8,
+        ws = torch.empty(max(16, wsfn(ctx, N_Q, N_KV, HEAD_DIM, M)), dtype=torch.uint8,
                          device=dev)
         for i in range(args.launches):
             Kc, Vc = caches[i % copies]

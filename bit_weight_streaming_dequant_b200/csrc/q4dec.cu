@@ -347,11 +347,6 @@ q4d_status launch_attn_tc(const q4d::AttnArgs& a, const q4d_attn_plan& p, int n_
 // with 32 MMA columns, whose shared memory holds only one next to two stages.
 int tca_pbufs(int nr, bool q8) { return (q8 && nr == 32) ? 1 : 2; }
 
-// Attention workspace: a header of split counters (4-byte, one per KV head and
-// row group; zero at rest) at a fixed offset, so that no call of another shape
-// or variant ever writes split states over them, then the split states.
-constexpr size_t kAttnCounterBytes = 4096;
-
 q4d_status plan_attn_impl(int ctx_len, int n_q_heads, int n_kv_heads, int head_dim, int M,
                           int num_sms, bool q8, q4d_attn_plan* plan);
 
@@ -386,10 +381,8 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
   a.K = static_cast<const uint8_t*>(Kq4);
   a.V = static_cast<const uint8_t*>(Vq4);
   a.out = out;
-  if (p.n_splits > 1) {  // the counter header, then the split states
-    a.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kAttnCounterBytes);
-    a.ws_ml = a.ws_o + size_t(p.n_splits) * M * n_q * 256;
-  }
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_ml = a.ws_o ? a.ws_o + size_t(p.n_splits) * M * n_q * 256 : nullptr;
   a.err = s->err;
   a.ctx_len = ctx_len;
   a.n_q = n_q;
@@ -403,13 +396,7 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
   a.rows_per_cta = p.rows_per_cta;
   a.stages = p.stages;
 
-  const bool rows8 = !q8 && p.rows_per_cta <= 8;
-  // the warp-local kernel merges in the same launch (its last split per KV
-  // head and row group), counting in the workspace header
-  const bool one_launch =
-      rows8 && p.n_splits > 1 && size_t(n_kv) * p.row_groups * 4 <= kAttnCounterBytes;
-  if (one_launch) a.merge_cnt = static_cast<unsigned*>(workspace);
-  if (rows8)
+  if (!q8 && p.rows_per_cta <= 8)
     st = launch_attn_rows8(a, p, n_kv, dev, *s, stream);
   else if (p.rows_per_cta <= 16)
     st = q8 ? launch_attn_tc<16, true, 2>(a, p, n_kv, dev, *s, stream)
@@ -418,7 +405,7 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
     st = q8 ? launch_attn_tc<32, true, 1>(a, p, n_kv, dev, *s, stream)
             : launch_attn_tc<32, false, 2>(a, p, n_kv, dev, *s, stream);
   if (st != Q4D_OK) return st;
-  if (p.n_splits > 1 && !one_launch) {
+  if (p.n_splits > 1) {
     // the merge may launch while the split kernel runs; it waits for it on
     // the device (griddepcontrol.wait) before reading the split states
     cudaLaunchConfig_t cfg;
@@ -526,11 +513,8 @@ q4d_status plan_attn_impl(int ctx_len, int n_q_heads, int n_kv_heads, int head_d
   plan->threads = rows8 ? q4d::kR8Threads : q4d::kTcaThreads;
   plan->smem_bytes =
       rows8 ? q4d::attn_rows8_smem_bytes(stages) : q4d::tca_smem_bytes(nr, stages, q8, pb);
-  // a fixed header of split counters (used by the one-launch merge), then
-  // the split states
   plan->workspace_bytes =
-      n_splits > 1 ? kAttnCounterBytes + size_t(n_splits) * M * n_q_heads * (q4d::kHeadDim + 2) * 4
-                   : 0;
+      n_splits > 1 ? size_t(n_splits) * M * n_q_heads * (q4d::kHeadDim + 2) * 4 : 0;
   return Q4D_OK;
 }
 

@@ -48,8 +48,6 @@ struct AttnArgs {
   float* out;          // [M][n_q][256]
   float* ws_o;         // [n_splits][M*n_q][256]
   float* ws_ml;        // [n_splits][M*n_q][2] (running max in log2 units, sum)
-  unsigned* merge_cnt; // [n_kv][row groups] splits finished, zero between launches;
-                       // set: the split kernel merges (the last split to finish)
   unsigned* err;
   int ctx_len, n_q, n_kv, M, g, kv_stride;
   float scale_log2;    // softmax scale * log2(e)
@@ -156,7 +154,7 @@ constexpr uint32_t kR8StageBytes = 2u * kR8Tile * kRowBytes;   // K tile + V til
 
 // Shared memory of the warp-local variant: the ring (which also holds the
 // final cross-warp combine, 96 KB), Q fragments of 8 rows, per-warp and
-// per-row statistics, barriers, the abort and last-split flags (padded to 16).
+// per-row statistics, barriers, the abort flag (padded to 16).
 __host__ __device__ constexpr size_t attn_rows8_smem_bytes(int stages) {
   return size_t(stages) * kR8StageBytes + 8 * kR8QPitch + size_t(kR8Warps) * 8 * 2 * 4 +
          8 * 2 * 4 + size_t(stages) * 16 + 16;
@@ -184,7 +182,6 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
   // set by the first wait that times out: from then on no wait blocks and no
   // further copy is issued (the results are void; the error word says so)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + S);
-  volatile int* last_flag = abort_flag + 1;  // this CTA merges the splits
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x, kh = blockIdx.y, rgrp = blockIdx.z;
@@ -452,56 +449,6 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
         a.ws_ml[(size_t(split) * rows_total + row) * 2 + 1] = rml[r * 2 + 1];
       }
     }
-  }
-  if (a.n_splits == 1 || a.merge_cnt == nullptr) return;
-  // ---- The last split of this (KV head, row group) to finish merges the
-  // states of all splits (log-sum-exp, base 2) into out: each CTA's state
-  // writes, a release fence, its count; the last one, after an acquire fence,
-  // reads them all and sets the count back to zero for the next launch.
-  __threadfence();
-  __syncthreads();
-  unsigned* cnt = a.merge_cnt + size_t(kh) * gridDim.z + rgrp;
-  if (tid == 0) *last_flag = atomicAdd(cnt, 1u) == unsigned(a.n_splits - 1);
-  __syncthreads();
-  if (!*last_flag) return;
-  __threadfence();
-  if (tid == 0) *cnt = 0u;
-  const int n = a.n_splits;
-  // per row (one warp each): the maximum over the splits and the total weight
-  if (warp < R) {
-    const int rr = row0 + warp, m = rr / a.g, j = rr - m * a.g;
-    const size_t row = size_t(m) * a.n_q + kh * a.g + j;
-    float mx = -INFINITY;
-    for (int c = lane; c < n; c += 32) mx = fmaxf(mx, __ldcg(a.ws_ml + (c * rows_total + row) * 2));
-    #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-    float L = 0.f;
-    for (int c = lane; c < n; c += 32) {
-      const float mc = __ldcg(a.ws_ml + (c * rows_total + row) * 2);
-      if (mc != -INFINITY) L += __ldcg(a.ws_ml + (c * rows_total + row) * 2 + 1) * ex2(mc - mx);
-    }
-    #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, off);
-    if (lane == 0) {
-      rml[warp * 2 + 0] = mx;
-      rml[warp * 2 + 1] = L;
-    }
-  }
-  __syncthreads();
-  // every output element: the splits' vectors weighted, in split order
-  for (int i = tid; i < R * kHeadDim; i += kR8Threads) {
-    const int r = i / kHeadDim, dim = i - r * kHeadDim;
-    const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
-    const size_t row = size_t(m) * a.n_q + kh * a.g + j;
-    const float mx = rml[r * 2 + 0];
-    float acc = 0.f;
-    #pragma unroll 4
-    for (int c = 0; c < n; ++c) {
-      const float mc = __ldcg(a.ws_ml + (c * rows_total + row) * 2);
-      const float v = __ldcg(a.ws_o + (c * rows_total + row) * kHeadDim + dim);
-      acc = fmaf(mc == -INFINITY ? 0.f : ex2(mc - mx), v, acc);
-    }
-    a.out[row * kHeadDim + dim] = acc / rml[r * 2 + 1];
   }
 }
 

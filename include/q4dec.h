@@ -258,16 +258,6 @@ q4d_status q4_gemv_batch_ex(const void* desc_host, void* desc_dev, void* stream,
  * rules as q4_gemv).  The _ex form takes all of them explicitly and never
  * allocates; workspace must hold q4d_attn_workspace_bytes(...) bytes.
  *
- * The context is cut into splits whose softmax states go to the workspace
- * and are merged by log-sum-exp.  With at most 8 query rows per KV head and
- * CTA (the warp-local kernel) the last split of a KV head to finish merges
- * them in the same launch, counting the finished splits in the workspace's
- * first 4 KB (the split states follow, for every variant): the workspace must
- * be zero-filled before its first use, and every launch that returns Q4D_OK
- * with the device error word at 0 leaves those counters at zero again (as for
- * q4_gemv_ex; re-zero it after a reported error).  More rows per CTA take a
- * second, dependent launch for the merge.
- *
  * Supported value range (the same for every M and both cache formats): the
  * kernels feed Q and the dequantised K/V values to the tensor cores as IEEE
  * fp16, so

@@ -142,29 +142,3 @@ def test_plain_entry_point(cuda_ok):
     torch.cuda.synchronize()
     assert st == 0
     assert_attn_close(out, ref, "plain entry")
-
-
-@pytest.mark.parametrize("ctx,n_q,n_kv,M", [(4096, 24, 4, 1), (65536, 24, 4, 1), (3000, 8, 1, 1)])
-def test_one_launch_merge_keeps_its_counters_zero(cuda_ok, ctx, n_q, n_kv, M):
-    # with at most 8 query rows per KV head and CTA the last split to finish
-    # merges in the same launch, counting finished splits in the first 4 KB of
-    # the caller's zero-filled workspace: the counts are back at zero after
-    # every call, repeated calls are bit-identical and match the oracle
-    p = q4dec.plan_attn(ctx, n_q, n_kv, 256, M, torch.cuda.get_device_properties(0).multi_processor_count)
-    assert p.rows_per_cta <= 8 and p.n_splits > 1
-    L = q4dec.lib()
-    need = L.q4d_attn_workspace_bytes(ctx, n_q, n_kv, 256, M)
-    states = p.n_splits * M * n_q * 258 * 4
-    assert need == 4096 + states
-    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
-    Q, K, V = _case(900 + ctx, ctx, n_q, n_kv, M)
-    Qd, Kd, Vd = dev_bf16(Q.reshape(M, n_q, 256)), dev_bytes(K), dev_bytes(V)
-    outs = []
-    for _ in range(3):
-        outs.append(q4dec.q4kv_attn_decode(Qd, Kd, Vd, ctx_len=ctx, n_kv_heads=n_kv, workspace=ws))
-        torch.cuda.synchronize()
-        assert int(torch.count_nonzero(ws[:4096])) == 0
-    assert all(torch.equal(o, outs[0]) for o in outs)
-    ref = oracle.attn_decode(Q, K, V, ctx, n_q, n_kv, 256, M)
-    assert_attn_close(outs[0], ref, f"one-launch merge ctx={ctx} M={M}")
-    assert q4dec.device_error() == 0

@@ -114,7 +114,7 @@ def test_decode_layer_calls_replay_as_one_cuda_graph(cuda_ok):
 
     def buffers():
         L = q4dec.lib()
-        ws = {"attn": torch.zeros(max(16, L.q4d_attn_workspace_bytes(ctx, n_q, n_kv, 256, M)),
+        ws = {"attn": torch.empty(max(16, L.q4d_attn_workspace_bytes(ctx, n_q, n_kv, 256, M)),
                                   dtype=torch.uint8, device=dev),
               # GEMV workspaces: zero-filled before first use
               "o": torch.zeros(max(16, L.q4d_gemv_workspace_bytes(M, hid, n_q * 256)),

@@ -369,7 +369,7 @@ def _tc_layout_checks(nr):
     assert sorted(dims) == list(range(256))
 
 
-def _attn_q_and_workspace(p, M, nq, nkv, g, q8=False):
+def _attn_q_and_workspace(p, M, nq, nkv, g):
     # Q reads (global, 8-byte vectors) stay inside [M][n_q][256]
     q_elems = M * nq * 256
     for kh in range(nkv):
@@ -381,15 +381,10 @@ def _attn_q_and_workspace(p, M, nq, nkv, g, q8=False):
                 for t in range(4):
                     e = row * 256 + b * 32 + 4 * t
                     assert e % 4 == 0 and e + 16 + 4 <= q_elems
-    # workspace: a fixed 4 KB header of split counters (one per KV head and row
-    # group, used by the warp-local kernel's one-launch merge), then the split
-    # outputs and (max, sum) pairs
+    # workspace: split outputs then (max, sum) pairs
     nrows = M * nq
     if p.n_splits > 1:
-        states = p.n_splits * nrows * 258 * 4
-        assert p.workspace_bytes == 4096 + states
-        if p.rows_per_cta <= 8 and not q8:
-            assert nkv * p.row_groups * 4 <= 4096
+        assert p.workspace_bytes == p.n_splits * nrows * 258 * 4
     else:
         assert p.workspace_bytes == 0
 
@@ -507,7 +502,7 @@ def test_attn_q8_geometry(ctx, nq, nkv, M, stride_extra):
     for col in range(0, ROW_Q8, 16):
         assert len(_chunks([r * ROW_Q8 + col for r in range(8)])) == 8
     _tc_layout_checks(nr)
-    _attn_q_and_workspace(p, M, nq, nkv, g, q8=True)
+    _attn_q_and_workspace(p, M, nq, nkv, g)
     assert p.workspace_bytes == q4dec.lib().q8kv_attn_workspace_bytes(ctx, nq, nkv, 256, M) or \
         sms != 148
 
