@@ -47,12 +47,13 @@
 //    clearing keeps replays of a captured launch (same tag) correct.
 //  * Several matrices ("jobs") can run in one launch.  The producer keeps
 //    streaming the next job's weights (they depend on nothing) while a job's
-//    activations wait for the job they depend on: whoever writes a row block's
-//    final values counts it on a per-job counter, and a job's activation
-//    copies are issued only once its prerequisite's count has reached that
-//    job's number of row blocks.  These counters live in the launch
-//    descriptor, which the host hands over zeroed; the last CTA to leave the
-//    launch sets them back to zero.
+//    activations wait for the job they depend on: whichever epilogue warp
+//    writes half of a row block in final form counts it on a per-job counter
+//    (a release reduction), and a job's activation copies are issued only
+//    once its prerequisite's count has reached twice that job's number of row
+//    blocks (an acquire load).  These counters live in the launch descriptor,
+//    which the host hands over zeroed; the last CTA to leave the launch sets
+//    them back to zero.
 //  * Weights are stored super-block-column-major: the 128 rows of a row block
 //    are one contiguous piece of each column, so a unit is two bulk copies of
 //    18 KB plus one copy of each activation row's 1 KB, issued by a producer
@@ -100,10 +101,15 @@ constexpr uint32_t kGemvWBox = kGemvRows * kSbBytes;       // one column of a ro
 constexpr uint32_t kJobOutBf16 = 1u;                       // y stored as bf16 (RNE)
 constexpr uint32_t kJobSwiglu = 2u;                        // rows are gate / up pairs
 
+// Activation rows of a stage: two columns (1 KB) each, at a pitch of 1056
+// bytes, so that the fragment loads of up to 8 rows (lanes g = row) fall on
+// distinct banks.
+constexpr uint32_t kGemvXPitch = kGemvCols * 512u + 32u;
 // One pipeline stage: the unit's two weight pieces, then M activation rows of
-// two columns (1 KB each, the second half unused when the unit has one column).
+// two columns (the second half unused when the unit has one column), rounded
+// up to 128 bytes.
 __host__ __device__ constexpr uint32_t gemv_stage_bytes(int M) {
-  return kGemvCols * kGemvWBox + uint32_t(M) * kGemvCols * 512u;
+  return (kGemvCols * kGemvWBox + uint32_t(M) * kGemvXPitch + 127u) / 128u * 128u;
 }
 // Reduction buffers (consumers -> epilogue): two for M <= 2, one otherwise
 // (shared memory), each 16 warp slots of [M][kGemvRedStride] fp32.
@@ -508,7 +514,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
       const int kc = min(kGemvCols, xs.nsb - col0);
       #pragma unroll
       for (int m = 0; m < M; ++m)
-        bulk_g2s_nohint(dst + uint32_t(m) * (kGemvCols * 512u),
+        bulk_g2s_nohint(dst + uint32_t(m) * kGemvXPitch,
                         xs.x + (size_t(m) * xs.nsb + col0) * 256, uint32_t(kc) * 512u, bar);
       ++stx;
       if (++x_slot == S) x_slot = 0;
@@ -564,7 +570,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
       const int col0 = 2 * xs.cp;
       const int kc = min(kGemvCols, xs.nsb - col0);
       for (int m = 0; m < M; ++m)
-        bulk_g2s_nohint(dst + uint32_t(m) * (kGemvCols * 512u),
+        bulk_g2s_nohint(dst + uint32_t(m) * kGemvXPitch,
                         xs.x + (size_t(m) * xs.nsb + col0) * 256, uint32_t(kc) * 512u, bar);
       if (++x_slot == S) x_slot = 0;
       cursor_next(xs, a);
@@ -643,7 +649,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
   const int g = lane >> 2, t = lane & 3;
   const int task_col = warp >> 3, task_blk = warp & 7;
   const uint32_t mask = 0x000F000Fu, magic = 0x43004300u, c136 = 0x43084308u;  // bf16 136
-  const uint32_t x_lane = kXOff + g * (kGemvCols * 512) + task_col * 512 + (task_blk * 32 + 4 * t) * 2;
+  const uint32_t x_lane = kXOff + g * kGemvXPitch + task_col * 512 + (task_blk * 32 + 4 * t) * 2;
   const uint32_t w_lane = task_col * kGemvWBox + g * kSbBytes + task_blk * 16 + t * 4;
   const uint32_t d_lane = task_col * kGemvWBox + g * kSbBytes + 128 + task_blk * 2;
   int slot = 0, seg = 0;

@@ -191,10 +191,13 @@ size_t q4d_gemv_workspace_bytes(int M, int N, int K);
  *               the stream has completed (every job can use -1 when no job of
  *               the batch writes another job's x);
  *               j (0 <= j < this job's index) -- x is read only after job j
- *               and every job before it have written their outputs, e.g. x is
- *               job j's y.
+ *               has written all of its output, e.g. x is job j's y.  Only job
+ *               j is waited for: a job that reads the outputs of several
+ *               earlier jobs needs them ordered by a chain of waits (job j
+ *               itself waiting, directly or through others, for the rest).
  *   Each job must also not overwrite an x or y that an earlier job, not yet
- *   finished, still uses: give it a wait_for at least as late as that job.
+ *   finished, still uses: make it wait, directly or through a chain of
+ *   waits, for that job.
  *
  *   q4d_gemv_batch_desc_bytes(n_jobs): bytes of the launch descriptor.
  *   q4d_gemv_batch_prepare: host only (no CUDA call).  Validates every job as
@@ -205,15 +208,16 @@ size_t q4d_gemv_workspace_bytes(int M, int N, int K);
  *   q4_gemv_batch_ex: launches the batch on `stream`.  desc_host is the
  *     prepared host buffer, desc_dev a byte-for-byte copy of it in device
  *     memory (16-byte aligned): copy it once, launch many times.  Its tail
- *     holds the per-job completion counters (row blocks written), zero as
- *     prepared; a launch counts on them and sets them back to zero before it
- *     ends, so launches that may
- *     overlap on the GPU must not share a descriptor copy, and a copy must not
- *     be rewritten while a launch may run.  num_sms
+ *     holds the per-job completion counters (row-block halves written in
+ *     final form), zero as prepared; a launch counts on them and sets them
+ *     back to zero before it ends, so launches that may overlap on the GPU
+ *     must not share a descriptor copy, and a copy must not be rewritten while
+ *     a launch may run.  num_sms
  *     must be the current device's SM count, else Q4D_ERR_INVALID_ARG.
  *     workspace: device memory of at least *workspace_bytes (16-byte aligned;
  *     zero-filled before first use and kept so, as for q4_gemv_ex; launches
- *     that may overlap on the GPU must not share it), else Q4D_ERR_WORKSPACE.  flags: 0 or
+ *     that may overlap on the GPU must not share it), else
+ *     Q4D_ERR_WORKSPACE.  flags: 0 or
  *     Q4D_GEMV_WEIGHT_PREFETCH (as q4_gemv_ex2: the first weights stream while
  *     the previous kernel on the stream still runs).  Never allocates; the
  *     launch can be captured into a CUDA graph and replayed.

@@ -16,8 +16,11 @@ GEMV_ROWS, GEMV_COLS, GEMV_WARPS, GEMV_THREADS = 128, 2, 16, 608
 GEMV_WBOX = GEMV_ROWS * 144
 
 
+GEMV_XPITCH = GEMV_COLS * 512 + 32   # activation rows of a stage: 1 KB at a 1056-byte pitch
+
+
 def _gemv_stage_bytes(M):
-    return GEMV_COLS * GEMV_WBOX + M * GEMV_COLS * 512
+    return -(-(GEMV_COLS * GEMV_WBOX + M * GEMV_XPITCH) // 128) * 128
 
 
 def _unit_begin(c, U, G):
@@ -96,7 +99,8 @@ def test_gemv_geometry(M, N, K, sms):
             for m in range(M):
                 xsrc = (m * nsb + col0) * 256 * 2
                 assert xsrc % 16 == 0 and xsrc + kc * 512 <= x_bytes
-                assert GEMV_COLS * GEMV_WBOX + m * 1024 + kc * 512 <= stage
+                dst = GEMV_COLS * GEMV_WBOX + m * GEMV_XPITCH
+                assert dst % 16 == 0 and dst + kc * 512 <= stage
     # per-warp shared-memory reads stay inside the stage: weights (rows g and
     # g + 8 of 8 tiles), scales, activations (column g < M)
     for warp in range(GEMV_WARPS):
@@ -108,12 +112,21 @@ def test_gemv_geometry(M, N, K, sms):
                 pd = col * GEMV_WBOX + g * 144 + 128 + blk * 2
                 assert pd + (16 * 7 + 8) * 144 + 2 <= (col + 1) * GEMV_WBOX
                 if g < M:
-                    xo = GEMV_COLS * GEMV_WBOX + g * 1024 + col * 512 + (blk * 32 + 4 * t) * 2
-                    assert xo + 32 + 8 <= stage
+                    xo = GEMV_COLS * GEMV_WBOX + g * GEMV_XPITCH + col * 512 + (blk * 32 + 4 * t) * 2
+                    assert xo % 8 == 0 and xo + 32 + 8 <= stage
     # bank pattern of the A-word loads: 32 lanes (g, t) read row g, word t at a
     # 144-byte pitch
     banks = {((g * 144 + 4 * t) // 4) % 32 for g in range(8) for t in range(4)}
     assert len(banks) == 32
+    # activation fragment loads (8 bytes per lane, a half-warp per pass): the
+    # rows g < M of either half-warp hit distinct banks
+    for half in (range(0, 4), range(4, 8)):
+        for col in range(2):
+            for blk in range(8):
+                words = [(GEMV_COLS * GEMV_WBOX + g * GEMV_XPITCH + col * 512 +
+                          (blk * 32 + 4 * t) * 2) // 4 + i
+                         for g in half if g < M for t in range(4) for i in range(2)]
+                assert len({w % 32 for w in words}) == len(words)
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 17408, 5120), (3, 5120, 17408), (2, 6144, 5120),
