@@ -223,3 +223,66 @@ def test_wait_selftest_rejects_bad_arguments_without_cuda():
     assert L.q4d_wait_selftest(FAKE, 0, 0, None) == 1
     assert L.q4d_wait_selftest(FAKE, 10_000_001, 0, None) == 1
     assert L.q4d_wait_selftest(FAKE + 2, 1000, 0, None) == 3
+
+
+def _contributors(rbs, upr, U, G):
+    slots = 0
+    for rb in range(rbs):
+        first = ((rb * upr + 1) * G - 1) // U
+        last = ((rb * upr + upr) * G - 1) // U
+        if last > first:
+            slots = max(slots, last - first + 1)
+    return slots
+
+
+@pytest.mark.parametrize("M,sms", [(1, 148), (5, 148), (3, 132)])
+def test_gemv_batch_descriptor_matches_the_planning_model(M, sms):
+    # a decode-like batch (two layers of gate, up, down, in, out; a fused gate /
+    # up job; a tiny job) prepared on the host and read back field by field:
+    # header, then one job descriptor per job (pointers, rows, K / 256, flags,
+    # wait_for, row blocks, units per row block, units, CTAs, partial slots,
+    # rotation, partial-slot offset), against a plain model of the partition
+    import struct
+    shapes = [(17408, 5120, 0), (17408, 5120, 0), (5120, 17408, 0), (6144, 5120, 0),
+              (5120, 6144, 0)] * 2 + [(1024, 5120, q4dec.GEMV_SWIGLU), (37, 256, 2)]
+    n = len(shapes)
+    jobs = (q4dec.GemvJob * n)()
+    for i, (N, K, fl) in enumerate(shapes):
+        jobs[i] = q4dec.GemvJob(FAKE + 16 * i, FAKE + 32 * i, FAKE + 64 * i, N, K, fl, i - 1)
+    L = q4dec.lib()
+    nbytes = L.q4d_gemv_batch_desc_bytes(n)
+    buf = ctypes.create_string_buffer(nbytes)
+    ws = ctypes.c_size_t(0)
+    assert L.q4d_gemv_batch_prepare(jobs, n, M, sms, buf, nbytes, ctypes.byref(ws)) == 0
+    raw = buf.raw
+    magic, n_jobs, M_h, sms_h, grid = struct.unpack_from("<Iiiii", raw, 0)
+    assert (n_jobs, M_h, sms_h) == (n, M, sms) and magic != 0
+    (ws_bytes,) = struct.unpack_from("<Q", raw, 24)
+    assert ws_bytes == ws.value
+    model, units_before, entries, launch_grid = [], 0, 0, 1
+    for N, K, fl in shapes:
+        rows = 2 * N if fl & q4dec.GEMV_SWIGLU else N
+        rbs, upr = -(-rows // 128), -(-(K // 256) // 2)
+        launch_grid = max(launch_grid, min(sms, rbs * upr))
+    assert grid == launch_grid
+    for i, (N, K, fl) in enumerate(shapes):
+        rows = 2 * N if fl & q4dec.GEMV_SWIGLU else N
+        rbs, upr = -(-rows // 128), -(-(K // 256) // 2)
+        U = rbs * upr
+        G = min(launch_grid, U)
+        slots = _contributors(rbs, upr, U, G)
+        off = 64 + i * 80
+        W, x, y, part_off = struct.unpack_from("<QQQq", raw, off)
+        (Nd, nsb, flags, wait_for, rbs_d, upr_d, units, G_d, slots_d, _, rot, _) = \
+            struct.unpack_from("<12i", raw, off + 32)
+        assert (W, x, y) == (FAKE + 16 * i, FAKE + 32 * i, FAKE + 64 * i)
+        assert (Nd, nsb, wait_for) == (rows, K // 256, i - 1)
+        assert bool(flags & 2) == bool(fl & q4dec.GEMV_SWIGLU) and bool(flags & 1) == bool(fl & 2)
+        assert (rbs_d, upr_d, units, G_d, slots_d) == (rbs, upr, U, G, slots)
+        assert rot == units_before % launch_grid
+        assert part_off == entries
+        units_before += U
+        entries += rbs * slots * M * 128 if slots else 0
+    assert ws.value == entries * 8
+    # the completion counters after the jobs are zero as prepared
+    assert set(raw[64 + n * 80:nbytes]) == {0}
