@@ -141,3 +141,36 @@ def test_batch_replays_as_a_cuda_graph(cuda_ok):
             assert torch.equal(j["y"], eager[i]), f"replay job {i}"
     del g
     assert q4dec.device_error() == 0
+
+
+def test_wait_for_orders_a_write_after_an_earlier_jobs_read(cuda_ok):
+    # job 0 reads x0; job 2 (no data dependence on job 0) writes its output
+    # into x0's memory and waits for job 0, so job 0 must still see the old x0;
+    # job 1 is independent and runs in between; job 3 waits for job 1, two jobs
+    # back
+    M, K = 2, 5120
+    x0 = dev_bf16(synth.activations(800, M, K))
+    x0_copy = x0.clone()
+    x1 = dev_bf16(synth.activations(801, M, K))
+    W = [_weights(810 + i, 5120, K, device_gen=True) for i in range(4)]
+    y = [torch.empty((M, 5120), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
+    jobs = [dict(W=W[0], x=x0, y=y[0], N=5120, K=K),
+            dict(W=W[1], x=x1, y=y[1], N=5120, K=K),
+            dict(W=W[2], x=x1, y=x0, N=5120, K=K, wait_for=0),   # overwrites job 0's input
+            dict(W=W[3], x=y[1], y=y[3], N=5120, K=K, wait_for=1)]
+    ref0 = q4dec.q4_gemv(W[0], x0_copy, N=5120, K=K, out_dtype=torch.bfloat16)
+    ref1 = q4dec.q4_gemv(W[1], x1, N=5120, K=K, out_dtype=torch.bfloat16)
+    ref2 = q4dec.q4_gemv(W[2], x1, N=5120, K=K, out_dtype=torch.bfloat16)
+    ref3 = q4dec.q4_gemv(W[3], ref1, N=5120, K=K, out_dtype=torch.bfloat16)
+    b = q4dec.GemvBatch(jobs)
+    for launch in range(3):
+        x0.copy_(x0_copy)
+        for t in y:
+            t.fill_(float("nan"))
+        torch.cuda.synchronize()
+        b.run()
+        torch.cuda.synchronize()
+        assert torch.equal(y[0], ref0), f"launch {launch}: job 0 saw the later x0"
+        assert torch.equal(y[1], ref1) and torch.equal(x0, ref2) and torch.equal(y[3], ref3), launch
+        assert int(torch.count_nonzero(b.workspace)) == 0
+    assert q4dec.device_error() == 0
