@@ -631,22 +631,42 @@ class DecodeStep:
         # the step's inputs (the activation rows of each width, every attention
         # layer's queries) come from pinned host memory; its results (the last
         # output of each matrix type, the logits, every attention output) go
-        # back to it; the kernels are the timed step's
+        # back to it; the kernels are the timed step's.  As a decode loop would,
+        # the copies that nothing waits for run on a second stream beside the
+        # kernels: the queries go up while the weight stream runs, the GEMV
+        # results and each attention layer's output come down while the next
+        # layers run; the step ends when both streams have finished (every
+        # copy is inside the timed region).
+        torch = self.torch
+        main = torch.cuda.current_stream()
+        if not hasattr(self, "side"):
+            self.side = torch.cuda.Stream(device=main.device)
+        side = self.side
         self.h2d = self.d2h = 0
         for K in self.xs:
             self.xs[K].copy_(self.h_x[K], non_blocking=True)
             self.h2d += self.xs[K].numel() * 2
-        for q, h in zip(self.Qs, self.h_q):
-            q.copy_(h, non_blocking=True)
-            self.h2d += q.numel() * 2
+        side.wait_stream(main)      # after the previous step, inside this one
+        with torch.cuda.stream(side):
+            for q, h in zip(self.Qs, self.h_q):
+                q.copy_(h, non_blocking=True)
+                self.h2d += q.numel() * 2
+        q_ready = side.record_event()
         self.gemv_stream()
-        self.attn_stream()
-        for n, y in self.ys.items():
-            self.h_y[n].copy_(y, non_blocking=True)
-            self.d2h += y.numel() * 4
-        for o, h in zip(self.outs, self.h_o):
-            h.copy_(o, non_blocking=True)
+        gemv_done = main.record_event()
+        side.wait_event(gemv_done)
+        with torch.cuda.stream(side):
+            for n, y in self.ys.items():
+                self.h_y[n].copy_(y, non_blocking=True)
+                self.d2h += y.numel() * y.element_size()
+        main.wait_event(q_ready)
+        for l, (o, h) in enumerate(zip(self.outs, self.h_o)):
+            self.attn(l)
+            side.wait_event(main.record_event())   # layer l's output is written
+            with torch.cuda.stream(side):
+                h.copy_(o, non_blocking=True)
             self.d2h += o.numel() * 4
+        main.wait_stream(side)      # the step ends with both streams
 
 
 def per_call_table(torch, L, dev, layers, kv, peak_gbs, reps=15):
