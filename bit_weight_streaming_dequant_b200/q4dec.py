@@ -377,10 +377,14 @@ class GemvBatch:
     ``jobs``: list of dicts with keys ``W`` (uint8 weights), ``x`` (bf16
     [M][K]), ``y`` (fp32 or bf16 output [M][N]), ``N``, ``K`` and optional
     ``swiglu`` (W holds 2N interleaved gate / up rows, y = h [M][N]) and
-    ``wait_for`` (-1, or the index of the job whose outputs, and those of every
-    job before it, must be written before this job reads x).  All tensors must
-    stay alive and in place for as long as the batch is used.  The descriptor
-    is prepared and copied to the device once; :meth:`run` only launches."""
+    ``wait_for`` (-1, or the index of the job whose output must be written
+    before this job reads x; only that job is waited for, so jobs depending on
+    several earlier ones, or overwriting memory an earlier job reads, need a
+    chain of waits).  All tensors must stay alive and in place for as long as
+    the batch is used.  The descriptor is prepared and copied to the device
+    once; :meth:`run` only launches.  The workspace is allocated zero-filled,
+    and every successful launch leaves it so (if a launch reports a device
+    error, zero it again before the next)."""
 
     def __init__(self, jobs, *, device=None):
         torch = _torch()
