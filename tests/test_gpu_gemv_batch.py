@@ -174,3 +174,43 @@ def test_wait_for_orders_a_write_after_an_earlier_jobs_read(cuda_ok):
         assert torch.equal(y[1], ref1) and torch.equal(x0, ref2) and torch.equal(y[3], ref3), launch
         assert int(torch.count_nonzero(b.workspace)) == 0
     assert q4dec.device_error() == 0
+
+
+def test_ffn_chain_in_one_launch(cuda_ok):
+    # the feed-forward block as a batch: fused gate / up + SwiGLU writing bf16 h,
+    # then the down projection reading h (waits for it); beside them a fused
+    # job whose 2N = 2000 rows end in a ragged row block of gate / up pairs
+    for M in (1, 4):
+        hid, ffn = 1024, 2048
+        Wgu = _weights(830, 2 * ffn, hid)
+        Wdn = _weights(831, hid, ffn)
+        Wr = _weights(832, 2 * 1000, hid)
+        x = dev_bf16(synth.activations(833 + M, M, hid))
+        h = torch.empty((M, ffn), dtype=torch.bfloat16, device="cuda")
+        y = torch.empty((M, hid), device="cuda")
+        hr = torch.empty((M, 1000), device="cuda")
+        b = q4dec.GemvBatch([dict(W=Wgu, x=x, y=h, N=ffn, K=hid, swiglu=True),
+                             dict(W=Wr, x=x, y=hr, N=1000, K=hid, swiglu=True),
+                             dict(W=Wdn, x=h, y=y, N=hid, K=ffn, wait_for=0)])
+        h_ref = q4dec.q4_gemv_swiglu(Wgu, x, N=ffn, K=hid, out_dtype=torch.bfloat16)
+        hr_ref = q4dec.q4_gemv_swiglu(Wr, x, N=1000, K=hid)
+        y_ref = q4dec.q4_gemv(Wdn, h_ref, N=hid, K=ffn)
+        for launch in range(2):
+            for t in (h, y, hr):
+                t.fill_(float("nan"))
+            b.run(weight_prefetch=bool(launch))
+            torch.cuda.synchronize()
+            assert torch.equal(h, h_ref) and torch.equal(hr, hr_ref), (M, launch)
+            assert torch.equal(y, y_ref), (M, launch)
+            assert int(torch.count_nonzero(b.workspace)) == 0
+    # the ragged job against the oracle's SwiGLU bound
+    Wr_np = synth.q4_0_weights(840, 2 * 1000, 1024)
+    xr_np = synth.activations(841, 2, 1024)
+    hr2 = torch.empty((2, 1000), device="cuda")
+    q4dec.GemvBatch([dict(W=dev_bytes(Wr_np), x=dev_bf16(xr_np), y=hr2, N=1000, K=1024,
+                          swiglu=True)]).run()
+    torch.cuda.synchronize()
+    h_o, tol = oracle.gemv_swiglu(Wr_np, xr_np, 2, 1000, 1024)
+    err = np.abs(hr2.cpu().numpy().astype(np.float64) - h_o)
+    assert (err <= tol).all(), float((err / tol).max())
+    assert q4dec.device_error() == 0
