@@ -415,7 +415,8 @@ def main():
         g5 = time_region(torch, stream, m5.gemv_stream, k5)
         a5 = time_region(torch, stream, m5.attn_stream, k5)
         t5 = time_region(torch, stream, lambda: (m5.gemv_stream(), m5.attn_stream()), k5)
-        g5, a5, t5 = reduce_over_ranks([g5, a5, t5], dev, world)
+        s5 = time_region(torch, stream, m5.gemv_stream_per_matrix, k5)
+        g5, a5, t5, s5 = reduce_over_ranks([g5, a5, t5, s5], dev, world)
         gb5 = gemv_step_bytes(5) / (g5 * 1e-3) / 1e9
         ab5 = ATTN_LAYERS * attn_alg_bytes(5, CTX) / (a5 * 1e-3) / 1e9
         m5_rec = {"M": 5, "steps": k5, "ms_per_step": t5,
@@ -425,7 +426,10 @@ def main():
                                "achieved": gb5, "peak": peak_gbs, "unit": "GB/s",
                                "frac": gb5 / peak_gbs, "launch_us": g5 * 1e3},
                   "attention": {"achieved_gbs": ab5, "frac": ab5 / peak_gbs,
-                                "us_per_layer": a5 * 1e3 / ATTN_LAYERS}}
+                                "us_per_layer": a5 * 1e3 / ATTN_LAYERS},
+                  "gemv_one_launch_per_matrix": {
+                      "ms_per_step": s5, "value": gemv_step_bytes(5) / (s5 * 1e-3) / 1e12,
+                      "unit": "TB/s", "launches_per_step": m5.n_gemv}}
         del m5
 
     # -------- the same step replayed as one CUDA graph

@@ -1,9 +1,11 @@
-"""Build libq4dec.so in-tree with nvcc for sm_100a.
+"""Build libq4dec.so in-tree with nvcc for sm_100a, and beside it
+libq4dec_debug.so: the same sources with Q4D_DEBUG defined (every global
+access of every kernel index-checked into the device error record).
 
 Usage: ``python -m bit_weight_streaming_dequant_b200.build`` (or
-``__graft_entry__.build()``).  The library links the CUDA runtime statically,
-so loading it needs no CUDA library path; it only needs the NVIDIA driver
-once a compute entry point is called.
+``__graft_entry__.build()``).  The libraries link the CUDA runtime
+statically, so loading them needs no CUDA library path; they only need the
+NVIDIA driver once a compute entry point is called.
 """
 from __future__ import annotations
 
@@ -17,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libq4dec.so")
+LIB_DEBUG = os.path.join(PKG, "libq4dec_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -33,14 +36,20 @@ def nvcc() -> str:
     return path
 
 
-def build(verbose: bool = False, extra_flags=None) -> str:
+def _compile(out: str, flags, verbose: bool):
     srcs = [os.path.join(CSRC, "q4dec.cu"), os.path.join(CSRC, "q4d_selftest.cu")]
-    cmd = [nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC,
-           *srcs, "-o", LIB + ".tmp"]
+    cmd = [nvcc(), *NVCC_FLAGS, *flags, "-I", INCLUDE, "-I", CSRC, *srcs, "-o", out + ".tmp"]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(out + ".tmp", out)
+
+
+def build(verbose: bool = False, extra_flags=None, debug: bool = True) -> str:
+    """Compile the release library (and, with `debug`, the debug one)."""
+    _compile(LIB, list(extra_flags or []), verbose)
+    if debug:
+        _compile(LIB_DEBUG, ["-DQ4D_DEBUG", *(extra_flags or [])], verbose)
     return LIB
 
 

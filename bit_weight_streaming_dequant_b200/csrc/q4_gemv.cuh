@@ -42,9 +42,9 @@
 //    the entries until they are valid -- those of a partner that finished
 //    early are read while its own sums are still being made -- adds the slots
 //    in slot order, its own from registers, writes the rows and clears the
-//    entries.  An entry holding another value (left over by another use of
-//    the memory) is not valid, so the workspace needs no clearing, and the
-//    clearing keeps replays of a captured launch (same tag) correct.
+//    entries.  The workspace is handed over zero-filled, and the clearing
+//    leaves it so after every launch; a cleared entry is never valid (tags
+//    are non-zero), and replays of a captured launch (same tag) stay correct.
 //  * Several matrices ("jobs") can run in one launch.  The producer keeps
 //    streaming the next job's weights (they depend on nothing) while a job's
 //    activations wait for the job they depend on: whichever epilogue warp
@@ -67,6 +67,10 @@
 //    the sums out (y, the partial slot, or the sum of the slots) and count the
 //    halves written in final form for their job, so no global write, atomic
 //    or cross-warp reduction stalls the consumers.
+//  * Built with Q4D_DEBUG, every global access above is index-checked
+//    against its buffer's extent (Q4D_CHECK): a failure is recorded in the
+//    device error record and the access skipped, or a copy redirected to the
+//    buffer's first bytes.
 //  * Every wait is bounded in time.  A wait that runs out sets the device
 //    error word and a per-CTA abort flag; from then on no wait blocks, the
 //    producer issues no further copies and waits for the ones in flight, and
@@ -150,9 +154,8 @@ struct alignas(16) GemvJobDesc {
   int units;             // rbs * upr
   int grid;              // CTAs that work on this job (min(launch grid, units))
   int slots;             // partial slots per row block (0: no row block is shared)
-  int pad0_;
   int rot;               // job-local CTA index = (blockIdx.x + rot) mod launch grid
-  int pad_;
+  long long w_bytes;     // extent of W that index checks allow (N * nsb * 144 or less)
 };
 
 struct GemvArgs {
@@ -165,6 +168,7 @@ struct GemvArgs {
   int grid;                       // CTAs of the launch
   int stages;                     // ring stages
   int pad_;
+  long long ws_entries;           // entries of the partial area that index checks allow
   GemvJobDesc job;                // the single job of a one-matrix launch
 };
 
@@ -266,6 +270,7 @@ struct UnitCursor {
   const uint16_t* x;
   int N, nsb, upr, wait_for;
   unsigned wait_rbs;  // count of job wait_for once finished (row-block halves)
+  long long w_bytes;
 };
 
 __device__ __forceinline__ void cursor_enter(UnitCursor& c, const GemvArgs& a, int i) {
@@ -283,10 +288,24 @@ __device__ __forceinline__ void cursor_enter(UnitCursor& c, const GemvArgs& a, i
     c.nsb = J->nsb;
     c.upr = J->upr;
     c.wait_for = J->wait_for;
+    if (!Q4D_CHECK(c.wait_for < i, a.err, kSiteGemvCounters, c.wait_for)) c.wait_for = -1;
+    c.w_bytes = J->w_bytes;
     c.wait_rbs = c.wait_for >= 0 ? unsigned(kGemvEpilogueWarps * gemv_job(a, c.wait_for)->rbs) : 0u;
     break;
   }
   c.job = i;
+}
+
+// Element offset in x of row m's columns [col0, col0 + kc) of 256 elements;
+// a failed index check gives the first element instead (memory that exists).
+template <int M>
+__device__ __forceinline__ size_t x_offset_m(const UnitCursor& c, int m, int col0, int kc,
+                                             unsigned* err) {
+  const size_t o = (size_t(m) * c.nsb + col0) * 256;
+  return Q4D_CHECK(m < M && o + size_t(kc) * 256 <= size_t(M) * c.nsb * 256, err,
+                   kSiteGemvActivations, o)
+             ? o
+             : 0;
 }
 
 __device__ __forceinline__ void cursor_next(UnitCursor& c, const GemvArgs& a) {
@@ -310,7 +329,7 @@ __device__ __forceinline__ int seg_index(int e, int lane, int k) {
 // and 2j + 1, held by neighbouring lanes).
 template <int M>
 __device__ __forceinline__ void gemv_store_rows(const GemvJobDesc* J, int rb, int e, int lane,
-                                                const float (&v)[2 * M]) {
+                                                unsigned* err, const float (&v)[2 * M]) {
   const bool bf16 = (J->flags & kJobOutBf16) != 0;
   const int r0 = rb * kGemvRows;
   if (J->flags & kJobSwiglu) {
@@ -319,15 +338,18 @@ __device__ __forceinline__ void gemv_store_rows(const GemvJobDesc* J, int rb, in
     for (int k = 0; k < 2 * M; ++k) {
       const int m = k >> 1, r = seg_row(e, lane, k);
       const float other = __shfl_down_sync(0xFFFFFFFFu, v[k], 1);
-      if ((r & 1) == 0 && r0 + r + 1 < J->N)
-        store_out(J->y, size_t(m) * n_out + ((r0 + r) >> 1), v[k] / (1.f + expf(-v[k])) * other,
-                  bf16);
+      const size_t i = size_t(m) * n_out + ((r0 + r) >> 1);
+      if ((r & 1) == 0 && r0 + r + 1 < J->N &&
+          Q4D_CHECK(i < size_t(M) * n_out, err, kSiteGemvOutput, i))
+        store_out(J->y, i, v[k] / (1.f + expf(-v[k])) * other, bf16);
     }
   } else {
     #pragma unroll
     for (int k = 0; k < 2 * M; ++k) {
       const int m = k >> 1, r = seg_row(e, lane, k);
-      if (r0 + r < J->N) store_out(J->y, size_t(m) * J->N + r0 + r, v[k], bf16);
+      const size_t i = size_t(m) * J->N + r0 + r;
+      if (r0 + r < J->N && Q4D_CHECK(i < size_t(M) * J->N, err, kSiteGemvOutput, i))
+        store_out(J->y, i, v[k], bf16);
     }
   }
 }
@@ -348,6 +370,17 @@ template <int M>
 __device__ __forceinline__ unsigned long long* slot_entries(const GemvArgs& a,
                                                             const GemvJobDesc* J, int rb, int sl) {
   return a.partials + J->part_off + (size_t(rb) * J->slots + sl) * M * kGemvRows;
+}
+
+// Index check of slot sl of row block rb (always true without Q4D_DEBUG).
+template <int M>
+__device__ __forceinline__ bool slot_in_range(const GemvArgs& a, const GemvJobDesc* J, int rb,
+                                              int sl) {
+  return Q4D_CHECK(rb < J->rbs && sl < J->slots &&
+                       J->part_off + ((long long)rb * J->slots + sl + 1) * M * kGemvRows <=
+                           a.ws_entries,
+                   a.err, kSiteGemvPartials,
+                   J->part_off + ((long long)rb * J->slots + sl) * M * kGemvRows);
 }
 
 // Read this lane's entries (epilogue warp e's half) of a slot if they are all
@@ -401,14 +434,16 @@ __device__ __forceinline__ bool gemv_segment_write(const GemvArgs& a, const Gemv
   const RowBlockShare sh = row_block_share(J, cj, rb);
   const unsigned tag32 = unsigned(a.tag);
   if (sh.n == 1) {
-    gemv_store_rows<M>(J, rb, e, lane, v);
+    gemv_store_rows<M>(J, rb, e, lane, a.err, v);
     return true;
   }
   if (sh.my != 0) {
     unsigned long long* s_e = slot_entries<M>(a, J, rb, sh.my);
-    #pragma unroll
-    for (int k = 0; k < 2 * M; ++k)
-      st_relaxed_gpu_u64(s_e + seg_index(e, lane, k), slot_entry(v[k], tag32));
+    if (slot_in_range<M>(a, J, rb, sh.my)) {
+      #pragma unroll
+      for (int k = 0; k < 2 * M; ++k)
+        st_relaxed_gpu_u64(s_e + seg_index(e, lane, k), slot_entry(v[k], tag32));
+    }
     return false;
   }
   // the finisher: slot 0 (its own, from registers), then the others in order
@@ -419,6 +454,9 @@ __device__ __forceinline__ bool gemv_segment_write(const GemvArgs& a, const Gemv
     if (sl == 1 && pre) {
       #pragma unroll
       for (int k = 0; k < 2 * M; ++k) w[k] = pv[k];
+    } else if (!slot_in_range<M>(a, J, rb, sl)) {
+      #pragma unroll
+      for (int k = 0; k < 2 * M; ++k) w[k] = 0.f;
     } else {
       const unsigned long long* s_e = slot_entries<M>(a, J, rb, sl);
       const unsigned long long t0 = global_timer_ns();
@@ -439,10 +477,11 @@ __device__ __forceinline__ bool gemv_segment_write(const GemvArgs& a, const Gemv
   // which starts only after this one has ended
   for (int sl = 1; sl < sh.n; ++sl) {
     unsigned long long* s_e = slot_entries<M>(a, J, rb, sl);
+    if (!slot_in_range<M>(a, J, rb, sl)) continue;
     #pragma unroll
     for (int k = 0; k < 2 * M; ++k) s_e[seg_index(e, lane, k)] = 0ull;
   }
-  gemv_store_rows<M>(J, rb, e, lane, v);
+  gemv_store_rows<M>(J, rb, e, lane, a.err, v);
   return true;
 }
 
@@ -515,7 +554,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
       #pragma unroll
       for (int m = 0; m < M; ++m)
         bulk_g2s_nohint(dst + uint32_t(m) * kGemvXPitch,
-                        xs.x + (size_t(m) * xs.nsb + col0) * 256, uint32_t(kc) * 512u, bar);
+                        xs.x + x_offset_m<M>(xs, m, col0, kc, a.err), uint32_t(kc) * 512u, bar);
       ++stx;
       if (++x_slot == S) x_slot = 0;
       cursor_next(xs, a);
@@ -533,10 +572,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
         const uint32_t bar = smem_addr(&full[w_slot]);
         const uint32_t dst = smem_addr(ring + size_t(w_slot) * kStage);
         mbar_arrive_expect_tx(bar, uint32_t(kc) * (uint32_t(rows) * kSbBytes + uint32_t(M) * 512u));
-        for (int j = 0; j < kc; ++j)
-          bulk_g2s(dst + uint32_t(j) * kGemvWBox,
-                   w.W + (size_t(col0 + j) * w.N + size_t(w.rb) * kGemvRows) * kSbBytes,
-                   uint32_t(rows) * kSbBytes, bar, pol);
+        for (int j = 0; j < kc; ++j) {
+          size_t off = (size_t(col0 + j) * w.N + size_t(w.rb) * kGemvRows) * kSbBytes;
+          // a failed check copies the matrix's first rows instead (memory that exists)
+          if (!Q4D_CHECK(off + uint32_t(rows) * kSbBytes <= size_t(w.w_bytes), a.err,
+                         kSiteGemvWeights, off))
+            off = 0;
+          bulk_g2s(dst + uint32_t(j) * kGemvWBox, w.W + off, uint32_t(rows) * kSbBytes, bar, pol);
+        }
         ++stw;
         if (++w_slot == S) {
           w_slot = 0;
@@ -571,7 +614,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
       const int kc = min(kGemvCols, xs.nsb - col0);
       for (int m = 0; m < M; ++m)
         bulk_g2s_nohint(dst + uint32_t(m) * kGemvXPitch,
-                        xs.x + (size_t(m) * xs.nsb + col0) * 256, uint32_t(kc) * 512u, bar);
+                        xs.x + x_offset_m<M>(xs, m, col0, kc, a.err), uint32_t(kc) * 512u, bar);
       if (++x_slot == S) x_slot = 0;
       cursor_next(xs, a);
     }
@@ -612,7 +655,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
         bool pre = false;
         float pv[2 * M];
         const RowBlockShare sh = row_block_share(J, r.cj, rb);
-        if (sh.n == 2 && sh.my == 0) {
+        if (sh.n == 2 && sh.my == 0 && slot_in_range<M>(a, J, rb, 1)) {
           const unsigned long long* s_e = slot_entries<M>(a, J, rb, 1);
           while (!pre && !mbar_test_wait(fb, fpar) && !*abort_flag) {
             pre = read_slot<M>(s_e, e, lane, unsigned(a.tag), pv);

@@ -1,10 +1,11 @@
-// Self-test of the bounded in-kernel wait that every pipeline of the library
-// relies on to terminate: one CTA waits, by phase parity, on an mbarrier that
-// (unless asked to) nobody arrives on, with the same try-wait and wall-clock
-// check the kernels use but a caller-chosen limit.  When the limit runs out
-// the kernel records it in a caller-owned word and returns normally, so the
-// CUDA context stays usable.  Nothing here faults, traps or spins without a
-// bound.
+// Self-tests of the library's two failure reports.  First the bounded
+// in-kernel wait that every pipeline of the library relies on to terminate:
+// one CTA waits, by phase parity, on an mbarrier that (unless asked to)
+// nobody arrives on, with the same try-wait and wall-clock check the kernels
+// use but a caller-chosen limit.  When the limit runs out the kernel records
+// it in a caller-owned word and returns normally, so the CUDA context stays
+// usable.  Then the record of a failed index check (below).  Nothing here
+// faults, traps or spins without a bound.
 #include <cuda_runtime.h>
 
 #include "q4dec.h"
@@ -44,5 +45,34 @@ extern "C" q4d_status q4d_wait_selftest(unsigned* word, unsigned limit_us, int a
   if (reinterpret_cast<uintptr_t>(word) % 4) return Q4D_ERR_MISALIGNED;
   q4d_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       word, 1000ull * limit_us, arrive ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? Q4D_OK : Q4D_ERR_CUDA;
+}
+
+// Self-test of the index-check record: the first n_fail of 64 threads fail a
+// check (site kSiteSelftest, index base + thread), through Q4D_CHECK in a
+// debug build and through the recording function itself in a release build
+// (whose Q4D_CHECK is the constant true).  A check that does not return its
+// condition ORs 4 into word 0.
+namespace {
+
+__global__ void q4d_index_check_selftest_kernel(unsigned* record, long long base, int n_fail) {
+  const int t = threadIdx.x;
+  const bool ok = t >= n_fail;
+#ifdef Q4D_DEBUG
+  const bool seen = Q4D_CHECK(ok, record, q4d::kSiteSelftest, base + t);
+#else
+  const bool seen = ok || (q4d::index_check_failed(record, q4d::kSiteSelftest, base + t), false);
+#endif
+  if (seen != ok) atomicOr(record, 4u);
+}
+
+}  // namespace
+
+extern "C" q4d_status q4d_index_check_selftest(unsigned* record, long long base, int n_fail,
+                                               void* stream) {
+  if (!record || n_fail < 0 || n_fail > 64) return Q4D_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(record) % 4) return Q4D_ERR_MISALIGNED;
+  q4d_index_check_selftest_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(record, base,
+                                                                                  n_fail);
   return cudaGetLastError() == cudaSuccess ? Q4D_OK : Q4D_ERR_CUDA;
 }

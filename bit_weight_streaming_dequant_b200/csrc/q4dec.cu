@@ -19,8 +19,10 @@
 #include "q4kv_attn_tc.cuh"
 #include "q4kv_append.cuh"
 
-// Device error word (bit q4d::kDevErrWaitTimeout: a bounded wait ran out).
-__device__ unsigned q4d_error_word;
+// Device error record: word 0 holds the bits (q4d::kDevErrWaitTimeout: a
+// bounded wait ran out; q4d::kDevErrIndex: an index check of a Q4D_DEBUG
+// build failed), words 1..3 the first failed check's site and index.
+__device__ unsigned q4d_error_word[q4d::kDevErrRecordWords];
 
 namespace {
 
@@ -220,6 +222,16 @@ q4d_status plan_gemv_rows(int M, int rows, int K, int num_sms, int smem_optin,
 
 std::atomic<unsigned long long> g_gemv_tag{0};
 
+// Weight extent that GEMV index checks allow, if a test has capped it
+// (q4d_debug_limit_weights; 0: none): the true N * K / 256 * 144 bytes, or
+// the cap when that is smaller.
+std::atomic<unsigned long long> g_weight_limit{0};
+long long declared_weight_bytes(int rows, int nsb) {
+  const unsigned long long full = (unsigned long long)rows * nsb * 144ull;
+  const unsigned long long cap = g_weight_limit.load(std::memory_order_relaxed);
+  return (long long)((cap > 0 && cap < full) ? cap : full);
+}
+
 // A fresh tag for every launch; its low 32 bits, the ones partial-slot entries
 // carry, are never 0 (a cleared entry is 0).
 unsigned long long next_gemv_tag() {
@@ -299,6 +311,7 @@ q4d_status gemv_impl(const void* W_q4, const void* x, void* y, int M, int N, int
   if (p.workspace_bytes > 0) {
     a.partials = static_cast<unsigned long long*>(workspace);
   }
+  a.ws_entries = (long long)(p.workspace_bytes / kGemvEntryBytes);
   q4d::GemvJobDesc& J = a.job;
   J.W = static_cast<const uint8_t*>(W_q4);
   J.x = static_cast<const uint16_t*>(x);
@@ -314,6 +327,7 @@ q4d_status gemv_impl(const void* W_q4, const void* x, void* y, int M, int N, int
   J.grid = p.grid;
   J.slots = p.slots;
   J.rot = 0;
+  J.w_bytes = declared_weight_bytes(rows, K / 256);
   if ((st = launch_gemv(M, a, p.smem_bytes, dev, *s, stream, pdl)) != Q4D_OK) return st;
   if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
   return Q4D_OK;
@@ -395,6 +409,7 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
   a.split_tokens = p.split_tokens;
   a.rows_per_cta = p.rows_per_cta;
   a.stages = p.stages;
+  a.ws_floats = (long long)(p.workspace_bytes / 4);
 
   if (!q8 && p.rows_per_cta <= 8)
     st = launch_attn_rows8(a, p, n_kv, dev, *s, stream);
@@ -449,6 +464,7 @@ const char* q4d_status_string(int status) {
     case Q4D_ERR_WORKSPACE: return "workspace missing or too small";
     case Q4D_ERR_CUDA: return "CUDA runtime error";
     case Q4D_ERR_DEVICE_TIMEOUT: return "in-kernel wait timed out";
+    case Q4D_ERR_DEVICE_INDEX: return "index check failed (debug build)";
     default: return "unknown status";
   }
 }
@@ -658,6 +674,7 @@ q4d_status q4d_gemv_batch_prepare(const q4d_gemv_job* jobs, int n_jobs, int M, i
     d.slots = sh.slots;
     d.part_off = (long long)partials;
     d.rot = int(units_before % grid);
+    d.w_bytes = declared_weight_bytes(rows, j.K / 256);
     units_before += sh.units;
     if (sh.slots > 0) {
       partials += size_t(sh.rbs) * sh.slots * M * q4d::kGemvRows;
@@ -710,6 +727,7 @@ q4d_status q4_gemv_batch_ex(const void* desc_host, void* desc_dev, void* stream,
   a.err = s->err;
   a.tag = next_gemv_tag();
   a.partials = static_cast<unsigned long long*>(workspace);
+  a.ws_entries = (long long)(h.workspace_bytes / kGemvEntryBytes);
   if ((st = launch_gemv(h.M, a, q4d::gemv_smem_bytes(h.M, stages), dev, *s,
                         static_cast<cudaStream_t>(stream), (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0)) !=
       Q4D_OK)
@@ -766,6 +784,7 @@ extern "C" q4d_status q4kv_append(void* Kq4, void* Vq4, const float* k_new, cons
   a.kv_stride = kv_stride_tokens;
   a.pos = pos;
   a.M = M;
+  a.err = s->err;
   q4d::q4kv_append_kernel<<<dim3(M * n_kv_heads, 2), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return cudaGetLastError() == cudaSuccess ? Q4D_OK : Q4D_ERR_CUDA;
 }
@@ -833,23 +852,45 @@ q4d_status q4d_unpack_q4_0_rows(const void* rows_q4, void* blocks18, int rows, i
 }  // extern "C"
 
 extern "C" {
-q4d_status q4d_device_error(int reset) {
+q4d_status q4d_device_error_record(unsigned* record, int reset) {
   int dev = 0;
   DeviceState* s = nullptr;
   q4d_status st = current_device(&dev, &s);
   if (st != Q4D_OK) return st;
-  unsigned word = 0;
+  unsigned rec[q4d::kDevErrRecordWords] = {0u, 0u, 0u, 0u};
   if (cudaDeviceSynchronize() != cudaSuccess ||
-      cudaMemcpy(&word, s->err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+      cudaMemcpy(rec, s->err, sizeof(rec), cudaMemcpyDeviceToHost) != cudaSuccess) {
     cudaGetLastError();
     return Q4D_ERR_CUDA;
   }
-  if (reset && word) {
-    const unsigned zero = 0;
-    if (cudaMemcpy(s->err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+  if (record) std::memcpy(record, rec, sizeof(rec));
+  if (reset && (rec[0] | rec[1] | rec[2] | rec[3])) {
+    const unsigned zero[q4d::kDevErrRecordWords] = {0u, 0u, 0u, 0u};
+    if (cudaMemcpy(s->err, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
       return Q4D_ERR_CUDA;
   }
-  return word ? Q4D_ERR_DEVICE_TIMEOUT : Q4D_OK;
+  if (rec[0] & q4d::kDevErrIndex) return Q4D_ERR_DEVICE_INDEX;
+  return rec[0] ? Q4D_ERR_DEVICE_TIMEOUT : Q4D_OK;
+}
+
+q4d_status q4d_device_error(int reset) { return q4d_device_error_record(nullptr, reset); }
+
+int q4d_debug_build(void) {
+#ifdef Q4D_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+q4d_status q4d_debug_limit_weights(unsigned long long bytes) {
+#ifdef Q4D_DEBUG
+  g_weight_limit.store(bytes, std::memory_order_relaxed);
+  return Q4D_OK;
+#else
+  (void)bytes;
+  return Q4D_ERR_INVALID_ARG;
+#endif
 }
 
 }  // extern "C"

@@ -11,6 +11,50 @@ namespace q4d {
 
 // Bits of the device error word.
 constexpr unsigned kDevErrWaitTimeout = 1u;
+constexpr unsigned kDevErrIndex = 2u;  // an index check of a Q4D_DEBUG build failed
+
+// The device error record: word 0 holds the bits above; words 1..3 the first
+// failed index check (its site, then the offending index, low word first).
+constexpr int kDevErrRecordWords = 4;
+
+// Where an index check sits (the site recorded with the first failure).
+enum IndexCheckSite : unsigned {
+  kSiteGemvWeights = 1,      // bulk copy of a unit's weight column
+  kSiteGemvActivations = 2,  // bulk copy of an activation row piece
+  kSiteGemvOutput = 3,       // store of an output element
+  kSiteGemvPartials = 4,     // a row block's partial-slot entries
+  kSiteGemvCounters = 5,     // a batch job's completion counter
+  kSiteAttnKV = 16,          // bulk copy of a K / V tile
+  kSiteAttnQuery = 17,       // load of a query element
+  kSiteAttnOutput = 18,      // store of an output element
+  kSiteAttnStates = 19,      // a split's state (partial output, max, sum)
+  kSiteAppend = 32,          // the super-block an appended row goes to
+  kSiteSelftest = 255,       // the check self-test
+};
+
+// Record a failed index check in the error record at err: the bit, and for
+// the first failure of all its site and index.  Also compiled into release
+// builds, where only the self-test calls it.
+static __device__ __noinline__ void index_check_failed(unsigned* err, unsigned site,
+                                                       long long index) {
+  atomicOr(err, kDevErrIndex);
+  if (atomicCAS(err + 1, 0u, site) == 0u) {
+    err[2] = unsigned(static_cast<unsigned long long>(index));
+    err[3] = unsigned(static_cast<unsigned long long>(index) >> 32);
+  }
+}
+
+// Index checks: Q4D_CHECK(ok, err, site, index) is `ok`, and records a
+// failure when it is false, in a build with Q4D_DEBUG defined; otherwise it
+// is the constant true and its arguments are not evaluated.  A failed check
+// never traps: the caller skips the access, or redirects a load to the first
+// element of its buffer (memory that exists), and the kernel runs to its end.
+#ifdef Q4D_DEBUG
+#define Q4D_CHECK(ok, err, site, index) \
+  ((ok) ? true : (::q4d::index_check_failed((err), (site), (long long)(index)), false))
+#else
+#define Q4D_CHECK(ok, err, site, index) true
+#endif
 
 // A pipeline wait gives up after this many nanoseconds (far above any normal
 // stage latency, which is microseconds); the kernel then flags the error word

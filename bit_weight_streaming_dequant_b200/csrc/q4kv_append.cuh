@@ -23,6 +23,7 @@ struct AppendArgs {
   uint8_t* V;
   const float* k_new;  // [M][n_kv][256]
   const float* v_new;
+  unsigned* err;       // device error record (index checks of a Q4D_DEBUG build)
   int n_kv, kv_stride, pos, M;
 };
 
@@ -57,6 +58,9 @@ __global__ void __launch_bounds__(256) q4kv_append_kernel(const AppendArgs a) {
   }
   const int q_hi = __shfl_down_sync(0xFFFFFFFFu, q, 16);
   uint8_t* sb = (is_v ? a.V : a.K) + (size_t(h) * a.kv_stride + a.pos + m) * 144;
+  if (!Q4D_CHECK(m < a.M && h < a.n_kv && a.pos >= 0 && a.pos + m < a.kv_stride, a.err,
+                 kSiteAppend, (long long)h * a.kv_stride + a.pos + m))
+    return;
   if (lane < 16) sb[blk * 16 + lane] = uint8_t(q | (q_hi << 4));
   if (lane == 0) *reinterpret_cast<__half*>(sb + 128 + 2 * blk) = d16;
 }

@@ -31,6 +31,8 @@
 // Each warp owns its own tokens, softmax state and full O^T.  More query rows
 // per CTA (9..32) go to the tensor-memory kernel in q4kv_attn_tc.cuh; both
 // write the same split states for the merge kernel at the end of this file.
+// Built with Q4D_DEBUG, the K / V copies, the query loads and the output and
+// state stores are index-checked (the *_in_range helpers below).
 #pragma once
 
 #include "q4dec_device.cuh"
@@ -52,7 +54,29 @@ struct AttnArgs {
   int ctx_len, n_q, n_kv, M, g, kv_stride;
   float scale_log2;    // softmax scale * log2(e)
   int n_splits, split_tokens, rows_per_cta, stages;
+  long long ws_floats; // floats of the workspace (split states) that index checks allow
 };
+
+// Index checks shared by the attention kernels (always true without
+// Q4D_DEBUG).  Token rows [t0, t0 + n) of KV head kh lie in the cache.
+__device__ __forceinline__ bool kv_rows_in_range(const AttnArgs& a, int kh, int t0, int n) {
+  return Q4D_CHECK(kh < a.n_kv && t0 >= 0 && n >= 1 && t0 + n <= a.kv_stride, a.err, kSiteAttnKV,
+                   (long long)kh * a.kv_stride + t0);
+}
+// Query row m, head h exists.
+__device__ __forceinline__ bool query_in_range(const AttnArgs& a, int m, int h) {
+  return Q4D_CHECK(m < a.M && h < a.n_q, a.err, kSiteAttnQuery, (long long)m * a.n_q + h);
+}
+// Output row `row` (m * n_q + h) exists, and so does split `split`'s state
+// for it, with every split's states inside the workspace.
+__device__ __forceinline__ bool out_row_in_range(const AttnArgs& a, size_t row) {
+  return Q4D_CHECK(row < size_t(a.M) * a.n_q, a.err, kSiteAttnOutput, row);
+}
+__device__ __forceinline__ bool state_in_range(const AttnArgs& a, int split, size_t row) {
+  return Q4D_CHECK(split < a.n_splits && row < size_t(a.M) * a.n_q &&
+                       size_t(a.n_splits) * a.M * a.n_q * (kHeadDim + 2) <= size_t(a.ws_floats),
+                   a.err, kSiteAttnStates, (long long)split * a.M * a.n_q + row);
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
@@ -195,14 +219,21 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
   const uint8_t* Vh = a.V + size_t(kh) * a.kv_stride * kRowBytes;
   const uint64_t pol = l2_evict_first_policy();
   auto issue = [&](int tile) {
-    const int t0 = t_begin + tile * TT;
-    const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * kRowBytes;
+    int t0 = t_begin + tile * TT, n = min(TT, t_end - t0);
+    const uint8_t *kp = Kh, *vp = Vh;
+    if (!kv_rows_in_range(a, kh, t0, n)) {  // copy rows of the first head instead
+      kp = a.K;
+      vp = a.V;
+      t0 = 0;
+      n = max(1, min(n, a.ctx_len));
+    }
+    const uint32_t bytes = uint32_t(n) * kRowBytes;
     const int slot = tile % S;
     const uint32_t bar = smem_addr(&full[slot]);
     const uint32_t dk = smem_addr(ring + size_t(slot) * kR8StageBytes);
     mbar_arrive_expect_tx(bar, 2 * bytes);
-    bulk_g2s(dk, Kh + size_t(t0) * kRowBytes, bytes, bar, pol);
-    bulk_g2s(dk + TT * kRowBytes, Vh + size_t(t0) * kRowBytes, bytes, bar, pol);
+    bulk_g2s(dk, kp + size_t(t0) * kRowBytes, bytes, bar, pol);
+    bulk_g2s(dk + TT * kRowBytes, vp + size_t(t0) * kRowBytes, bytes, bar, pol);
   };
 
   int issued = 0;
@@ -223,7 +254,8 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (r < R) {
       const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
-      v = q_frag_f16(a.Q + (size_t(m) * a.n_q + kh * a.g + j) * kHeadDim + b * 32 + 4 * tt);
+      if (query_in_range(a, m, kh * a.g + j))
+        v = q_frag_f16(a.Q + (size_t(m) * a.n_q + kh * a.g + j) * kHeadDim + b * 32 + 4 * tt);
     }
     *reinterpret_cast<uint4*>(Qf + r * kR8QPitch + (i & 31) * 16) = v;
   }
@@ -441,8 +473,8 @@ __global__ void __launch_bounds__(kR8Threads, 1) q4kv_attn_split_rows8_kernel(co
     const int rr = row0 + r, m = rr / a.g, j = rr - m * a.g;
     const size_t row = size_t(m) * a.n_q + kh * a.g + j;
     if (a.n_splits == 1) {
-      a.out[row * kHeadDim + dim] = acc / rml[r * 2 + 1];
-    } else {
+      if (out_row_in_range(a, row)) a.out[row * kHeadDim + dim] = acc / rml[r * 2 + 1];
+    } else if (state_in_range(a, split, row)) {
       a.ws_o[(size_t(split) * rows_total + row) * kHeadDim + dim] = acc;
       if (dim == 0) {
         a.ws_ml[(size_t(split) * rows_total + row) * 2 + 0] = rml[r * 2 + 0];
@@ -465,6 +497,7 @@ __global__ void __launch_bounds__(256) q4kv_attn_merge_kernel(const AttnArgs a) 
   if (tid == 0) griddep_launch_dependents();
   griddep_wait();  // the split kernel has finished: its states are visible
   const size_t rows = size_t(a.M) * a.n_q;
+  if (!state_in_range(a, a.n_splits - 1, row)) return;  // every split's state of this row
   __shared__ float part[8 * kHeadDim];
   const int n = a.n_splits;
   float mx = -INFINITY;
@@ -500,7 +533,7 @@ __global__ void __launch_bounds__(256) q4kv_attn_merge_kernel(const AttnArgs a) 
   float sum = 0.f;
   #pragma unroll
   for (int w = 0; w < 8; ++w) sum += part[w * kHeadDim + tid];
-  a.out[size_t(row) * kHeadDim + tid] = sum / L;
+  if (out_row_in_range(a, row)) a.out[size_t(row) * kHeadDim + tid] = sum / L;
 }
 
 }  // namespace q4d

@@ -203,7 +203,8 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
     if (n < R) {
       const int rr = row0 + n, m = rr / a.g, j = rr - m * a.g;
       const int e = (kp & ~31) + tca_element<Q8>(kp & 31);
-      v = bf16_bits_to_float(a.Q[(size_t(m) * a.n_q + kh * a.g + j) * kHeadDim + e]);
+      if (query_in_range(a, m, kh * a.g + j))
+        v = bf16_bits_to_float(a.Q[(size_t(m) * a.n_q + kh * a.g + j) * kHeadDim + e]);
     }
     *reinterpret_cast<__half*>(Qs + (kp >> 3) * (NR * 16) + (n >> 3) * 128 + (n & 7) * 16 +
                                (kp & 7) * 2) = __float2half_rn(v);
@@ -239,13 +240,20 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
         if (tile >= S && !mbar_wait_or_abort(smem_addr(&empty[slot]), uint32_t(tile / S - 1) & 1u,
                                              a.err, abort_flag))
           break;  // no further copies after a time-out
-        const int t0 = t_begin + tile * TT;
-        const uint32_t bytes = uint32_t(min(TT, t_end - t0)) * RB;
+        int t0 = t_begin + tile * TT, n = min(TT, t_end - t0);
+        const uint8_t *kp = Kh, *vp = Vh;
+        if (!kv_rows_in_range(a, kh, t0, n)) {  // copy rows of the first head instead
+          kp = a.K;
+          vp = a.V;
+          t0 = 0;
+          n = max(1, min(n, a.ctx_len));
+        }
+        const uint32_t bytes = uint32_t(n) * RB;
         const uint32_t bar = smem_addr(&full[slot]);
         const uint32_t dk = smem_addr(ring + size_t(slot) * kStage);
         mbar_arrive_expect_tx(bar, 2 * bytes);
-        bulk_g2s(dk, Kh + size_t(t0) * RB, bytes, bar, pol);
-        bulk_g2s(dk + TT * RB, Vh + size_t(t0) * RB, bytes, bar, pol);
+        bulk_g2s(dk, kp + size_t(t0) * RB, bytes, bar, pol);
+        bulk_g2s(dk + TT * RB, vp + size_t(t0) * RB, bytes, bar, pol);
         issued = tile + 1;
       }
       // after a time-out: wait (bounded) for the copies still in flight, the
@@ -489,8 +497,8 @@ __global__ void __launch_bounds__(kTcaThreads, 1) q4kv_attn_tc_kernel(const Attn
         const size_t orow = size_t(m) * a.n_q + kh * a.g + j;
         const float ov = __uint_as_float(o[i]);
         if (a.n_splits == 1) {
-          a.out[orow * kHeadDim + dim] = ov / lsum[n];
-        } else {
+          if (out_row_in_range(a, orow)) a.out[orow * kHeadDim + dim] = ov / lsum[n];
+        } else if (state_in_range(a, split, orow)) {
           a.ws_o[(size_t(split) * rows_total + orow) * kHeadDim + dim] = ov;
           if (mm == 0) {
             a.ws_ml[(size_t(split) * rows_total + orow) * 2 + 0] = m_run[n];

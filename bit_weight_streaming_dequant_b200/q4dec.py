@@ -11,7 +11,12 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libq4dec.so")
+RELEASE_LIB_PATH = os.path.join(_HERE, "libq4dec.so")
+# libq4dec_debug.so: the same library built with Q4D_DEBUG (index checks of
+# every global access into the device error record); chosen with
+# Q4D_DEBUG=1 in the environment or use_debug_library().
+DEBUG_LIB_PATH = os.path.join(_HERE, "libq4dec_debug.so")
+LIB_PATH = DEBUG_LIB_PATH if os.environ.get("Q4D_DEBUG") == "1" else RELEASE_LIB_PATH
 
 STATUS = {
     0: "Q4D_OK",
@@ -21,6 +26,14 @@ STATUS = {
     4: "Q4D_ERR_WORKSPACE",
     5: "Q4D_ERR_CUDA",
     6: "Q4D_ERR_DEVICE_TIMEOUT",
+    7: "Q4D_ERR_DEVICE_INDEX",
+}
+
+# Sites of the device error record's first failed index check.
+CHECK_SITES = {
+    1: "gemv weights", 2: "gemv activations", 3: "gemv output", 4: "gemv partial slots",
+    5: "gemv batch counters", 16: "attention K/V", 17: "attention query",
+    18: "attention output", 19: "attention split states", 32: "K/V append", 255: "self-test",
 }
 
 EXPORTS = (
@@ -34,6 +47,8 @@ EXPORTS = (
     "q4d_gemv_swiglu_workspace_bytes", "q8kv_attn_decode_ex", "q8kv_attn_workspace_bytes",
     "q8kv_plan_attn", "q4d_wait_selftest",
     "q4d_gemv_batch_desc_bytes", "q4d_gemv_batch_prepare", "q4_gemv_batch_ex",
+    "q4d_device_error_record", "q4d_debug_build", "q4d_debug_limit_weights",
+    "q4d_index_check_selftest",
 )
 
 
@@ -69,8 +84,20 @@ class AttnPlan(ctypes.Structure):
 _lib = None
 
 
+def use_debug_library(debug: bool = True) -> str:
+    """Make the next lib() load the debug (or the release) library; calls
+    made through the other one before keep their results.  Returns the path."""
+    global _lib, LIB_PATH
+    path = DEBUG_LIB_PATH if debug else RELEASE_LIB_PATH
+    if path != LIB_PATH:
+        LIB_PATH = path
+        _lib = None
+    return path
+
+
 def lib() -> ctypes.CDLL:
-    """Load libq4dec.so (built in-tree); raise if it is not there."""
+    """Load the library at LIB_PATH (libq4dec.so, built in-tree, unless the
+    debug build was chosen); raise if it is not there."""
     global _lib
     if _lib is not None:
         return _lib
@@ -120,6 +147,14 @@ def lib() -> ctypes.CDLL:
     L.q8kv_plan_attn.restype = i
     L.q4d_wait_selftest.argtypes = [vp, ctypes.c_uint, i, vp]
     L.q4d_wait_selftest.restype = i
+    L.q4d_device_error_record.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
+    L.q4d_device_error_record.restype = i
+    L.q4d_debug_build.argtypes = []
+    L.q4d_debug_build.restype = i
+    L.q4d_debug_limit_weights.argtypes = [ctypes.c_ulonglong]
+    L.q4d_debug_limit_weights.restype = i
+    L.q4d_index_check_selftest.argtypes = [vp, ctypes.c_longlong, i, vp]
+    L.q4d_index_check_selftest.restype = i
     for fn in ("q4_gemv", "q4_gemv_ex", "q4_gemv_ex2", "q4kv_attn_decode", "q4kv_attn_decode_ex",
                "q4d_plan_gemv", "q4d_plan_attn", "q4d_device_error",
                "q4kv_attn_decode_noalloc"):
@@ -472,3 +507,26 @@ def q4kv_attn_decode_noalloc(Q, Kq4, Vq4, out, *, ctx_len: int, n_kv_heads: int,
 def device_error(reset: bool = False) -> int:
     """Synchronise and read the device error word (0 = clear)."""
     return lib().q4d_device_error(1 if reset else 0)
+
+
+def device_error_record(reset: bool = False):
+    """Synchronise and read the device error record: (status, bits, site,
+    index) -- site and index of the first failed index check of a debug
+    build (0, 0 when none failed)."""
+    rec = (ctypes.c_uint * 4)()
+    st = lib().q4d_device_error_record(rec, 1 if reset else 0)
+    if st not in (0, 6, 7):
+        _check(st, "q4d_device_error_record")
+    index = rec[2] | (rec[3] << 32)
+    return st, rec[0], rec[1], index - (1 << 64) if index >= 1 << 63 else index
+
+
+def debug_build() -> bool:
+    """Whether the loaded library is the debug (index-checked) build."""
+    return lib().q4d_debug_build() == 1
+
+
+def debug_limit_weights(nbytes: int) -> None:
+    """Debug build only: declare the weight extent of GEMVs launched or
+    batches prepared from now on as min(true extent, nbytes) (0: true)."""
+    _check(lib().q4d_debug_limit_weights(int(nbytes)), "q4d_debug_limit_weights")

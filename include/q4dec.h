@@ -80,7 +80,8 @@ typedef enum {
   Q4D_ERR_MISALIGNED = 3,        /* pointer alignment below the stated minimum */
   Q4D_ERR_WORKSPACE = 4,         /* workspace missing or smaller than required */
   Q4D_ERR_CUDA = 5,              /* CUDA runtime error (launch, device query, malloc) */
-  Q4D_ERR_DEVICE_TIMEOUT = 6     /* a bounded in-kernel wait ran out (q4d_device_error) */
+  Q4D_ERR_DEVICE_TIMEOUT = 6,    /* a bounded in-kernel wait ran out (q4d_device_error) */
+  Q4D_ERR_DEVICE_INDEX = 7       /* an index check of a debug build failed (q4d_device_error) */
 } q4d_status;
 
 /* Library version, Q4D_VERSION of the build. */
@@ -425,12 +426,52 @@ q4d_status q4d_pack_q4_0_rows(const void* blocks18, void* rows_q4, int rows, int
 q4d_status q4d_unpack_q4_0_rows(const void* rows_q4, void* blocks18, int rows, int K);
 
 /* ------------------------------------------------------- device errors --
- * Synchronises the current device and reads the library's device error word
- * (set when an in-kernel wait exceeded its time limit).  Returns Q4D_OK when
- * clear, Q4D_ERR_DEVICE_TIMEOUT when set, Q4D_ERR_CUDA if the device cannot
- * be queried.  reset != 0 clears the word after reading.
+ * Synchronises the current device and reads the library's device error
+ * record: a word of bits (1: an in-kernel wait exceeded its time limit; 2: an
+ * index check of a debug build failed) and the first failed index check.
+ * Returns Q4D_OK when clear, Q4D_ERR_DEVICE_INDEX when bit 2 is set, else
+ * Q4D_ERR_DEVICE_TIMEOUT when bit 1 is set, Q4D_ERR_CUDA if the device
+ * cannot be queried.  reset != 0 clears the record after reading.
  */
 q4d_status q4d_device_error(int reset);
+
+/* The same, also copying the record into record[0..3] (HOST memory, 4
+ * unsigned, may be NULL): record[0] the bits, record[1] the site of the first
+ * failed index check (0: none; 1..5 the GEMV's weight copy, activation copy,
+ * output store, partial slots and batch counters; 16..19 attention's K / V
+ * copy, query load, output store and split states; 32 the K/V append; 255
+ * the self-test below), record[2] / record[3] the low / high word of the
+ * offending index (a byte offset for copies, an element or row index
+ * otherwise).
+ */
+q4d_status q4d_device_error_record(unsigned* record, int reset);
+
+/* ------------------------------------------------------ debug build --
+ * libq4dec_debug.so is the same library built with Q4D_DEBUG: every global
+ * access of every kernel (bulk copies of weights, activations, K and V;
+ * query loads; output, partial-slot, state and cache stores; batch counter
+ * loads) is first checked against its buffer's extent.  A failed check never
+ * traps: it sets bit 2 of the device error record (site and index of the
+ * first failure), skips the access or redirects a copy to its buffer's first
+ * bytes, and the kernel runs to its end; results of that launch are void.
+ * No counterpart in the source pages: a test facility of this library.
+ *
+ * q4d_debug_build: 1 in the debug build, 0 otherwise.
+ * q4d_debug_limit_weights: the GEMV launches and batch descriptors prepared
+ *   after this call declare each matrix's weight extent as min(true extent,
+ *   bytes) (0: the true extent), so that a test can make the weight-copy
+ *   check fail on memory that exists.  Debug build: Q4D_OK.  Release build:
+ *   Q4D_ERR_INVALID_ARG, nothing changes.
+ * q4d_index_check_selftest: one CTA of 64 threads, the first n_fail of which
+ *   (0..64) fail a check with site 255 and index base + thread into the
+ *   caller's record (DEVICE pointer to 4 unsigned, 4-byte aligned, zeroed by
+ *   the caller); a check that does not return its own condition ORs 4 into
+ *   record[0].  Runs in both builds.  Returns Q4D_ERR_INVALID_ARG /
+ *   Q4D_ERR_MISALIGNED (nothing launched) or the launch status.
+ */
+int q4d_debug_build(void);
+q4d_status q4d_debug_limit_weights(unsigned long long bytes);
+q4d_status q4d_index_check_selftest(unsigned* record, long long base, int n_fail, void* stream);
 
 /* Self-test of the bounded in-kernel wait (the mechanism behind
  * Q4D_ERR_DEVICE_TIMEOUT), for failure-detection tests: one CTA waits on an

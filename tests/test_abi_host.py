@@ -30,8 +30,8 @@ def test_library_exports_every_declared_function():
 def test_version_and_status_strings():
     L = q4dec.lib()
     assert L.q4d_version() == 20000
-    for code in range(7):
-        assert L.q4d_status_string(code)
+    for code in range(8):
+        assert L.q4d_status_string(code) != b"unknown status"
     assert L.q4d_status_string(99) == b"unknown status"
 
 
@@ -273,8 +273,10 @@ def test_gemv_batch_descriptor_matches_the_planning_model(M, sms):
         slots = _contributors(rbs, upr, U, G)
         off = 64 + i * 80
         W, x, y, part_off = struct.unpack_from("<QQQq", raw, off)
-        (Nd, nsb, flags, wait_for, rbs_d, upr_d, units, G_d, slots_d, _, rot, _) = \
-            struct.unpack_from("<12i", raw, off + 32)
+        (Nd, nsb, flags, wait_for, rbs_d, upr_d, units, G_d, slots_d, rot) = \
+            struct.unpack_from("<10i", raw, off + 32)
+        (w_bytes,) = struct.unpack_from("<q", raw, off + 72)
+        assert w_bytes == rows * (K // 256) * 144  # the index checks' weight extent
         assert (W, x, y) == (FAKE + 16 * i, FAKE + 32 * i, FAKE + 64 * i)
         assert (Nd, nsb, wait_for) == (rows, K // 256, i - 1)
         assert bool(flags & 2) == bool(fl & q4dec.GEMV_SWIGLU) and bool(flags & 1) == bool(fl & 2)
@@ -286,3 +288,84 @@ def test_gemv_batch_descriptor_matches_the_planning_model(M, sms):
     assert ws.value == entries * 8
     # the completion counters after the jobs are zero as prepared
     assert set(raw[64 + n * 80:nbytes]) == {0}
+
+
+# ---- the debug build (libq4dec_debug.so: the same sources with Q4D_DEBUG)
+
+def _debug_lib():
+    assert os.path.exists(q4dec.DEBUG_LIB_PATH), "libq4dec_debug.so is built beside libq4dec.so"
+    D = ctypes.CDLL(q4dec.DEBUG_LIB_PATH)
+    D.q4d_debug_build.restype = ctypes.c_int
+    D.q4d_debug_limit_weights.argtypes = [ctypes.c_ulonglong]
+    D.q4d_debug_limit_weights.restype = ctypes.c_int
+    D.q4d_gemv_batch_desc_bytes.argtypes = [ctypes.c_int]
+    D.q4d_gemv_batch_desc_bytes.restype = ctypes.c_size_t
+    D.q4d_gemv_batch_prepare.argtypes = [ctypes.POINTER(q4dec.GemvJob), ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                         ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)]
+    D.q4d_gemv_batch_prepare.restype = ctypes.c_int
+    D.q4d_index_check_selftest.argtypes = [ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int,
+                                           ctypes.c_void_p]
+    D.q4d_index_check_selftest.restype = ctypes.c_int
+    return D
+
+
+def test_debug_library_exports_every_declared_function_and_says_it_is_the_debug_build():
+    D = _debug_lib()
+    for name in _declared_functions():
+        assert hasattr(D, name), name
+    assert D.q4d_debug_build() == 1
+    assert q4dec.lib().q4d_debug_build() == 0
+
+
+def test_index_check_selftest_validates_before_launching():
+    for L in (q4dec.lib(), _debug_lib()):
+        assert L.q4d_index_check_selftest(None, 0, 1, None) == 1
+        assert L.q4d_index_check_selftest(FAKE, 0, -1, None) == 1
+        assert L.q4d_index_check_selftest(FAKE, 0, 65, None) == 1
+        assert L.q4d_index_check_selftest(FAKE + 2, 0, 1, None) == 3
+
+
+def test_weight_limit_is_a_debug_build_hook_and_caps_the_declared_extent():
+    import struct
+    assert q4dec.lib().q4d_debug_limit_weights(4096) == 1  # release: refused, nothing set
+    D = _debug_lib()
+    shapes = [(512, 1024), (16, 256)]                       # 294912 and 2304 bytes of weights
+    jobs = (q4dec.GemvJob * 2)()
+    for i, (N, K) in enumerate(shapes):
+        jobs[i] = q4dec.GemvJob(FAKE, FAKE, FAKE, N, K, 0, -1)
+    nbytes = D.q4d_gemv_batch_desc_bytes(2)
+    for limit, expect in ((4096, [4096, 2304]), (0, [294912, 2304])):
+        assert D.q4d_debug_limit_weights(limit) == 0
+        buf = ctypes.create_string_buffer(nbytes)
+        ws = ctypes.c_size_t(0)
+        assert D.q4d_gemv_batch_prepare(jobs, 2, 1, 148, buf, nbytes, ctypes.byref(ws)) == 0
+        got = [struct.unpack_from("<q", buf.raw, 64 + i * 80 + 72)[0] for i in range(2)]
+        assert got == expect
+    assert D.q4d_debug_limit_weights(0) == 0
+
+
+def _kernel_sources():
+    csrc = os.path.join(ROOT, "bit_weight_streaming_dequant_b200", "csrc")
+    return {n: open(os.path.join(csrc, n)).read() for n in sorted(os.listdir(csrc))
+            if n.endswith(".cuh") and n != "q4dec_device.cuh"}
+
+
+def test_every_bulk_copy_and_global_store_of_the_kernels_is_index_checked():
+    """Each bulk copy's source and each plain global store of the kernels is
+    guarded by an index check within the few lines before it (a lint: the
+    debug-build parity runs show that no check fails on valid inputs)."""
+    guards = ("Q4D_CHECK", "_in_range", "x_offset_m<")
+    stores = re.compile(r"\b(a\.out|a\.ws_o|a\.ws_ml|sb)\[[^\]]*\]\s*=[^=]|store_out\(J->y|"
+                        r"st_relaxed_gpu_u64\(s_e|s_e\[seg_index\([^)]*\)\]\s*=|"
+                        r"reinterpret_cast<__half\*>\(sb")
+    for name, text in _kernel_sources().items():
+        lines = text.splitlines()
+        for i, line in enumerate(lines):
+            code = line.split("//")[0]
+            if re.search(r"\bbulk_g2s(_nohint)?\(", code) and "__device__" not in code:
+                window = "\n".join(lines[max(0, i - 12):i + 2])
+                assert any(g in window for g in guards), f"{name}:{i + 1}: {line.strip()}"
+            if stores.search(code):
+                window = "\n".join(lines[max(0, i - 6):i + 1])
+                assert any(g in window for g in guards), f"{name}:{i + 1}: {line.strip()}"
