@@ -60,13 +60,15 @@
 //    warp into a ring of stages that complete on "full" mbarriers.  Sixteen
 //    consumer warps take one (column, block) task each per stage and release
 //    it on an "empty" mbarrier.  At the end of each row block segment each
-//    consumer warp stores its partial sums into its own slot of a reduction
-//    buffer, signals it on an mbarrier and goes on with the next stage -- no
-//    CTA-wide barrier; two epilogue warps, each taking one half (64 rows) of
-//    every segment, add the 16 slots in warp order, release the buffer, write
-//    the sums out (y, the partial slot, or the sum of the slots) and count the
-//    halves written in final form for their job, so no global write, atomic
-//    or cross-warp reduction stalls the consumers.
+//    consumer warp of column 0 stores its partial sums into the slot of its
+//    block index in a reduction buffer and signals it on an mbarrier; the
+//    column-1 warp of the same block adds its sums to that slot, signals the
+//    slot complete and goes on with the next stage -- no CTA-wide barrier;
+//    two epilogue warps, each taking one half (64 rows) of every segment, add
+//    the 8 slots in block order, release the buffer, write the sums out (y,
+//    the partial slot, or the sum of the slots) and count the halves written
+//    in final form for their job, so no global write or atomic stalls the
+//    consumers, and a consumer warp waits at most for its column partner.
 //  * Built with Q4D_DEBUG, every global access above is index-checked
 //    against its buffer's extent (Q4D_CHECK): a failure is recorded in the
 //    device error record and the access skipped, or a copy redirected to the
@@ -109,23 +111,42 @@ constexpr uint32_t kJobSwiglu = 2u;                        // rows are gate / up
 // bytes, so that the fragment loads of up to 8 rows (lanes g = row) fall on
 // distinct banks.
 constexpr uint32_t kGemvXPitch = kGemvCols * 512u + 32u;
+// Reduction slots (consumers -> epilogue), [M][kGemvRedStride] fp32 each.  At
+// M <= 3 one per consumer warp; at M >= 4 one per block index ("pair slots":
+// the column-1 warp adds its sums to those the column-0 warp of its block
+// stored), half the shared memory, which leaves room for a fifth ring stage.
+// The epilogue adds, block index by block index, column 0 + column 1, then
+// the block indices in order: the same roundings at every M.
+__host__ __device__ constexpr bool gemv_pair_slots(int M) { return M >= 4; }
+__host__ __device__ constexpr int gemv_red_slots(int M) { return gemv_pair_slots(M) ? 8 : 16; }
 // One pipeline stage: the unit's two weight pieces, then M activation rows of
 // two columns (the second half unused when the unit has one column), rounded
-// up to 128 bytes.
+// up to 128 bytes, or to 16 (every bulk copy's alignment) with pair slots,
+// so that five stages fit at M = 5 (a stage's bank pattern does not depend
+// on where it starts: all its addresses shift alike).
 __host__ __device__ constexpr uint32_t gemv_stage_bytes(int M) {
-  return (kGemvCols * kGemvWBox + uint32_t(M) * kGemvXPitch + 127u) / 128u * 128u;
+  return gemv_pair_slots(M)
+             ? (kGemvCols * kGemvWBox + uint32_t(M) * kGemvXPitch + 15u) / 16u * 16u
+             : (kGemvCols * kGemvWBox + uint32_t(M) * kGemvXPitch + 127u) / 128u * 128u;
 }
-// Reduction buffers (consumers -> epilogue): two for M <= 2, one otherwise
-// (shared memory), each 16 warp slots of [M][kGemvRedStride] fp32.
+// Reduction buffers: two for M <= 2, one otherwise.
 __host__ __device__ constexpr int gemv_red_bufs(int M) { return M <= 2 ? 2 : 1; }
 __host__ __device__ constexpr uint32_t gemv_red_bytes(int M) {
-  return uint32_t(gemv_red_bufs(M)) * kGemvConsumerWarps * uint32_t(M) * kGemvRedStride * 4u;
+  return uint32_t(gemv_red_bufs(M)) * uint32_t(gemv_red_slots(M)) * uint32_t(M) * kGemvRedStride *
+         4u;
+}
+// Reduction buffer b of the [bufs] at `red` (consumers and epilogue alike).
+template <int M>
+__device__ __forceinline__ float* gemv_red_buffer(float* red, int b) {
+  return red + size_t(b) * gemv_red_slots(M) * M * kGemvRedStride;
 }
 // Shared memory: ring, reduction buffers, the abort flag (padded to 16), 2
-// barriers per stage and 2 per reduction buffer.
+// barriers per stage, 2 per reduction buffer and, with pair slots, one per
+// slot of each buffer.
 __host__ __device__ constexpr size_t gemv_smem_bytes(int M, int stages) {
   return size_t(stages) * gemv_stage_bytes(M) + gemv_red_bytes(M) + 16 + size_t(stages) * 16 +
-         size_t(gemv_red_bufs(M)) * 16;
+         size_t(gemv_red_bufs(M)) * 16 +
+         (gemv_pair_slots(M) ? size_t(gemv_red_bufs(M)) * gemv_red_slots(M) * 8 : 0);
 }
 
 // First unit of (job-local) CTA c when U units are shared out over G CTAs
@@ -402,17 +423,27 @@ __device__ __forceinline__ bool read_slot(const unsigned long long* s_e, int e, 
 }
 
 // This CTA's sums of a row block segment, epilogue side (warp e: rows [64 e,
-// 64 e + 64)): the 16 consumer warps' slots of reduction buffer `buf` added in
-// warp order into v; then the buffer is released (this warp's arrival).
+// 64 e + 64)): the slots of reduction buffer `buf` added into v, block index
+// by block index (column 0 + column 1: the sum a pair slot already holds),
+// in block order; then the buffer is released (this warp's arrival).
 template <int M>
 __device__ __forceinline__ void gemv_segment_sum(const float* buf, uint64_t* buf_empty, int e,
                                                  int lane, float (&v)[2 * M]) {
   #pragma unroll
   for (int k = 0; k < 2 * M; ++k) {
     const float* col = buf + (k >> 1) * kGemvRedStride + seg_row(e, lane, k);
-    float acc = col[0];
-    #pragma unroll
-    for (int w = 1; w < kGemvConsumerWarps; ++w) acc += col[w * M * kGemvRedStride];
+    float acc;
+    if constexpr (gemv_pair_slots(M)) {
+      acc = col[0];
+      #pragma unroll
+      for (int w = 1; w < 8; ++w) acc += col[w * M * kGemvRedStride];
+    } else {
+      constexpr int kCol1 = 8 * M * kGemvRedStride;     // the column-1 warps' slots
+      acc = col[0] + col[kCol1];
+      #pragma unroll
+      for (int w = 1; w < 8; ++w)
+        acc += col[w * M * kGemvRedStride] + col[kCol1 + w * M * kGemvRedStride];
+    }
     v[k] = acc;
   }
   __syncwarp();
@@ -494,12 +525,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
   constexpr uint32_t kXOff = kGemvCols * kGemvWBox;
   uint8_t* ring = smem;
   constexpr int kRedBufs = gemv_red_bufs(M);
-  float* red = reinterpret_cast<float*>(smem + size_t(S) * kStage);  // [bufs][16 warps][M][stride]
+  float* red = reinterpret_cast<float*>(smem + size_t(S) * kStage);  // [bufs][8 slots][M][stride]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(red + gemv_red_bytes(M) / 4);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(S) * kStage + gemv_red_bytes(M) + 16);
   uint64_t* empty = full + S;
-  uint64_t* red_full = empty + S;            // [bufs] every consumer warp's slot written
+  uint64_t* red_full = empty + S;            // [bufs] every slot holds both columns' sums
   uint64_t* red_empty = red_full + kRedBufs; // [bufs] buffer read by both epilogue warps
+  uint64_t* red_pair = red_empty + kRedBufs; // pair slots: [bufs][8] column 0's sums are in
 
   if (tid == 0) {
     griddep_launch_dependents();  // the next kernel on the stream may start its prologue
@@ -508,8 +540,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
       mbar_init(smem_addr(&empty[s]), kGemvConsumerWarps);
     }
     for (int b = 0; b < kRedBufs; ++b) {
-      mbar_init(smem_addr(&red_full[b]), kGemvConsumerWarps);
+      mbar_init(smem_addr(&red_full[b]), gemv_red_slots(M));
       mbar_init(smem_addr(&red_empty[b]), kGemvEpilogueWarps);
+      if constexpr (gemv_pair_slots(M))
+        for (int k = 0; k < 8; ++k) mbar_init(smem_addr(&red_pair[b * 8 + k]), 1);
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -664,8 +698,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
         }
         gemv_wait(fb, fpar, a.err, abort_flag);
         float v[2 * M];
-        gemv_segment_sum<M>(red + size_t(b) * kGemvConsumerWarps * M * kGemvRedStride,
-                            &red_empty[b], e, lane, v);
+        gemv_segment_sum<M>(gemv_red_buffer<M>(red, b), &red_empty[b], e, lane, v);
         const bool wrote =
             gemv_segment_write<M>(a, J, r.cj, rb, e, lane, abort_flag, pre, pv, v);
         if (wrote && a.n_jobs > 1) {
@@ -755,22 +788,42 @@ __global__ void __launch_bounds__(kGemvThreads, 1) q4_gemv_kernel(const __grid_c
       }
       // hand this warp's sums of the row block to the epilogue: its slot of
       // reduction buffer seg % bufs (released by the epilogue after segment
-      // seg - bufs), element (m, row) at m * stride + row
+      // seg - bufs), element (m, row) at m * stride + row.  With pair slots
+      // the column-0 warp stores its sums into the slot of its block index,
+      // and the column-1 warp adds its own once they are there and reports
+      // the slot complete.
       const int b = seg % kRedBufs;
       if (seg >= kRedBufs)
         gemv_wait(smem_addr(&red_empty[b]), uint32_t((seg - kRedBufs) / kRedBufs) & 1u, a.err,
                   abort_flag);
-      float* slot = red + (size_t(b) * kGemvConsumerWarps + warp) * M * kGemvRedStride;
-      #pragma unroll
-      for (int p = 0; p < kGemvTiles; ++p)
+      constexpr bool kPair = gemv_pair_slots(M);
+      float* slot =
+          gemv_red_buffer<M>(red, b) + size_t(kPair ? task_blk : warp) * M * kGemvRedStride;
+      const uint32_t pair = kPair ? smem_addr(&red_pair[b * 8 + task_blk]) : 0u;
+      if (!kPair || task_col == 0) {
         #pragma unroll
-        for (int e = 0; e < 2; ++e)
-          if (2 * t + e < M) {
-            slot[(2 * t + e) * kGemvRedStride + 16 * p + g] = acc[p][e];
-            slot[(2 * t + e) * kGemvRedStride + 16 * p + g + 8] = acc[p][2 + e];
-          }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&red_full[b]));
+        for (int p = 0; p < kGemvTiles; ++p)
+          #pragma unroll
+          for (int e = 0; e < 2; ++e)
+            if (2 * t + e < M) {
+              slot[(2 * t + e) * kGemvRedStride + 16 * p + g] = acc[p][e];
+              slot[(2 * t + e) * kGemvRedStride + 16 * p + g + 8] = acc[p][2 + e];
+            }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(kPair ? pair : smem_addr(&red_full[b]));
+      } else {
+        gemv_wait(pair, uint32_t(seg / kRedBufs) & 1u, a.err, abort_flag);
+        #pragma unroll
+        for (int p = 0; p < kGemvTiles; ++p)
+          #pragma unroll
+          for (int e = 0; e < 2; ++e)
+            if (2 * t + e < M) {
+              slot[(2 * t + e) * kGemvRedStride + 16 * p + g] += acc[p][e];
+              slot[(2 * t + e) * kGemvRedStride + 16 * p + g + 8] += acc[p][2 + e];
+            }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&red_full[b]));
+      }
       ++seg;
       u += n_units;
     }

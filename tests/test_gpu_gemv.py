@@ -177,15 +177,18 @@ def test_output_head_sampled_rows(cuda_ok):
         assert_gemv_close(y[:, torch.from_numpy(rows).cuda()], y_ref, S, f"head M={M}")
 
 
-@pytest.mark.parametrize("N,K", [(2048, 5120), (300, 1280), (64, 65536)])
-def test_verify_rows_equal_single_row_calls_bitwise(cuda_ok, N, K):
-    # row m of an M = 5 verification call is the M = 1 call on x[m], bit for
+@pytest.mark.parametrize("N,K", [(2048, 5120), (300, 1280), (64, 65536), (17408, 5120)])
+@pytest.mark.parametrize("M", [3, 4, 5])
+def test_verify_rows_equal_single_row_calls_bitwise(cuda_ok, N, K, M):
+    # row m of an M-row verification call is the M = 1 call on x[m], bit for
     # bit: the rows are independent columns of the MMAs and every row sees the
-    # same blocking, K ranges and summation order
+    # same blocking, K ranges and summation order -- also across the change of
+    # reduction slots (one per consumer warp up to M = 3, one per block index
+    # from M = 4: column 0 + column 1 first in both)
     W = dev_bytes(synth.q4_0_weights(600 + N, N, K))
-    x = synth.activations(601 + N, 5, K)
-    y5 = q4dec.q4_gemv(W, dev_bf16(x), N=N, K=K)
-    for m in range(5):
+    x = synth.activations(601 + N, M, K)
+    yM = q4dec.q4_gemv(W, dev_bf16(x), N=N, K=K)
+    for m in range(M):
         y1 = q4dec.q4_gemv(W, dev_bf16(x[m:m + 1]), N=N, K=K)
         torch.cuda.synchronize()
-        assert torch.equal(y5[m:m + 1], y1), f"row {m}"
+        assert torch.equal(yM[m:m + 1], y1), f"row {m} of M={M}"

@@ -19,8 +19,20 @@ GEMV_WBOX = GEMV_ROWS * 144
 GEMV_XPITCH = GEMV_COLS * 512 + 32   # activation rows of a stage: 1 KB at a 1056-byte pitch
 
 
+def _gemv_pair_slots(M):
+    # one reduction slot per block index (column 1 adds to column 0) at M >= 4
+    return M >= 4
+
+
 def _gemv_stage_bytes(M):
-    return -(-(GEMV_COLS * GEMV_WBOX + M * GEMV_XPITCH) // 128) * 128
+    align = 16 if _gemv_pair_slots(M) else 128
+    return -(-(GEMV_COLS * GEMV_WBOX + M * GEMV_XPITCH) // align) * align
+
+
+def _gemv_red_layout(M):
+    # (buffers, slots per buffer): two buffers for M <= 2; a slot per consumer
+    # warp, or per block index with pair slots
+    return (2 if M <= 2 else 1), (8 if _gemv_pair_slots(M) else 16)
 
 
 def _unit_begin(c, U, G):
@@ -49,13 +61,17 @@ def test_gemv_geometry(M, N, K, sms):
     assert p.threads == GEMV_THREADS and p.row_blocks == rbs and p.units_per_row_block == upr
     assert p.units == U and 1 <= G <= min(sms, U)
     stage = _gemv_stage_bytes(M)
-    assert stage % 128 == 0 and (p.stages * stage) % 128 == 0
-    # reduction buffers (consumers -> epilogue): 2 for M <= 2, else 1, each a
-    # slot per consumer warp of [M][132] fp32 (128 rows + 4 floats of padding:
-    # the 8 rows x 4 columns a warp stores at once hit distinct banks)
-    bufs = 2 if M <= 2 else 1
-    red = bufs * 16 * M * 132 * 4
-    assert p.smem_bytes == p.stages * stage + red + 16 + p.stages * 16 + bufs * 16
+    assert stage % 16 == 0                    # every stage starts where a bulk copy may land
+    # reduction buffers (consumers -> epilogue), slots of [M][132] fp32 (128
+    # rows + 4 floats of padding: the 8 rows x 4 columns a warp stores at once
+    # hit distinct banks), with pair slots one barrier per slot (the column-0
+    # warp's sums are in) besides the two per buffer
+    bufs, slots_per_buf = _gemv_red_layout(M)
+    red = bufs * slots_per_buf * M * 132 * 4
+    assert p.smem_bytes == (p.stages * stage + red + 16 + p.stages * 16 + bufs * 16 +
+                            (bufs * 8 * 8 if _gemv_pair_slots(M) else 0))
+    if sms == 148:
+        assert p.stages == 5                  # five stages at every M on B200
     banks = {((2 * t + e) * 132 + g) % 32 for t in range(4) for g in range(8) for e in (0,)
              if 2 * t + e < M}
     assert len(banks) == 8 * len([t for t in range(4) if 2 * t < M])
@@ -132,7 +148,7 @@ def test_gemv_geometry(M, N, K, sms):
 @pytest.mark.parametrize("M,N,K", [(1, 17408, 5120), (3, 5120, 17408), (2, 6144, 5120),
                                    (5, 37, 4352), (1, 300, 1280), (4, 1000, 2048)])
 def test_gemv_stream_k_sums_every_product_once(M, N, K):
-    # a model of the partition and of the last-arriver reduction: partial sums
+    # a model of the partition and of the finisher's reduction: partial sums
     # of each CTA's segments, slot by slot, rebuild the full product exactly
     p = q4dec.plan_gemv(M, N, K, 148)
     nsb = K // 256
@@ -571,3 +587,42 @@ def test_q4_unpack_constants_give_exact_codes():
         # each fma is exact (the result is a small integer), so fp16 rounding is moot
         assert float(np.float16(lo * 1.0 - 1032.0)) == q - 8
         assert float(np.float16(hi * (1.0 / 16) - 72.0)) == q - 8
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5])
+def test_gemv_shared_memory_carve_up(M):
+    """Every shared-memory access of the GEMV in bounds, for the planned ring:
+    consumer slot stores (and, with pair slots, column-1 adds), the
+    epilogue's sums, for every reduction buffer; then the abort flag and the
+    barriers (2 per stage, 2 per buffer, with pair slots one per slot of each
+    buffer), ending at the planned size."""
+    p = q4dec.plan_gemv(M, 17408, 5120, 148)
+    S, stage = p.stages, _gemv_stage_bytes(M)
+    bufs, nslot = _gemv_red_layout(M)
+    red_floats = bufs * nslot * M * 132
+    buf_base = lambda b: b * nslot * M * 132               # the kernel's gemv_red_buffer
+    for b in range(bufs):
+        top = buf_base(b) + nslot * M * 132
+        assert top <= red_floats
+        for blk in range(nslot):                            # consumer: its slot
+            for t in range(4):
+                for e in range(2):
+                    m = 2 * t + e
+                    if m >= M:
+                        continue
+                    for p_ in range(8):
+                        for g in range(8):
+                            for r in (g, g + 8):
+                                i = buf_base(b) + blk * M * 132 + m * 132 + 16 * p_ + r
+                                assert buf_base(b) <= i < top
+        for e in range(2):                                  # epilogue warp e: rows 64e..64e+63
+            for lane in range(32):
+                for k in range(2 * M):
+                    row = 64 * e + 32 * (k & 1) + lane
+                    for w in range(nslot):
+                        i = buf_base(b) + (k >> 1) * 132 + row + w * M * 132
+                        assert buf_base(b) <= i < top
+    red_off = S * stage
+    bars = red_off + red_floats * 4 + 16                    # abort flag (padded to 16) first
+    n_bars = 2 * S + 2 * bufs + (8 * bufs if _gemv_pair_slots(M) else 0)
+    assert bars % 8 == 0 and bars + 8 * n_bars == p.smem_bytes <= SMEM_OPTIN
