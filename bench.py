@@ -303,7 +303,11 @@ def main():
     ap.add_argument("--ctx", type=int, default=65536, help="--case attn: ctx_len")
     ap.add_argument("--launches", type=int, default=8, help="--case gemv/attn: launches")
     ap.add_argument("--q8", action="store_true", help="--case attn: the Q8_0 K/V cache")
+    ap.add_argument("--nvtx", action="store_true",
+                    help="mark the step's weight stream and attention layers as NVTX ranges "
+                         "(for a profiler's range filters; off for the reported numbers)")
     args = ap.parse_args()
+    DecodeStep.nvtx = args.nvtx
     ARGS = args
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -600,10 +604,22 @@ class DecodeStep:
         self.h_o = [torch.empty((M, N_Q, HEAD_DIM), dtype=torch.float32, pin_memory=True)
                     for _ in self.outs]
 
+    nvtx = False   # NVTX ranges around the step's phases (bench.py --nvtx)
+
+    def _range(self, name):
+        if self.nvtx:
+            self.torch.cuda.nvtx.range_push(name)
+
+    def _end(self):
+        if self.nvtx:
+            self.torch.cuda.nvtx.range_pop()
+
     def gemv_stream(self):
         # one launch; the weights of later matrices stream while earlier ones
         # finish (programmatic dependent launch against the previous kernel)
+        self._range(f"weight stream M={self.M}")
         self.batch.run(weight_prefetch=True)
+        self._end()
         self.launches += 1
 
     def gemv_stream_per_matrix(self):
@@ -629,7 +645,9 @@ class DecodeStep:
 
     def attn_stream(self):
         for l in range(ATTN_LAYERS):
+            self._range(f"attention layer {l}")
             self.attn(l)
+            self._end()
 
     def e2e_step(self):
         # the step's inputs (the activation rows of each width, every attention
