@@ -428,9 +428,11 @@ def main():
                   "bytes_per_step": step_bytes(5),
                   "roofline": {"bound": "hbm", "kernel": "q4_gemv_kernel<5> (one launch)",
                                "achieved": gb5, "peak": peak_gbs, "unit": "GB/s",
-                               "frac": gb5 / peak_gbs, "launch_us": g5 * 1e3},
+                               "frac": gb5 / peak_gbs, "launch_us": g5 * 1e3,
+                               "traffic": recorded_traffic("q4_gemv_kernel", 5)},
                   "attention": {"achieved_gbs": ab5, "frac": ab5 / peak_gbs,
-                                "us_per_layer": a5 * 1e3 / ATTN_LAYERS},
+                                "us_per_layer": a5 * 1e3 / ATTN_LAYERS,
+                                "traffic": recorded_traffic("q4kv_attn", 5)},
                   "gemv_one_launch_per_matrix": {
                       "ms_per_step": s5, "value": gemv_step_bytes(5) / (s5 * 1e-3) / 1e12,
                       "unit": "TB/s", "launches_per_step": m5.n_gemv}}

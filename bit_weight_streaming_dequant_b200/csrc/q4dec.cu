@@ -72,6 +72,35 @@ q4d_status current_device(int* dev_out, DeviceState** st_out) {
   return Q4D_OK;
 }
 
+// The end of a compute call.  In a debug build (Q4D_DEBUG) the call waits for
+// its stream and reports the device error record -- a failed index check, or
+// a bounded wait that ran out -- as its own status (the record stays set
+// until q4d_device_error(1) clears it); work captured into a graph is not
+// waited for.  In a release build it only returns the launch status.
+q4d_status finish_call(cudaStream_t stream, const DeviceState& s) {
+  if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
+#ifdef Q4D_DEBUG
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &capture) != cudaSuccess) {
+    cudaGetLastError();
+    return Q4D_ERR_CUDA;
+  }
+  if (capture != cudaStreamCaptureStatusNone) return Q4D_OK;
+  unsigned word = 0;
+  if (cudaStreamSynchronize(stream) != cudaSuccess ||
+      cudaMemcpy(&word, s.err, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return Q4D_ERR_CUDA;
+  }
+  if (word & q4d::kDevErrIndex) return Q4D_ERR_DEVICE_INDEX;
+  if (word) return Q4D_ERR_DEVICE_TIMEOUT;
+#else
+  (void)stream;
+  (void)s;
+#endif
+  return Q4D_OK;
+}
+
 // Raise a kernel's dynamic shared-memory limit to the device maximum, once
 // per (kernel, device).
 template <typename Kernel>
@@ -329,8 +358,7 @@ q4d_status gemv_impl(const void* W_q4, const void* x, void* y, int M, int N, int
   J.rot = 0;
   J.w_bytes = declared_weight_bytes(rows, K / 256);
   if ((st = launch_gemv(M, a, p.smem_bytes, dev, *s, stream, pdl)) != Q4D_OK) return st;
-  if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
-  return Q4D_OK;
+  return finish_call(stream, *s);
 }
 
 // The warp-local mma.sync kernel (at most 8 query rows per CTA).
@@ -438,8 +466,7 @@ q4d_status attn_impl(const void* Q, const void* Kq4, const void* Vq4, float* out
       return Q4D_ERR_CUDA;
     }
   }
-  if (cudaGetLastError() != cudaSuccess) return Q4D_ERR_CUDA;
-  return Q4D_OK;
+  return finish_call(stream, *s);
 }
 
 int planning_sms() {
@@ -732,7 +759,7 @@ q4d_status q4_gemv_batch_ex(const void* desc_host, void* desc_dev, void* stream,
                         static_cast<cudaStream_t>(stream), (flags & Q4D_GEMV_WEIGHT_PREFETCH) != 0)) !=
       Q4D_OK)
     return st;
-  return cudaGetLastError() == cudaSuccess ? Q4D_OK : Q4D_ERR_CUDA;
+  return finish_call(static_cast<cudaStream_t>(stream), *s);
 }
 
 q4d_status q4kv_attn_decode(const void* Q, const void* Kq4, const void* Vq4, float* out,
@@ -786,7 +813,7 @@ extern "C" q4d_status q4kv_append(void* Kq4, void* Vq4, const float* k_new, cons
   a.M = M;
   a.err = s->err;
   q4d::q4kv_append_kernel<<<dim3(M * n_kv_heads, 2), 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
-  return cudaGetLastError() == cudaSuccess ? Q4D_OK : Q4D_ERR_CUDA;
+  return finish_call(static_cast<cudaStream_t>(stream), *s);
 }
 
 // ---- host layout helpers: canonical 18-byte blocks <-> 144-byte super-blocks

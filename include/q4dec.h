@@ -454,6 +454,10 @@ q4d_status q4d_device_error_record(unsigned* record, int reset);
  * traps: it sets bit 2 of the device error record (site and index of the
  * first failure), skips the access or redirects a copy to its buffer's first
  * bytes, and the kernel runs to its end; results of that launch are void.
+ * Every compute entry point of the debug build also waits for its stream
+ * and returns Q4D_ERR_DEVICE_INDEX or Q4D_ERR_DEVICE_TIMEOUT while the record
+ * is set (it stays set until q4d_device_error(1) clears it); on a stream that
+ * is being captured into a graph it does not wait.
  * No counterpart in the source pages: a test facility of this library.
  *
  * q4d_debug_build: 1 in the debug build, 0 otherwise.

@@ -4,7 +4,8 @@ error record).  On valid inputs no check fails and every result is bit for
 bit the release build's (the checks change no arithmetic); a check made to
 fail -- a declared weight extent smaller than the real buffer, so that the
 redirected copies still read memory that exists -- is reported with its site
-and offset, and the launch ends normally."""
+and offset (by the failing call itself: a debug-build call waits for its
+work and returns the record's status), and the launch ends normally."""
 import numpy as np
 import pytest
 import torch
@@ -141,9 +142,13 @@ def test_weight_copy_check_reports_site_and_offset(debug_lib):
     W, x = dev_bytes(Wnp), dev_bf16(xnp)
     limit = 100_000                             # the copies past it read the first rows instead
     q4dec.debug_limit_weights(limit)
-    q4dec.q4_gemv(W, x, N=N, K=K)
-    torch.cuda.synchronize()
-    q4dec.debug_limit_weights(0)
+    try:
+        # a debug-build call waits for its work and reports the record itself
+        with pytest.raises(q4dec.Q4DecError) as failed:
+            q4dec.q4_gemv(W, x, N=N, K=K)
+        assert failed.value.status == 7
+    finally:
+        q4dec.debug_limit_weights(0)
     st, bits, site, index = q4dec.device_error_record(reset=True)
     assert st == 7 and bits == 2, (st, bits)                 # Q4D_ERR_DEVICE_INDEX, no time-out
     assert q4dec.CHECK_SITES[site] == "gemv weights"
