@@ -369,3 +369,26 @@ def test_every_bulk_copy_and_global_store_of_the_kernels_is_index_checked():
             if stores.search(code):
                 window = "\n".join(lines[max(0, i - 6):i + 1])
                 assert any(g in window for g in guards), f"{name}:{i + 1}: {line.strip()}"
+
+
+def test_check_sites_of_the_binding_match_the_device_enum():
+    # the site numbers the binding names are the kernels' IndexCheckSite values
+    text = open(os.path.join(ROOT, "bit_weight_streaming_dequant_b200", "csrc",
+                             "q4dec_device.cuh")).read()
+    body = text[text.index("enum IndexCheckSite"):]
+    body = body[:body.index("};")]
+    sites = {int(v) for v in re.findall(r"kSite\w+\s*=\s*(\d+)", body)}
+    assert sites == set(q4dec.CHECK_SITES)
+    assert q4dec.STATUS[7] == "Q4D_ERR_DEVICE_INDEX"
+    header = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    assert re.search(r"Q4D_ERR_DEVICE_INDEX\s*=\s*7", header)
+
+
+def test_use_debug_library_switches_the_loaded_library_and_back():
+    try:
+        assert q4dec.use_debug_library(True) == q4dec.DEBUG_LIB_PATH
+        assert q4dec.debug_build()
+        assert q4dec.use_debug_library(False) == q4dec.RELEASE_LIB_PATH
+        assert not q4dec.debug_build()
+    finally:
+        q4dec.use_debug_library(False)
