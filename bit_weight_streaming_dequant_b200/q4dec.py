@@ -85,8 +85,10 @@ _lib = None
 
 
 def use_debug_library(debug: bool = True) -> str:
-    """Make the next lib() load the debug (or the release) library; calls
-    made through the other one before keep their results.  Returns the path."""
+    """Choose the library that lib() returns from now on: the debug build
+    (True) or the release build (False).  Both can be loaded in one process;
+    work already launched through the other one is unaffected, and a
+    prepared GemvBatch descriptor serves either.  Returns the chosen path."""
     global _lib, LIB_PATH
     path = DEBUG_LIB_PATH if debug else RELEASE_LIB_PATH
     if path != LIB_PATH:
@@ -505,7 +507,9 @@ def q4kv_attn_decode_noalloc(Q, Kq4, Vq4, out, *, ctx_len: int, n_kv_heads: int,
 
 
 def device_error(reset: bool = False) -> int:
-    """Synchronise and read the device error word (0 = clear)."""
+    """Synchronise and read the device error word: 0 when clear, else the
+    status it stands for (6: a bounded wait ran out, 7: an index check of the
+    debug build failed)."""
     return lib().q4d_device_error(1 if reset else 0)
 
 
