@@ -108,11 +108,11 @@ const char* q4d_status_string(int status);
  * Partition (q4d_plan_gemv): rows are cut into blocks of 128 and K into units
  * of 512 elements; the units are shared out in equal contiguous ranges over
  * one CTA per SM, so a row block may be summed by several CTAs.  All but
- * one of them write fp32 partial sums into the workspace and raise a flag;
- * the CTA whose range ends in the row block waits for the flags and adds the
- * partial sums in a fixed (K) order, so results are deterministic.  Each
- * workspace entry (8 bytes) holds a partial sum and the launch's tag, which
- * marks it as written.  The workspace must therefore be zero-filled before
+ * one of them write their fp32 partial sums into the workspace, each entry
+ * (8 bytes) holding a partial sum and the launch's tag, which marks it as
+ * written; the CTA whose range ends in the row block waits until the entries
+ * carry the tag, adds the partial sums in a fixed (K) order, so results are
+ * deterministic, and clears the entries.  The workspace must therefore be zero-filled before
  * its first use; every launch that returns Q4D_OK and leaves the device error
  * word at 0 leaves it zero-filled again, so one zeroing serves any number of
  * GEMV calls of any shape (zero it again after a reported error, and do not
