@@ -311,7 +311,7 @@ size_t q8kv_attn_workspace_bytes(int ctx_len, int n_q_heads, int n_kv_heads, int
                                  int M);
 
 /* ------------------------------------------- attention, allocation-free --
- * The paper has no counterpart to this entry point; it exists for deployment.
+ * The pages have no counterpart to this entry point; it exists for deployment.
  *
  * Some callers may not allocate device memory once they are running: runtimes
  * that reserve all device memory in their own arena at start-up and forbid
@@ -356,7 +356,7 @@ typedef struct {
   int stages;            /* shared-memory pipeline depth (one unit per stage)      */
   int reserved;
   size_t smem_bytes;     /* dynamic shared memory per CTA                          */
-  size_t workspace_bytes;/* counters + fp32 partial sums of shared row blocks      */
+  size_t workspace_bytes;/* tagged 8-byte partial-sum entries of shared row blocks */
 } q4d_gemv_plan;
 
 typedef struct {
