@@ -82,3 +82,46 @@ def test_reference_arm_prints_from_rank_zero_only():
     for key in ("metric", "value", "unit", "higher_is_better", "cpu_baseline", "e2e", "config"):
         assert key in line
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
+
+
+def test_algorithmic_bytes_of_the_step():
+    # Q4_0: 18 bytes per 32 weights; x bf16 in, y fp32 out per matrix; K and V
+    # super-blocks (144 B) per token and KV head, bf16 queries, fp32 outputs
+    hidden, ffn, qkv, head_n = 5120, 17408, 6144, 151936
+    layer = [(ffn, hidden), (ffn, hidden), (hidden, ffn), (qkv, hidden), (hidden, qkv)]
+    for M in (1, 5):
+        mats = layer * 64 + [(head_n, hidden)]
+        gemv = sum(N * K // 32 * 18 + 2 * M * K + 4 * M * N for N, K in mats)
+        attn = 16 * (2 * 4 * 262144 * 144 + M * 24 * 256 * 6)
+        assert bench.gemv_step_bytes(M) == gemv
+        assert bench.step_bytes(M) == gemv + attn
+    assert bench.gemv_step_bytes(1) == 12347133440      # the 12.35 GB quoted for M = 1
+    assert bench.gemv_step_bytes(5) == 12421957120
+    assert bench.attn_alg_bytes(1, 262144) == 302026752
+    assert bench.step_bytes(1) == 17179561472
+
+
+def test_recorded_traffic_follows_the_source_hash(monkeypatch):
+    rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: rec["source_hash"])
+    got = bench.recorded_traffic("q4_gemv_kernel", 1)
+    assert got == rec["step"]["q4_gemv_kernel"]["M1"]["bytes_per_launch"]
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
+    assert bench.recorded_traffic("q4_gemv_kernel", 1) is None
+
+
+def test_kernel_source_hash_covers_the_kernels_but_not_the_self_tests():
+    import hashlib
+    csrc = os.path.join(ROOT, "bit_weight_streaming_dequant_b200", "csrc")
+    names = sorted(os.listdir(csrc))
+    assert "q4_gemv.cuh" in names and "q4d_selftest.cu" in names
+
+    def digest(skip):
+        h = hashlib.sha256()
+        for n in names:
+            if n not in skip:
+                h.update(n.encode() + open(os.path.join(csrc, n), "rb").read())
+        return h.hexdigest()[:16]
+
+    assert bench.kernel_source_hash() == digest({"q4d_selftest.cu"})
+    assert bench.kernel_source_hash() != digest(set())
